@@ -1,0 +1,150 @@
+"""fp64 CPU oracle for the gated delta rule -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The product path (``libgdn`` and its
+binding ``gated_deltanet_04_b200``) never imports, links or calls it, and the
+two share no code: the oracle is plain C (``gdn_oracle.c``) compiled with gcc,
+driven here through ctypes on numpy float64 arrays.
+
+Method (page "Qwen3.8-27B 架构深读 ...", section 三): the gated delta rule
+    S_t = a_t S_{t-1} (I - b_t k_t k_t^T) + b_t v_t k_t^T,   o_t = S_t q_t,
+with a_t = exp(g_t), b_t = beta_t, plus the page's illustrative step order
+(recall S k taken before the decay) as a flagged variant, and an fp64
+chunk-parallel form used only to cross-check the recurrence.
+
+Every function is pinned by tests/test_oracle_pins.py (invariants, closed
+forms, brute force) and tests/golden/ (hand-worked example).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "gdn_oracle.c")
+_LIB = os.path.join(_HERE, "libgdn_oracle.so")
+_lock = threading.Lock()
+_lib = None
+
+ORDER_STANDARD = 0
+ORDER_ILLUSTRATIVE = 1
+GATE_LOG = 0
+GATE_LINEAR = 1
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle shared library with gcc (fp64, OpenMP)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        cmd = ["gcc", "-O2", "-std=c99", "-fopenmp", "-fPIC", "-shared",
+               "-fno-fast-math", "-ffp-contract=off", _SRC, "-o", tmp, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            lib = ctypes.CDLL(_LIB)
+            dp = ctypes.POINTER(ctypes.c_double)
+            i64p = ctypes.POINTER(ctypes.c_int64)
+            i64 = ctypes.c_int64
+            lib.gdn_oracle_recurrent.argtypes = [dp, dp, dp, dp, dp, dp, i64p, i64, i64, i64, i64,
+                                                 i64, i64, ctypes.c_int, ctypes.c_int,
+                                                 ctypes.c_void_p, dp, dp]
+            lib.gdn_oracle_recurrent.restype = ctypes.c_int
+            lib.gdn_oracle_chunked.argtypes = [dp, dp, dp, dp, dp, dp, i64p, i64, i64, i64, i64,
+                                               i64, i64, i64, dp, dp]
+            lib.gdn_oracle_chunked.restype = ctypes.c_int
+            _lib = lib
+    return _lib
+
+
+def _f64(x):
+    if x is None:
+        return None
+    if hasattr(x, "detach"):  # torch tensor -> exact fp64 copy on the host
+        x = x.detach().to("cpu").double().numpy()
+    return np.ascontiguousarray(x, dtype=np.float64)
+
+
+def _ptr(a, ctype=ctypes.c_double):
+    if a is None:
+        return None
+    return a.ctypes.data_as(ctypes.POINTER(ctype))
+
+
+def _prep(q, k, v, gate, beta, s0, cu_seqlens):
+    q, k, v, gate, beta, s0 = (_f64(x) for x in (q, k, v, gate, beta, s0))
+    T, Hqk, Dk = q.shape
+    Hv, Dv = v.shape[1], v.shape[2]
+    assert k.shape == q.shape and v.shape[0] == T
+    assert gate.shape == (T, Hv) and beta.shape == (T, Hv)
+    if cu_seqlens is None:
+        cu = np.array([0, T], dtype=np.int64)
+    else:
+        if hasattr(cu_seqlens, "detach"):
+            cu_seqlens = cu_seqlens.detach().cpu().numpy()
+        cu = np.ascontiguousarray(cu_seqlens, dtype=np.int64)
+    N = cu.shape[0] - 1
+    if s0 is not None:
+        assert s0.shape == (N, Hv, Dv, Dk)
+    return q, k, v, gate, beta, s0, cu, N, T, Hqk, Hv, Dk, Dv
+
+
+def recurrent(q, k, v, gate, beta, s0=None, cu_seqlens=None, *, order=ORDER_STANDARD,
+              gate_kind=GATE_LOG, heads=None, want_o=True):
+    """Token-by-token fp64 recurrence.
+
+    Shapes: q,k [T,Hqk,Dk]; v [T,Hv,Dv]; gate,beta [T,Hv]; s0 [N,Hv,Dv,Dk] or None;
+    cu_seqlens [N+1] or None (one sequence).  ``gate`` is g (a = exp(g)) for
+    GATE_LOG, or a itself for GATE_LINEAR.  ``heads``: optional iterable of
+    v-heads to compute (others are left as zeros).
+    Returns (o [T,Hv,Dv] or None, final_state [N,Hv,Dv,Dk]) in float64.
+    """
+    lib = _load()
+    q, k, v, gate, beta, s0, cu, N, T, Hqk, Hv, Dk, Dv = _prep(q, k, v, gate, beta, s0, cu_seqlens)
+    o = np.zeros((T, Hv, Dv), dtype=np.float64) if want_o else None
+    sT = np.zeros((N, Hv, Dv, Dk), dtype=np.float64)
+    mask = None
+    if heads is not None:
+        m = np.zeros(Hv, dtype=np.uint8)
+        m[list(heads)] = 1
+        mask = m
+    rc = lib.gdn_oracle_recurrent(_ptr(q), _ptr(k), _ptr(v), _ptr(gate), _ptr(beta), _ptr(s0),
+                                  _ptr(cu, ctypes.c_int64), N, T, Hqk, Hv, Dk, Dv, order,
+                                  gate_kind, None if mask is None else mask.ctypes.data,
+                                  _ptr(o), _ptr(sT))
+    if rc != 0:
+        raise ValueError(f"gdn_oracle_recurrent failed with code {rc}")
+    return o, sT
+
+
+def chunked(q, k, v, g, beta, s0=None, cu_seqlens=None, *, chunk=64):
+    """fp64 chunk-parallel form (standard order, log gate). Same shapes as recurrent()."""
+    lib = _load()
+    q, k, v, g, beta, s0, cu, N, T, Hqk, Hv, Dk, Dv = _prep(q, k, v, g, beta, s0, cu_seqlens)
+    o = np.zeros((T, Hv, Dv), dtype=np.float64)
+    sT = np.zeros((N, Hv, Dv, Dk), dtype=np.float64)
+    rc = lib.gdn_oracle_chunked(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(s0),
+                                _ptr(cu, ctypes.c_int64), N, T, Hqk, Hv, Dk, Dv, int(chunk),
+                                _ptr(o), _ptr(sT))
+    if rc != 0:
+        raise ValueError(f"gdn_oracle_chunked failed with code {rc}")
+    return o, sT
+
+
+def decode_step(q, k, v, g, beta, state, *, order=ORDER_STANDARD):
+    """One-token update of N independent sequences: q,k [N,Hqk,Dk], v [N,Hv,Dv],
+    g,beta [N,Hv], state [N,Hv,Dv,Dk].  Returns (o [N,Hv,Dv], new_state).
+    This is the recurrence with every sequence of length one."""
+    N = q.shape[0]
+    cu = np.arange(N + 1, dtype=np.int64)
+    return recurrent(q, k, v, g, beta, state, cu, order=order)

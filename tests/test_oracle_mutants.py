@@ -1,0 +1,56 @@
+"""The oracle's pins must fail when a plausible mistake is planted in the oracle.
+
+Each case copies oracle/ to a temporary directory, plants one mistake in the
+C source (dropped decay, wrong sign of the delta write, transposed recall,
+read-out with the wrong vector, wrong head grouping, inverted decay mask,
+missing cumulative decay in W, strict instead of inclusive output mask),
+rebuilds it and runs tests/test_oracle_pins.py against the mutant.  At least
+one pin must fail for every mutant.  Mistakes are planted in the oracle on
+the CPU only.
+"""
+import os
+import shutil
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+MUTANTS = {
+    "drop_decay": ("for (int64_t x = 0; x < Dv * Dk; ++x) S[x] *= a;\n            for (int64_t i = 0;",
+                   "for (int64_t x = 0; x < Dv * Dk; ++x) S[x] *= 1.0;\n            for (int64_t i = 0;"),
+    "sign_of_write": ("const double u = b * (vt[i] - r[i]);", "const double u = b * (vt[i] + r[i]);"),
+    "transposed_recall": ("acc += S[i * Dk + d] * kt[d];\n                r[i] = acc;\n            }\n        }",
+                          "acc += S[d * Dk + i] * kt[d];\n                r[i] = acc;\n            }\n        }"),
+    "readout_with_key": ("acc += S[i * Dk + d] * qt[d];", "acc += S[i * Dk + d] * kt[d];"),
+    "head_group_modulo": ("const int64_t j = h / (Hv / Hqk);", "const int64_t j = h % Hqk;"),
+    "chunk_mask_inverted": ("val = GB(beta, r) * kk * exp(gam[r] - gam[i]);",
+                            "val = GB(beta, r) * kk * exp(gam[i] - gam[r]);"),
+    "chunk_W_without_decay": ("GB(beta, i) *\n                                     exp(gam[i]) * KR(i)[d];",
+                              "GB(beta, i) *\n                                     1.0 * KR(i)[d];"),
+    "chunk_output_mask_strict": ("for (int64_t i = 0; i <= r; ++i) {\n                                double qk",
+                                 "for (int64_t i = 0; i < r; ++i) {\n                                double qk"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_mutant(name, tmp_path):
+    src = open(os.path.join(ROOT, "oracle", "gdn_oracle.c")).read()
+    old, new = MUTANTS[name]
+    assert src.count(old) == 1, f"mutation site for {name} not found exactly once"
+    work = tmp_path / "repo"
+    shutil.copytree(os.path.join(ROOT, "oracle"), work / "oracle",
+                    ignore=shutil.ignore_patterns("*.so", "__pycache__"))
+    shutil.copytree(os.path.join(ROOT, "gated_deltanet_04_b200"), work / "gated_deltanet_04_b200",
+                    ignore=shutil.ignore_patterns("*.so", "__pycache__", "csrc"))
+    (work / "tests").mkdir()
+    for f in ("conftest.py", "test_oracle_pins.py"):
+        shutil.copy(os.path.join(ROOT, "tests", f), work / "tests" / f)
+    shutil.copytree(os.path.join(ROOT, "tests", "golden"), work / "tests" / "golden")
+    (work / "oracle" / "gdn_oracle.c").write_text(src.replace(old, new))
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-p", "no:cacheprovider",
+                        "tests/test_oracle_pins.py"], cwd=work, capture_output=True, text=True,
+                       timeout=600)
+    tail = r.stdout.strip().splitlines()[-1] if r.stdout.strip() else r.stderr[-500:]
+    assert r.returncode != 0 and "failed" in tail, f"mutant {name} survived: {tail}"

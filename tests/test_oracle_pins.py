@@ -1,0 +1,356 @@
+"""Pins of the fp64 oracle against facts fixed by the pages and by mathematics.
+
+None of these re-types the oracle's formula: each checks a property that a
+plausible mistake in it (a dropped decay, a wrong sign, a transposed state,
+recall taken from the wrong state, a mis-indexed head group, a wrong mask)
+would break.  Source of the rule: page "Qwen3.8-27B 架构深读: Gated DeltaNet
+混合线性注意力与 262K 长上下文", section 三.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from oracle import GATE_LINEAR, GATE_LOG, ORDER_ILLUSTRATIVE, ORDER_STANDARD
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def rnd(seed):
+    return np.random.default_rng(seed)
+
+
+def unit_rows(x):
+    return x / np.linalg.norm(x, axis=-1, keepdims=True)
+
+
+def make(seed, T=24, Hqk=2, Hv=4, Dk=8, Dv=6, N=1, s0_std=0.5):
+    r = rnd(seed)
+    q = unit_rows(r.standard_normal((T, Hqk, Dk)))
+    k = unit_rows(r.standard_normal((T, Hqk, Dk)))
+    v = r.standard_normal((T, Hv, Dv))
+    g = -np.log1p(np.exp(r.standard_normal((T, Hv))))
+    beta = 1 / (1 + np.exp(-r.standard_normal((T, Hv))))
+    s0 = s0_std * r.standard_normal((N, Hv, Dv, Dk)) if s0_std else None
+    return q, k, v, g, beta, s0
+
+
+def fro(x):
+    return float(np.sqrt(np.sum(x * x)))
+
+
+# ---------------------------------------------------------------- golden ---
+
+def load_worked():
+    toks, illus = [], None
+    with open(os.path.join(GOLDEN, "worked_2x2.txt")) as f:
+        for line in f:
+            if line.startswith("#") or not line.strip():
+                continue
+            head, state, out = (p.split() for p in line.split("|"))
+            if head[0] == "token":
+                vals = [float(x) for x in head[2:]]
+                toks.append((vals, [float(x) for x in state], [float(x) for x in out]))
+            else:
+                illus = ([float(x) for x in state], [float(x) for x in out])
+    return toks, illus
+
+
+@pytest.mark.parametrize("gate_kind", [GATE_LINEAR, GATE_LOG])
+def test_golden_worked_example(gate_kind):
+    toks, illus = load_worked()
+    T = len(toks)
+    a = np.array([t[0][0] for t in toks])
+    b = np.array([t[0][1] for t in toks])
+    k = np.array([t[0][2:4] for t in toks]).reshape(T, 1, 2)
+    v = np.array([t[0][4:6] for t in toks]).reshape(T, 1, 2)
+    q = np.array([t[0][6:8] for t in toks]).reshape(T, 1, 2)
+    gate = a if gate_kind == GATE_LINEAR else np.log(a)
+    tol = 1e-15 if gate_kind == GATE_LINEAR else 1e-14
+    # step by step, carrying the state, so every intermediate state is checked
+    s = None
+    for t in range(T):
+        sl = slice(t, t + 1)
+        o, s = oracle.recurrent(q[sl], k[sl], v[sl], gate[sl].reshape(1, 1), b[sl].reshape(1, 1),
+                                s, gate_kind=gate_kind)
+        np.testing.assert_allclose(s.reshape(4), toks[t][1], rtol=0, atol=tol)
+        np.testing.assert_allclose(o.reshape(2), toks[t][2], rtol=0, atol=tol)
+    # the page's illustrative order differs only at token 4
+    s = None
+    for t in range(T):
+        sl = slice(t, t + 1)
+        o, s = oracle.recurrent(q[sl], k[sl], v[sl], gate[sl].reshape(1, 1), b[sl].reshape(1, 1),
+                                s, gate_kind=gate_kind, order=ORDER_ILLUSTRATIVE)
+        want_s = toks[t][1] if t < 3 else illus[0]
+        want_o = toks[t][2] if t < 3 else illus[1]
+        np.testing.assert_allclose(s.reshape(4), want_s, rtol=0, atol=tol)
+        np.testing.assert_allclose(o.reshape(2), want_o, rtol=0, atol=tol)
+    # and the chunked form reaches the same sequence of outputs
+    if gate_kind == GATE_LOG:
+        for C in (1, 2, 3, 4):
+            o, s = oracle.chunked(q, k, v, gate.reshape(T, 1), b.reshape(T, 1), chunk=C)
+            np.testing.assert_allclose(o.reshape(T, 2), [t[2] for t in toks], atol=1e-14)
+            np.testing.assert_allclose(s.reshape(4), toks[-1][1], atol=1e-14)
+
+
+def test_accounting_pins_workload_shapes():
+    vals = {}
+    with open(os.path.join(GOLDEN, "accounting.txt")) as f:
+        for line in f:
+            if line.strip() and not line.startswith("#"):
+                name, val = line.split()
+                vals[name] = int(val)
+    from gated_deltanet_04_b200.inputs import WORKLOADS
+    wl = WORKLOADS["long256k"]
+    # 48 layers of fp32 state per sequence == about 144 MiB (exactly, with these heads)
+    assert 48 * wl.Hv * wl.Dv * wl.Dk * 4 == vals["gdn_state_48_layers_fp32"] == 144 * 2**20
+    assert 16 * wl.T * 2 * 4 * 256 * 2 == vals["attention_kv_16_layers_262144"] == 16 * 2**30
+    d = WORKLOADS["decode256"]
+    assert d.N * d.Hv * d.Dv * d.Dk * 4 == vals["decode_state_per_layer_256_seqs"]
+    assert d.layers == 48 and wl.Hv // wl.Hqk == 3
+
+
+# ----------------------------------------------------------- invariants ---
+
+def test_P1_identity_step_keeps_state():
+    """a = 1, b = 0: S unchanged (bitwise) and o_t = S0 q_t."""
+    q, k, v, g, beta, s0 = make(1)
+    g[:] = 0.0
+    beta[:] = 0.0
+    o, sT = oracle.recurrent(q, k, v, g, beta, s0)
+    assert np.array_equal(sT, s0)
+    G = 2
+    for h in range(4):
+        want = np.einsum("ed,td->te", s0[0, h], q[:, h // G])
+        np.testing.assert_allclose(o[:, h], want, rtol=0, atol=1e-14)
+
+
+@pytest.mark.parametrize("a_val", [1.0, 0.7, 0.05])
+def test_P2_erase_then_write_unit_key(a_val):
+    """|k| = 1 exactly and b = 1: after the step, S_t k_t = v_t (erase-then-write)."""
+    r = rnd(2)
+    Dk, Dv = 16, 5
+    k = (r.integers(0, 2, (1, 1, Dk)) * 2 - 1) / 4.0  # entries +-1/4 -> |k|^2 = 1 exactly
+    q = unit_rows(r.standard_normal((1, 1, Dk)))
+    v = r.standard_normal((1, 1, Dv))
+    s0 = r.standard_normal((1, 1, Dv, Dk))
+    _, s1 = oracle.recurrent(q, k, v, np.full((1, 1), a_val), np.ones((1, 1)), s0,
+                             gate_kind=GATE_LINEAR)
+    np.testing.assert_allclose(s1[0, 0] @ k[0, 0], v[0, 0], rtol=0, atol=1e-14)
+    # basis key: only column j is rewritten, the rest only decays
+    e = np.zeros((1, 1, Dk)); e[0, 0, 3] = 1.0
+    _, s2 = oracle.recurrent(q, e, v, np.full((1, 1), a_val), np.ones((1, 1)), s0,
+                             gate_kind=GATE_LINEAR)
+    np.testing.assert_allclose(s2[0, 0][:, 3], v[0, 0], rtol=0, atol=1e-15)
+    others = [d for d in range(Dk) if d != 3]
+    assert np.array_equal(s2[0, 0][:, others], a_val * s0[0, 0][:, others])
+
+
+def test_P3_zero_decay_erases_history():
+    """a = 0: S_t = b_t v_t k_t^T and o_t = b_t (k_t . q_t) v_t, whatever came before."""
+    q, k, v, g, beta, s0 = make(3, T=5)
+    a = np.full_like(g, 0.0)
+    o, sT = oracle.recurrent(q, k, v, a, beta, s0, gate_kind=GATE_LINEAR)
+    for h in range(4):
+        kt, qt = k[-1, h // 2], q[-1, h // 2]
+        np.testing.assert_allclose(sT[0, h], beta[-1, h] * np.outer(v[-1, h], kt), atol=1e-15)
+        for t in range(5):
+            want = beta[t, h] * np.dot(k[t, h // 2], q[t, h // 2]) * v[t, h]
+            np.testing.assert_allclose(o[t, h], want, atol=1e-14)
+
+
+def test_P4_linear_in_v_and_state():
+    """At fixed k, b, g the map (S0, V) -> (O, S_T) is linear: superposition holds."""
+    q, k, v, g, beta, s0 = make(4)
+    o_full, s_full = oracle.recurrent(q, k, v, g, beta, s0)
+    o_s0, s_s0 = oracle.recurrent(q, k, np.zeros_like(v), g, beta, s0)
+    o_v, s_v = oracle.recurrent(q, k, v, g, beta, None)
+    np.testing.assert_allclose(o_full, o_s0 + o_v, atol=1e-12)
+    np.testing.assert_allclose(s_full, s_s0 + s_v, atol=1e-12)
+    o_2v, s_2v = oracle.recurrent(q, k, 2.5 * v, g, beta, None)
+    np.testing.assert_allclose(o_2v, 2.5 * o_v, atol=1e-12)
+    np.testing.assert_allclose(s_2v, 2.5 * s_v, atol=1e-12)
+
+
+@pytest.mark.parametrize("C", [1, 4, 16, 64])
+def test_P5_chunked_equals_recurrent(C):
+    q, k, v, g, beta, s0 = make(5, T=150, Dk=16, Dv=16)
+    o1, s1 = oracle.recurrent(q, k, v, g, beta, s0)
+    o2, s2 = oracle.chunked(q, k, v, g, beta, s0, chunk=C)
+    scale = max(1.0, np.abs(o1).max())
+    np.testing.assert_allclose(o2, o1, rtol=0, atol=1e-12 * scale)
+    np.testing.assert_allclose(s2, s1, rtol=0, atol=1e-12)
+
+
+def test_P5_chunked_equals_recurrent_tiny_workload():
+    from gated_deltanet_04_b200.inputs import make_prefill
+    inp = make_prefill("tiny")
+    o1, s1 = oracle.recurrent(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"])
+    o2, s2 = oracle.chunked(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], chunk=16)
+    np.testing.assert_allclose(o2, o1, atol=1e-12)
+    np.testing.assert_allclose(s2, s1, atol=1e-12)
+
+
+def test_P6_split_and_carry_is_bitwise_and_packing_is_independent():
+    q, k, v, g, beta, s0 = make(6, T=40)
+    o, sT = oracle.recurrent(q, k, v, g, beta, s0)
+    for p in (1, 7, 16, 39):
+        oa, sa = oracle.recurrent(q[:p], k[:p], v[:p], g[:p], beta[:p], s0)
+        ob, sb = oracle.recurrent(q[p:], k[p:], v[p:], g[p:], beta[p:], sa)
+        assert np.array_equal(np.concatenate([oa, ob]), o)
+        assert np.array_equal(sb, sT)
+    # three sequences packed with cu_seqlens == three separate runs
+    cu = np.array([0, 9, 9, 40])
+    s03 = np.concatenate([s0, 0.3 * s0, -s0])
+    op, sp = oracle.recurrent(q, k, v, g, beta, s03, cu)
+    for n in range(3):
+        a, b = cu[n], cu[n + 1]
+        on, sn = oracle.recurrent(q[a:b], k[a:b], v[a:b], g[a:b], beta[a:b], s03[n:n + 1])
+        assert np.array_equal(op[a:b], on)
+        assert np.array_equal(sp[n], sn[0])
+    assert np.array_equal(sp[1], s03[1])  # an empty sequence leaves its state alone
+
+
+def orthonormal_keys(seed, T, Dk):
+    r = rnd(seed)
+    Qm, _ = np.linalg.qr(r.standard_normal((Dk, Dk)))
+    return Qm[:T]  # rows orthonormal
+
+
+def test_P7_linear_attention_closed_form():
+    """Orthonormal keys, a = b = 1, S0 = 0: S_T = sum_i v_i k_i^T (linear attention)."""
+    T, Dk, Dv = 10, 12, 7
+    kk = orthonormal_keys(7, T, Dk)
+    r = rnd(70)
+    v = r.standard_normal((T, 1, Dv))
+    q = unit_rows(r.standard_normal((T, 1, Dk)))
+    o, sT = oracle.recurrent(q, kk.reshape(T, 1, Dk), v, np.zeros((T, 1)), np.ones((T, 1)))
+    np.testing.assert_allclose(sT[0, 0], v[:, 0].T @ kk, atol=1e-13)
+    for t in range(T):
+        np.testing.assert_allclose(o[t, 0], (v[: t + 1, 0].T @ kk[: t + 1]) @ q[t, 0], atol=1e-13)
+
+
+def test_P8_orthogonal_keys_brute_force_decay_mask():
+    """Orthonormal keys, general a, b, S0 = 0:
+    o_t = sum_{i<=t} (Gamma_t / Gamma_i) b_i (k_i . q_t) v_i   (O(T^2) brute force)."""
+    T, Dk, Dv = 16, 16, 5
+    kk = orthonormal_keys(8, T, Dk)
+    r = rnd(80)
+    v = r.standard_normal((T, 1, Dv))
+    q = r.standard_normal((T, 1, Dk))
+    g = -r.uniform(0.0, 1.5, (T, 1))
+    b = r.uniform(0.0, 1.0, (T, 1))
+    o, sT = oracle.recurrent(q, kk.reshape(T, 1, Dk), v, g, b)
+    gam = np.cumsum(g[:, 0])
+    for t in range(T):
+        want = np.zeros(Dv)
+        for i in range(t + 1):
+            want += math.exp(gam[t] - gam[i]) * b[i, 0] * np.dot(kk[i], q[t, 0]) * v[i, 0]
+        np.testing.assert_allclose(o[t, 0], want, atol=1e-13)
+    want_S = sum(math.exp(gam[-1] - gam[i]) * b[i, 0] * np.outer(v[i, 0], kk[i]) for i in range(T))
+    np.testing.assert_allclose(sT[0, 0], want_S, atol=1e-13)
+
+
+def test_P9_repeated_key_overwrites():
+    """A key written twice with b = 1 recalls only the latest value (any decay)."""
+    T, Dk, Dv = 6, 8, 3
+    r = rnd(9)
+    key = unit_rows(r.standard_normal(Dk))
+    k = np.tile(key, (T, 1)).reshape(T, 1, Dk)
+    v = r.standard_normal((T, 1, Dv))
+    q = np.tile(key, (T, 1)).reshape(T, 1, Dk)
+    g = -r.uniform(0, 1, (T, 1))
+    o, sT = oracle.recurrent(q, k, v, g, np.ones((T, 1)), r.standard_normal((1, 1, Dv, Dk)))
+    # querying with the key itself returns exactly the latest value
+    np.testing.assert_allclose(o[:, 0], v[:, 0], atol=1e-13)
+    np.testing.assert_allclose(sT[0, 0] @ key, v[-1, 0], atol=1e-13)
+
+
+def test_P10_householder_norm():
+    """b = 2, |k| = 1, v = 0: S (I - 2 k k^T) is a reflection, |S|_F is kept;
+    with decay, |S_t|_F = Gamma_t |S_0|_F."""
+    T, Dk, Dv = 12, 8, 5
+    q, k, v, g, beta, s0 = make(10, T=T, Hqk=1, Hv=1, Dk=Dk, Dv=Dv)
+    v[:] = 0.0
+    beta[:] = 2.0
+    _, sT = oracle.recurrent(q, k, v, np.zeros_like(g), beta, s0)
+    assert abs(fro(sT) - fro(s0)) < 1e-12 * fro(s0)
+    _, sT = oracle.recurrent(q, k, v, g, beta, s0)
+    assert abs(fro(sT) - math.exp(g.sum()) * fro(s0)) < 1e-12 * fro(s0)
+
+
+def test_P11_contractive_when_v_zero():
+    T = 20
+    q, k, v, g, beta, s0 = make(11, T=T, Hqk=1, Hv=1)
+    v[:] = 0.0
+    s = s0
+    prev = fro(s)
+    for t in range(T):
+        sl = slice(t, t + 1)
+        _, s = oracle.recurrent(q[sl], k[sl], v[sl], g[sl], beta[sl], s)
+        cur = fro(s)
+        assert cur <= prev * (1 + 1e-15)
+        assert cur <= math.exp(g[t, 0]) * prev * (1 + 1e-15)
+        prev = cur
+
+
+def test_P13_illustrative_order_difference():
+    """illustrative - standard = -b (1 - a) (S_{t-1} k) k^T for one step; equal when a = 1 or b = 0."""
+    q, k, v, g, beta, s0 = make(13, T=1, Hqk=1, Hv=1)
+    _, s_std = oracle.recurrent(q, k, v, g, beta, s0)
+    _, s_ill = oracle.recurrent(q, k, v, g, beta, s0, order=ORDER_ILLUSTRATIVE)
+    a, b = math.exp(g[0, 0]), beta[0, 0]
+    kt = k[0, 0]
+    diff = -b * (1 - a) * np.outer(s0[0, 0] @ kt, kt)
+    np.testing.assert_allclose(s_ill - s_std, diff.reshape(s_std.shape), atol=1e-14)
+    _, s_std = oracle.recurrent(q, k, v, np.zeros_like(g), beta, s0)
+    _, s_ill = oracle.recurrent(q, k, v, np.zeros_like(g), beta, s0, order=ORDER_ILLUSTRATIVE)
+    assert np.array_equal(s_std, s_ill)
+
+
+def test_head_grouping_is_contiguous():
+    """v-heads h and h' read the same q/k head iff h // G == h' // G."""
+    q, k, v, g, beta, s0 = make(14, Hqk=2, Hv=4)
+    v[:, 1] = v[:, 0]; g[:, 1] = g[:, 0]; beta[:, 1] = beta[:, 0]; s0[:, 1] = s0[:, 0]
+    v[:, 2] = v[:, 0]; g[:, 2] = g[:, 0]; beta[:, 2] = beta[:, 0]; s0[:, 2] = s0[:, 0]
+    o, sT = oracle.recurrent(q, k, v, g, beta, s0)
+    assert np.array_equal(o[:, 0], o[:, 1])            # same group -> identical
+    assert not np.allclose(o[:, 0], o[:, 2])           # other group -> different keys
+
+
+def test_state_orientation_recall():
+    """The state maps keys to values: after one write from S0 = 0 with b = 1,
+    S k = v, i.e. S is Dv x Dk (not its transpose)."""
+    Dk, Dv = 6, 3
+    r = rnd(15)
+    k = unit_rows(r.standard_normal((1, 1, Dk)))
+    v = r.standard_normal((1, 1, Dv))
+    _, s = oracle.recurrent(k, k, v, np.zeros((1, 1)), np.ones((1, 1)))
+    assert s.shape == (1, 1, Dv, Dk)
+    np.testing.assert_allclose(s[0, 0] @ k[0, 0], v[0, 0], atol=1e-15)
+
+
+def test_decode_step_is_length_one_recurrence():
+    r = rnd(16)
+    N, Hqk, Hv, D = 5, 2, 4, 8
+    q = unit_rows(r.standard_normal((N, Hqk, D)))
+    k = unit_rows(r.standard_normal((N, Hqk, D)))
+    v = r.standard_normal((N, Hv, D))
+    g = -r.uniform(0, 1, (N, Hv))
+    b = r.uniform(0, 1, (N, Hv))
+    S = r.standard_normal((N, Hv, D, D))
+    o, S1 = oracle.decode_step(q, k, v, g, b, S)
+    for n in range(N):
+        on, sn = oracle.recurrent(q[n:n + 1], k[n:n + 1], v[n:n + 1], g[n:n + 1], b[n:n + 1],
+                                  S[n:n + 1])
+        assert np.array_equal(o[n], on[0]) and np.array_equal(S1[n], sn[0])
+
+
+def test_bad_seqlens_rejected():
+    q, k, v, g, beta, s0 = make(17, T=8)
+    with pytest.raises(ValueError):
+        oracle.recurrent(q, k, v, g, beta, None, np.array([0, 5, 3, 8]))
+    with pytest.raises(ValueError):
+        oracle.recurrent(q, k, v, g, beta, None, np.array([0, 9]))
