@@ -1,0 +1,416 @@
+#!/usr/bin/env python
+"""Benchmark of libgdn, the gated delta rule on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step is one pass of the whole hot path over one batch of synthetic input:
+  * prefill: gdn_prefill over one 262,144-token layer (B=1, 48 v-heads /
+    16 q-k heads, Dk=Dv=128, chunk 64, bf16 q/k/v, fp32 g/beta/state,
+    zero initial state) -- the headline, in Mtok/s per layer;
+  * decode: gdn_decode_step for 256 sequences through 48 layers, each layer
+    with its own 768 MiB fp32 state updated in place -- reported as state
+    GB/s (bytes read + written) in the "decode" object.
+Inputs are drawn on the device by the seeded generator and are larger than
+L2 (8.7 GB per prefill step, 38.6 GB of decode states), so no flush is needed.
+For N > 1 (torchrun) every rank runs the same workload on its own GPU with no
+data-path collective (weak scaling); timings are the max over ranks.
+
+``--impl reference`` times the fp64 CPU oracle on the host cores instead, on a
+bounded sample of the prefill workload (the only other use of oracle/ here).
+Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "GDN prefill Mtok/s per layer; decode-step state GB/s vs 8 TB/s HBM peak"
+PREFILL_WL = "long256k"
+DECODE_WL = "decode256"
+# per-token algorithmic work of the chunked prefill (Dk = Dv = 128, C = 64,
+# Hv = 48, Hqk = 16), Gram matrices shared by the 3 v-heads of a q/k head:
+#   flops = Hv (4 C Dv + 2 C Dk + 6 Dk Dv) + Hqk 4 C Dk   = 7,602,176
+#   bytes = q,k (2*16*128*2) + v (48*128*2) + o (48*128*2) + g,beta (2*48*4) = 33,152
+PREFILL_FLOP_PER_TOKEN = 48 * (4 * 64 * 128 + 2 * 64 * 128 + 6 * 128 * 128) + 16 * 4 * 64 * 128
+PREFILL_BYTES_PER_TOKEN = 2 * 16 * 128 * 2 + 48 * 128 * 2 * 2 + 2 * 48 * 4
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=10)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    return p.parse_args()
+
+
+# ------------------------------------------------------------ distributed --
+
+class Dist:
+    def __init__(self):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = False
+
+    def init(self, backend):
+        if self.world > 1:
+            import torch.distributed as dist
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+            self.pg = True
+
+    def barrier(self):
+        if self.pg:
+            import torch.distributed as dist
+            if dist.get_backend() == "nccl":
+                dist.barrier(device_ids=[self.local_rank])
+            else:
+                dist.barrier()
+
+    def max(self, x: float) -> float:
+        """Max of a float over ranks (the only collective: timing, not data)."""
+        if not self.pg:
+            return x
+        import torch.distributed as dist
+        dev = torch.device("cuda", self.local_rank) if dist.get_backend() == "nccl" else "cpu"
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+def weak_scaling_value(units_per_rank: float, seconds_max: float, world: int) -> float:
+    """Whole-job throughput: every rank processed units_per_rank in the timed region."""
+    return units_per_rank * world / seconds_max
+
+
+# ------------------------------------------------------------------ clocks --
+
+class ClockSampler:
+    """Samples nvidia-smi clocks and throttle reasons while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.lines = []
+        self.active = False
+
+    def _reader(self):
+        for line in self.proc.stdout:
+            if self.active:
+                self.lines.append(line.strip())
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.gpu_index), "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            threading.Thread(target=self._reader, daemon=True).start()
+        except OSError:
+            self.proc = None
+
+    def mark(self, on: bool):
+        self.active = on
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# -------------------------------------------------------------- roofline ---
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+def traffic_for(kernel_key, src_file):
+    """DRAM bytes per launch from the committed ncu summary, or None when the
+    kernel source changed since the counters were taken."""
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    src = os.path.join(ROOT, "gated_deltanet_04_b200", "csrc", src_file)
+    try:
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        with open(path) as f:
+            for line in f:
+                parts = line.split()
+                if len(parts) >= 3 and not line.startswith("#") and parts[0] == kernel_key \
+                        and parts[1] == sha:
+                    return float(parts[2])
+    except OSError:
+        pass
+    return None
+
+
+# ------------------------------------------------------------------ timing --
+
+def time_launches(fn, K, W, dist, stream, sampler=None):
+    """W warm-up calls, then K timed calls bracketed by barrier + synchronize.
+    Returns (total ms, list of per-call ms) measured with CUDA events on ``stream``."""
+    for _ in range(W):
+        fn()
+    torch.cuda.synchronize()
+    dist.barrier()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(K)]
+    if sampler:
+        sampler.mark(True)
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for a, b in evs:
+        a.record(stream)
+        fn()
+        b.record(stream)
+    end.record(stream)
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.mark(False)
+    dist.barrier()
+    torch.cuda.synchronize()
+    return start.elapsed_time(end), [a.elapsed_time(b) for a, b in evs]
+
+
+def cpu_baseline_prefill(tokens: int):
+    """The fp64 oracle on the host cores, on the first ``tokens`` tokens of the
+    prefill workload (all 48 heads).  Returns (Mtok/s, seconds, threads)."""
+    import oracle
+    from gated_deltanet_04_b200 import inputs
+    oracle.build()
+    inp = inputs.make_prefill(PREFILL_WL, device="cpu", T=tokens)
+    t0 = time.perf_counter()
+    oracle.recurrent(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"])
+    dt = time.perf_counter() - t0
+    threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    return tokens / dt / 1e6, dt, threads
+
+
+def run_reference(args, dist):
+    """Reference arm: the fp64 CPU oracle, timed as it stands, on rank 0 only."""
+    if dist.rank != 0:
+        return 0
+    tokens = 2048
+    vals = []
+    for _ in range(args.warmup):
+        cpu_baseline_prefill(tokens)
+    secs = []
+    for _ in range(args.steps):
+        _, dt, threads = cpu_baseline_prefill(tokens)
+        secs.append(dt)
+    total = sum(secs)
+    value = tokens * args.steps / total / 1e6
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "Mtok/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000 * total / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{PREFILL_WL}: B=1 T=262144 Hv=48 Hqk=16 D=128 chunk=64 "
+                               f"(sample: first {tokens} tokens, all 48 heads, per step)"},
+        "cpu_baseline": {"value": value, "unit": "Mtok/s", "cores": threads, "kind": "oracle",
+                         "sample": f"first {tokens} tokens x 48 heads of the 262,144-token layer"},
+        "e2e": {"value": value, "unit": "Mtok/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse()
+    dist = Dist()
+    if args.impl == "reference":
+        dist.init("gloo")
+        rc = run_reference(args, dist)
+        dist.close()
+        return rc
+
+    import gated_deltanet_04_b200 as gdn
+    from gated_deltanet_04_b200 import inputs
+
+    assert torch.cuda.is_available(), "bench.py needs a CUDA device"
+    torch.cuda.set_device(dist.local_rank)
+    dist.init("nccl")
+    gdn.library()  # fails loudly when libgdn.so is missing
+    dev = torch.device("cuda", dist.local_rank)
+    stream = torch.cuda.current_stream()
+    K, W = args.steps, max(3, args.warmup)
+    peaks = measured_peaks()
+    sampler = ClockSampler(dist.local_rank)
+    sampler.start()
+
+    # ---------------------------------------------------------- prefill --
+    inp = inputs.make_prefill(PREFILL_WL, device=dev)
+    T = inp["T"]
+    o = torch.empty_like(inp["v"])
+    sT = torch.empty((1, 48, 128, 128), dtype=torch.float32, device=dev)
+
+    def prefill():
+        gdn.gdn_prefill(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], None, None,
+                        chunk=64, o=o, final_state=sT)
+
+    p_total, p_each = time_launches(prefill, K, W, dist, stream, sampler)
+    p_ms = dist.max(p_total / K)
+    p_launch_ms = dist.max(sum(p_each) / K)
+
+    # ----------------------------------------------------------- decode --
+    dwl = inputs.WORKLOADS[DECODE_WL]
+    layers = [inputs.make_decode_layer(l, device=dev) for l in range(dwl.layers)]
+    d_outs = [torch.empty_like(L["v"]) for L in layers]
+
+    def decode_step():
+        for L, out in zip(layers, d_outs):
+            gdn.gdn_decode_step(L["q"], L["k"], L["v"], L["g"], L["beta"], L["state"], o=out)
+
+    d_total, _ = time_launches(decode_step, K, W, dist, stream, sampler)
+    d_ms = dist.max(d_total / K)
+    state_bytes_layer = dwl.N * dwl.Hv * dwl.Dv * dwl.Dk * 4 * 2
+    io_bytes_layer = dwl.N * (2 * dwl.Hqk * dwl.Dk * 2 + 2 * dwl.Hv * dwl.Dv * 2 + 2 * dwl.Hv * 4)
+    d_state_gbs = weak_scaling_value(state_bytes_layer * dwl.layers, d_ms / 1e3, dist.world) / 1e9
+    # per-launch timing of the decode kernel (one layer), for its roofline
+    L0, out0 = layers[0], d_outs[0]
+    d1_total, _ = time_launches(
+        lambda: gdn.gdn_decode_step(L0["q"], L0["k"], L0["v"], L0["g"], L0["beta"], L0["state"],
+                                    o=out0), K, W, dist, stream)
+    d1_ms = dist.max(d1_total / K)
+    del layers, d_outs
+    torch.cuda.empty_cache()
+    clocks = sampler.stop()
+
+    # -------------------------------------------------------------- e2e --
+    e2e = None
+    if not args.no_e2e:
+        host = {key: inp[key].cpu().pin_memory() for key in ("q", "k", "v", "g", "beta")}
+        o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        s_host = torch.empty(sT.shape, dtype=sT.dtype).pin_memory()
+        dev_in = {key: inp[key] for key in host}
+
+        def e2e_step():
+            for key in host:
+                dev_in[key].copy_(host[key], non_blocking=True)
+            gdn.gdn_prefill(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["g"], dev_in["beta"],
+                            None, None, chunk=64, o=o, final_state=sT)
+            o_host.copy_(o, non_blocking=True)
+            s_host.copy_(sT, non_blocking=True)
+
+        e_total, _ = time_launches(e2e_step, K, W, dist, stream)
+        e_ms = dist.max(e_total / K)
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        d2h = o_host.numel() * o_host.element_size() + s_host.numel() * s_host.element_size()
+        e2e = {"value": weak_scaling_value(T, e_ms / 1e3, dist.world) / 1e6, "unit": "Mtok/s",
+               "ms_per_step": e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    # --------------------------------------------------------- roofline --
+    tc_path = True  # Dk = Dv = 128, bf16, chunk 64 -> tensor-core chunked kernel
+    flops = PREFILL_FLOP_PER_TOKEN * T
+    achieved_tf = flops / (p_launch_ms / 1e3) / 1e12
+    achieved_gbs = PREFILL_BYTES_PER_TOKEN * T / (p_launch_ms / 1e3) / 1e9
+    roofline = {"bound": "tensor", "achieved": achieved_tf, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": achieved_tf / peaks["bf16_tflops"],
+                "traffic": traffic_for("gdn_prefill_tc", "prefill_tc.cu"),
+                "peak_source": f"{peaks['source']} bf16 burst",
+                "kernel": "gdn_prefill_tc" if tc_path else "gdn_prefill_recurrent",
+                "algorithmic_flop_per_launch": flops,
+                "hbm": {"achieved": achieved_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                        "frac": achieved_gbs / peaks["hbm_gbs"],
+                        "algorithmic_bytes_per_launch": PREFILL_BYTES_PER_TOKEN * T}}
+    d_gbs_launch = (state_bytes_layer + io_bytes_layer) / (d1_ms / 1e3) / 1e9
+    decode = {"value": d_state_gbs, "unit": "GB/s", "ms_per_step": d_ms,
+              "layers_per_step": dwl.layers, "sequences": dwl.N,
+              "roofline": {"bound": "hbm", "achieved": d_gbs_launch, "peak": peaks["hbm_gbs"],
+                           "unit": "GB/s", "frac": d_gbs_launch / peaks["hbm_gbs"],
+                           "traffic": traffic_for("gdn_decode", "decode.cu"),
+                           "peak_source": f"{peaks['source']} copy",
+                           "kernel": "gdn_decode_kernel<128>",
+                           "algorithmic_bytes_per_launch": state_bytes_layer + io_bytes_layer},
+              "frac_of_8TBps": d_state_gbs / dist.world / 8000.0}
+
+    cpu = None
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
+        tokens = 4096
+        val, dt, threads = cpu_baseline_prefill(tokens)
+        cpu = {"value": val, "unit": "Mtok/s", "cores": threads, "kind": "oracle",
+               "sample": f"first {tokens} tokens x 48 heads of the 262,144-token layer, "
+                         f"{dt:.1f} s"}
+
+    line = {
+        "metric": METRIC,
+        "value": weak_scaling_value(T, p_ms / 1e3, dist.world) / 1e6,
+        "unit": "Mtok/s",
+        "n_gpus": dist.world, "steps": K, "warmup": W, "ms_per_step": p_ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": f"{PREFILL_WL}: prefill B=1 T=262144 Hv=48 Hqk=16 Dk=Dv=128 "
+                               f"chunk=64 bf16 q/k/v, fp32 g/beta/state; plus {DECODE_WL}: "
+                               "decode N=256 x 48 layers (see 'decode')",
+                   "l2": "inputs larger than L2 (8.7 GB per prefill, 38.6 GB decode states)",
+                   "parallelism": f"replica x{dist.world} (no data-path collective)"},
+        "roofline": roofline,
+        "decode": decode,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": K * (1 + dwl.layers + 1) + K * (0 if args.no_e2e else 1),
+        "clocks": clocks,
+    }
+    if dist.rank == 0:
+        print(json.dumps(line), flush=True)
+    dist.close()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

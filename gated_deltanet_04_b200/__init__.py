@@ -1,0 +1,173 @@
+"""Python binding of libgdn: the gated delta rule on B200 (sm_100a).
+
+Argument marshalling only.  Every step of the computation runs in libgdn's
+CUDA kernels; this module checks tensor shapes/dtypes, allocates outputs with
+torch (device memory is the only thing torch is used for), and passes raw
+device pointers plus the current CUDA stream to the C ABI declared in
+include/gdn.h.  There is no CPU path: if libgdn.so is missing or no CUDA device
+is present, the calls raise.
+
+Entry points (same names as the C ABI):
+    gdn_prefill(q, k, v, g, beta, initial_state=None, cu_seqlens=None, ...)
+    gdn_decode_step(q, k, v, g, beta, state, ...)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+__all__ = ["gdn_prefill", "gdn_decode_step", "gdn_prefill_workspace_bytes", "library",
+           "GdnError", "LIB_PATH", "STATUS"]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgdn.so")
+
+STATUS = {0: "GDN_OK", 1: "GDN_ERR_INVALID_ARGUMENT", 2: "GDN_ERR_UNSUPPORTED", 3: "GDN_ERR_CUDA",
+          4: "GDN_ERR_TIMEOUT", 5: "GDN_ERR_BAD_SEQLENS"}
+DTYPE = {torch.bfloat16: 0, torch.float32: 1}
+
+_lib = None
+_lock = threading.Lock()
+
+
+class GdnError(RuntimeError):
+    def __init__(self, code, where):
+        self.code = int(code)
+        super().__init__(f"{where} failed: {STATUS.get(self.code, self.code)}")
+
+
+def library():
+    """Load libgdn.so (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise ImportError(f"libgdn.so not built at {LIB_PATH}; run "
+                                  "`python -m gated_deltanet_04_b200.build`")
+            lib = ctypes.CDLL(LIB_PATH)
+            vp, i32, i64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+            lib.gdn_prefill.argtypes = [vp, vp, vp, ctypes.c_int, vp, vp, vp, vp, i32, i64, i32, i32,
+                                        i32, i32, i32, vp, vp, vp, sz, vp, vp]
+            lib.gdn_prefill.restype = ctypes.c_int
+            lib.gdn_decode_step.argtypes = [vp, vp, vp, ctypes.c_int, vp, vp, vp, i32, i32, i32, i32,
+                                            i32, vp, vp, vp]
+            lib.gdn_decode_step.restype = ctypes.c_int
+            lib.gdn_prefill_workspace_bytes.argtypes = [i32, i64, i32, i32, i32, i32, i32]
+            lib.gdn_prefill_workspace_bytes.restype = sz
+            lib.gdn_status_string.argtypes = [ctypes.c_int]
+            lib.gdn_status_string.restype = ctypes.c_char_p
+            lib.gdn_version.argtypes = []
+            lib.gdn_version.restype = i32
+            _lib = lib
+    return _lib
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(t, name, shape, dtype, device):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def gdn_prefill_workspace_bytes(N, T, Hqk, Hv, Dk, Dv, chunk=0):
+    return int(library().gdn_prefill_workspace_bytes(N, T, Hqk, Hv, Dk, Dv, chunk))
+
+
+def gdn_prefill(q, k, v, g, beta, initial_state=None, cu_seqlens=None, *, chunk=0, o=None,
+                final_state=None, output_final_state=True, workspace=None, error_flag=None,
+                stream=None):
+    """Chunk-parallel prefill of the gated delta rule on the GPU.
+
+    q, k [T,Hqk,Dk] and v [T,Hv,Dv] (bf16 or fp32, same dtype); g, beta [T,Hv] fp32;
+    initial_state [N,Hv,Dv,Dk] fp32 or None; cu_seqlens int32 [N+1] on the device or None.
+    Returns (o [T,Hv,Dv], final_state [N,Hv,Dv,Dk] or None).  ``final_state`` may be
+    ``initial_state`` for an in-place update.  Asynchronous on the current stream.
+    """
+    lib = library()
+    dev = q.device
+    if dev.type != "cuda":
+        raise ValueError("gdn_prefill runs on CUDA tensors only")
+    T, Hqk, Dk = q.shape
+    Hv, Dv = v.shape[1], v.shape[2]
+    if q.dtype not in DTYPE:
+        raise ValueError(f"unsupported io dtype {q.dtype}")
+    _check(k, "k", (T, Hqk, Dk), q.dtype, dev)
+    _check(q, "q", (T, Hqk, Dk), q.dtype, dev)
+    _check(v, "v", (T, Hv, Dv), q.dtype, dev)
+    _check(g, "g", (T, Hv), torch.float32, dev)
+    _check(beta, "beta", (T, Hv), torch.float32, dev)
+    if cu_seqlens is None:
+        N = 1
+    else:
+        N = cu_seqlens.shape[0] - 1
+        _check(cu_seqlens, "cu_seqlens", (N + 1,), torch.int32, dev)
+    if initial_state is not None:
+        _check(initial_state, "initial_state", (N, Hv, Dv, Dk), torch.float32, dev)
+    if o is None:
+        o = torch.empty((T, Hv, Dv), dtype=q.dtype, device=dev)
+    _check(o, "o", (T, Hv, Dv), q.dtype, dev)
+    if final_state is None and output_final_state:
+        final_state = torch.empty((N, Hv, Dv, Dk), dtype=torch.float32, device=dev)
+    if final_state is not None:
+        _check(final_state, "final_state", (N, Hv, Dv, Dk), torch.float32, dev)
+    ws_bytes = 0
+    if workspace is not None:
+        ws_bytes = workspace.numel() * workspace.element_size()
+    else:
+        need = int(lib.gdn_prefill_workspace_bytes(N, T, Hqk, Hv, Dk, Dv, chunk))
+        if need:
+            workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+            ws_bytes = need
+    rc = lib.gdn_prefill(_ptr(q), _ptr(k), _ptr(v), DTYPE[q.dtype], _ptr(g), _ptr(beta),
+                         _ptr(initial_state), _ptr(cu_seqlens), N, T, Hqk, Hv, Dk, Dv, chunk,
+                         _ptr(o), _ptr(final_state), _ptr(workspace), ws_bytes, _ptr(error_flag),
+                         _stream(stream))
+    if rc != 0:
+        raise GdnError(rc, "gdn_prefill")
+    return o, final_state
+
+
+def gdn_decode_step(q, k, v, g, beta, state, *, o=None, error_flag=None, stream=None):
+    """One-token update of N sequences, in place on ``state`` [N,Hv,Dv,Dk] fp32.
+
+    q, k [N,Hqk,Dk], v [N,Hv,Dv] (bf16 or fp32); g, beta [N,Hv] fp32.  Returns o [N,Hv,Dv].
+    """
+    lib = library()
+    dev = q.device
+    if dev.type != "cuda":
+        raise ValueError("gdn_decode_step runs on CUDA tensors only")
+    N, Hqk, Dk = q.shape
+    Hv, Dv = v.shape[1], v.shape[2]
+    if q.dtype not in DTYPE:
+        raise ValueError(f"unsupported io dtype {q.dtype}")
+    _check(k, "k", (N, Hqk, Dk), q.dtype, dev)
+    _check(v, "v", (N, Hv, Dv), q.dtype, dev)
+    _check(g, "g", (N, Hv), torch.float32, dev)
+    _check(beta, "beta", (N, Hv), torch.float32, dev)
+    _check(state, "state", (N, Hv, Dv, Dk), torch.float32, dev)
+    if o is None:
+        o = torch.empty((N, Hv, Dv), dtype=q.dtype, device=dev)
+    _check(o, "o", (N, Hv, Dv), q.dtype, dev)
+    rc = lib.gdn_decode_step(_ptr(q), _ptr(k), _ptr(v), DTYPE[q.dtype], _ptr(g), _ptr(beta),
+                             _ptr(state), N, Hqk, Hv, Dk, Dv, _ptr(o), _ptr(error_flag),
+                             _stream(stream))
+    if rc != 0:
+        raise GdnError(rc, "gdn_decode_step")
+    return o

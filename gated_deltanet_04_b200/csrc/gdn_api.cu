@@ -1,0 +1,97 @@
+// libgdn C ABI: argument validation and kernel dispatch.  See include/gdn.h
+// for the contract of every entry point.
+#include <stdint.h>
+
+#include "gdn_internal.cuh"
+
+namespace {
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool supported_dim(int32_t d) { return d == 16 || d == 32 || d == 64 || d == 128; }
+
+bool tc_path(gdn_dtype dt, int32_t Dk, int32_t Dv, int32_t chunk) {
+    return dt == GDN_DTYPE_BF16 && Dk == 128 && Dv == 128 && (chunk == 0 || chunk == 64);
+}
+
+gdn_status from_cuda(cudaError_t e) { return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+const char *gdn_status_string(gdn_status s) {
+    switch (s) {
+        case GDN_OK: return "GDN_OK";
+        case GDN_ERR_INVALID_ARGUMENT: return "GDN_ERR_INVALID_ARGUMENT";
+        case GDN_ERR_UNSUPPORTED: return "GDN_ERR_UNSUPPORTED";
+        case GDN_ERR_CUDA: return "GDN_ERR_CUDA";
+        case GDN_ERR_TIMEOUT: return "GDN_ERR_TIMEOUT";
+        case GDN_ERR_BAD_SEQLENS: return "GDN_ERR_BAD_SEQLENS";
+    }
+    return "GDN_ERR_UNKNOWN";
+}
+
+int32_t gdn_version(void) { return 1 * 10000 + 0 * 100 + 0; }
+
+size_t gdn_prefill_workspace_bytes(int32_t N, int64_t T, int32_t Hqk, int32_t Hv, int32_t Dk,
+                                   int32_t Dv, int32_t chunk) {
+    (void)N; (void)T; (void)Hqk; (void)Hv; (void)Dk; (void)Dv; (void)chunk;
+    return 0;
+}
+
+gdn_status gdn_prefill(const void *q, const void *k, const void *v, gdn_dtype io_dtype,
+                       const float *g, const float *beta, const float *initial_state,
+                       const int32_t *cu_seqlens, int32_t N, int64_t T, int32_t Hqk, int32_t Hv,
+                       int32_t Dk, int32_t Dv, int32_t chunk, void *o, float *final_state,
+                       void *workspace, size_t workspace_bytes, int32_t *dev_error_flag,
+                       void *stream) {
+    if (io_dtype != GDN_DTYPE_BF16 && io_dtype != GDN_DTYPE_F32) return GDN_ERR_INVALID_ARGUMENT;
+    if (N < 0 || T < 0 || Hqk <= 0 || Hv <= 0 || Dk <= 0 || Dv <= 0 || chunk < 0)
+        return GDN_ERR_INVALID_ARGUMENT;
+    if (Hv % Hqk != 0) return GDN_ERR_INVALID_ARGUMENT;
+    if (cu_seqlens == nullptr && N != 1) return GDN_ERR_INVALID_ARGUMENT;
+    if (N == 0) return T == 0 ? GDN_OK : GDN_ERR_INVALID_ARGUMENT;
+    if (T > 0 && (!q || !k || !v || !g || !beta || !o)) return GDN_ERR_INVALID_ARGUMENT;
+    const void *ptrs[] = {q, k, v, g, beta, initial_state, cu_seqlens, o, final_state, workspace,
+                          dev_error_flag};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return GDN_ERR_INVALID_ARGUMENT;
+    if (o && (o == q || o == k || o == v)) return GDN_ERR_INVALID_ARGUMENT;
+    if (!supported_dim(Dk) || !supported_dim(Dv) || chunk > 64) return GDN_ERR_UNSUPPORTED;
+    const size_t need = gdn_prefill_workspace_bytes(N, T, Hqk, Hv, Dk, Dv, chunk);
+    if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return GDN_ERR_INVALID_ARGUMENT;
+    if (T == 0 && final_state == nullptr) return GDN_OK;  // nothing observable to do
+
+    gdn::PrefillArgs a;
+    a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.s0 = initial_state; a.cu = cu_seqlens;
+    a.o = o; a.sT = final_state; a.err = dev_error_flag; a.T = T; a.N = N; a.Hqk = Hqk;
+    a.Hv = Hv; a.Dk = Dk; a.Dv = Dv; a.chunk = chunk == 0 ? 64 : chunk; a.dtype = io_dtype;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (tc_path(io_dtype, Dk, Dv, chunk)) return from_cuda(gdn::launch_prefill_tc(a, s));
+    return from_cuda(gdn::launch_prefill_recurrent(a, s));
+}
+
+gdn_status gdn_decode_step(const void *q, const void *k, const void *v, gdn_dtype io_dtype,
+                           const float *g, const float *beta, float *state, int32_t N,
+                           int32_t Hqk, int32_t Hv, int32_t Dk, int32_t Dv, void *o,
+                           int32_t *dev_error_flag, void *stream) {
+    if (io_dtype != GDN_DTYPE_BF16 && io_dtype != GDN_DTYPE_F32) return GDN_ERR_INVALID_ARGUMENT;
+    if (N < 0 || Hqk <= 0 || Hv <= 0 || Dk <= 0 || Dv <= 0) return GDN_ERR_INVALID_ARGUMENT;
+    if (Hv % Hqk != 0) return GDN_ERR_INVALID_ARGUMENT;
+    if ((int64_t)N * Hv > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
+    if (N == 0) return GDN_OK;
+    if (!q || !k || !v || !g || !beta || !state || !o) return GDN_ERR_INVALID_ARGUMENT;
+    const void *ptrs[] = {q, k, v, g, beta, state, o, dev_error_flag};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return GDN_ERR_INVALID_ARGUMENT;
+    if (o == q || o == k || o == v || o == state) return GDN_ERR_INVALID_ARGUMENT;
+    if (!supported_dim(Dk)) return GDN_ERR_UNSUPPORTED;
+    gdn::DecodeArgs a;
+    a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.state = state; a.o = o;
+    a.err = dev_error_flag; a.N = N; a.Hqk = Hqk; a.Hv = Hv; a.Dk = Dk; a.Dv = Dv;
+    a.dtype = io_dtype;
+    return from_cuda(gdn::launch_decode(a, static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,80 @@
+// Internal declarations shared by libgdn's translation units (not installed).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "gdn.h"
+
+namespace gdn {
+
+// Everything a prefill kernel needs; pointers are device pointers.
+struct PrefillArgs {
+    const void *q, *k, *v;
+    const float *g, *beta;
+    const float *s0;        // may be null (zeros)
+    const int32_t *cu;      // may be null (one sequence)
+    void *o;
+    float *sT;              // may be null
+    int32_t *err;           // may be null
+    int64_t T;
+    int32_t N, Hqk, Hv, Dk, Dv, chunk;
+    gdn_dtype dtype;
+};
+
+struct DecodeArgs {
+    const void *q, *k, *v;
+    const float *g, *beta;
+    float *state;
+    void *o;
+    int32_t *err;
+    int32_t N, Hqk, Hv, Dk, Dv;
+    gdn_dtype dtype;
+};
+
+// Host launchers (return cudaGetLastError() of the launch).
+cudaError_t launch_prefill_recurrent(const PrefillArgs &a, cudaStream_t s);
+cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s);
+// Tensor-core chunked prefill, Dk = Dv = 128, bf16, chunk 64.
+cudaError_t launch_prefill_tc(const PrefillArgs &a, cudaStream_t s);
+
+// ---------------------------------------------------------------- device --
+
+__device__ __forceinline__ float load_io(const void *p, int64_t idx, gdn_dtype dt) {
+    if (dt == GDN_DTYPE_BF16) return __bfloat162float(static_cast<const __nv_bfloat16 *>(p)[idx]);
+    return static_cast<const float *>(p)[idx];
+}
+
+__device__ __forceinline__ void store_io(void *p, int64_t idx, float x, gdn_dtype dt) {
+    if (dt == GDN_DTYPE_BF16)
+        static_cast<__nv_bfloat16 *>(p)[idx] = __float2bfloat16_rn(x);
+    else
+        static_cast<float *>(p)[idx] = x;
+}
+
+__device__ __forceinline__ void raise_error(int32_t *flag, int code) {
+    if (flag) atomicCAS(flag, 0, code);
+}
+
+// Reads and validates sequence n's token range.  Returns false (and raises
+// GDN_ERR_BAD_SEQLENS) when cu_seqlens is malformed around n; the range is
+// then not to be used.  Uniform across a CTA when every thread passes the
+// same n.
+__device__ __forceinline__ bool seq_range(const int32_t *cu, int32_t n, int32_t N, int64_t T,
+                                          int32_t *err, int64_t &t0, int64_t &t1) {
+    if (cu == nullptr) {
+        t0 = 0;
+        t1 = T;
+        return true;
+    }
+    t0 = cu[n];
+    t1 = cu[n + 1];
+    bool ok = (t0 >= 0) && (t0 <= t1) && (t1 <= T);
+    if (n == 0) ok = ok && (t0 == 0);
+    if (n == N - 1) ok = ok && (t1 == T);
+    if (!ok) raise_error(err, GDN_ERR_BAD_SEQLENS);
+    return ok;
+}
+
+}  // namespace gdn

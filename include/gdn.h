@@ -1,0 +1,151 @@
+/*
+ * gdn.h -- C ABI of libgdn, the gated delta rule on NVIDIA B200 (sm_100a).
+ *
+ * The operation (page "Qwen3.8-27B 架构深读: Gated DeltaNet 混合线性注意力与
+ * 262K 长上下文", section 三, "Gated DeltaNet: 把注意力变成可读写的记忆"):
+ * a fixed-size matrix memory per head that is decayed by a per-token gate and
+ * then edited by the delta rule (erase what the key recalls, write the new
+ * value), read out by the query.  In the standard step order implemented here
+ *
+ *     S_t = a_t S_{t-1} (I - b_t k_t k_t^T) + b_t v_t k_t^T,   o_t = S_t q_t,
+ *     a_t = exp(g_t),  b_t = beta_t,
+ *
+ * i.e. S <- a S; r = S k; S <- S + b (v - r) k^T; o = S q.  The same section
+ * says training/prefill accumulates the state chunk-parallel and inference
+ * does one fixed-size matrix update per token: gdn_prefill is the former,
+ * gdn_decode_step the latter.  Readings of points the page leaves open: the
+ * state is Dv x Dk (S k is a Dv-vector); the gate is one scalar per token and
+ * v-head, passed as its logarithm g; o_t uses the updated state; there is no
+ * 1/sqrt(Dk) scale and no feature map or normalisation inside the operation.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * Layouts are token-major and packed over sequences, row-major, contiguous:
+ *     q, k        [T][Hqk][Dk]        io_dtype
+ *     v, o        [T][Hv][Dv]         io_dtype
+ *     g, beta     [T][Hv]             fp32  (g finite and <= 0; beta finite)
+ *     state       [N][Hv][Dv][Dk]     fp32  (row i of a head's state is S[i,:])
+ *     cu_seqlens  [N+1]               int32, cu[0] = 0, non-decreasing, cu[N] = T
+ * v-head h reads q/k head h / (Hv / Hqk): groups of Hv/Hqk consecutive v-heads
+ * share one q/k head.
+ *
+ * Ownership: every pointer is a DEVICE pointer owned by the caller.  The
+ * library allocates nothing, frees nothing and never synchronises; all work
+ * is enqueued on `stream` (a cudaStream_t; NULL is the legacy default stream)
+ * and completes asynchronously.  Inputs are only read.  Outputs must not alias
+ * inputs, except where stated.  Every pointer must be 16-byte aligned.
+ *
+ * Errors: argument errors are returned synchronously and nothing is launched.
+ * A failed launch returns GDN_ERR_CUDA (cudaGetLastError, no synchronisation).
+ * Errors only the device can see (a malformed cu_seqlens, a bounded wait that
+ * expired) are written as a gdn_status value to *dev_error_flag when that
+ * optional device int32 is given; the caller zeroes it beforehand and reads it
+ * after synchronising.  A unit (sequence, head) that detects such an error
+ * writes no output for itself.  No C++ exception crosses this interface.  The
+ * calls keep no global mutable state and are safe to call from any thread.
+ */
+#ifndef GDN_H_
+#define GDN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define GDN_API __attribute__((visibility("default")))
+#else
+#define GDN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum gdn_status {
+    GDN_OK = 0,
+    GDN_ERR_INVALID_ARGUMENT = 1, /* null/misaligned pointer, bad size, bad enum */
+    GDN_ERR_UNSUPPORTED = 2,      /* valid but not implemented (head dims, dtype) */
+    GDN_ERR_CUDA = 3,             /* a CUDA runtime call or launch failed */
+    GDN_ERR_TIMEOUT = 4,          /* device: a bounded wait expired */
+    GDN_ERR_BAD_SEQLENS = 5       /* device: cu_seqlens malformed */
+} gdn_status;
+
+typedef enum gdn_dtype {
+    GDN_DTYPE_BF16 = 0, /* q, k, v, o in bfloat16; o rounded once, to nearest even */
+    GDN_DTYPE_F32 = 1   /* q, k, v, o in fp32 */
+} gdn_dtype;
+
+/*
+ * gdn_prefill -- chunk-parallel prefill/training forward of the gated delta
+ * rule over a packed batch of N sequences (section 三 of the page above:
+ * "the state is accumulated chunk-parallel").
+ *
+ *   q, k, v, io_dtype   token inputs, layouts above.
+ *   g, beta             per-token log-decay and write strength, fp32 [T][Hv].
+ *   initial_state       fp32 [N][Hv][Dv][Dk] state entering each sequence,
+ *                       or NULL for zeros.
+ *   cu_seqlens          device int32 [N+1] sequence offsets, or NULL for a
+ *                       single sequence (then N must be 1).  Never read on
+ *                       the host.  Empty sequences are allowed: their final
+ *                       state equals their initial state.
+ *   N, T                number of sequences and total tokens (T >= 0).
+ *   Hqk, Hv, Dk, Dv     head counts (Hv % Hqk == 0) and head dimensions.
+ *   chunk               chunk length of the chunk-parallel form; 0 picks the
+ *                       default.  It changes rounding only, never the result.
+ *   o                   output [T][Hv][Dv] in io_dtype.
+ *   final_state         fp32 [N][Hv][Dv][Dk] state after each sequence, or
+ *                       NULL to skip.  May equal initial_state (in place).
+ *   workspace, workspace_bytes
+ *                       scratch of at least gdn_prefill_workspace_bytes();
+ *                       may be NULL when that is 0.
+ *   dev_error_flag      optional device int32 (see Errors above).
+ *   stream              cudaStream_t.
+ *
+ * Supported: Dk = Dv = 128 with bf16 I/O and chunk 0 or 64 runs the tensor-core
+ * (tcgen05) chunked kernel; every other combination with Dk, Dv in
+ * {16, 32, 64, 128} and either dtype runs an exact fp32 token-recurrent CUDA
+ * kernel.  Anything else returns GDN_ERR_UNSUPPORTED.
+ */
+GDN_API gdn_status gdn_prefill(const void *q, const void *k, const void *v, gdn_dtype io_dtype,
+                       const float *g, const float *beta, const float *initial_state,
+                       const int32_t *cu_seqlens, int32_t N, int64_t T, int32_t Hqk, int32_t Hv,
+                       int32_t Dk, int32_t Dv, int32_t chunk, void *o, float *final_state,
+                       void *workspace, size_t workspace_bytes, int32_t *dev_error_flag,
+                       void *stream);
+
+/*
+ * gdn_prefill_workspace_bytes -- scratch bytes gdn_prefill needs for these
+ * sizes (0 when none).  Pure function of its arguments; no device access.
+ */
+GDN_API size_t gdn_prefill_workspace_bytes(int32_t N, int64_t T, int32_t Hqk, int32_t Hv, int32_t Dk,
+                                   int32_t Dv, int32_t chunk);
+
+/*
+ * gdn_decode_step -- one-token inference update of N independent sequences
+ * (section 三 of the page above: "each inference step does one fixed-size
+ * matrix update"), in place on the state.
+ *
+ *   q, k                [N][Hqk][Dk] io_dtype, this step's query and key.
+ *   v                   [N][Hv][Dv]  io_dtype.
+ *   g, beta             fp32 [N][Hv].
+ *   state               fp32 [N][Hv][Dv][Dk], read and overwritten in place.
+ *   o                   [N][Hv][Dv] io_dtype output; must not alias anything.
+ *   dev_error_flag      optional (this call detects no device-side errors
+ *                       today and never writes it).
+ * Supported: Dk in {16, 32, 64, 128}, any Dv >= 1, either dtype.
+ */
+GDN_API gdn_status gdn_decode_step(const void *q, const void *k, const void *v, gdn_dtype io_dtype,
+                           const float *g, const float *beta, float *state, int32_t N,
+                           int32_t Hqk, int32_t Hv, int32_t Dk, int32_t Dv, void *o,
+                           int32_t *dev_error_flag, void *stream);
+
+/* Human-readable name of a status code (static storage, never NULL). */
+GDN_API const char *gdn_status_string(gdn_status status);
+
+/* Library ABI version: major * 10000 + minor * 100 + patch. */
+GDN_API int32_t gdn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_H_ */

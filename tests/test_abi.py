@@ -1,0 +1,143 @@
+"""Host-only checks of the C ABI: the library loads, exports every symbol the
+header declares, and rejects bad arguments synchronously without touching a
+GPU (every call below returns before any CUDA runtime call)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import gated_deltanet_04_b200 as gdn
+from gated_deltanet_04_b200 import build as gdn_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    gdn_build.build()
+    return gdn.library()
+
+
+def declared_functions():
+    names = []
+    for h in os.listdir(os.path.join(ROOT, "include")):
+        if h.endswith(".h"):
+            txt = open(os.path.join(ROOT, "include", h)).read()
+            names += re.findall(r"GDN_API\s+[\w\s\*]+?\b(gdn_\w+)\s*\(", txt)
+    return sorted(set(names))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert {"gdn_prefill", "gdn_decode_step", "gdn_prefill_workspace_bytes",
+            "gdn_status_string", "gdn_version"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), f"libgdn.so does not export {n}"
+
+
+def test_status_strings_and_version(lib):
+    for code, name in gdn.STATUS.items():
+        assert lib.gdn_status_string(code).decode() == name
+    assert lib.gdn_status_string(99).decode() == "GDN_ERR_UNKNOWN"
+    assert lib.gdn_version() >= 10000
+
+
+def test_workspace_bytes_is_pure(lib):
+    a = lib.gdn_prefill_workspace_bytes(1, 262144, 16, 48, 128, 128, 64)
+    b = lib.gdn_prefill_workspace_bytes(1, 262144, 16, 48, 128, 128, 64)
+    assert a == b and a >= 0
+
+
+# fake, 16-byte aligned "device" addresses: validation rejects the call before
+# any of them could be dereferenced
+P = 0x10000
+MIS = 0x10008
+
+
+def prefill(lib, **kw):
+    args = dict(q=P, k=P + 0x1000, v=P + 0x2000, dt=0, g=P + 0x3000, beta=P + 0x4000, s0=None,
+                cu=None, N=1, T=64, Hqk=16, Hv=48, Dk=128, Dv=128, chunk=64, o=P + 0x5000,
+                sT=None, ws=None, wsb=0, err=None, stream=None)
+    args.update(kw)
+    return lib.gdn_prefill(args["q"], args["k"], args["v"], args["dt"], args["g"], args["beta"],
+                           args["s0"], args["cu"], args["N"], args["T"], args["Hqk"], args["Hv"],
+                           args["Dk"], args["Dv"], args["chunk"], args["o"], args["sT"], args["ws"],
+                           args["wsb"], args["err"], args["stream"])
+
+
+INVALID, UNSUPPORTED = 1, 2
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), INVALID),
+    (dict(o=None), INVALID),
+    (dict(g=None), INVALID),
+    (dict(q=MIS), INVALID),
+    (dict(s0=MIS), INVALID),
+    (dict(err=MIS), INVALID),
+    (dict(dt=7), INVALID),
+    (dict(N=-1), INVALID),
+    (dict(T=-5), INVALID),
+    (dict(Hv=47), INVALID),          # Hv % Hqk != 0
+    (dict(Hqk=0), INVALID),
+    (dict(N=2, cu=None), INVALID),   # several sequences need cu_seqlens
+    (dict(o=P), INVALID),            # o aliases q
+    (dict(chunk=-1), INVALID),
+    (dict(Dk=96), UNSUPPORTED),
+    (dict(Dv=256), UNSUPPORTED),
+    (dict(chunk=128), UNSUPPORTED),
+])
+def test_prefill_rejects(lib, kw, code):
+    assert prefill(lib, **kw) == code
+
+
+def test_prefill_nothing_to_do_is_ok(lib):
+    assert prefill(lib, N=0, T=0, cu=P + 0x6000) == 0
+    assert prefill(lib, T=0, sT=None) == 0
+
+
+def decode(lib, **kw):
+    args = dict(q=P, k=P + 0x1000, v=P + 0x2000, dt=0, g=P + 0x3000, beta=P + 0x4000,
+                state=P + 0x7000, N=256, Hqk=16, Hv=48, Dk=128, Dv=128, o=P + 0x5000, err=None,
+                stream=None)
+    args.update(kw)
+    return lib.gdn_decode_step(args["q"], args["k"], args["v"], args["dt"], args["g"],
+                               args["beta"], args["state"], args["N"], args["Hqk"], args["Hv"],
+                               args["Dk"], args["Dv"], args["o"], args["err"], args["stream"])
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(state=None), INVALID),
+    (dict(k=MIS), INVALID),
+    (dict(o=P + 0x7000), INVALID),   # o aliases the state
+    (dict(Hv=40), INVALID),
+    (dict(dt=2), INVALID),
+    (dict(Dk=24), UNSUPPORTED),
+])
+def test_decode_rejects(lib, kw, code):
+    assert decode(lib, **kw) == code
+
+
+def test_decode_empty_batch_is_ok(lib):
+    assert decode(lib, N=0) == 0
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    x = torch.zeros(4, 2, 16)
+    with pytest.raises(ValueError):
+        gdn.gdn_prefill(x, x, x, torch.zeros(4, 2), torch.zeros(4, 2))
+    with pytest.raises(ValueError):
+        gdn.gdn_decode_step(x, x, x, torch.zeros(4, 2), torch.zeros(4, 2), torch.zeros(4, 2, 16, 16))
+
+
+def test_product_path_never_imports_the_oracle():
+    """The library binding and the CUDA sources must not reach the oracle."""
+    pkg = os.path.join(ROOT, "gated_deltanet_04_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                txt = open(os.path.join(dirpath, f), encoding="utf-8").read()
+                assert "import oracle" not in txt and "from oracle" not in txt, f
+                assert "gdn_oracle" not in txt, f

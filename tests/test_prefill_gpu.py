@@ -1,0 +1,207 @@
+"""GPU parity of gdn_prefill against the fp64 oracle (called through the C ABI).
+
+Covers the workloads' own shapes (tiny fp32 heads, one 4096-token layer,
+the 262,144-token layer on sampled heads, the 32-sequence varlen batch with
+split-and-carry), ragged tails around the 64-token chunk, empty sequences,
+in-place state update, and degenerate gates (b = 0, b = 1, a = 1, very strong
+decay, orthonormal keys).  Tolerances: tests/helpers.py.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import gated_deltanet_04_b200 as gdn
+from gated_deltanet_04_b200 import inputs
+from tests.helpers import check_o, check_state
+
+pytestmark = pytest.mark.gpu
+DEV = torch.device("cuda:0")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    from gated_deltanet_04_b200 import build
+    build.build()
+
+
+def run_gpu(inp, s0=None, cu=None, chunk=0, dev=DEV):
+    t = lambda x: None if x is None else x.to(dev).contiguous()
+    o, sT = gdn.gdn_prefill(t(inp["q"]), t(inp["k"]), t(inp["v"]), t(inp["g"]), t(inp["beta"]),
+                            t(s0), None if cu is None else cu.to(torch.int32).to(dev), chunk=chunk)
+    torch.cuda.synchronize()
+    return o.cpu(), sT.cpu()
+
+
+def run_oracle(inp, s0=None, cu=None):
+    return oracle.recurrent(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], s0,
+                            None if cu is None else cu.to(torch.int64))
+
+
+def synth(T, Hqk, Hv, D, dtype, seed, s0_std=0.0, N=1, g_scale=inputs.G_SCALE_097):
+    gen = torch.Generator().manual_seed(seed)
+    q, k, v, g, beta = inputs.make_tokens(T, Hqk, Hv, D, D, dtype, g_scale, gen)
+    s0 = inputs.make_state(N, Hv, D, D, s0_std, gen) if s0_std else None
+    return {"q": q, "k": k, "v": v, "g": g, "beta": beta}, s0
+
+
+def test_tiny_workload_fp32():
+    inp = inputs.make_prefill("tiny")
+    o, sT = run_gpu(inp, chunk=16)
+    o_ref, s_ref = run_oracle(inp)
+    check_o(o, o_ref)
+    check_state(sT, s_ref)
+
+
+def test_layer4k_workload():
+    inp = inputs.make_prefill("layer4k")
+    o, sT = run_gpu(inp, chunk=64)
+    o_ref, s_ref = run_oracle(inp)
+    check_o(o, o_ref)
+    check_state(sT, s_ref)
+
+
+@pytest.mark.parametrize("T", [1, 63, 64, 65, 127, 200, 333])
+def test_ragged_lengths_d128_bf16(T):
+    inp, s0 = synth(T, 2, 6, 128, torch.bfloat16, seed=100 + T, s0_std=0.05)
+    o, sT = run_gpu(inp, s0)
+    o_ref, s_ref = run_oracle(inp, s0)
+    check_o(o, o_ref)
+    check_state(sT, s_ref)
+
+
+@pytest.mark.parametrize("D,dtype", [(16, torch.float32), (32, torch.bfloat16),
+                                     (64, torch.float32), (128, torch.float32)])
+def test_other_head_sizes(D, dtype):
+    inp, s0 = synth(150, 2, 4, D, dtype, seed=200 + D, s0_std=0.05)
+    o, sT = run_gpu(inp, s0)
+    o_ref, s_ref = run_oracle(inp, s0)
+    check_o(o, o_ref)
+    check_state(sT, s_ref)
+
+
+def test_packed_with_empty_sequences_and_in_place_state():
+    lengths = [0, 65, 0, 64, 1, 200, 0]
+    cu = inputs.cu_from_lengths(lengths)
+    inp, s0 = synth(int(cu[-1]), 2, 6, 128, torch.bfloat16, seed=300, s0_std=0.05,
+                    N=len(lengths))
+    o_ref, s_ref = run_oracle(inp, s0, cu)
+    t = lambda x: x.to(DEV).contiguous()
+    state = t(s0)
+    o, sT = gdn.gdn_prefill(t(inp["q"]), t(inp["k"]), t(inp["v"]), t(inp["g"]), t(inp["beta"]),
+                            state, cu.to(torch.int32).to(DEV), final_state=state)
+    torch.cuda.synchronize()
+    assert sT.data_ptr() == state.data_ptr()
+    check_o(o.cpu(), o_ref)
+    check_state(state.cpu(), s_ref)
+    for n, L in enumerate(lengths):
+        if L == 0:  # empty sequence: final state is the initial state, bit for bit
+            assert torch.equal(state[n].cpu(), s0[n])
+
+
+@pytest.mark.parametrize("case", ["b0", "b1", "a1", "strong_decay", "orthonormal_keys"])
+def test_degenerate_gates(case):
+    T, D = 130, 128
+    inp, s0 = synth(T, 1, 3, D, torch.bfloat16, seed=400, s0_std=0.05)
+    if case == "b0":
+        inp["beta"].zero_()
+    elif case == "b1":
+        inp["beta"].fill_(1.0)
+    elif case == "a1":
+        inp["g"].zero_()
+    elif case == "strong_decay":
+        inp["g"].fill_(-30.0)
+    elif case == "orthonormal_keys":
+        gen = torch.Generator().manual_seed(401)
+        basis, _ = torch.linalg.qr(torch.randn(D, D, generator=gen, dtype=torch.float64))
+        idx = torch.arange(T) % D
+        inp["k"] = basis[idx].reshape(T, 1, D).to(torch.bfloat16)
+    o, sT = run_gpu(inp, s0)
+    o_ref, s_ref = run_oracle(inp, s0)
+    check_o(o, o_ref)
+    check_state(sT, s_ref)
+    if case == "b0":  # no writes at all: S_T = exp(sum g) S_0 exactly in exact arithmetic
+        decay = torch.exp(inp["g"].double().sum(0))  # [Hv]
+        want = s0.double() * decay.view(1, -1, 1, 1)
+        np.testing.assert_allclose(sT.double().numpy(), want.numpy(), rtol=2e-5, atol=1e-7)
+
+
+def test_bad_cu_seqlens_sets_flag_without_writing():
+    inp, _ = synth(64, 1, 3, 128, torch.bfloat16, seed=500)
+    t = lambda x: x.to(DEV).contiguous()
+    for bad in ([0, 10, 5, 64], [0, 10, 20, 63], [1, 10, 20, 64]):
+        cu = torch.tensor(bad, dtype=torch.int32, device=DEV)
+        flag = torch.zeros(4, dtype=torch.int32, device=DEV)
+        o = torch.full((64, 3, 128), 7.0, dtype=torch.bfloat16, device=DEV)
+        gdn.gdn_prefill(t(inp["q"]), t(inp["k"]), t(inp["v"]), t(inp["g"]), t(inp["beta"]), None,
+                        cu, o=o, error_flag=flag)
+        torch.cuda.synchronize()
+        assert int(flag[0]) == 5, bad  # GDN_ERR_BAD_SEQLENS
+    # a valid call leaves the flag at zero
+    cu = torch.tensor([0, 10, 20, 64], dtype=torch.int32, device=DEV)
+    flag = torch.zeros(4, dtype=torch.int32, device=DEV)
+    gdn.gdn_prefill(t(inp["q"]), t(inp["k"]), t(inp["v"]), t(inp["g"]), t(inp["beta"]), None,
+                    cu, error_flag=flag)
+    torch.cuda.synchronize()
+    assert int(flag[0]) == 0
+
+
+def test_chunk_length_changes_rounding_only():
+    inp, s0 = synth(300, 2, 6, 128, torch.bfloat16, seed=600, s0_std=0.05)
+    o64, s64 = run_gpu(inp, s0, chunk=64)
+    o16, s16 = run_gpu(inp, s0, chunk=16)
+    check_o(o16, o64.double())
+    check_state(s16, s64.double())
+
+
+def test_varlen32_split_and_carry():
+    """32 packed sequences, lengths U[512,16384], nonzero initial states; every
+    sequence split at a random point and run as two calls carrying the state
+    must match the one-shot run and the oracle (sampled v-heads)."""
+    inp = inputs.make_prefill("varlen32")
+    cu = inputs.cu_from_lengths(inp["lengths"])
+    s0 = inp["s0"]
+    o1, s1 = run_gpu(inp, s0, cu)
+    first, second = inputs.split_packed(inp)
+    oa, sa = run_gpu(first, s0, first["cu_seqlens"])
+    ob, sb = run_gpu(second, sa, second["cu_seqlens"])
+    # reassemble the two halves in the packed order of the one-shot run
+    o2 = torch.empty_like(o1)
+    cua, cub = first["cu_seqlens"].tolist(), second["cu_seqlens"].tolist()
+    for n in range(len(inp["lengths"])):
+        base, sp = int(cu[n]), int(inp["split"][n])
+        o2[base:base + sp] = oa[cua[n]:cua[n + 1]]
+        o2[base + sp:int(cu[n + 1])] = ob[cub[n]:cub[n + 1]]
+    check_o(o2, o1.double(), "segmented vs one-shot o")
+    check_state(sb, s1.double(), "segmented vs one-shot state")
+    heads = [0, 1, 2, 25, 47]  # groups 0, 8, 15 of the 16 q/k heads
+    sub, cols = head_subset(inp, heads)
+    o_ref, s_ref = run_oracle(sub, s0[:, heads], cu)
+    check_o(o1[:, heads], o_ref, "one-shot o, sampled heads")
+    check_state(s1[:, heads], s_ref, "one-shot state, sampled heads")
+    check_o(o2[:, heads], o_ref, "segmented o, sampled heads")
+    check_state(sb[:, heads], s_ref, "segmented state, sampled heads")
+
+
+def head_subset(inp, heads):
+    """Inputs restricted to the given v-heads, each paired with its own q/k head
+    (Hqk = Hv = len(heads) in the result, so the grouping is the identity)."""
+    G = inp["wl"].Hv // inp["wl"].Hqk
+    js = [h // G for h in heads]
+    pick = lambda x, idx: x[:, idx].cpu().contiguous()
+    return ({"q": pick(inp["q"], js), "k": pick(inp["k"], js), "v": pick(inp["v"], heads),
+             "g": pick(inp["g"], heads), "beta": pick(inp["beta"], heads)}, js)
+
+
+def test_long256k_sampled_heads():
+    """The 262,144-token layer, in the bench's launch configuration (inputs drawn
+    on the device by the seeded generator), checked on sampled v-heads."""
+    inp = inputs.make_prefill("long256k", device="cuda")
+    o, sT = gdn.gdn_prefill(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], chunk=64)
+    torch.cuda.synchronize()
+    heads = [0, 29, 47]
+    sub, _ = head_subset(inp, heads)
+    o_ref, s_ref = run_oracle(sub)
+    check_o(o[:, heads].cpu(), o_ref, "o, sampled heads")
+    check_state(sT[:, heads].cpu(), s_ref, "state, sampled heads")
