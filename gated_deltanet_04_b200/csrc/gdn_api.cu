@@ -68,7 +68,7 @@ gdn_status gdn_prefill(const void *q, const void *k, const void *v, gdn_dtype io
     a.o = o; a.sT = final_state; a.err = dev_error_flag; a.T = T; a.N = N; a.Hqk = Hqk;
     a.Hv = Hv; a.Dk = Dk; a.Dv = Dv; a.chunk = chunk == 0 ? 64 : chunk; a.dtype = io_dtype;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (tc_path(io_dtype, Dk, Dv, chunk)) return from_cuda(gdn::launch_prefill_tc(a, s));
+    if (T > 0 && tc_path(io_dtype, Dk, Dv, chunk)) return from_cuda(gdn::launch_prefill_tc(a, s));
     return from_cuda(gdn::launch_prefill_recurrent(a, s));
 }
 
