@@ -21,14 +21,16 @@
 //     accumulation) whose result rows are state rows or chunk rows:
 //       Gram   [K;Q] K^T            -> K K^T (lanes 0-63), Q K^T (lanes 64-127)
 //       U~^T = V^T (T diag b)^T      (T split into fp16 hi + lo: 2 passes)
-//       W^T  = K^T (T diag(b Gamma))^T
-//       S Q^T, R = S W^T             (state times chunk keys/queries)
+//       W^T  = K^T (T diag(b Gamma))^T  (2 passes)
+//       S Q^T, R = S W^T             (R: S and W^T both split, 3 passes)
 //       S   += [U'hi | U'lo] [K ; K] (U' = U diag(Gamma_C/Gamma), split)
 //       U^T P^T                      (P = Q K^T (.) M)
 //     q/k/v tiles arrive by TMA (128-byte swizzle, no multicast) and are
 //     converted in place from bf16 to fp16 (exact for |x| in [6e-5, 6.5e4]).
-//     fp16 operands keep 11 significant bits, so only T diag(b) and U' need
-//     a second (low-part) pass to hold the fp32 state within 1e-4 of fp64.
+//     fp16 operands keep 11 significant bits.  T diag(b), T diag(b Gamma) and
+//     U' get a second (low-part) pass and S W^T three (hi.hi + hi.lo + lo.hi):
+//     without them the rounding of the undecayed (a = 1) state accumulates
+//     past 1e-4 of fp64 within a few chunks.
 //   * The unit lower-triangular solve T = (I + A)^-1 runs on CUDA cores in
 //     fp32 by 16 x 16 blocks.
 //   * Rows past the end of a sequence inside the last chunk are zeroed and
@@ -53,20 +55,25 @@ constexpr long long kWaitLimit = 1ll << 31;  // SM clocks (about a second)
 // ---- shared memory map (bytes from a 1024-aligned base) ----
 constexpr uint32_t OFF_KQ = 0;          // 2 halves x [K 64 rows | Q 64 rows] x 128 B
 constexpr uint32_t OFF_V = 32768;       // 2 halves x 64 rows x 128 B
-constexpr uint32_t OFF_S16 = 49152;     // 2 K-halves x 128 rows x 128 B   (A: S fp16)
-constexpr uint32_t OFF_UP = 81920;      // hi, lo x 128 rows x 128 B       (A: U')
-constexpr uint32_t OFF_U16 = 114688;    // 128 rows x 128 B                 (A: U^T)
-constexpr uint32_t OFF_WST = 131072;    // 128 rows(d) x 128 B              (B: W^T, MN-major)
-constexpr uint32_t OFF_P16 = 147456;    // 64 rows x 128 B                  (B: P, K-major)
-constexpr uint32_t OFF_TBH = 155648;    // 64 rows x 128 B                  (B: T diag b, hi)
-constexpr uint32_t OFF_TBL = 163840;    //                                  (B: T diag b, lo)
-constexpr uint32_t OFF_TBG = 172032;    //                                  (B: T diag(b Gamma))
-constexpr uint32_t OFF_MISC = 180224;
-// the triangular-solve scratch reuses the U'/U16 region (free at that time)
-constexpr uint32_t OFF_AS = OFF_UP;                 // float [64][65]
-constexpr uint32_t OFF_TS = OFF_UP + 64 * 65 * 4;   // float [64][65]
+constexpr uint32_t OFF_S16H = 49152;    // 2 K-halves x 128 rows x 128 B   (A: S fp16 hi)
+constexpr uint32_t OFF_S16L = 81920;    //                                  (A: S fp16 lo)
+// One 48 KB region holds, in turn within a chunk: the triangular-solve
+// scratch, then W^T (hi, lo), then U' (hi, lo) and U^T.  Each use starts
+// only after the MMAs reading the previous one have completed.
+constexpr uint32_t OFF_X = 114688;
+constexpr uint32_t OFF_UP = OFF_X;            // hi, lo x 128 rows x 128 B  (A: U')
+constexpr uint32_t OFF_U16 = OFF_X + 32768;   // 128 rows x 128 B           (A: U^T)
+constexpr uint32_t OFF_WST = OFF_X;           // hi, lo x 128 rows(d) x 128 B (B: W^T, MN-major)
+constexpr uint32_t OFF_AS = OFF_X;                  // float [64][65]
+constexpr uint32_t OFF_TS = OFF_X + 64 * 65 * 4;    // float [64][65]
 constexpr uint32_t OFF_XS = OFF_TS + 64 * 65 * 4;   // float [3][16][16]
-static_assert(OFF_XS + 3 * 256 * 4 <= OFF_WST, "solve scratch overflows");
+constexpr uint32_t OFF_P16 = 163840;    // 64 rows x 128 B                  (B: P, K-major)
+constexpr uint32_t OFF_TBH = 172032;    // 64 rows x 128 B                  (B: T diag b, hi)
+constexpr uint32_t OFF_TBL = 180224;    //                                  (B: T diag b, lo)
+constexpr uint32_t OFF_TGH = 188416;    //                                  (B: T diag(b Gamma), hi)
+constexpr uint32_t OFF_TGL = 196608;    //                                  (B: T diag(b Gamma), lo)
+constexpr uint32_t OFF_MISC = 204800;
+static_assert(OFF_XS + 3 * 256 * 4 <= OFF_P16, "solve scratch overflows");
 
 struct Misc {
     float gam[kC];    // cumulative log-decay within the chunk
@@ -116,6 +123,18 @@ __device__ __forceinline__ uint4 pack8(const float *x) {
 __device__ __forceinline__ void st_row_chunk(uint8_t *tile, uint32_t row, uint32_t chunk,
                                              uint4 val) {
     *reinterpret_cast<uint4 *>(tile + sw128(row, chunk * 16)) = val;
+}
+
+// row i, columns [c, c + 16) of S -> fp16 hi and lo A-operand tiles
+__device__ __forceinline__ void store_state_split(uint8_t *sm, int i, int c, const float *v) {
+    const uint32_t half = (c / 64) * 16384, ch = (c % 64) / 8;
+    uint4 hi, lo;
+    split8(v, hi, lo);
+    st_row_chunk(sm + OFF_S16H + half, i, ch, hi);
+    st_row_chunk(sm + OFF_S16L + half, i, ch, lo);
+    split8(v + 8, hi, lo);
+    st_row_chunk(sm + OFF_S16H + half, i, ch + 1, hi);
+    st_row_chunk(sm + OFF_S16L + half, i, ch + 1, lo);
 }
 
 struct TcParams {
@@ -191,9 +210,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 v[x] = f.x; v[x + 1] = f.y; v[x + 2] = f.z; v[x + 3] = f.w;
             }
             tmem_st16(trow + TM_S + c, v);
-            uint8_t *tile = sm + OFF_S16 + (c / 64) * 16384;
-            st_row_chunk(tile, i, (c % 64) / 8, pack8(v));
-            st_row_chunk(tile, i, (c % 64) / 8 + 1, pack8(v + 8));
+            store_state_split(sm, i, c, v);
         }
         tmem_wait_st();
     }
@@ -376,7 +393,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncthreads();
         }
 
-        // ---- B operands from T: rows r of T diag(b) (hi, lo) and T diag(b Gamma) ----
+        // ---- B operands from T: rows r of T diag(b) and T diag(b Gamma), hi and lo ----
         {
             const int r = tid & 63;
 #pragma unroll 1
@@ -388,19 +405,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const float t = (i <= r) ? Ts[r * 65 + i] : 0.f;
                     x[e] = (tid < kC) ? t * ms->bb[i] : t * ms->bb[i] * ms->Gam[i];
                 }
-                if (tid < kC) {
-                    uint4 hi, lo;
-                    split8(x, hi, lo);
-                    st_row_chunk(sm + OFF_TBH, r, c / 8, hi);
-                    st_row_chunk(sm + OFF_TBL, r, c / 8, lo);
-                } else {
-                    st_row_chunk(sm + OFF_TBG, r, c / 8, pack8(x));
-                }
+                uint4 hi, lo;
+                split8(x, hi, lo);
+                st_row_chunk(sm + (tid < kC ? OFF_TBH : OFF_TGH), r, c / 8, hi);
+                st_row_chunk(sm + (tid < kC ? OFF_TBL : OFF_TGL), r, c / 8, lo);
             }
         }
         publish();
 
-        // ---- U~^T = V^T (T diag b)^T (2 passes), W^T = K^T (T diag(b Gamma))^T, S Q^T ----
+        // ---- U~^T = V^T (T diag b)^T, W^T = K^T (T diag(b Gamma))^T (2 passes each), S Q^T ----
         if (tid == 0) {
 #pragma unroll
             for (int pass = 0; pass < 2; ++pass)
@@ -412,15 +425,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mma_f16_ss(tmem + TM_U, a, b, IDESC_MK_N64, (pass | ks) != 0);
                 }
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-                const uint64_t a = make_sdesc(sbase + OFF_KQ + ks * 2048, 16384, 1024);
-                const uint64_t b = make_sdesc(sbase + OFF_TBG + ks * 32, 16, 1024);
-                mma_f16_ss(tmem + TM_WT, a, b, IDESC_MK_N64, ks > 0);
-            }
+            for (int pass = 0; pass < 2; ++pass)
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks) {
+                    const uint64_t a = make_sdesc(sbase + OFF_KQ + ks * 2048, 16384, 1024);
+                    const uint64_t b =
+                        make_sdesc(sbase + (pass ? OFF_TGL : OFF_TGH) + ks * 32, 16, 1024);
+                    mma_f16_ss(tmem + TM_WT, a, b, IDESC_MK_N64, (pass | ks) != 0);
+                }
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
                 const uint64_t a =
-                    make_sdesc(sbase + OFF_S16 + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
+                    make_sdesc(sbase + OFF_S16H + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
                 const uint64_t b =
                     make_sdesc(sbase + OFF_KQ + (ks >> 2) * 16384 + 8192 + (ks & 3) * 32, 16, 1024);
                 mma_f16_ss(tmem + TM_O, a, b, IDESC_KK_N64, ks > 0);
@@ -428,7 +444,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (mma_sync_point()) { aborted = true; break; }
 
-        // ---- W^T rows -> fp16 B tile (MN-major); master state *= Gamma_C ----
+        // ---- W^T rows -> fp16 hi/lo B tiles (MN-major); master state *= Gamma_C ----
         {
             const float gC = ms->Gam[kC - 1];
 #pragma unroll 1
@@ -436,8 +452,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 float v[16];
                 tmem_ld16(trow + TM_WT + c, v);
                 tmem_wait_ld();
-                st_row_chunk(sm + OFF_WST, tid, c / 8, pack8(v));
-                st_row_chunk(sm + OFF_WST, tid, c / 8 + 1, pack8(v + 8));
+                uint4 hi, lo;
+                split8(v, hi, lo);
+                st_row_chunk(sm + OFF_WST, tid, c / 8, hi);
+                st_row_chunk(sm + OFF_WST + 16384, tid, c / 8, lo);
+                split8(v + 8, hi, lo);
+                st_row_chunk(sm + OFF_WST, tid, c / 8 + 1, hi);
+                st_row_chunk(sm + OFF_WST + 16384, tid, c / 8 + 1, lo);
             }
 #pragma unroll 1
             for (int c = 0; c < kD; c += 16) {
@@ -451,15 +472,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         publish();
 
-        // ---- R = S W^T ----
+        // ---- R = S W^T = Sh Wh^T + Sh Wl^T + Sl Wh^T ----
         if (tid == 0) {
 #pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-                const uint64_t a =
-                    make_sdesc(sbase + OFF_S16 + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
-                const uint64_t b = make_sdesc(sbase + OFF_WST + ks * 2048, 16384, 1024);
-                mma_f16_ss(tmem + TM_R, a, b, IDESC_KM_N64, ks > 0);
-            }
+            for (int pass = 0; pass < 3; ++pass)
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {
+                    const uint32_t s_off = pass == 2 ? OFF_S16L : OFF_S16H;
+                    const uint32_t w_off = pass == 1 ? OFF_WST + 16384 : OFF_WST;
+                    const uint64_t a = make_sdesc(
+                        sbase + s_off + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
+                    const uint64_t b = make_sdesc(sbase + w_off + ks * 2048, 16384, 1024);
+                    mma_f16_ss(tmem + TM_R, a, b, IDESC_KM_N64, (pass | ks) != 0);
+                }
         }
         if (mma_sync_point()) { aborted = true; break; }
 
@@ -510,7 +535,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // next chunk's tiles can land while we finish this one (all MMAs reading them are done)
         if (tid == 0 && c0 + kC < t_end) issue_tma(c0 + kC);
 
-        // ---- o = diag(Gamma) S Q^T + U^T P^T (transposed), new S -> fp16 copy ----
+        // ---- o = diag(Gamma) S Q^T + U^T P^T (transposed), new S -> fp16 hi/lo copies ----
         {
             const int i = tid;
 #pragma unroll 1
@@ -537,9 +562,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 float v[16];
                 tmem_ld16(trow + TM_S + c, v);
                 tmem_wait_ld();
-                uint8_t *tile = sm + OFF_S16 + (c / 64) * 16384;
-                st_row_chunk(tile, i, (c % 64) / 8, pack8(v));
-                st_row_chunk(tile, i, (c % 64) / 8 + 1, pack8(v + 8));
+                store_state_split(sm, i, c, v);
             }
         }
         publish();
