@@ -56,6 +56,10 @@ def parse():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--case", default=None,
+                   help="profiling mode: run one operation of a named workload (layer4k, "
+                        "long256k, varlen32: one gdn_prefill call; decode256: one layer's "
+                        "gdn_decode_step) W + K times and print its per-call time; no bench line")
     return p.parse_args()
 
 
@@ -270,8 +274,34 @@ def run_reference(args, dist):
     return 0
 
 
+def run_case(args):
+    """Profiling mode: W + K calls of one operation on one GPU, per-call device time."""
+    import gated_deltanet_04_b200 as gdn
+    from gated_deltanet_04_b200 import inputs
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream()
+    if args.case == "decode256":
+        L = inputs.make_decode_layer(0, device=dev)
+        out = torch.empty_like(L["v"])
+        fn = lambda: gdn.gdn_decode_step(L["q"], L["k"], L["v"], L["g"], L["beta"], L["state"], o=out)
+    else:
+        inp = inputs.make_prefill(args.case, device=dev)
+        o = torch.empty_like(inp["v"])
+        N = inp["N"]
+        sT = torch.empty((N, inp["wl"].Hv, 128, 128), dtype=torch.float32, device=dev)
+        fn = lambda: gdn.gdn_prefill(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"],
+                                     inp["s0"], inp["cu_seqlens"], chunk=inp["wl"].chunk,
+                                     o=o, final_state=sT)
+    total, each = time_launches(fn, args.steps, args.warmup, Dist(), stream)
+    print(json.dumps({"case": args.case, "calls": args.steps, "ms_per_call": total / args.steps,
+                      "ms_min": min(each), "ms_max": max(each)}), flush=True)
+    return 0
+
+
 def main():
     args = parse()
+    if args.case:
+        return run_case(args)
     dist = Dist()
     if args.impl == "reference":
         dist.init("gloo")
