@@ -12,27 +12,34 @@
 //     O   = diag(Gamma) Q S^T + (Q K^T (.) M) U
 //     S'  = Gamma_C S + U^T diag(Gamma_C / Gamma) K
 //
-// Kernel design (one CTA of 4 warps per (sequence, v-head); thread i <-> TMEM
-// lane i <-> state row i):
+// Kernel design (one CTA of 8 warps per (sequence, v-head)).  TMEM lane i is
+// state row i (or chunk row i); warps w and w + 4 share lane quadrant w % 4
+// and split the columns of every accumulator between them.
 //   * The fp32 state S lives in tensor memory as an MMA accumulator for the
-//     whole sequence (no HBM round trip between chunks).  Its fp16 copy in
-//     shared memory is the A operand of the state-side products.
+//     whole sequence (no HBM round trip between chunks).  Its fp16 hi/lo
+//     copies in shared memory are the A operand of the state-side products.
 //   * Every product is a tcgen05.mma (M = 128, fp16 operands, fp32
 //     accumulation) whose result rows are state rows or chunk rows:
 //       Gram   [K;Q] K^T            -> K K^T (lanes 0-63), Q K^T (lanes 64-127)
 //       U~^T = V^T (T diag b)^T      (T split into fp16 hi + lo: 2 passes)
-//       W^T  = K^T (T diag(b Gamma))^T  (2 passes)
-//       S Q^T, R = S W^T             (R: S and W^T both split, 3 passes)
+//       W^T  = K^T (T diag(b Gamma))^T
+//       S Q^T, R = S W^T             (state times chunk queries / W)
 //       S   += [U'hi | U'lo] [K ; K] (U' = U diag(Gamma_C/Gamma), split)
-//       U^T P^T                      (P = Q K^T (.) M)
+//       O   += U^T P^T               (P = Q K^T (.) M, onto diag(Gamma) S Q^T)
 //     q/k/v tiles arrive by TMA (128-byte swizzle, no multicast) and are
 //     converted in place from bf16 to fp16 (exact for |x| in [6e-5, 6.5e4]).
-//     fp16 operands keep 11 significant bits.  T diag(b), T diag(b Gamma) and
-//     U' get a second (low-part) pass and S W^T three (hi.hi + hi.lo + lo.hi):
-//     without them the rounding of the undecayed (a = 1) state accumulates
-//     past 1e-4 of fp64 within a few chunks.
-//   * The unit lower-triangular solve T = (I + A)^-1 runs on CUDA cores in
-//     fp32 by 16 x 16 blocks.
+//   * Precision: fp16 operands keep 11 significant bits.  T diag(b) and U'
+//     always get a second (low-part) pass.  W and S W^T get extra passes
+//     (W: 2, S W^T: 3 = hi.hi + hi.lo + lo.hi) only in chunks whose total
+//     decay Gamma_C is at least 0.2: a chunk's rounding error is carried into
+//     later chunks scaled by their decay, so it only accumulates when decay
+//     is weak; with the threshold the fp32 state stays within 4e-5 of fp64
+//     in every regime from no decay (a = 1) to the strong decay of the
+//     benchmark workloads (emulated, and checked by the GPU tests).
+//   * The decay factors exp(gamma_r - gamma_i) are formed as
+//     Gamma_r * exp(-gamma_i) when |gamma| <= 60 over the chunk (no overflow),
+//     else elementwise.
+//   * T = (I + A)^-1 is solved on CUDA cores in fp32 by 16 x 16 blocks.
 //   * Rows past the end of a sequence inside the last chunk are zeroed and
 //     get b = g = 0, which makes them contribute nothing.
 // The phases of a chunk run in order, separated by MMA commits; every wait
@@ -42,6 +49,20 @@
 #include "gdn_internal.cuh"
 #include "sm100.cuh"
 
+#ifdef GDN_TC_PHASES
+__device__ long long gdn_tc_phase_clk[16];
+#define GDN_TC_PHASE(k)                                             \
+    do {                                                            \
+        if (threadIdx.x == 0 && blockIdx.x == 0) {                  \
+            const long long now_ = clock64();                       \
+            gdn_tc_phase_clk[(k)] += now_ - phase_t_;               \
+            phase_t_ = now_;                                        \
+        }                                                           \
+    } while (0)
+#else
+#define GDN_TC_PHASE(k) ((void)0)
+#endif
+
 namespace gdn {
 namespace {
 
@@ -49,8 +70,9 @@ using namespace sm100;
 
 constexpr int kC = 64;      // chunk length
 constexpr int kD = 128;     // Dk = Dv
-constexpr int kThreads = 128;
+constexpr int kThreads = 256;
 constexpr long long kWaitLimit = 1ll << 31;  // SM clocks (about a second)
+constexpr float kHighPrecisionDecay = 0.2f;  // Gamma_C at or above -> extra passes
 
 // ---- shared memory map (bytes from a 1024-aligned base) ----
 constexpr uint32_t OFF_KQ = 0;          // 2 halves x [K 64 rows | Q 64 rows] x 128 B
@@ -64,32 +86,39 @@ constexpr uint32_t OFF_X = 114688;
 constexpr uint32_t OFF_UP = OFF_X;            // hi, lo x 128 rows x 128 B  (A: U')
 constexpr uint32_t OFF_U16 = OFF_X + 32768;   // 128 rows x 128 B           (A: U^T)
 constexpr uint32_t OFF_WST = OFF_X;           // hi, lo x 128 rows(d) x 128 B (B: W^T, MN-major)
-constexpr uint32_t OFF_AS = OFF_X;                  // float [64][65]
-constexpr uint32_t OFF_TS = OFF_X + 64 * 65 * 4;    // float [64][65]
-constexpr uint32_t OFF_XS = OFF_TS + 64 * 65 * 4;   // float [3][16][16]
+constexpr int kAS = 65;  // row stride of A (scalar, conflict-free column access)
+constexpr int kTS = 68;  // row stride of T (16-byte aligned rows for float4 access)
+constexpr uint32_t OFF_AS = OFF_X;                   // float [64][kAS]
+constexpr uint32_t OFF_TS = OFF_X + 64 * kAS * 4;       // float [64][kTS], 16-byte aligned
+constexpr uint32_t OFF_XS = OFF_TS + 64 * kTS * 4;   // float [3][16][16]
 constexpr uint32_t OFF_P16 = 163840;    // 64 rows x 128 B                  (B: P, K-major)
 constexpr uint32_t OFF_TBH = 172032;    // 64 rows x 128 B                  (B: T diag b, hi)
 constexpr uint32_t OFF_TBL = 180224;    //                                  (B: T diag b, lo)
 constexpr uint32_t OFF_TGH = 188416;    //                                  (B: T diag(b Gamma), hi)
 constexpr uint32_t OFF_TGL = 196608;    //                                  (B: T diag(b Gamma), lo)
+constexpr uint32_t OFF_OST = OFF_TBH;   // o staging [64 tokens][128] bf16 (TB tiles are dead)
 constexpr uint32_t OFF_MISC = 204800;
 static_assert(OFF_XS + 3 * 256 * 4 <= OFF_P16, "solve scratch overflows");
+static_assert(OFF_TS % 16 == 0 && OFF_XS % 16 == 0, "float4 scratch must be aligned");
 
 struct Misc {
     float gam[kC];    // cumulative log-decay within the chunk
     float Gam[kC];    // exp(gam)
+    float iGam[kC];   // exp(-gam) (only when the chunk is "safe")
     float eC[kC];     // exp(gam_C - gam_r)
     float bb[kC];     // beta (0 for padding rows)
+    float bG[kC];     // beta * Gamma
     uint64_t tma_bar;
     uint64_t mma_bar;
     uint32_t tmem_base;
-    int32_t abort;
+    int32_t safe;     // |gamma| <= 60 over the chunk
+    int32_t hp;       // Gamma_C >= kHighPrecisionDecay
+    float gsum_next;  // sum of g over the next (or first) chunk
 };
 constexpr uint32_t kSmemBytes = OFF_MISC + sizeof(Misc) + 1024;  // + alignment slack
 
-// TMEM column map (fp32 columns; 512 allocated)
-constexpr uint32_t TM_S = 0, TM_G = 128, TM_U = 192, TM_WT = 256, TM_O = 320, TM_R = 384,
-                   TM_P = 448;
+// TMEM column map (fp32 columns; 512 allocated, 448 used)
+constexpr uint32_t TM_S = 0, TM_G = 128, TM_U = 192, TM_WT = 256, TM_O = 320, TM_R = 384;
 
 constexpr uint32_t IDESC_KK_N64 = make_idesc_f16(128, 64, 0, 0);
 constexpr uint32_t IDESC_MK_N64 = make_idesc_f16(128, 64, 1, 0);
@@ -125,16 +154,54 @@ __device__ __forceinline__ void st_row_chunk(uint8_t *tile, uint32_t row, uint32
     *reinterpret_cast<uint4 *>(tile + sw128(row, chunk * 16)) = val;
 }
 
-// row i, columns [c, c + 16) of S -> fp16 hi and lo A-operand tiles
-__device__ __forceinline__ void store_state_split(uint8_t *sm, int i, int c, const float *v) {
-    const uint32_t half = (c / 64) * 16384, ch = (c % 64) / 8;
-    uint4 hi, lo;
-    split8(v, hi, lo);
-    st_row_chunk(sm + OFF_S16H + half, i, ch, hi);
-    st_row_chunk(sm + OFF_S16L + half, i, ch, lo);
-    split8(v + 8, hi, lo);
-    st_row_chunk(sm + OFF_S16H + half, i, ch + 1, hi);
-    st_row_chunk(sm + OFF_S16L + half, i, ch + 1, lo);
+// Writes 32 consecutive values (columns c .. c+31 of row `row`) of a 128-byte
+// swizzled fp16 tile as hi (and, if `with_lo`, lo) parts.
+__device__ __forceinline__ void store_split32(uint8_t *hi_tile, uint8_t *lo_tile, int row, int c,
+                                              const float *v, bool with_lo) {
+#pragma unroll
+    for (int e = 0; e < 32; e += 8) {
+        uint4 hi, lo;
+        split8(v + e, hi, lo);
+        st_row_chunk(hi_tile, row, (c + e) / 8, hi);
+        if (with_lo) st_row_chunk(lo_tile, row, (c + e) / 8, lo);
+    }
+}
+
+// One block-distance level of the triangular inverse (see the solve phase).
+template <int D>
+__device__ __forceinline__ void solve_level(const float *As, float *Ts, float *Xs, int tid) {
+    constexpr int kBlocks = 4 - D;
+    const bool act = tid < kBlocks * 64;
+    const int blk = tid >> 6, r = (tid >> 2) & 15, c4 = 4 * (tid & 3);
+    const int bi = blk + D, bk = blk;
+    if (act) {
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        const float *arow = As + (16 * bi + r) * kAS + 16 * bk;
+        const float *tcol = Ts + (16 * bk) * kTS + 16 * bk + c4;
+#pragma unroll
+        for (int m = 0; m < 16 * D; ++m) {
+            const float a = arow[m];
+            const float4 t = *reinterpret_cast<const float4 *>(tcol + m * kTS);
+            acc.x = fmaf(a, t.x, acc.x); acc.y = fmaf(a, t.y, acc.y);
+            acc.z = fmaf(a, t.z, acc.z); acc.w = fmaf(a, t.w, acc.w);
+        }
+        *reinterpret_cast<float4 *>(Xs + (blk << 8) + r * 16 + c4) = acc;
+    }
+    __syncthreads();
+    if (act) {
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        const float *drow = Ts + (16 * bi + r) * kTS + 16 * bi;
+#pragma unroll
+        for (int m = 0; m < 16; ++m) {
+            const float d = drow[m];
+            const float4 x = *reinterpret_cast<const float4 *>(Xs + (blk << 8) + m * 16 + c4);
+            acc.x = fmaf(d, x.x, acc.x); acc.y = fmaf(d, x.y, acc.y);
+            acc.z = fmaf(d, x.z, acc.z); acc.w = fmaf(d, x.w, acc.w);
+        }
+        *reinterpret_cast<float4 *>(Ts + (16 * bi + r) * kTS + 16 * bk + c4) =
+            make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
+    }
+    __syncthreads();
 }
 
 struct TcParams {
@@ -145,15 +212,14 @@ struct TcParams {
     int32_t *err;
     int64_t T;
     int32_t N, Hqk, Hv;
-    int32_t o_f32;  // o dtype: 0 = bf16, 1 = fp32
 };
 
-// Ends the CTA's work when `bad` is set on any thread: raises the status and
-// returns true for every thread.
-__device__ __forceinline__ bool cta_abort(bool bad, Misc *ms, int32_t *err) {
-    const int any = __syncthreads_or(bad ? 1 : 0);
-    if (any && threadIdx.x == 0) raise_error(err, GDN_ERR_TIMEOUT);
-    return any != 0;
+// Sum over warp 0 of one value per lane (each lane holding the sum of its
+// two gates); lane 0 writes it to *dst.
+__device__ __forceinline__ void warp0_sum_to(float x, float *dst) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+    if (threadIdx.x == 0) *dst = x;
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -167,6 +233,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t sbase = smem_u32(sm);
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
+    const int lane = tid & 31;
+    const int quad = warp & 3;          // TMEM lane quadrant
+    const int half = warp >> 2;         // which half of the columns this warp handles
+    const int row = quad * 32 + lane;   // TMEM lane = accumulator row
+#ifdef GDN_TC_PHASES
+    long long phase_t_ = clock64();
+#endif
 
     const int unit = blockIdx.x;  // n * Hv + h
     const int h = unit % p.Hv;
@@ -179,7 +252,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (tid == 0) {
         mbar_init(&ms->tma_bar, 1);
         mbar_init(&ms->mma_bar, 1);
-        ms->abort = 0;
         fence_mbarrier_init();
         tma_prefetch_desc(&tm_q);
         tma_prefetch_desc(&tm_k);
@@ -189,55 +261,71 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_alloc(&ms->tmem_base, 512);
         tmem_relinquish();
     }
+    // gates of the first chunk (warp 0: lane l holds tokens 2l, 2l+1), and its total decay
+    float gpre0 = 0.f, gpre1 = 0.f, bpre0 = 0.f, bpre1 = 0.f;
+    auto load_gates = [&](int64_t tok0) {
+        gpre0 = gpre1 = bpre0 = bpre1 = 0.f;
+        const int64_t t0_ = tok0 + 2 * lane, t1_ = t0_ + 1;
+        if (t0_ < t_end) { gpre0 = p.g[t0_ * p.Hv + h]; bpre0 = p.beta[t0_ * p.Hv + h]; }
+        if (t1_ < t_end) { gpre1 = p.g[t1_ * p.Hv + h]; bpre1 = p.beta[t1_ * p.Hv + h]; }
+    };
+    if (warp == 0) {
+        load_gates(t_begin);
+        warp0_sum_to(gpre0 + gpre1, &ms->gsum_next);
+    }
     tc_fence_before_sync();
     __syncthreads();
     tc_fence_after_sync();
     const uint32_t tmem = ms->tmem_base;
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;  // this warp's TMEM lanes
-    const uint32_t trow = tmem + lane_off;                  // + column
+    const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);  // + column
 
-    // ---- initial state: S (fp32) -> TMEM accumulator, fp16 copy -> S16 ----
+    // ---- initial state: Gamma_C(first chunk) * S -> TMEM accumulator; S -> fp16 hi/lo ----
     {
-        const int i = tid;
-        const float *src = p.s0 ? p.s0 + (((int64_t)n * p.Hv + h) * kD + i) * kD : nullptr;
+        const float scale0 = t_begin < t_end ? expf(ms->gsum_next) : 1.f;
+        const float *src = p.s0 ? p.s0 + (((int64_t)n * p.Hv + h) * kD + row) * kD : nullptr;
 #pragma unroll 1
-        for (int c = 0; c < kD; c += 16) {
-            float v[16];
+        for (int c = 64 * half; c < 64 * half + 64; c += 32) {
+            float v[32];
 #pragma unroll
-            for (int x = 0; x < 16; x += 4) {
-                float4 f = src ? *reinterpret_cast<const float4 *>(src + c + x)
-                               : make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int x = 0; x < 32; x += 4) {
+                const float4 f = src ? *reinterpret_cast<const float4 *>(src + c + x)
+                                     : make_float4(0.f, 0.f, 0.f, 0.f);
                 v[x] = f.x; v[x + 1] = f.y; v[x + 2] = f.z; v[x + 3] = f.w;
             }
-            tmem_st16(trow + TM_S + c, v);
-            store_state_split(sm, i, c, v);
+            store_split32(sm + OFF_S16H + (c / 64) * 16384, sm + OFF_S16L + (c / 64) * 16384, row,
+                          c % 64, v, true);
+#pragma unroll
+            for (int x = 0; x < 32; ++x) v[x] *= scale0;
+            tmem_st32(trow + TM_S + c, v);
         }
-        tmem_wait_st();
     }
     fence_proxy_async_smem();
+    tmem_wait_st();
     tc_fence_before_sync();
     __syncthreads();
+    tc_fence_after_sync();
 
     uint32_t tma_phase = 0, mma_phase = 0;
     bool aborted = false;
+    bool timed_out = false;  // this thread saw a bounded wait expire (voted on once per chunk)
+    bool tma_outstanding = false;  // a tile load was issued and not yet waited for
 
     auto issue_tma = [&](int64_t tok0) {
         mbar_arrive_expect_tx(&ms->tma_bar, 6 * 8192);
         const int32_t t32 = (int32_t)tok0;
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-            tma_load_3d(sm + OFF_KQ + half * 16384, &tm_k, &ms->tma_bar, 64 * half, j, t32);
-            tma_load_3d(sm + OFF_KQ + half * 16384 + 8192, &tm_q, &ms->tma_bar, 64 * half, j, t32);
-            tma_load_3d(sm + OFF_V + half * 8192, &tm_v, &ms->tma_bar, 64 * half, h, t32);
+        for (int hf = 0; hf < 2; ++hf) {
+            tma_load_3d(sm + OFF_KQ + hf * 16384, &tm_k, &ms->tma_bar, 64 * hf, j, t32);
+            tma_load_3d(sm + OFF_KQ + hf * 16384 + 8192, &tm_q, &ms->tma_bar, 64 * hf, j, t32);
+            tma_load_3d(sm + OFF_V + hf * 8192, &tm_v, &ms->tma_bar, 64 * hf, h, t32);
         }
     };
     // commit the MMAs issued by thread 0, then everyone waits for them
-    auto mma_sync_point = [&]() -> bool {
+    auto mma_sync_point = [&]() {
         if (tid == 0) mma_commit(&ms->mma_bar);
-        const bool ok = mbar_wait_bounded(&ms->mma_bar, mma_phase, kWaitLimit);
+        if (!mbar_wait_bounded(&ms->mma_bar, mma_phase, kWaitLimit)) timed_out = true;
         mma_phase ^= 1;
         tc_fence_after_sync();
-        return cta_abort(!ok, ms, p.err);
     };
     // generic smem / TMEM writes of every thread -> visible to the MMA issuer
     auto publish = [&]() {
@@ -248,50 +336,61 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after_sync();
     };
 
-    if (t_begin < t_end && tid == 0) issue_tma(t_begin);
+    if (t_begin < t_end) {
+        if (tid == 0) issue_tma(t_begin);
+        tma_outstanding = true;
+    }
+    GDN_TC_PHASE(0);
 
 #pragma unroll 1
     for (int64_t c0 = t_begin; c0 < t_end && !aborted; c0 += kC) {
         const int L = (int)((t_end - c0) < kC ? (t_end - c0) : kC);
+        const bool has_next = c0 + kC < t_end;
 
-        // ---- gates of the chunk (threads 0..63), cumulative log-decay ----
-        float gr = 0.f, br = 0.f;
-        if (tid < kC && tid < L) {
-            gr = p.g[(c0 + tid) * p.Hv + h];
-            br = p.beta[(c0 + tid) * p.Hv + h];
-        }
-        if (tid < kC) {
-            float x = gr;  // inclusive scan over 64 lanes (two warps)
+        // ---- gates (warp 0, two tokens per lane): cumulative log-decay, factors, flags ----
+        if (warp == 0) {
+            float x1 = gpre0 + gpre1;  // inclusive scan of pair sums
 #pragma unroll
             for (int off = 1; off < 32; off <<= 1) {
-                const float y = __shfl_up_sync(0xffffffffu, x, off);
-                if ((tid & 31) >= off) x += y;
+                const float y = __shfl_up_sync(0xffffffffu, x1, off);
+                if (lane >= off) x1 += y;
             }
-            ms->gam[tid] = x;  // partial (per warp)
-            ms->bb[tid] = br;
+            const float x0 = x1 - gpre1;  // gamma at token 2l
+            const float gC = __shfl_sync(0xffffffffu, x1, 31);
+            float m = fmaxf(fabsf(x0), fabsf(x1));
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+            const bool safe_ = m <= 60.f;
+            const float G0 = expf(x0), G1 = expf(x1);
+            const int r0 = 2 * lane;
+            ms->gam[r0] = x0;                ms->gam[r0 + 1] = x1;
+            ms->Gam[r0] = G0;                ms->Gam[r0 + 1] = G1;
+            ms->iGam[r0] = safe_ ? expf(-x0) : 0.f;
+            ms->iGam[r0 + 1] = safe_ ? expf(-x1) : 0.f;
+            ms->eC[r0] = expf(gC - x0);      ms->eC[r0 + 1] = expf(gC - x1);
+            ms->bb[r0] = bpre0;              ms->bb[r0 + 1] = bpre1;
+            ms->bG[r0] = bpre0 * G0;         ms->bG[r0 + 1] = bpre1 * G1;
+            if (lane == 0) {
+                ms->safe = safe_;
+                ms->hp = expf(gC) >= kHighPrecisionDecay;
+            }
+            if (has_next) load_gates(c0 + kC);  // prefetch the next chunk's gates
         }
-        __syncthreads();
-        if (tid >= 32 && tid < kC) ms->gam[tid] += ms->gam[31];
-        __syncthreads();
-        if (tid < kC) {
-            const float gm = ms->gam[tid];
-            ms->Gam[tid] = expf(gm);
-            ms->eC[tid] = expf(ms->gam[kC - 1] - gm);
-        }
+        GDN_TC_PHASE(1);
 
         // ---- wait for the tiles, convert bf16 -> fp16 in place, zero padding rows ----
-        {
-            const bool ok = mbar_wait_bounded(&ms->tma_bar, tma_phase, kWaitLimit);
-            tma_phase ^= 1;
-            if (cta_abort(!ok, ms, p.err)) { aborted = true; break; }
-        }
+        if (!mbar_wait_bounded(&ms->tma_bar, tma_phase, kWaitLimit)) timed_out = true;
+        tma_phase ^= 1;
+        tma_outstanding = false;
+        GDN_TC_PHASE(2);
         // 48 KB = 3072 chunks of 16 bytes; row = token index (offset / 128 within each 8 KB box)
-#pragma unroll 4
-        for (int x = tid; x < 3072; x += kThreads) {
+#pragma unroll
+        for (int k = 0; k < 3072 / kThreads; ++k) {
+            const int x = tid + k * kThreads;
             uint4 *ptr = reinterpret_cast<uint4 *>(sm + OFF_KQ) + x;  // KQ and V are contiguous
-            const int row = (x >> 3) & 63;
+            const int r = (x >> 3) & 63;
             uint4 val = *ptr;
-            if (row >= L) {
+            if (r >= L) {
                 val = make_uint4(0u, 0u, 0u, 0u);
             } else {
                 uint32_t w[4] = {val.x, val.y, val.z, val.w};
@@ -306,6 +405,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             *ptr = val;
         }
         publish();
+        const bool hp = ms->hp;
+        const bool safe = ms->safe;
+        GDN_TC_PHASE(3);
 
         // ---- Gram: [K;Q] K^T -> TM_G ----
         if (tid == 0) {
@@ -316,104 +418,95 @@ __global__ void __launch_bounds__(kThreads, 1)
                            IDESC_KK_N64, ks > 0);
             }
         }
-        if (mma_sync_point()) { aborted = true; break; }
+        mma_sync_point();
+        GDN_TC_PHASE(4);
 
-        // ---- A (rows 0..63) and P (rows 64..127) from the Gram rows ----
+        // ---- A (lanes 0..63) and P (lanes 64..127) from the Gram rows ----
         float *As = reinterpret_cast<float *>(sm + OFF_AS);
         float *Ts = reinterpret_cast<float *>(sm + OFF_TS);
         float *Xs = reinterpret_cast<float *>(sm + OFF_XS);
         {
-            const int r = tid & 63;
-            const float gr_ = ms->gam[r];
-            const float br_ = ms->bb[r];
-#pragma unroll 1
-            for (int c = 0; c < kC; c += 16) {
-                float v[16];
-                tmem_ld16(trow + TM_G + c, v);
-                tmem_wait_ld();
-                if (tid < kC) {
+            const int r = row & 63;
+            const int c = 32 * half;
+            float v[32];
+            tmem_ld32(trow + TM_G + c, v);
+            tmem_wait_ld();
+            if (safe) {  // exp(gam_r - gam_i) = Gamma_r * exp(-gam_i), no overflow
+                const float sr = row < kC ? ms->bG[r] : ms->Gam[r];
 #pragma unroll
-                    for (int x = 0; x < 16; ++x) {
-                        const int i = c + x;
-                        As[r * 65 + i] = (i < r) ? br_ * v[x] * expf(gr_ - ms->gam[i]) : 0.f;
-                    }
-                } else {
-                    float pr[16];
+                for (int x = 0; x < 32; ++x) v[x] *= sr * ms->iGam[c + x];
+            } else {
+                const float gr = ms->gam[r];
+                const float sr = row < kC ? ms->bb[r] : 1.f;
 #pragma unroll
-                    for (int x = 0; x < 16; ++x) {
-                        const int i = c + x;
-                        pr[x] = (i <= r) ? v[x] * expf(gr_ - ms->gam[i]) : 0.f;
-                    }
-                    uint8_t *tile = sm + OFF_P16;
-                    st_row_chunk(tile, r, c / 8, pack8(pr));
-                    st_row_chunk(tile, r, c / 8 + 1, pack8(pr + 8));
-                }
+                for (int x = 0; x < 32; ++x) v[x] *= sr * expf(gr - ms->gam[c + x]);
+            }
+            if (row < kC) {  // A = strictly lower part
+#pragma unroll
+                for (int x = 0; x < 32; ++x) As[r * kAS + c + x] = (c + x < r) ? v[x] : 0.f;
+            } else {         // P = lower part including the diagonal
+#pragma unroll
+                for (int x = 0; x < 32; ++x) v[x] = (c + x <= r) ? v[x] : 0.f;
+#pragma unroll
+                for (int e = 0; e < 32; e += 8) st_row_chunk(sm + OFF_P16, r, (c + e) / 8, pack8(v + e));
             }
         }
         __syncthreads();
+        GDN_TC_PHASE(5);
 
         // ---- T = (I + A)^-1 by 16 x 16 blocks (fp32, CUDA cores) ----
-        if (tid < kC) {  // diagonal blocks: thread = (block, column)
+        // Diagonal blocks D_i = (I + A_ii)^-1 by forward substitution, one thread per
+        // (block, column); then, by block distance d = 1..3,
+        //   X = sum_{m = k}^{i-1} A_im T_mk,   T_ik = -D_i X,   i = k + d,
+        // each thread producing four adjacent columns of one row.
+        if (tid < kC) {
             const int bi = tid >> 4, col = tid & 15;
+            const float *Ab = As + (16 * bi) * kAS + 16 * bi;
             float x[16];
 #pragma unroll
             for (int rr = 0; rr < 16; ++rr) {
-                float acc = (rr == col) ? 1.f : 0.f;
+                float a0 = (rr == col) ? 1.f : 0.f, a1 = 0.f;
 #pragma unroll
-                for (int ii = 0; ii < rr; ++ii) acc -= As[(16 * bi + rr) * 65 + 16 * bi + ii] * x[ii];
-                x[rr] = acc;
+                for (int ii = 0; ii + 1 < rr; ii += 2) {
+                    a0 -= Ab[rr * kAS + ii] * x[ii];
+                    a1 -= Ab[rr * kAS + ii + 1] * x[ii + 1];
+                }
+                if (rr & 1) a0 -= Ab[rr * kAS + rr - 1] * x[rr - 1];
+                x[rr] = a0 + a1;
             }
 #pragma unroll
-            for (int rr = 0; rr < 16; ++rr) Ts[(16 * bi + rr) * 65 + 16 * bi + col] = x[rr];
+            for (int rr = 0; rr < 16; ++rr) Ts[(16 * bi + rr) * kTS + 16 * bi + col] = x[rr];
         }
         __syncthreads();
-#pragma unroll 1
-        for (int d = 1; d < 4; ++d) {
-            const int nblk = 4 - d;
-            // X_blk = sum_{m = 16k}^{16i - 1} A[16i + r][m] T[m][16k + c],  i = k + d
-            for (int e = tid; e < nblk * 256; e += kThreads) {
-                const int blk = e >> 8, r = (e >> 4) & 15, c = e & 15;
-                const int bi = blk + d, bk = blk;
-                float acc = 0.f;
-                for (int m = 16 * bk; m < 16 * bi; ++m)
-                    acc += As[(16 * bi + r) * 65 + m] * Ts[m * 65 + 16 * bk + c];
-                Xs[e] = acc;
-            }
-            __syncthreads();
-            // T[16i + r][16k + c] = - sum_m T[16i + r][16i + m] X[m][c]
-            for (int e = tid; e < nblk * 256; e += kThreads) {
-                const int blk = e >> 8, r = (e >> 4) & 15, c = e & 15;
-                const int bi = blk + d, bk = blk;
-                float acc = 0.f;
-#pragma unroll
-                for (int m = 0; m < 16; ++m)
-                    acc += Ts[(16 * bi + r) * 65 + 16 * bi + m] * Xs[(blk << 8) + m * 16 + c];
-                Ts[(16 * bi + r) * 65 + 16 * bk + c] = -acc;
-            }
-            __syncthreads();
-        }
+        solve_level<1>(As, Ts, Xs, tid);
+        solve_level<2>(As, Ts, Xs, tid);
+        solve_level<3>(As, Ts, Xs, tid);
+        GDN_TC_PHASE(6);
 
-        // ---- B operands from T: rows r of T diag(b) and T diag(b Gamma), hi and lo ----
+        // ---- B operands: rows r of T diag(b) and T diag(b Gamma), fp16 hi / lo ----
         {
-            const int r = tid & 63;
-#pragma unroll 1
-            for (int c = 0; c < kC; c += 8) {
-                float x[8];
+            const int grp = tid >> 6, r = tid & 63;
+            const bool tg = grp >= 2;
+            const int c = 32 * (grp & 1);
+            const float *scale = tg ? ms->bG : ms->bb;
+            float x[32];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const int i = c + e;
-                    const float t = (i <= r) ? Ts[r * 65 + i] : 0.f;
-                    x[e] = (tid < kC) ? t * ms->bb[i] : t * ms->bb[i] * ms->Gam[i];
+            for (int e = 0; e < 32; e += 4) {
+                const float4 t4 = *reinterpret_cast<const float4 *>(Ts + r * kTS + c + e);
+                const float tv[4] = {t4.x, t4.y, t4.z, t4.w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int i = c + e + q;
+                    x[e + q] = (i <= r) ? tv[q] * scale[i] : 0.f;
                 }
-                uint4 hi, lo;
-                split8(x, hi, lo);
-                st_row_chunk(sm + (tid < kC ? OFF_TBH : OFF_TGH), r, c / 8, hi);
-                st_row_chunk(sm + (tid < kC ? OFF_TBL : OFF_TGL), r, c / 8, lo);
             }
+            store_split32(sm + (tg ? OFF_TGH : OFF_TBH), sm + (tg ? OFF_TGL : OFF_TBL), r, c, x,
+                          !tg || hp);
         }
         publish();
+        GDN_TC_PHASE(7);
 
-        // ---- U~^T = V^T (T diag b)^T, W^T = K^T (T diag(b Gamma))^T (2 passes each), S Q^T ----
+        // ---- U~^T = V^T (T diag b)^T, W^T = K^T (T diag(b Gamma))^T, S Q^T ----
         if (tid == 0) {
 #pragma unroll
             for (int pass = 0; pass < 2; ++pass)
@@ -424,8 +517,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         make_sdesc(sbase + (pass ? OFF_TBL : OFF_TBH) + ks * 32, 16, 1024);
                     mma_f16_ss(tmem + TM_U, a, b, IDESC_MK_N64, (pass | ks) != 0);
                 }
-#pragma unroll
-            for (int pass = 0; pass < 2; ++pass)
+            for (int pass = 0; pass < (hp ? 2 : 1); ++pass)
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks) {
                     const uint64_t a = make_sdesc(sbase + OFF_KQ + ks * 2048, 16384, 1024);
@@ -442,40 +534,28 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mma_f16_ss(tmem + TM_O, a, b, IDESC_KK_N64, ks > 0);
             }
         }
-        if (mma_sync_point()) { aborted = true; break; }
+        mma_sync_point();
+        GDN_TC_PHASE(8);
 
-        // ---- W^T rows -> fp16 hi/lo B tiles (MN-major); master state *= Gamma_C ----
+        // ---- W^T rows -> fp16 B tiles (MN-major); S Q^T rows scaled by Gamma (in place) ----
         {
-            const float gC = ms->Gam[kC - 1];
-#pragma unroll 1
-            for (int c = 0; c < kC; c += 16) {
-                float v[16];
-                tmem_ld16(trow + TM_WT + c, v);
-                tmem_wait_ld();
-                uint4 hi, lo;
-                split8(v, hi, lo);
-                st_row_chunk(sm + OFF_WST, tid, c / 8, hi);
-                st_row_chunk(sm + OFF_WST + 16384, tid, c / 8, lo);
-                split8(v + 8, hi, lo);
-                st_row_chunk(sm + OFF_WST, tid, c / 8 + 1, hi);
-                st_row_chunk(sm + OFF_WST + 16384, tid, c / 8 + 1, lo);
-            }
-#pragma unroll 1
-            for (int c = 0; c < kD; c += 16) {
-                float v[16];
-                tmem_ld16(trow + TM_S + c, v);
-                tmem_wait_ld();
+            const int c = 32 * half;
+            float v[32];
+            tmem_ld32(trow + TM_WT + c, v);
+            tmem_wait_ld();
+            store_split32(sm + OFF_WST, sm + OFF_WST + 16384, row, c, v, hp);
+            tmem_ld32(trow + TM_O + c, v);
+            tmem_wait_ld();
 #pragma unroll
-                for (int x = 0; x < 16; ++x) v[x] *= gC;
-                tmem_st16(trow + TM_S + c, v);
-            }
+            for (int x = 0; x < 32; ++x) v[x] *= ms->Gam[c + x];
+            tmem_st32(trow + TM_O + c, v);
         }
         publish();
+        GDN_TC_PHASE(9);
 
-        // ---- R = S W^T = Sh Wh^T + Sh Wl^T + Sl Wh^T ----
+        // ---- R = S W^T (hp: Sh Wh^T + Sh Wl^T + Sl Wh^T) ----
         if (tid == 0) {
-#pragma unroll
-            for (int pass = 0; pass < 3; ++pass)
+            for (int pass = 0; pass < (hp ? 3 : 1); ++pass)
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks) {
                     const uint32_t s_off = pass == 2 ? OFF_S16L : OFF_S16H;
@@ -486,35 +566,30 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mma_f16_ss(tmem + TM_R, a, b, IDESC_KM_N64, (pass | ks) != 0);
                 }
         }
-        if (mma_sync_point()) { aborted = true; break; }
+        mma_sync_point();
+        GDN_TC_PHASE(10);
 
         // ---- U = U~ - R (row i of U^T), U' = U diag(Gamma_C/Gamma) split, U fp16 ----
         {
-#pragma unroll 1
-            for (int c = 0; c < kC; c += 16) {
-                float u0[16], r0[16], up[16];
-                tmem_ld16(trow + TM_U + c, u0);
-                tmem_ld16(trow + TM_R + c, r0);
-                tmem_wait_ld();
+            const int c = 32 * half;
+            float u[32], r0[32];
+            tmem_ld32(trow + TM_U + c, u);
+            tmem_ld32(trow + TM_R + c, r0);
+            tmem_wait_ld();
 #pragma unroll
-                for (int x = 0; x < 16; ++x) {
-                    u0[x] -= r0[x];
-                    up[x] = u0[x] * ms->eC[c + x];
-                }
-                uint4 hi, lo;
-                split8(up, hi, lo);
-                st_row_chunk(sm + OFF_UP, tid, c / 8, hi);
-                st_row_chunk(sm + OFF_UP + 16384, tid, c / 8, lo);
-                split8(up + 8, hi, lo);
-                st_row_chunk(sm + OFF_UP, tid, c / 8 + 1, hi);
-                st_row_chunk(sm + OFF_UP + 16384, tid, c / 8 + 1, lo);
-                st_row_chunk(sm + OFF_U16, tid, c / 8, pack8(u0));
-                st_row_chunk(sm + OFF_U16, tid, c / 8 + 1, pack8(u0 + 8));
+            for (int x = 0; x < 32; ++x) {
+                u[x] -= r0[x];
+                r0[x] = u[x] * ms->eC[c + x];
             }
+            store_split32(sm + OFF_UP, sm + OFF_UP + 16384, row, c, r0, true);
+#pragma unroll
+            for (int e = 0; e < 32; e += 8) st_row_chunk(sm + OFF_U16, row, (c + e) / 8, pack8(u + e));
+            if (warp == 0) warp0_sum_to(gpre0 + gpre1, &ms->gsum_next);  // next chunk's log-decay
         }
         publish();
+        GDN_TC_PHASE(11);
 
-        // ---- S += [U'hi | U'lo] [K ; K];  U^T P^T ----
+        // ---- S += [U'hi | U'lo] [K ; K];  O += U^T P^T ----
         if (tid == 0) {
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
@@ -527,64 +602,84 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int ks = 0; ks < 4; ++ks) {
                 const uint64_t a = make_sdesc(sbase + OFF_U16 + ks * 32, 16, 1024);
                 const uint64_t b = make_sdesc(sbase + OFF_P16 + ks * 32, 16, 1024);
-                mma_f16_ss(tmem + TM_P, a, b, IDESC_KK_N64, ks > 0);
+                mma_f16_ss(tmem + TM_O, a, b, IDESC_KK_N64, 1);
             }
         }
-        if (mma_sync_point()) { aborted = true; break; }
-
+        mma_sync_point();
         // next chunk's tiles can land while we finish this one (all MMAs reading them are done)
-        if (tid == 0 && c0 + kC < t_end) issue_tma(c0 + kC);
+        if (has_next) {
+            if (tid == 0) issue_tma(c0 + kC);
+            tma_outstanding = true;
+        }
+        GDN_TC_PHASE(12);
 
-        // ---- o = diag(Gamma) S Q^T + U^T P^T (transposed), new S -> fp16 hi/lo copies ----
+        // ---- o rows -> staging tile; new S -> fp16 hi/lo; master *= Gamma_C(next) ----
         {
-            const int i = tid;
-#pragma unroll 1
-            for (int c = 0; c < kC; c += 16) {
-                float so[16], pu[16];
-                tmem_ld16(trow + TM_O + c, so);
-                tmem_ld16(trow + TM_P + c, pu);
-                tmem_wait_ld();
+            const int c = 32 * half;
+            float v[32];
+            tmem_ld32(trow + TM_O + c, v);
+            tmem_wait_ld();
+            __nv_bfloat16 *ost = reinterpret_cast<__nv_bfloat16 *>(sm + OFF_OST);
 #pragma unroll
-                for (int x = 0; x < 16; ++x) {
-                    const int r = c + x;
-                    if (r < L) {
-                        const float val = fmaf(ms->Gam[r], so[x], pu[x]);
-                        const int64_t idx = ((c0 + r) * p.Hv + h) * (int64_t)kD + i;
-                        if (p.o_f32)
-                            static_cast<float *>(p.o)[idx] = val;
-                        else
-                            static_cast<__nv_bfloat16 *>(p.o)[idx] = __float2bfloat16_rn(val);
-                    }
+            for (int x = 0; x < 32; ++x) ost[(c + x) * kD + row] = __float2bfloat16_rn(v[x]);
+            const float gnext = has_next ? expf(ms->gsum_next) : 1.f;
+            const bool lo_next = gnext >= kHighPrecisionDecay;
+#pragma unroll 1
+            for (int cc = 64 * half; cc < 64 * half + 64; cc += 32) {
+                tmem_ld32(trow + TM_S + cc, v);
+                tmem_wait_ld();
+                store_split32(sm + OFF_S16H + (cc / 64) * 16384, sm + OFF_S16L + (cc / 64) * 16384,
+                              row, cc % 64, v, lo_next);
+                if (has_next) {
+#pragma unroll
+                    for (int x = 0; x < 32; ++x) v[x] *= gnext;
+                    tmem_st32(trow + TM_S + cc, v);
                 }
             }
-#pragma unroll 1
-            for (int c = 0; c < kD; c += 16) {
-                float v[16];
-                tmem_ld16(trow + TM_S + c, v);
-                tmem_wait_ld();
-                store_state_split(sm, i, c, v);
+        }
+        __syncthreads();
+        {
+            const uint4 *ost = reinterpret_cast<const uint4 *>(sm + OFF_OST);
+#pragma unroll
+            for (int k = 0; k < (kC * kD * 2 / 16) / kThreads; ++k) {
+                const int x = tid + k * kThreads;
+                const int r = x >> 4, c16 = x & 15;
+                if (r < L) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.o) +
+                                                           ((c0 + r) * p.Hv + h) * (int64_t)kD) + c16;
+                    *dst = ost[x];
+                }
             }
         }
-        publish();
+        fence_proxy_async_smem();
+        tmem_wait_st();
+        tc_fence_before_sync();
+        if (__syncthreads_or(timed_out ? 1 : 0)) {  // a bounded wait expired: stop here
+            if (tid == 0) raise_error(p.err, GDN_ERR_TIMEOUT);
+            aborted = true;
+        }
+        tc_fence_after_sync();
+        GDN_TC_PHASE(13);
     }
 
     // ---- final state ----
     if (!aborted && p.sT) {
-        float *dst = p.sT + (((int64_t)n * p.Hv + h) * kD + tid) * kD;
+        float *dst = p.sT + (((int64_t)n * p.Hv + h) * kD + row) * kD;
 #pragma unroll 1
-        for (int c = 0; c < kD; c += 16) {
-            float v[16];
-            tmem_ld16(trow + TM_S + c, v);
+        for (int c = 64 * half; c < 64 * half + 64; c += 32) {
+            float v[32];
+            tmem_ld32(trow + TM_S + c, v);
             tmem_wait_ld();
 #pragma unroll
-            for (int x = 0; x < 16; x += 4)
+            for (int x = 0; x < 32; x += 4)
                 *reinterpret_cast<float4 *>(dst + c + x) = make_float4(v[x], v[x + 1], v[x + 2], v[x + 3]);
         }
     }
     if (aborted) {
-        // give MMAs / copies still in flight a bounded chance to drain before freeing TMEM
-        mbar_wait_bounded(&ms->mma_bar, mma_phase, kWaitLimit);
-        mbar_wait_bounded(&ms->tma_bar, tma_phase, kWaitLimit);
+        // Give the last committed MMAs and an outstanding tile load a bounded
+        // chance to drain before TMEM is freed (parities of the latest phases).
+        mbar_wait_bounded(&ms->mma_bar, mma_phase ^ 1, kWaitLimit);
+        if (tma_outstanding) mbar_wait_bounded(&ms->tma_bar, tma_phase, kWaitLimit);
     }
     tc_fence_before_sync();
     __syncthreads();
@@ -638,7 +733,7 @@ cudaError_t launch_prefill_tc(const PrefillArgs &a, cudaStream_t s) {
         return cudaErrorInvalidValue;
     TcParams p;
     p.g = a.g; p.beta = a.beta; p.s0 = a.s0; p.cu = a.cu; p.o = a.o; p.sT = a.sT; p.err = a.err;
-    p.T = a.T; p.N = a.N; p.Hqk = a.Hqk; p.Hv = a.Hv; p.o_f32 = a.dtype == GDN_DTYPE_F32;
+    p.T = a.T; p.N = a.N; p.Hqk = a.Hqk; p.Hv = a.Hv;
     cudaError_t e = cudaFuncSetAttribute(gdn_prefill_tc_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
@@ -648,3 +743,16 @@ cudaError_t launch_prefill_tc(const PrefillArgs &a, cudaStream_t s) {
 }
 
 }  // namespace gdn
+
+#ifdef GDN_TC_PHASES
+extern "C" GDN_API int gdn_debug_tc_phases(long long *out, int n, int reset) {
+    long long host[16];
+    if (cudaMemcpyFromSymbol(host, gdn_tc_phase_clk, sizeof(host)) != cudaSuccess) return -1;
+    for (int i = 0; i < n && i < 16; ++i) out[i] = host[i];
+    if (reset) {
+        const long long zero[16] = {0};
+        cudaMemcpyToSymbol(gdn_tc_phase_clk, zero, sizeof(zero));
+    }
+    return 0;
+}
+#endif
