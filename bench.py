@@ -248,8 +248,7 @@ def run_reference(args, dist):
     """Reference arm: the fp64 CPU oracle, timed as it stands, on rank 0 only."""
     if dist.rank != 0:
         return 0
-    tokens = 2048
-    vals = []
+    tokens = 16384
     for _ in range(args.warmup):
         cpu_baseline_prefill(tokens)
     secs = []
@@ -405,13 +404,13 @@ def main():
                            "unit": "GB/s", "frac": d_gbs_launch / peaks["hbm_gbs"],
                            "traffic": traffic_for("gdn_decode", "decode.cu"),
                            "peak_source": f"{peaks['source']} copy",
-                           "kernel": "gdn_decode_kernel<128>",
+                           "kernel": "gdn_decode_staged_kernel",
                            "algorithmic_bytes_per_launch": state_bytes_layer + io_bytes_layer},
               "frac_of_8TBps": d_state_gbs / dist.world / 8000.0}
 
     cpu = None
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
-        tokens = 4096
+        tokens = 65536
         val, dt, threads = cpu_baseline_prefill(tokens)
         cpu = {"value": val, "unit": "Mtok/s", "cores": threads, "kind": "oracle",
                "sample": f"first {tokens} tokens x 48 heads of the 262,144-token layer, "

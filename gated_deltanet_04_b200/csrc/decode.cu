@@ -11,13 +11,22 @@
 // and q, rewritten and stored by the same lanes, so the kernel is bound by
 // HBM bandwidth on 2 * Dv * Dk * 4 bytes per (n, h).
 //
-// Mapping: one CTA of 8 warps per (n, h).  A row of Dk fp32 values is spread
+// Two kernels:
+//  * Dk = Dv = 128 (the workload shape): a persistent kernel, one CTA per SM,
+//    that streams each 64 KB head state through shared memory with bulk TMA
+//    copies (3 states in flight per SM: loads of the next two overlap the
+//    update of the current one, and the updated state leaves by a bulk store
+//    while the next is computed).  Threads only read and write shared memory.
+//  * other head sizes: the direct kernel below.
+//
+// Direct kernel: one CTA of 8 warps per (n, h).  A row of Dk fp32 values is spread
 // over LPR = Dk/4 lanes as float4 (Dk = 128: a full warp per row, 512
 // contiguous bytes, fully coalesced).  Each warp keeps ROWS_IN_FLIGHT rows
 // loaded before reducing them, so every lane has several independent 16-byte
 // loads outstanding.  Streaming cache hints keep the once-touched state from
 // displacing other data in L2.
 #include "gdn_internal.cuh"
+#include "sm100.cuh"
 
 namespace gdn {
 namespace {
@@ -109,10 +118,156 @@ __global__ void __launch_bounds__(kDecodeWarps * 32)
     }
 }
 
+
+// ---------------------------------------------------------------- staged --
+
+constexpr int kStStages = 3;
+constexpr int kStThreads = 256;                 // 8 warps x 16 state rows
+constexpr uint32_t kStUnitFloats = 128 * 128;   // one (n, h) state
+constexpr uint32_t kStUnitBytes = kStUnitFloats * 4;
+constexpr long long kStWaitLimit = 1ll << 31;   // SM clocks (about a second)
+
+struct StagedSmem {
+    float state[kStStages][kStUnitFloats];
+    float o[2][128];
+    uint64_t full[kStStages];
+};
+constexpr size_t kStSmemBytes = sizeof(StagedSmem) + 128;
+
+struct UnitInputs {
+    float4 k, q;
+    float g, b, v;  // v: lanes 0..15 hold rows 16*warp + lane
+};
+
+__device__ __forceinline__ UnitInputs load_unit_inputs(const DecodeArgs &a, int u, int warp,
+                                                       int lane) {
+    UnitInputs in;
+    const int h = u % a.Hv, n = u / a.Hv;
+    const int j = h / (a.Hv / a.Hqk);
+    const int64_t qk = ((int64_t)n * a.Hqk + j) * 128 + 4 * lane;
+    in.k = load_vec4(a.k, qk, a.dtype);
+    in.q = load_vec4(a.q, qk, a.dtype);
+    in.g = a.g[u];
+    in.b = a.beta[u];
+    in.v = lane < 16 ? load_io(a.v, (int64_t)u * 128 + 16 * warp + lane, a.dtype) : 0.f;
+    return in;
+}
+
+__global__ void __launch_bounds__(kStThreads, 1)
+    gdn_decode_staged_kernel(DecodeArgs a, int units) {
+    using namespace sm100;
+    extern __shared__ uint8_t smem_raw[];
+    StagedSmem &sm = *reinterpret_cast<StagedSmem *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int first = blockIdx.x, stride = gridDim.x;
+    if (first >= units) return;
+    const int count = (units - first + stride - 1) / stride;  // units of this CTA
+
+    if (tid == 0) {
+        for (int s = 0; s < kStStages; ++s) mbar_init(&sm.full[s], 1);
+        fence_mbarrier_init();
+    }
+    __syncthreads();
+    int issued = 0;  // units whose state load has been issued (thread 0's view)
+    if (tid == 0) {
+        for (; issued < count && issued < kStStages; ++issued) {
+            const int u = first + issued * stride;
+            mbar_arrive_expect_tx(&sm.full[issued], kStUnitBytes);
+            bulk_load(sm.state[issued], a.state + (int64_t)u * kStUnitFloats, kStUnitBytes,
+                      &sm.full[issued]);
+        }
+    }
+    UnitInputs nxt = load_unit_inputs(a, first, warp, lane);
+    bool timed_out = false;
+    int li = 0;
+#pragma unroll 1
+    for (; li < count; ++li) {
+        const int u = first + li * stride;
+        const int s = li % kStStages;
+        const UnitInputs cur = nxt;
+        if (li + 1 < count) nxt = load_unit_inputs(a, u + stride, warp, lane);
+        if (!mbar_wait_bounded(&sm.full[s], (li / kStStages) & 1, kStWaitLimit)) timed_out = true;
+
+        const float dec = expf(cur.g);
+        float kq = cur.k.x * cur.q.x + cur.k.y * cur.q.y + cur.k.z * cur.q.z + cur.k.w * cur.q.w;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) kq += __shfl_xor_sync(0xffffffffu, kq, off);
+        float *st = sm.state[s];
+#pragma unroll
+        for (int r0 = 0; r0 < 16; r0 += 4) {
+            float4 row[4];
+            float sk[4], sq[4];
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                row[r] = *reinterpret_cast<const float4 *>(st + (16 * warp + r0 + r) * 128 + 4 * lane);
+                sk[r] = row[r].x * cur.k.x + row[r].y * cur.k.y + row[r].z * cur.k.z + row[r].w * cur.k.w;
+                sq[r] = row[r].x * cur.q.x + row[r].y * cur.q.y + row[r].z * cur.q.z + row[r].w * cur.q.w;
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1)
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    sk[r] += __shfl_xor_sync(0xffffffffu, sk[r], off);
+                    sq[r] += __shfl_xor_sync(0xffffffffu, sq[r], off);
+                }
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                const int i = 16 * warp + r0 + r;
+                const float vi = __shfl_sync(0xffffffffu, cur.v, r0 + r);
+                const float uu = cur.b * (vi - dec * sk[r]);
+                float4 w;
+                w.x = fmaf(uu, cur.k.x, dec * row[r].x);
+                w.y = fmaf(uu, cur.k.y, dec * row[r].y);
+                w.z = fmaf(uu, cur.k.z, dec * row[r].z);
+                w.w = fmaf(uu, cur.k.w, dec * row[r].w);
+                *reinterpret_cast<float4 *>(st + i * 128 + 4 * lane) = w;
+                if (lane == 0) sm.o[li & 1][i] = fmaf(uu, kq, dec * sq[r]);
+            }
+        }
+        fence_proxy_async_smem();  // updated state -> visible to the bulk store
+        if (__syncthreads_or(timed_out ? 1 : 0)) {
+            if (tid == 0) raise_error(a.err, GDN_ERR_TIMEOUT);
+            break;
+        }
+        if (tid < 128) store_io(a.o, (int64_t)u * 128 + tid, sm.o[li & 1][tid], a.dtype);
+        if (tid == 0) {
+            bulk_store(a.state + (int64_t)u * kStUnitFloats, st, kStUnitBytes);
+            bulk_commit();
+            if (issued < count) {  // refill this stage with the unit kStStages ahead
+                bulk_wait_read_all();
+                const int un = first + issued * stride;
+                mbar_arrive_expect_tx(&sm.full[s], kStUnitBytes);
+                bulk_load(st, a.state + (int64_t)un * kStUnitFloats, kStUnitBytes, &sm.full[s]);
+                ++issued;
+            }
+        }
+    }
+    if (tid == 0) {
+        // loads issued but not consumed (only after a timeout): let them land
+        for (int l = li; l < issued; ++l)
+            mbar_wait_bounded(&sm.full[l % kStStages], (l / kStStages) & 1, kStWaitLimit);
+        bulk_wait_all();
+    }
+}
+
 }  // namespace
 
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s) {
-    const dim3 grid((unsigned)((int64_t)a.N * a.Hv));
+    const int units = a.N * a.Hv;
+    if (a.Dk == 128 && a.Dv == 128) {
+        int dev = 0, sms = 0;
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(gdn_decode_staged_kernel,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kStSmemBytes);
+        if (e != cudaSuccess) return e;
+        const int grid = units < sms ? units : sms;
+        gdn_decode_staged_kernel<<<grid, kStThreads, kStSmemBytes, s>>>(a, units);
+        return cudaGetLastError();
+    }
+    const dim3 grid((unsigned)units);
     const dim3 block(kDecodeWarps * 32);
     switch (a.Dk) {
         case 16: gdn_decode_kernel<16><<<grid, block, 0, s>>>(a); break;
