@@ -384,15 +384,15 @@ def main():
                "ms_per_step": e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     # --------------------------------------------------------- roofline --
-    tc_path = True  # Dk = Dv = 128, bf16, chunk 64 -> tensor-core chunked kernel
+    # Dk = Dv = 128, bf16, chunk 64: the library's default is the cluster kernel
     flops = PREFILL_FLOP_PER_TOKEN * T
     achieved_tf = flops / (p_launch_ms / 1e3) / 1e12
     achieved_gbs = PREFILL_BYTES_PER_TOKEN * T / (p_launch_ms / 1e3) / 1e9
     roofline = {"bound": "tensor", "achieved": achieved_tf, "peak": peaks["bf16_tflops"],
                 "unit": "TFLOP/s", "frac": achieved_tf / peaks["bf16_tflops"],
-                "traffic": traffic_for("gdn_prefill_tc", "prefill_tc.cu"),
+                "traffic": traffic_for("gdn_prefill_cluster", "prefill_cluster.cu"),
                 "peak_source": f"{peaks['source']} bf16 burst",
-                "kernel": "gdn_prefill_tc" if tc_path else "gdn_prefill_recurrent",
+                "kernel": "gdn_prefill_cluster_kernel",
                 "algorithmic_flop_per_launch": flops,
                 "hbm": {"achieved": achieved_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                         "frac": achieved_gbs / peaks["hbm_gbs"],

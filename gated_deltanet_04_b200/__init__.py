@@ -20,13 +20,15 @@ import threading
 import torch
 
 __all__ = ["gdn_prefill", "gdn_decode_step", "gdn_prefill_workspace_bytes", "library",
-           "GdnError", "LIB_PATH", "STATUS"]
+           "GdnError", "LIB_PATH", "STATUS", "KERNELS"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgdn.so")
 
 STATUS = {0: "GDN_OK", 1: "GDN_ERR_INVALID_ARGUMENT", 2: "GDN_ERR_UNSUPPORTED", 3: "GDN_ERR_CUDA",
           4: "GDN_ERR_TIMEOUT", 5: "GDN_ERR_BAD_SEQLENS"}
 DTYPE = {torch.bfloat16: 0, torch.float32: 1}
+# gdn_prefill_kernel values of include/gdn.h
+KERNELS = {"auto": 0, "cluster": 1, "single_cta": 2, "recurrent": 3}
 
 _lib = None
 _lock = threading.Lock()
@@ -51,6 +53,8 @@ def library():
             lib.gdn_prefill.argtypes = [vp, vp, vp, ctypes.c_int, vp, vp, vp, vp, i32, i64, i32, i32,
                                         i32, i32, i32, vp, vp, vp, sz, vp, vp]
             lib.gdn_prefill.restype = ctypes.c_int
+            lib.gdn_prefill_ex.argtypes = lib.gdn_prefill.argtypes + [ctypes.c_int]
+            lib.gdn_prefill_ex.restype = ctypes.c_int
             lib.gdn_decode_step.argtypes = [vp, vp, vp, ctypes.c_int, vp, vp, vp, i32, i32, i32, i32,
                                             i32, vp, vp, vp]
             lib.gdn_decode_step.restype = ctypes.c_int
@@ -92,13 +96,14 @@ def gdn_prefill_workspace_bytes(N, T, Hqk, Hv, Dk, Dv, chunk=0):
 
 def gdn_prefill(q, k, v, g, beta, initial_state=None, cu_seqlens=None, *, chunk=0, o=None,
                 final_state=None, output_final_state=True, workspace=None, error_flag=None,
-                stream=None):
+                stream=None, kernel="auto"):
     """Chunk-parallel prefill of the gated delta rule on the GPU.
 
     q, k [T,Hqk,Dk] and v [T,Hv,Dv] (bf16 or fp32, same dtype); g, beta [T,Hv] fp32;
     initial_state [N,Hv,Dv,Dk] fp32 or None; cu_seqlens int32 [N+1] on the device or None.
     Returns (o [T,Hv,Dv], final_state [N,Hv,Dv,Dk] or None).  ``final_state`` may be
     ``initial_state`` for an in-place update.  Asynchronous on the current stream.
+    ``kernel``: "auto", "cluster", "single_cta" or "recurrent" (see gdn_prefill_ex).
     """
     lib = library()
     dev = q.device
@@ -135,10 +140,10 @@ def gdn_prefill(q, k, v, g, beta, initial_state=None, cu_seqlens=None, *, chunk=
         if need:
             workspace = torch.empty(need, dtype=torch.uint8, device=dev)
             ws_bytes = need
-    rc = lib.gdn_prefill(_ptr(q), _ptr(k), _ptr(v), DTYPE[q.dtype], _ptr(g), _ptr(beta),
-                         _ptr(initial_state), _ptr(cu_seqlens), N, T, Hqk, Hv, Dk, Dv, chunk,
-                         _ptr(o), _ptr(final_state), _ptr(workspace), ws_bytes, _ptr(error_flag),
-                         _stream(stream))
+    rc = lib.gdn_prefill_ex(_ptr(q), _ptr(k), _ptr(v), DTYPE[q.dtype], _ptr(g), _ptr(beta),
+                            _ptr(initial_state), _ptr(cu_seqlens), N, T, Hqk, Hv, Dk, Dv, chunk,
+                            _ptr(o), _ptr(final_state), _ptr(workspace), ws_bytes,
+                            _ptr(error_flag), _stream(stream), KERNELS[kernel])
     if rc != 0:
         raise GdnError(rc, "gdn_prefill")
     return o, final_state

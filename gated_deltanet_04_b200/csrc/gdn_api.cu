@@ -46,6 +46,18 @@ gdn_status gdn_prefill(const void *q, const void *k, const void *v, gdn_dtype io
                        int32_t Dk, int32_t Dv, int32_t chunk, void *o, float *final_state,
                        void *workspace, size_t workspace_bytes, int32_t *dev_error_flag,
                        void *stream) {
+    return gdn_prefill_ex(q, k, v, io_dtype, g, beta, initial_state, cu_seqlens, N, T, Hqk, Hv,
+                          Dk, Dv, chunk, o, final_state, workspace, workspace_bytes,
+                          dev_error_flag, stream, GDN_PREFILL_AUTO);
+}
+
+gdn_status gdn_prefill_ex(const void *q, const void *k, const void *v, gdn_dtype io_dtype,
+                          const float *g, const float *beta, const float *initial_state,
+                          const int32_t *cu_seqlens, int32_t N, int64_t T, int32_t Hqk,
+                          int32_t Hv, int32_t Dk, int32_t Dv, int32_t chunk, void *o,
+                          float *final_state, void *workspace, size_t workspace_bytes,
+                          int32_t *dev_error_flag, void *stream, gdn_prefill_kernel kernel) {
+    if (kernel < GDN_PREFILL_AUTO || kernel > GDN_PREFILL_RECURRENT) return GDN_ERR_INVALID_ARGUMENT;
     if (io_dtype != GDN_DTYPE_BF16 && io_dtype != GDN_DTYPE_F32) return GDN_ERR_INVALID_ARGUMENT;
     if (N < 0 || T < 0 || Hqk <= 0 || Hv <= 0 || Dk <= 0 || Dv <= 0 || chunk < 0)
         return GDN_ERR_INVALID_ARGUMENT;
@@ -68,8 +80,13 @@ gdn_status gdn_prefill(const void *q, const void *k, const void *v, gdn_dtype io
     a.o = o; a.sT = final_state; a.err = dev_error_flag; a.T = T; a.N = N; a.Hqk = Hqk;
     a.Hv = Hv; a.Dk = Dk; a.Dv = Dv; a.chunk = chunk == 0 ? 64 : chunk; a.dtype = io_dtype;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (T > 0 && tc_path(io_dtype, Dk, Dv, chunk)) return from_cuda(gdn::launch_prefill_tc(a, s));
-    return from_cuda(gdn::launch_prefill_recurrent(a, s));
+    const bool tc_ok = tc_path(io_dtype, Dk, Dv, chunk);
+    if ((kernel == GDN_PREFILL_CLUSTER || kernel == GDN_PREFILL_SINGLE_CTA) && !tc_ok)
+        return GDN_ERR_UNSUPPORTED;
+    if (kernel == GDN_PREFILL_AUTO) kernel = tc_ok ? GDN_PREFILL_CLUSTER : GDN_PREFILL_RECURRENT;
+    if (T == 0 || kernel == GDN_PREFILL_RECURRENT) return from_cuda(gdn::launch_prefill_recurrent(a, s));
+    if (kernel == GDN_PREFILL_SINGLE_CTA) return from_cuda(gdn::launch_prefill_tc(a, s));
+    return from_cuda(gdn::launch_prefill_cluster(a, s));
 }
 
 gdn_status gdn_decode_step(const void *q, const void *k, const void *v, gdn_dtype io_dtype,

@@ -36,8 +36,10 @@ struct DecodeArgs {
 // Host launchers (return cudaGetLastError() of the launch).
 cudaError_t launch_prefill_recurrent(const PrefillArgs &a, cudaStream_t s);
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s);
-// Tensor-core chunked prefill, Dk = Dv = 128, bf16, chunk 64.
+// Tensor-core chunked prefill, Dk = Dv = 128, bf16, chunk 64: one CTA per
+// (sequence, head), or a 3-CTA cluster per (sequence, head).
 cudaError_t launch_prefill_tc(const PrefillArgs &a, cudaStream_t s);
+cudaError_t launch_prefill_cluster(const PrefillArgs &a, cudaStream_t s);
 
 // ---------------------------------------------------------------- device --
 

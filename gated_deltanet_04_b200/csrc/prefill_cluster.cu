@@ -1,0 +1,738 @@
+// Chunk-parallel prefill of the gated delta rule on a 3-CTA thread-block
+// cluster per (sequence, v-head).
+//
+// The math is the chunk step of the single-CTA kernel (see prefill_tc.cu):
+//     A = strict-lower(diag(b)(K K^T (.) M)),   T = (I + A)^-1
+//     U~ = T diag(b) V,   W = T diag(b Gamma) K,   U = U~ - W S^T
+//     O = diag(Gamma) Q S^T + (Q K^T (.) M) U,   S' = Gamma_C S + U^T diag(Gamma_C/Gamma) K
+// from the rule of page "Qwen3.8-27B 架构深读: Gated DeltaNet 混合线性注意力与 262K
+// 长上下文", section 三.  Only U (through S) links one chunk to the next; every
+// other quantity of a chunk depends on that chunk's inputs alone.
+//
+// Work split (one SM per CTA):
+//   * rank 0, the chain CTA, keeps the fp32 state as a TMEM accumulator and
+//     its fp16 hi/lo copies as TMEM A operands, and runs only the state-
+//     dependent products of each chunk: S Q^T, R = S W^T, U = U~ - R, the state
+//     update S += U'^T K, O += U^T P^T, and the output stores.
+//   * ranks 1 and 2, the producer CTAs, take alternate chunks (rank 1 even,
+//     rank 2 odd): TMA tile loads, bf16 -> fp16, Gram matrices, decay factors,
+//     the triangular solve, U~ and W on tensor cores.  Each finished chunk
+//     (K, Q, W^T hi/lo, U~, P, gates: up to 105 KB) is copied by bulk copies
+//     into one of two hand-off slots in the chain CTA's shared memory.
+// With the producers a chunk ahead, the chain CTA's per-chunk time is its own
+// chain of two MMA groups and two row epilogues.
+//
+// Flow control (all mbarrier waits bounded; a wait that expires is voted on
+// once per chunk, reports GDN_ERR_TIMEOUT and ends the CTA's loop):
+//   full[k]  (chain)    : producer k's expect-tx arrival + its bulk copies
+//   copied   (producer) : the chain received the producer's last delivery, so
+//                         the producer may reuse its tile buffers and staging
+//   freed    (producer) : the chain finished the chunk in slot k
+// A cluster barrier after set-up and another before exit keep every CTA's
+// shared memory alive while the others may still address it.  No TMA load
+// uses multicast.
+#include <mutex>
+
+#include "gdn_internal.cuh"
+#include "sm100.cuh"
+#include "tc_common.cuh"
+
+namespace gdn {
+namespace {
+
+using namespace sm100;
+using namespace tc;
+
+constexpr int kThreads = 256;
+constexpr int kCluster = 3;
+
+// ---- chain CTA: two hand-off slots (offsets inside a slot) ----
+constexpr uint32_t SL_K16 = 0;         // K fp16: d-halves at +0 / +8192 ([64 rows][128 B], SW128)
+constexpr uint32_t SL_Q16 = 16384;     // Q fp16, same layout
+constexpr uint32_t SL_WH = 32768;      // W^T hi, MN-major [128 d][128 B]
+constexpr uint32_t SL_WL = 49152;      // W^T lo
+constexpr uint32_t SL_UT = 65536;      // U~^T fp32 [128 rows][64], 16-byte chunks XOR-swizzled by row
+constexpr uint32_t SL_P16 = 98304;     // P fp16 [64 rows][128 B], SW128
+constexpr uint32_t SL_GATES = 106496;  // GatesBlock
+constexpr uint32_t SLOT_BYTES = 107520;
+// reuse of a slot's regions once the chain has consumed them
+constexpr uint32_t SL_UP = SL_UT;      // U' hi then lo (K-major A operand), after U~ is read
+constexpr uint32_t SL_U16 = SL_WH;     // U^T fp16 (K-major A operand), after R
+constexpr uint32_t SL_OST = SL_Q16;    // o staging [64 tokens][128] bf16, after S Q^T
+constexpr uint32_t C_MISC = 2 * SLOT_BYTES;
+
+struct GatesBlock {
+    float Gam[kC];   // exp(gamma_r)
+    float eC[kC];    // exp(gamma_C - gamma_r)
+    int32_t hp;      // extra precision passes for this chunk
+    int32_t pad[3];
+};
+static_assert(sizeof(GatesBlock) % 16 == 0, "bulk copies move multiples of 16 bytes");
+
+struct ChainMisc {
+    uint64_t full[2];
+    uint64_t mma_bar;
+    uint32_t tmem_base;
+};
+
+// chain TMEM columns (512 allocated)
+constexpr uint32_t CT_S = 0, CT_SH = 128, CT_SL = 192, CT_R = 256, CT_O = 320;
+
+// ---- producer CTA ----
+constexpr uint32_t P_KQV = 0;           // 2 buffers: [K|Q] d-half 0, [K|Q] d-half 1, V halves
+constexpr uint32_t P_KQV_BYTES = 49152;
+constexpr uint32_t P_X = 98304;         // 48 KB: solve scratch, then W^T hi/lo + gates staging
+constexpr uint32_t P_WST = P_X;
+constexpr uint32_t P_GST = P_X + 32768;
+constexpr uint32_t P_AS = P_X;
+constexpr uint32_t P_TS = P_X + 64 * kAS * 4;
+constexpr uint32_t P_XS = P_TS + 64 * kTS * 4;
+constexpr uint32_t P_UTS = 147456;      // U~^T staging (same layout as SL_UT)
+constexpr uint32_t P_P16 = 180224;
+constexpr uint32_t P_TBH = 188416, P_TBL = 196608, P_TGH = 204800, P_TGL = 212992;
+constexpr uint32_t P_MISC = 221184;
+static_assert(P_XS + 3 * 256 * 4 <= P_UTS, "solve scratch overflows");
+static_assert(P_GST >= P_XS + 3 * 256 * 4 || P_GST + sizeof(GatesBlock) <= P_X + 49152,
+              "gates staging stays inside the scratch region");
+static_assert(P_TS % 16 == 0 && P_XS % 16 == 0, "float4 scratch must be aligned");
+
+struct ProdMisc {
+    float gam[kC], Gam[kC], iGam[kC], eC[kC], bb[kC], bG[kC];
+    uint64_t tma_bar[2];
+    uint64_t mma_bar;
+    uint64_t copied;
+    uint64_t freed;
+    uint32_t tmem_base;
+    int32_t safe, hp;
+    float gsum;
+};
+constexpr uint32_t kSmemBytes = P_MISC + sizeof(ProdMisc) + 1024;
+static_assert(C_MISC + sizeof(ChainMisc) <= P_MISC + sizeof(ProdMisc), "chain misc fits");
+
+// producer TMEM columns (128 allocated)
+constexpr uint32_t PT_G = 0, PT_U = 64;
+
+struct ClusterParams {
+    const float *g, *beta, *s0;
+    const int32_t *cu;
+    void *o;
+    float *sT;
+    int32_t *err;
+    int64_t T;
+    int32_t N, Hqk, Hv;
+};
+
+// byte offset of 16-byte chunk q of row i in a [128][64] fp32 U~ tile
+__device__ __forceinline__ uint32_t ut_off(int i, int q) {
+    return (uint32_t)i * 256u + (uint32_t)((q ^ (i & 15)) << 4);
+}
+
+// ------------------------------------------------------------- producer --
+
+__device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtensorMap *tm_k,
+                              const CUtensorMap *tm_v, const ClusterParams &p, int k, int h,
+                              int j, int64_t t_begin, int64_t t_end, int nch) {
+    ProdMisc *ms = reinterpret_cast<ProdMisc *>(sm + P_MISC);
+    const uint32_t sbase = smem_u32(sm);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quad = warp & 3, half = warp >> 2, row = quad * 32 + lane;
+    const uint32_t tmem = ms->tmem_base;
+    const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
+    // chain-CTA addresses (rank 0)
+    const uint32_t c_base = mapa_shared(sbase, 0);
+    const uint32_t c_full = mapa_shared(sbase + C_MISC + (uint32_t)offsetof(ChainMisc, full) + 8u * k, 0);
+    const int nmine = nch > k ? (nch - k + 1) / 2 : 0;
+
+    uint32_t mma_phase = 0;
+    bool timed_out = false;
+    float gpre0 = 0.f, gpre1 = 0.f, bpre0 = 0.f, bpre1 = 0.f;
+    auto load_gates = [&](int64_t tok0) {
+        gpre0 = gpre1 = bpre0 = bpre1 = 0.f;
+        const int64_t t0_ = tok0 + 2 * lane, t1_ = t0_ + 1;
+        if (t0_ < t_end) { gpre0 = p.g[t0_ * p.Hv + h]; bpre0 = p.beta[t0_ * p.Hv + h]; }
+        if (t1_ < t_end) { gpre1 = p.g[t1_ * p.Hv + h]; bpre1 = p.beta[t1_ * p.Hv + h]; }
+    };
+    auto issue_tma = [&](int buf, int64_t tok0) {
+        uint8_t *b = sm + P_KQV + buf * P_KQV_BYTES;
+        mbar_arrive_expect_tx(&ms->tma_bar[buf], 6 * 8192);
+        const int32_t t32 = (int32_t)tok0;
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+            tma_load_3d(b + hf * 16384, tm_k, &ms->tma_bar[buf], 64 * hf, j, t32);
+            tma_load_3d(b + hf * 16384 + 8192, tm_q, &ms->tma_bar[buf], 64 * hf, j, t32);
+            tma_load_3d(b + 32768 + hf * 8192, tm_v, &ms->tma_bar[buf], 64 * hf, h, t32);
+        }
+    };
+    auto mma_sync_point = [&]() {
+        if (tid == 0) mma_commit(&ms->mma_bar);
+        if (!mbar_wait_bounded(&ms->mma_bar, mma_phase, kWaitLimit)) timed_out = true;
+        mma_phase ^= 1;
+        tc_fence_after_sync();
+    };
+    auto publish = [&]() {
+        fence_proxy_async_smem();
+        tmem_wait_st();
+        tc_fence_before_sync();
+        __syncthreads();
+        tc_fence_after_sync();
+    };
+
+    int tma_issued = 0;  // tile loads issued (local chunk indices 0 .. tma_issued-1)
+    if (nmine > 0) {
+        if (tid == 0) issue_tma(0, t_begin + (int64_t)kC * k);
+        tma_issued = 1;
+        if (warp == 0) load_gates(t_begin + (int64_t)kC * k);
+    }
+    int jj = 0;
+#pragma unroll 1
+    for (; jj < nmine; ++jj) {
+        const int c = k + 2 * jj;
+        const int64_t c0 = t_begin + (int64_t)kC * c;
+        const int L = (int)((t_end - c0) < kC ? (t_end - c0) : kC);
+        const int buf = jj & 1;
+        const bool more = jj + 1 < nmine;
+
+        // ---- gates (warp 0, two tokens per lane) ----
+        if (warp == 0) {
+            float x1 = gpre0 + gpre1;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const float y = __shfl_up_sync(0xffffffffu, x1, off);
+                if (lane >= off) x1 += y;
+            }
+            const float x0 = x1 - gpre1;
+            const float gC = __shfl_sync(0xffffffffu, x1, 31);
+            float m = fmaxf(fabsf(x0), fabsf(x1));
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+            const bool safe_ = m <= 60.f;
+            const float G0 = expf(x0), G1 = expf(x1);
+            const int r0 = 2 * lane;
+            ms->gam[r0] = x0;                ms->gam[r0 + 1] = x1;
+            ms->Gam[r0] = G0;                ms->Gam[r0 + 1] = G1;
+            ms->iGam[r0] = safe_ ? expf(-x0) : 0.f;
+            ms->iGam[r0 + 1] = safe_ ? expf(-x1) : 0.f;
+            ms->eC[r0] = expf(gC - x0);      ms->eC[r0 + 1] = expf(gC - x1);
+            ms->bb[r0] = bpre0;              ms->bb[r0 + 1] = bpre1;
+            ms->bG[r0] = bpre0 * G0;         ms->bG[r0 + 1] = bpre1 * G1;
+            if (lane == 0) {
+                ms->safe = safe_;
+                ms->hp = expf(gC) >= kHighPrecisionDecay;
+            }
+            if (more) load_gates(c0 + 2 * kC);
+        }
+
+        // ---- the chain has taken our previous delivery: buffers and staging are free ----
+        if (jj >= 1 && !mbar_wait_cluster_bounded(&ms->copied, (jj - 1) & 1, kWaitLimit))
+            timed_out = true;
+        if (more) {
+            if (tid == 0) issue_tma(buf ^ 1, c0 + 2 * kC);
+            tma_issued = jj + 2;
+        }
+        if (!mbar_wait_bounded(&ms->tma_bar[buf], (jj >> 1) & 1, kWaitLimit)) timed_out = true;
+
+        // ---- bf16 -> fp16 in place, zero padding rows ----
+        uint8_t *kqv = sm + P_KQV + buf * P_KQV_BYTES;
+        const uint32_t skqv = sbase + P_KQV + buf * P_KQV_BYTES;
+#pragma unroll
+        for (int q = 0; q < 3072 / kThreads; ++q) {
+            const int x = tid + q * kThreads;
+            uint4 *ptr = reinterpret_cast<uint4 *>(kqv) + x;
+            const int r = (x >> 3) & 63;
+            uint4 val = *ptr;
+            if (r >= L) {
+                val = make_uint4(0u, 0u, 0u, 0u);
+            } else {
+                uint32_t w[4] = {val.x, val.y, val.z, val.w};
+#pragma unroll
+                for (int q2 = 0; q2 < 4; ++q2) {
+                    const __nv_bfloat162 b2 = *reinterpret_cast<const __nv_bfloat162 *>(&w[q2]);
+                    const float2 f = __bfloat1622float2(b2);
+                    w[q2] = pack_half2(f.x, f.y);
+                }
+                val = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+            *ptr = val;
+        }
+        publish();
+        const bool hp = ms->hp;
+        const bool safe = ms->safe;
+
+        // ---- Gram: [K;Q] K^T ----
+        if (tid == 0) {
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                const uint32_t a = skqv + (ks >> 2) * 16384 + (ks & 3) * 32;
+                mma_f16_ss(tmem + PT_G, make_sdesc(a, 16, 1024), make_sdesc(a, 16, 1024),
+                           IDESC_KK_N64, ks > 0);
+            }
+        }
+        mma_sync_point();
+
+        // ---- A (lanes 0..63) and P (lanes 64..127) ----
+        float *As = reinterpret_cast<float *>(sm + P_AS);
+        float *Ts = reinterpret_cast<float *>(sm + P_TS);
+        float *Xs = reinterpret_cast<float *>(sm + P_XS);
+        {
+            const int r = row & 63;
+            const int c = 32 * half;
+            float v[32];
+            tmem_ld32(trow + PT_G + c, v);
+            tmem_wait_ld();
+            if (safe) {
+                const float sr = row < kC ? ms->bG[r] : ms->Gam[r];
+#pragma unroll
+                for (int x = 0; x < 32; ++x) v[x] *= sr * ms->iGam[c + x];
+            } else {
+                const float gr = ms->gam[r];
+                const float sr = row < kC ? ms->bb[r] : 1.f;
+#pragma unroll
+                for (int x = 0; x < 32; ++x) v[x] *= sr * expf(gr - ms->gam[c + x]);
+            }
+            if (row < kC) {
+#pragma unroll
+                for (int x = 0; x < 32; ++x) As[r * kAS + c + x] = (c + x < r) ? v[x] : 0.f;
+            } else {
+#pragma unroll
+                for (int x = 0; x < 32; ++x) v[x] = (c + x <= r) ? v[x] : 0.f;
+#pragma unroll
+                for (int e = 0; e < 32; e += 8) st_row_chunk(sm + P_P16, r, (c + e) / 8, pack8(v + e));
+            }
+        }
+        __syncthreads();
+
+        // ---- T = (I + A)^-1 ----
+        if (tid < kC) {
+            const int bi = tid >> 4, col = tid & 15;
+            const float *Ab = As + (16 * bi) * kAS + 16 * bi;
+            float x[16];
+#pragma unroll
+            for (int rr = 0; rr < 16; ++rr) {
+                float a0 = (rr == col) ? 1.f : 0.f, a1 = 0.f;
+#pragma unroll
+                for (int ii = 0; ii + 1 < rr; ii += 2) {
+                    a0 -= Ab[rr * kAS + ii] * x[ii];
+                    a1 -= Ab[rr * kAS + ii + 1] * x[ii + 1];
+                }
+                if (rr & 1) a0 -= Ab[rr * kAS + rr - 1] * x[rr - 1];
+                x[rr] = a0 + a1;
+            }
+#pragma unroll
+            for (int rr = 0; rr < 16; ++rr) Ts[(16 * bi + rr) * kTS + 16 * bi + col] = x[rr];
+        }
+        __syncthreads();
+        solve_level<1>(As, Ts, Xs, tid);
+        solve_level<2>(As, Ts, Xs, tid);
+        solve_level<3>(As, Ts, Xs, tid);
+
+        // ---- rows of T diag(b), T diag(b Gamma): fp16 hi / lo ----
+        {
+            const int grp = tid >> 6, r = tid & 63;
+            const bool tg = grp >= 2;
+            const int c = 32 * (grp & 1);
+            const float *scale = tg ? ms->bG : ms->bb;
+            float x[32];
+#pragma unroll
+            for (int e = 0; e < 32; e += 4) {
+                const float4 t4 = *reinterpret_cast<const float4 *>(Ts + r * kTS + c + e);
+                const float tv[4] = {t4.x, t4.y, t4.z, t4.w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int i = c + e + q;
+                    x[e + q] = (i <= r) ? tv[q] * scale[i] : 0.f;
+                }
+            }
+            store_split32(sm + (tg ? P_TGH : P_TBH), sm + (tg ? P_TGL : P_TBL), r, c, x, !tg || hp);
+        }
+        publish();
+
+        // ---- U~^T = V^T (T diag b)^T,  W^T = K^T (T diag(b Gamma))^T ----
+        if (tid == 0) {
+#pragma unroll
+            for (int pass = 0; pass < 2; ++pass)
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks) {
+                    const uint64_t a = make_sdesc(skqv + 32768 + ks * 2048, 8192, 1024);
+                    const uint64_t b = make_sdesc(sbase + (pass ? P_TBL : P_TBH) + ks * 32, 16, 1024);
+                    mma_f16_ss(tmem + PT_U, a, b, IDESC_MK_N64, (pass | ks) != 0);
+                }
+            for (int pass = 0; pass < (hp ? 2 : 1); ++pass)
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks) {
+                    const uint64_t a = make_sdesc(skqv + ks * 2048, 16384, 1024);
+                    const uint64_t b = make_sdesc(sbase + (pass ? P_TGL : P_TGH) + ks * 32, 16, 1024);
+                    mma_f16_ss(tmem + PT_G, a, b, IDESC_MK_N64, (pass | ks) != 0);
+                }
+        }
+        mma_sync_point();
+
+        // ---- staging: W^T hi/lo (MN-major), U~^T (swizzled fp32), gates ----
+        {
+            const int c = 32 * half;
+            float v[32];
+            tmem_ld32(trow + PT_G + c, v);
+            tmem_wait_ld();
+            store_split32(sm + P_WST, sm + P_WST + 16384, row, c, v, hp);
+            tmem_ld32(trow + PT_U + c, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                *reinterpret_cast<float4 *>(sm + P_UTS + ut_off(row, c / 4 + q)) =
+                    make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+            GatesBlock *gs = reinterpret_cast<GatesBlock *>(sm + P_GST);
+            if (tid < kC) {
+                gs->Gam[tid] = ms->Gam[tid];
+                gs->eC[tid] = ms->eC[tid];
+            }
+            if (tid == 0) gs->hp = hp;
+        }
+        fence_proxy_async_smem();  // staged data -> visible to the bulk copies
+        __syncthreads();
+
+        // ---- deliver into slot k of the chain CTA, once it is free ----
+        if (jj >= 1 && !mbar_wait_cluster_bounded(&ms->freed, (jj - 1) & 1, kWaitLimit))
+            timed_out = true;
+        if (__syncthreads_or(timed_out ? 1 : 0)) {
+            if (tid == 0) raise_error(p.err, GDN_ERR_TIMEOUT);
+            break;
+        }
+        if (tid == 0) {
+            const uint32_t slot = c_base + (uint32_t)k * SLOT_BYTES;
+            const uint32_t bytes = 4 * 8192 + 16384 * (hp ? 2 : 1) + 32768 + 8192 +
+                                   (uint32_t)sizeof(GatesBlock);
+            mbar_arrive_expect_tx_remote(c_full, bytes);
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                bulk_copy_to_cluster(slot + SL_K16 + hf * 8192, kqv + hf * 16384, 8192, c_full);
+                bulk_copy_to_cluster(slot + SL_Q16 + hf * 8192, kqv + hf * 16384 + 8192, 8192, c_full);
+            }
+            bulk_copy_to_cluster(slot + SL_WH, sm + P_WST, 16384, c_full);
+            if (hp) bulk_copy_to_cluster(slot + SL_WL, sm + P_WST + 16384, 16384, c_full);
+            bulk_copy_to_cluster(slot + SL_UT, sm + P_UTS, 32768, c_full);
+            bulk_copy_to_cluster(slot + SL_P16, sm + P_P16, 8192, c_full);
+            bulk_copy_to_cluster(slot + SL_GATES, sm + P_GST, (uint32_t)sizeof(GatesBlock), c_full);
+        }
+    }
+    // let the last delivery land, and a prefetched tile load that was never
+    // consumed, before this CTA's shared memory can go away
+    if (jj > 0) mbar_wait_cluster_bounded(&ms->copied, (jj - 1) & 1, kWaitLimit);
+    if (tma_issued > jj + 1) {
+        const int l = tma_issued - 1;
+        mbar_wait_bounded(&ms->tma_bar[l & 1], (l >> 1) & 1, kWaitLimit);
+    }
+}
+
+// ---------------------------------------------------------------- chain --
+
+__device__ void chain_role(uint8_t *sm, const ClusterParams &p, int n, int h, int64_t t_begin,
+                           int64_t t_end, int nch) {
+    ChainMisc *ms = reinterpret_cast<ChainMisc *>(sm + C_MISC);
+    const uint32_t sbase = smem_u32(sm);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quad = warp & 3, half = warp >> 2, row = quad * 32 + lane;
+    const uint32_t tmem = ms->tmem_base;
+    const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
+    // producer-CTA barrier addresses (rank 1 + k)
+    const uint32_t prod_copied_local = sbase + P_MISC + (uint32_t)offsetof(ProdMisc, copied);
+    const uint32_t prod_freed_local = sbase + P_MISC + (uint32_t)offsetof(ProdMisc, freed);
+
+    // ---- initial state: fp32 -> TMEM accumulator, fp16 hi/lo -> TMEM A operands ----
+    {
+        const float *src = p.s0 ? p.s0 + (((int64_t)n * p.Hv + h) * kD + row) * kD + 64 * half : nullptr;
+        float v[32];
+        uint32_t hi[32], lo[32];
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {
+#pragma unroll
+            for (int x = 0; x < 32; x += 4) {
+                const float4 f = src ? *reinterpret_cast<const float4 *>(src + 32 * part + x)
+                                     : make_float4(0.f, 0.f, 0.f, 0.f);
+                v[x] = f.x; v[x + 1] = f.y; v[x + 2] = f.z; v[x + 3] = f.w;
+            }
+            tmem_st32(trow + CT_S + 64 * half + 32 * part, v);
+#pragma unroll
+            for (int x = 0; x < 32; x += 2) {
+                const __half2 hh = __floats2half2_rn(v[x], v[x + 1]);
+                const float2 hf = __half22float2(hh);
+                hi[16 * part + x / 2] = *reinterpret_cast<const uint32_t *>(&hh);
+                lo[16 * part + x / 2] = pack_half2(v[x] - hf.x, v[x + 1] - hf.y);
+            }
+        }
+        tmem_st32u(trow + CT_SH + 32 * half, hi);
+        tmem_st32u(trow + CT_SL + 32 * half, lo);
+        tmem_wait_st();
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+
+    uint32_t mma_phase = 0;
+    bool timed_out = false, aborted = false;
+    auto mma_sync_point = [&]() {
+        if (tid == 0) mma_commit(&ms->mma_bar);
+        if (!mbar_wait_bounded(&ms->mma_bar, mma_phase, kWaitLimit)) timed_out = true;
+        mma_phase ^= 1;
+        tc_fence_after_sync();
+    };
+    auto publish = [&]() {
+        fence_proxy_async_smem();
+        tmem_wait_st();
+        tc_fence_before_sync();
+        __syncthreads();
+        tc_fence_after_sync();
+    };
+
+    int c = 0;
+#pragma unroll 1
+    for (; c < nch && !aborted; ++c) {
+        const int k = c & 1;
+        uint8_t *slot = sm + k * SLOT_BYTES;
+        const uint32_t sslot = sbase + k * SLOT_BYTES;
+        const int64_t c0 = t_begin + (int64_t)kC * c;
+        const int L = (int)((t_end - c0) < kC ? (t_end - c0) : kC);
+
+        if (!mbar_wait_cluster_bounded(&ms->full[k], (c >> 1) & 1, kWaitLimit)) timed_out = true;
+        if (tid == 0) mbar_arrive_remote(mapa_shared(prod_copied_local, 1 + k));
+        const GatesBlock *gb = reinterpret_cast<const GatesBlock *>(slot + SL_GATES);
+        const bool hp = gb->hp != 0;
+        const float gC = gb->Gam[kC - 1];
+
+        // ---- S Q^T -> O, R = S W^T (A operands from TMEM) ----
+        if (tid == 0) {
+            tc_fence_after_sync();
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)
+                mma_f16_ts(tmem + CT_O, tmem + CT_SH + 8 * ks,
+                           make_sdesc(sslot + SL_Q16 + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024),
+                           IDESC_KK_N64, ks > 0);
+            for (int pass = 0; pass < (hp ? 3 : 1); ++pass)
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {
+                    const uint32_t a_col = pass == 2 ? CT_SL : CT_SH;
+                    const uint32_t w_off = pass == 1 ? SL_WL : SL_WH;
+                    mma_f16_ts(tmem + CT_R, tmem + a_col + 8 * ks,
+                               make_sdesc(sslot + w_off + ks * 2048, 16384, 1024), IDESC_KM_N64,
+                               (pass | ks) != 0);
+                }
+            mma_commit(&ms->mma_bar);
+        }
+        // master state *= Gamma_C while those run (they do not touch CT_S)
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {
+            float v[32];
+            tmem_ld32(trow + CT_S + 64 * half + 32 * part, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int x = 0; x < 32; ++x) v[x] *= gC;
+            tmem_st32(trow + CT_S + 64 * half + 32 * part, v);
+        }
+        if (!mbar_wait_bounded(&ms->mma_bar, mma_phase, kWaitLimit)) timed_out = true;
+        mma_phase ^= 1;
+        tc_fence_after_sync();
+
+        // ---- O *= Gamma (rows of the transposed output); U = U~ - R; U', U ----
+        {
+            const int c32 = 32 * half;
+            float v[32], r0[32];
+            tmem_ld32(trow + CT_O + c32, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int x = 0; x < 32; ++x) v[x] *= gb->Gam[c32 + x];
+            tmem_st32(trow + CT_O + c32, v);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const float4 f = *reinterpret_cast<const float4 *>(slot + SL_UT + ut_off(row, c32 / 4 + q));
+                v[4 * q] = f.x; v[4 * q + 1] = f.y; v[4 * q + 2] = f.z; v[4 * q + 3] = f.w;
+            }
+            tmem_ld32(trow + CT_R + c32, r0);
+            tmem_wait_ld();
+            __syncthreads();  // every U~ row is read before U' overwrites the region
+#pragma unroll
+            for (int x = 0; x < 32; ++x) {
+                v[x] -= r0[x];
+                r0[x] = v[x] * gb->eC[c32 + x];
+            }
+            store_split32(slot + SL_UP, slot + SL_UP + 16384, row, c32, r0, true);
+#pragma unroll
+            for (int e = 0; e < 32; e += 8) st_row_chunk(slot + SL_U16, row, (c32 + e) / 8, pack8(v + e));
+        }
+        publish();
+
+        // ---- S += [U'hi | U'lo] [K ; K];  O += U^T P^T ----
+        if (tid == 0) {
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)
+                mma_f16_ss(tmem + CT_S,
+                           make_sdesc(sslot + SL_UP + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024),
+                           make_sdesc(sslot + SL_K16 + (ks & 3) * 2048, 8192, 1024), IDESC_KM_N128, 1);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_f16_ss(tmem + CT_O, make_sdesc(sslot + SL_U16 + ks * 32, 16, 1024),
+                           make_sdesc(sslot + SL_P16 + ks * 32, 16, 1024), IDESC_KK_N64, 1);
+        }
+        mma_sync_point();
+
+        // ---- o -> staging -> global; new S -> fp16 hi/lo TMEM operands ----
+        {
+            const int c32 = 32 * half;
+            float v[32];
+            tmem_ld32(trow + CT_O + c32, v);
+            tmem_wait_ld();
+            __nv_bfloat16 *ost = reinterpret_cast<__nv_bfloat16 *>(slot + SL_OST);
+#pragma unroll
+            for (int x = 0; x < 32; ++x) ost[(c32 + x) * kD + row] = __float2bfloat16_rn(v[x]);
+            uint32_t hi[32], lo[32];
+#pragma unroll
+            for (int part = 0; part < 2; ++part) {
+                tmem_ld32(trow + CT_S + 64 * half + 32 * part, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int x = 0; x < 32; x += 2) {
+                    const __half2 hh = __floats2half2_rn(v[x], v[x + 1]);
+                    const float2 hf = __half22float2(hh);
+                    hi[16 * part + x / 2] = *reinterpret_cast<const uint32_t *>(&hh);
+                    lo[16 * part + x / 2] = pack_half2(v[x] - hf.x, v[x + 1] - hf.y);
+                }
+            }
+            tmem_st32u(trow + CT_SH + 32 * half, hi);
+            tmem_st32u(trow + CT_SL + 32 * half, lo);
+        }
+        __syncthreads();
+        {
+            const uint4 *ost = reinterpret_cast<const uint4 *>(slot + SL_OST);
+#pragma unroll
+            for (int q = 0; q < (kC * kD * 2 / 16) / kThreads; ++q) {
+                const int x = tid + q * kThreads;
+                const int r = x >> 4, c16 = x & 15;
+                if (r < L) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.o) +
+                                                           ((c0 + r) * p.Hv + h) * (int64_t)kD) + c16;
+                    *dst = ost[x];
+                }
+            }
+        }
+        fence_proxy_async_smem();  // our writes to the slot precede the producer's next copies
+        tmem_wait_st();
+        tc_fence_before_sync();
+        if (__syncthreads_or(timed_out ? 1 : 0)) {
+            if (tid == 0) raise_error(p.err, GDN_ERR_TIMEOUT);
+            aborted = true;
+        } else if (tid == 0) {
+            mbar_arrive_remote(mapa_shared(prod_freed_local, 1 + k));
+        }
+        tc_fence_after_sync();
+    }
+
+    if (!aborted && p.sT) {
+        float *dst = p.sT + (((int64_t)n * p.Hv + h) * kD + row) * kD;
+#pragma unroll 1
+        for (int cc = 64 * half; cc < 64 * half + 64; cc += 32) {
+            float v[32];
+            tmem_ld32(trow + CT_S + cc, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int x = 0; x < 32; x += 4)
+                *reinterpret_cast<float4 *>(dst + cc + x) = make_float4(v[x], v[x + 1], v[x + 2], v[x + 3]);
+        }
+    }
+    if (aborted) {
+        // a delivery for the next chunk may be on its way: let it land, acknowledge it
+        if (c < nch) {
+            const int k2 = c & 1;
+            if (mbar_wait_cluster_bounded(&ms->full[k2], (c >> 1) & 1, kWaitLimit) && tid == 0)
+                mbar_arrive_remote(mapa_shared(prod_copied_local, 1 + k2));
+        }
+        mbar_wait_bounded(&ms->mma_bar, mma_phase ^ 1, kWaitLimit);
+    }
+}
+
+__global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
+    gdn_prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
+                               const __grid_constant__ CUtensorMap tm_k,
+                               const __grid_constant__ CUtensorMap tm_v, ClusterParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~uintptr_t(1023));
+    const int rank = (int)cluster_ctarank();
+    const int unit = blockIdx.x / kCluster;  // n * Hv + h
+    const int h = unit % p.Hv;
+    const int n = unit / p.Hv;
+    const int j = h / (p.Hv / p.Hqk);
+    const int tid = threadIdx.x, warp = tid >> 5;
+
+    int64_t t_begin, t_end;
+    if (!seq_range(p.cu, n, p.N, p.T, p.err, t_begin, t_end)) return;  // uniform per cluster
+    const int nch = (int)((t_end - t_begin + kC - 1) / kC);
+
+    uint32_t *tmem_slot;
+    uint32_t ncols;
+    if (rank == 0) {
+        ChainMisc *ms = reinterpret_cast<ChainMisc *>(sm + C_MISC);
+        tmem_slot = &ms->tmem_base;
+        ncols = 512;
+        if (tid == 0) {
+            mbar_init(&ms->full[0], 1);
+            mbar_init(&ms->full[1], 1);
+            mbar_init(&ms->mma_bar, 1);
+            fence_mbarrier_init();
+        }
+    } else {
+        ProdMisc *ms = reinterpret_cast<ProdMisc *>(sm + P_MISC);
+        tmem_slot = &ms->tmem_base;
+        ncols = 128;
+        if (tid == 0) {
+            mbar_init(&ms->tma_bar[0], 1);
+            mbar_init(&ms->tma_bar[1], 1);
+            mbar_init(&ms->mma_bar, 1);
+            mbar_init(&ms->copied, 1);
+            mbar_init(&ms->freed, 1);
+            fence_mbarrier_init();
+            tma_prefetch_desc(&tm_q);
+            tma_prefetch_desc(&tm_k);
+            tma_prefetch_desc(&tm_v);
+        }
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, ncols);
+        tmem_relinquish();
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    cluster_sync();  // every CTA's barriers exist before anyone signals them
+    tc_fence_after_sync();
+
+    if (rank == 0)
+        chain_role(sm, p, n, h, t_begin, t_end, nch);
+    else
+        producer_role(sm, &tm_q, &tm_k, &tm_v, p, rank - 1, h, j, t_begin, t_end, nch);
+
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    if (warp == 0) tmem_dealloc(*tmem_slot, ncols);
+    cluster_sync();  // nobody's shared memory goes away while another CTA may address it
+}
+
+}  // namespace
+
+bool make_tile_map_bf16_128(CUtensorMap *m, const void *base, int64_t T, int32_t H);
+
+cudaError_t launch_prefill_cluster(const PrefillArgs &a, cudaStream_t s) {
+    if (a.T > 0x7fffffffLL) return cudaErrorInvalidValue;
+    CUtensorMap mq, mk, mv;
+    const int64_t Tm = a.T > 0 ? a.T : 1;
+    if (!make_tile_map_bf16_128(&mq, a.q, Tm, a.Hqk) || !make_tile_map_bf16_128(&mk, a.k, Tm, a.Hqk) ||
+        !make_tile_map_bf16_128(&mv, a.v, Tm, a.Hv))
+        return cudaErrorInvalidValue;
+    ClusterParams p;
+    p.g = a.g; p.beta = a.beta; p.s0 = a.s0; p.cu = a.cu; p.o = a.o; p.sT = a.sT; p.err = a.err;
+    p.T = a.T; p.N = a.N; p.Hqk = a.Hqk; p.Hv = a.Hv;
+    cudaError_t e = cudaFuncSetAttribute(gdn_prefill_cluster_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) return e;
+    const dim3 grid((unsigned)((int64_t)a.N * a.Hv * kCluster));
+    gdn_prefill_cluster_kernel<<<grid, kThreads, kSmemBytes, s>>>(mq, mk, mv, p);
+    return cudaGetLastError();
+}
+
+}  // namespace gdn

@@ -48,6 +48,7 @@
 
 #include "gdn_internal.cuh"
 #include "sm100.cuh"
+#include "tc_common.cuh"
 
 #ifdef GDN_TC_PHASES
 __device__ long long gdn_tc_phase_clk[16];
@@ -67,12 +68,9 @@ namespace gdn {
 namespace {
 
 using namespace sm100;
+using namespace tc;
 
-constexpr int kC = 64;      // chunk length
-constexpr int kD = 128;     // Dk = Dv
 constexpr int kThreads = 256;
-constexpr long long kWaitLimit = 1ll << 31;  // SM clocks (about a second)
-constexpr float kHighPrecisionDecay = 0.2f;  // Gamma_C at or above -> extra passes
 
 // ---- shared memory map (bytes from a 1024-aligned base) ----
 constexpr uint32_t OFF_KQ = 0;          // 2 halves x [K 64 rows | Q 64 rows] x 128 B
@@ -86,8 +84,6 @@ constexpr uint32_t OFF_X = 114688;
 constexpr uint32_t OFF_UP = OFF_X;            // hi, lo x 128 rows x 128 B  (A: U')
 constexpr uint32_t OFF_U16 = OFF_X + 32768;   // 128 rows x 128 B           (A: U^T)
 constexpr uint32_t OFF_WST = OFF_X;           // hi, lo x 128 rows(d) x 128 B (B: W^T, MN-major)
-constexpr int kAS = 65;  // row stride of A (scalar, conflict-free column access)
-constexpr int kTS = 68;  // row stride of T (16-byte aligned rows for float4 access)
 constexpr uint32_t OFF_AS = OFF_X;                   // float [64][kAS]
 constexpr uint32_t OFF_TS = OFF_X + 64 * kAS * 4;       // float [64][kTS], 16-byte aligned
 constexpr uint32_t OFF_XS = OFF_TS + 64 * kTS * 4;   // float [3][16][16]
@@ -120,89 +116,6 @@ constexpr uint32_t kSmemBytes = OFF_MISC + sizeof(Misc) + 1024;  // + alignment 
 // TMEM column map (fp32 columns; 512 allocated, 448 used)
 constexpr uint32_t TM_S = 0, TM_G = 128, TM_U = 192, TM_WT = 256, TM_O = 320, TM_R = 384;
 
-constexpr uint32_t IDESC_KK_N64 = make_idesc_f16(128, 64, 0, 0);
-constexpr uint32_t IDESC_MK_N64 = make_idesc_f16(128, 64, 1, 0);
-constexpr uint32_t IDESC_KM_N64 = make_idesc_f16(128, 64, 0, 1);
-constexpr uint32_t IDESC_KM_N128 = make_idesc_f16(128, 128, 0, 1);
-
-__device__ __forceinline__ uint32_t pack_half2(float a, float b) {
-    const __half2 h = __floats2half2_rn(a, b);
-    return *reinterpret_cast<const uint32_t *>(&h);
-}
-
-// hi = fp16(x), lo = fp16(x - hi) for 8 values, packed as two uint4
-__device__ __forceinline__ void split8(const float *x, uint4 &hi, uint4 &lo) {
-    uint32_t h[4], l[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        const __half2 hh = __floats2half2_rn(x[2 * j], x[2 * j + 1]);
-        const float2 hf = __half22float2(hh);
-        h[j] = *reinterpret_cast<const uint32_t *>(&hh);
-        l[j] = pack_half2(x[2 * j] - hf.x, x[2 * j + 1] - hf.y);
-    }
-    hi = make_uint4(h[0], h[1], h[2], h[3]);
-    lo = make_uint4(l[0], l[1], l[2], l[3]);
-}
-
-__device__ __forceinline__ uint4 pack8(const float *x) {
-    return make_uint4(pack_half2(x[0], x[1]), pack_half2(x[2], x[3]), pack_half2(x[4], x[5]),
-                      pack_half2(x[6], x[7]));
-}
-
-__device__ __forceinline__ void st_row_chunk(uint8_t *tile, uint32_t row, uint32_t chunk,
-                                             uint4 val) {
-    *reinterpret_cast<uint4 *>(tile + sw128(row, chunk * 16)) = val;
-}
-
-// Writes 32 consecutive values (columns c .. c+31 of row `row`) of a 128-byte
-// swizzled fp16 tile as hi (and, if `with_lo`, lo) parts.
-__device__ __forceinline__ void store_split32(uint8_t *hi_tile, uint8_t *lo_tile, int row, int c,
-                                              const float *v, bool with_lo) {
-#pragma unroll
-    for (int e = 0; e < 32; e += 8) {
-        uint4 hi, lo;
-        split8(v + e, hi, lo);
-        st_row_chunk(hi_tile, row, (c + e) / 8, hi);
-        if (with_lo) st_row_chunk(lo_tile, row, (c + e) / 8, lo);
-    }
-}
-
-// One block-distance level of the triangular inverse (see the solve phase).
-template <int D>
-__device__ __forceinline__ void solve_level(const float *As, float *Ts, float *Xs, int tid) {
-    constexpr int kBlocks = 4 - D;
-    const bool act = tid < kBlocks * 64;
-    const int blk = tid >> 6, r = (tid >> 2) & 15, c4 = 4 * (tid & 3);
-    const int bi = blk + D, bk = blk;
-    if (act) {
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        const float *arow = As + (16 * bi + r) * kAS + 16 * bk;
-        const float *tcol = Ts + (16 * bk) * kTS + 16 * bk + c4;
-#pragma unroll
-        for (int m = 0; m < 16 * D; ++m) {
-            const float a = arow[m];
-            const float4 t = *reinterpret_cast<const float4 *>(tcol + m * kTS);
-            acc.x = fmaf(a, t.x, acc.x); acc.y = fmaf(a, t.y, acc.y);
-            acc.z = fmaf(a, t.z, acc.z); acc.w = fmaf(a, t.w, acc.w);
-        }
-        *reinterpret_cast<float4 *>(Xs + (blk << 8) + r * 16 + c4) = acc;
-    }
-    __syncthreads();
-    if (act) {
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        const float *drow = Ts + (16 * bi + r) * kTS + 16 * bi;
-#pragma unroll
-        for (int m = 0; m < 16; ++m) {
-            const float d = drow[m];
-            const float4 x = *reinterpret_cast<const float4 *>(Xs + (blk << 8) + m * 16 + c4);
-            acc.x = fmaf(d, x.x, acc.x); acc.y = fmaf(d, x.y, acc.y);
-            acc.z = fmaf(d, x.z, acc.z); acc.w = fmaf(d, x.w, acc.w);
-        }
-        *reinterpret_cast<float4 *>(Ts + (16 * bi + r) * kTS + 16 * bk + c4) =
-            make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
-    }
-    __syncthreads();
-}
 
 struct TcParams {
     const float *g, *beta, *s0;
@@ -689,6 +602,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ---------------------------------------------------------------- host --
 
+}  // namespace
+
+namespace {
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
@@ -708,8 +625,11 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// [T][H][128] bf16 tensor, boxes of 64 (features) x 1 (head) x 64 (tokens), 128-byte swizzle
-bool make_map(CUtensorMap *m, const void *base, int64_t T, int32_t H) {
+}  // namespace
+
+// [T][H][128] bf16 tensor map with 64 x 1 x 64 boxes and the 128-byte swizzle,
+// shared by the tensor-core prefill kernels.
+bool make_tile_map_bf16_128(CUtensorMap *m, const void *base, int64_t T, int32_t H) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)H, (cuuint64_t)T};
@@ -722,14 +642,13 @@ bool make_map(CUtensorMap *m, const void *base, int64_t T, int32_t H) {
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-}  // namespace
 
 cudaError_t launch_prefill_tc(const PrefillArgs &a, cudaStream_t s) {
     if (a.T > 0x7fffffffLL) return cudaErrorInvalidValue;  // TMA coordinates are 32-bit
     CUtensorMap mq, mk, mv;
     const int64_t Tm = a.T > 0 ? a.T : 1;
-    if (!make_map(&mq, a.q, Tm, a.Hqk) || !make_map(&mk, a.k, Tm, a.Hqk) ||
-        !make_map(&mv, a.v, Tm, a.Hv))
+    if (!make_tile_map_bf16_128(&mq, a.q, Tm, a.Hqk) || !make_tile_map_bf16_128(&mk, a.k, Tm, a.Hqk) ||
+        !make_tile_map_bf16_128(&mv, a.v, Tm, a.Hv))
         return cudaErrorInvalidValue;
     TcParams p;
     p.g = a.g; p.beta = a.beta; p.s0 = a.s0; p.cu = a.cu; p.o = a.o; p.sT = a.sT; p.err = a.err;

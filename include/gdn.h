@@ -100,10 +100,11 @@ typedef enum gdn_dtype {
  *   dev_error_flag      optional device int32 (see Errors above).
  *   stream              cudaStream_t.
  *
- * Supported: Dk = Dv = 128 with bf16 I/O and chunk 0 or 64 runs the tensor-core
+ * Supported: Dk = Dv = 128 with bf16 I/O and chunk 0 or 64 runs a tensor-core
  * (tcgen05) chunked kernel; every other combination with Dk, Dv in
  * {16, 32, 64, 128} and either dtype runs an exact fp32 token-recurrent CUDA
- * kernel.  Anything else returns GDN_ERR_UNSUPPORTED.
+ * kernel.  Anything else returns GDN_ERR_UNSUPPORTED.  gdn_prefill_ex below
+ * selects the kernel explicitly.
  */
 GDN_API gdn_status gdn_prefill(const void *q, const void *k, const void *v, gdn_dtype io_dtype,
                        const float *g, const float *beta, const float *initial_state,
@@ -111,6 +112,32 @@ GDN_API gdn_status gdn_prefill(const void *q, const void *k, const void *v, gdn_
                        int32_t Dk, int32_t Dv, int32_t chunk, void *o, float *final_state,
                        void *workspace, size_t workspace_bytes, int32_t *dev_error_flag,
                        void *stream);
+
+/*
+ * Which prefill kernel runs.  AUTO picks the tensor-core cluster kernel for
+ * Dk = Dv = 128, bf16 and chunk 0 or 64, and the exact recurrent kernel
+ * otherwise.  Naming a tensor-core kernel for a shape it does not support
+ * returns GDN_ERR_UNSUPPORTED.
+ */
+typedef enum gdn_prefill_kernel {
+    GDN_PREFILL_AUTO = 0,
+    GDN_PREFILL_CLUSTER = 1,     /* tcgen05, a 3-CTA cluster per (sequence, head): one CTA
+                                    holds the state, two prepare alternate chunks */
+    GDN_PREFILL_SINGLE_CTA = 2,  /* tcgen05, one CTA per (sequence, head) */
+    GDN_PREFILL_RECURRENT = 3    /* exact fp32 token recurrence on CUDA cores, any shape */
+} gdn_prefill_kernel;
+
+/*
+ * gdn_prefill_ex -- gdn_prefill with an explicit kernel choice (all other
+ * arguments and behaviour as gdn_prefill).  The kernels differ in speed and
+ * rounding only; each meets the same tolerances.
+ */
+GDN_API gdn_status gdn_prefill_ex(const void *q, const void *k, const void *v, gdn_dtype io_dtype,
+                                  const float *g, const float *beta, const float *initial_state,
+                                  const int32_t *cu_seqlens, int32_t N, int64_t T, int32_t Hqk,
+                                  int32_t Hv, int32_t Dk, int32_t Dv, int32_t chunk, void *o,
+                                  float *final_state, void *workspace, size_t workspace_bytes,
+                                  int32_t *dev_error_flag, void *stream, gdn_prefill_kernel kernel);
 
 /*
  * gdn_prefill_workspace_bytes -- scratch bytes gdn_prefill needs for these

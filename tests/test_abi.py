@@ -30,7 +30,7 @@ def declared_functions():
 
 def test_exports_every_declared_symbol(lib):
     names = declared_functions()
-    assert {"gdn_prefill", "gdn_decode_step", "gdn_prefill_workspace_bytes",
+    assert {"gdn_prefill", "gdn_prefill_ex", "gdn_decode_step", "gdn_prefill_workspace_bytes",
             "gdn_status_string", "gdn_version"} <= set(names)
     for n in names:
         assert hasattr(lib, n), f"libgdn.so does not export {n}"
@@ -90,6 +90,29 @@ INVALID, UNSUPPORTED = 1, 2
 ])
 def test_prefill_rejects(lib, kw, code):
     assert prefill(lib, **kw) == code
+
+
+def prefill_ex(lib, kernel, **kw):
+    args = dict(q=P, k=P + 0x1000, v=P + 0x2000, dt=0, g=P + 0x3000, beta=P + 0x4000, s0=None,
+                cu=None, N=1, T=64, Hqk=16, Hv=48, Dk=128, Dv=128, chunk=64, o=P + 0x5000,
+                sT=None, ws=None, wsb=0, err=None, stream=None)
+    args.update(kw)
+    return lib.gdn_prefill_ex(args["q"], args["k"], args["v"], args["dt"], args["g"], args["beta"],
+                              args["s0"], args["cu"], args["N"], args["T"], args["Hqk"], args["Hv"],
+                              args["Dk"], args["Dv"], args["chunk"], args["o"], args["sT"],
+                              args["ws"], args["wsb"], args["err"], args["stream"], kernel)
+
+
+@pytest.mark.parametrize("kernel,kw,code", [
+    (7, {}, INVALID),                              # no such kernel
+    (1, dict(Dk=64, Dv=64), UNSUPPORTED),          # tensor-core kernels need D = 128
+    (2, dict(dt=1), UNSUPPORTED),                  # ... and bf16
+    (1, dict(chunk=32), UNSUPPORTED),              # ... and chunk 64
+    (3, dict(q=None), INVALID),
+])
+def test_prefill_ex_rejects(lib, kernel, kw, code):
+    lib.gdn_prefill_ex.argtypes = lib.gdn_prefill.argtypes + [ctypes.c_int]
+    assert prefill_ex(lib, kernel, **kw) == code
 
 
 def test_prefill_nothing_to_do_is_ok(lib):

@@ -26,10 +26,14 @@ def _gpu():
     build.build()
 
 
-def run_gpu(inp, s0=None, cu=None, chunk=0, dev=DEV):
+TC_KERNELS = ["cluster", "single_cta"]
+
+
+def run_gpu(inp, s0=None, cu=None, chunk=0, dev=DEV, kernel="auto"):
     t = lambda x: None if x is None else x.to(dev).contiguous()
     o, sT = gdn.gdn_prefill(t(inp["q"]), t(inp["k"]), t(inp["v"]), t(inp["g"]), t(inp["beta"]),
-                            t(s0), None if cu is None else cu.to(torch.int32).to(dev), chunk=chunk)
+                            t(s0), None if cu is None else cu.to(torch.int32).to(dev), chunk=chunk,
+                            kernel=kernel)
     torch.cuda.synchronize()
     return o.cpu(), sT.cpu()
 
@@ -54,18 +58,20 @@ def test_tiny_workload_fp32():
     check_state(sT, s_ref)
 
 
-def test_layer4k_workload():
+@pytest.mark.parametrize("kernel", TC_KERNELS + ["recurrent"])
+def test_layer4k_workload(kernel):
     inp = inputs.make_prefill("layer4k")
-    o, sT = run_gpu(inp, chunk=64)
+    o, sT = run_gpu(inp, chunk=64, kernel=kernel)
     o_ref, s_ref = run_oracle(inp)
     check_o(o, o_ref)
     check_state(sT, s_ref)
 
 
-@pytest.mark.parametrize("T", [1, 63, 64, 65, 127, 200, 333])
-def test_ragged_lengths_d128_bf16(T):
+@pytest.mark.parametrize("kernel", TC_KERNELS)
+@pytest.mark.parametrize("T", [1, 63, 64, 65, 127, 128, 129, 200, 333])
+def test_ragged_lengths_d128_bf16(T, kernel):
     inp, s0 = synth(T, 2, 6, 128, torch.bfloat16, seed=100 + T, s0_std=0.05)
-    o, sT = run_gpu(inp, s0)
+    o, sT = run_gpu(inp, s0, kernel=kernel)
     o_ref, s_ref = run_oracle(inp, s0)
     check_o(o, o_ref)
     check_state(sT, s_ref)
@@ -81,7 +87,8 @@ def test_other_head_sizes(D, dtype):
     check_state(sT, s_ref)
 
 
-def test_packed_with_empty_sequences_and_in_place_state():
+@pytest.mark.parametrize("kernel", TC_KERNELS)
+def test_packed_with_empty_sequences_and_in_place_state(kernel):
     lengths = [0, 65, 0, 64, 1, 200, 0]
     cu = inputs.cu_from_lengths(lengths)
     inp, s0 = synth(int(cu[-1]), 2, 6, 128, torch.bfloat16, seed=300, s0_std=0.05,
@@ -90,7 +97,7 @@ def test_packed_with_empty_sequences_and_in_place_state():
     t = lambda x: x.to(DEV).contiguous()
     state = t(s0)
     o, sT = gdn.gdn_prefill(t(inp["q"]), t(inp["k"]), t(inp["v"]), t(inp["g"]), t(inp["beta"]),
-                            state, cu.to(torch.int32).to(DEV), final_state=state)
+                            state, cu.to(torch.int32).to(DEV), final_state=state, kernel=kernel)
     torch.cuda.synchronize()
     assert sT.data_ptr() == state.data_ptr()
     check_o(o.cpu(), o_ref)
@@ -100,8 +107,9 @@ def test_packed_with_empty_sequences_and_in_place_state():
             assert torch.equal(state[n].cpu(), s0[n])
 
 
+@pytest.mark.parametrize("kernel", TC_KERNELS)
 @pytest.mark.parametrize("case", ["b0", "b1", "a1", "strong_decay", "orthonormal_keys"])
-def test_degenerate_gates(case):
+def test_degenerate_gates(case, kernel):
     T, D = 130, 128
     inp, s0 = synth(T, 1, 3, D, torch.bfloat16, seed=400, s0_std=0.05)
     if case == "b0":
@@ -117,7 +125,7 @@ def test_degenerate_gates(case):
         basis, _ = torch.linalg.qr(torch.randn(D, D, generator=gen, dtype=torch.float64))
         idx = torch.arange(T) % D
         inp["k"] = basis[idx].reshape(T, 1, D).to(torch.bfloat16)
-    o, sT = run_gpu(inp, s0)
+    o, sT = run_gpu(inp, s0, kernel=kernel)
     o_ref, s_ref = run_oracle(inp, s0)
     check_o(o, o_ref)
     check_state(sT, s_ref)
@@ -127,7 +135,8 @@ def test_degenerate_gates(case):
         np.testing.assert_allclose(sT.double().numpy(), want.numpy(), rtol=2e-5, atol=1e-7)
 
 
-def test_bad_cu_seqlens_sets_flag_without_writing():
+@pytest.mark.parametrize("kernel", TC_KERNELS + ["recurrent"])
+def test_bad_cu_seqlens_sets_flag_without_writing(kernel):
     inp, _ = synth(64, 1, 3, 128, torch.bfloat16, seed=500)
     t = lambda x: x.to(DEV).contiguous()
     for bad in ([0, 10, 5, 64], [0, 10, 20, 63], [1, 10, 20, 64]):
@@ -135,37 +144,41 @@ def test_bad_cu_seqlens_sets_flag_without_writing():
         flag = torch.zeros(4, dtype=torch.int32, device=DEV)
         o = torch.full((64, 3, 128), 7.0, dtype=torch.bfloat16, device=DEV)
         gdn.gdn_prefill(t(inp["q"]), t(inp["k"]), t(inp["v"]), t(inp["g"]), t(inp["beta"]), None,
-                        cu, o=o, error_flag=flag)
+                        cu, o=o, error_flag=flag, kernel=kernel)
         torch.cuda.synchronize()
         assert int(flag[0]) == 5, bad  # GDN_ERR_BAD_SEQLENS
     # a valid call leaves the flag at zero
     cu = torch.tensor([0, 10, 20, 64], dtype=torch.int32, device=DEV)
     flag = torch.zeros(4, dtype=torch.int32, device=DEV)
     gdn.gdn_prefill(t(inp["q"]), t(inp["k"]), t(inp["v"]), t(inp["g"]), t(inp["beta"]), None,
-                    cu, error_flag=flag)
+                    cu, error_flag=flag, kernel=kernel)
     torch.cuda.synchronize()
     assert int(flag[0]) == 0
 
 
-def test_chunk_length_changes_rounding_only():
+def test_kernels_agree_with_each_other():
+    """chunk 64 (tensor cores, both kernels), chunk 16 and the recurrent kernel:
+    the chunk length and the kernel change rounding only."""
     inp, s0 = synth(300, 2, 6, 128, torch.bfloat16, seed=600, s0_std=0.05)
-    o64, s64 = run_gpu(inp, s0, chunk=64)
-    o16, s16 = run_gpu(inp, s0, chunk=16)
-    check_o(o16, o64.double())
-    check_state(s16, s64.double())
+    o64, s64 = run_gpu(inp, s0, chunk=64, kernel="cluster")
+    for kw in (dict(chunk=64, kernel="single_cta"), dict(chunk=16), dict(kernel="recurrent")):
+        o2, s2 = run_gpu(inp, s0, **kw)
+        check_o(o2, o64.double())
+        check_state(s2, s64.double())
 
 
-def test_varlen32_split_and_carry():
+@pytest.mark.parametrize("kernel", TC_KERNELS)
+def test_varlen32_split_and_carry(kernel):
     """32 packed sequences, lengths U[512,16384], nonzero initial states; every
     sequence split at a random point and run as two calls carrying the state
     must match the one-shot run and the oracle (sampled v-heads)."""
     inp = inputs.make_prefill("varlen32")
     cu = inputs.cu_from_lengths(inp["lengths"])
     s0 = inp["s0"]
-    o1, s1 = run_gpu(inp, s0, cu)
+    o1, s1 = run_gpu(inp, s0, cu, kernel=kernel)
     first, second = inputs.split_packed(inp)
-    oa, sa = run_gpu(first, s0, first["cu_seqlens"])
-    ob, sb = run_gpu(second, sa, second["cu_seqlens"])
+    oa, sa = run_gpu(first, s0, first["cu_seqlens"], kernel=kernel)
+    ob, sb = run_gpu(second, sa, second["cu_seqlens"], kernel=kernel)
     # reassemble the two halves in the packed order of the one-shot run
     o2 = torch.empty_like(o1)
     cua, cub = first["cu_seqlens"].tolist(), second["cu_seqlens"].tolist()
@@ -194,11 +207,13 @@ def head_subset(inp, heads):
              "g": pick(inp["g"], heads), "beta": pick(inp["beta"], heads)}, js)
 
 
-def test_long256k_sampled_heads():
+@pytest.mark.parametrize("kernel", TC_KERNELS)
+def test_long256k_sampled_heads(kernel):
     """The 262,144-token layer, in the bench's launch configuration (inputs drawn
     on the device by the seeded generator), checked on sampled v-heads."""
     inp = inputs.make_prefill("long256k", device="cuda")
-    o, sT = gdn.gdn_prefill(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], chunk=64)
+    o, sT = gdn.gdn_prefill(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], chunk=64,
+                            kernel=kernel)
     torch.cuda.synchronize()
     heads = [0, 29, 47]
     sub, _ = head_subset(inp, heads)
