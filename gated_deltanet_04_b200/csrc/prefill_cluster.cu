@@ -37,6 +37,21 @@
 #include "sm100.cuh"
 #include "tc_common.cuh"
 
+#ifdef GDN_TC_PHASES
+// per-phase SM clocks of cluster 0: [0] chain CTA, [1] first producer CTA
+__device__ long long gdn_cl_phase_clk[2][16];
+#define GDN_CL_PHASE(role, k)                                          \
+    do {                                                               \
+        if (threadIdx.x == 0 && blockIdx.x < 2) {                      \
+            const long long now_ = clock64();                          \
+            gdn_cl_phase_clk[(role)][(k)] += now_ - phase_t_;          \
+            phase_t_ = now_;                                           \
+        }                                                              \
+    } while (0)
+#else
+#define GDN_CL_PHASE(role, k) ((void)0)
+#endif
+
 namespace gdn {
 namespace {
 
@@ -75,8 +90,9 @@ struct ChainMisc {
     uint32_t tmem_base;
 };
 
-// chain TMEM columns (512 allocated)
-constexpr uint32_t CT_S = 0, CT_SH = 128, CT_SL = 192, CT_R = 256, CT_O = 320;
+// chain TMEM columns (512 allocated): state, this chunk's state increment,
+// fp16 hi/lo copies of the state (A operands), R = S W^T, output
+constexpr uint32_t CT_S = 0, CT_D = 128, CT_SH = 256, CT_SL = 320, CT_R = 384, CT_O = 448;
 
 // ---- producer CTA ----
 constexpr uint32_t P_KQV = 0;           // 2 buffers: [K|Q] d-half 0, [K|Q] d-half 1, V halves
@@ -91,9 +107,8 @@ constexpr uint32_t P_UTS = 147456;      // U~^T staging (same layout as SL_UT)
 constexpr uint32_t P_P16 = 180224;
 constexpr uint32_t P_TBH = 188416, P_TBL = 196608, P_TGH = 204800, P_TGL = 212992;
 constexpr uint32_t P_MISC = 221184;
-static_assert(P_XS + 3 * 256 * 4 <= P_UTS, "solve scratch overflows");
-static_assert(P_GST >= P_XS + 3 * 256 * 4 || P_GST + sizeof(GatesBlock) <= P_X + 49152,
-              "gates staging stays inside the scratch region");
+static_assert(P_XS + 1024 * 4 <= P_UTS, "solve scratch overflows");
+static_assert(P_GST + sizeof(GatesBlock) <= P_X + 49152, "gates staging stays inside the region");
 static_assert(P_TS % 16 == 0 && P_XS % 16 == 0, "float4 scratch must be aligned");
 
 struct ProdMisc {
@@ -183,6 +198,9 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
         tma_issued = 1;
         if (warp == 0) load_gates(t_begin + (int64_t)kC * k);
     }
+#ifdef GDN_TC_PHASES
+    long long phase_t_ = clock64();
+#endif
     int jj = 0;
 #pragma unroll 1
     for (; jj < nmine; ++jj) {
@@ -222,6 +240,7 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
             if (more) load_gates(c0 + 2 * kC);
         }
 
+        GDN_CL_PHASE(1, 0);  // gates
         // ---- the chain has taken our previous delivery: buffers and staging are free ----
         if (jj >= 1 && !mbar_wait_cluster_bounded(&ms->copied, (jj - 1) & 1, kWaitLimit))
             timed_out = true;
@@ -229,7 +248,9 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
             if (tid == 0) issue_tma(buf ^ 1, c0 + 2 * kC);
             tma_issued = jj + 2;
         }
+        GDN_CL_PHASE(1, 1);  // wait: chain received our previous delivery
         if (!mbar_wait_bounded(&ms->tma_bar[buf], (jj >> 1) & 1, kWaitLimit)) timed_out = true;
+        GDN_CL_PHASE(1, 2);  // wait: tiles
 
         // ---- bf16 -> fp16 in place, zero padding rows ----
         uint8_t *kqv = sm + P_KQV + buf * P_KQV_BYTES;
@@ -257,6 +278,7 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
         publish();
         const bool hp = ms->hp;
         const bool safe = ms->safe;
+        GDN_CL_PHASE(1, 3);  // convert
 
         // ---- Gram: [K;Q] K^T ----
         if (tid == 0) {
@@ -268,6 +290,7 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
             }
         }
         mma_sync_point();
+        GDN_CL_PHASE(1, 4);  // Gram MMA
 
         // ---- A (lanes 0..63) and P (lanes 64..127) ----
         float *As = reinterpret_cast<float *>(sm + P_AS);
@@ -300,6 +323,7 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
             }
         }
         __syncthreads();
+        GDN_CL_PHASE(1, 5);  // A / P
 
         // ---- T = (I + A)^-1 ----
         if (tid < kC) {
@@ -324,6 +348,7 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
         solve_level<1>(As, Ts, Xs, tid);
         solve_level<2>(As, Ts, Xs, tid);
         solve_level<3>(As, Ts, Xs, tid);
+        GDN_CL_PHASE(1, 6);  // solve
 
         // ---- rows of T diag(b), T diag(b Gamma): fp16 hi / lo ----
         {
@@ -345,6 +370,7 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
             store_split32(sm + (tg ? P_TGH : P_TBH), sm + (tg ? P_TGL : P_TBL), r, c, x, !tg || hp);
         }
         publish();
+        GDN_CL_PHASE(1, 7);  // T tiles
 
         // ---- U~^T = V^T (T diag b)^T,  W^T = K^T (T diag(b Gamma))^T ----
         if (tid == 0) {
@@ -365,6 +391,7 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
                 }
         }
         mma_sync_point();
+        GDN_CL_PHASE(1, 8);  // U~ / W MMAs
 
         // ---- staging: W^T hi/lo (MN-major), U~^T (swizzled fp32), gates ----
         {
@@ -388,6 +415,7 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
         }
         fence_proxy_async_smem();  // staged data -> visible to the bulk copies
         __syncthreads();
+        GDN_CL_PHASE(1, 9);  // staging
 
         // ---- deliver into slot k of the chain CTA, once it is free ----
         if (jj >= 1 && !mbar_wait_cluster_bounded(&ms->freed, (jj - 1) & 1, kWaitLimit))
@@ -396,22 +424,32 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
             if (tid == 0) raise_error(p.err, GDN_ERR_TIMEOUT);
             break;
         }
-        if (tid == 0) {
+        GDN_CL_PHASE(1, 10);  // wait: slot free
+        if (warp == 1) {  // one bulk copy per lane; warp 0 moves on to the next gates
             const uint32_t slot = c_base + (uint32_t)k * SLOT_BYTES;
-            const uint32_t bytes = 4 * 8192 + 16384 * (hp ? 2 : 1) + 32768 + 8192 +
-                                   (uint32_t)sizeof(GatesBlock);
-            mbar_arrive_expect_tx_remote(c_full, bytes);
-#pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
-                bulk_copy_to_cluster(slot + SL_K16 + hf * 8192, kqv + hf * 16384, 8192, c_full);
-                bulk_copy_to_cluster(slot + SL_Q16 + hf * 8192, kqv + hf * 16384 + 8192, 8192, c_full);
+            if (lane == 0) {
+                const uint32_t bytes = 4 * 8192 + 16384 * (hp ? 2 : 1) + 32768 + 8192 +
+                                       (uint32_t)sizeof(GatesBlock);
+                mbar_arrive_expect_tx_remote(c_full, bytes);
             }
-            bulk_copy_to_cluster(slot + SL_WH, sm + P_WST, 16384, c_full);
-            if (hp) bulk_copy_to_cluster(slot + SL_WL, sm + P_WST + 16384, 16384, c_full);
-            bulk_copy_to_cluster(slot + SL_UT, sm + P_UTS, 32768, c_full);
-            bulk_copy_to_cluster(slot + SL_P16, sm + P_P16, 8192, c_full);
-            bulk_copy_to_cluster(slot + SL_GATES, sm + P_GST, (uint32_t)sizeof(GatesBlock), c_full);
+            __syncwarp();
+            uint32_t dst = 0, bytes = 0;
+            const uint8_t *src = nullptr;
+            switch (lane) {
+                case 0: dst = SL_K16; src = kqv; bytes = 8192; break;
+                case 1: dst = SL_K16 + 8192; src = kqv + 16384; bytes = 8192; break;
+                case 2: dst = SL_Q16; src = kqv + 8192; bytes = 8192; break;
+                case 3: dst = SL_Q16 + 8192; src = kqv + 16384 + 8192; bytes = 8192; break;
+                case 4: dst = SL_WH; src = sm + P_WST; bytes = 16384; break;
+                case 5: dst = SL_WL; src = sm + P_WST + 16384; bytes = hp ? 16384 : 0; break;
+                case 6: dst = SL_UT; src = sm + P_UTS; bytes = 32768; break;
+                case 7: dst = SL_P16; src = sm + P_P16; bytes = 8192; break;
+                case 8: dst = SL_GATES; src = sm + P_GST; bytes = (uint32_t)sizeof(GatesBlock); break;
+                default: break;
+            }
+            if (bytes) bulk_copy_to_cluster(slot + dst, src, bytes, c_full);
         }
+        GDN_CL_PHASE(1, 11);  // deliver (issue)
     }
     // let the last delivery land, and a prefetched tile load that was never
     // consumed, before this CTA's shared memory can go away
@@ -482,6 +520,20 @@ __device__ void chain_role(uint8_t *sm, const ClusterParams &p, int n, int h, in
         tc_fence_after_sync();
     };
 
+#ifdef GDN_TC_PHASES
+    long long phase_t_ = clock64();
+#endif
+    // Thread 0 acknowledges each delivery as soon as it sees it complete (the
+    // producer may then reuse its buffers), polling for chunk c + 1 while
+    // chunk c is processed.
+    int acked = -1;
+    auto poll_next = [&](int cur) {
+        if (tid == 0 && acked == cur && cur + 1 < nch &&
+            mbar_try_wait_cluster(&ms->full[(cur + 1) & 1], ((cur + 1) >> 1) & 1)) {
+            mbar_arrive_remote(mapa_shared(prod_copied_local, 1 + ((cur + 1) & 1)));
+            acked = cur + 1;
+        }
+    };
     int c = 0;
 #pragma unroll 1
     for (; c < nch && !aborted; ++c) {
@@ -492,7 +544,11 @@ __device__ void chain_role(uint8_t *sm, const ClusterParams &p, int n, int h, in
         const int L = (int)((t_end - c0) < kC ? (t_end - c0) : kC);
 
         if (!mbar_wait_cluster_bounded(&ms->full[k], (c >> 1) & 1, kWaitLimit)) timed_out = true;
-        if (tid == 0) mbar_arrive_remote(mapa_shared(prod_copied_local, 1 + k));
+        GDN_CL_PHASE(0, 0);  // wait: delivery
+        if (tid == 0 && acked < c) {
+            mbar_arrive_remote(mapa_shared(prod_copied_local, 1 + k));
+            acked = c;
+        }
         const GatesBlock *gb = reinterpret_cast<const GatesBlock *>(slot + SL_GATES);
         const bool hp = gb->hp != 0;
         const float gC = gb->Gam[kC - 1];
@@ -516,19 +572,12 @@ __device__ void chain_role(uint8_t *sm, const ClusterParams &p, int n, int h, in
                 }
             mma_commit(&ms->mma_bar);
         }
-        // master state *= Gamma_C while those run (they do not touch CT_S)
-#pragma unroll
-        for (int part = 0; part < 2; ++part) {
-            float v[32];
-            tmem_ld32(trow + CT_S + 64 * half + 32 * part, v);
-            tmem_wait_ld();
-#pragma unroll
-            for (int x = 0; x < 32; ++x) v[x] *= gC;
-            tmem_st32(trow + CT_S + 64 * half + 32 * part, v);
-        }
+        poll_next(c);
+        GDN_CL_PHASE(0, 1);  // issue S Q^T, R
         if (!mbar_wait_bounded(&ms->mma_bar, mma_phase, kWaitLimit)) timed_out = true;
         mma_phase ^= 1;
         tc_fence_after_sync();
+        GDN_CL_PHASE(0, 2);  // wait: S Q^T, R
 
         // ---- O *= Gamma (rows of the transposed output); U = U~ - R; U', U ----
         {
@@ -557,22 +606,27 @@ __device__ void chain_role(uint8_t *sm, const ClusterParams &p, int n, int h, in
             for (int e = 0; e < 32; e += 8) st_row_chunk(slot + SL_U16, row, (c32 + e) / 8, pack8(v + e));
         }
         publish();
+        poll_next(c);
+        GDN_CL_PHASE(0, 3);  // O scale, U, U'
 
-        // ---- S += [U'hi | U'lo] [K ; K];  O += U^T P^T ----
+        // ---- dS = [U'hi | U'lo] [K ; K];  O += U^T P^T ----
         if (tid == 0) {
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks)
-                mma_f16_ss(tmem + CT_S,
+                mma_f16_ss(tmem + CT_D,
                            make_sdesc(sslot + SL_UP + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024),
-                           make_sdesc(sslot + SL_K16 + (ks & 3) * 2048, 8192, 1024), IDESC_KM_N128, 1);
+                           make_sdesc(sslot + SL_K16 + (ks & 3) * 2048, 8192, 1024), IDESC_KM_N128,
+                           ks > 0);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
                 mma_f16_ss(tmem + CT_O, make_sdesc(sslot + SL_U16 + ks * 32, 16, 1024),
                            make_sdesc(sslot + SL_P16 + ks * 32, 16, 1024), IDESC_KK_N64, 1);
         }
+        poll_next(c);
         mma_sync_point();
+        GDN_CL_PHASE(0, 4);  // state update + P MMAs
 
-        // ---- o -> staging -> global; new S -> fp16 hi/lo TMEM operands ----
+        // ---- o -> staging -> global; S' = Gamma_C S + dS, its fp16 hi/lo TMEM operands ----
         {
             const int c32 = 32 * half;
             float v[32];
@@ -584,8 +638,13 @@ __device__ void chain_role(uint8_t *sm, const ClusterParams &p, int n, int h, in
             uint32_t hi[32], lo[32];
 #pragma unroll
             for (int part = 0; part < 2; ++part) {
+                float d[32];
                 tmem_ld32(trow + CT_S + 64 * half + 32 * part, v);
+                tmem_ld32(trow + CT_D + 64 * half + 32 * part, d);
                 tmem_wait_ld();
+#pragma unroll
+                for (int x = 0; x < 32; ++x) v[x] = fmaf(gC, v[x], d[x]);  // S' = Gamma_C S + dS
+                tmem_st32(trow + CT_S + 64 * half + 32 * part, v);
 #pragma unroll
                 for (int x = 0; x < 32; x += 2) {
                     const __half2 hh = __floats2half2_rn(v[x], v[x + 1]);
@@ -611,6 +670,8 @@ __device__ void chain_role(uint8_t *sm, const ClusterParams &p, int n, int h, in
                 }
             }
         }
+        poll_next(c);
+        GDN_CL_PHASE(0, 5);  // o staging + stores, S copies
         fence_proxy_async_smem();  // our writes to the slot precede the producer's next copies
         tmem_wait_st();
         tc_fence_before_sync();
@@ -621,6 +682,7 @@ __device__ void chain_role(uint8_t *sm, const ClusterParams &p, int n, int h, in
             mbar_arrive_remote(mapa_shared(prod_freed_local, 1 + k));
         }
         tc_fence_after_sync();
+        GDN_CL_PHASE(0, 6);  // vote, free the slot
     }
 
     if (!aborted && p.sT) {
@@ -637,7 +699,7 @@ __device__ void chain_role(uint8_t *sm, const ClusterParams &p, int n, int h, in
     }
     if (aborted) {
         // a delivery for the next chunk may be on its way: let it land, acknowledge it
-        if (c < nch) {
+        if (c < nch && acked < c) {
             const int k2 = c & 1;
             if (mbar_wait_cluster_bounded(&ms->full[k2], (c >> 1) & 1, kWaitLimit) && tid == 0)
                 mbar_arrive_remote(mapa_shared(prod_copied_local, 1 + k2));
@@ -736,3 +798,16 @@ cudaError_t launch_prefill_cluster(const PrefillArgs &a, cudaStream_t s) {
 }
 
 }  // namespace gdn
+
+#ifdef GDN_TC_PHASES
+extern "C" GDN_API int gdn_debug_cluster_phases(long long *out, int reset) {
+    long long host[32];
+    if (cudaMemcpyFromSymbol(host, gdn_cl_phase_clk, sizeof(host)) != cudaSuccess) return -1;
+    for (int i = 0; i < 32; ++i) out[i] = host[i];
+    if (reset) {
+        const long long zero[32] = {0};
+        cudaMemcpyToSymbol(gdn_cl_phase_clk, zero, sizeof(zero));
+    }
+    return 0;
+}
+#endif

@@ -86,7 +86,7 @@ constexpr uint32_t OFF_U16 = OFF_X + 32768;   // 128 rows x 128 B           (A: 
 constexpr uint32_t OFF_WST = OFF_X;           // hi, lo x 128 rows(d) x 128 B (B: W^T, MN-major)
 constexpr uint32_t OFF_AS = OFF_X;                   // float [64][kAS]
 constexpr uint32_t OFF_TS = OFF_X + 64 * kAS * 4;       // float [64][kTS], 16-byte aligned
-constexpr uint32_t OFF_XS = OFF_TS + 64 * kTS * 4;   // float [3][16][16]
+constexpr uint32_t OFF_XS = OFF_TS + 64 * kTS * 4;   // float [1024] level partials
 constexpr uint32_t OFF_P16 = 163840;    // 64 rows x 128 B                  (B: P, K-major)
 constexpr uint32_t OFF_TBH = 172032;    // 64 rows x 128 B                  (B: T diag b, hi)
 constexpr uint32_t OFF_TBL = 180224;    //                                  (B: T diag b, lo)
@@ -94,7 +94,7 @@ constexpr uint32_t OFF_TGH = 188416;    //                                  (B: 
 constexpr uint32_t OFF_TGL = 196608;    //                                  (B: T diag(b Gamma), lo)
 constexpr uint32_t OFF_OST = OFF_TBH;   // o staging [64 tokens][128] bf16 (TB tiles are dead)
 constexpr uint32_t OFF_MISC = 204800;
-static_assert(OFF_XS + 3 * 256 * 4 <= OFF_P16, "solve scratch overflows");
+static_assert(OFF_XS + 1024 * 4 <= OFF_P16, "solve scratch overflows");
 static_assert(OFF_TS % 16 == 0 && OFF_XS % 16 == 0, "float4 scratch must be aligned");
 
 struct Misc {

@@ -68,7 +68,9 @@ __device__ __forceinline__ void store_split32(uint8_t *hi_tile, uint8_t *lo_tile
     }
 }
 
-// One block-distance level of the triangular inverse (see the solve phase).
+// One block-distance level D of the triangular inverse (see the solve phase):
+//   X = sum_{m = k}^{i-1} A_im T_mk,   T_ik = -D_i X,   i = k + D,
+// each thread producing four adjacent columns of one row of one block.
 template <int D>
 __device__ __forceinline__ void solve_level(const float *As, float *Ts, float *Xs, int tid) {
     constexpr int kBlocks = 4 - D;
@@ -104,7 +106,6 @@ __device__ __forceinline__ void solve_level(const float *As, float *Ts, float *X
     }
     __syncthreads();
 }
-
 
 }  // namespace tc
 }  // namespace gdn
