@@ -60,6 +60,8 @@ def parse():
                    help="profiling mode: run one operation of a named workload (layer4k, "
                         "long256k, varlen32: one gdn_prefill call; decode256: one layer's "
                         "gdn_decode_step) W + K times and print its per-call time; no bench line")
+    p.add_argument("--kernel", default="auto", choices=["auto", "cluster", "single_cta", "recurrent"],
+                   help="prefill kernel for --case")
     return p.parse_args()
 
 
@@ -288,11 +290,14 @@ def run_case(args):
         o = torch.empty_like(inp["v"])
         N = inp["N"]
         sT = torch.empty((N, inp["wl"].Hv, 128, 128), dtype=torch.float32, device=dev)
+        kern = args.kernel
+        ws = torch.empty(max(1, gdn.gdn_prefill_workspace_bytes(N, inp["T"], 16, 48, 128, 128, 64,
+                                                                kern)), dtype=torch.uint8, device=dev)
         fn = lambda: gdn.gdn_prefill(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"],
                                      inp["s0"], inp["cu_seqlens"], chunk=inp["wl"].chunk,
-                                     o=o, final_state=sT)
+                                     o=o, final_state=sT, workspace=ws, kernel=kern)
     total, each = time_launches(fn, args.steps, args.warmup, Dist(), stream)
-    print(json.dumps({"case": args.case, "calls": args.steps, "ms_per_call": total / args.steps,
+    print(json.dumps({"case": args.case, "kernel": args.kernel, "calls": args.steps, "ms_per_call": total / args.steps,
                       "ms_min": min(each), "ms_max": max(each)}), flush=True)
     return 0
 
@@ -327,10 +332,12 @@ def main():
     T = inp["T"]
     o = torch.empty_like(inp["v"])
     sT = torch.empty((1, 48, 128, 128), dtype=torch.float32, device=dev)
+    ws = torch.empty(max(1, gdn.gdn_prefill_workspace_bytes(1, T, 16, 48, 128, 128, 64)),
+                     dtype=torch.uint8, device=dev)
 
     def prefill():
         gdn.gdn_prefill(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], None, None,
-                        chunk=64, o=o, final_state=sT)
+                        chunk=64, o=o, final_state=sT, workspace=ws)
 
     p_total, p_each = time_launches(prefill, K, W, dist, stream, sampler)
     p_ms = dist.max(p_total / K)
@@ -372,7 +379,7 @@ def main():
             for key in host:
                 dev_in[key].copy_(host[key], non_blocking=True)
             gdn.gdn_prefill(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["g"], dev_in["beta"],
-                            None, None, chunk=64, o=o, final_state=sT)
+                            None, None, chunk=64, o=o, final_state=sT, workspace=ws)
             o_host.copy_(o, non_blocking=True)
             s_host.copy_(sT, non_blocking=True)
 

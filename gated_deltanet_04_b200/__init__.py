@@ -60,6 +60,9 @@ def library():
             lib.gdn_decode_step.restype = ctypes.c_int
             lib.gdn_prefill_workspace_bytes.argtypes = [i32, i64, i32, i32, i32, i32, i32]
             lib.gdn_prefill_workspace_bytes.restype = sz
+            lib.gdn_prefill_ex_workspace_bytes.argtypes = [i32, i64, i32, i32, i32, i32, i32,
+                                                           ctypes.c_int]
+            lib.gdn_prefill_ex_workspace_bytes.restype = sz
             lib.gdn_status_string.argtypes = [ctypes.c_int]
             lib.gdn_status_string.restype = ctypes.c_char_p
             lib.gdn_version.argtypes = []
@@ -90,8 +93,9 @@ def _check(t, name, shape, dtype, device):
         raise ValueError(f"{name} must be contiguous")
 
 
-def gdn_prefill_workspace_bytes(N, T, Hqk, Hv, Dk, Dv, chunk=0):
-    return int(library().gdn_prefill_workspace_bytes(N, T, Hqk, Hv, Dk, Dv, chunk))
+def gdn_prefill_workspace_bytes(N, T, Hqk, Hv, Dk, Dv, chunk=0, kernel="auto"):
+    return int(library().gdn_prefill_ex_workspace_bytes(N, T, Hqk, Hv, Dk, Dv, chunk,
+                                                        KERNELS[kernel]))
 
 
 def gdn_prefill(q, k, v, g, beta, initial_state=None, cu_seqlens=None, *, chunk=0, o=None,
@@ -136,7 +140,7 @@ def gdn_prefill(q, k, v, g, beta, initial_state=None, cu_seqlens=None, *, chunk=
     if workspace is not None:
         ws_bytes = workspace.numel() * workspace.element_size()
     else:
-        need = int(lib.gdn_prefill_workspace_bytes(N, T, Hqk, Hv, Dk, Dv, chunk))
+        need = int(lib.gdn_prefill_ex_workspace_bytes(N, T, Hqk, Hv, Dk, Dv, chunk, KERNELS[kernel]))
         if need:
             workspace = torch.empty(need, dtype=torch.uint8, device=dev)
             ws_bytes = need

@@ -34,10 +34,25 @@ const char *gdn_status_string(gdn_status s) {
 
 int32_t gdn_version(void) { return 1 * 10000 + 0 * 100 + 0; }
 
+// The kernel gdn_prefill_ex runs for these arguments (kernel AUTO resolved).
+gdn_prefill_kernel resolve_kernel(gdn_prefill_kernel kernel, bool tc_ok, int64_t units) {
+    if (kernel != GDN_PREFILL_AUTO) return kernel;
+    if (!tc_ok) return GDN_PREFILL_RECURRENT;
+    return units <= gdn::kClusterMaxUnits ? GDN_PREFILL_CLUSTER : GDN_PREFILL_SINGLE_CTA;
+}
+
+size_t gdn_prefill_ex_workspace_bytes(int32_t N, int64_t T, int32_t Hqk, int32_t Hv, int32_t Dk,
+                                      int32_t Dv, int32_t chunk, gdn_prefill_kernel kernel) {
+    (void)T; (void)Hqk;
+    if (N <= 0 || Hv <= 0) return 0;
+    const bool shape_ok = Dk == 128 && Dv == 128 && (chunk == 0 || chunk == 64);
+    if (resolve_kernel(kernel, shape_ok, (int64_t)N * Hv) != GDN_PREFILL_CLUSTER || !shape_ok) return 0;
+    return gdn::prefill_cluster_workspace_bytes((int64_t)N * Hv);
+}
+
 size_t gdn_prefill_workspace_bytes(int32_t N, int64_t T, int32_t Hqk, int32_t Hv, int32_t Dk,
                                    int32_t Dv, int32_t chunk) {
-    (void)N; (void)T; (void)Hqk; (void)Hv; (void)Dk; (void)Dv; (void)chunk;
-    return 0;
+    return gdn_prefill_ex_workspace_bytes(N, T, Hqk, Hv, Dk, Dv, chunk, GDN_PREFILL_AUTO);
 }
 
 gdn_status gdn_prefill(const void *q, const void *k, const void *v, gdn_dtype io_dtype,
@@ -71,19 +86,21 @@ gdn_status gdn_prefill_ex(const void *q, const void *k, const void *v, gdn_dtype
         if (p && !aligned16(p)) return GDN_ERR_INVALID_ARGUMENT;
     if (o && (o == q || o == k || o == v)) return GDN_ERR_INVALID_ARGUMENT;
     if (!supported_dim(Dk) || !supported_dim(Dv) || chunk > 64) return GDN_ERR_UNSUPPORTED;
-    const size_t need = gdn_prefill_workspace_bytes(N, T, Hqk, Hv, Dk, Dv, chunk);
+    const bool tc_ok = tc_path(io_dtype, Dk, Dv, chunk);
+    if ((kernel == GDN_PREFILL_CLUSTER || kernel == GDN_PREFILL_SINGLE_CTA) && !tc_ok)
+        return GDN_ERR_UNSUPPORTED;
+    kernel = resolve_kernel(kernel, tc_ok, (int64_t)N * Hv);
+    const size_t need = (kernel == GDN_PREFILL_CLUSTER && T > 0)
+                            ? gdn::prefill_cluster_workspace_bytes((int64_t)N * Hv)
+                            : 0;
     if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return GDN_ERR_INVALID_ARGUMENT;
     if (T == 0 && final_state == nullptr) return GDN_OK;  // nothing observable to do
 
     gdn::PrefillArgs a;
     a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.s0 = initial_state; a.cu = cu_seqlens;
-    a.o = o; a.sT = final_state; a.err = dev_error_flag; a.T = T; a.N = N; a.Hqk = Hqk;
+    a.o = o; a.sT = final_state; a.err = dev_error_flag; a.ws = workspace; a.T = T; a.N = N; a.Hqk = Hqk;
     a.Hv = Hv; a.Dk = Dk; a.Dv = Dv; a.chunk = chunk == 0 ? 64 : chunk; a.dtype = io_dtype;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const bool tc_ok = tc_path(io_dtype, Dk, Dv, chunk);
-    if ((kernel == GDN_PREFILL_CLUSTER || kernel == GDN_PREFILL_SINGLE_CTA) && !tc_ok)
-        return GDN_ERR_UNSUPPORTED;
-    if (kernel == GDN_PREFILL_AUTO) kernel = tc_ok ? GDN_PREFILL_CLUSTER : GDN_PREFILL_RECURRENT;
     if (T == 0 || kernel == GDN_PREFILL_RECURRENT) return from_cuda(gdn::launch_prefill_recurrent(a, s));
     if (kernel == GDN_PREFILL_SINGLE_CTA) return from_cuda(gdn::launch_prefill_tc(a, s));
     return from_cuda(gdn::launch_prefill_cluster(a, s));

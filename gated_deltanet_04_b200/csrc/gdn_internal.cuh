@@ -18,6 +18,7 @@ struct PrefillArgs {
     void *o;
     float *sT;              // may be null
     int32_t *err;           // may be null
+    void *ws;               // workspace (cluster kernel's L2 ring)
     int64_t T;
     int32_t N, Hqk, Hv, Dk, Dv, chunk;
     gdn_dtype dtype;
@@ -40,6 +41,10 @@ cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s);
 // (sequence, head), or a 3-CTA cluster per (sequence, head).
 cudaError_t launch_prefill_tc(const PrefillArgs &a, cudaStream_t s);
 cudaError_t launch_prefill_cluster(const PrefillArgs &a, cudaStream_t s);
+// Workspace of the cluster kernel: a 4-slot ring per (sequence, head).
+size_t prefill_cluster_workspace_bytes(int64_t units);
+// AUTO uses the cluster kernel up to this many (sequence, head) units.
+constexpr int64_t kClusterMaxUnits = 64;
 
 // ---------------------------------------------------------------- device --
 

@@ -16,18 +16,24 @@
 //     update S += U'^T K, O += U^T P^T, and the output stores.
 //   * ranks 1 and 2, the producer CTAs, take alternate chunks (rank 1 even,
 //     rank 2 odd): TMA tile loads, bf16 -> fp16, Gram matrices, decay factors,
-//     the triangular solve, U~ and W on tensor cores.  Each finished chunk
-//     (K, Q, W^T hi/lo, U~, P, gates: up to 105 KB) is copied by bulk copies
-//     into one of two hand-off slots in the chain CTA's shared memory.
-// With the producers a chunk ahead, the chain CTA's per-chunk time is its own
-// chain of two MMA groups and two row epilogues.
+//     the triangular solve, U~ and W on tensor cores.
+// A finished chunk (K, Q, W^T hi/lo, U~, P, gates: one 105 KB block laid out
+// exactly like a chain slot) goes through L2: the producer bulk-stores it
+// into a ring of 2 slots per producer in the caller's workspace, the chain
+// bulk-loads it into one of its two shared-memory slots while it computes
+// the previous chunk.  Distributed shared memory carries only the signals
+// (it moves bulk data far more slowly than L2); the ring is 420 KB per
+// (sequence, head) and stays resident in L2.
 //
-// Flow control (all mbarrier waits bounded; a wait that expires is voted on
-// once per chunk, reports GDN_ERR_TIMEOUT and ends the CTA's loop):
-//   full[k]  (chain)    : producer k's expect-tx arrival + its bulk copies
-//   copied   (producer) : the chain received the producer's last delivery, so
-//                         the producer may reuse its tile buffers and staging
-//   freed    (producer) : the chain finished the chunk in slot k
+// Flow control (all waits bounded; a wait that expires is voted on once per
+// chunk, reports GDN_ERR_TIMEOUT and ends the CTA's loop):
+//   ready[k] (chain)    : producer k's stores of its next chunk are complete
+//   full[i]  (chain)    : the bulk load into shared slot i has landed
+//   taken    (producer) : the chain has loaded this producer's last delivery
+// A producer delivers chunk j only after the chain has taken chunk j - 1:
+// then no barrier ever runs more than one phase ahead of its waiter (a
+// parity wait cannot tell phase n from phase n + 2), and the ring slot of
+// chunk j, last used by chunk j - 2, is free.
 // A cluster barrier after set-up and another before exit keep every CTA's
 // shared memory alive while the others may still address it.  No TMA load
 // uses multicast.
@@ -86,6 +92,7 @@ static_assert(sizeof(GatesBlock) % 16 == 0, "bulk copies move multiples of 16 by
 
 struct ChainMisc {
     uint64_t full[2];
+    uint64_t ready[2];
     uint64_t mma_bar;
     uint32_t tmem_base;
 };
@@ -115,8 +122,7 @@ struct ProdMisc {
     float gam[kC], Gam[kC], iGam[kC], eC[kC], bb[kC], bG[kC];
     uint64_t tma_bar[2];
     uint64_t mma_bar;
-    uint64_t copied;
-    uint64_t freed;
+    uint64_t taken;
     uint32_t tmem_base;
     int32_t safe, hp;
     float gsum;
@@ -128,6 +134,7 @@ static_assert(C_MISC + sizeof(ChainMisc) <= P_MISC + sizeof(ProdMisc), "chain mi
 constexpr uint32_t PT_G = 0, PT_U = 64;
 
 struct ClusterParams {
+    uint8_t *ws;  // ring: [unit][producer][2 slots][SLOT_BYTES]
     const float *g, *beta, *s0;
     const int32_t *cu;
     void *o;
@@ -137,6 +144,10 @@ struct ClusterParams {
     int32_t N, Hqk, Hv;
 };
 
+__device__ __forceinline__ uint8_t *ring_slot(const ClusterParams &p, int unit, int k, int s) {
+    return p.ws + ((size_t)(unit * 2 + k) * 2 + s) * SLOT_BYTES;
+}
+
 // byte offset of 16-byte chunk q of row i in a [128][64] fp32 U~ tile
 __device__ __forceinline__ uint32_t ut_off(int i, int q) {
     return (uint32_t)i * 256u + (uint32_t)((q ^ (i & 15)) << 4);
@@ -145,17 +156,17 @@ __device__ __forceinline__ uint32_t ut_off(int i, int q) {
 // ------------------------------------------------------------- producer --
 
 __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtensorMap *tm_k,
-                              const CUtensorMap *tm_v, const ClusterParams &p, int k, int h,
-                              int j, int64_t t_begin, int64_t t_end, int nch) {
+                              const CUtensorMap *tm_v, const ClusterParams &p, int unit, int k,
+                              int h, int j, int64_t t_begin, int64_t t_end, int nch) {
     ProdMisc *ms = reinterpret_cast<ProdMisc *>(sm + P_MISC);
     const uint32_t sbase = smem_u32(sm);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quad = warp & 3, half = warp >> 2, row = quad * 32 + lane;
     const uint32_t tmem = ms->tmem_base;
     const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
-    // chain-CTA addresses (rank 0)
-    const uint32_t c_base = mapa_shared(sbase, 0);
-    const uint32_t c_full = mapa_shared(sbase + C_MISC + (uint32_t)offsetof(ChainMisc, full) + 8u * k, 0);
+    // the chain CTA's ready barrier for this producer (rank 0)
+    const uint32_t c_ready =
+        mapa_shared(sbase + C_MISC + (uint32_t)offsetof(ChainMisc, ready) + 8u * k, 0);
     const int nmine = nch > k ? (nch - k + 1) / 2 : 0;
 
     uint32_t mma_phase = 0;
@@ -192,12 +203,14 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
         tc_fence_after_sync();
     };
 
+    // Tile loads: local chunks 0 and 1 now; chunk jj + 2 by the delivery thread
+    // of chunk jj, into the buffer its stores have just drained.
     int tma_issued = 0;  // tile loads issued (local chunk indices 0 .. tma_issued-1)
-    if (nmine > 0) {
-        if (tid == 0) issue_tma(0, t_begin + (int64_t)kC * k);
-        tma_issued = 1;
-        if (warp == 0) load_gates(t_begin + (int64_t)kC * k);
+    for (int l = 0; l < 2 && l < nmine; ++l) {
+        if (tid == 32) issue_tma(l, t_begin + (int64_t)kC * (k + 2 * l));
+        tma_issued = l + 1;
     }
+    if (nmine > 0 && warp == 0) load_gates(t_begin + (int64_t)kC * k);
 #ifdef GDN_TC_PHASES
     long long phase_t_ = clock64();
 #endif
@@ -241,14 +254,7 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
         }
 
         GDN_CL_PHASE(1, 0);  // gates
-        // ---- the chain has taken our previous delivery: buffers and staging are free ----
-        if (jj >= 1 && !mbar_wait_cluster_bounded(&ms->copied, (jj - 1) & 1, kWaitLimit))
-            timed_out = true;
-        if (more) {
-            if (tid == 0) issue_tma(buf ^ 1, c0 + 2 * kC);
-            tma_issued = jj + 2;
-        }
-        GDN_CL_PHASE(1, 1);  // wait: chain received our previous delivery
+        GDN_CL_PHASE(1, 1);  // (no wait)
         if (!mbar_wait_bounded(&ms->tma_bar[buf], (jj >> 1) & 1, kWaitLimit)) timed_out = true;
         GDN_CL_PHASE(1, 2);  // wait: tiles
 
@@ -417,62 +423,52 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
         __syncthreads();
         GDN_CL_PHASE(1, 9);  // staging
 
-        // ---- deliver into slot k of the chain CTA, once it is free ----
-        if (jj >= 1 && !mbar_wait_cluster_bounded(&ms->freed, (jj - 1) & 1, kWaitLimit))
+        // ---- deliver through the L2 ring, once the chain has taken our previous chunk ----
+        const int rs = jj & 1;
+        if (jj >= 1 && !mbar_wait_cluster_bounded(&ms->taken, (jj - 1) & 1, kWaitLimit))
             timed_out = true;
         if (__syncthreads_or(timed_out ? 1 : 0)) {
             if (tid == 0) raise_error(p.err, GDN_ERR_TIMEOUT);
             break;
         }
-        GDN_CL_PHASE(1, 10);  // wait: slot free
-        if (warp == 1) {  // one bulk copy per lane; warp 0 moves on to the next gates
-            const uint32_t slot = c_base + (uint32_t)k * SLOT_BYTES;
-            if (lane == 0) {
-                const uint32_t bytes = 4 * 8192 + 16384 * (hp ? 2 : 1) + 32768 + 8192 +
-                                       (uint32_t)sizeof(GatesBlock);
-                mbar_arrive_expect_tx_remote(c_full, bytes);
-            }
-            __syncwarp();
-            uint32_t dst = 0, bytes = 0;
-            const uint8_t *src = nullptr;
-            switch (lane) {
-                case 0: dst = SL_K16; src = kqv; bytes = 8192; break;
-                case 1: dst = SL_K16 + 8192; src = kqv + 16384; bytes = 8192; break;
-                case 2: dst = SL_Q16; src = kqv + 8192; bytes = 8192; break;
-                case 3: dst = SL_Q16 + 8192; src = kqv + 16384 + 8192; bytes = 8192; break;
-                case 4: dst = SL_WH; src = sm + P_WST; bytes = 16384; break;
-                case 5: dst = SL_WL; src = sm + P_WST + 16384; bytes = hp ? 16384 : 0; break;
-                case 6: dst = SL_UT; src = sm + P_UTS; bytes = 32768; break;
-                case 7: dst = SL_P16; src = sm + P_P16; bytes = 8192; break;
-                case 8: dst = SL_GATES; src = sm + P_GST; bytes = (uint32_t)sizeof(GatesBlock); break;
-                default: break;
-            }
-            if (bytes) bulk_copy_to_cluster(slot + dst, src, bytes, c_full);
+        GDN_CL_PHASE(1, 10);  // wait: ring slot free
+        if (tid == 32) {  // one thread of warp 1 issues the stores; warp 0 moves on to the gates
+            uint8_t *dst = ring_slot(p, unit, k, rs);
+            bulk_store(dst + SL_K16, kqv, 8192);
+            bulk_store(dst + SL_K16 + 8192, kqv + 16384, 8192);
+            bulk_store(dst + SL_Q16, kqv + 8192, 8192);
+            bulk_store(dst + SL_Q16 + 8192, kqv + 16384 + 8192, 8192);
+            bulk_store(dst + SL_WH, sm + P_WST, hp ? 32768 : 16384);
+            bulk_store(dst + SL_UT, sm + P_UTS, 32768);
+            bulk_store(dst + SL_P16, sm + P_P16, 8192);
+            bulk_store(dst + SL_GATES, sm + P_GST, (uint32_t)sizeof(GatesBlock));
+            bulk_commit();
+            bulk_wait_all();              // written to global memory
+            fence_proxy_async_global();   // ... ordered before the signal below
+            mbar_arrive_remote(c_ready);
+            if (jj + 2 < nmine) issue_tma(buf, c0 + 4 * kC);  // this buffer is free now
         }
+        if (jj + 2 < nmine) tma_issued = jj + 3;
         GDN_CL_PHASE(1, 11);  // deliver (issue)
     }
-    // let the last delivery land, and a prefetched tile load that was never
-    // consumed, before this CTA's shared memory can go away
-    if (jj > 0) mbar_wait_cluster_bounded(&ms->copied, (jj - 1) & 1, kWaitLimit);
-    if (tma_issued > jj + 1) {
-        const int l = tma_issued - 1;
+    // a prefetched tile load that was never consumed must land before this
+    // CTA's shared memory can go away (every delivery's stores have drained)
+    for (int l = jj + 1; l < tma_issued; ++l)
         mbar_wait_bounded(&ms->tma_bar[l & 1], (l >> 1) & 1, kWaitLimit);
-    }
 }
 
 // ---------------------------------------------------------------- chain --
 
-__device__ void chain_role(uint8_t *sm, const ClusterParams &p, int n, int h, int64_t t_begin,
-                           int64_t t_end, int nch) {
+__device__ void chain_role(uint8_t *sm, const ClusterParams &p, int unit, int n, int h,
+                           int64_t t_begin, int64_t t_end, int nch) {
     ChainMisc *ms = reinterpret_cast<ChainMisc *>(sm + C_MISC);
     const uint32_t sbase = smem_u32(sm);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quad = warp & 3, half = warp >> 2, row = quad * 32 + lane;
     const uint32_t tmem = ms->tmem_base;
     const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
-    // producer-CTA barrier addresses (rank 1 + k)
-    const uint32_t prod_copied_local = sbase + P_MISC + (uint32_t)offsetof(ProdMisc, copied);
-    const uint32_t prod_freed_local = sbase + P_MISC + (uint32_t)offsetof(ProdMisc, freed);
+    // producer-CTA "taken" barriers (rank 1 + k)
+    const uint32_t prod_taken_local = sbase + P_MISC + (uint32_t)offsetof(ProdMisc, taken);
 
     // ---- initial state: fp32 -> TMEM accumulator, fp16 hi/lo -> TMEM A operands ----
     {
@@ -523,15 +519,22 @@ __device__ void chain_role(uint8_t *sm, const ClusterParams &p, int n, int h, in
 #ifdef GDN_TC_PHASES
     long long phase_t_ = clock64();
 #endif
-    // Thread 0 acknowledges each delivery as soon as it sees it complete (the
-    // producer may then reuse its buffers), polling for chunk c + 1 while
-    // chunk c is processed.
-    int acked = -1;
+    // Thread 0 loads chunk c + 1 from the ring into shared slot (c + 1) & 1 as
+    // soon as its producer reports it ready, while chunk c is processed; the
+    // slot held chunk c - 1, which is finished.
+    int loaded = 0;  // chunks whose load has been issued
+    auto issue_load = [&](int cc) {
+        const int kk = cc & 1, rs = (cc >> 1) & 1;
+        fence_proxy_async_global();  // the producer's stores, acquired, precede our bulk load
+        mbar_arrive_expect_tx(&ms->full[cc & 1], SLOT_BYTES);
+        bulk_load(sm + (cc & 1) * SLOT_BYTES, ring_slot(p, unit, kk, rs), SLOT_BYTES,
+                  &ms->full[cc & 1]);
+    };
     auto poll_next = [&](int cur) {
-        if (tid == 0 && acked == cur && cur + 1 < nch &&
-            mbar_try_wait_cluster(&ms->full[(cur + 1) & 1], ((cur + 1) >> 1) & 1)) {
-            mbar_arrive_remote(mapa_shared(prod_copied_local, 1 + ((cur + 1) & 1)));
-            acked = cur + 1;
+        if (tid == 0 && loaded == cur + 1 && cur + 1 < nch &&
+            mbar_try_wait_cluster(&ms->ready[(cur + 1) & 1], ((cur + 1) >> 1) & 1)) {
+            issue_load(cur + 1);
+            loaded = cur + 2;
         }
     };
     int c = 0;
@@ -543,12 +546,15 @@ __device__ void chain_role(uint8_t *sm, const ClusterParams &p, int n, int h, in
         const int64_t c0 = t_begin + (int64_t)kC * c;
         const int L = (int)((t_end - c0) < kC ? (t_end - c0) : kC);
 
-        if (!mbar_wait_cluster_bounded(&ms->full[k], (c >> 1) & 1, kWaitLimit)) timed_out = true;
-        GDN_CL_PHASE(0, 0);  // wait: delivery
-        if (tid == 0 && acked < c) {
-            mbar_arrive_remote(mapa_shared(prod_copied_local, 1 + k));
-            acked = c;
+        if (tid == 0 && loaded == c) {  // not prefetched: wait for the producer, then load
+            if (!mbar_wait_cluster_bounded(&ms->ready[k], (c >> 1) & 1, kWaitLimit)) timed_out = true;
+            issue_load(c);
+            loaded = c + 1;
         }
+        if (!mbar_wait_bounded(&ms->full[k], (c >> 1) & 1, kWaitLimit)) timed_out = true;
+        GDN_CL_PHASE(0, 0);  // wait: delivery
+        if (tid == 0)  // the chunk is out of the ring: its producer may deliver the next one
+            mbar_arrive_remote(mapa_shared(prod_taken_local, 1 + k));
         const GatesBlock *gb = reinterpret_cast<const GatesBlock *>(slot + SL_GATES);
         const bool hp = gb->hp != 0;
         const float gC = gb->Gam[kC - 1];
@@ -678,8 +684,6 @@ __device__ void chain_role(uint8_t *sm, const ClusterParams &p, int n, int h, in
         if (__syncthreads_or(timed_out ? 1 : 0)) {
             if (tid == 0) raise_error(p.err, GDN_ERR_TIMEOUT);
             aborted = true;
-        } else if (tid == 0) {
-            mbar_arrive_remote(mapa_shared(prod_freed_local, 1 + k));
         }
         tc_fence_after_sync();
         GDN_CL_PHASE(0, 6);  // vote, free the slot
@@ -698,12 +702,8 @@ __device__ void chain_role(uint8_t *sm, const ClusterParams &p, int n, int h, in
         }
     }
     if (aborted) {
-        // a delivery for the next chunk may be on its way: let it land, acknowledge it
-        if (c < nch && acked < c) {
-            const int k2 = c & 1;
-            if (mbar_wait_cluster_bounded(&ms->full[k2], (c >> 1) & 1, kWaitLimit) && tid == 0)
-                mbar_arrive_remote(mapa_shared(prod_copied_local, 1 + k2));
-        }
+        // a prefetched load may still be landing in shared memory: let it finish
+        if (loaded > c + 1) mbar_wait_bounded(&ms->full[(c + 1) & 1], ((c + 1) >> 1) & 1, kWaitLimit);
         mbar_wait_bounded(&ms->mma_bar, mma_phase ^ 1, kWaitLimit);
     }
 }
@@ -735,6 +735,8 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
         if (tid == 0) {
             mbar_init(&ms->full[0], 1);
             mbar_init(&ms->full[1], 1);
+            mbar_init(&ms->ready[0], 1);
+            mbar_init(&ms->ready[1], 1);
             mbar_init(&ms->mma_bar, 1);
             fence_mbarrier_init();
         }
@@ -746,8 +748,7 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
             mbar_init(&ms->tma_bar[0], 1);
             mbar_init(&ms->tma_bar[1], 1);
             mbar_init(&ms->mma_bar, 1);
-            mbar_init(&ms->copied, 1);
-            mbar_init(&ms->freed, 1);
+            mbar_init(&ms->taken, 1);
             fence_mbarrier_init();
             tma_prefetch_desc(&tm_q);
             tma_prefetch_desc(&tm_k);
@@ -764,9 +765,9 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
     tc_fence_after_sync();
 
     if (rank == 0)
-        chain_role(sm, p, n, h, t_begin, t_end, nch);
+        chain_role(sm, p, unit, n, h, t_begin, t_end, nch);
     else
-        producer_role(sm, &tm_q, &tm_k, &tm_v, p, rank - 1, h, j, t_begin, t_end, nch);
+        producer_role(sm, &tm_q, &tm_k, &tm_v, p, unit, rank - 1, h, j, t_begin, t_end, nch);
 
     tc_fence_before_sync();
     __syncthreads();
@@ -777,6 +778,10 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
+size_t prefill_cluster_workspace_bytes(int64_t units) {
+    return (size_t)units * 4 * SLOT_BYTES;
+}
+
 bool make_tile_map_bf16_128(CUtensorMap *m, const void *base, int64_t T, int32_t H);
 
 cudaError_t launch_prefill_cluster(const PrefillArgs &a, cudaStream_t s) {
@@ -786,7 +791,9 @@ cudaError_t launch_prefill_cluster(const PrefillArgs &a, cudaStream_t s) {
     if (!make_tile_map_bf16_128(&mq, a.q, Tm, a.Hqk) || !make_tile_map_bf16_128(&mk, a.k, Tm, a.Hqk) ||
         !make_tile_map_bf16_128(&mv, a.v, Tm, a.Hv))
         return cudaErrorInvalidValue;
+    if (a.ws == nullptr) return cudaErrorInvalidValue;
     ClusterParams p;
+    p.ws = static_cast<uint8_t *>(a.ws);
     p.g = a.g; p.beta = a.beta; p.s0 = a.s0; p.cu = a.cu; p.o = a.o; p.sT = a.sT; p.err = a.err;
     p.T = a.T; p.N = a.N; p.Hqk = a.Hqk; p.Hv = a.Hv;
     cudaError_t e = cudaFuncSetAttribute(gdn_prefill_cluster_kernel,

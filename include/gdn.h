@@ -114,15 +114,18 @@ GDN_API gdn_status gdn_prefill(const void *q, const void *k, const void *v, gdn_
                        void *stream);
 
 /*
- * Which prefill kernel runs.  AUTO picks the tensor-core cluster kernel for
- * Dk = Dv = 128, bf16 and chunk 0 or 64, and the exact recurrent kernel
- * otherwise.  Naming a tensor-core kernel for a shape it does not support
- * returns GDN_ERR_UNSUPPORTED.
+ * Which prefill kernel runs.  For Dk = Dv = 128, bf16 and chunk 0 or 64, AUTO
+ * picks the cluster kernel when there are at most 64 (sequence, v-head) units
+ * (few, long sequences: it puts three SMs on every unit) and the single-CTA
+ * kernel otherwise; every other shape runs the exact recurrent kernel.
+ * Naming a tensor-core kernel for a shape it does not support returns
+ * GDN_ERR_UNSUPPORTED.  The cluster kernel needs a workspace (see below).
  */
 typedef enum gdn_prefill_kernel {
     GDN_PREFILL_AUTO = 0,
     GDN_PREFILL_CLUSTER = 1,     /* tcgen05, a 3-CTA cluster per (sequence, head): one CTA
-                                    holds the state, two prepare alternate chunks */
+                                    holds the state, two prepare alternate chunks and
+                                    hand them over through an L2-resident workspace ring */
     GDN_PREFILL_SINGLE_CTA = 2,  /* tcgen05, one CTA per (sequence, head) */
     GDN_PREFILL_RECURRENT = 3    /* exact fp32 token recurrence on CUDA cores, any shape */
 } gdn_prefill_kernel;
@@ -141,10 +144,19 @@ GDN_API gdn_status gdn_prefill_ex(const void *q, const void *k, const void *v, g
 
 /*
  * gdn_prefill_workspace_bytes -- scratch bytes gdn_prefill needs for these
- * sizes (0 when none).  Pure function of its arguments; no device access.
+ * sizes (0 when none): 430,080 bytes per (sequence, v-head) unit when AUTO
+ * would run the cluster kernel.  Pure function of its arguments (it cannot see
+ * the dtype, so it may ask for a workspace an fp32 call does not use); no
+ * device access.  The workspace is device memory, 256-byte aligned, owned by
+ * the caller; its contents need no initialisation and are garbage afterwards.
  */
 GDN_API size_t gdn_prefill_workspace_bytes(int32_t N, int64_t T, int32_t Hqk, int32_t Hv, int32_t Dk,
                                    int32_t Dv, int32_t chunk);
+
+/* Scratch bytes gdn_prefill_ex needs with this kernel choice. */
+GDN_API size_t gdn_prefill_ex_workspace_bytes(int32_t N, int64_t T, int32_t Hqk, int32_t Hv,
+                                              int32_t Dk, int32_t Dv, int32_t chunk,
+                                              gdn_prefill_kernel kernel);
 
 /*
  * gdn_decode_step -- one-token inference update of N independent sequences

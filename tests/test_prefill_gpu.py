@@ -31,10 +31,12 @@ TC_KERNELS = ["cluster", "single_cta"]
 
 def run_gpu(inp, s0=None, cu=None, chunk=0, dev=DEV, kernel="auto"):
     t = lambda x: None if x is None else x.to(dev).contiguous()
+    flag = torch.zeros(4, dtype=torch.int32, device=dev)
     o, sT = gdn.gdn_prefill(t(inp["q"]), t(inp["k"]), t(inp["v"]), t(inp["g"]), t(inp["beta"]),
                             t(s0), None if cu is None else cu.to(torch.int32).to(dev), chunk=chunk,
-                            kernel=kernel)
+                            kernel=kernel, error_flag=flag)
     torch.cuda.synchronize()
+    assert int(flag[0]) == 0, f"device error {gdn.STATUS.get(int(flag[0]))}"
     return o.cpu(), sT.cpu()
 
 
