@@ -43,6 +43,7 @@ cudaError_t launch_prefill_tc(const PrefillArgs &a, cudaStream_t s);
 cudaError_t launch_prefill_cluster(const PrefillArgs &a, cudaStream_t s);
 // Workspace of the cluster kernel: a 4-slot ring per (sequence, head).
 size_t prefill_cluster_workspace_bytes(int64_t units);
+constexpr size_t kClusterWorkspaceBytesPerUnit = 430080;
 // AUTO uses the cluster kernel up to this many (sequence, head) units.
 constexpr int64_t kClusterMaxUnits = 64;
 

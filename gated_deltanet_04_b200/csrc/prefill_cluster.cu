@@ -778,6 +778,8 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
+static_assert(4 * SLOT_BYTES == kClusterWorkspaceBytesPerUnit, "ring size per unit");
+
 size_t prefill_cluster_workspace_bytes(int64_t units) {
     return (size_t)units * 4 * SLOT_BYTES;
 }

@@ -177,6 +177,46 @@ GDN_API gdn_status gdn_decode_step(const void *q, const void *k, const void *v, 
                            int32_t Hqk, int32_t Hv, int32_t Dk, int32_t Dv, void *o,
                            int32_t *dev_error_flag, void *stream);
 
+/*
+ * gdn_prefill_static_workspace -- gdn_prefill_ex with kernel
+ * GDN_PREFILL_CLUSTER, but the cluster kernel's workspace ring lives in a
+ * fixed device array inside libgdn, so the call allocates nothing and takes
+ * no workspace argument.  The paper has no counterpart to this entry point; it exists
+ * for callers that cannot hand out device memory at call time: a host program
+ * that links only this C ABI and has no device allocator of its own, or a
+ * runtime whose device memory is planned once up front and may not grow or be
+ * carved up per call.
+ *
+ * All other arguments, layouts and results are those of gdn_prefill_ex; the
+ * results are bit-identical to gdn_prefill_ex(..., GDN_PREFILL_CLUSTER) with
+ * a caller-supplied workspace.
+ *
+ * Limit: N * Hv <= GDN_STATIC_WORKSPACE_MAX_UNITS (48 units, a 20,643,840-byte
+ * array, 430,080 bytes per unit).  Larger calls return GDN_ERR_UNSUPPORTED
+ * before any CUDA call; use gdn_prefill_ex with a workspace for them.
+ * Shapes the cluster kernel does not take (not bf16, Dk or Dv != 128, chunk
+ * not 0 or 64) also return GDN_ERR_UNSUPPORTED.
+ *
+ * Set-up: the first call on a device (with that device current) looks up the
+ * array's device address once and caches it per device; a failure there
+ * returns GDN_ERR_CUDA.  Make that first call before any stream capture.
+ * Depending on the CUDA module loading mode, the array's device memory is
+ * reserved when libgdn's module is loaded or at that first call.
+ *
+ * Nothing in the array has to start at zero: within one call every ring slot
+ * is written before it is read.  There is one array per device, so calls whose
+ * execution overlaps on the same device (different streams, or threads not
+ * ordered on one stream) race on it and give wrong results; order them.
+ */
+#define GDN_STATIC_WORKSPACE_MAX_UNITS 48
+GDN_API gdn_status gdn_prefill_static_workspace(const void *q, const void *k, const void *v,
+                                                gdn_dtype io_dtype, const float *g,
+                                                const float *beta, const float *initial_state,
+                                                const int32_t *cu_seqlens, int32_t N, int64_t T,
+                                                int32_t Hqk, int32_t Hv, int32_t Dk, int32_t Dv,
+                                                int32_t chunk, void *o, float *final_state,
+                                                int32_t *dev_error_flag, void *stream);
+
 /* Human-readable name of a status code (static storage, never NULL). */
 GDN_API const char *gdn_status_string(gdn_status status);
 
