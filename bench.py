@@ -60,7 +60,7 @@ def parse():
                    help="profiling mode: run one operation of a named workload (layer4k, "
                         "long256k, varlen32: one gdn_prefill call; decode256: one layer's "
                         "gdn_decode_step) W + K times and print its per-call time; no bench line")
-    p.add_argument("--kernel", default="auto", choices=["auto", "cluster", "single_cta", "recurrent"],
+    p.add_argument("--kernel", default="auto", choices=["auto", "pool", "cluster", "single_cta", "recurrent"],
                    help="prefill kernel for --case")
     return p.parse_args()
 
@@ -391,15 +391,15 @@ def main():
                "ms_per_step": e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     # --------------------------------------------------------- roofline --
-    # Dk = Dv = 128, bf16, chunk 64: the library's default is the cluster kernel
+    # Dk = Dv = 128, bf16, chunk 64, 48 units: the library's default is the pool kernel
     flops = PREFILL_FLOP_PER_TOKEN * T
     achieved_tf = flops / (p_launch_ms / 1e3) / 1e12
     achieved_gbs = PREFILL_BYTES_PER_TOKEN * T / (p_launch_ms / 1e3) / 1e9
     roofline = {"bound": "tensor", "achieved": achieved_tf, "peak": peaks["bf16_tflops"],
                 "unit": "TFLOP/s", "frac": achieved_tf / peaks["bf16_tflops"],
-                "traffic": traffic_for("gdn_prefill_cluster", "prefill_cluster.cu"),
+                "traffic": traffic_for("gdn_prefill_pool", "prefill_chain.cu"),
                 "peak_source": f"{peaks['source']} bf16 burst",
-                "kernel": "gdn_prefill_cluster_kernel",
+                "kernel": "gdn_prefill_pool_kernel",
                 "algorithmic_flop_per_launch": flops,
                 "hbm": {"achieved": achieved_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                         "frac": achieved_gbs / peaks["hbm_gbs"],

@@ -28,7 +28,7 @@ STATUS = {0: "GDN_OK", 1: "GDN_ERR_INVALID_ARGUMENT", 2: "GDN_ERR_UNSUPPORTED", 
           4: "GDN_ERR_TIMEOUT", 5: "GDN_ERR_BAD_SEQLENS"}
 DTYPE = {torch.bfloat16: 0, torch.float32: 1}
 # gdn_prefill_kernel values of include/gdn.h
-KERNELS = {"auto": 0, "cluster": 1, "single_cta": 2, "recurrent": 3}
+KERNELS = {"auto": 0, "cluster": 1, "single_cta": 2, "recurrent": 3, "pool": 4}
 
 _lib = None
 _lock = threading.Lock()
@@ -107,7 +107,7 @@ def gdn_prefill(q, k, v, g, beta, initial_state=None, cu_seqlens=None, *, chunk=
     initial_state [N,Hv,Dv,Dk] fp32 or None; cu_seqlens int32 [N+1] on the device or None.
     Returns (o [T,Hv,Dv], final_state [N,Hv,Dv,Dk] or None).  ``final_state`` may be
     ``initial_state`` for an in-place update.  Asynchronous on the current stream.
-    ``kernel``: "auto", "cluster", "single_cta" or "recurrent" (see gdn_prefill_ex).
+    ``kernel``: "auto", "pool", "cluster", "single_cta" or "recurrent" (see gdn_prefill_ex).
     """
     lib = library()
     dev = q.device

@@ -38,7 +38,14 @@ int32_t gdn_version(void) { return 1 * 10000 + 0 * 100 + 0; }
 gdn_prefill_kernel resolve_kernel(gdn_prefill_kernel kernel, bool tc_ok, int64_t units) {
     if (kernel != GDN_PREFILL_AUTO) return kernel;
     if (!tc_ok) return GDN_PREFILL_RECURRENT;
-    return units <= gdn::kClusterMaxUnits ? GDN_PREFILL_CLUSTER : GDN_PREFILL_SINGLE_CTA;
+    return units <= gdn::kPoolMaxUnits ? GDN_PREFILL_POOL : GDN_PREFILL_SINGLE_CTA;
+}
+
+// Scratch bytes of a resolved kernel choice.
+size_t workspace_need(gdn_prefill_kernel kernel, int64_t units) {
+    if (kernel == GDN_PREFILL_CLUSTER) return gdn::prefill_cluster_workspace_bytes(units);
+    if (kernel == GDN_PREFILL_POOL) return gdn::prefill_pool_workspace_bytes(units);
+    return 0;
 }
 
 size_t gdn_prefill_ex_workspace_bytes(int32_t N, int64_t T, int32_t Hqk, int32_t Hv, int32_t Dk,
@@ -46,8 +53,8 @@ size_t gdn_prefill_ex_workspace_bytes(int32_t N, int64_t T, int32_t Hqk, int32_t
     (void)T; (void)Hqk;
     if (N <= 0 || Hv <= 0) return 0;
     const bool shape_ok = Dk == 128 && Dv == 128 && (chunk == 0 || chunk == 64);
-    if (resolve_kernel(kernel, shape_ok, (int64_t)N * Hv) != GDN_PREFILL_CLUSTER || !shape_ok) return 0;
-    return gdn::prefill_cluster_workspace_bytes((int64_t)N * Hv);
+    if (!shape_ok) return 0;
+    return workspace_need(resolve_kernel(kernel, shape_ok, (int64_t)N * Hv), (int64_t)N * Hv);
 }
 
 size_t gdn_prefill_workspace_bytes(int32_t N, int64_t T, int32_t Hqk, int32_t Hv, int32_t Dk,
@@ -72,7 +79,7 @@ gdn_status gdn_prefill_ex(const void *q, const void *k, const void *v, gdn_dtype
                           int32_t Hv, int32_t Dk, int32_t Dv, int32_t chunk, void *o,
                           float *final_state, void *workspace, size_t workspace_bytes,
                           int32_t *dev_error_flag, void *stream, gdn_prefill_kernel kernel) {
-    if (kernel < GDN_PREFILL_AUTO || kernel > GDN_PREFILL_RECURRENT) return GDN_ERR_INVALID_ARGUMENT;
+    if (kernel < GDN_PREFILL_AUTO || kernel > GDN_PREFILL_POOL) return GDN_ERR_INVALID_ARGUMENT;
     if (io_dtype != GDN_DTYPE_BF16 && io_dtype != GDN_DTYPE_F32) return GDN_ERR_INVALID_ARGUMENT;
     if (N < 0 || T < 0 || Hqk <= 0 || Hv <= 0 || Dk <= 0 || Dv <= 0 || chunk < 0)
         return GDN_ERR_INVALID_ARGUMENT;
@@ -87,12 +94,12 @@ gdn_status gdn_prefill_ex(const void *q, const void *k, const void *v, gdn_dtype
     if (o && (o == q || o == k || o == v)) return GDN_ERR_INVALID_ARGUMENT;
     if (!supported_dim(Dk) || !supported_dim(Dv) || chunk > 64) return GDN_ERR_UNSUPPORTED;
     const bool tc_ok = tc_path(io_dtype, Dk, Dv, chunk);
-    if ((kernel == GDN_PREFILL_CLUSTER || kernel == GDN_PREFILL_SINGLE_CTA) && !tc_ok)
+    if ((kernel == GDN_PREFILL_CLUSTER || kernel == GDN_PREFILL_SINGLE_CTA ||
+         kernel == GDN_PREFILL_POOL) && !tc_ok)
         return GDN_ERR_UNSUPPORTED;
+    if (kernel == GDN_PREFILL_POOL && (int64_t)N * Hv > gdn::kPoolMaxUnits) return GDN_ERR_UNSUPPORTED;
     kernel = resolve_kernel(kernel, tc_ok, (int64_t)N * Hv);
-    const size_t need = (kernel == GDN_PREFILL_CLUSTER && T > 0)
-                            ? gdn::prefill_cluster_workspace_bytes((int64_t)N * Hv)
-                            : 0;
+    const size_t need = T > 0 ? workspace_need(kernel, (int64_t)N * Hv) : 0;
     if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return GDN_ERR_INVALID_ARGUMENT;
     if (T == 0 && final_state == nullptr) return GDN_OK;  // nothing observable to do
 
@@ -103,6 +110,7 @@ gdn_status gdn_prefill_ex(const void *q, const void *k, const void *v, gdn_dtype
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (T == 0 || kernel == GDN_PREFILL_RECURRENT) return from_cuda(gdn::launch_prefill_recurrent(a, s));
     if (kernel == GDN_PREFILL_SINGLE_CTA) return from_cuda(gdn::launch_prefill_tc(a, s));
+    if (kernel == GDN_PREFILL_POOL) return from_cuda(gdn::launch_prefill_pool(a, s));
     return from_cuda(gdn::launch_prefill_cluster(a, s));
 }
 

@@ -41,11 +41,19 @@ cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s);
 // (sequence, head), or a 3-CTA cluster per (sequence, head).
 cudaError_t launch_prefill_tc(const PrefillArgs &a, cudaStream_t s);
 cudaError_t launch_prefill_cluster(const PrefillArgs &a, cudaStream_t s);
+// Chain CTA per (sequence, head) plus producer CTAs on every other SM, one
+// cooperative launch.  Falls back to launch_prefill_tc on a GPU with too few
+// SMs for the units.
+cudaError_t launch_prefill_pool(const PrefillArgs &a, cudaStream_t s);
 // Workspace of the cluster kernel: a 4-slot ring per (sequence, head).
 size_t prefill_cluster_workspace_bytes(int64_t units);
 constexpr size_t kClusterWorkspaceBytesPerUnit = 430080;
-// AUTO uses the cluster kernel up to this many (sequence, head) units.
-constexpr int64_t kClusterMaxUnits = 64;
+// Workspace of the pool kernel: hand-off flags, then the same ring.
+size_t prefill_pool_workspace_bytes(int64_t units);
+// AUTO uses the pool kernel up to this many (sequence, head) units.
+constexpr int64_t kPoolMaxUnits = 64;
+// Whether the current device has SMs enough for the pool kernel with `units`.
+bool prefill_pool_fits(int64_t units);
 
 // ---------------------------------------------------------------- device --
 

@@ -1,5 +1,6 @@
-// Chunk-parallel prefill of the gated delta rule on a 3-CTA thread-block
-// cluster per (sequence, v-head).
+// Chunk-parallel prefill of the gated delta rule split across CTAs: one
+// "chain" CTA per (sequence, v-head) carries the state from chunk to chunk,
+// and "producer" CTAs prepare the chunks.
 //
 // The math is the chunk step of the single-CTA kernel (see prefill_tc.cu):
 //     A = strict-lower(diag(b)(K K^T (.) M)),   T = (I + A)^-1
@@ -9,46 +10,58 @@
 // 长上下文", section 三.  Only U (through S) links one chunk to the next; every
 // other quantity of a chunk depends on that chunk's inputs alone.
 //
-// Work split (one SM per CTA):
-//   * rank 0, the chain CTA, keeps the fp32 state as a TMEM accumulator and
-//     its fp16 hi/lo copies as TMEM A operands, and runs only the state-
-//     dependent products of each chunk: S Q^T, R = S W^T, U = U~ - R, the state
-//     update S += U'^T K, O += U^T P^T, and the output stores.
-//   * ranks 1 and 2, the producer CTAs, take alternate chunks (rank 1 even,
-//     rank 2 odd): TMA tile loads, bf16 -> fp16, Gram matrices, decay factors,
-//     the triangular solve, U~ and W on tensor cores.
+// Roles (one SM per CTA):
+//   * the chain CTA keeps the fp32 state as a TMEM accumulator and its fp16
+//     hi/lo copies as TMEM A operands, and runs only the state-dependent
+//     products of each chunk: S Q^T, R = S W^T, U = U~ - R, the state update
+//     S += U'^T K, O += U^T P^T, and the output stores.
+//   * a producer CTA takes whole chunks: TMA tile loads, bf16 -> fp16, Gram
+//     matrices, decay factors, the triangular solve, U~ and W on tensor cores.
 // A finished chunk (K, Q, W^T hi/lo, U~, P, gates: one 105 KB block laid out
 // exactly like a chain slot) goes through L2: the producer bulk-stores it
-// into a ring of 2 slots per producer in the caller's workspace, the chain
-// bulk-loads it into one of its two shared-memory slots while it computes
-// the previous chunk.  Distributed shared memory carries only the signals
-// (it moves bulk data far more slowly than L2); the ring is 420 KB per
-// (sequence, head) and stays resident in L2.
+// into a ring of kRingSlots slots per (sequence, head) in the caller's
+// workspace, and the chain bulk-loads it into one of its two shared-memory
+// slots while it computes the previous chunk.  Chunk c of a unit always uses
+// ring slot c % kRingSlots.
 //
-// Flow control (all waits bounded; a wait that expires is voted on once per
-// chunk, reports GDN_ERR_TIMEOUT and ends the CTA's loop):
-//   ready[k] (chain)    : producer k's stores of its next chunk are complete
-//   full[i]  (chain)    : the bulk load into shared slot i has landed
-//   taken    (producer) : the chain has loaded this producer's last delivery
-// A producer delivers chunk j only after the chain has taken chunk j - 1:
-// then no barrier ever runs more than one phase ahead of its waiter (a
-// parity wait cannot tell phase n from phase n + 2), and the ring slot of
-// chunk j, last used by chunk j - 2, is free.
-// A cluster barrier after set-up and another before exit keep every CTA's
-// shared memory alive while the others may still address it.  No TMA load
-// uses multicast.
-#include <mutex>
-
+// Two ways to schedule the producers:
+//   * cluster kernel: a 3-CTA cluster per unit, rank 0 the chain, ranks 1 and
+//     2 producers of the even and odd chunks.  Signals are mbarriers reached
+//     through distributed shared memory:
+//         ready[k] (chain)    producer k's stores of its next chunk are complete
+//         full[i]  (chain)    the bulk load into shared slot i has landed
+//         taken    (producer) the chain has loaded this producer's last delivery
+//     A producer delivers its chunk only after the chain has taken its
+//     previous one, so no barrier runs more than one phase ahead of its waiter
+//     (a parity wait cannot tell phase n from n + 2).  A B200 holds at most 45
+//     such clusters at once, so more than 45 units run in two waves.
+//   * pool kernel: a cooperative launch of one CTA per SM; CTA u < units is
+//     the chain of unit u, every other CTA is a producer that takes chunks
+//     from a global counter in chunk-major order (chunk 0 of every unit, then
+//     chunk 1, ...).  Signals are 32-bit flags in the workspace with gpu-scope
+//     release / acquire:
+//         ready[u][s]  = c + 1   chunk c of unit u is in ring slot s
+//         taken[u]     = c + 1   the chain of unit u has loaded chunks 0..c
+//     A producer writes chunk c only after taken[u] >= c - kRingSlots + 1.
+//     Every wait is on a chunk of lower counter index, and a producer works
+//     through its chunks in counter order, so the lowest unfinished chunk can
+//     always proceed: no deadlock while every CTA is resident, which the
+//     cooperative launch guarantees.
+//
+// Every wait is bounded; an expired wait is voted on once per chunk, reports
+// GDN_ERR_TIMEOUT and ends the CTA's loop (the pool kernel also raises its
+// abort flag so that every other CTA stops waiting).  No TMA load uses
+// multicast.
 #include "gdn_internal.cuh"
 #include "sm100.cuh"
 #include "tc_common.cuh"
 
 #ifdef GDN_TC_PHASES
-// per-phase SM clocks of cluster 0: [0] chain CTA, [1] first producer CTA
+// per-phase SM clocks: [0] the first chain CTA, [1] the first producer CTA
 __device__ long long gdn_cl_phase_clk[2][16];
 #define GDN_CL_PHASE(role, k)                                          \
     do {                                                               \
-        if (threadIdx.x == 0 && blockIdx.x < 2) {                      \
+        if (threadIdx.x == 0 && phase_on_) {                           \
             const long long now_ = clock64();                          \
             gdn_cl_phase_clk[(role)][(k)] += now_ - phase_t_;          \
             phase_t_ = now_;                                           \
@@ -66,6 +79,7 @@ using namespace tc;
 
 constexpr int kThreads = 256;
 constexpr int kCluster = 3;
+constexpr int kRingSlots = 4;
 
 // ---- chain CTA: two hand-off slots (offsets inside a slot) ----
 constexpr uint32_t SL_K16 = 0;         // K fp16: d-halves at +0 / +8192 ([64 rows][128 B], SW128)
@@ -118,8 +132,17 @@ static_assert(P_XS + 1024 * 4 <= P_UTS, "solve scratch overflows");
 static_assert(P_GST + sizeof(GatesBlock) <= P_X + 49152, "gates staging stays inside the region");
 static_assert(P_TS % 16 == 0 && P_XS % 16 == 0, "float4 scratch must be aligned");
 
+// One chunk of one unit, as a producer sees it.
+struct Item {
+    int64_t c0;       // first token
+    int32_t unit, c;  // unit = n * Hv + h; chunk index within the sequence
+    int32_t h, j, L;  // v head, q/k head, valid rows
+    int32_t valid;
+};
+
 struct ProdMisc {
     float gam[kC], Gam[kC], iGam[kC], eC[kC], bb[kC], bG[kC];
+    Item items[4];    // this CTA's chunks l .. l + 2, by l % 4
     uint64_t tma_bar[2];
     uint64_t mma_bar;
     uint64_t taken;
@@ -129,23 +152,39 @@ struct ProdMisc {
 };
 constexpr uint32_t kSmemBytes = P_MISC + sizeof(ProdMisc) + 1024;
 static_assert(C_MISC + sizeof(ChainMisc) <= P_MISC + sizeof(ProdMisc), "chain misc fits");
+static_assert(kSmemBytes <= 232448, "fits the 227 KB opt-in shared memory of a CTA");
 
 // producer TMEM columns (128 allocated)
 constexpr uint32_t PT_G = 0, PT_U = 64;
 
-struct ClusterParams {
-    uint8_t *ws;  // ring: [unit][producer][2 slots][SLOT_BYTES]
+// pool flags: a header of kFlagHeader words ([0] the chunk counter, [1] the
+// abort flag), then 8 words per unit ([0] taken, [1 + s] ready of slot s)
+constexpr int kFlagHeader = 64;
+constexpr int kFlagsPerUnit = 8;
+static_assert(1 + kRingSlots <= kFlagsPerUnit, "flag words per unit");
+
+struct ChainParams {
+    uint8_t *ring;    // [unit][kRingSlots][SLOT_BYTES]
+    uint32_t *flags;  // pool kernel only
     const float *g, *beta, *s0;
     const int32_t *cu;
     void *o;
     float *sT;
     int32_t *err;
     int64_t T;
-    int32_t N, Hqk, Hv;
+    int32_t N, Hqk, Hv, units, max_chunks;
 };
 
-__device__ __forceinline__ uint8_t *ring_slot(const ClusterParams &p, int unit, int k, int s) {
-    return p.ws + ((size_t)(unit * 2 + k) * 2 + s) * SLOT_BYTES;
+__device__ __forceinline__ uint8_t *ring_slot(const ChainParams &p, int unit, int c) {
+    return p.ring + ((size_t)unit * kRingSlots + (c % kRingSlots)) * SLOT_BYTES;
+}
+
+__device__ __forceinline__ uint32_t *unit_flags(const ChainParams &p, int unit) {
+    return p.flags + kFlagHeader + kFlagsPerUnit * unit;
+}
+
+__device__ __forceinline__ void pool_abort(const ChainParams &p) {
+    atomicExch(p.flags + 1, 1u);
 }
 
 // byte offset of 16-byte chunk q of row i in a [128][64] fp32 U~ tile
@@ -153,10 +192,40 @@ __device__ __forceinline__ uint32_t ut_off(int i, int q) {
     return (uint32_t)i * 256u + (uint32_t)((q ^ (i & 15)) << 4);
 }
 
+// The next chunk of the pool kernel's chunk-major order that exists (invalid
+// once the order is exhausted or the abort flag is up).  One thread calls it.
+__device__ Item pool_fetch(const ChainParams &p) {
+    Item it;
+    it.valid = 0;
+    for (;;) {
+        if (ld_relaxed_gpu(p.flags + 1) != 0u) return it;
+        const uint32_t i = atomicAdd(p.flags, 1u);
+        const int c = (int)(i / (uint32_t)p.units);
+        const int unit = (int)(i % (uint32_t)p.units);
+        if (c >= p.max_chunks) return it;
+        const int n = unit / p.Hv;
+        int64_t t0, t1;
+        if (!seq_range(p.cu, n, p.N, p.T, nullptr, t0, t1)) continue;  // the chain reports it
+        const int64_t c0 = t0 + (int64_t)kC * c;
+        if (c0 >= t1) continue;  // a shorter sequence
+        it.c0 = c0;
+        it.unit = unit;
+        it.c = c;
+        it.h = unit % p.Hv;
+        it.j = it.h / (p.Hv / p.Hqk);
+        it.L = (int)((t1 - c0) < kC ? (t1 - c0) : kC);
+        it.valid = 1;
+        return it;
+    }
+}
+
 // ------------------------------------------------------------- producer --
 
+// kPool: the pool kernel (chunks from the global counter); otherwise producer
+// k of a cluster, whose chunks are k, k + 2, ... of `unit`.
+template <bool kPool>
 __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtensorMap *tm_k,
-                              const CUtensorMap *tm_v, const ClusterParams &p, int unit, int k,
+                              const CUtensorMap *tm_v, const ChainParams &p, int unit, int k,
                               int h, int j, int64_t t_begin, int64_t t_end, int nch) {
     ProdMisc *ms = reinterpret_cast<ProdMisc *>(sm + P_MISC);
     const uint32_t sbase = smem_u32(sm);
@@ -164,29 +233,45 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
     const int quad = warp & 3, half = warp >> 2, row = quad * 32 + lane;
     const uint32_t tmem = ms->tmem_base;
     const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
-    // the chain CTA's ready barrier for this producer (rank 0)
+    // cluster: the chain CTA's ready barrier for this producer (rank 0)
     const uint32_t c_ready =
-        mapa_shared(sbase + C_MISC + (uint32_t)offsetof(ChainMisc, ready) + 8u * k, 0);
-    const int nmine = nch > k ? (nch - k + 1) / 2 : 0;
+        kPool ? 0u : mapa_shared(sbase + C_MISC + (uint32_t)offsetof(ChainMisc, ready) + 8u * k, 0);
+
+    auto fetch = [&](int l) -> Item {
+        if constexpr (kPool) {
+            return pool_fetch(p);
+        } else {
+            Item it;
+            const int c = k + 2 * l;
+            it.valid = c < nch;
+            it.c0 = t_begin + (int64_t)kC * c;
+            it.unit = unit;
+            it.c = c;
+            it.h = h;
+            it.j = j;
+            it.L = (int)((t_end - it.c0) < kC ? (t_end - it.c0) : kC);
+            return it;
+        }
+    };
 
     uint32_t mma_phase = 0;
     bool timed_out = false;
     float gpre0 = 0.f, gpre1 = 0.f, bpre0 = 0.f, bpre1 = 0.f;
-    auto load_gates = [&](int64_t tok0) {
+    auto load_gates = [&](const Item &it) {
         gpre0 = gpre1 = bpre0 = bpre1 = 0.f;
-        const int64_t t0_ = tok0 + 2 * lane, t1_ = t0_ + 1;
-        if (t0_ < t_end) { gpre0 = p.g[t0_ * p.Hv + h]; bpre0 = p.beta[t0_ * p.Hv + h]; }
-        if (t1_ < t_end) { gpre1 = p.g[t1_ * p.Hv + h]; bpre1 = p.beta[t1_ * p.Hv + h]; }
+        const int64_t t0_ = it.c0 + 2 * lane, t1_ = t0_ + 1, te = it.c0 + it.L;
+        if (t0_ < te) { gpre0 = p.g[t0_ * p.Hv + it.h]; bpre0 = p.beta[t0_ * p.Hv + it.h]; }
+        if (t1_ < te) { gpre1 = p.g[t1_ * p.Hv + it.h]; bpre1 = p.beta[t1_ * p.Hv + it.h]; }
     };
-    auto issue_tma = [&](int buf, int64_t tok0) {
+    auto issue_tma = [&](int buf, const Item &it) {
         uint8_t *b = sm + P_KQV + buf * P_KQV_BYTES;
         mbar_arrive_expect_tx(&ms->tma_bar[buf], 6 * 8192);
-        const int32_t t32 = (int32_t)tok0;
+        const int32_t t32 = (int32_t)it.c0;
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
-            tma_load_3d(b + hf * 16384, tm_k, &ms->tma_bar[buf], 64 * hf, j, t32);
-            tma_load_3d(b + hf * 16384 + 8192, tm_q, &ms->tma_bar[buf], 64 * hf, j, t32);
-            tma_load_3d(b + 32768 + hf * 8192, tm_v, &ms->tma_bar[buf], 64 * hf, h, t32);
+            tma_load_3d(b + hf * 16384, tm_k, &ms->tma_bar[buf], 64 * hf, it.j, t32);
+            tma_load_3d(b + hf * 16384 + 8192, tm_q, &ms->tma_bar[buf], 64 * hf, it.j, t32);
+            tma_load_3d(b + 32768 + hf * 8192, tm_v, &ms->tma_bar[buf], 64 * hf, it.h, t32);
         }
     };
     auto mma_sync_point = [&]() {
@@ -203,25 +288,31 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
         tc_fence_after_sync();
     };
 
-    // Tile loads: local chunks 0 and 1 now; chunk jj + 2 by the delivery thread
-    // of chunk jj, into the buffer its stores have just drained.
-    int tma_issued = 0;  // tile loads issued (local chunk indices 0 .. tma_issued-1)
-    for (int l = 0; l < 2 && l < nmine; ++l) {
-        if (tid == 32) issue_tma(l, t_begin + (int64_t)kC * (k + 2 * l));
-        tma_issued = l + 1;
+    // Chunks l and l + 1 are known (and their tile loads issued) when chunk l
+    // starts; the delivery thread fetches chunk l + 2 before the vote of chunk
+    // l and issues its tile loads into chunk l's buffer once that buffer's
+    // stores have drained.
+    if (tid == 32) {
+        for (int l = 0; l < 2; ++l) {
+            const Item it = fetch(l);
+            ms->items[l] = it;
+            if (it.valid) issue_tma(l, it);
+        }
     }
-    if (nmine > 0 && warp == 0) load_gates(t_begin + (int64_t)kC * k);
+    __syncthreads();
+    if (warp == 0 && ms->items[0].valid) load_gates(ms->items[0]);
 #ifdef GDN_TC_PHASES
     long long phase_t_ = clock64();
+    const bool phase_on_ = blockIdx.x == (kPool ? (unsigned)p.units : 1u);
 #endif
-    int jj = 0;
+    int l = 0;
+    bool broke = false;
 #pragma unroll 1
-    for (; jj < nmine; ++jj) {
-        const int c = k + 2 * jj;
-        const int64_t c0 = t_begin + (int64_t)kC * c;
-        const int L = (int)((t_end - c0) < kC ? (t_end - c0) : kC);
-        const int buf = jj & 1;
-        const bool more = jj + 1 < nmine;
+    for (;; ++l) {
+        const Item it = ms->items[l & 3];
+        if (!it.valid) break;
+        const int L = it.L;
+        const int buf = l & 1;
 
         // ---- gates (warp 0, two tokens per lane) ----
         if (warp == 0) {
@@ -250,12 +341,13 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
                 ms->safe = safe_;
                 ms->hp = expf(gC) >= kHighPrecisionDecay;
             }
-            if (more) load_gates(c0 + 2 * kC);
+            const Item nx = ms->items[(l + 1) & 3];
+            if (nx.valid) load_gates(nx);
         }
 
         GDN_CL_PHASE(1, 0);  // gates
         GDN_CL_PHASE(1, 1);  // (no wait)
-        if (!mbar_wait_bounded(&ms->tma_bar[buf], (jj >> 1) & 1, kWaitLimit)) timed_out = true;
+        if (!mbar_wait_bounded(&ms->tma_bar[buf], (l >> 1) & 1, kWaitLimit)) timed_out = true;
         GDN_CL_PHASE(1, 2);  // wait: tiles
 
         // ---- bf16 -> fp16 in place, zero padding rows ----
@@ -423,17 +515,31 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
         __syncthreads();
         GDN_CL_PHASE(1, 9);  // staging
 
-        // ---- deliver through the L2 ring, once the chain has taken our previous chunk ----
-        const int rs = jj & 1;
-        if (jj >= 1 && !mbar_wait_cluster_bounded(&ms->taken, (jj - 1) & 1, kWaitLimit))
-            timed_out = true;
+        // ---- deliver through the L2 ring once its slot is free ----
+        if (tid == 32) {
+            ms->items[(l + 2) & 3] = fetch(l + 2);
+            if constexpr (kPool) {
+                if (it.c >= kRingSlots &&
+                    !wait_flag_geq(unit_flags(p, it.unit), (uint32_t)(it.c - kRingSlots + 1),
+                                   p.flags + 1, kWaitLimit))
+                    timed_out = true;
+            } else {
+                if (l >= 1 && !mbar_wait_cluster_bounded(&ms->taken, (l - 1) & 1, kWaitLimit))
+                    timed_out = true;
+            }
+        }
         if (__syncthreads_or(timed_out ? 1 : 0)) {
-            if (tid == 0) raise_error(p.err, GDN_ERR_TIMEOUT);
+            if (tid == 0) {
+                raise_error(p.err, GDN_ERR_TIMEOUT);
+                if constexpr (kPool) pool_abort(p);
+            }
+            broke = true;
             break;
         }
         GDN_CL_PHASE(1, 10);  // wait: ring slot free
         if (tid == 32) {  // one thread of warp 1 issues the stores; warp 0 moves on to the gates
-            uint8_t *dst = ring_slot(p, unit, k, rs);
+            uint8_t *dst = ring_slot(p, it.unit, it.c);
+            fence_proxy_async_global();  // the chain's reads of this slot precede our writes
             bulk_store(dst + SL_K16, kqv, 8192);
             bulk_store(dst + SL_K16 + 8192, kqv + 16384, 8192);
             bulk_store(dst + SL_Q16, kqv + 8192, 8192);
@@ -445,21 +551,26 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
             bulk_commit();
             bulk_wait_all();              // written to global memory
             fence_proxy_async_global();   // ... ordered before the signal below
-            mbar_arrive_remote(c_ready);
-            if (jj + 2 < nmine) issue_tma(buf, c0 + 4 * kC);  // this buffer is free now
+            if constexpr (kPool)
+                st_release_gpu(unit_flags(p, it.unit) + 1 + it.c % kRingSlots, (uint32_t)(it.c + 1));
+            else
+                mbar_arrive_remote(c_ready);
+            const Item nx2 = ms->items[(l + 2) & 3];
+            if (nx2.valid) issue_tma(buf, nx2);  // this buffer is free now
         }
-        if (jj + 2 < nmine) tma_issued = jj + 3;
         GDN_CL_PHASE(1, 11);  // deliver (issue)
     }
-    // a prefetched tile load that was never consumed must land before this
-    // CTA's shared memory can go away (every delivery's stores have drained)
-    for (int l = jj + 1; l < tma_issued; ++l)
-        mbar_wait_bounded(&ms->tma_bar[l & 1], (l >> 1) & 1, kWaitLimit);
+    // A tile load issued for a chunk this loop never reached must land before
+    // this CTA's shared memory can go away (chunk l + 1's, after a timeout;
+    // on a normal exit chunks l and l + 1 do not exist).
+    if (broke && ms->items[(l + 1) & 3].valid)
+        mbar_wait_bounded(&ms->tma_bar[(l + 1) & 1], ((l + 1) >> 1) & 1, kWaitLimit);
 }
 
 // ---------------------------------------------------------------- chain --
 
-__device__ void chain_role(uint8_t *sm, const ClusterParams &p, int unit, int n, int h,
+template <bool kPool>
+__device__ void chain_role(uint8_t *sm, const ChainParams &p, int unit, int n, int h,
                            int64_t t_begin, int64_t t_end, int nch) {
     ChainMisc *ms = reinterpret_cast<ChainMisc *>(sm + C_MISC);
     const uint32_t sbase = smem_u32(sm);
@@ -467,8 +578,10 @@ __device__ void chain_role(uint8_t *sm, const ClusterParams &p, int unit, int n,
     const int quad = warp & 3, half = warp >> 2, row = quad * 32 + lane;
     const uint32_t tmem = ms->tmem_base;
     const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
-    // producer-CTA "taken" barriers (rank 1 + k)
+    // cluster: producer-CTA "taken" barriers (rank 1 + k)
     const uint32_t prod_taken_local = sbase + P_MISC + (uint32_t)offsetof(ProdMisc, taken);
+    uint32_t *uflags = kPool ? unit_flags(p, unit) : nullptr;
+    (void)warp;
 
     // ---- initial state: fp32 -> TMEM accumulator, fp16 hi/lo -> TMEM A operands ----
     {
@@ -515,24 +628,36 @@ __device__ void chain_role(uint8_t *sm, const ClusterParams &p, int unit, int n,
         __syncthreads();
         tc_fence_after_sync();
     };
+    // has chunk cc reached the ring?  (thread 0)
+    auto ready_try = [&](int cc) -> bool {
+        if constexpr (kPool)
+            return ld_acquire_gpu(uflags + 1 + cc % kRingSlots) >= (uint32_t)(cc + 1);
+        else
+            return mbar_try_wait_cluster(&ms->ready[cc & 1], ((cc >> 1) & 1));
+    };
+    auto ready_wait = [&](int cc) -> bool {
+        if constexpr (kPool)
+            return wait_flag_geq(uflags + 1 + cc % kRingSlots, (uint32_t)(cc + 1), p.flags + 1,
+                                 kWaitLimit);
+        else
+            return mbar_wait_cluster_bounded(&ms->ready[cc & 1], (cc >> 1) & 1, kWaitLimit);
+    };
 
 #ifdef GDN_TC_PHASES
     long long phase_t_ = clock64();
+    const bool phase_on_ = blockIdx.x == 0;
 #endif
     // Thread 0 loads chunk c + 1 from the ring into shared slot (c + 1) & 1 as
-    // soon as its producer reports it ready, while chunk c is processed; the
+    // soon as it is reported ready, while chunk c is processed; the shared
     // slot held chunk c - 1, which is finished.
     int loaded = 0;  // chunks whose load has been issued
     auto issue_load = [&](int cc) {
-        const int kk = cc & 1, rs = (cc >> 1) & 1;
         fence_proxy_async_global();  // the producer's stores, acquired, precede our bulk load
         mbar_arrive_expect_tx(&ms->full[cc & 1], SLOT_BYTES);
-        bulk_load(sm + (cc & 1) * SLOT_BYTES, ring_slot(p, unit, kk, rs), SLOT_BYTES,
-                  &ms->full[cc & 1]);
+        bulk_load(sm + (cc & 1) * SLOT_BYTES, ring_slot(p, unit, cc), SLOT_BYTES, &ms->full[cc & 1]);
     };
     auto poll_next = [&](int cur) {
-        if (tid == 0 && loaded == cur + 1 && cur + 1 < nch &&
-            mbar_try_wait_cluster(&ms->ready[(cur + 1) & 1], ((cur + 1) >> 1) & 1)) {
+        if (tid == 0 && loaded == cur + 1 && cur + 1 < nch && ready_try(cur + 1)) {
             issue_load(cur + 1);
             loaded = cur + 2;
         }
@@ -546,15 +671,27 @@ __device__ void chain_role(uint8_t *sm, const ClusterParams &p, int unit, int n,
         const int64_t c0 = t_begin + (int64_t)kC * c;
         const int L = (int)((t_end - c0) < kC ? (t_end - c0) : kC);
 
+        bool have = true;
         if (tid == 0 && loaded == c) {  // not prefetched: wait for the producer, then load
-            if (!mbar_wait_cluster_bounded(&ms->ready[k], (c >> 1) & 1, kWaitLimit)) timed_out = true;
-            issue_load(c);
-            loaded = c + 1;
+            if (ready_wait(c)) {
+                issue_load(c);
+                loaded = c + 1;
+            } else {
+                // Nothing will land: complete the slot's phase by hand so that no
+                // thread waits for it; the vote at the end of the chunk aborts.
+                timed_out = true;
+                have = false;
+                mbar_arrive(&ms->full[k]);
+            }
         }
         if (!mbar_wait_bounded(&ms->full[k], (c >> 1) & 1, kWaitLimit)) timed_out = true;
         GDN_CL_PHASE(0, 0);  // wait: delivery
-        if (tid == 0)  // the chunk is out of the ring: its producer may deliver the next one
-            mbar_arrive_remote(mapa_shared(prod_taken_local, 1 + k));
+        if (tid == 0 && have) {  // the chunk is out of the ring: its slot may be refilled
+            if constexpr (kPool)
+                st_release_gpu(uflags, (uint32_t)(c + 1));
+            else
+                mbar_arrive_remote(mapa_shared(prod_taken_local, 1 + k));
+        }
         const GatesBlock *gb = reinterpret_cast<const GatesBlock *>(slot + SL_GATES);
         const bool hp = gb->hp != 0;
         const float gC = gb->Gam[kC - 1];
@@ -678,11 +815,14 @@ __device__ void chain_role(uint8_t *sm, const ClusterParams &p, int unit, int n,
         }
         poll_next(c);
         GDN_CL_PHASE(0, 5);  // o staging + stores, S copies
-        fence_proxy_async_smem();  // our writes to the slot precede the producer's next copies
+        fence_proxy_async_smem();  // our writes to the slot precede the next bulk load into it
         tmem_wait_st();
         tc_fence_before_sync();
         if (__syncthreads_or(timed_out ? 1 : 0)) {
-            if (tid == 0) raise_error(p.err, GDN_ERR_TIMEOUT);
+            if (tid == 0) {
+                raise_error(p.err, GDN_ERR_TIMEOUT);
+                if constexpr (kPool) pool_abort(p);
+            }
             aborted = true;
         }
         tc_fence_after_sync();
@@ -702,33 +842,21 @@ __device__ void chain_role(uint8_t *sm, const ClusterParams &p, int unit, int n,
         }
     }
     if (aborted) {
-        // a prefetched load may still be landing in shared memory: let it finish
-        if (loaded > c + 1) mbar_wait_bounded(&ms->full[(c + 1) & 1], ((c + 1) >> 1) & 1, kWaitLimit);
+        // A prefetch still landing in shared memory must finish (c is one past
+        // the chunk that voted; every earlier load has been waited for).
+        for (int cc = c; cc < loaded; ++cc)
+            mbar_wait_bounded(&ms->full[cc & 1], (cc >> 1) & 1, kWaitLimit);
         mbar_wait_bounded(&ms->mma_bar, mma_phase ^ 1, kWaitLimit);
     }
 }
 
-__global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
-    gdn_prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
-                               const __grid_constant__ CUtensorMap tm_k,
-                               const __grid_constant__ CUtensorMap tm_v, ClusterParams p) {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                              ~uintptr_t(1023));
-    const int rank = (int)cluster_ctarank();
-    const int unit = blockIdx.x / kCluster;  // n * Hv + h
-    const int h = unit % p.Hv;
-    const int n = unit / p.Hv;
-    const int j = h / (p.Hv / p.Hqk);
-    const int tid = threadIdx.x, warp = tid >> 5;
-
-    int64_t t_begin, t_end;
-    if (!seq_range(p.cu, n, p.N, p.T, p.err, t_begin, t_end)) return;  // uniform per cluster
-    const int nch = (int)((t_end - t_begin + kC - 1) / kC);
-
+// Barrier set-up and TMEM allocation of either role.
+__device__ __forceinline__ uint32_t *setup_role(uint8_t *sm, bool chain, uint32_t &ncols,
+                                                const CUtensorMap *tm_q, const CUtensorMap *tm_k,
+                                                const CUtensorMap *tm_v) {
+    const int tid = threadIdx.x;
     uint32_t *tmem_slot;
-    uint32_t ncols;
-    if (rank == 0) {
+    if (chain) {
         ChainMisc *ms = reinterpret_cast<ChainMisc *>(sm + C_MISC);
         tmem_slot = &ms->tmem_base;
         ncols = 512;
@@ -750,59 +878,181 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
             mbar_init(&ms->mma_bar, 1);
             mbar_init(&ms->taken, 1);
             fence_mbarrier_init();
-            tma_prefetch_desc(&tm_q);
-            tma_prefetch_desc(&tm_k);
-            tma_prefetch_desc(&tm_v);
+            tma_prefetch_desc(tm_q);
+            tma_prefetch_desc(tm_k);
+            tma_prefetch_desc(tm_v);
         }
     }
-    if (warp == 0) {
+    if ((tid >> 5) == 0) {
         tmem_alloc(tmem_slot, ncols);
         tmem_relinquish();
     }
+    return tmem_slot;
+}
+
+__device__ __forceinline__ uint8_t *aligned_smem(uint8_t *raw) {
+    return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
+}
+
+__global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
+    gdn_prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
+                               const __grid_constant__ CUtensorMap tm_k,
+                               const __grid_constant__ CUtensorMap tm_v, ChainParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = aligned_smem(smem_raw);
+    const int rank = (int)cluster_ctarank();
+    const int unit = blockIdx.x / kCluster;  // n * Hv + h
+    const int h = unit % p.Hv;
+    const int n = unit / p.Hv;
+    const int j = h / (p.Hv / p.Hqk);
+
+    int64_t t_begin, t_end;
+    if (!seq_range(p.cu, n, p.N, p.T, p.err, t_begin, t_end)) return;  // uniform per cluster
+    const int nch = (int)((t_end - t_begin + kC - 1) / kC);
+
+    uint32_t ncols;
+    uint32_t *tmem_slot = setup_role(sm, rank == 0, ncols, &tm_q, &tm_k, &tm_v);
     tc_fence_before_sync();
     __syncthreads();
     cluster_sync();  // every CTA's barriers exist before anyone signals them
     tc_fence_after_sync();
 
     if (rank == 0)
-        chain_role(sm, p, unit, n, h, t_begin, t_end, nch);
+        chain_role<false>(sm, p, unit, n, h, t_begin, t_end, nch);
     else
-        producer_role(sm, &tm_q, &tm_k, &tm_v, p, unit, rank - 1, h, j, t_begin, t_end, nch);
+        producer_role<false>(sm, &tm_q, &tm_k, &tm_v, p, unit, rank - 1, h, j, t_begin, t_end, nch);
 
     tc_fence_before_sync();
     __syncthreads();
     tc_fence_after_sync();
-    if (warp == 0) tmem_dealloc(*tmem_slot, ncols);
+    if ((threadIdx.x >> 5) == 0) tmem_dealloc(*tmem_slot, ncols);
     cluster_sync();  // nobody's shared memory goes away while another CTA may address it
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    gdn_prefill_pool_kernel(const __grid_constant__ CUtensorMap tm_q,
+                            const __grid_constant__ CUtensorMap tm_k,
+                            const __grid_constant__ CUtensorMap tm_v, ChainParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = aligned_smem(smem_raw);
+    const bool chain = (int)blockIdx.x < p.units;
+    int unit = 0, n = 0, h = 0, nch = 0;
+    int64_t t_begin = 0, t_end = 0;
+    if (chain) {
+        unit = blockIdx.x;
+        h = unit % p.Hv;
+        n = unit / p.Hv;
+        if (!seq_range(p.cu, n, p.N, p.T, p.err, t_begin, t_end)) return;  // producers skip it too
+        nch = (int)((t_end - t_begin + kC - 1) / kC);
+    }
+    uint32_t ncols;
+    uint32_t *tmem_slot = setup_role(sm, chain, ncols, &tm_q, &tm_k, &tm_v);
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+
+    if (chain)
+        chain_role<true>(sm, p, unit, n, h, t_begin, t_end, nch);
+    else
+        producer_role<true>(sm, &tm_q, &tm_k, &tm_v, p, 0, 0, 0, 0, 0, 0, 0);
+
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    if ((threadIdx.x >> 5) == 0) tmem_dealloc(*tmem_slot, ncols);
+}
+
+size_t pool_flag_bytes(int64_t units) {
+    const size_t b = (size_t)(kFlagHeader + kFlagsPerUnit * units) * sizeof(uint32_t);
+    return (b + 1023) & ~size_t(1023);
+}
+
+bool fill_params(const PrefillArgs &a, ChainParams &p, CUtensorMap &mq, CUtensorMap &mk,
+                 CUtensorMap &mv);
+
+int sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    return n;
 }
 
 }  // namespace
 
-static_assert(4 * SLOT_BYTES == kClusterWorkspaceBytesPerUnit, "ring size per unit");
+static_assert(kRingSlots * SLOT_BYTES == kClusterWorkspaceBytesPerUnit, "ring size per unit");
 
 size_t prefill_cluster_workspace_bytes(int64_t units) {
-    return (size_t)units * 4 * SLOT_BYTES;
+    return (size_t)units * kRingSlots * SLOT_BYTES;
+}
+
+size_t prefill_pool_workspace_bytes(int64_t units) {
+    return pool_flag_bytes(units) + (size_t)units * kRingSlots * SLOT_BYTES;
+}
+
+bool prefill_pool_fits(int64_t units) {
+    const int sms = sm_count();
+    return units >= 1 && units <= kPoolMaxUnits && units + 16 <= sms;
 }
 
 bool make_tile_map_bf16_128(CUtensorMap *m, const void *base, int64_t T, int32_t H);
 
-cudaError_t launch_prefill_cluster(const PrefillArgs &a, cudaStream_t s) {
-    if (a.T > 0x7fffffffLL) return cudaErrorInvalidValue;
-    CUtensorMap mq, mk, mv;
+namespace {
+bool fill_params(const PrefillArgs &a, ChainParams &p, CUtensorMap &mq, CUtensorMap &mk,
+                 CUtensorMap &mv) {
+    if (a.T > 0x7fffffffLL || a.ws == nullptr) return false;
     const int64_t Tm = a.T > 0 ? a.T : 1;
     if (!make_tile_map_bf16_128(&mq, a.q, Tm, a.Hqk) || !make_tile_map_bf16_128(&mk, a.k, Tm, a.Hqk) ||
         !make_tile_map_bf16_128(&mv, a.v, Tm, a.Hv))
-        return cudaErrorInvalidValue;
-    if (a.ws == nullptr) return cudaErrorInvalidValue;
-    ClusterParams p;
-    p.ws = static_cast<uint8_t *>(a.ws);
+        return false;
+    p.ring = static_cast<uint8_t *>(a.ws);
+    p.flags = nullptr;
     p.g = a.g; p.beta = a.beta; p.s0 = a.s0; p.cu = a.cu; p.o = a.o; p.sT = a.sT; p.err = a.err;
     p.T = a.T; p.N = a.N; p.Hqk = a.Hqk; p.Hv = a.Hv;
+    p.units = a.N * a.Hv;
+    p.max_chunks = (int)((a.T + kC - 1) / kC);
+    return true;
+}
+}  // namespace
+
+cudaError_t launch_prefill_cluster(const PrefillArgs &a, cudaStream_t s) {
+    ChainParams p;
+    CUtensorMap mq, mk, mv;
+    if (!fill_params(a, p, mq, mk, mv)) return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(gdn_prefill_cluster_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
     const dim3 grid((unsigned)((int64_t)a.N * a.Hv * kCluster));
     gdn_prefill_cluster_kernel<<<grid, kThreads, kSmemBytes, s>>>(mq, mk, mv, p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_prefill_pool(const PrefillArgs &a, cudaStream_t s) {
+    ChainParams p;
+    CUtensorMap mq, mk, mv;
+    if (!fill_params(a, p, mq, mk, mv)) return cudaErrorInvalidValue;
+    const int sms = sm_count();
+    if (!prefill_pool_fits(p.units) || sms <= 0) return launch_prefill_tc(a, s);
+    const size_t fb = pool_flag_bytes(p.units);
+    p.flags = static_cast<uint32_t *>(a.ws);
+    p.ring = static_cast<uint8_t *>(a.ws) + fb;
+    // the chunk counter, abort flag and hand-off flags start at zero
+    cudaError_t e = cudaMemsetAsync(a.ws, 0, fb, s);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(gdn_prefill_pool_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kSmemBytes);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)sms);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;  // every CTA resident at once, or no launch
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, gdn_prefill_pool_kernel, mq, mk, mv, p);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

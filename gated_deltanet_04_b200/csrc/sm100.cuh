@@ -215,6 +215,38 @@ __device__ __forceinline__ void bulk_copy_to_cluster(uint32_t dst_cluster, const
         : "memory");
 }
 
+// ------------------------------------------------- global-memory flags --
+// Device-wide (gpu scope) acquire / release accesses of 32-bit flag words
+// that CTAs outside one cluster use to hand work to one another.
+
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t *p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ uint32_t ld_relaxed_gpu(const uint32_t *p) {
+    uint32_t v;
+    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void st_release_gpu(uint32_t *p, uint32_t v) {
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Spins until *flag >= want (acquire).  Returns false, without waiting
+// further, once *abort is non-zero or after `limit` SM clocks.
+__device__ __forceinline__ bool wait_flag_geq(const uint32_t *flag, uint32_t want,
+                                              const uint32_t *abort, long long limit) {
+    const long long t0 = clock64();
+    for (;;) {
+        if (ld_acquire_gpu(flag) >= want) return true;
+        if (ld_relaxed_gpu(abort) != 0u || clock64() - t0 > limit) return false;
+        __nanosleep(32);
+    }
+}
+
 // --------------------------------------------------------- tensor memory --
 
 // Allocates `ncols` TMEM columns (power of two >= 32); the whole warp calls.

@@ -115,11 +115,12 @@ GDN_API gdn_status gdn_prefill(const void *q, const void *k, const void *v, gdn_
 
 /*
  * Which prefill kernel runs.  For Dk = Dv = 128, bf16 and chunk 0 or 64, AUTO
- * picks the cluster kernel when there are at most 64 (sequence, v-head) units
- * (few, long sequences: it puts three SMs on every unit) and the single-CTA
+ * picks the pool kernel when there are at most 64 (sequence, v-head) units
+ * (few, long sequences: every SM of the GPU works on them) and the single-CTA
  * kernel otherwise; every other shape runs the exact recurrent kernel.
  * Naming a tensor-core kernel for a shape it does not support returns
- * GDN_ERR_UNSUPPORTED.  The cluster kernel needs a workspace (see below).
+ * GDN_ERR_UNSUPPORTED, and so does the pool kernel for more than 64 units.
+ * The cluster and pool kernels need a workspace (see below).
  */
 typedef enum gdn_prefill_kernel {
     GDN_PREFILL_AUTO = 0,
@@ -127,7 +128,12 @@ typedef enum gdn_prefill_kernel {
                                     holds the state, two prepare alternate chunks and
                                     hand them over through an L2-resident workspace ring */
     GDN_PREFILL_SINGLE_CTA = 2,  /* tcgen05, one CTA per (sequence, head) */
-    GDN_PREFILL_RECURRENT = 3    /* exact fp32 token recurrence on CUDA cores, any shape */
+    GDN_PREFILL_RECURRENT = 3,   /* exact fp32 token recurrence on CUDA cores, any shape */
+    GDN_PREFILL_POOL = 4         /* tcgen05, one cooperative launch over every SM: a CTA per
+                                    (sequence, head) holds the state, the other CTAs
+                                    prepare chunks in chunk-major order and hand them
+                                    over through the workspace ring (at most 64 units;
+                                    on a GPU with too few SMs it runs as SINGLE_CTA) */
 } gdn_prefill_kernel;
 
 /*
@@ -144,11 +150,14 @@ GDN_API gdn_status gdn_prefill_ex(const void *q, const void *k, const void *v, g
 
 /*
  * gdn_prefill_workspace_bytes -- scratch bytes gdn_prefill needs for these
- * sizes (0 when none): 430,080 bytes per (sequence, v-head) unit when AUTO
- * would run the cluster kernel.  Pure function of its arguments (it cannot see
- * the dtype, so it may ask for a workspace an fp32 call does not use); no
- * device access.  The workspace is device memory, 256-byte aligned, owned by
- * the caller; its contents need no initialisation and are garbage afterwards.
+ * sizes (0 when none): 430,080 bytes per (sequence, v-head) unit, plus a
+ * flag block of 1 KB or more for the pool kernel, when AUTO would run the
+ * pool kernel.  Pure function of its arguments (it cannot see the dtype, so
+ * it may ask for a workspace an fp32 call does not use); no device access.
+ * The workspace is device memory, 256-byte aligned, owned by the caller; its
+ * contents need no initialisation (the pool kernel clears its flag block on
+ * the stream before it starts) and are garbage afterwards.  One workspace
+ * must not serve two calls that may run at the same time.
  */
 GDN_API size_t gdn_prefill_workspace_bytes(int32_t N, int64_t T, int32_t Hqk, int32_t Hv, int32_t Dk,
                                    int32_t Dv, int32_t chunk);

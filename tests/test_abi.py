@@ -105,6 +105,8 @@ def prefill_ex(lib, kernel, **kw):
 
 @pytest.mark.parametrize("kernel,kw,code", [
     (7, {}, INVALID),                              # no such kernel
+    (4, dict(N=2, cu=P + 0x6000), UNSUPPORTED),    # the pool kernel takes at most 64 units
+    (4, dict(dt=1), UNSUPPORTED),
     (1, dict(Dk=64, Dv=64), UNSUPPORTED),          # tensor-core kernels need D = 128
     (2, dict(dt=1), UNSUPPORTED),                  # ... and bf16
     (1, dict(chunk=32), UNSUPPORTED),              # ... and chunk 64

@@ -26,7 +26,7 @@ def _gpu():
     build.build()
 
 
-TC_KERNELS = ["cluster", "single_cta"]
+TC_KERNELS = ["pool", "cluster", "single_cta"]
 
 
 def run_gpu(inp, s0=None, cu=None, chunk=0, dev=DEV, kernel="auto"):
@@ -163,13 +163,14 @@ def test_kernels_agree_with_each_other():
     the chunk length and the kernel change rounding only."""
     inp, s0 = synth(300, 2, 6, 128, torch.bfloat16, seed=600, s0_std=0.05)
     o64, s64 = run_gpu(inp, s0, chunk=64, kernel="cluster")
-    for kw in (dict(chunk=64, kernel="single_cta"), dict(chunk=16), dict(kernel="recurrent")):
+    for kw in (dict(chunk=64, kernel="single_cta"), dict(chunk=64, kernel="pool"), dict(chunk=16),
+               dict(kernel="recurrent")):
         o2, s2 = run_gpu(inp, s0, **kw)
         check_o(o2, o64.double())
         check_state(s2, s64.double())
 
 
-@pytest.mark.parametrize("kernel", TC_KERNELS)
+@pytest.mark.parametrize("kernel", ["cluster", "single_cta"])  # 1536 units: over the pool's 64
 def test_varlen32_split_and_carry(kernel):
     """32 packed sequences, lengths U[512,16384], nonzero initial states; every
     sequence split at a random point and run as two calls carrying the state
@@ -197,6 +198,44 @@ def test_varlen32_split_and_carry(kernel):
     check_state(s1[:, heads], s_ref, "one-shot state, sampled heads")
     check_o(o2[:, heads], o_ref, "segmented o, sampled heads")
     check_state(sb[:, heads], s_ref, "segmented state, sampled heads")
+
+
+def test_pool_kernel_rejects_more_than_64_units():
+    inp = inputs.make_prefill("varlen32")
+    with pytest.raises(gdn.GdnError, match="UNSUPPORTED"):
+        run_gpu(inp, inp["s0"], inputs.cu_from_lengths(inp["lengths"]), kernel="pool")
+
+
+@pytest.mark.parametrize("kernel", ["pool", "cluster"])
+def test_few_units_varlen_split_and_carry(kernel):
+    """Six packed sequences (one empty, one a single chunk, ragged tails) x 8
+    v-heads = 48 units, the size the multi-CTA kernels are for; nonzero
+    initial states; each sequence split and carried must match the one-shot
+    run, and both must match the oracle on every head."""
+    lengths = [5000, 700, 12000, 64, 0, 3001]
+    T = sum(lengths)
+    gen = torch.Generator().manual_seed(2201)
+    q, k, v, g, beta = inputs.make_tokens(T, 2, 8, 128, 128, torch.bfloat16, inputs.G_SCALE_097, gen)
+    s0 = inputs.make_state(len(lengths), 8, 128, 128, 0.05, gen)
+    inp = {"q": q, "k": k, "v": v, "g": g, "beta": beta, "lengths": torch.tensor(lengths),
+           "split": torch.tensor([2500, 333, 64, 1, 0, 1500])}
+    cu = inputs.cu_from_lengths(lengths)
+    o1, s1 = run_gpu(inp, s0, cu, kernel=kernel)
+    o_ref, s_ref = run_oracle(inp, s0, cu)
+    check_o(o1, o_ref, "one-shot o")
+    check_state(s1, s_ref, "one-shot state")
+    inp["cu_seqlens"] = cu
+    first, second = inputs.split_packed(inp)
+    oa, sa = run_gpu(first, s0, first["cu_seqlens"], kernel=kernel)
+    ob, sb = run_gpu(second, sa, second["cu_seqlens"], kernel=kernel)
+    cua, cub = first["cu_seqlens"].tolist(), second["cu_seqlens"].tolist()
+    o2 = torch.empty_like(o1)
+    for n in range(len(lengths)):
+        base, sp = int(cu[n]), int(inp["split"][n])
+        o2[base:base + sp] = oa[cua[n]:cua[n + 1]]
+        o2[base + sp:int(cu[n + 1])] = ob[cub[n]:cub[n + 1]]
+    check_o(o2, o_ref, "segmented o")
+    check_state(sb, s_ref, "segmented state")
 
 
 def head_subset(inp, heads):
