@@ -112,23 +112,52 @@ def weak_scaling_value(units_per_rank: float, seconds_max: float, world: int) ->
 # ------------------------------------------------------------------ clocks --
 
 class ClockSampler:
-    """Samples nvidia-smi clocks and throttle reasons while the timed region runs."""
+    """Samples SM clocks and throttle reasons every 20 ms while the timed
+    region runs (NVML reads only; nvidia-smi at 200 ms when NVML is missing)."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clock-event reason bits
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "sw_power_cap": 0x4}
 
     def __init__(self, gpu_index):
         self.gpu_index = gpu_index
         self.proc = None
+        self.nvml = None
         self.lines = []
+        self.samples = []  # (sm_mhz, max_mhz, reason bits)
         self.active = False
+        self.stopping = False
 
     def _reader(self):
         for line in self.proc.stdout:
             if self.active:
                 self.lines.append(line.strip())
 
+    def _poll(self):
+        nv, h = self.nvml
+        while not self.stopping:
+            if self.active:
+                try:
+                    sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                    mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+                    rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                    self.samples.append((float(sm), float(mx), int(rs)))
+                except Exception:
+                    pass
+            time.sleep(0.02)
+
     def start(self):
+        try:
+            import pynvml as nv
+            nv.nvmlInit()
+            self.nvml = (nv, nv.nvmlDeviceGetHandleByIndex(self._physical_index()))
+            self.thread = threading.Thread(target=self._poll, daemon=True)
+            self.thread.start()
+            return
+        except Exception:
+            self.nvml = None
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
@@ -138,35 +167,54 @@ class ClockSampler:
         except OSError:
             self.proc = None
 
+    def _physical_index(self):
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+        ids = [x for x in vis.split(",") if x.strip()]
+        if ids and ids[0].strip().isdigit() and self.gpu_index < len(ids):
+            return int(ids[self.gpu_index])
+        return self.gpu_index
+
     def mark(self, on: bool):
         self.active = on
 
     def stop(self):
-        if self.proc is None:
-            return None
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
         sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in self.lines:
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 9:
-                continue
+        if self.nvml is not None:
+            self.stopping = True
+            self.thread.join(timeout=2)
+            for s_mhz, m_mhz, bits in self.samples:
+                sm.append(s_mhz)
+                mx = m_mhz
+                for name, bit in self.REASONS.items():
+                    if bits & bit:
+                        reasons.add(name)
+            src = "nvml 20 ms"
+        elif self.proc is not None:
+            self.proc.terminate()
             try:
-                sm.append(float(parts[1]))
-                mx = float(parts[2])
-            except ValueError:
-                continue
-            for name, val in zip(names, parts[5:9]):
-                if val.lower() == "active":
-                    reasons.add(name)
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+            for line in self.lines:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx = float(parts[2])
+                except ValueError:
+                    continue
+                for name, val in zip(names, parts[5:9]):
+                    if val.lower() == "active":
+                        reasons.add(name)
+            src = "nvidia-smi 200 ms"
+        else:
+            return None
         if not sm:
             return None
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "sampler": src}
 
 
 # -------------------------------------------------------------- roofline ---
