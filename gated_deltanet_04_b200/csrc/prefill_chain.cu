@@ -19,10 +19,10 @@
 //     matrices, decay factors, the triangular solve, U~ and W on tensor cores.
 // A finished chunk (K, Q, W^T hi/lo, U~, P, gates: one 105 KB block laid out
 // exactly like a chain slot) goes through L2: the producer bulk-stores it
-// into a ring of kRingSlots slots per (sequence, head) in the caller's
-// workspace, and the chain bulk-loads it into one of its two shared-memory
-// slots while it computes the previous chunk.  Chunk c of a unit always uses
-// ring slot c % kRingSlots.
+// into a ring of R slots per (sequence, head) in the caller's workspace (R = 4
+// for the cluster kernel, 8 for the pool kernel), and the chain bulk-loads
+// it into one of its two shared-memory slots while it computes the previous
+// chunk.  Chunk c of a unit always uses ring slot c % R.
 //
 // Two ways to schedule the producers:
 //   * cluster kernel: a 3-CTA cluster per unit, rank 0 the chain, ranks 1 and
@@ -42,7 +42,7 @@
 //     release / acquire:
 //         ready[u][s]  = c + 1   chunk c of unit u is in ring slot s
 //         taken[u]     = c + 1   the chain of unit u has loaded chunks 0..c
-//     A producer writes chunk c only after taken[u] >= c - kRingSlots + 1.
+//     A producer writes chunk c only after taken[u] >= c - R + 1.
 //     Every wait is on a chunk of lower counter index, and a producer works
 //     through its chunks in counter order, so the lowest unfinished chunk can
 //     always proceed: no deadlock while every CTA is resident, which the
@@ -57,18 +57,35 @@
 #include "tc_common.cuh"
 
 #ifdef GDN_TC_PHASES
-// per-phase SM clocks: [0] the first chain CTA, [1] the first producer CTA
-__device__ long long gdn_cl_phase_clk[2][16];
+// Per-phase SM clocks of thread 0: [0] the first chain CTA, [1] the first
+// producer CTA.  Accumulated in shared memory (a global read-modify-write per
+// marker would stall thread 0 and distort the phases) and added to the
+// global totals once, at the end of the role.
+__device__ unsigned long long gdn_cl_phase_clk[2][16];
+static __shared__ unsigned int gdn_phase_acc_[16];
 #define GDN_CL_PHASE(role, k)                                          \
     do {                                                               \
         if (threadIdx.x == 0 && phase_on_) {                           \
             const long long now_ = clock64();                          \
-            gdn_cl_phase_clk[(role)][(k)] += now_ - phase_t_;          \
+            gdn_phase_acc_[(k)] += (unsigned int)(now_ - phase_t_);    \
             phase_t_ = now_;                                           \
         }                                                              \
     } while (0)
+#define GDN_CL_PHASE_BEGIN()                                           \
+    long long phase_t_ = clock64();                                    \
+    if (threadIdx.x == 0)                                              \
+        for (int i_ = 0; i_ < 16; ++i_) gdn_phase_acc_[i_] = 0u
+#define GDN_CL_PHASE_END(role)                                         \
+    do {                                                               \
+        if (threadIdx.x == 0 && phase_on_)                             \
+            for (int i_ = 0; i_ < 16; ++i_)                            \
+                atomicAdd(&gdn_cl_phase_clk[(role)][i_],               \
+                          (unsigned long long)gdn_phase_acc_[i_]);     \
+    } while (0)
 #else
 #define GDN_CL_PHASE(role, k) ((void)0)
+#define GDN_CL_PHASE_BEGIN() ((void)0)
+#define GDN_CL_PHASE_END(role) ((void)0)
 #endif
 
 namespace gdn {
@@ -79,21 +96,23 @@ using namespace tc;
 
 constexpr int kThreads = 256;
 constexpr int kCluster = 3;
-constexpr int kRingSlots = 4;
+constexpr int kClusterRingSlots = 4;
+constexpr int kPoolRingSlots = 8;
 
 // ---- chain CTA: two hand-off slots (offsets inside a slot) ----
 constexpr uint32_t SL_K16 = 0;         // K fp16: d-halves at +0 / +8192 ([64 rows][128 B], SW128)
-constexpr uint32_t SL_Q16 = 16384;     // Q fp16, same layout
-constexpr uint32_t SL_WH = 32768;      // W^T hi, MN-major [128 d][128 B]
-constexpr uint32_t SL_WL = 49152;      // W^T lo
+constexpr uint32_t SL_QT = 16384;      // Q^T fp16, MN-major [128 d][128 B] (SW128)
+constexpr uint32_t SL_WH = 32768;      // W^T hi, same layout
+constexpr uint32_t SL_WL = 49152;      // W^T lo, same layout
+// Q^T, W^T hi and W^T lo are 16 KB apart: one MN-major B operand of N = 128
+// ([Q | W hi]) or N = 192 ([Q | W hi | W lo]) tokens with that atom stride.
+static_assert(SL_WH - SL_QT == 16384 && SL_WL - SL_WH == 16384, "stacked B operand");
 constexpr uint32_t SL_UT = 65536;      // U~^T fp32 [128 rows][64], 16-byte chunks XOR-swizzled by row
 constexpr uint32_t SL_P16 = 98304;     // P fp16 [64 rows][128 B], SW128
 constexpr uint32_t SL_GATES = 106496;  // GatesBlock
 constexpr uint32_t SLOT_BYTES = 107520;
-// reuse of a slot's regions once the chain has consumed them
-constexpr uint32_t SL_UP = SL_UT;      // U' hi then lo (K-major A operand), after U~ is read
-constexpr uint32_t SL_U16 = SL_WH;     // U^T fp16 (K-major A operand), after R
-constexpr uint32_t SL_OST = SL_Q16;    // o staging [64 tokens][128] bf16, after S Q^T
+// reuse of a slot's region once the chain has consumed it
+constexpr uint32_t SL_OST = SL_QT;     // o staging [64 tokens][128] bf16, after S Q^T
 constexpr uint32_t C_MISC = 2 * SLOT_BYTES;
 
 struct GatesBlock {
@@ -111,26 +130,33 @@ struct ChainMisc {
     uint32_t tmem_base;
 };
 
-// chain TMEM columns (512 allocated): state, this chunk's state increment,
-// fp16 hi/lo copies of the state (A operands), R = S W^T, output
-constexpr uint32_t CT_S = 0, CT_D = 128, CT_SH = 256, CT_SL = 320, CT_R = 384, CT_O = 448;
+// chain TMEM columns (512 allocated):
+//   S    0..127   fp32 state (accumulator of nothing: read, scaled, rewritten)
+//   SH 128..191   fp16 hi copy of S (A operand); SL 192..255 its lo part,
+//                 whose columns 192..223 then hold U^T fp16 (A operand)
+//   O  256..319   S Q^T, then the whole transposed chunk output
+//   R  320..383   S W^T (S_hi W_hi [+ S_lo W_hi]); R2 384..447 S_hi W_lo;
+//                 once both are read, D 320..447 takes the state increment
+//   UP 448..511   U' = U diag(Gamma_C / Gamma) as fp16 hi | lo (A operand, K = 128)
+constexpr uint32_t CT_S = 0, CT_SH = 128, CT_SL = 192, CT_U16 = 192, CT_O = 256, CT_R = 320,
+                   CT_R2 = 384, CT_D = 320, CT_UP = 448;
 
 // ---- producer CTA ----
 constexpr uint32_t P_KQV = 0;           // 2 buffers: [K|Q] d-half 0, [K|Q] d-half 1, V halves
 constexpr uint32_t P_KQV_BYTES = 49152;
-constexpr uint32_t P_X = 98304;         // 48 KB: solve scratch, then W^T hi/lo + gates staging
+constexpr uint32_t P_X = 98304;         // solve scratch: A, T, X (fp32); then W^T hi/lo staging
 constexpr uint32_t P_WST = P_X;
-constexpr uint32_t P_GST = P_X + 32768;
 constexpr uint32_t P_AS = P_X;
 constexpr uint32_t P_TS = P_X + 64 * kAS * 4;
 constexpr uint32_t P_XS = P_TS + 64 * kTS * 4;
-constexpr uint32_t P_UTS = 147456;      // U~^T staging (same layout as SL_UT)
-constexpr uint32_t P_P16 = 180224;
-constexpr uint32_t P_TBH = 188416, P_TBL = 196608, P_TGH = 204800, P_TGL = 212992;
-constexpr uint32_t P_MISC = 221184;
-static_assert(P_XS + 1024 * 4 <= P_UTS, "solve scratch overflows");
-static_assert(P_GST + sizeof(GatesBlock) <= P_X + 49152, "gates staging stays inside the region");
+constexpr uint32_t P_P16 = 137216;      // P fp16 [64 rows][128 B], SW128
+constexpr uint32_t P_TBH = 145408, P_TBL = 153600, P_TGH = 161792, P_TGL = 169984;  // T tiles
+constexpr uint32_t P_UTS = P_TBH;       // then U~^T staging (same layout as SL_UT)
+constexpr uint32_t P_MISC = 178176;
+static_assert(P_WST + 32768 <= P_P16 && P_UTS + 32768 <= P_MISC, "staging fits its region");
+static_assert(P_XS + 1024 * 4 <= P_P16, "solve scratch overflows");
 static_assert(P_TS % 16 == 0 && P_XS % 16 == 0, "float4 scratch must be aligned");
+static_assert(P_P16 % 1024 == 0 && P_TBH % 1024 == 0, "swizzled tiles start on 1 KB");
 
 // One chunk of one unit, as a producer sees it.
 struct Item {
@@ -140,18 +166,25 @@ struct Item {
     int32_t valid;
 };
 
-struct ProdMisc {
+// Decay and gate factors of one chunk (double-buffered by chunk parity: the
+// next chunk's are computed while this chunk's U~ / W products run).
+struct ProdGates {
     float gam[kC], Gam[kC], iGam[kC], eC[kC], bb[kC], bG[kC];
+    int32_t safe, hp, pad[2];
+};
+
+struct ProdMisc {
+    GatesBlock gst;   // gates staging of the chunk being delivered
+    ProdGates gt[2];
     Item items[4];    // this CTA's chunks l .. l + 2, by l % 4
     uint64_t tma_bar[2];
     uint64_t mma_bar;
     uint64_t taken;
     uint32_t tmem_base;
-    int32_t safe, hp;
-    float gsum;
 };
-constexpr uint32_t kSmemBytes = P_MISC + sizeof(ProdMisc) + 1024;
-static_assert(C_MISC + sizeof(ChainMisc) <= P_MISC + sizeof(ProdMisc), "chain misc fits");
+constexpr uint32_t kProdBytes = P_MISC + sizeof(ProdMisc);
+constexpr uint32_t kChainBytes = C_MISC + sizeof(ChainMisc);
+constexpr uint32_t kSmemBytes = (kProdBytes > kChainBytes ? kProdBytes : kChainBytes) + 1024;
 static_assert(kSmemBytes <= 232448, "fits the 227 KB opt-in shared memory of a CTA");
 
 // producer TMEM columns (128 allocated)
@@ -160,11 +193,11 @@ constexpr uint32_t PT_G = 0, PT_U = 64;
 // pool flags: a header of kFlagHeader words ([0] the chunk counter, [1] the
 // abort flag), then 8 words per unit ([0] taken, [1 + s] ready of slot s)
 constexpr int kFlagHeader = 64;
-constexpr int kFlagsPerUnit = 8;
-static_assert(1 + kRingSlots <= kFlagsPerUnit, "flag words per unit");
+constexpr int kFlagsPerUnit = 16;
+static_assert(1 + kPoolRingSlots <= kFlagsPerUnit, "flag words per unit");
 
 struct ChainParams {
-    uint8_t *ring;    // [unit][kRingSlots][SLOT_BYTES]
+    uint8_t *ring;    // [unit][ring_slots][SLOT_BYTES]
     uint32_t *flags;  // pool kernel only
     const float *g, *beta, *s0;
     const int32_t *cu;
@@ -173,10 +206,11 @@ struct ChainParams {
     int32_t *err;
     int64_t T;
     int32_t N, Hqk, Hv, units, max_chunks;
+    int32_t ring_slots;  // a power of two
 };
 
 __device__ __forceinline__ uint8_t *ring_slot(const ChainParams &p, int unit, int c) {
-    return p.ring + ((size_t)unit * kRingSlots + (c % kRingSlots)) * SLOT_BYTES;
+    return p.ring + ((size_t)unit * p.ring_slots + (c & (p.ring_slots - 1))) * SLOT_BYTES;
 }
 
 __device__ __forceinline__ uint32_t *unit_flags(const ChainParams &p, int unit) {
@@ -256,7 +290,7 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
 
     uint32_t mma_phase = 0;
     bool timed_out = false;
-    float gpre0 = 0.f, gpre1 = 0.f, bpre0 = 0.f, bpre1 = 0.f;
+    float gpre0 = 0.f, gpre1 = 0.f, bpre0 = 0.f, bpre1 = 0.f;  // warp 0: the next chunk's g, beta
     auto load_gates = [&](const Item &it) {
         gpre0 = gpre1 = bpre0 = bpre1 = 0.f;
         const int64_t t0_ = it.c0 + 2 * lane, t1_ = t0_ + 1, te = it.c0 + it.L;
@@ -288,10 +322,63 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
         tc_fence_after_sync();
     };
 
-    // Chunks l and l + 1 are known (and their tile loads issued) when chunk l
-    // starts; the delivery thread fetches chunk l + 2 before the vote of chunk
-    // l and issues its tile loads into chunk l's buffer once that buffer's
-    // stores have drained.
+    // The delivery thread's last chunk whose ring stores are in flight and not
+    // yet reported ready (valid == 0: none).
+    Item pending;
+    pending.valid = 0;
+    auto flush_delivery = [&]() {  // delivery thread only
+        if (!pending.valid) return;
+        bulk_wait_all();              // written to global memory
+        fence_proxy_async_global();   // ... ordered before the signal below
+        if constexpr (kPool)
+            st_release_gpu(unit_flags(p, pending.unit) + 1 + (pending.c & (p.ring_slots - 1)),
+                           (uint32_t)(pending.c + 1));
+        else
+            mbar_arrive_remote(c_ready);
+        pending.valid = 0;
+    };
+
+    // Gates of a chunk from the g, beta values in gpre / bpre (warp 0, two
+    // tokens per lane): cumulative log-decay gamma, Gamma = exp(gamma), the
+    // factors of A, P, W and U', and the precision choice.
+    auto compute_gates = [&](ProdGates &gt) {
+        float x1 = gpre0 + gpre1;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const float y = __shfl_up_sync(0xffffffffu, x1, off);
+            if (lane >= off) x1 += y;
+        }
+        const float x0 = x1 - gpre1;
+        const float gC = __shfl_sync(0xffffffffu, x1, 31);
+        float m = fmaxf(fabsf(x0), fabsf(x1));
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+        const bool safe_ = m <= 60.f;  // every exp(+-gamma) a normal float
+        const float G0 = expf(x0), G1 = expf(x1);
+        const float GC = __shfl_sync(0xffffffffu, G1, 31);
+        const int r0 = 2 * lane;
+        gt.gam[r0] = x0;                gt.gam[r0 + 1] = x1;
+        gt.Gam[r0] = G0;                gt.Gam[r0 + 1] = G1;
+        if (safe_) {  // 1 / Gamma and Gamma_C / Gamma from the exponentials above
+            const float i0 = 1.f / G0, i1 = 1.f / G1;
+            gt.iGam[r0] = i0;           gt.iGam[r0 + 1] = i1;
+            gt.eC[r0] = GC * i0;        gt.eC[r0 + 1] = GC * i1;
+        } else {
+            gt.iGam[r0] = 0.f;          gt.iGam[r0 + 1] = 0.f;
+            gt.eC[r0] = expf(gC - x0);  gt.eC[r0 + 1] = expf(gC - x1);
+        }
+        gt.bb[r0] = bpre0;              gt.bb[r0 + 1] = bpre1;
+        gt.bG[r0] = bpre0 * G0;         gt.bG[r0 + 1] = bpre1 * G1;
+        if (lane == 0) {
+            gt.safe = safe_;
+            gt.hp = GC >= kHighPrecisionDecay;
+        }
+    };
+
+    // Chunks l and l + 1 are known when chunk l starts (tile loads of chunks
+    // 0 and 1 are issued here, those of chunk l + 1 > 1 during chunk l, once
+    // the stores of chunk l - 1 have read its buffer); the delivery thread
+    // fetches chunk l + 2 before the vote of chunk l.
     if (tid == 32) {
         for (int l = 0; l < 2; ++l) {
             const Item it = fetch(l);
@@ -300,11 +387,15 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
         }
     }
     __syncthreads();
-    if (warp == 0 && ms->items[0].valid) load_gates(ms->items[0]);
+    if (warp == 0 && ms->items[0].valid) {
+        load_gates(ms->items[0]);
+        compute_gates(ms->gt[0]);
+    }
+    __syncthreads();
 #ifdef GDN_TC_PHASES
-    long long phase_t_ = clock64();
     const bool phase_on_ = blockIdx.x == (kPool ? (unsigned)p.units : 1u);
 #endif
+    GDN_CL_PHASE_BEGIN();
     int l = 0;
     bool broke = false;
 #pragma unroll 1
@@ -313,51 +404,36 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
         if (!it.valid) break;
         const int L = it.L;
         const int buf = l & 1;
+        const ProdGates &gt = ms->gt[l & 1];
 
-        // ---- gates (warp 0, two tokens per lane) ----
+        // the next chunk's g, beta: in flight until its gates are computed
         if (warp == 0) {
-            float x1 = gpre0 + gpre1;
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const float y = __shfl_up_sync(0xffffffffu, x1, off);
-                if (lane >= off) x1 += y;
-            }
-            const float x0 = x1 - gpre1;
-            const float gC = __shfl_sync(0xffffffffu, x1, 31);
-            float m = fmaxf(fabsf(x0), fabsf(x1));
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-            const bool safe_ = m <= 60.f;
-            const float G0 = expf(x0), G1 = expf(x1);
-            const int r0 = 2 * lane;
-            ms->gam[r0] = x0;                ms->gam[r0 + 1] = x1;
-            ms->Gam[r0] = G0;                ms->Gam[r0 + 1] = G1;
-            ms->iGam[r0] = safe_ ? expf(-x0) : 0.f;
-            ms->iGam[r0 + 1] = safe_ ? expf(-x1) : 0.f;
-            ms->eC[r0] = expf(gC - x0);      ms->eC[r0 + 1] = expf(gC - x1);
-            ms->bb[r0] = bpre0;              ms->bb[r0 + 1] = bpre1;
-            ms->bG[r0] = bpre0 * G0;         ms->bG[r0 + 1] = bpre1 * G1;
-            if (lane == 0) {
-                ms->safe = safe_;
-                ms->hp = expf(gC) >= kHighPrecisionDecay;
-            }
             const Item nx = ms->items[(l + 1) & 3];
             if (nx.valid) load_gates(nx);
         }
-
         GDN_CL_PHASE(1, 0);  // gates
         GDN_CL_PHASE(1, 1);  // (no wait)
         if (!mbar_wait_bounded(&ms->tma_bar[buf], (l >> 1) & 1, kWaitLimit)) timed_out = true;
         GDN_CL_PHASE(1, 2);  // wait: tiles
 
-        // ---- bf16 -> fp16 in place, zero padding rows ----
+        // ---- Gram [K;Q] K^T straight from the bf16 tiles (exact products either way) ----
         uint8_t *kqv = sm + P_KQV + buf * P_KQV_BYTES;
         const uint32_t skqv = sbase + P_KQV + buf * P_KQV_BYTES;
+        if (tid == 0) {
 #pragma unroll
-        for (int q = 0; q < 3072 / kThreads; ++q) {
-            const int x = tid + q * kThreads;
-            uint4 *ptr = reinterpret_cast<uint4 *>(kqv) + x;
-            const int r = (x >> 3) & 63;
+            for (int ks = 0; ks < 8; ++ks) {
+                const uint32_t a = skqv + (ks >> 2) * 16384 + (ks & 3) * 32;
+                mma_f16_ss(tmem + PT_G, make_sdesc(a, 16, 1024), make_sdesc(a, 16, 1024),
+                           IDESC_KK_N64_BF16, ks > 0);
+            }
+            mma_commit(&ms->mma_bar);
+        }
+        // bf16 -> fp16 in place with padding rows zeroed: V (A operand of U~)
+        // while the Gram products run, then K once they have read it.  Q goes
+        // to fp16 in the Q^T transpose.
+        auto convert16 = [&](uint8_t *base, int x) {  // 16-byte chunk x of a [64][128 B] tile
+            uint4 *ptr = reinterpret_cast<uint4 *>(base) + x;
+            const int r = x >> 3;
             uint4 val = *ptr;
             if (r >= L) {
                 val = make_uint4(0u, 0u, 0u, 0u);
@@ -372,23 +448,28 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
                 val = make_uint4(w[0], w[1], w[2], w[3]);
             }
             *ptr = val;
-        }
-        publish();
-        const bool hp = ms->hp;
-        const bool safe = ms->safe;
-        GDN_CL_PHASE(1, 3);  // convert
-
-        // ---- Gram: [K;Q] K^T ----
-        if (tid == 0) {
+        };
 #pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-                const uint32_t a = skqv + (ks >> 2) * 16384 + (ks & 3) * 32;
-                mma_f16_ss(tmem + PT_G, make_sdesc(a, 16, 1024), make_sdesc(a, 16, 1024),
-                           IDESC_KK_N64, ks > 0);
-            }
+        for (int q = 0; q < 1024 / kThreads; ++q) {
+            const int x = tid + q * kThreads;  // V halves: 2 x 512 chunks
+            convert16(kqv + 32768 + (x >> 9) * 8192, x & 511);
         }
-        mma_sync_point();
-        GDN_CL_PHASE(1, 4);  // Gram MMA
+        if (!mbar_wait_bounded(&ms->mma_bar, mma_phase, kWaitLimit)) timed_out = true;
+        mma_phase ^= 1;
+        tc_fence_after_sync();
+        // A / P, the solve and the W^T staging rewrite what the previous chunk's
+        // first store group (W^T, P, gates) reads: wait until it has been read.
+        if (tid == 32) bulk_wait_read_all_but_one();
+        __syncthreads();
+#pragma unroll
+        for (int q = 0; q < 1024 / kThreads; ++q) {
+            const int x = tid + q * kThreads;  // K halves: 2 x 512 chunks
+            convert16(kqv + (x >> 9) * 16384, x & 511);
+        }
+        const bool hp = gt.hp;
+        const bool safe = gt.safe;
+        GDN_CL_PHASE(1, 3);  // Gram + convert
+        GDN_CL_PHASE(1, 4);  // (merged)
 
         // ---- A (lanes 0..63) and P (lanes 64..127) ----
         float *As = reinterpret_cast<float *>(sm + P_AS);
@@ -401,14 +482,14 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
             tmem_ld32(trow + PT_G + c, v);
             tmem_wait_ld();
             if (safe) {
-                const float sr = row < kC ? ms->bG[r] : ms->Gam[r];
+                const float sr = row < kC ? gt.bG[r] : gt.Gam[r];
 #pragma unroll
-                for (int x = 0; x < 32; ++x) v[x] *= sr * ms->iGam[c + x];
+                for (int x = 0; x < 32; ++x) v[x] *= sr * gt.iGam[c + x];
             } else {
-                const float gr = ms->gam[r];
-                const float sr = row < kC ? ms->bb[r] : 1.f;
+                const float gr = gt.gam[r];
+                const float sr = row < kC ? gt.bb[r] : 1.f;
 #pragma unroll
-                for (int x = 0; x < 32; ++x) v[x] *= sr * expf(gr - ms->gam[c + x]);
+                for (int x = 0; x < 32; ++x) v[x] *= sr * expf(gr - gt.gam[c + x]);
             }
             if (row < kC) {
 #pragma unroll
@@ -423,29 +504,17 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
         __syncthreads();
         GDN_CL_PHASE(1, 5);  // A / P
 
-        // ---- T = (I + A)^-1 ----
-        if (tid < kC) {
-            const int bi = tid >> 4, col = tid & 15;
-            const float *Ab = As + (16 * bi) * kAS + 16 * bi;
-            float x[16];
-#pragma unroll
-            for (int rr = 0; rr < 16; ++rr) {
-                float a0 = (rr == col) ? 1.f : 0.f, a1 = 0.f;
-#pragma unroll
-                for (int ii = 0; ii + 1 < rr; ii += 2) {
-                    a0 -= Ab[rr * kAS + ii] * x[ii];
-                    a1 -= Ab[rr * kAS + ii + 1] * x[ii + 1];
-                }
-                if (rr & 1) a0 -= Ab[rr * kAS + rr - 1] * x[rr - 1];
-                x[rr] = a0 + a1;
-            }
-#pragma unroll
-            for (int rr = 0; rr < 16; ++rr) Ts[(16 * bi + rr) * kTS + 16 * bi + col] = x[rr];
+        // The previous chunk's stores have had the Gram, A / P time to land:
+        // report it ready, and refill its tile buffer with chunk l + 1 (the T
+        // tiles below also overwrite its U~ staging, read by then).
+        if (tid == 32) {
+            flush_delivery();
+            const Item nx = ms->items[(l + 1) & 3];
+            if (l >= 1 && nx.valid) issue_tma((l + 1) & 1, nx);
         }
-        __syncthreads();
-        solve_level<1>(As, Ts, Xs, tid);
-        solve_level<2>(As, Ts, Xs, tid);
-        solve_level<3>(As, Ts, Xs, tid);
+
+        // ---- T = (I + A)^-1 ----
+        solve_tril64(As, Ts, Xs, tid);
         GDN_CL_PHASE(1, 6);  // solve
 
         // ---- rows of T diag(b), T diag(b Gamma): fp16 hi / lo ----
@@ -453,7 +522,7 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
             const int grp = tid >> 6, r = tid & 63;
             const bool tg = grp >= 2;
             const int c = 32 * (grp & 1);
-            const float *scale = tg ? ms->bG : ms->bb;
+            const float *scale = tg ? gt.bG : gt.bb;
             float x[32];
 #pragma unroll
             for (int e = 0; e < 32; e += 4) {
@@ -487,11 +556,15 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
                     const uint64_t b = make_sdesc(sbase + (pass ? P_TGL : P_TGH) + ks * 32, 16, 1024);
                     mma_f16_ss(tmem + PT_G, a, b, IDESC_MK_N64, (pass | ks) != 0);
                 }
+            mma_commit(&ms->mma_bar);
         }
-        mma_sync_point();
+        if (warp == 0 && ms->items[(l + 1) & 3].valid) compute_gates(ms->gt[(l + 1) & 1]);
+        if (!mbar_wait_bounded(&ms->mma_bar, mma_phase, kWaitLimit)) timed_out = true;
+        mma_phase ^= 1;
+        tc_fence_after_sync();
         GDN_CL_PHASE(1, 8);  // U~ / W MMAs
 
-        // ---- staging: W^T hi/lo (MN-major), U~^T (swizzled fp32), gates ----
+        // ---- staging: W^T hi/lo (MN-major), U~^T (swizzled fp32), gates, Q^T ----
         {
             const int c = 32 * half;
             float v[32];
@@ -504,23 +577,43 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
             for (int q = 0; q < 8; ++q)
                 *reinterpret_cast<float4 *>(sm + P_UTS + ut_off(row, c / 4 + q)) =
                     make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-            GatesBlock *gs = reinterpret_cast<GatesBlock *>(sm + P_GST);
             if (tid < kC) {
-                gs->Gam[tid] = ms->Gam[tid];
-                gs->eC[tid] = ms->eC[tid];
+                ms->gst.Gam[tid] = gt.Gam[tid];
+                ms->gst.eC[tid] = gt.eC[tid];
             }
-            if (tid == 0) gs->hp = hp;
+            if (tid == 0) ms->gst.hp = hp;
+        }
+        {   // Q^T fp16 (MN-major: row d holds 64 tokens) from the bf16 Q tile into
+            // the V half of the tile buffer, which the U~ product has finished reading
+            const int d = tid & 127, tq = (tid >> 7) * 32;
+            const uint8_t *qsrc = kqv + (d >> 6) * 16384 + 8192;
+            const uint32_t dbyte = (uint32_t)(d & 63) * 2u;
+#pragma unroll
+            for (int g8 = 0; g8 < 4; ++g8) {
+                uint32_t w[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const uint32_t t = (uint32_t)(tq + 8 * g8 + 2 * e);
+                    const float a = (int)t < L
+                        ? __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(qsrc + sw128(t, dbyte)))
+                        : 0.f;
+                    const float b = (int)t + 1 < L
+                        ? __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(qsrc + sw128(t + 1, dbyte)))
+                        : 0.f;
+                    w[e] = pack_half2(a, b);
+                }
+                st_row_chunk(kqv + 32768, d, (tq >> 3) + g8, make_uint4(w[0], w[1], w[2], w[3]));
+            }
         }
         fence_proxy_async_smem();  // staged data -> visible to the bulk copies
-        __syncthreads();
         GDN_CL_PHASE(1, 9);  // staging
 
-        // ---- deliver through the L2 ring once its slot is free ----
+        // ---- the ring slot must be free; then deliver with asynchronous stores ----
         if (tid == 32) {
             ms->items[(l + 2) & 3] = fetch(l + 2);
             if constexpr (kPool) {
-                if (it.c >= kRingSlots &&
-                    !wait_flag_geq(unit_flags(p, it.unit), (uint32_t)(it.c - kRingSlots + 1),
+                if (it.c >= p.ring_slots &&
+                    !wait_flag_geq(unit_flags(p, it.unit), (uint32_t)(it.c - p.ring_slots + 1),
                                    p.flags + 1, kWaitLimit))
                     timed_out = true;
             } else {
@@ -537,29 +630,26 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
             break;
         }
         GDN_CL_PHASE(1, 10);  // wait: ring slot free
-        if (tid == 32) {  // one thread of warp 1 issues the stores; warp 0 moves on to the gates
+        if (tid == 32) {
             uint8_t *dst = ring_slot(p, it.unit, it.c);
             fence_proxy_async_global();  // the chain's reads of this slot precede our writes
+            // group 1: what the next chunk rewrites first (read before its A / P)
+            bulk_store(dst + SL_WH, sm + P_WST, hp ? 32768 : 16384);
+            bulk_store(dst + SL_P16, sm + P_P16, 8192);
+            bulk_store(dst + SL_GATES, &ms->gst, (uint32_t)sizeof(GatesBlock));
+            bulk_commit();
+            // group 2: U~ (in the T tiles' space), K and Q^T (in the tile buffer)
+            bulk_store(dst + SL_UT, sm + P_UTS, 32768);
             bulk_store(dst + SL_K16, kqv, 8192);
             bulk_store(dst + SL_K16 + 8192, kqv + 16384, 8192);
-            bulk_store(dst + SL_Q16, kqv + 8192, 8192);
-            bulk_store(dst + SL_Q16 + 8192, kqv + 16384 + 8192, 8192);
-            bulk_store(dst + SL_WH, sm + P_WST, hp ? 32768 : 16384);
-            bulk_store(dst + SL_UT, sm + P_UTS, 32768);
-            bulk_store(dst + SL_P16, sm + P_P16, 8192);
-            bulk_store(dst + SL_GATES, sm + P_GST, (uint32_t)sizeof(GatesBlock));
+            bulk_store(dst + SL_QT, kqv + 32768, 16384);
             bulk_commit();
-            bulk_wait_all();              // written to global memory
-            fence_proxy_async_global();   // ... ordered before the signal below
-            if constexpr (kPool)
-                st_release_gpu(unit_flags(p, it.unit) + 1 + it.c % kRingSlots, (uint32_t)(it.c + 1));
-            else
-                mbar_arrive_remote(c_ready);
-            const Item nx2 = ms->items[(l + 2) & 3];
-            if (nx2.valid) issue_tma(buf, nx2);  // this buffer is free now
+            pending = it;
         }
         GDN_CL_PHASE(1, 11);  // deliver (issue)
     }
+    if (tid == 32) flush_delivery();  // the last chunk delivered
+    GDN_CL_PHASE_END(1);
     // A tile load issued for a chunk this loop never reached must land before
     // this CTA's shared memory can go away (chunk l + 1's, after a timeout;
     // on a normal exit chunks l and l + 1 do not exist).
@@ -628,38 +718,70 @@ __device__ void chain_role(uint8_t *sm, const ChainParams &p, int unit, int n, i
         __syncthreads();
         tc_fence_after_sync();
     };
-    // has chunk cc reached the ring?  (thread 0)
+    // Has chunk cc reached the ring?  (thread 0)  The pool kernel reads the
+    // flag with a relaxed load whose value is only examined on a later call,
+    // so the L2 round trip overlaps other work; an observed flag is turned
+    // into an acquire by a fence.
+    uint32_t polled = 0;
+    int polled_for = -1;  // the chunk whose flag `polled` holds
+    auto read_flag = [&](int cc) {
+        if constexpr (kPool) {
+            polled = ld_relaxed_gpu(uflags + 1 + (cc & (p.ring_slots - 1)));
+            polled_for = cc;
+        }
+    };
     auto ready_try = [&](int cc) -> bool {
-        if constexpr (kPool)
-            return ld_acquire_gpu(uflags + 1 + cc % kRingSlots) >= (uint32_t)(cc + 1);
-        else
+        if constexpr (kPool) {
+            if (polled_for == cc && polled >= (uint32_t)(cc + 1)) {
+                fence_acq_rel_gpu();
+                polled_for = -1;
+                return true;
+            }
+            read_flag(cc);
+            return false;
+        } else {
             return mbar_try_wait_cluster(&ms->ready[cc & 1], ((cc >> 1) & 1));
+        }
     };
     auto ready_wait = [&](int cc) -> bool {
         if constexpr (kPool)
-            return wait_flag_geq(uflags + 1 + cc % kRingSlots, (uint32_t)(cc + 1), p.flags + 1,
+            return wait_flag_geq(uflags + 1 + (cc & (p.ring_slots - 1)), (uint32_t)(cc + 1), p.flags + 1,
                                  kWaitLimit);
         else
             return mbar_wait_cluster_bounded(&ms->ready[cc & 1], (cc >> 1) & 1, kWaitLimit);
     };
 
 #ifdef GDN_TC_PHASES
-    long long phase_t_ = clock64();
     const bool phase_on_ = blockIdx.x == 0;
 #endif
+    GDN_CL_PHASE_BEGIN();
     // Thread 0 loads chunk c + 1 from the ring into shared slot (c + 1) & 1 as
     // soon as it is reported ready, while chunk c is processed; the shared
     // slot held chunk c - 1, which is finished.
     int loaded = 0;  // chunks whose load has been issued
-    auto issue_load = [&](int cc) {
+    auto issue_load = [&](int cc) {  // four copies, which the copy engine can overlap
         fence_proxy_async_global();  // the producer's stores, acquired, precede our bulk load
-        mbar_arrive_expect_tx(&ms->full[cc & 1], SLOT_BYTES);
-        bulk_load(sm + (cc & 1) * SLOT_BYTES, ring_slot(p, unit, cc), SLOT_BYTES, &ms->full[cc & 1]);
+        uint64_t *bar = &ms->full[cc & 1];
+        mbar_arrive_expect_tx(bar, SLOT_BYTES);
+        uint8_t *dst = sm + (cc & 1) * SLOT_BYTES;
+        const uint8_t *src = ring_slot(p, unit, cc);
+        bulk_load(dst, src, SL_WH, bar);                                   // K, Q^T
+        bulk_load(dst + SL_WH, src + SL_WH, SL_UT - SL_WH, bar);           // W^T hi, lo
+        bulk_load(dst + SL_UT, src + SL_UT, SL_P16 - SL_UT, bar);          // U~^T
+        bulk_load(dst + SL_P16, src + SL_P16, SLOT_BYTES - SL_P16, bar);   // P, gates
     };
+    // cur: the chunk in progress; the shared slot of chunk cur + 1 is free.
+    // Loads chunk cur + 1 once it is ready; when it is loaded already, starts
+    // reading the flag of chunk cur + 2 (its slot frees up with chunk cur).
     auto poll_next = [&](int cur) {
-        if (tid == 0 && loaded == cur + 1 && cur + 1 < nch && ready_try(cur + 1)) {
-            issue_load(cur + 1);
-            loaded = cur + 2;
+        if (tid != 0) return;
+        if (loaded == cur + 1 && cur + 1 < nch) {
+            if (ready_try(cur + 1)) {
+                issue_load(cur + 1);
+                loaded = cur + 2;
+            }
+        } else if (loaded == cur + 2 && cur + 2 < nch && polled_for != cur + 2) {
+            read_flag(cur + 2);
         }
     };
     int c = 0;
@@ -684,11 +806,12 @@ __device__ void chain_role(uint8_t *sm, const ChainParams &p, int unit, int n, i
                 mbar_arrive(&ms->full[k]);
             }
         }
+        poll_next(c);  // chunk c + 1 may be ready already: load it while c computes
         if (!mbar_wait_bounded(&ms->full[k], (c >> 1) & 1, kWaitLimit)) timed_out = true;
         GDN_CL_PHASE(0, 0);  // wait: delivery
         if (tid == 0 && have) {  // the chunk is out of the ring: its slot may be refilled
             if constexpr (kPool)
-                st_release_gpu(uflags, (uint32_t)(c + 1));
+                st_relaxed_gpu(uflags, (uint32_t)(c + 1));
             else
                 mbar_arrive_remote(mapa_shared(prod_taken_local, 1 + k));
         }
@@ -696,23 +819,20 @@ __device__ void chain_role(uint8_t *sm, const ChainParams &p, int unit, int n, i
         const bool hp = gb->hp != 0;
         const float gC = gb->Gam[kC - 1];
 
-        // ---- S Q^T -> O, R = S W^T (A operands from TMEM) ----
+        // ---- [O | R | R2] = S_hi [Q^T | W^T hi | W^T lo]  (+ S_lo W^T hi into R) ----
         if (tid == 0) {
             tc_fence_after_sync();
+            const uint32_t idesc = hp ? IDESC_KM_N192 : IDESC_KM_N128;
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks)
                 mma_f16_ts(tmem + CT_O, tmem + CT_SH + 8 * ks,
-                           make_sdesc(sslot + SL_Q16 + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024),
-                           IDESC_KK_N64, ks > 0);
-            for (int pass = 0; pass < (hp ? 3 : 1); ++pass)
+                           make_sdesc(sslot + SL_QT + ks * 2048, 16384, 1024), idesc, ks > 0);
+            if (hp) {
 #pragma unroll
-                for (int ks = 0; ks < 8; ++ks) {
-                    const uint32_t a_col = pass == 2 ? CT_SL : CT_SH;
-                    const uint32_t w_off = pass == 1 ? SL_WL : SL_WH;
-                    mma_f16_ts(tmem + CT_R, tmem + a_col + 8 * ks,
-                               make_sdesc(sslot + w_off + ks * 2048, 16384, 1024), IDESC_KM_N64,
-                               (pass | ks) != 0);
-                }
+                for (int ks = 0; ks < 8; ++ks)
+                    mma_f16_ts(tmem + CT_R, tmem + CT_SL + 8 * ks,
+                               make_sdesc(sslot + SL_WH + ks * 2048, 16384, 1024), IDESC_KM_N64, 1);
+            }
             mma_commit(&ms->mma_bar);
         }
         poll_next(c);
@@ -722,12 +842,20 @@ __device__ void chain_role(uint8_t *sm, const ChainParams &p, int unit, int n, i
         tc_fence_after_sync();
         GDN_CL_PHASE(0, 2);  // wait: S Q^T, R
 
-        // ---- O *= Gamma (rows of the transposed output); U = U~ - R; U', U ----
+        // ---- O *= Gamma (rows of the transposed output); U = U~ - R; U', U -> TMEM ----
         {
             const int c32 = 32 * half;
             float v[32], r0[32];
             tmem_ld32(trow + CT_O + c32, v);
+            tmem_ld32(trow + CT_R + c32, r0);
             tmem_wait_ld();
+            if (hp) {
+                float r2[32];
+                tmem_ld32(trow + CT_R2 + c32, r2);
+                tmem_wait_ld();
+#pragma unroll
+                for (int x = 0; x < 32; ++x) r0[x] += r2[x];
+            }
 #pragma unroll
             for (int x = 0; x < 32; ++x) v[x] *= gb->Gam[c32 + x];
             tmem_st32(trow + CT_O + c32, v);
@@ -736,33 +864,38 @@ __device__ void chain_role(uint8_t *sm, const ChainParams &p, int unit, int n, i
                 const float4 f = *reinterpret_cast<const float4 *>(slot + SL_UT + ut_off(row, c32 / 4 + q));
                 v[4 * q] = f.x; v[4 * q + 1] = f.y; v[4 * q + 2] = f.z; v[4 * q + 3] = f.w;
             }
-            tmem_ld32(trow + CT_R + c32, r0);
-            tmem_wait_ld();
-            __syncthreads();  // every U~ row is read before U' overwrites the region
+            uint32_t uh[16], ul[16], u16[16];
 #pragma unroll
-            for (int x = 0; x < 32; ++x) {
-                v[x] -= r0[x];
-                r0[x] = v[x] * gb->eC[c32 + x];
+            for (int x = 0; x < 32; x += 2) {
+                const float u0 = v[x] - r0[x], u1 = v[x + 1] - r0[x + 1];
+                const float p0 = u0 * gb->eC[c32 + x], p1 = u1 * gb->eC[c32 + x + 1];
+                const __half2 hh = __floats2half2_rn(p0, p1);
+                const float2 hf = __half22float2(hh);
+                uh[x / 2] = *reinterpret_cast<const uint32_t *>(&hh);
+                ul[x / 2] = pack_half2(p0 - hf.x, p1 - hf.y);
+                u16[x / 2] = pack_half2(u0, u1);
             }
-            store_split32(slot + SL_UP, slot + SL_UP + 16384, row, c32, r0, true);
-#pragma unroll
-            for (int e = 0; e < 32; e += 8) st_row_chunk(slot + SL_U16, row, (c32 + e) / 8, pack8(v + e));
+            tmem_st16u(trow + CT_UP + c32 / 2, uh);
+            tmem_st16u(trow + CT_UP + 32 + c32 / 2, ul);
+            tmem_st16u(trow + CT_U16 + c32 / 2, u16);
         }
-        publish();
+        tmem_wait_st();
+        tc_fence_before_sync();
+        __syncthreads();
+        tc_fence_after_sync();
         poll_next(c);
         GDN_CL_PHASE(0, 3);  // O scale, U, U'
 
-        // ---- dS = [U'hi | U'lo] [K ; K];  O += U^T P^T ----
+        // ---- dS = [U'hi | U'lo] [K ; K];  O += U^T P^T  (A operands from TMEM) ----
         if (tid == 0) {
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks)
-                mma_f16_ss(tmem + CT_D,
-                           make_sdesc(sslot + SL_UP + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024),
+                mma_f16_ts(tmem + CT_D, tmem + CT_UP + 8 * ks,
                            make_sdesc(sslot + SL_K16 + (ks & 3) * 2048, 8192, 1024), IDESC_KM_N128,
                            ks > 0);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
-                mma_f16_ss(tmem + CT_O, make_sdesc(sslot + SL_U16 + ks * 32, 16, 1024),
+                mma_f16_ts(tmem + CT_O, tmem + CT_U16 + 8 * ks,
                            make_sdesc(sslot + SL_P16 + ks * 32, 16, 1024), IDESC_KK_N64, 1);
         }
         poll_next(c);
@@ -841,6 +974,7 @@ __device__ void chain_role(uint8_t *sm, const ChainParams &p, int unit, int n, i
                 *reinterpret_cast<float4 *>(dst + cc + x) = make_float4(v[x], v[x + 1], v[x + 2], v[x + 3]);
         }
     }
+    GDN_CL_PHASE_END(0);
     if (aborted) {
         // A prefetch still landing in shared memory must finish (c is one past
         // the chunk that voted; every earlier load has been waited for).
@@ -979,14 +1113,14 @@ int sm_count() {
 
 }  // namespace
 
-static_assert(kRingSlots * SLOT_BYTES == kClusterWorkspaceBytesPerUnit, "ring size per unit");
+static_assert(kClusterRingSlots * SLOT_BYTES == kClusterWorkspaceBytesPerUnit, "ring size per unit");
 
 size_t prefill_cluster_workspace_bytes(int64_t units) {
-    return (size_t)units * kRingSlots * SLOT_BYTES;
+    return (size_t)units * kClusterRingSlots * SLOT_BYTES;
 }
 
 size_t prefill_pool_workspace_bytes(int64_t units) {
-    return pool_flag_bytes(units) + (size_t)units * kRingSlots * SLOT_BYTES;
+    return pool_flag_bytes(units) + (size_t)units * kPoolRingSlots * SLOT_BYTES;
 }
 
 bool prefill_pool_fits(int64_t units) {
@@ -1010,6 +1144,7 @@ bool fill_params(const PrefillArgs &a, ChainParams &p, CUtensorMap &mq, CUtensor
     p.T = a.T; p.N = a.N; p.Hqk = a.Hqk; p.Hv = a.Hv;
     p.units = a.N * a.Hv;
     p.max_chunks = (int)((a.T + kC - 1) / kC);
+    p.ring_slots = kClusterRingSlots;
     return true;
 }
 }  // namespace
@@ -1035,6 +1170,7 @@ cudaError_t launch_prefill_pool(const PrefillArgs &a, cudaStream_t s) {
     const size_t fb = pool_flag_bytes(p.units);
     p.flags = static_cast<uint32_t *>(a.ws);
     p.ring = static_cast<uint8_t *>(a.ws) + fb;
+    p.ring_slots = kPoolRingSlots;
     // the chunk counter, abort flag and hand-off flags start at zero
     cudaError_t e = cudaMemsetAsync(a.ws, 0, fb, s);
     if (e != cudaSuccess) return e;
@@ -1060,11 +1196,11 @@ cudaError_t launch_prefill_pool(const PrefillArgs &a, cudaStream_t s) {
 
 #ifdef GDN_TC_PHASES
 extern "C" GDN_API int gdn_debug_cluster_phases(long long *out, int reset) {
-    long long host[32];
+    unsigned long long host[32];
     if (cudaMemcpyFromSymbol(host, gdn_cl_phase_clk, sizeof(host)) != cudaSuccess) return -1;
-    for (int i = 0; i < 32; ++i) out[i] = host[i];
+    for (int i = 0; i < 32; ++i) out[i] = (long long)host[i];
     if (reset) {
-        const long long zero[32] = {0};
+        const unsigned long long zero[32] = {0};
         cudaMemcpyToSymbol(gdn_cl_phase_clk, zero, sizeof(zero));
     }
     return 0;

@@ -136,6 +136,12 @@ __device__ __forceinline__ void bulk_wait_read_all() {
     asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
 
+// Waits until the sources of all but the most recent committed bulk store
+// group have been read.
+__device__ __forceinline__ void bulk_wait_read_all_but_one() {
+    asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
+
 // Waits until every committed bulk store has completed.
 __device__ __forceinline__ void bulk_wait_all() {
     asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
@@ -235,6 +241,15 @@ __device__ __forceinline__ void st_release_gpu(uint32_t *p, uint32_t v) {
     asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
+__device__ __forceinline__ void st_relaxed_gpu(uint32_t *p, uint32_t v) {
+    asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Turns an earlier relaxed load that observed a flag into an acquire.
+__device__ __forceinline__ void fence_acq_rel_gpu() {
+    asm volatile("fence.acq_rel.gpu;" ::: "memory");
+}
+
 // Spins until *flag >= want (acquire).  Returns false, without waiting
 // further, once *abort is non-zero or after `limit` SM clocks.
 __device__ __forceinline__ bool wait_flag_geq(const uint32_t *flag, uint32_t want,
@@ -332,6 +347,16 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) 
         : "memory");
 }
 
+__device__ __forceinline__ void tmem_st16u(uint32_t taddr, const uint32_t (&v)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+        "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+        "r"(v[15])
+        : "memory");
+}
+
 __device__ __forceinline__ void tmem_st32u(uint32_t taddr, const uint32_t (&v)[32]) {
     asm volatile(
         "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
@@ -369,13 +394,13 @@ __device__ __forceinline__ uint64_t make_sdesc(uint32_t saddr, uint32_t lbo_byte
     return d;
 }
 
-// kind::f16 instruction descriptor: fp32 accumulator, fp16 A and B,
+// kind::f16 instruction descriptor: fp32 accumulator, A and B both fp16 or both bf16,
 // A/B major-ness (0 = K-major, 1 = MN-major), N >> 3 at bit 17, M >> 4 at bit 24.
 __host__ __device__ constexpr uint32_t make_idesc_f16(int M, int N, int a_mn_major,
-                                                      int b_mn_major) {
+                                                      int b_mn_major, int bf16 = 0) {
     return (1u << 4)                          // D format: f32
-           | (0u << 7)                        // A format: f16
-           | (0u << 10)                       // B format: f16
+           | ((uint32_t)bf16 << 7)            // A format: f16 (0) or bf16 (1)
+           | ((uint32_t)bf16 << 10)           // B format: same as A
            | ((uint32_t)a_mn_major << 15)     // A major
            | ((uint32_t)b_mn_major << 16)     // B major
            | ((uint32_t)(N >> 3) << 17)       // N

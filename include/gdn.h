@@ -150,9 +150,9 @@ GDN_API gdn_status gdn_prefill_ex(const void *q, const void *k, const void *v, g
 
 /*
  * gdn_prefill_workspace_bytes -- scratch bytes gdn_prefill needs for these
- * sizes (0 when none): 430,080 bytes per (sequence, v-head) unit, plus a
- * flag block of 1 KB or more for the pool kernel, when AUTO would run the
- * pool kernel.  Pure function of its arguments (it cannot see the dtype, so
+ * sizes (0 when none): when AUTO would run the pool kernel, 860,160 bytes per
+ * (sequence, v-head) unit plus a flag block of 4 KB or more (the cluster
+ * kernel, chosen explicitly, takes 430,080 bytes per unit).  Pure function of its arguments (it cannot see the dtype, so
  * it may ask for a workspace an fp32 call does not use); no device access.
  * The workspace is device memory, 256-byte aligned, owned by the caller; its
  * contents need no initialisation (the pool kernel clears its flag block on
