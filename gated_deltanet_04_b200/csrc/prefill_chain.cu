@@ -147,7 +147,7 @@ constexpr uint32_t P_KQV_BYTES = 49152;
 constexpr uint32_t P_X = 98304;         // solve scratch: A, T, X (fp32); then W^T hi/lo staging
 constexpr uint32_t P_WST = P_X;
 constexpr uint32_t P_AS = P_X;
-constexpr uint32_t P_TS = P_X + 64 * kAS * 4;
+constexpr uint32_t P_TS = P_X + 64 * kAS4 * 4;
 constexpr uint32_t P_XS = P_TS + 64 * kTS * 4;
 constexpr uint32_t P_P16 = 137216;      // P fp16 [64 rows][128 B], SW128
 constexpr uint32_t P_TBH = 145408, P_TBL = 153600, P_TGH = 161792, P_TGL = 169984;  // T tiles
@@ -376,9 +376,9 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
     };
 
     // Chunks l and l + 1 are known when chunk l starts (tile loads of chunks
-    // 0 and 1 are issued here, those of chunk l + 1 > 1 during chunk l, once
-    // the stores of chunk l - 1 have read its buffer); the delivery thread
-    // fetches chunk l + 2 before the vote of chunk l.
+    // 0 and 1 are issued here, those of chunk l + 1 > 1 during the U~ / W
+    // products of chunk l, after the stores of chunk l - 1 have landed); the
+    // delivery thread fetches chunk l + 2 before the vote of chunk l.
     if (tid == 32) {
         for (int l = 0; l < 2; ++l) {
             const Item it = fetch(l);
@@ -493,7 +493,10 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
             }
             if (row < kC) {
 #pragma unroll
-                for (int x = 0; x < 32; ++x) As[r * kAS + c + x] = (c + x < r) ? v[x] : 0.f;
+                for (int x = 0; x < 32; x += 4)  // 16-byte stores: conflict-free at stride kAS4
+                    *reinterpret_cast<float4 *>(As + r * kAS4 + c + x) =
+                        make_float4((c + x < r) ? v[x] : 0.f, (c + x + 1 < r) ? v[x + 1] : 0.f,
+                                    (c + x + 2 < r) ? v[x + 2] : 0.f, (c + x + 3 < r) ? v[x + 3] : 0.f);
             } else {
 #pragma unroll
                 for (int x = 0; x < 32; ++x) v[x] = (c + x <= r) ? v[x] : 0.f;
@@ -504,14 +507,10 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
         __syncthreads();
         GDN_CL_PHASE(1, 5);  // A / P
 
-        // The previous chunk's stores have had the Gram, A / P time to land:
-        // report it ready, and refill its tile buffer with chunk l + 1 (the T
-        // tiles below also overwrite its U~ staging, read by then).
-        if (tid == 32) {
-            flush_delivery();
-            const Item nx = ms->items[(l + 1) & 3];
-            if (l >= 1 && nx.valid) issue_tma((l + 1) & 1, nx);
-        }
+        // The T tiles below overwrite the previous chunk's U~ staging: its
+        // stores must have read it (long done by now; the solve's first
+        // barrier orders this before every thread's writes).
+        if (tid == 32) bulk_wait_read_all();
 
         // ---- T = (I + A)^-1 ----
         solve_tril64(As, Ts, Xs, tid);
@@ -559,6 +558,11 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
             mma_commit(&ms->mma_bar);
         }
         if (warp == 0 && ms->items[(l + 1) & 3].valid) compute_gates(ms->gt[(l + 1) & 1]);
+        if (tid == 32) {  // idle during these products: report the previous chunk
+            flush_delivery();  // ready once its stores have landed, refill its buffer
+            const Item nx = ms->items[(l + 1) & 3];
+            if (l >= 1 && nx.valid) issue_tma((l + 1) & 1, nx);
+        }
         if (!mbar_wait_bounded(&ms->mma_bar, mma_phase, kWaitLimit)) timed_out = true;
         mma_phase ^= 1;
         tc_fence_after_sync();

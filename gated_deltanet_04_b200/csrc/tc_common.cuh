@@ -19,6 +19,7 @@ constexpr int kD = 128;     // Dk = Dv
 constexpr long long kWaitLimit = 1ll << 31;  // SM clocks (about a second)
 constexpr float kHighPrecisionDecay = 0.2f;  // Gamma_C at or above -> extra passes
 constexpr int kAS = 65;  // row stride of A (scalar, conflict-free column access)
+constexpr int kAS4 = 68; // row stride of A for solve_tril64 (16-byte aligned rows)
 constexpr int kTS = 68;  // row stride of T (16-byte aligned rows for float4 access)
 
 constexpr uint32_t IDESC_KK_N64 = make_idesc_f16(128, 64, 0, 0);
@@ -109,100 +110,141 @@ __device__ __forceinline__ void solve_level(const float *As, float *Ts, float *X
     __syncthreads();
 }
 
-// T = (I + A)^-1 for the 64 x 64 strictly lower A in As (row stride kAS), into
-// Ts (row stride kTS), fp32, 256 threads.  Three steps:
+// T = (I + A)^-1 for the 64 x 64 strictly lower A in As (row stride kAS4),
+// into Ts (row stride kTS), fp32, 256 threads.  Three steps:
 //   1. the four 16 x 16 diagonal blocks D_i = (I + A_ii)^-1, by forward
-//      substitution (one thread per (block, column));
-//   2. T_10 = -D_1 A_10 D_0 and T_32 = -D_3 A_32 D_2 (upper 32 x 32 halves);
-//   3. the lower-left 32 x 32 block T_bl = -T_bot (A_bl T_top), where T_top
-//      and T_bot are the two lower-triangular 32 x 32 diagonal halves.
-// Each step keeps most threads busy; block-triangular zeros are skipped.  The
-// entries above the diagonal blocks of Ts are left unwritten and never read.
-// Xs needs 1024 floats.  Callers synchronise before (As complete) and after.
+//      substitution (one thread per (block, column)); the threads idle there
+//      write zeros above the diagonal blocks;
+//   2. T_10 = -D_1 A_10 D_0 and T_32 = -D_3 A_32 D_2 (the 32 x 32 halves);
+//   3. the lower-left 32 x 32 block T_bl = -T_bot (A_bl T_top), where T_top and
+//      T_bot are the two lower-triangular 32 x 32 diagonal halves.
+// The block products map a lane to an output column and a warp to four output
+// rows: the right operand is one conflict-free 32-bit load per term, the left
+// operand a broadcast 16-byte load per four terms, which keeps the products off
+// the shared-memory wavefront limit.  The 16 x 16 products split their sums over
+// the two half-warps.  As must hold explicit zeros on and above its diagonal
+// and have 16-byte aligned rows.  Xs needs 1024 floats.  Callers synchronise
+// before (As complete); the function ends with a barrier.
 __device__ __forceinline__ void solve_tril64(const float *As, float *Ts, float *Xs, int tid) {
+    const int warp = tid >> 5, lane = tid & 31;
     if (tid < kC) {  // 1. diagonal blocks
         const int bi = tid >> 4, col = tid & 15;
-        const float *Ab = As + (16 * bi) * kAS + 16 * bi;
+        const float *Ab = As + (16 * bi) * kAS4 + 16 * bi;
         float x[16];
 #pragma unroll
         for (int rr = 0; rr < 16; ++rr) {
             float a0 = (rr == col) ? 1.f : 0.f, a1 = 0.f;
 #pragma unroll
             for (int ii = 0; ii + 1 < rr; ii += 2) {
-                a0 -= Ab[rr * kAS + ii] * x[ii];
-                a1 -= Ab[rr * kAS + ii + 1] * x[ii + 1];
+                a0 -= Ab[rr * kAS4 + ii] * x[ii];
+                a1 -= Ab[rr * kAS4 + ii + 1] * x[ii + 1];
             }
-            if (rr & 1) a0 -= Ab[rr * kAS + rr - 1] * x[rr - 1];
+            if (rr & 1) a0 -= Ab[rr * kAS4 + rr - 1] * x[rr - 1];
             x[rr] = a0 + a1;
         }
 #pragma unroll
         for (int rr = 0; rr < 16; ++rr) Ts[(16 * bi + rr) * kTS + 16 * bi + col] = x[rr];
+    } else {  // zeros above the diagonal blocks: 6 blocks of 16 x 16, 8 floats per thread
+        const int z = tid - kC;              // 0 .. 191
+        const int blk = z >> 5, part = z & 31;
+        // upper blocks (bi, bj), bi < bj: (0,1) (0,2) (0,3) (1,2) (1,3) (2,3)
+        const int bi = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
+        const int bj = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
+        const int rr = part >> 1, c8 = 8 * (part & 1);
+        float *dst = Ts + (16 * bi + rr) * kTS + 16 * bj + c8;
+        *reinterpret_cast<float4 *>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
+        *reinterpret_cast<float4 *>(dst + 4) = make_float4(0.f, 0.f, 0.f, 0.f);
     }
     __syncthreads();
-    {   // 2a. X = A_{i,i-1} D_{i-1} for i = 1, 3
-        const int blk = tid >> 6;            // 0, 1 active (128 threads)
-        const int r = (tid >> 2) & 15, c4 = 4 * (tid & 3);
-        if (blk < 2) {
-            const int bi = 2 * blk + 1, bk = bi - 1;
-            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-            const float *arow = As + (16 * bi + r) * kAS + 16 * bk;
-            const float *tcol = Ts + (16 * bk) * kTS + 16 * bk + c4;
+    // 2.: warp -> block b (i = 2b + 1, k = 2b) and rows rq .. rq + 3; lane -> column
+    // (lane & 15) and half of the 16-term sum (lane >> 4)
+    const int b2 = warp >> 2, rq = 4 * (warp & 3), col = lane & 15, kh = lane >> 4;
+    const int bi = 2 * b2 + 1, bk = bi - 1;
+    {   // 2a. X = A_{i,k} D_k
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int m = 0; m < 16; ++m) {
-                const float a = arow[m];
-                const float4 t = *reinterpret_cast<const float4 *>(tcol + m * kTS);
-                acc.x = fmaf(a, t.x, acc.x); acc.y = fmaf(a, t.y, acc.y);
-                acc.z = fmaf(a, t.z, acc.z); acc.w = fmaf(a, t.w, acc.w);
-            }
-            *reinterpret_cast<float4 *>(Xs + (blk << 8) + r * 16 + c4) = acc;
-        }
-    }
-    __syncthreads();
-    {   // 2b. T_{i,i-1} = -D_i X
-        const int blk = tid >> 6;
-        const int r = (tid >> 2) & 15, c4 = 4 * (tid & 3);
-        if (blk < 2) {
-            const int bi = 2 * blk + 1, bk = bi - 1;
-            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-            const float *drow = Ts + (16 * bi + r) * kTS + 16 * bi;
+        for (int mg = 0; mg < 8; mg += 4) {
+            const int m = 8 * kh + mg;
+            float4 a4[4];
 #pragma unroll
-            for (int m = 0; m < 16; ++m) {
-                const float d = drow[m];
-                const float4 x = *reinterpret_cast<const float4 *>(Xs + (blk << 8) + m * 16 + c4);
-                acc.x = fmaf(d, x.x, acc.x); acc.y = fmaf(d, x.y, acc.y);
-                acc.z = fmaf(d, x.z, acc.z); acc.w = fmaf(d, x.w, acc.w);
-            }
-            *reinterpret_cast<float4 *>(Ts + (16 * bi + r) * kTS + 16 * bk + c4) =
-                make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
+            for (int j = 0; j < 4; ++j)
+                a4[j] = *reinterpret_cast<const float4 *>(As + (16 * bi + rq + j) * kAS4 + 16 * bk + m);
+            float y[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) y[q] = Ts[(16 * bk + m + q) * kTS + 16 * bk + col];
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                acc[j] = fmaf(a4[j].x, y[0], fmaf(a4[j].y, y[1], fmaf(a4[j].z, y[2], fmaf(a4[j].w, y[3], acc[j]))));
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], 16);
+        if (kh == 0) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) Xs[(b2 << 8) + (rq + j) * 16 + col] = acc[j];
         }
     }
     __syncthreads();
-    const int r = tid >> 3, c4 = 4 * (tid & 7);  // 32 rows x 8 column groups
-    {   // 3a. X = A_bl T_top   (T_top[m][c] = 0 for m < c)
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        const float *arow = As + (32 + r) * kAS;
-#pragma unroll 4
-        for (int m = c4; m < 32; ++m) {
-            const float a = arow[m];
-            const float4 t = *reinterpret_cast<const float4 *>(Ts + m * kTS + c4);
-            acc.x = fmaf(a, t.x, acc.x); acc.y = fmaf(a, t.y, acc.y);
-            acc.z = fmaf(a, t.z, acc.z); acc.w = fmaf(a, t.w, acc.w);
+    {   // 2b. T_{i,k} = -D_i X
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int mg = 0; mg < 8; mg += 4) {
+            const int m = 8 * kh + mg;
+            float4 d4[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                d4[j] = *reinterpret_cast<const float4 *>(Ts + (16 * bi + rq + j) * kTS + 16 * bi + m);
+            float y[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) y[q] = Xs[(b2 << 8) + (m + q) * 16 + col];
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                acc[j] = fmaf(d4[j].x, y[0], fmaf(d4[j].y, y[1], fmaf(d4[j].z, y[2], fmaf(d4[j].w, y[3], acc[j]))));
         }
-        *reinterpret_cast<float4 *>(Xs + r * 32 + c4) = acc;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], 16);
+        if (kh == 0) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) Ts[(16 * bi + rq + j) * kTS + 16 * bk + col] = -acc[j];
+        }
     }
     __syncthreads();
-    {   // 3b. T_bl = -T_bot X   (T_bot[r][m] = 0 for m > r)
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        const float *brow = Ts + (32 + r) * kTS + 32;
-#pragma unroll 4
-        for (int m = 0; m <= r; ++m) {
-            const float b = brow[m];
-            const float4 x = *reinterpret_cast<const float4 *>(Xs + m * 32 + c4);
-            acc.x = fmaf(b, x.x, acc.x); acc.y = fmaf(b, x.y, acc.y);
-            acc.z = fmaf(b, x.z, acc.z); acc.w = fmaf(b, x.w, acc.w);
+    const int r4 = 4 * warp;  // 3.: rows r4 .. r4 + 3 of the 32 x 32 block, lane = column
+    {   // 3a. X = A_bl T_top
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int m = 0; m < 32; m += 4) {
+            float4 a4[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                a4[j] = *reinterpret_cast<const float4 *>(As + (32 + r4 + j) * kAS4 + m);
+            float y[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) y[q] = Ts[(m + q) * kTS + lane];
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                acc[j] = fmaf(a4[j].x, y[0], fmaf(a4[j].y, y[1], fmaf(a4[j].z, y[2], fmaf(a4[j].w, y[3], acc[j]))));
         }
-        *reinterpret_cast<float4 *>(Ts + (32 + r) * kTS + c4) =
-            make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) Xs[(r4 + j) * 32 + lane] = acc[j];
+    }
+    __syncthreads();
+    {   // 3b. T_bl = -T_bot X
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int m = 0; m < 32; m += 4) {
+            float4 t4[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                t4[j] = *reinterpret_cast<const float4 *>(Ts + (32 + r4 + j) * kTS + 32 + m);
+            float y[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) y[q] = Xs[(m + q) * 32 + lane];
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                acc[j] = fmaf(t4[j].x, y[0], fmaf(t4[j].y, y[1], fmaf(t4[j].z, y[2], fmaf(t4[j].w, y[3], acc[j]))));
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) Ts[(32 + r4 + j) * kTS + lane] = -acc[j];
     }
     __syncthreads();
 }
