@@ -96,6 +96,11 @@ using namespace tc;
 
 constexpr int kThreads = 256;
 constexpr int kCluster = 3;
+// producer threads with side duties (first lanes of warps that would otherwise
+// reach the end-of-chunk vote early): ring stores, ready signals and tile
+// refills; the chunk counter and the ring-slot check
+constexpr int kDeliverTid = 64;
+constexpr int kFetchTid = 96;
 constexpr int kClusterRingSlots = 4;
 constexpr int kPoolRingSlots = 8;
 
@@ -226,30 +231,47 @@ __device__ __forceinline__ uint32_t ut_off(int i, int q) {
     return (uint32_t)i * 256u + (uint32_t)((q ^ (i & 15)) << 4);
 }
 
-// The next chunk of the pool kernel's chunk-major order that exists (invalid
-// once the order is exhausted or the abort flag is up).  One thread calls it.
-__device__ Item pool_fetch(const ChainParams &p) {
+// The chunk at index i of the pool kernel's chunk-major order (valid == 0 once
+// the order is exhausted).  `skip` is set when index i names no chunk (a
+// shorter or malformed sequence): the caller then takes another index.
+__device__ Item pool_item(const ChainParams &p, uint32_t i, bool &skip) {
     Item it;
     it.valid = 0;
-    for (;;) {
-        if (ld_relaxed_gpu(p.flags + 1) != 0u) return it;
-        const uint32_t i = atomicAdd(p.flags, 1u);
-        const int c = (int)(i / (uint32_t)p.units);
-        const int unit = (int)(i % (uint32_t)p.units);
-        if (c >= p.max_chunks) return it;
-        const int n = unit / p.Hv;
-        int64_t t0, t1;
-        if (!seq_range(p.cu, n, p.N, p.T, nullptr, t0, t1)) continue;  // the chain reports it
-        const int64_t c0 = t0 + (int64_t)kC * c;
-        if (c0 >= t1) continue;  // a shorter sequence
-        it.c0 = c0;
-        it.unit = unit;
-        it.c = c;
-        it.h = unit % p.Hv;
-        it.j = it.h / (p.Hv / p.Hqk);
-        it.L = (int)((t1 - c0) < kC ? (t1 - c0) : kC);
-        it.valid = 1;
+    skip = false;
+    const int c = (int)(i / (uint32_t)p.units);
+    const int unit = (int)(i % (uint32_t)p.units);
+    if (c >= p.max_chunks) return it;
+    const int n = unit / p.Hv;
+    int64_t t0, t1;
+    if (!seq_range(p.cu, n, p.N, p.T, nullptr, t0, t1)) {  // the chain reports it
+        skip = true;
         return it;
+    }
+    const int64_t c0 = t0 + (int64_t)kC * c;
+    if (c0 >= t1) {  // a shorter sequence
+        skip = true;
+        return it;
+    }
+    it.c0 = c0;
+    it.unit = unit;
+    it.c = c;
+    it.h = unit % p.Hv;
+    it.j = it.h / (p.Hv / p.Hqk);
+    it.L = (int)((t1 - c0) < kC ? (t1 - c0) : kC);
+    it.valid = 1;
+    return it;
+}
+
+// The next chunk of the order that exists, from index `first` on (invalid once
+// the order is exhausted or the abort flag is up).  One thread calls it.
+__device__ Item pool_fetch(const ChainParams &p, uint32_t first) {
+    uint32_t i = first;
+    for (;;) {
+        bool skip;
+        const Item it = pool_item(p, i, skip);
+        if (!skip) return it;
+        if (ld_relaxed_gpu(p.flags + 1) != 0u) return Item{0, 0, 0, 0, 0, 0, 0};
+        i = atomicAdd(p.flags, 1u);
     }
 }
 
@@ -271,9 +293,16 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
     const uint32_t c_ready =
         kPool ? 0u : mapa_shared(sbase + C_MISC + (uint32_t)offsetof(ChainMisc, ready) + 8u * k, 0);
 
+    // pool: the counter index of the chunk after next, taken at the start of a
+    // chunk so that its L2 round trip is over by the time it is decoded
+    uint32_t pre_index = 0;
     auto fetch = [&](int l) -> Item {
         if constexpr (kPool) {
-            return pool_fetch(p);
+            if (l < 2) {
+                if (ld_relaxed_gpu(p.flags + 1) != 0u) return Item{0, 0, 0, 0, 0, 0, 0};
+                return pool_fetch(p, atomicAdd(p.flags, 1u));
+            }
+            return pool_fetch(p, pre_index);
         } else {
             Item it;
             const int c = k + 2 * l;
@@ -377,9 +406,9 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
 
     // Chunks l and l + 1 are known when chunk l starts (tile loads of chunks
     // 0 and 1 are issued here, those of chunk l + 1 > 1 during the U~ / W
-    // products of chunk l, after the stores of chunk l - 1 have landed); the
-    // delivery thread fetches chunk l + 2 before the vote of chunk l.
-    if (tid == 32) {
+    // products of chunk l, after the stores of chunk l - 1 have landed); chunk
+    // l + 2 is fetched during those products too.
+    if (tid == kFetchTid) {
         for (int l = 0; l < 2; ++l) {
             const Item it = fetch(l);
             ms->items[l] = it;
@@ -410,6 +439,15 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
         if (warp == 0) {
             const Item nx = ms->items[(l + 1) & 3];
             if (nx.valid) load_gates(nx);
+        }
+        // pool: the index of chunk l + 2 and an early look at this chunk's ring
+        // slot, both consumed at the end of the chunk
+        uint32_t early_taken = 0;
+        if constexpr (kPool) {
+            if (tid == kFetchTid) {
+                pre_index = atomicAdd(p.flags, 1u);
+                if (it.c >= p.ring_slots) early_taken = ld_relaxed_gpu(unit_flags(p, it.unit));
+            }
         }
         GDN_CL_PHASE(1, 0);  // gates
         GDN_CL_PHASE(1, 1);  // (no wait)
@@ -459,7 +497,7 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
         tc_fence_after_sync();
         // A / P, the solve and the W^T staging rewrite what the previous chunk's
         // first store group (W^T, P, gates) reads: wait until it has been read.
-        if (tid == 32) bulk_wait_read_all_but_one();
+        if (tid == kDeliverTid) bulk_wait_read_all_but_one();
         __syncthreads();
 #pragma unroll
         for (int q = 0; q < 1024 / kThreads; ++q) {
@@ -510,7 +548,7 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
         // The T tiles below overwrite the previous chunk's U~ staging: its
         // stores must have read it (long done by now; the solve's first
         // barrier orders this before every thread's writes).
-        if (tid == 32) bulk_wait_read_all();
+        if (tid == kDeliverTid) bulk_wait_read_all();
 
         // ---- T = (I + A)^-1 ----
         solve_tril64(As, Ts, Xs, tid);
@@ -558,10 +596,26 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
             mma_commit(&ms->mma_bar);
         }
         if (warp == 0 && ms->items[(l + 1) & 3].valid) compute_gates(ms->gt[(l + 1) & 1]);
-        if (tid == 32) {  // idle during these products: report the previous chunk
-            flush_delivery();  // ready once its stores have landed, refill its buffer
+        // side duties while these products run
+        if (tid == kDeliverTid) {  // report the previous chunk ready, refill its buffer
+            flush_delivery();
             const Item nx = ms->items[(l + 1) & 3];
             if (l >= 1 && nx.valid) issue_tma((l + 1) & 1, nx);
+        }
+        if (tid == kFetchTid) {
+            ms->items[(l + 2) & 3] = fetch(l + 2);  // decode chunk l + 2,
+            if constexpr (kPool) {  // and make sure this chunk's ring slot is free
+                const uint32_t need = (uint32_t)(it.c - p.ring_slots + 1);
+                // a free slot seen early needs no fence: the stores that refill it
+                // depend on that observation, and the chain publishes it only after
+                // its load of the slot has completed
+                if (it.c >= p.ring_slots && early_taken < need &&
+                    !wait_flag_geq(unit_flags(p, it.unit), need, p.flags + 1, kWaitLimit))
+                    timed_out = true;
+            } else {
+                if (l >= 1 && !mbar_wait_cluster_bounded(&ms->taken, (l - 1) & 1, kWaitLimit))
+                    timed_out = true;
+            }
         }
         if (!mbar_wait_bounded(&ms->mma_bar, mma_phase, kWaitLimit)) timed_out = true;
         mma_phase ^= 1;
@@ -612,19 +666,7 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
         fence_proxy_async_smem();  // staged data -> visible to the bulk copies
         GDN_CL_PHASE(1, 9);  // staging
 
-        // ---- the ring slot must be free; then deliver with asynchronous stores ----
-        if (tid == 32) {
-            ms->items[(l + 2) & 3] = fetch(l + 2);
-            if constexpr (kPool) {
-                if (it.c >= p.ring_slots &&
-                    !wait_flag_geq(unit_flags(p, it.unit), (uint32_t)(it.c - p.ring_slots + 1),
-                                   p.flags + 1, kWaitLimit))
-                    timed_out = true;
-            } else {
-                if (l >= 1 && !mbar_wait_cluster_bounded(&ms->taken, (l - 1) & 1, kWaitLimit))
-                    timed_out = true;
-            }
-        }
+        // ---- deliver with asynchronous stores (the ring slot is free: see above) ----
         if (__syncthreads_or(timed_out ? 1 : 0)) {
             if (tid == 0) {
                 raise_error(p.err, GDN_ERR_TIMEOUT);
@@ -634,7 +676,7 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
             break;
         }
         GDN_CL_PHASE(1, 10);  // wait: ring slot free
-        if (tid == 32) {
+        if (tid == kDeliverTid) {
             uint8_t *dst = ring_slot(p, it.unit, it.c);
             fence_proxy_async_global();  // the chain's reads of this slot precede our writes
             // group 1: what the next chunk rewrites first (read before its A / P)
@@ -652,7 +694,7 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
         }
         GDN_CL_PHASE(1, 11);  // deliver (issue)
     }
-    if (tid == 32) flush_delivery();  // the last chunk delivered
+    if (tid == kDeliverTid) flush_delivery();  // the last chunk delivered
     GDN_CL_PHASE_END(1);
     // A tile load issued for a chunk this loop never reached must land before
     // this CTA's shared memory can go away (chunk l + 1's, after a timeout;
@@ -788,15 +830,29 @@ __device__ void chain_role(uint8_t *sm, const ChainParams &p, int unit, int n, i
             read_flag(cur + 2);
         }
     };
+    // Chunk cc's output from its staging area (the consumed Q^T region of its
+    // shared slot) to global memory, 16 bytes per thread and store.
+    auto store_o = [&](int cc) {
+        const int64_t cc0 = t_begin + (int64_t)kC * cc;
+        const int cL = (int)((t_end - cc0) < kC ? (t_end - cc0) : kC);
+        const uint4 *ost = reinterpret_cast<const uint4 *>(sm + (cc & 1) * SLOT_BYTES + SL_OST);
+#pragma unroll
+        for (int q = 0; q < (kC * kD * 2 / 16) / kThreads; ++q) {
+            const int x = tid + q * kThreads;
+            const int r = x >> 4, c16 = x & 15;
+            if (r < cL) {
+                uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.o) +
+                                                       ((cc0 + r) * p.Hv + h) * (int64_t)kD) + c16;
+                *dst = ost[x];
+            }
+        }
+    };
     int c = 0;
 #pragma unroll 1
     for (; c < nch && !aborted; ++c) {
         const int k = c & 1;
         uint8_t *slot = sm + k * SLOT_BYTES;
         const uint32_t sslot = sbase + k * SLOT_BYTES;
-        const int64_t c0 = t_begin + (int64_t)kC * c;
-        const int L = (int)((t_end - c0) < kC ? (t_end - c0) : kC);
-
         bool have = true;
         if (tid == 0 && loaded == c) {  // not prefetched: wait for the producer, then load
             if (ready_wait(c)) {
@@ -810,7 +866,6 @@ __device__ void chain_role(uint8_t *sm, const ChainParams &p, int unit, int n, i
                 mbar_arrive(&ms->full[k]);
             }
         }
-        poll_next(c);  // chunk c + 1 may be ready already: load it while c computes
         if (!mbar_wait_bounded(&ms->full[k], (c >> 1) & 1, kWaitLimit)) timed_out = true;
         GDN_CL_PHASE(0, 0);  // wait: delivery
         if (tid == 0 && have) {  // the chunk is out of the ring: its slot may be refilled
@@ -839,7 +894,10 @@ __device__ void chain_role(uint8_t *sm, const ChainParams &p, int unit, int n, i
             }
             mma_commit(&ms->mma_bar);
         }
-        poll_next(c);
+        // the previous chunk's output, staged in its shared slot, goes out while
+        // these products run; its slot may be refilled after the next barrier
+        if (c > 0) store_o(c - 1);
+        fence_proxy_async_smem();
         GDN_CL_PHASE(0, 1);  // issue S Q^T, R
         if (!mbar_wait_bounded(&ms->mma_bar, mma_phase, kWaitLimit)) timed_out = true;
         mma_phase ^= 1;
@@ -906,7 +964,8 @@ __device__ void chain_role(uint8_t *sm, const ChainParams &p, int unit, int n, i
         mma_sync_point();
         GDN_CL_PHASE(0, 4);  // state update + P MMAs
 
-        // ---- o -> staging -> global; S' = Gamma_C S + dS, its fp16 hi/lo TMEM operands ----
+        // ---- o -> staging (stored during the next chunk); S' = Gamma_C S + dS and its
+        //      fp16 hi/lo TMEM operands ----
         {
             const int c32 = 32 * half;
             float v[32];
@@ -936,22 +995,8 @@ __device__ void chain_role(uint8_t *sm, const ChainParams &p, int unit, int n, i
             tmem_st32u(trow + CT_SH + 32 * half, hi);
             tmem_st32u(trow + CT_SL + 32 * half, lo);
         }
-        __syncthreads();
-        {
-            const uint4 *ost = reinterpret_cast<const uint4 *>(slot + SL_OST);
-#pragma unroll
-            for (int q = 0; q < (kC * kD * 2 / 16) / kThreads; ++q) {
-                const int x = tid + q * kThreads;
-                const int r = x >> 4, c16 = x & 15;
-                if (r < L) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.o) +
-                                                           ((c0 + r) * p.Hv + h) * (int64_t)kD) + c16;
-                    *dst = ost[x];
-                }
-            }
-        }
         poll_next(c);
-        GDN_CL_PHASE(0, 5);  // o staging + stores, S copies
+        GDN_CL_PHASE(0, 5);  // o staging, S copies
         fence_proxy_async_smem();  // our writes to the slot precede the next bulk load into it
         tmem_wait_st();
         tc_fence_before_sync();
@@ -978,6 +1023,7 @@ __device__ void chain_role(uint8_t *sm, const ChainParams &p, int unit, int n, i
                 *reinterpret_cast<float4 *>(dst + cc + x) = make_float4(v[x], v[x + 1], v[x + 2], v[x + 3]);
         }
     }
+    if (!aborted && nch > 0) store_o(nch - 1);  // the last chunk's output
     GDN_CL_PHASE_END(0);
     if (aborted) {
         // A prefetch still landing in shared memory must finish (c is one past
