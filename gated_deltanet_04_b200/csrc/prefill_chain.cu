@@ -101,6 +101,9 @@ constexpr int kCluster = 3;
 // refills; the chunk counter and the ring-slot check
 constexpr int kDeliverTid = 64;
 constexpr int kFetchTid = 96;
+constexpr int kRefillTid = 128;
+constexpr int kSlotTid = 192;
+constexpr int kGatesWarp = 5;  // loads g, beta and computes the next chunk's gates
 constexpr int kClusterRingSlots = 4;
 constexpr int kPoolRingSlots = 8;
 
@@ -124,7 +127,8 @@ struct GatesBlock {
     float Gam[kC];   // exp(gamma_r)
     float eC[kC];    // exp(gamma_C - gamma_r)
     int32_t hp;      // extra precision passes for this chunk
-    int32_t pad[3];
+    int32_t qs;      // Q^T arrives scaled by Gamma (so the chain need not scale O)
+    int32_t pad[2];
 };
 static_assert(sizeof(GatesBlock) % 16 == 0, "bulk copies move multiples of 16 bytes");
 
@@ -175,7 +179,7 @@ struct Item {
 // next chunk's are computed while this chunk's U~ / W products run).
 struct ProdGates {
     float gam[kC], Gam[kC], iGam[kC], eC[kC], bb[kC], bG[kC];
-    int32_t safe, hp, pad[2];
+    int32_t safe, hp, qs, pad;
 };
 
 struct ProdMisc {
@@ -319,7 +323,7 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
 
     uint32_t mma_phase = 0;
     bool timed_out = false;
-    float gpre0 = 0.f, gpre1 = 0.f, bpre0 = 0.f, bpre1 = 0.f;  // warp 0: the next chunk's g, beta
+    float gpre0 = 0.f, gpre1 = 0.f, bpre0 = 0.f, bpre1 = 0.f;  // gates warp: next chunk's g, beta
     auto load_gates = [&](const Item &it) {
         gpre0 = gpre1 = bpre0 = bpre1 = 0.f;
         const int64_t t0_ = it.c0 + 2 * lane, t1_ = t0_ + 1, te = it.c0 + it.L;
@@ -367,7 +371,7 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
         pending.valid = 0;
     };
 
-    // Gates of a chunk from the g, beta values in gpre / bpre (warp 0, two
+    // Gates of a chunk from the g, beta values in gpre / bpre (the gates warp, two
     // tokens per lane): cumulative log-decay gamma, Gamma = exp(gamma), the
     // factors of A, P, W and U', and the precision choice.
     auto compute_gates = [&](ProdGates &gt) {
@@ -379,9 +383,12 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
         }
         const float x0 = x1 - gpre1;
         const float gC = __shfl_sync(0xffffffffu, x1, 31);
-        float m = fmaxf(fabsf(x0), fabsf(x1));
+        float m = fmaxf(fabsf(x0), fabsf(x1)), top = fmaxf(x0, x1);
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+        for (int off = 16; off > 0; off >>= 1) {
+            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+            top = fmaxf(top, __shfl_xor_sync(0xffffffffu, top, off));
+        }
         const bool safe_ = m <= 60.f;  // every exp(+-gamma) a normal float
         const float G0 = expf(x0), G1 = expf(x1);
         const float GC = __shfl_sync(0xffffffffu, G1, 31);
@@ -401,6 +408,8 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
         if (lane == 0) {
             gt.safe = safe_;
             gt.hp = GC >= kHighPrecisionDecay;
+            // Q^T is scaled by Gamma <= 1 only: Gamma q then cannot overflow fp16
+            gt.qs = safe_ && top <= 0.f;
         }
     };
 
@@ -416,7 +425,7 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
         }
     }
     __syncthreads();
-    if (warp == 0 && ms->items[0].valid) {
+    if (warp == kGatesWarp && ms->items[0].valid) {
         load_gates(ms->items[0]);
         compute_gates(ms->gt[0]);
     }
@@ -436,7 +445,7 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
         const ProdGates &gt = ms->gt[l & 1];
 
         // the next chunk's g, beta: in flight until its gates are computed
-        if (warp == 0) {
+        if (warp == kGatesWarp) {
             const Item nx = ms->items[(l + 1) & 3];
             if (nx.valid) load_gates(nx);
         }
@@ -444,10 +453,9 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
         // slot, both consumed at the end of the chunk
         uint32_t early_taken = 0;
         if constexpr (kPool) {
-            if (tid == kFetchTid) {
-                pre_index = atomicAdd(p.flags, 1u);
-                if (it.c >= p.ring_slots) early_taken = ld_relaxed_gpu(unit_flags(p, it.unit));
-            }
+            if (tid == kFetchTid) pre_index = atomicAdd(p.flags, 1u);
+            if (tid == kSlotTid && it.c >= p.ring_slots)
+                early_taken = ld_relaxed_gpu(unit_flags(p, it.unit));
         }
         GDN_CL_PHASE(1, 0);  // gates
         GDN_CL_PHASE(1, 1);  // (no wait)
@@ -595,16 +603,16 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
                 }
             mma_commit(&ms->mma_bar);
         }
-        if (warp == 0 && ms->items[(l + 1) & 3].valid) compute_gates(ms->gt[(l + 1) & 1]);
+        if (warp == kGatesWarp && ms->items[(l + 1) & 3].valid) compute_gates(ms->gt[(l + 1) & 1]);
         // side duties while these products run
-        if (tid == kDeliverTid) {  // report the previous chunk ready, refill its buffer
-            flush_delivery();
+        if (tid == kDeliverTid) flush_delivery();  // report the previous chunk ready
+        if (tid == kRefillTid) {  // refill its tile buffer (its stores have read it)
             const Item nx = ms->items[(l + 1) & 3];
             if (l >= 1 && nx.valid) issue_tma((l + 1) & 1, nx);
         }
-        if (tid == kFetchTid) {
-            ms->items[(l + 2) & 3] = fetch(l + 2);  // decode chunk l + 2,
-            if constexpr (kPool) {  // and make sure this chunk's ring slot is free
+        if (tid == kFetchTid) ms->items[(l + 2) & 3] = fetch(l + 2);  // decode chunk l + 2
+        if (tid == kSlotTid) {  // make sure this chunk's ring slot is free
+            if constexpr (kPool) {
                 const uint32_t need = (uint32_t)(it.c - p.ring_slots + 1);
                 // a free slot seen early needs no fence: the stores that refill it
                 // depend on that observation, and the chain publishes it only after
@@ -639,25 +647,34 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
                 ms->gst.Gam[tid] = gt.Gam[tid];
                 ms->gst.eC[tid] = gt.eC[tid];
             }
-            if (tid == 0) ms->gst.hp = hp;
+            if (tid == 0) {
+                ms->gst.hp = hp;
+                ms->gst.qs = gt.qs;
+            }
         }
         {   // Q^T fp16 (MN-major: row d holds 64 tokens) from the bf16 Q tile into
-            // the V half of the tile buffer, which the U~ product has finished reading
+            // the V half of the tile buffer, which the U~ product has finished
+            // reading; scaled by Gamma when the gates allow (qs)
             const int d = tid & 127, tq = (tid >> 7) * 32;
             const uint8_t *qsrc = kqv + (d >> 6) * 16384 + 8192;
             const uint32_t dbyte = (uint32_t)(d & 63) * 2u;
+            const bool qs = gt.qs;
 #pragma unroll
             for (int g8 = 0; g8 < 4; ++g8) {
                 uint32_t w[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const uint32_t t = (uint32_t)(tq + 8 * g8 + 2 * e);
-                    const float a = (int)t < L
+                    float a = (int)t < L
                         ? __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(qsrc + sw128(t, dbyte)))
                         : 0.f;
-                    const float b = (int)t + 1 < L
+                    float b = (int)t + 1 < L
                         ? __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(qsrc + sw128(t + 1, dbyte)))
                         : 0.f;
+                    if (qs) {
+                        a *= gt.Gam[t];
+                        b *= gt.Gam[t + 1];
+                    }
                     w[e] = pack_half2(a, b);
                 }
                 st_row_chunk(kqv + 32768, d, (tq >> 3) + g8, make_uint4(w[0], w[1], w[2], w[3]));
@@ -830,17 +847,26 @@ __device__ void chain_role(uint8_t *sm, const ChainParams &p, int unit, int n, i
             read_flag(cur + 2);
         }
     };
+    // Only starts reading chunk cur + 1's flag (no fence, no load): where thread
+    // 0 is about to issue MMAs and must not stall.
+    auto poll_read = [&](int cur) {
+        if (tid == 0 && loaded == cur + 1 && cur + 1 < nch) read_flag(cur + 1);
+    };
     // Chunk cc's output from its staging area (the consumed Q^T region of its
-    // shared slot) to global memory, 16 bytes per thread and store.
+    // shared slot) to global memory, 16 bytes per store.  Warp 0 takes no part:
+    // thread 0 fences before its ring loads, and a fence waits for the issuing
+    // thread's own outstanding stores.
     auto store_o = [&](int cc) {
+        if (warp == 0) return;
         const int64_t cc0 = t_begin + (int64_t)kC * cc;
         const int cL = (int)((t_end - cc0) < kC ? (t_end - cc0) : kC);
         const uint4 *ost = reinterpret_cast<const uint4 *>(sm + (cc & 1) * SLOT_BYTES + SL_OST);
+        constexpr int kStorers = kThreads - 32;
 #pragma unroll
-        for (int q = 0; q < (kC * kD * 2 / 16) / kThreads; ++q) {
-            const int x = tid + q * kThreads;
+        for (int q = 0; q < (kC * kD * 2 / 16 + kStorers - 1) / kStorers; ++q) {
+            const int x = (tid - 32) + q * kStorers;
             const int r = x >> 4, c16 = x & 15;
-            if (r < cL) {
+            if (x < kC * kD * 2 / 16 && r < cL) {
                 uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.o) +
                                                        ((cc0 + r) * p.Hv + h) * (int64_t)kD) + c16;
                 *dst = ost[x];
@@ -904,11 +930,12 @@ __device__ void chain_role(uint8_t *sm, const ChainParams &p, int unit, int n, i
         tc_fence_after_sync();
         GDN_CL_PHASE(0, 2);  // wait: S Q^T, R
 
-        // ---- O *= Gamma (rows of the transposed output); U = U~ - R; U', U -> TMEM ----
+        // ---- O *= Gamma unless Q^T came scaled; U = U~ - R; U', U -> TMEM ----
         {
             const int c32 = 32 * half;
             float v[32], r0[32];
-            tmem_ld32(trow + CT_O + c32, v);
+            const bool qs = gb->qs != 0;
+            if (!qs) tmem_ld32(trow + CT_O + c32, v);
             tmem_ld32(trow + CT_R + c32, r0);
             tmem_wait_ld();
             if (hp) {
@@ -918,9 +945,11 @@ __device__ void chain_role(uint8_t *sm, const ChainParams &p, int unit, int n, i
 #pragma unroll
                 for (int x = 0; x < 32; ++x) r0[x] += r2[x];
             }
+            if (!qs) {  // O = diag(Gamma) Q S^T, unless Q^T came scaled
 #pragma unroll
-            for (int x = 0; x < 32; ++x) v[x] *= gb->Gam[c32 + x];
-            tmem_st32(trow + CT_O + c32, v);
+                for (int x = 0; x < 32; ++x) v[x] *= gb->Gam[c32 + x];
+                tmem_st32(trow + CT_O + c32, v);
+            }
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
                 const float4 f = *reinterpret_cast<const float4 *>(slot + SL_UT + ut_off(row, c32 / 4 + q));
@@ -945,7 +974,7 @@ __device__ void chain_role(uint8_t *sm, const ChainParams &p, int unit, int n, i
         tc_fence_before_sync();
         __syncthreads();
         tc_fence_after_sync();
-        poll_next(c);
+        poll_read(c);  // the load itself is issued under the next products
         GDN_CL_PHASE(0, 3);  // O scale, U, U'
 
         // ---- dS = [U'hi | U'lo] [K ; K];  O += U^T P^T  (A operands from TMEM) ----
