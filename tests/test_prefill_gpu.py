@@ -261,3 +261,49 @@ def test_long256k_sampled_heads(kernel):
     o_ref, s_ref = run_oracle(sub)
     check_o(o[:, heads].cpu(), o_ref, "o, sampled heads")
     check_state(sT[:, heads].cpu(), s_ref, "state, sampled heads")
+
+
+@pytest.mark.parametrize("kernel", ["pool", "single_cta"])
+def test_weak_decay_long_sequence(kernel):
+    """8192 tokens with a = 0.999 per token: every chunk has Gamma_C >= 0.2, so
+    the extra-precision passes run everywhere, and the state's rounding errors
+    accumulate over 128 chunks instead of decaying away."""
+    T, Hqk, Hv = 8192, 1, 4
+    inp, s0 = synth(T, Hqk, Hv, 128, torch.bfloat16, seed=2301, s0_std=0.05)
+    inp["g"].fill_(float(np.log(0.999)))
+    o, sT = run_gpu(inp, s0, kernel=kernel)
+    o_ref, s_ref = run_oracle(inp, s0)
+    check_o(o, o_ref)
+    check_state(sT, s_ref)
+
+
+def test_pool_kernel_at_its_unit_limit():
+    """64 units (4 sequences x 16 v-heads), the most the pool kernel takes,
+    against the oracle; the single-CTA kernel must agree."""
+    lengths = [300, 64, 0, 517]
+    cu = inputs.cu_from_lengths(lengths)
+    inp, s0 = synth(int(cu[-1]), 4, 16, 128, torch.bfloat16, seed=2302, s0_std=0.05,
+                    N=len(lengths))
+    o, sT = run_gpu(inp, s0, cu, kernel="pool")
+    o_ref, s_ref = run_oracle(inp, s0, cu)
+    check_o(o, o_ref)
+    check_state(sT, s_ref)
+    o2, s2 = run_gpu(inp, s0, cu, kernel="single_cta")
+    check_o(o2, o.double())
+    check_state(s2, sT.double())
+
+
+def test_auto_past_the_pool_limit():
+    """65 units: AUTO takes the single-CTA kernel (the pool kernel refuses),
+    and its result still matches the oracle."""
+    lengths = [70] * 65
+    cu = inputs.cu_from_lengths(lengths)
+    inp, s0 = synth(int(cu[-1]), 1, 1, 128, torch.bfloat16, seed=2303, s0_std=0.05,
+                    N=len(lengths))
+    with pytest.raises(gdn.GdnError, match="UNSUPPORTED"):
+        run_gpu(inp, s0, cu, kernel="pool")
+    assert gdn.gdn_prefill_workspace_bytes(65, int(cu[-1]), 1, 1, 128, 128, 64) == 0
+    o, sT = run_gpu(inp, s0, cu)
+    o_ref, s_ref = run_oracle(inp, s0, cu)
+    check_o(o, o_ref)
+    check_state(sT, s_ref)
