@@ -51,17 +51,28 @@
 #include "tc_common.cuh"
 
 #ifdef GDN_TC_PHASES
-__device__ long long gdn_tc_phase_clk[16];
+// Per-phase SM clocks of thread 0 of CTA 0, accumulated in shared memory (a
+// global read-modify-write per marker would stall thread 0 and distort the
+// phases) and added to the global totals once, at the end.
+__device__ unsigned long long gdn_tc_phase_clk[16];
+static __shared__ unsigned int gdn_tc_acc_[16];
 #define GDN_TC_PHASE(k)                                             \
     do {                                                            \
         if (threadIdx.x == 0 && blockIdx.x == 0) {                  \
             const long long now_ = clock64();                       \
-            gdn_tc_phase_clk[(k)] += now_ - phase_t_;               \
+            gdn_tc_acc_[(k)] += (unsigned int)(now_ - phase_t_);    \
             phase_t_ = now_;                                        \
         }                                                           \
     } while (0)
+#define GDN_TC_PHASE_FLUSH()                                        \
+    do {                                                            \
+        if (threadIdx.x == 0 && blockIdx.x == 0)                    \
+            for (int i_ = 0; i_ < 16; ++i_)                         \
+                atomicAdd(&gdn_tc_phase_clk[i_], (unsigned long long)gdn_tc_acc_[i_]); \
+    } while (0)
 #else
 #define GDN_TC_PHASE(k) ((void)0)
+#define GDN_TC_PHASE_FLUSH() ((void)0)
 #endif
 
 namespace gdn {
@@ -84,8 +95,8 @@ constexpr uint32_t OFF_X = 114688;
 constexpr uint32_t OFF_UP = OFF_X;            // hi, lo x 128 rows x 128 B  (A: U')
 constexpr uint32_t OFF_U16 = OFF_X + 32768;   // 128 rows x 128 B           (A: U^T)
 constexpr uint32_t OFF_WST = OFF_X;           // hi, lo x 128 rows(d) x 128 B (B: W^T, MN-major)
-constexpr uint32_t OFF_AS = OFF_X;                   // float [64][kAS]
-constexpr uint32_t OFF_TS = OFF_X + 64 * kAS * 4;       // float [64][kTS], 16-byte aligned
+constexpr uint32_t OFF_AS = OFF_X;                   // float [64][kAS4]
+constexpr uint32_t OFF_TS = OFF_X + 64 * kAS4 * 4;      // float [64][kTS], 16-byte aligned
 constexpr uint32_t OFF_XS = OFF_TS + 64 * kTS * 4;   // float [1024] level partials
 constexpr uint32_t OFF_P16 = 163840;    // 64 rows x 128 B                  (B: P, K-major)
 constexpr uint32_t OFF_TBH = 172032;    // 64 rows x 128 B                  (B: T diag b, hi)
@@ -152,6 +163,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = quad * 32 + lane;   // TMEM lane = accumulator row
 #ifdef GDN_TC_PHASES
     long long phase_t_ = clock64();
+    if (threadIdx.x == 0)
+        for (int i_ = 0; i_ < 16; ++i_) gdn_tc_acc_[i_] = 0u;
 #endif
 
     const int unit = blockIdx.x;  // n * Hv + h
@@ -273,34 +286,49 @@ __global__ void __launch_bounds__(kThreads, 1)
             float m = fmaxf(fabsf(x0), fabsf(x1));
 #pragma unroll
             for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-            const bool safe_ = m <= 60.f;
+            const bool safe_ = m <= 60.f;  // every exp(+-gamma) a normal float
             const float G0 = expf(x0), G1 = expf(x1);
+            const float GC = __shfl_sync(0xffffffffu, G1, 31);
             const int r0 = 2 * lane;
             ms->gam[r0] = x0;                ms->gam[r0 + 1] = x1;
             ms->Gam[r0] = G0;                ms->Gam[r0 + 1] = G1;
-            ms->iGam[r0] = safe_ ? expf(-x0) : 0.f;
-            ms->iGam[r0 + 1] = safe_ ? expf(-x1) : 0.f;
-            ms->eC[r0] = expf(gC - x0);      ms->eC[r0 + 1] = expf(gC - x1);
+            if (safe_) {  // 1 / Gamma and Gamma_C / Gamma from the exponentials above
+                const float i0 = 1.f / G0, i1 = 1.f / G1;
+                ms->iGam[r0] = i0;           ms->iGam[r0 + 1] = i1;
+                ms->eC[r0] = GC * i0;        ms->eC[r0 + 1] = GC * i1;
+            } else {
+                ms->iGam[r0] = 0.f;          ms->iGam[r0 + 1] = 0.f;
+                ms->eC[r0] = expf(gC - x0);  ms->eC[r0 + 1] = expf(gC - x1);
+            }
             ms->bb[r0] = bpre0;              ms->bb[r0 + 1] = bpre1;
             ms->bG[r0] = bpre0 * G0;         ms->bG[r0 + 1] = bpre1 * G1;
             if (lane == 0) {
                 ms->safe = safe_;
-                ms->hp = expf(gC) >= kHighPrecisionDecay;
+                ms->hp = GC >= kHighPrecisionDecay;
             }
             if (has_next) load_gates(c0 + kC);  // prefetch the next chunk's gates
         }
         GDN_TC_PHASE(1);
 
-        // ---- wait for the tiles, convert bf16 -> fp16 in place, zero padding rows ----
+        // ---- wait for the tiles; Gram [K;Q] K^T -> TM_G straight from the bf16 tiles
+        //      (exact products either way), bf16 -> fp16 in place meanwhile ----
         if (!mbar_wait_bounded(&ms->tma_bar, tma_phase, kWaitLimit)) timed_out = true;
         tma_phase ^= 1;
         tma_outstanding = false;
         GDN_TC_PHASE(2);
-        // 48 KB = 3072 chunks of 16 bytes; row = token index (offset / 128 within each 8 KB box)
+        if (tid == 0) {
 #pragma unroll
-        for (int k = 0; k < 3072 / kThreads; ++k) {
-            const int x = tid + k * kThreads;
-            uint4 *ptr = reinterpret_cast<uint4 *>(sm + OFF_KQ) + x;  // KQ and V are contiguous
+            for (int ks = 0; ks < 8; ++ks) {
+                const uint32_t a = sbase + OFF_KQ + (ks >> 2) * 16384 + (ks & 3) * 32;
+                mma_f16_ss(tmem + TM_G, make_sdesc(a, 16, 1024), make_sdesc(a, 16, 1024),
+                           IDESC_KK_N64_BF16, ks > 0);
+            }
+            mma_commit(&ms->mma_bar);
+        }
+        // 16-byte chunk x of the tile region starting at `base`; row = token
+        // (offset / 128 within each 8 KB box); padding rows become zeros
+        auto convert16 = [&](uint8_t *base, int x) {
+            uint4 *ptr = reinterpret_cast<uint4 *>(base) + x;
             const int r = (x >> 3) & 63;
             uint4 val = *ptr;
             if (r >= L) {
@@ -316,22 +344,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                 val = make_uint4(w[0], w[1], w[2], w[3]);
             }
             *ptr = val;
-        }
-        publish();
+        };
+#pragma unroll
+        for (int k = 0; k < 1024 / kThreads; ++k) convert16(sm + OFF_V, tid + k * kThreads);  // V
+        if (!mbar_wait_bounded(&ms->mma_bar, mma_phase, kWaitLimit)) timed_out = true;
+        mma_phase ^= 1;
+        tc_fence_after_sync();
+#pragma unroll
+        for (int k = 0; k < 2048 / kThreads; ++k) convert16(sm + OFF_KQ, tid + k * kThreads);  // K, Q
         const bool hp = ms->hp;
         const bool safe = ms->safe;
         GDN_TC_PHASE(3);
-
-        // ---- Gram: [K;Q] K^T -> TM_G ----
-        if (tid == 0) {
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-                const uint32_t a = sbase + OFF_KQ + (ks >> 2) * 16384 + (ks & 3) * 32;
-                mma_f16_ss(tmem + TM_G, make_sdesc(a, 16, 1024), make_sdesc(a, 16, 1024),
-                           IDESC_KK_N64, ks > 0);
-            }
-        }
-        mma_sync_point();
         GDN_TC_PHASE(4);
 
         // ---- A (lanes 0..63) and P (lanes 64..127) from the Gram rows ----
@@ -354,9 +377,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int x = 0; x < 32; ++x) v[x] *= sr * expf(gr - ms->gam[c + x]);
             }
-            if (row < kC) {  // A = strictly lower part
+            if (row < kC) {  // A = strictly lower part (16-byte stores: conflict-free at stride kAS4)
 #pragma unroll
-                for (int x = 0; x < 32; ++x) As[r * kAS + c + x] = (c + x < r) ? v[x] : 0.f;
+                for (int x = 0; x < 32; x += 4)
+                    *reinterpret_cast<float4 *>(As + r * kAS4 + c + x) =
+                        make_float4((c + x < r) ? v[x] : 0.f, (c + x + 1 < r) ? v[x + 1] : 0.f,
+                                    (c + x + 2 < r) ? v[x + 2] : 0.f, (c + x + 3 < r) ? v[x + 3] : 0.f);
             } else {         // P = lower part including the diagonal
 #pragma unroll
                 for (int x = 0; x < 32; ++x) v[x] = (c + x <= r) ? v[x] : 0.f;
@@ -367,33 +393,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncthreads();
         GDN_TC_PHASE(5);
 
-        // ---- T = (I + A)^-1 by 16 x 16 blocks (fp32, CUDA cores) ----
-        // Diagonal blocks D_i = (I + A_ii)^-1 by forward substitution, one thread per
-        // (block, column); then, by block distance d = 1..3,
-        //   X = sum_{m = k}^{i-1} A_im T_mk,   T_ik = -D_i X,   i = k + d,
-        // each thread producing four adjacent columns of one row.
-        if (tid < kC) {
-            const int bi = tid >> 4, col = tid & 15;
-            const float *Ab = As + (16 * bi) * kAS + 16 * bi;
-            float x[16];
-#pragma unroll
-            for (int rr = 0; rr < 16; ++rr) {
-                float a0 = (rr == col) ? 1.f : 0.f, a1 = 0.f;
-#pragma unroll
-                for (int ii = 0; ii + 1 < rr; ii += 2) {
-                    a0 -= Ab[rr * kAS + ii] * x[ii];
-                    a1 -= Ab[rr * kAS + ii + 1] * x[ii + 1];
-                }
-                if (rr & 1) a0 -= Ab[rr * kAS + rr - 1] * x[rr - 1];
-                x[rr] = a0 + a1;
-            }
-#pragma unroll
-            for (int rr = 0; rr < 16; ++rr) Ts[(16 * bi + rr) * kTS + 16 * bi + col] = x[rr];
-        }
-        __syncthreads();
-        solve_level<1>(As, Ts, Xs, tid);
-        solve_level<2>(As, Ts, Xs, tid);
-        solve_level<3>(As, Ts, Xs, tid);
+        // ---- T = (I + A)^-1 (fp32, CUDA cores) ----
+        solve_tril64(As, Ts, Xs, tid);
         GDN_TC_PHASE(6);
 
         // ---- B operands: rows r of T diag(b) and T diag(b Gamma), fp16 hi / lo ----
@@ -597,6 +598,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_before_sync();
     __syncthreads();
     tc_fence_after_sync();
+    GDN_TC_PHASE_FLUSH();
     if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
@@ -665,11 +667,11 @@ cudaError_t launch_prefill_tc(const PrefillArgs &a, cudaStream_t s) {
 
 #ifdef GDN_TC_PHASES
 extern "C" GDN_API int gdn_debug_tc_phases(long long *out, int n, int reset) {
-    long long host[16];
+    unsigned long long host[16];
     if (cudaMemcpyFromSymbol(host, gdn_tc_phase_clk, sizeof(host)) != cudaSuccess) return -1;
-    for (int i = 0; i < n && i < 16; ++i) out[i] = host[i];
+    for (int i = 0; i < n && i < 16; ++i) out[i] = (long long)host[i];
     if (reset) {
-        const long long zero[16] = {0};
+        const unsigned long long zero[16] = {0};
         cudaMemcpyToSymbol(gdn_tc_phase_clk, zero, sizeof(zero));
     }
     return 0;

@@ -18,7 +18,6 @@ constexpr int kC = 64;      // chunk length
 constexpr int kD = 128;     // Dk = Dv
 constexpr long long kWaitLimit = 1ll << 31;  // SM clocks (about a second)
 constexpr float kHighPrecisionDecay = 0.2f;  // Gamma_C at or above -> extra passes
-constexpr int kAS = 65;  // row stride of A (scalar, conflict-free column access)
 constexpr int kAS4 = 68; // row stride of A for solve_tril64 (16-byte aligned rows)
 constexpr int kTS = 68;  // row stride of T (16-byte aligned rows for float4 access)
 
@@ -69,45 +68,6 @@ __device__ __forceinline__ void store_split32(uint8_t *hi_tile, uint8_t *lo_tile
         st_row_chunk(hi_tile, row, (c + e) / 8, hi);
         if (with_lo) st_row_chunk(lo_tile, row, (c + e) / 8, lo);
     }
-}
-
-// One block-distance level D of the triangular inverse (see the solve phase):
-//   X = sum_{m = k}^{i-1} A_im T_mk,   T_ik = -D_i X,   i = k + D,
-// each thread producing four adjacent columns of one row of one block.
-template <int D>
-__device__ __forceinline__ void solve_level(const float *As, float *Ts, float *Xs, int tid) {
-    constexpr int kBlocks = 4 - D;
-    const bool act = tid < kBlocks * 64;
-    const int blk = tid >> 6, r = (tid >> 2) & 15, c4 = 4 * (tid & 3);
-    const int bi = blk + D, bk = blk;
-    if (act) {
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        const float *arow = As + (16 * bi + r) * kAS + 16 * bk;
-        const float *tcol = Ts + (16 * bk) * kTS + 16 * bk + c4;
-#pragma unroll
-        for (int m = 0; m < 16 * D; ++m) {
-            const float a = arow[m];
-            const float4 t = *reinterpret_cast<const float4 *>(tcol + m * kTS);
-            acc.x = fmaf(a, t.x, acc.x); acc.y = fmaf(a, t.y, acc.y);
-            acc.z = fmaf(a, t.z, acc.z); acc.w = fmaf(a, t.w, acc.w);
-        }
-        *reinterpret_cast<float4 *>(Xs + (blk << 8) + r * 16 + c4) = acc;
-    }
-    __syncthreads();
-    if (act) {
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        const float *drow = Ts + (16 * bi + r) * kTS + 16 * bi;
-#pragma unroll
-        for (int m = 0; m < 16; ++m) {
-            const float d = drow[m];
-            const float4 x = *reinterpret_cast<const float4 *>(Xs + (blk << 8) + m * 16 + c4);
-            acc.x = fmaf(d, x.x, acc.x); acc.y = fmaf(d, x.y, acc.y);
-            acc.z = fmaf(d, x.z, acc.z); acc.w = fmaf(d, x.w, acc.w);
-        }
-        *reinterpret_cast<float4 *>(Ts + (16 * bi + r) * kTS + 16 * bk + c4) =
-            make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
-    }
-    __syncthreads();
 }
 
 // T = (I + A)^-1 for the 64 x 64 strictly lower A in As (row stride kAS4),
