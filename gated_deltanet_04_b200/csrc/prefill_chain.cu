@@ -103,6 +103,9 @@ constexpr int kDeliverTid = 64;
 constexpr int kFetchTid = 96;
 constexpr int kRefillTid = 128;
 constexpr int kSlotTid = 192;
+// chain thread that polls the ring, loads it, signals taken chunks and stores
+// output tiles (thread 0 only issues MMAs, and never waits on L2)
+constexpr int kLoadTid = 32;
 constexpr int kGatesWarp = 5;  // loads g, beta and computes the next chunk's gates
 constexpr int kClusterRingSlots = 4;
 constexpr int kPoolRingSlots = 8;
@@ -555,8 +558,13 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
 
         // The T tiles below overwrite the previous chunk's U~ staging: its
         // stores must have read it (long done by now; the solve's first
-        // barrier orders this before every thread's writes).
-        if (tid == kDeliverTid) bulk_wait_read_all();
+        // barrier orders this before every thread's writes).  The same thread
+        // reports that chunk ready: step 1 of the solve keeps warps 0 and 1
+        // busy while the others, this one included, would wait.
+        if (tid == kDeliverTid) {
+            bulk_wait_read_all();
+            flush_delivery();
+        }
 
         // ---- T = (I + A)^-1 ----
         solve_tril64(As, Ts, Xs, tid);
@@ -605,7 +613,6 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
         }
         if (warp == kGatesWarp && ms->items[(l + 1) & 3].valid) compute_gates(ms->gt[(l + 1) & 1]);
         // side duties while these products run
-        if (tid == kDeliverTid) flush_delivery();  // report the previous chunk ready
         if (tid == kRefillTid) {  // refill its tile buffer (its stores have read it)
             const Item nx = ms->items[(l + 1) & 3];
             if (l >= 1 && nx.valid) issue_tma((l + 1) & 1, nx);
@@ -723,8 +730,8 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
 // ---------------------------------------------------------------- chain --
 
 template <bool kPool>
-__device__ void chain_role(uint8_t *sm, const ChainParams &p, int unit, int n, int h,
-                           int64_t t_begin, int64_t t_end, int nch) {
+__device__ void chain_role(uint8_t *sm, const CUtensorMap *tm_o, const ChainParams &p, int unit,
+                           int n, int h, int64_t t_begin, int64_t t_end, int nch) {
     ChainMisc *ms = reinterpret_cast<ChainMisc *>(sm + C_MISC);
     const uint32_t sbase = smem_u32(sm);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -781,7 +788,7 @@ __device__ void chain_role(uint8_t *sm, const ChainParams &p, int unit, int n, i
         __syncthreads();
         tc_fence_after_sync();
     };
-    // Has chunk cc reached the ring?  (thread 0)  The pool kernel reads the
+    // Has chunk cc reached the ring?  (load thread)  The pool kernel reads the
     // flag with a relaxed load whose value is only examined on a later call,
     // so the L2 round trip overlaps other work; an observed flag is turned
     // into an acquire by a fence.
@@ -818,11 +825,12 @@ __device__ void chain_role(uint8_t *sm, const ChainParams &p, int unit, int n, i
     const bool phase_on_ = blockIdx.x == 0;
 #endif
     GDN_CL_PHASE_BEGIN();
-    // Thread 0 loads chunk c + 1 from the ring into shared slot (c + 1) & 1 as
+    // The load thread loads chunk c + 1 from the ring into shared slot (c + 1) & 1 as
     // soon as it is reported ready, while chunk c is processed; the shared
     // slot held chunk c - 1, which is finished.
     int loaded = 0;  // chunks whose load has been issued
     auto issue_load = [&](int cc) {  // four copies, which the copy engine can overlap
+        bulk_wait_read_all();        // an output tile store from this shared slot has read it
         fence_proxy_async_global();  // the producer's stores, acquired, precede our bulk load
         uint64_t *bar = &ms->full[cc & 1];
         mbar_arrive_expect_tx(bar, SLOT_BYTES);
@@ -837,7 +845,7 @@ __device__ void chain_role(uint8_t *sm, const ChainParams &p, int unit, int n, i
     // Loads chunk cur + 1 once it is ready; when it is loaded already, starts
     // reading the flag of chunk cur + 2 (its slot frees up with chunk cur).
     auto poll_next = [&](int cur) {
-        if (tid != 0) return;
+        if (tid != kLoadTid) return;
         if (loaded == cur + 1 && cur + 1 < nch) {
             if (ready_try(cur + 1)) {
                 issue_load(cur + 1);
@@ -847,24 +855,34 @@ __device__ void chain_role(uint8_t *sm, const ChainParams &p, int unit, int n, i
             read_flag(cur + 2);
         }
     };
-    // Only starts reading chunk cur + 1's flag (no fence, no load): where thread
-    // 0 is about to issue MMAs and must not stall.
+    // Only starts reading chunk cur + 1's flag (no fence, no load).
     auto poll_read = [&](int cur) {
-        if (tid == 0 && loaded == cur + 1 && cur + 1 < nch) read_flag(cur + 1);
+        if (tid == kLoadTid && loaded == cur + 1 && cur + 1 < nch) read_flag(cur + 1);
     };
     // Chunk cc's output from its staging area (the consumed Q^T region of its
-    // shared slot) to global memory, 16 bytes per store.  Warp 0 takes no part:
-    // thread 0 fences before its ring loads, and a fence waits for the issuing
-    // thread's own outstanding stores.
+    // shared slot) to global memory: a full chunk as one tile store issued by
+    // the load thread (read back before the slot is reloaded, see issue_load);
+    // the last, partial chunk of a sequence with 16-byte stores of warps 2..7,
+    // so nothing past the sequence is written.  Warps 0 and 1 take no part in
+    // those: the load thread fences before its ring loads, and a fence waits
+    // for the issuing thread's own outstanding stores.
     auto store_o = [&](int cc) {
-        if (warp == 0) return;
         const int64_t cc0 = t_begin + (int64_t)kC * cc;
         const int cL = (int)((t_end - cc0) < kC ? (t_end - cc0) : kC);
-        const uint4 *ost = reinterpret_cast<const uint4 *>(sm + (cc & 1) * SLOT_BYTES + SL_OST);
-        constexpr int kStorers = kThreads - 32;
+        const uint8_t *ostb = sm + (cc & 1) * SLOT_BYTES + SL_OST;
+        if (cL == kC) {
+            if (tid == kLoadTid) {
+                tma_store_3d(tm_o, ostb, 0, h, (int32_t)cc0);
+                bulk_commit();
+            }
+            return;
+        }
+        if (warp <= 1) return;
+        const uint4 *ost = reinterpret_cast<const uint4 *>(ostb);
+        constexpr int kStorers = kThreads - 64;
 #pragma unroll
         for (int q = 0; q < (kC * kD * 2 / 16 + kStorers - 1) / kStorers; ++q) {
-            const int x = (tid - 32) + q * kStorers;
+            const int x = (tid - 64) + q * kStorers;
             const int r = x >> 4, c16 = x & 15;
             if (x < kC * kD * 2 / 16 && r < cL) {
                 uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.o) +
@@ -880,7 +898,7 @@ __device__ void chain_role(uint8_t *sm, const ChainParams &p, int unit, int n, i
         uint8_t *slot = sm + k * SLOT_BYTES;
         const uint32_t sslot = sbase + k * SLOT_BYTES;
         bool have = true;
-        if (tid == 0 && loaded == c) {  // not prefetched: wait for the producer, then load
+        if (tid == kLoadTid && loaded == c) {  // not prefetched: wait for the producer, then load
             if (ready_wait(c)) {
                 issue_load(c);
                 loaded = c + 1;
@@ -894,7 +912,7 @@ __device__ void chain_role(uint8_t *sm, const ChainParams &p, int unit, int n, i
         }
         if (!mbar_wait_bounded(&ms->full[k], (c >> 1) & 1, kWaitLimit)) timed_out = true;
         GDN_CL_PHASE(0, 0);  // wait: delivery
-        if (tid == 0 && have) {  // the chunk is out of the ring: its slot may be refilled
+        if (tid == kLoadTid && have) {  // the chunk is out of the ring: its slot may be refilled
             if constexpr (kPool)
                 st_relaxed_gpu(uflags, (uint32_t)(c + 1));
             else
@@ -1053,6 +1071,7 @@ __device__ void chain_role(uint8_t *sm, const ChainParams &p, int unit, int n, i
         }
     }
     if (!aborted && nch > 0) store_o(nch - 1);  // the last chunk's output
+    if (tid == kLoadTid) bulk_wait_all();  // every output tile store has landed
     GDN_CL_PHASE_END(0);
     if (aborted) {
         // A prefetch still landing in shared memory must finish (c is one past
@@ -1110,7 +1129,8 @@ __device__ __forceinline__ uint8_t *aligned_smem(uint8_t *raw) {
 __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
     gdn_prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
                                const __grid_constant__ CUtensorMap tm_k,
-                               const __grid_constant__ CUtensorMap tm_v, ChainParams p) {
+                               const __grid_constant__ CUtensorMap tm_v,
+                               const __grid_constant__ CUtensorMap tm_o, ChainParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = aligned_smem(smem_raw);
     const int rank = (int)cluster_ctarank();
@@ -1131,7 +1151,7 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
     tc_fence_after_sync();
 
     if (rank == 0)
-        chain_role<false>(sm, p, unit, n, h, t_begin, t_end, nch);
+        chain_role<false>(sm, &tm_o, p, unit, n, h, t_begin, t_end, nch);
     else
         producer_role<false>(sm, &tm_q, &tm_k, &tm_v, p, unit, rank - 1, h, j, t_begin, t_end, nch);
 
@@ -1145,7 +1165,8 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
 __global__ void __launch_bounds__(kThreads, 1)
     gdn_prefill_pool_kernel(const __grid_constant__ CUtensorMap tm_q,
                             const __grid_constant__ CUtensorMap tm_k,
-                            const __grid_constant__ CUtensorMap tm_v, ChainParams p) {
+                            const __grid_constant__ CUtensorMap tm_v,
+                            const __grid_constant__ CUtensorMap tm_o, ChainParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = aligned_smem(smem_raw);
     const bool chain = (int)blockIdx.x < p.units;
@@ -1165,7 +1186,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after_sync();
 
     if (chain)
-        chain_role<true>(sm, p, unit, n, h, t_begin, t_end, nch);
+        chain_role<true>(sm, &tm_o, p, unit, n, h, t_begin, t_end, nch);
     else
         producer_role<true>(sm, &tm_q, &tm_k, &tm_v, p, 0, 0, 0, 0, 0, 0, 0);
 
@@ -1181,7 +1202,7 @@ size_t pool_flag_bytes(int64_t units) {
 }
 
 bool fill_params(const PrefillArgs &a, ChainParams &p, CUtensorMap &mq, CUtensorMap &mk,
-                 CUtensorMap &mv);
+                 CUtensorMap &mv, CUtensorMap &mo);
 
 int sm_count() {
     int dev = 0, n = 0;
@@ -1208,14 +1229,15 @@ bool prefill_pool_fits(int64_t units) {
 }
 
 bool make_tile_map_bf16_128(CUtensorMap *m, const void *base, int64_t T, int32_t H);
+bool make_store_map_bf16_128(CUtensorMap *m, void *base, int64_t T, int32_t H);
 
 namespace {
 bool fill_params(const PrefillArgs &a, ChainParams &p, CUtensorMap &mq, CUtensorMap &mk,
-                 CUtensorMap &mv) {
+                 CUtensorMap &mv, CUtensorMap &mo) {
     if (a.T > 0x7fffffffLL || a.ws == nullptr) return false;
     const int64_t Tm = a.T > 0 ? a.T : 1;
     if (!make_tile_map_bf16_128(&mq, a.q, Tm, a.Hqk) || !make_tile_map_bf16_128(&mk, a.k, Tm, a.Hqk) ||
-        !make_tile_map_bf16_128(&mv, a.v, Tm, a.Hv))
+        !make_tile_map_bf16_128(&mv, a.v, Tm, a.Hv) || !make_store_map_bf16_128(&mo, a.o, Tm, a.Hv))
         return false;
     p.ring = static_cast<uint8_t *>(a.ws);
     p.flags = nullptr;
@@ -1230,20 +1252,20 @@ bool fill_params(const PrefillArgs &a, ChainParams &p, CUtensorMap &mq, CUtensor
 
 cudaError_t launch_prefill_cluster(const PrefillArgs &a, cudaStream_t s) {
     ChainParams p;
-    CUtensorMap mq, mk, mv;
-    if (!fill_params(a, p, mq, mk, mv)) return cudaErrorInvalidValue;
+    CUtensorMap mq, mk, mv, mo;
+    if (!fill_params(a, p, mq, mk, mv, mo)) return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(gdn_prefill_cluster_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
     const dim3 grid((unsigned)((int64_t)a.N * a.Hv * kCluster));
-    gdn_prefill_cluster_kernel<<<grid, kThreads, kSmemBytes, s>>>(mq, mk, mv, p);
+    gdn_prefill_cluster_kernel<<<grid, kThreads, kSmemBytes, s>>>(mq, mk, mv, mo, p);
     return cudaGetLastError();
 }
 
 cudaError_t launch_prefill_pool(const PrefillArgs &a, cudaStream_t s) {
     ChainParams p;
-    CUtensorMap mq, mk, mv;
-    if (!fill_params(a, p, mq, mk, mv)) return cudaErrorInvalidValue;
+    CUtensorMap mq, mk, mv, mo;
+    if (!fill_params(a, p, mq, mk, mv, mo)) return cudaErrorInvalidValue;
     const int sms = sm_count();
     if (!prefill_pool_fits(p.units) || sms <= 0) return launch_prefill_tc(a, s);
     const size_t fb = pool_flag_bytes(p.units);
@@ -1266,7 +1288,7 @@ cudaError_t launch_prefill_pool(const PrefillArgs &a, cudaStream_t s) {
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, gdn_prefill_pool_kernel, mq, mk, mv, p);
+    e = cudaLaunchKernelEx(&cfg, gdn_prefill_pool_kernel, mq, mk, mv, mo, p);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }

@@ -106,6 +106,17 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, u
         : "memory");
 }
 
+// 3-D tile store shared -> global (bulk-group completion: commit, then wait
+// with bulk_wait_read_all / bulk_wait_all).  The innermost coordinate must be
+// a multiple of 16 bytes and no coordinate may be negative.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap *map, const void *src, int32_t c0,
+                                             int32_t c1, int32_t c2) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4}], [%1];"
+        ::"l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
+}
+
 // ------------------------------------------------------------ bulk copies --
 
 // Contiguous global -> shared copy of `bytes` (multiple of 16, both addresses

@@ -70,6 +70,60 @@ __device__ __forceinline__ void store_split32(uint8_t *hi_tile, uint8_t *lo_tile
     }
 }
 
+// ---- warp-level tf32 tensor-core products (mma.sync m16n8k8) ----
+
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+
+// x = hi + lo with both parts tf32 (about 21 significant bits together)
+__device__ __forceinline__ void split_tf32(float x, uint32_t &hi, uint32_t &lo) {
+    hi = to_tf32(x);
+    lo = to_tf32(x - __uint_as_float(hi));
+}
+
+__device__ __forceinline__ void mma_tf32_16x8x8(float (&d)[4], const uint32_t (&a)[4],
+                                                const uint32_t (&b)[2]) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+// D = L R for 32 x 32 fp32 matrices on one warp's 16 x 8 tile per call site:
+// warp w (0..7) computes rows 16 (w >> 2) .. + 15, columns 8 (w & 3) .. + 7.
+// L(r, m) = Lp[r * ls + m], R(m, c) = Rp[m * rs + c].  Three tf32 passes
+// (hi hi, hi lo, lo hi, in separate accumulators) give nearly fp32 products.
+// The result goes to store(r, c, value), two columns per lane and row.
+template <class Store>
+__device__ __forceinline__ void mm32_tf32(const float *Lp, int ls, const float *Rp, int rs,
+                                          int warp, int lane, Store store) {
+    const int mt = warp >> 2, nt = warp & 3, gid = lane >> 2, tig = lane & 3;
+    float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f}, d2[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks) {
+        const int r0 = 16 * mt + gid, k0 = 8 * ks + tig, c0 = 8 * nt + gid;
+        uint32_t ah[4], al[4], bh[2], bl[2];
+        split_tf32(Lp[r0 * ls + k0], ah[0], al[0]);
+        split_tf32(Lp[(r0 + 8) * ls + k0], ah[1], al[1]);
+        split_tf32(Lp[r0 * ls + k0 + 4], ah[2], al[2]);
+        split_tf32(Lp[(r0 + 8) * ls + k0 + 4], ah[3], al[3]);
+        split_tf32(Rp[k0 * rs + c0], bh[0], bl[0]);
+        split_tf32(Rp[(k0 + 4) * rs + c0], bh[1], bl[1]);
+        mma_tf32_16x8x8(d0, ah, bh);
+        mma_tf32_16x8x8(d1, ah, bl);
+        mma_tf32_16x8x8(d2, al, bh);
+    }
+    const int rr = 16 * mt + gid, cc = 8 * nt + 2 * tig;
+    store(rr, cc, d0[0] + (d1[0] + d2[0]));
+    store(rr, cc + 1, d0[1] + (d1[1] + d2[1]));
+    store(rr + 8, cc, d0[2] + (d1[2] + d2[2]));
+    store(rr + 8, cc + 1, d0[3] + (d1[3] + d2[3]));
+}
+
 // T = (I + A)^-1 for the 64 x 64 strictly lower A in As (row stride kAS4),
 // into Ts (row stride kTS), fp32, 256 threads.  Three steps:
 //   1. the four 16 x 16 diagonal blocks D_i = (I + A_ii)^-1, by forward
@@ -77,12 +131,12 @@ __device__ __forceinline__ void store_split32(uint8_t *hi_tile, uint8_t *lo_tile
 //      write zeros above the diagonal blocks;
 //   2. T_10 = -D_1 A_10 D_0 and T_32 = -D_3 A_32 D_2 (the 32 x 32 halves);
 //   3. the lower-left 32 x 32 block T_bl = -T_bot (A_bl T_top), where T_top and
-//      T_bot are the two lower-triangular 32 x 32 diagonal halves.
-// The block products map a lane to an output column and a warp to four output
-// rows: the right operand is one conflict-free 32-bit load per term, the left
-// operand a broadcast 16-byte load per four terms, which keeps the products off
-// the shared-memory wavefront limit.  The 16 x 16 products split their sums over
-// the two half-warps.  As must hold explicit zeros on and above its diagonal
+//      T_bot are the two lower-triangular 32 x 32 diagonal halves, on warp-level
+//      tf32 tensor cores (mm32_tf32).
+// The 16 x 16 products of step 2 map a lane to an output column and a warp to
+// four output rows: the right operand is one conflict-free 32-bit load per
+// term, the left operand a broadcast 16-byte load per four terms, and the sums
+// are split over the two half-warps.  As must hold explicit zeros on and above its diagonal
 // and have 16-byte aligned rows.  Xs needs 1024 floats.  Callers synchronise
 // before (As complete); the function ends with a barrier.
 __device__ __forceinline__ void solve_tril64(const float *As, float *Ts, float *Xs, int tid) {
@@ -168,44 +222,12 @@ __device__ __forceinline__ void solve_tril64(const float *As, float *Ts, float *
         }
     }
     __syncthreads();
-    const int r4 = 4 * warp;  // 3.: rows r4 .. r4 + 3 of the 32 x 32 block, lane = column
-    {   // 3a. X = A_bl T_top
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int m = 0; m < 32; m += 4) {
-            float4 a4[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-                a4[j] = *reinterpret_cast<const float4 *>(As + (32 + r4 + j) * kAS4 + m);
-            float y[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) y[q] = Ts[(m + q) * kTS + lane];
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-                acc[j] = fmaf(a4[j].x, y[0], fmaf(a4[j].y, y[1], fmaf(a4[j].z, y[2], fmaf(a4[j].w, y[3], acc[j]))));
-        }
-#pragma unroll
-        for (int j = 0; j < 4; ++j) Xs[(r4 + j) * 32 + lane] = acc[j];
-    }
+    // 3a. X = A_bl T_top;  3b. T_bl = -T_bot X  (warp-level tf32 tensor cores)
+    mm32_tf32(As + 32 * kAS4, kAS4, Ts, kTS, warp, lane,
+              [&](int r, int c, float v) { Xs[r * 32 + c] = v; });
     __syncthreads();
-    {   // 3b. T_bl = -T_bot X
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int m = 0; m < 32; m += 4) {
-            float4 t4[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-                t4[j] = *reinterpret_cast<const float4 *>(Ts + (32 + r4 + j) * kTS + 32 + m);
-            float y[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) y[q] = Xs[(m + q) * 32 + lane];
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-                acc[j] = fmaf(t4[j].x, y[0], fmaf(t4[j].y, y[1], fmaf(t4[j].z, y[2], fmaf(t4[j].w, y[3], acc[j]))));
-        }
-#pragma unroll
-        for (int j = 0; j < 4; ++j) Ts[(32 + r4 + j) * kTS + lane] = -acc[j];
-    }
+    mm32_tf32(Ts + 32 * kTS + 32, kTS, Xs, 32, warp, lane,
+              [&](int r, int c, float v) { Ts[(32 + r) * kTS + c] = -v; });
     __syncthreads();
 }
 
