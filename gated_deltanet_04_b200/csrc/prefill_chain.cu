@@ -165,6 +165,7 @@ constexpr uint32_t P_P16 = 137216;      // P fp16 [64 rows][128 B], SW128
 constexpr uint32_t P_TBH = 145408, P_TBL = 153600, P_TGH = 161792, P_TGL = 169984;  // T tiles
 constexpr uint32_t P_UTS = P_TBH;       // then U~^T staging (same layout as SL_UT)
 constexpr uint32_t P_MISC = 178176;
+constexpr uint32_t P_ID = 182272;       // bf16 identity [64][128 B] (B operand of the Q^T product)
 static_assert(P_WST + 32768 <= P_P16 && P_UTS + 32768 <= P_MISC, "staging fits its region");
 static_assert(P_XS + 1024 * 4 <= P_P16, "solve scratch overflows");
 static_assert(P_TS % 16 == 0 && P_XS % 16 == 0, "float4 scratch must be aligned");
@@ -192,15 +193,18 @@ struct ProdMisc {
     uint64_t tma_bar[2];
     uint64_t mma_bar;
     uint64_t taken;
+    uint64_t qt_bar;  // the Q^T product of the current chunk has landed
     uint32_t tmem_base;
 };
-constexpr uint32_t kProdBytes = P_MISC + sizeof(ProdMisc);
+static_assert(P_MISC + sizeof(ProdMisc) <= P_ID, "identity tile after the misc block");
+constexpr uint32_t kProdBytes = P_ID + 8192;
 constexpr uint32_t kChainBytes = C_MISC + sizeof(ChainMisc);
 constexpr uint32_t kSmemBytes = (kProdBytes > kChainBytes ? kProdBytes : kChainBytes) + 1024;
 static_assert(kSmemBytes <= 232448, "fits the 227 KB opt-in shared memory of a CTA");
 
 // producer TMEM columns (128 allocated)
-constexpr uint32_t PT_G = 0, PT_U = 64;
+// producer TMEM columns (256 allocated): Gram then W^T, U~^T, Q^T
+constexpr uint32_t PT_G = 0, PT_U = 64, PT_Q = 128;
 
 // pool flags: a header of kFlagHeader words ([0] the chunk counter, [1] the
 // abort flag), then 8 words per unit ([0] taken, [1 + s] ready of slot s)
@@ -427,6 +431,17 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
             if (it.valid) issue_tma(l, it);
         }
     }
+    // the bf16 identity, K-major with the 128-byte swizzle: row n holds 1 at k = n
+    for (int x = tid; x < 512; x += kThreads) {  // 512 chunks of 16 bytes
+        const int n = x >> 3, ch = x & 7;
+        uint4 w = make_uint4(0u, 0u, 0u, 0u);
+        if ((n >> 3) == ch) {
+            uint32_t *wp = reinterpret_cast<uint32_t *>(&w);
+            wp[(n & 7) >> 1] = (n & 1) ? 0x3f800000u : 0x00003f80u;  // bf16 1.0 in the right half
+        }
+        st_row_chunk(sm + P_ID, n, ch, w);
+    }
+    fence_proxy_async_smem();
     __syncthreads();
     if (warp == kGatesWarp && ms->items[0].valid) {
         load_gates(ms->items[0]);
@@ -566,6 +581,15 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
             flush_delivery();
         }
 
+        // ---- Q^T = Q^T I on the tensor cores while the solve runs (exact: bf16 x 1) ----
+        if (tid == 0) {
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_f16_ss(tmem + PT_Q, make_sdesc(skqv + 8192 + ks * 2048, 16384, 1024),
+                           make_sdesc(sbase + P_ID + ks * 32, 16, 1024), IDESC_MK_N64_BF16, ks > 0);
+            mma_commit(&ms->qt_bar);
+        }
+
         // ---- T = (I + A)^-1 ----
         solve_tril64(As, Ts, Xs, tid);
         GDN_CL_PHASE(1, 6);  // solve
@@ -659,33 +683,23 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
                 ms->gst.qs = gt.qs;
             }
         }
-        {   // Q^T fp16 (MN-major: row d holds 64 tokens) from the bf16 Q tile into
-            // the V half of the tile buffer, which the U~ product has finished
-            // reading; scaled by Gamma when the gates allow (qs)
-            const int d = tid & 127, tq = (tid >> 7) * 32;
-            const uint8_t *qsrc = kqv + (d >> 6) * 16384 + 8192;
-            const uint32_t dbyte = (uint32_t)(d & 63) * 2u;
+        {   // Q^T fp16 (MN-major: row d holds 64 tokens) from TMEM into the V half
+            // of the tile buffer, which the U~ product has finished reading;
+            // scaled by Gamma when the gates allow (qs); tokens past L zeroed
+            if (!mbar_wait_bounded(&ms->qt_bar, l & 1, kWaitLimit)) timed_out = true;
+            tc_fence_after_sync();
+            const int c = 32 * half;
+            float v[32];
+            tmem_ld32(trow + PT_Q + c, v);
+            tmem_wait_ld();
             const bool qs = gt.qs;
 #pragma unroll
-            for (int g8 = 0; g8 < 4; ++g8) {
-                uint32_t w[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const uint32_t t = (uint32_t)(tq + 8 * g8 + 2 * e);
-                    float a = (int)t < L
-                        ? __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(qsrc + sw128(t, dbyte)))
-                        : 0.f;
-                    float b = (int)t + 1 < L
-                        ? __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(qsrc + sw128(t + 1, dbyte)))
-                        : 0.f;
-                    if (qs) {
-                        a *= gt.Gam[t];
-                        b *= gt.Gam[t + 1];
-                    }
-                    w[e] = pack_half2(a, b);
-                }
-                st_row_chunk(kqv + 32768, d, (tq >> 3) + g8, make_uint4(w[0], w[1], w[2], w[3]));
+            for (int x = 0; x < 32; ++x) {
+                const float sc = qs ? gt.Gam[c + x] : 1.f;
+                v[x] = (c + x < L) ? v[x] * sc : 0.f;
             }
+#pragma unroll
+            for (int e = 0; e < 32; e += 8) st_row_chunk(kqv + 32768, row, (c + e) / 8, pack8(v + e));
         }
         fence_proxy_async_smem();  // staged data -> visible to the bulk copies
         GDN_CL_PHASE(1, 9);  // staging
@@ -1103,12 +1117,13 @@ __device__ __forceinline__ uint32_t *setup_role(uint8_t *sm, bool chain, uint32_
     } else {
         ProdMisc *ms = reinterpret_cast<ProdMisc *>(sm + P_MISC);
         tmem_slot = &ms->tmem_base;
-        ncols = 128;
+        ncols = 256;
         if (tid == 0) {
             mbar_init(&ms->tma_bar[0], 1);
             mbar_init(&ms->tma_bar[1], 1);
             mbar_init(&ms->mma_bar, 1);
             mbar_init(&ms->taken, 1);
+            mbar_init(&ms->qt_bar, 1);
             fence_mbarrier_init();
             tma_prefetch_desc(tm_q);
             tma_prefetch_desc(tm_k);

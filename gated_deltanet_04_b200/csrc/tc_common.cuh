@@ -27,6 +27,7 @@ constexpr uint32_t IDESC_KM_N64 = make_idesc_f16(128, 64, 0, 1);
 constexpr uint32_t IDESC_KM_N128 = make_idesc_f16(128, 128, 0, 1);
 constexpr uint32_t IDESC_KM_N192 = make_idesc_f16(128, 192, 0, 1);
 constexpr uint32_t IDESC_KK_N64_BF16 = make_idesc_f16(128, 64, 0, 0, 1);
+constexpr uint32_t IDESC_MK_N64_BF16 = make_idesc_f16(128, 64, 1, 0, 1);
 
 __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
     const __half2 h = __floats2half2_rn(a, b);
