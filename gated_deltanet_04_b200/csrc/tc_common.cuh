@@ -125,6 +125,34 @@ __device__ __forceinline__ void mm32_tf32(const float *Lp, int ls, const float *
     store(rr + 8, cc + 1, d0[3] + (d1[3] + d2[3]));
 }
 
+// D = L R for one 16 x 8 tile with a 16-term sum: L(r, m) = Lp[r * ls + m]
+// (16 x 16), R(m, c) = Rp[m * rs + c] (16 x 8), three tf32 passes; the warp's
+// lanes pass the result to store(r, c, value).
+template <class Store>
+__device__ __forceinline__ void mm16x8_tf32(const float *Lp, int ls, const float *Rp, int rs,
+                                            int lane, Store store) {
+    const int gid = lane >> 2, tig = lane & 3;
+    float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f}, d2[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int ks = 0; ks < 2; ++ks) {
+        const int k0 = 8 * ks + tig;
+        uint32_t ah[4], al[4], bh[2], bl[2];
+        split_tf32(Lp[gid * ls + k0], ah[0], al[0]);
+        split_tf32(Lp[(gid + 8) * ls + k0], ah[1], al[1]);
+        split_tf32(Lp[gid * ls + k0 + 4], ah[2], al[2]);
+        split_tf32(Lp[(gid + 8) * ls + k0 + 4], ah[3], al[3]);
+        split_tf32(Rp[k0 * rs + gid], bh[0], bl[0]);
+        split_tf32(Rp[(k0 + 4) * rs + gid], bh[1], bl[1]);
+        mma_tf32_16x8x8(d0, ah, bh);
+        mma_tf32_16x8x8(d1, ah, bl);
+        mma_tf32_16x8x8(d2, al, bh);
+    }
+    store(gid, 2 * tig, d0[0] + (d1[0] + d2[0]));
+    store(gid, 2 * tig + 1, d0[1] + (d1[1] + d2[1]));
+    store(gid + 8, 2 * tig, d0[2] + (d1[2] + d2[2]));
+    store(gid + 8, 2 * tig + 1, d0[3] + (d1[3] + d2[3]));
+}
+
 // T = (I + A)^-1 for the 64 x 64 strictly lower A in As (row stride kAS4),
 // into Ts (row stride kTS), fp32, 256 threads.  Three steps:
 //   1. the four 16 x 16 diagonal blocks D_i = (I + A_ii)^-1, by forward
@@ -132,12 +160,9 @@ __device__ __forceinline__ void mm32_tf32(const float *Lp, int ls, const float *
 //      write zeros above the diagonal blocks;
 //   2. T_10 = -D_1 A_10 D_0 and T_32 = -D_3 A_32 D_2 (the 32 x 32 halves);
 //   3. the lower-left 32 x 32 block T_bl = -T_bot (A_bl T_top), where T_top and
-//      T_bot are the two lower-triangular 32 x 32 diagonal halves, on warp-level
-//      tf32 tensor cores (mm32_tf32).
-// The 16 x 16 products of step 2 map a lane to an output column and a warp to
-// four output rows: the right operand is one conflict-free 32-bit load per
-// term, the left operand a broadcast 16-byte load per four terms, and the sums
-// are split over the two half-warps.  As must hold explicit zeros on and above its diagonal
+//      T_bot are the two lower-triangular 32 x 32 diagonal halves.
+// The block products of steps 2 and 3 run on warp-level tf32 tensor cores
+// (three hi/lo passes, so nearly fp32).  As must hold explicit zeros on and above its diagonal
 // and have 16-byte aligned rows.  Xs needs 1024 floats.  Callers synchronise
 // before (As complete); the function ends with a barrier.
 __device__ __forceinline__ void solve_tril64(const float *As, float *Ts, float *Xs, int tid) {
@@ -171,56 +196,18 @@ __device__ __forceinline__ void solve_tril64(const float *As, float *Ts, float *
         *reinterpret_cast<float4 *>(dst + 4) = make_float4(0.f, 0.f, 0.f, 0.f);
     }
     __syncthreads();
-    // 2.: warp -> block b (i = 2b + 1, k = 2b) and rows rq .. rq + 3; lane -> column
-    // (lane & 15) and half of the 16-term sum (lane >> 4)
-    const int b2 = warp >> 2, rq = 4 * (warp & 3), col = lane & 15, kh = lane >> 4;
-    const int bi = 2 * b2 + 1, bk = bi - 1;
-    {   // 2a. X = A_{i,k} D_k
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int mg = 0; mg < 8; mg += 4) {
-            const int m = 8 * kh + mg;
-            float4 a4[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-                a4[j] = *reinterpret_cast<const float4 *>(As + (16 * bi + rq + j) * kAS4 + 16 * bk + m);
-            float y[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) y[q] = Ts[(16 * bk + m + q) * kTS + 16 * bk + col];
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-                acc[j] = fmaf(a4[j].x, y[0], fmaf(a4[j].y, y[1], fmaf(a4[j].z, y[2], fmaf(a4[j].w, y[3], acc[j]))));
-        }
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], 16);
-        if (kh == 0) {
-#pragma unroll
-            for (int j = 0; j < 4; ++j) Xs[(b2 << 8) + (rq + j) * 16 + col] = acc[j];
-        }
+    // 2. (warps 0..3: block b = warp >> 1 with i = 2b + 1, k = 2b; output
+    //    columns 8 (warp & 1) .. + 7), warp-level tf32 tensor cores
+    if (warp < 4) {  // 2a. X = A_{i,k} D_k
+        const int b2 = warp >> 1, bi = 2 * b2 + 1, bk = bi - 1, c8 = 8 * (warp & 1);
+        mm16x8_tf32(As + (16 * bi) * kAS4 + 16 * bk, kAS4, Ts + (16 * bk) * kTS + 16 * bk + c8, kTS,
+                    lane, [&](int r, int c, float v) { Xs[(b2 << 8) + r * 16 + c8 + c] = v; });
     }
     __syncthreads();
-    {   // 2b. T_{i,k} = -D_i X
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int mg = 0; mg < 8; mg += 4) {
-            const int m = 8 * kh + mg;
-            float4 d4[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-                d4[j] = *reinterpret_cast<const float4 *>(Ts + (16 * bi + rq + j) * kTS + 16 * bi + m);
-            float y[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) y[q] = Xs[(b2 << 8) + (m + q) * 16 + col];
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-                acc[j] = fmaf(d4[j].x, y[0], fmaf(d4[j].y, y[1], fmaf(d4[j].z, y[2], fmaf(d4[j].w, y[3], acc[j]))));
-        }
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], 16);
-        if (kh == 0) {
-#pragma unroll
-            for (int j = 0; j < 4; ++j) Ts[(16 * bi + rq + j) * kTS + 16 * bk + col] = -acc[j];
-        }
+    if (warp < 4) {  // 2b. T_{i,k} = -D_i X
+        const int b2 = warp >> 1, bi = 2 * b2 + 1, bk = bi - 1, c8 = 8 * (warp & 1);
+        mm16x8_tf32(Ts + (16 * bi) * kTS + 16 * bi, kTS, Xs + (b2 << 8) + c8, 16, lane,
+                    [&](int r, int c, float v) { Ts[(16 * bi + r) * kTS + 16 * bk + c8 + c] = -v; });
     }
     __syncthreads();
     // 3a. X = A_bl T_top;  3b. T_bl = -T_bot X  (warp-level tf32 tensor cores)
