@@ -573,13 +573,10 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
 
         // The T tiles below overwrite the previous chunk's U~ staging: its
         // stores must have read it (long done by now; the solve's first
-        // barrier orders this before every thread's writes).  The same thread
-        // reports that chunk ready: step 1 of the solve keeps warps 0 and 1
-        // busy while the others, this one included, would wait.
-        if (tid == kDeliverTid) {
-            bulk_wait_read_all();
-            flush_delivery();
-        }
+        // barrier orders this before every thread's writes).  Waiting for
+        // those stores to land, and signalling the chunk ready, comes later,
+        // in the U~ / W window, where this warp idles.
+        if (tid == kDeliverTid) bulk_wait_read_all();
 
         // ---- Q^T = Q^T I on the tensor cores while the solve runs (exact: bf16 x 1) ----
         if (tid == 0) {
@@ -642,6 +639,7 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
             if (l >= 1 && nx.valid) issue_tma((l + 1) & 1, nx);
         }
         if (tid == kFetchTid) ms->items[(l + 2) & 3] = fetch(l + 2);  // decode chunk l + 2
+        if (tid == kDeliverTid) flush_delivery();  // the previous chunk, landed -> ready
         if (tid == kSlotTid) {  // make sure this chunk's ring slot is free
             if constexpr (kPool) {
                 const uint32_t need = (uint32_t)(it.c - p.ring_slots + 1);

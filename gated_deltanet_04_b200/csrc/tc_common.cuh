@@ -172,16 +172,11 @@ __device__ __forceinline__ void solve_tril64(const float *As, float *Ts, float *
         const float *Ab = As + (16 * bi) * kAS4 + 16 * bi;
         float x[16];
 #pragma unroll
-        for (int rr = 0; rr < 16; ++rr) {
-            float a0 = (rr == col) ? 1.f : 0.f, a1 = 0.f;
+        for (int rr = 0; rr < 16; ++rr) x[rr] = (rr == col) ? 1.f : 0.f;
 #pragma unroll
-            for (int ii = 0; ii + 1 < rr; ii += 2) {
-                a0 -= Ab[rr * kAS4 + ii] * x[ii];
-                a1 -= Ab[rr * kAS4 + ii + 1] * x[ii + 1];
-            }
-            if (rr & 1) a0 -= Ab[rr * kAS4 + rr - 1] * x[rr - 1];
-            x[rr] = a0 + a1;
-        }
+        for (int j = 0; j < 15; ++j)
+#pragma unroll
+            for (int i = j + 1; i < 16; ++i) x[i] -= Ab[i * kAS4 + j] * x[j];
 #pragma unroll
         for (int rr = 0; rr < 16; ++rr) Ts[(16 * bi + rr) * kTS + 16 * bi + col] = x[rr];
     } else {  // zeros above the diagonal blocks: 6 blocks of 16 x 16, 8 floats per thread
