@@ -17,6 +17,10 @@
 //    copies (3 states in flight per SM: loads of the next two overlap the
 //    update of the current one, and the updated state leaves by a bulk store
 //    while the next is computed).  Threads only read and write shared memory.
+//    Each CTA takes a contiguous range of (n, h) units, so every SM streams
+//    one contiguous stretch of the states (measured ~1% faster on B200 than
+//    dealing units round-robin).  The units % grid left over are split into
+//    single rows across all CTAs, so no SM runs a whole extra unit at the end.
 //  * other head sizes: the direct kernel below.
 //
 // Direct kernel: one CTA of 8 warps per (n, h).  A row of Dk fp32 values is spread
@@ -160,9 +164,11 @@ __global__ void __launch_bounds__(kStThreads, 1)
     StagedSmem &sm = *reinterpret_cast<StagedSmem *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int first = blockIdx.x, stride = gridDim.x;
-    if (first >= units) return;
-    const int count = (units - first + stride - 1) / stride;  // units of this CTA
+    const int per = units / (int)gridDim.x, extra = units % (int)gridDim.x;
+    const int b = blockIdx.x;
+    const int first = b * per, stride = 1;
+    const int count = per;  // units of this CTA: a contiguous range (grid <= units, so >= 1)
+    if (count <= 0) return;
 
     if (tid == 0) {
         for (int s = 0; s < kStStages; ++s) mbar_init(&sm.full[s], 1);
@@ -177,6 +183,38 @@ __global__ void __launch_bounds__(kStThreads, 1)
             bulk_load(sm.state[issued], a.state + (int64_t)u * kStUnitFloats, kStUnitBytes,
                       &sm.full[issued]);
         }
+    }
+    // The extra = units % grid leftover units (the last ones), as single rows
+    // spread over all CTAs, one row per warp at a time, while this CTA's first
+    // stage loads are in flight.  Same arithmetic as the staged update below;
+    // no other CTA touches these units.
+    for (int r = b + (int)gridDim.x * warp; r < extra * 128; r += (int)gridDim.x * (kStThreads / 32)) {
+        const int u = per * (int)gridDim.x + r / 128, i = r % 128;
+        const int h = u % a.Hv, n = u / a.Hv;
+        const int j = h / (a.Hv / a.Hqk);
+        const int64_t qk = ((int64_t)n * a.Hqk + j) * 128 + 4 * lane;
+        const float4 k4 = load_vec4(a.k, qk, a.dtype), q4 = load_vec4(a.q, qk, a.dtype);
+        float *srow = a.state + (int64_t)u * kStUnitFloats + i * 128 + 4 * lane;
+        const float4 row = *reinterpret_cast<const float4 *>(srow);
+        const float dec = expf(a.g[u]), bb = a.beta[u];
+        const float vi = load_io(a.v, (int64_t)u * 128 + i, a.dtype);
+        float kq = k4.x * q4.x + k4.y * q4.y + k4.z * q4.z + k4.w * q4.w;
+        float sk = row.x * k4.x + row.y * k4.y + row.z * k4.z + row.w * k4.w;
+        float sq = row.x * q4.x + row.y * q4.y + row.z * q4.z + row.w * q4.w;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            kq += __shfl_xor_sync(0xffffffffu, kq, off);
+            sk += __shfl_xor_sync(0xffffffffu, sk, off);
+            sq += __shfl_xor_sync(0xffffffffu, sq, off);
+        }
+        const float uu = bb * (vi - dec * sk);
+        float4 w;
+        w.x = fmaf(uu, k4.x, dec * row.x);
+        w.y = fmaf(uu, k4.y, dec * row.y);
+        w.z = fmaf(uu, k4.z, dec * row.z);
+        w.w = fmaf(uu, k4.w, dec * row.w);
+        *reinterpret_cast<float4 *>(srow) = w;
+        if (lane == 0) store_io(a.o, (int64_t)u * 128 + i, fmaf(uu, kq, dec * sq), a.dtype);
     }
     UnitInputs nxt = load_unit_inputs(a, first, warp, lane);
     bool timed_out = false;
