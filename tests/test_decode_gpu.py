@@ -42,6 +42,26 @@ def test_decode_small_shapes(Dk, Dv, dtype):
     check_state(st.cpu(), s_ref)
 
 
+@pytest.mark.parametrize("N,Hqk,Hv", [(1, 1, 1), (37, 2, 4), (38, 2, 4), (75, 2, 4),
+                                       (8, 16, 48)])
+def test_decode_staged_unit_counts(N, Hqk, Hv):
+    """The D = 128 kernel splits N * Hv units into one contiguous range per CTA
+    (one CTA per SM) and spreads the units % grid left over as single rows over
+    all CTAs.  Unit counts below, at and just past a 148-SM grid, and 2.6 grids
+    with 88 left over, must all match the oracle."""
+    gen = torch.Generator().manual_seed(N * 100 + Hv)
+    q, k, v, g, beta = inputs.make_tokens(N, Hqk, Hv, 128, 128, torch.bfloat16,
+                                          inputs.G_SCALE_097, gen)
+    state = 0.05 * torch.randn(N, Hv, 128, 128, generator=gen)
+    layer = {"q": q, "k": k, "v": v, "g": g, "beta": beta, "state": state}
+    o_ref, s_ref = oracle_step(layer)
+    st = state.to(DEV)
+    o = gdn.gdn_decode_step(q.to(DEV), k.to(DEV), v.to(DEV), g.to(DEV), beta.to(DEV), st)
+    torch.cuda.synchronize()
+    check_o(o.cpu(), o_ref)
+    check_state(st.cpu(), s_ref)
+
+
 def test_decode_repeated_steps_track_recurrence():
     """Eight decode steps in a row equal one 8-token prefill of each sequence."""
     gen = torch.Generator().manual_seed(77)
