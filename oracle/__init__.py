@@ -148,3 +148,38 @@ def decode_step(q, k, v, g, beta, state, *, order=ORDER_STANDARD):
     N = q.shape[0]
     cu = np.arange(N + 1, dtype=np.int64)
     return recurrent(q, k, v, g, beta, state, cu, order=order)
+
+
+def round_bf16(x):
+    """Round float64 values to the nearest bfloat16, ties to even, in one step.
+
+    bfloat16 is the upper half of an IEEE-754 binary32 (sign, 8 exponent bits,
+    7 stored fraction bits): 8 significant bits.  With x = m 2^e, 0.5 <= |m| < 1
+    (frexp), the nearest such value is rint(m 2^8) 2^(e-8), rint rounding
+    halfway cases to the even integer.  Normal range only: a nonzero |x| below
+    2^-126 (bfloat16 subnormals) or above the largest finite bfloat16 raises.
+    Returns float64 arrays holding bfloat16 values exactly.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    ax = np.abs(x)
+    if np.any((ax != 0) & (ax < 2.0 ** -126)) or np.any(ax > 3.3895313892515355e38):
+        raise ValueError("round_bf16: value outside the normal bfloat16 range")
+    m, e = np.frexp(x)
+    return np.ldexp(np.rint(np.ldexp(m, 8)), e - 8)
+
+
+def decode_step_bf16_state(q, k, v, g, beta, state, *, order=ORDER_STANDARD):
+    """decode_step for a state stored in bfloat16 between steps.
+
+    The stored values are exact in fp64; the step runs in fp64 as decode_step
+    does, and the new state is stored by rounding each element once to
+    bfloat16 (nearest, ties to even).  ``state`` holds bfloat16 values (a torch
+    bfloat16 tensor, or float64 values that are all bfloat16-representable).
+    Returns (o [N,Hv,Dv], new state before rounding, new state rounded), all
+    float64.
+    """
+    s = _f64(state)
+    if not np.array_equal(round_bf16(s), s):
+        raise ValueError("decode_step_bf16_state: state is not bfloat16-representable")
+    o, s_new = decode_step(q, k, v, g, beta, s, order=order)
+    return o, s_new, round_bf16(s_new)

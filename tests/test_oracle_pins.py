@@ -354,3 +354,51 @@ def test_bad_seqlens_rejected():
         oracle.recurrent(q, k, v, g, beta, None, np.array([0, 5, 3, 8]))
     with pytest.raises(ValueError):
         oracle.recurrent(q, k, v, g, beta, None, np.array([0, 9]))
+
+
+# ---- bfloat16 state storage for decode ----------------------------------------
+
+def test_round_bf16_agrees_with_torch_on_fp32_values():
+    """torch rounds fp32 -> bfloat16 to nearest, ties to even; on values that are
+    exactly fp32 the oracle's one-step rounding from fp64 must agree bit for bit
+    (random normals, powers of two, and values right at rounding boundaries)."""
+    import torch
+    r = rnd(21)
+    x = r.standard_normal(200000).astype(np.float32)
+    ulp = np.float32(2.0 ** -7)
+    edges = (np.float32(1.0) + np.arange(-64, 64, dtype=np.float32) * ulp / 2).astype(np.float32)
+    x = np.concatenate([x, edges, -edges, np.float32(2.0) ** np.arange(-60, 60, dtype=np.float32)])
+    want = torch.from_numpy(x).to(torch.bfloat16).double().numpy()
+    assert np.array_equal(oracle.round_bf16(x.astype(np.float64)), want)
+
+
+def test_round_bf16_ties_to_even_and_error_bound():
+    one = 1.0
+    # halfway between 1 and 1 + 2^-7 -> 1 (even); between 1 + 2^-7 and 1 + 2^-6 -> 1 + 2^-6
+    assert oracle.round_bf16(np.array([one + 2.0 ** -8]))[0] == one
+    assert oracle.round_bf16(np.array([one + 3 * 2.0 ** -8]))[0] == one + 2.0 ** -6
+    assert oracle.round_bf16(np.array([one + 2.0 ** -8 + 2.0 ** -40]))[0] == one + 2.0 ** -7
+    x = rnd(22).standard_normal(100000) * 10.0 ** rnd(23).uniform(-20, 20, 100000)
+    y = oracle.round_bf16(x)
+    _, e = np.frexp(x)                                           # x = m 2^e, 0.5 <= |m| < 1
+    assert np.all(np.abs(y - x) <= np.ldexp(1.0, e - 9))          # half an ulp (ulp = 2^(e-8))
+    assert np.array_equal(oracle.round_bf16(y), y)                # idempotent
+    with pytest.raises(ValueError):
+        oracle.round_bf16(np.array([1e-39]))
+
+
+def test_decode_bf16_state_identity_step_keeps_bf16_state():
+    """a = 1, b = 0 leaves the state unchanged, so a bfloat16 state comes back
+    bit-identical and o = S q (P1 through the bfloat16 storage)."""
+    r = rnd(24)
+    N, Hqk, Hv, D = 3, 2, 4, 8
+    q = unit_rows(r.standard_normal((N, Hqk, D)))
+    k = unit_rows(r.standard_normal((N, Hqk, D)))
+    v = r.standard_normal((N, Hv, D))
+    S = oracle.round_bf16(r.standard_normal((N, Hv, D, D)))
+    o, s_new, s_bf16 = oracle.decode_step_bf16_state(q, k, v, np.zeros((N, Hv)), np.zeros((N, Hv)), S)
+    assert np.array_equal(s_bf16, S) and np.array_equal(s_new, S)
+    heads = np.arange(Hv) // (Hv // Hqk)
+    assert np.allclose(o, np.einsum("nhij,nhj->nhi", S, q[:, heads]), rtol=1e-13, atol=1e-13)
+    with pytest.raises(ValueError):
+        oracle.decode_step_bf16_state(q, k, v, np.zeros((N, Hv)), np.zeros((N, Hv)), S + 2.0 ** -20)
