@@ -9,7 +9,9 @@ One step is one pass of the whole hot path over one batch of synthetic input:
     zero initial state) -- the headline, in Mtok/s per layer;
   * decode: gdn_decode_step for 256 sequences through 48 layers, each layer
     with its own 768 MiB fp32 state updated in place -- reported as state
-    GB/s (bytes read + written) in the "decode" object.
+    GB/s (bytes read + written) in the "decode" object; the same step with
+    the states stored in bfloat16 (gdn_decode_step_bf16_state) is its
+    "bf16_state" entry.
 Inputs are drawn on the device by the seeded generator and are larger than
 L2 (8.7 GB per prefill step, 38.6 GB of decode states), so no flush is needed.
 For N > 1 (torchrun) every rank runs the same workload on its own GPU with no
@@ -59,7 +61,8 @@ def parse():
     p.add_argument("--case", default=None,
                    help="profiling mode: run one operation of a named workload (layer4k, "
                         "long256k, varlen32: one gdn_prefill call; decode256: one layer's "
-                        "gdn_decode_step) W + K times and print its per-call time; no bench line")
+                        "gdn_decode_step; decode256_bf16: the same with a bfloat16 state) "
+                        "W + K times and print its per-call time; no bench line")
     p.add_argument("--kernel", default="auto", choices=["auto", "pool", "cluster", "single_cta", "recurrent"],
                    help="prefill kernel for --case")
     return p.parse_args()
@@ -333,6 +336,12 @@ def run_case(args):
         L = inputs.make_decode_layer(0, device=dev)
         out = torch.empty_like(L["v"])
         fn = lambda: gdn.gdn_decode_step(L["q"], L["k"], L["v"], L["g"], L["beta"], L["state"], o=out)
+    elif args.case == "decode256_bf16":
+        L = inputs.make_decode_layer(0, device=dev)
+        out = torch.empty_like(L["v"])
+        sb = L["state"].to(torch.bfloat16)
+        fn = lambda: gdn.gdn_decode_step_bf16_state(L["q"], L["k"], L["v"], L["g"], L["beta"], sb,
+                                                    o=out)
     else:
         inp = inputs.make_prefill(args.case, device=dev)
         o = torch.empty_like(inp["v"])
@@ -411,7 +420,18 @@ def main():
         lambda: gdn.gdn_decode_step(L0["q"], L0["k"], L0["v"], L0["g"], L0["beta"], L0["state"],
                                     o=out0), K, W, dist, stream)
     d1_ms = dist.max(d1_total / K)
-    del layers, d_outs
+    # the same step with each layer's state stored in bfloat16 (half the bytes)
+    b_states = [L["state"].to(torch.bfloat16) for L in layers]
+
+    def decode_step_bf16():
+        for L, st, out in zip(layers, b_states, d_outs):
+            gdn.gdn_decode_step_bf16_state(L["q"], L["k"], L["v"], L["g"], L["beta"], st, o=out)
+
+    b_total, _ = time_launches(decode_step_bf16, K, W, dist, stream, sampler)
+    b_ms = dist.max(b_total / K)
+    b_state_gbs = weak_scaling_value(state_bytes_layer // 2 * dwl.layers, b_ms / 1e3,
+                                     dist.world) / 1e9
+    del layers, d_outs, b_states
     torch.cuda.empty_cache()
     clocks = sampler.stop()
 
@@ -461,7 +481,12 @@ def main():
                            "peak_source": f"{peaks['source']} copy",
                            "kernel": "gdn_decode_staged_kernel",
                            "algorithmic_bytes_per_launch": state_bytes_layer + io_bytes_layer},
-              "frac_of_8TBps": d_state_gbs / dist.world / 8000.0}
+              "frac_of_8TBps": d_state_gbs / dist.world / 8000.0,
+              "bf16_state": {"value": b_state_gbs, "unit": "GB/s", "ms_per_step": b_ms,
+                             "note": "same 48-layer step with the state stored in bfloat16 "
+                                     "(gdn_decode_step_bf16_state); GB/s of bf16 state bytes",
+                             "frac_of_measured_copy": b_state_gbs / dist.world / peaks["hbm_gbs"],
+                             "frac_of_8TBps": b_state_gbs / dist.world / 8000.0}}
 
     cpu = None
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
@@ -487,7 +512,7 @@ def main():
         "decode": decode,
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": K * (1 + dwl.layers + 1) + K * (0 if args.no_e2e else 1),
+        "gpu_launches": K * (1 + dwl.layers + 1 + dwl.layers) + K * (0 if args.no_e2e else 1),
         "clocks": clocks,
     }
     if dist.rank == 0:

@@ -10,6 +10,7 @@ is present, the calls raise.
 Entry points (same names as the C ABI):
     gdn_prefill(q, k, v, g, beta, initial_state=None, cu_seqlens=None, ...)
     gdn_decode_step(q, k, v, g, beta, state, ...)
+    gdn_decode_step_bf16_state(q, k, v, g, beta, state, ...)
 """
 from __future__ import annotations
 
@@ -19,7 +20,8 @@ import threading
 
 import torch
 
-__all__ = ["gdn_prefill", "gdn_decode_step", "gdn_prefill_workspace_bytes", "library",
+__all__ = ["gdn_prefill", "gdn_decode_step", "gdn_decode_step_bf16_state",
+           "gdn_prefill_workspace_bytes", "library",
            "GdnError", "LIB_PATH", "STATUS", "KERNELS"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgdn.so")
@@ -58,6 +60,8 @@ def library():
             lib.gdn_decode_step.argtypes = [vp, vp, vp, ctypes.c_int, vp, vp, vp, i32, i32, i32, i32,
                                             i32, vp, vp, vp]
             lib.gdn_decode_step.restype = ctypes.c_int
+            lib.gdn_decode_step_bf16_state.argtypes = lib.gdn_decode_step.argtypes
+            lib.gdn_decode_step_bf16_state.restype = ctypes.c_int
             lib.gdn_prefill_workspace_bytes.argtypes = [i32, i64, i32, i32, i32, i32, i32]
             lib.gdn_prefill_workspace_bytes.restype = sz
             lib.gdn_prefill_ex_workspace_bytes.argtypes = [i32, i64, i32, i32, i32, i32, i32,
@@ -179,4 +183,33 @@ def gdn_decode_step(q, k, v, g, beta, state, *, o=None, error_flag=None, stream=
                              _stream(stream))
     if rc != 0:
         raise GdnError(rc, "gdn_decode_step")
+    return o
+
+
+def gdn_decode_step_bf16_state(q, k, v, g, beta, state, *, o=None, error_flag=None, stream=None):
+    """gdn_decode_step for a state stored in bfloat16: ``state`` [N,Hv,128,128]
+    bfloat16, updated in place (computed in fp32, rounded to nearest even).
+    q, k [N,Hqk,128], v [N,Hv,128] (bf16 or fp32); g, beta [N,Hv] fp32.
+    Returns o [N,Hv,128]."""
+    lib = library()
+    dev = q.device
+    if dev.type != "cuda":
+        raise ValueError("gdn_decode_step_bf16_state runs on CUDA tensors only")
+    N, Hqk, Dk = q.shape
+    Hv, Dv = v.shape[1], v.shape[2]
+    if q.dtype not in DTYPE:
+        raise ValueError(f"unsupported io dtype {q.dtype}")
+    _check(k, "k", (N, Hqk, Dk), q.dtype, dev)
+    _check(v, "v", (N, Hv, Dv), q.dtype, dev)
+    _check(g, "g", (N, Hv), torch.float32, dev)
+    _check(beta, "beta", (N, Hv), torch.float32, dev)
+    _check(state, "state", (N, Hv, Dv, Dk), torch.bfloat16, dev)
+    if o is None:
+        o = torch.empty((N, Hv, Dv), dtype=q.dtype, device=dev)
+    _check(o, "o", (N, Hv, Dv), q.dtype, dev)
+    rc = lib.gdn_decode_step_bf16_state(_ptr(q), _ptr(k), _ptr(v), DTYPE[q.dtype], _ptr(g),
+                                        _ptr(beta), _ptr(state), N, Hqk, Hv, Dk, Dv, _ptr(o),
+                                        _ptr(error_flag), _stream(stream))
+    if rc != 0:
+        raise GdnError(rc, "gdn_decode_step_bf16_state")
     return o

@@ -84,7 +84,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32)
     const float dec = expf(gate);
     const float b = a.beta[(int64_t)n * a.Hv + h];
 
-    float *st = a.state + (int64_t)unit * a.Dv * DK;
+    float *st = static_cast<float *>(a.state) + (int64_t)unit * a.Dv * DK;
     const int64_t vo_base = (int64_t)unit * a.Dv;
 
     // w0 is warp-uniform, so every lane runs every shuffle below; rows past Dv
@@ -125,24 +125,107 @@ __global__ void __launch_bounds__(kDecodeWarps * 32)
 
 // ---------------------------------------------------------------- staged --
 
-constexpr int kStStages = 3;
-constexpr int kStThreads = 256;                 // 8 warps x 16 state rows
-constexpr uint32_t kStUnitFloats = 128 * 128;   // one (n, h) state
-constexpr uint32_t kStUnitBytes = kStUnitFloats * 4;
+constexpr uint32_t kStUnitElems = 128 * 128;    // one (n, h) state
 constexpr long long kStWaitLimit = 1ll << 31;   // SM clocks (about a second)
 
-struct StagedSmem {
-    float state[kStStages][kStUnitFloats];
-    float o[2][128];
-    uint64_t full[kStStages];
+// State storage: fp32, or bfloat16 (computed in fp32, rounded to nearest even
+// when stored).  A bfloat16 state is half the bytes, so twice as many stages
+// fit in the same shared memory.
+template <class StateT>
+struct StagedCfg;
+// kStages: states in shared memory.  kWarps: warps per CTA, 128 / kWarps state
+// rows each.  kLateRefill: a stage is refilled one unit after its bulk store
+// was issued (its read is done by then, so the issuing thread never waits),
+// instead of right after the store has read it.  kIoInStage: a unit's k, q and
+// v rows come with its stage (bulk copies on the stage's mbarrier) instead of
+// per-thread loads one unit ahead.  Measured on B200 (48-layer step): the fp32
+// state is bandwidth-bound with 3 stages and prefers the register path (12.8
+// vs 13.5 ms), a bfloat16 state moves half the bytes and needs the deeper,
+// never-waiting pipeline (7.4 ms; 10.0 ms with the fp32 choices).
+template <>
+struct StagedCfg<float> {
+    static constexpr int kStages = 3, kWarps = 16, kLateRefill = 0, kIoInStage = 0;
 };
-constexpr size_t kStSmemBytes = sizeof(StagedSmem) + 128;
+template <>
+struct StagedCfg<__nv_bfloat16> {
+    static constexpr int kStages = 6, kWarps = 16, kLateRefill = 1, kIoInStage = 1;
+};
 
+template <class StateT>
+struct StagedSmem {
+    static constexpr int kStages = StagedCfg<StateT>::kStages;
+    StateT state[kStages][kStUnitElems];
+    uint8_t io[kStages][3][512];  // the unit's k, q and v rows (io dtype), loaded with its state
+    float o[2][128];
+    uint64_t full[kStages];
+};
+template <class StateT>
+constexpr size_t staged_smem_bytes() {
+    return sizeof(StagedSmem<StateT>) + 128;
+}
+static_assert(staged_smem_bytes<float>() <= 232448 && staged_smem_bytes<__nv_bfloat16>() <= 232448,
+              "stages fit the 227 KB of shared memory a CTA can opt into");
+
+// Four consecutive state elements of a row, as fp32 (a lane's share of a row).
+__device__ __forceinline__ float4 ld_state4(const float *p) {
+    return *reinterpret_cast<const float4 *>(p);
+}
+__device__ __forceinline__ float4 ld_state4(const __nv_bfloat16 *p) {
+    const uint2 raw = *reinterpret_cast<const uint2 *>(p);
+    const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.x));
+    const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.y));
+    return make_float4(lo.x, lo.y, hi.x, hi.y);
+}
+__device__ __forceinline__ void st_state4(float *p, float4 w) {
+    *reinterpret_cast<float4 *>(p) = w;
+}
+__device__ __forceinline__ void st_state4(__nv_bfloat16 *p, float4 w) {
+    const __nv_bfloat162 lo = __floats2bfloat162_rn(w.x, w.y);  // round to nearest even
+    const __nv_bfloat162 hi = __floats2bfloat162_rn(w.z, w.w);
+    uint2 raw;
+    raw.x = *reinterpret_cast<const uint32_t *>(&lo);
+    raw.y = *reinterpret_cast<const uint32_t *>(&hi);
+    *reinterpret_cast<uint2 *>(p) = raw;
+}
+
+// Sums, over the 32 lanes of a warp, the 8 per-lane partial values sk[0..3],
+// sq[0..3] (dot products of 4 state rows with k and with q) in 9 shuffles
+// instead of 8 x 5: each exchange level sends half of the values a lane still
+// holds and keeps the other half (recursive halving).  After the three halving
+// levels lane L holds 8-lane partial sums of one value -- S.k (L < 16) or S.q
+// (L >= 16) of row (L >> 2) & 3 -- and two plain butterfly levels complete it.
+__device__ __forceinline__ float reduce8_transposed(const float (&sk)[4], const float (&sq)[4],
+                                                    int lane) {
+    const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4;
+    float h[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {  // lanes < 16 keep the S.k partials, the others S.q
+        const float send = b4 ? sk[i] : sq[i];
+        const float keep = b4 ? sq[i] : sk[i];
+        h[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+    }
+    float h2[2];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {  // bit 3 of the lane: rows 0, 1 or rows 2, 3
+        const float send = b3 ? h[i] : h[i + 2];
+        const float keep = b3 ? h[i + 2] : h[i];
+        h2[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+    }
+    const float send = b2 ? h2[0] : h2[1];  // bit 2: the even or the odd row of the pair
+    float t = (b2 ? h2[1] : h2[0]) + __shfl_xor_sync(0xffffffffu, send, 4);
+    t += __shfl_xor_sync(0xffffffffu, t, 2);
+    t += __shfl_xor_sync(0xffffffffu, t, 1);
+    return t;
+}
+
+// Per-thread inputs of one unit (the register path): k, q as 4 values of a
+// lane, gates, and v of row R*warp + lane on lanes 0 .. R-1.
 struct UnitInputs {
     float4 k, q;
-    float g, b, v;  // v: lanes 0..15 hold rows 16*warp + lane
+    float g, b, v;
 };
 
+template <int R>
 __device__ __forceinline__ UnitInputs load_unit_inputs(const DecodeArgs &a, int u, int warp,
                                                        int lane) {
     UnitInputs in;
@@ -153,16 +236,24 @@ __device__ __forceinline__ UnitInputs load_unit_inputs(const DecodeArgs &a, int 
     in.q = load_vec4(a.q, qk, a.dtype);
     in.g = a.g[u];
     in.b = a.beta[u];
-    in.v = lane < 16 ? load_io(a.v, (int64_t)u * 128 + 16 * warp + lane, a.dtype) : 0.f;
+    in.v = lane < R ? load_io(a.v, (int64_t)u * 128 + R * warp + lane, a.dtype) : 0.f;
     return in;
 }
 
-__global__ void __launch_bounds__(kStThreads, 1)
+template <class StateT>
+__global__ void __launch_bounds__(StagedCfg<StateT>::kWarps * 32, 1)
     gdn_decode_staged_kernel(DecodeArgs a, int units) {
     using namespace sm100;
+    constexpr int kStStages = StagedCfg<StateT>::kStages;
+    constexpr int kStThreads = StagedCfg<StateT>::kWarps * 32;
+    constexpr int R = 128 / StagedCfg<StateT>::kWarps;  // state rows per warp
+    constexpr bool kLate = StagedCfg<StateT>::kLateRefill != 0;
+    constexpr bool kIo = StagedCfg<StateT>::kIoInStage != 0;
+    constexpr uint32_t kStUnitBytes = kStUnitElems * sizeof(StateT);
     extern __shared__ uint8_t smem_raw[];
-    StagedSmem &sm = *reinterpret_cast<StagedSmem *>(
+    StagedSmem<StateT> &sm = *reinterpret_cast<StagedSmem<StateT> *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+    StateT *state = static_cast<StateT *>(a.state);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int per = units / (int)gridDim.x, extra = units % (int)gridDim.x;
     const int b = blockIdx.x;
@@ -175,15 +266,25 @@ __global__ void __launch_bounds__(kStThreads, 1)
         fence_mbarrier_init();
     }
     __syncthreads();
-    int issued = 0;  // units whose state load has been issued (thread 0's view)
-    if (tid == 0) {
-        for (; issued < count && issued < kStStages; ++issued) {
-            const int u = first + issued * stride;
-            mbar_arrive_expect_tx(&sm.full[issued], kStUnitBytes);
-            bulk_load(sm.state[issued], a.state + (int64_t)u * kStUnitFloats, kStUnitBytes,
-                      &sm.full[issued]);
+    // A stage holds one unit: its state (and with kIo its k, q and v rows),
+    // bulk copies that complete one mbarrier (thread 0 issues them).
+    const uint32_t esz = a.dtype == GDN_DTYPE_BF16 ? 2u : 4u, row_bytes = 128u * esz;
+    auto issue_stage = [&](int stg, int u) {
+        mbar_arrive_expect_tx(&sm.full[stg], kStUnitBytes + (kIo ? 3u * row_bytes : 0u));
+        bulk_load(sm.state[stg], state + (int64_t)u * kStUnitElems, kStUnitBytes, &sm.full[stg]);
+        if constexpr (kIo) {
+            const int h = u % a.Hv, n = u / a.Hv;
+            const int64_t qk = ((int64_t)n * a.Hqk + h / (a.Hv / a.Hqk)) * 128;
+            const uint8_t *kp = static_cast<const uint8_t *>(a.k), *qp = static_cast<const uint8_t *>(a.q);
+            bulk_load(sm.io[stg][0], kp + qk * esz, row_bytes, &sm.full[stg]);
+            bulk_load(sm.io[stg][1], qp + qk * esz, row_bytes, &sm.full[stg]);
+            bulk_load(sm.io[stg][2], static_cast<const uint8_t *>(a.v) + (int64_t)u * 128 * esz,
+                      row_bytes, &sm.full[stg]);
         }
-    }
+    };
+    int issued = 0;  // units whose stage load has been issued (thread 0's view)
+    if (tid == 0)
+        for (; issued < count && issued < kStStages; ++issued) issue_stage(issued, first + issued * stride);
     // The extra = units % grid leftover units (the last ones), as single rows
     // spread over all CTAs, one row per warp at a time, while this CTA's first
     // stage loads are in flight.  Same arithmetic as the staged update below;
@@ -194,8 +295,8 @@ __global__ void __launch_bounds__(kStThreads, 1)
         const int j = h / (a.Hv / a.Hqk);
         const int64_t qk = ((int64_t)n * a.Hqk + j) * 128 + 4 * lane;
         const float4 k4 = load_vec4(a.k, qk, a.dtype), q4 = load_vec4(a.q, qk, a.dtype);
-        float *srow = a.state + (int64_t)u * kStUnitFloats + i * 128 + 4 * lane;
-        const float4 row = *reinterpret_cast<const float4 *>(srow);
+        StateT *srow = state + (int64_t)u * kStUnitElems + i * 128 + 4 * lane;
+        const float4 row = ld_state4(srow);
         const float dec = expf(a.g[u]), bb = a.beta[u];
         const float vi = load_io(a.v, (int64_t)u * 128 + i, a.dtype);
         float kq = k4.x * q4.x + k4.y * q4.y + k4.z * q4.z + k4.w * q4.w;
@@ -213,54 +314,89 @@ __global__ void __launch_bounds__(kStThreads, 1)
         w.y = fmaf(uu, k4.y, dec * row.y);
         w.z = fmaf(uu, k4.z, dec * row.z);
         w.w = fmaf(uu, k4.w, dec * row.w);
-        *reinterpret_cast<float4 *>(srow) = w;
+        st_state4(srow, w);
         if (lane == 0) store_io(a.o, (int64_t)u * 128 + i, fmaf(uu, kq, dec * sq), a.dtype);
     }
-    UnitInputs nxt = load_unit_inputs(a, first, warp, lane);
+    // kIo: gates two units ahead in registers, the rest comes with the stage;
+    // otherwise all of a unit's inputs one unit ahead in registers
+    float g1 = 0.f, b1 = 0.f, g2 = 0.f, b2 = 0.f;
+    UnitInputs nxt{};
+    if constexpr (kIo) {
+        g1 = a.g[first];
+        b1 = a.beta[first];
+        if (count > 1) {
+            g2 = a.g[first + 1];
+            b2 = a.beta[first + 1];
+        }
+    } else {
+        nxt = load_unit_inputs<R>(a, first, warp, lane);
+    }
     bool timed_out = false;
     int li = 0;
 #pragma unroll 1
     for (; li < count; ++li) {
         const int u = first + li * stride;
         const int s = li % kStStages;
-        const UnitInputs cur = nxt;
-        if (li + 1 < count) nxt = load_unit_inputs(a, u + stride, warp, lane);
+        float gcur, bcur;
+        UnitInputs cur{};
+        if constexpr (kIo) {
+            gcur = g1;
+            bcur = b1;
+            g1 = g2;
+            b1 = b2;
+            if (li + 2 < count) {
+                g2 = a.g[u + 2 * stride];
+                b2 = a.beta[u + 2 * stride];
+            }
+        } else {
+            cur = nxt;
+            if (li + 1 < count) nxt = load_unit_inputs<R>(a, u + stride, warp, lane);
+            gcur = cur.g;
+            bcur = cur.b;
+        }
         if (!mbar_wait_bounded(&sm.full[s], (li / kStStages) & 1, kStWaitLimit)) timed_out = true;
 
-        const float dec = expf(cur.g);
-        float kq = cur.k.x * cur.q.x + cur.k.y * cur.q.y + cur.k.z * cur.q.z + cur.k.w * cur.q.w;
+        const float dec = expf(gcur);
+        const float4 kv = kIo ? load_vec4(sm.io[s][0], 4 * lane, a.dtype) : cur.k;
+        const float4 qv = kIo ? load_vec4(sm.io[s][1], 4 * lane, a.dtype) : cur.q;
+        float kq = kv.x * qv.x + kv.y * qv.y + kv.z * qv.z + kv.w * qv.w;
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) kq += __shfl_xor_sync(0xffffffffu, kq, off);
-        float *st = sm.state[s];
+        StateT *st = sm.state[s];
 #pragma unroll
-        for (int r0 = 0; r0 < 16; r0 += 4) {
+        for (int r0 = 0; r0 < R; r0 += 4) {
             float4 row[4];
             float sk[4], sq[4];
 #pragma unroll
             for (int r = 0; r < 4; ++r) {
-                row[r] = *reinterpret_cast<const float4 *>(st + (16 * warp + r0 + r) * 128 + 4 * lane);
-                sk[r] = row[r].x * cur.k.x + row[r].y * cur.k.y + row[r].z * cur.k.z + row[r].w * cur.k.w;
-                sq[r] = row[r].x * cur.q.x + row[r].y * cur.q.y + row[r].z * cur.q.z + row[r].w * cur.q.w;
+                row[r] = ld_state4(st + (R * warp + r0 + r) * 128 + 4 * lane);
+                sk[r] = row[r].x * kv.x + row[r].y * kv.y + row[r].z * kv.z + row[r].w * kv.w;
+                sq[r] = row[r].x * qv.x + row[r].y * qv.y + row[r].z * qv.z + row[r].w * qv.w;
             }
+            // the 8 dot products of these 4 rows, summed over the warp at once:
+            // lane L ends with the full S.k (L < 16) or S.q (L >= 16) of row
+            // rr = (L >> 2) & 3
+            const int rr = (lane >> 2) & 3;
+            const float t = reduce8_transposed(sk, sq, lane);
+            // u of row rr on lanes 0..15, then to every lane
+            const float vi = kIo ? load_io(sm.io[s][2], R * warp + r0 + rr, a.dtype)
+                                 : __shfl_sync(0xffffffffu, cur.v, r0 + rr);
+            const float u = bcur * (vi - dec * t);
+            float uu[4];
 #pragma unroll
-            for (int off = 16; off > 0; off >>= 1)
-#pragma unroll
-                for (int r = 0; r < 4; ++r) {
-                    sk[r] += __shfl_xor_sync(0xffffffffu, sk[r], off);
-                    sq[r] += __shfl_xor_sync(0xffffffffu, sq[r], off);
-                }
+            for (int r = 0; r < 4; ++r) uu[r] = __shfl_sync(0xffffffffu, u, 4 * r);
+            const float u_o = __shfl_xor_sync(0xffffffffu, u, 16);  // lanes >= 16: u of row rr
+            if (lane >= 16 && (lane & 3) == 0)
+                sm.o[li & 1][R * warp + r0 + rr] = fmaf(u_o, kq, dec * t);
 #pragma unroll
             for (int r = 0; r < 4; ++r) {
-                const int i = 16 * warp + r0 + r;
-                const float vi = __shfl_sync(0xffffffffu, cur.v, r0 + r);
-                const float uu = cur.b * (vi - dec * sk[r]);
+                const int i = R * warp + r0 + r;
                 float4 w;
-                w.x = fmaf(uu, cur.k.x, dec * row[r].x);
-                w.y = fmaf(uu, cur.k.y, dec * row[r].y);
-                w.z = fmaf(uu, cur.k.z, dec * row[r].z);
-                w.w = fmaf(uu, cur.k.w, dec * row[r].w);
-                *reinterpret_cast<float4 *>(st + i * 128 + 4 * lane) = w;
-                if (lane == 0) sm.o[li & 1][i] = fmaf(uu, kq, dec * sq[r]);
+                w.x = fmaf(uu[r], kv.x, dec * row[r].x);
+                w.y = fmaf(uu[r], kv.y, dec * row[r].y);
+                w.z = fmaf(uu[r], kv.z, dec * row[r].z);
+                w.w = fmaf(uu[r], kv.w, dec * row[r].w);
+                st_state4(st + i * 128 + 4 * lane, w);
             }
         }
         fence_proxy_async_smem();  // updated state -> visible to the bulk store
@@ -270,13 +406,18 @@ __global__ void __launch_bounds__(kStThreads, 1)
         }
         if (tid < 128) store_io(a.o, (int64_t)u * 128 + tid, sm.o[li & 1][tid], a.dtype);
         if (tid == 0) {
-            bulk_store(a.state + (int64_t)u * kStUnitFloats, st, kStUnitBytes);
+            bulk_store(state + (int64_t)u * kStUnitElems, st, kStUnitBytes);
             bulk_commit();
-            if (issued < count) {  // refill this stage with the unit kStStages ahead
+            if constexpr (kLate) {
+                // refill the previous unit's stage: its store was issued a unit ago
+                if (li >= 1 && issued < count) {
+                    bulk_wait_read_all_but_one();
+                    issue_stage((li + kStStages - 1) % kStStages, first + issued * stride);
+                    ++issued;
+                }
+            } else if (issued < count) {  // refill this stage with the unit kStStages ahead
                 bulk_wait_read_all();
-                const int un = first + issued * stride;
-                mbar_arrive_expect_tx(&sm.full[s], kStUnitBytes);
-                bulk_load(st, a.state + (int64_t)un * kStUnitFloats, kStUnitBytes, &sm.full[s]);
+                issue_stage(s, first + issued * stride);
                 ++issued;
             }
         }
@@ -289,22 +430,31 @@ __global__ void __launch_bounds__(kStThreads, 1)
     }
 }
 
+template <class StateT>
+cudaError_t launch_staged(const DecodeArgs &a, int units, cudaStream_t s) {
+    int dev = 0, sms = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(gdn_decode_staged_kernel<StateT>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)staged_smem_bytes<StateT>());
+    if (e != cudaSuccess) return e;
+    const int grid = units < sms ? units : sms;
+    gdn_decode_staged_kernel<StateT>
+        <<<grid, StagedCfg<StateT>::kWarps * 32, staged_smem_bytes<StateT>(), s>>>(a, units);
+    return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s) {
     const int units = a.N * a.Hv;
-    if (a.Dk == 128 && a.Dv == 128) {
-        int dev = 0, sms = 0;
-        cudaError_t e = cudaGetDevice(&dev);
-        if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(gdn_decode_staged_kernel,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kStSmemBytes);
-        if (e != cudaSuccess) return e;
-        const int grid = units < sms ? units : sms;
-        gdn_decode_staged_kernel<<<grid, kStThreads, kStSmemBytes, s>>>(a, units);
-        return cudaGetLastError();
+    if (a.state_bf16) {  // bfloat16 state storage: the staged kernel only
+        if (a.Dk != 128 || a.Dv != 128) return cudaErrorInvalidValue;
+        return launch_staged<__nv_bfloat16>(a, units, s);
     }
+    if (a.Dk == 128 && a.Dv == 128) return launch_staged<float>(a, units, s);
     const dim3 grid((unsigned)units);
     const dim3 block(kDecodeWarps * 32);
     switch (a.Dk) {

@@ -136,4 +136,27 @@ gdn_status gdn_decode_step(const void *q, const void *k, const void *v, gdn_dtyp
     return from_cuda(gdn::launch_decode(a, static_cast<cudaStream_t>(stream)));
 }
 
+gdn_status gdn_decode_step_bf16_state(const void *q, const void *k, const void *v,
+                                      gdn_dtype io_dtype, const float *g, const float *beta,
+                                      void *state, int32_t N, int32_t Hqk, int32_t Hv, int32_t Dk,
+                                      int32_t Dv, void *o, int32_t *dev_error_flag, void *stream) {
+    if (io_dtype != GDN_DTYPE_BF16 && io_dtype != GDN_DTYPE_F32) return GDN_ERR_INVALID_ARGUMENT;
+    if (N < 0 || Hqk <= 0 || Hv <= 0 || Dk <= 0 || Dv <= 0) return GDN_ERR_INVALID_ARGUMENT;
+    if (Hv % Hqk != 0) return GDN_ERR_INVALID_ARGUMENT;
+    if ((int64_t)N * Hv > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
+    if (Dk != 128 || Dv != 128) return GDN_ERR_UNSUPPORTED;
+    if (N == 0) return GDN_OK;
+    if (!q || !k || !v || !g || !beta || !state || !o) return GDN_ERR_INVALID_ARGUMENT;
+    const void *ptrs[] = {q, k, v, g, beta, state, o, dev_error_flag};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return GDN_ERR_INVALID_ARGUMENT;
+    if (o == q || o == k || o == v || o == state) return GDN_ERR_INVALID_ARGUMENT;
+    gdn::DecodeArgs a;
+    a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.state = state; a.o = o;
+    a.state_bf16 = 1;
+    a.err = dev_error_flag; a.N = N; a.Hqk = Hqk; a.Hv = Hv; a.Dk = Dk; a.Dv = Dv;
+    a.dtype = io_dtype;
+    return from_cuda(gdn::launch_decode(a, static_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

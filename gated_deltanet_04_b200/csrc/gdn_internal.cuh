@@ -27,7 +27,8 @@ struct PrefillArgs {
 struct DecodeArgs {
     const void *q, *k, *v;
     const float *g, *beta;
-    float *state;
+    void *state;            // fp32, or bfloat16 when state_bf16
+    int32_t state_bf16 = 0;
     void *o;
     int32_t *err;
     int32_t N, Hqk, Hv, Dk, Dv;

@@ -187,6 +187,27 @@ GDN_API gdn_status gdn_decode_step(const void *q, const void *k, const void *v, 
                            int32_t *dev_error_flag, void *stream);
 
 /*
+ * gdn_decode_step_bf16_state -- gdn_decode_step for a state that is stored in
+ * bfloat16 between steps, which halves the state bytes a decode step moves.
+ * The page (section 一, the per-sequence state of the DeltaNet layers) counts
+ * that state in fp32 and notes that the byte count follows the runtime dtype;
+ * this entry point is that other dtype.
+ *
+ *   state               bfloat16 [N][Hv][Dv][Dk], read and overwritten in place.
+ *   everything else     as gdn_decode_step.
+ * Arithmetic: each element is widened to fp32 (exact), the step runs in fp32
+ * exactly as in gdn_decode_step, o comes from the fp32 values, and the new
+ * state is rounded once to bfloat16, to nearest, ties to even.
+ * Supported: Dk = Dv = 128, either io dtype; other head sizes return
+ * GDN_ERR_UNSUPPORTED.  Errors and ownership as gdn_decode_step.
+ */
+GDN_API gdn_status gdn_decode_step_bf16_state(const void *q, const void *k, const void *v,
+                                              gdn_dtype io_dtype, const float *g,
+                                              const float *beta, void *state, int32_t N,
+                                              int32_t Hqk, int32_t Hv, int32_t Dk, int32_t Dv,
+                                              void *o, int32_t *dev_error_flag, void *stream);
+
+/*
  * gdn_prefill_static_workspace -- gdn_prefill_ex with kernel
  * GDN_PREFILL_CLUSTER, but the cluster kernel's workspace ring lives in a
  * fixed device array inside libgdn, so the call allocates nothing and takes

@@ -148,6 +148,34 @@ def test_decode_empty_batch_is_ok(lib):
     assert decode(lib, N=0) == 0
 
 
+def decode_bf16_state(lib, **kw):
+    args = dict(q=P, k=P + 0x1000, v=P + 0x2000, dt=0, g=P + 0x3000, beta=P + 0x4000,
+                state=P + 0x7000, N=256, Hqk=16, Hv=48, Dk=128, Dv=128, o=P + 0x5000, err=None,
+                stream=None)
+    args.update(kw)
+    return lib.gdn_decode_step_bf16_state(args["q"], args["k"], args["v"], args["dt"], args["g"],
+                                          args["beta"], args["state"], args["N"], args["Hqk"],
+                                          args["Hv"], args["Dk"], args["Dv"], args["o"],
+                                          args["err"], args["stream"])
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(state=None), INVALID),
+    (dict(state=MIS), INVALID),
+    (dict(o=P + 0x7000), INVALID),   # o aliases the state
+    (dict(Hv=40), INVALID),
+    (dict(dt=2), INVALID),
+    (dict(Dk=64, Dv=64), UNSUPPORTED),   # the bfloat16 state kernel is D = 128 only
+    (dict(Dv=96), UNSUPPORTED),
+])
+def test_decode_bf16_state_rejects(lib, kw, code):
+    assert decode_bf16_state(lib, **kw) == code
+
+
+def test_decode_bf16_state_empty_batch_is_ok(lib):
+    assert decode_bf16_state(lib, N=0) == 0
+
+
 def test_binding_refuses_cpu_tensors():
     import torch
     x = torch.zeros(4, 2, 16)

@@ -103,3 +103,91 @@ def test_decode256_all_layers_sampled():
             check_o(o.cpu(), o_ref, f"layer {layer_id} o")
             check_state(layer["state"].cpu(), s_ref, f"layer {layer_id} state")
         del layer
+
+
+# ---- bfloat16 state storage ----------------------------------------------------
+# The kernel widens each stored bfloat16 element to fp32, steps in fp32 and
+# rounds the new state once to bfloat16 (nearest even); the oracle steps in
+# fp64 and rounds its result the same way.  Rounding moves an element by at
+# most half a bfloat16 ulp, 2^-8 of its magnitude in the worst case, so the
+# state's rel-L2 against the oracle's unrounded fp64 state is bounded by 2^-8
+# (plus fp32 arithmetic error, ~1e-6).  Element by element, the kernel's value
+# is the oracle's rounded value or a neighbour, the two rounding different
+# inputs (an fp32 and an fp64 value) that can straddle a rounding boundary --
+# up to fp32 error: a S + u k^T rounds its terms (|a S|, |u k| up to a few
+# times max|S'|) at 2^-24, which for an element that nearly cancels can be
+# several of its own (tiny) ulps, hence an absolute slack of 2^-22 max|S'|.
+
+BF16_STATE_REL_L2 = 2.0 ** -8
+
+
+def bf16_ulp(x):
+    _, e = np.frexp(np.asarray(x, dtype=np.float64))
+    return np.ldexp(1.0, e - 8)
+
+
+def check_bf16_state(s_gpu, s_new64, s_rounded):
+    g64 = s_gpu.double().numpy()
+    rl = np.linalg.norm((g64 - s_new64).ravel()) / np.linalg.norm(s_new64.ravel())
+    assert rl <= BF16_STATE_REL_L2, f"bf16 state rel-L2 {rl:.3e}"
+    diff = np.abs(g64 - s_rounded)
+    slack = 2.0 ** -22 * np.max(np.abs(s_new64))
+    assert np.all(diff <= bf16_ulp(s_rounded) * 1.0000001 + slack), \
+        "bf16 state off by more than 1 ulp plus fp32 error"
+    same = float(np.mean(diff == 0))
+    assert same >= 0.99, f"only {same:.4f} of the bf16 state equals the oracle's rounding"
+    return rl, same
+
+
+@pytest.mark.parametrize("N,Hqk,Hv,dtype", [(1, 1, 1, torch.bfloat16), (38, 2, 4, torch.bfloat16),
+                                            (8, 16, 48, torch.bfloat16), (9, 2, 6, torch.float32)])
+def test_decode_bf16_state(N, Hqk, Hv, dtype):
+    gen = torch.Generator().manual_seed(5000 + N * 10 + Hv)
+    q, k, v, g, beta = inputs.make_tokens(N, Hqk, Hv, 128, 128, dtype, inputs.G_SCALE_097, gen)
+    state = (0.05 * torch.randn(N, Hv, 128, 128, generator=gen)).to(torch.bfloat16)
+    o_ref, s_new, s_rounded = oracle.decode_step_bf16_state(q, k, v, g, beta, state)
+    st = state.to(DEV)
+    o = gdn.gdn_decode_step_bf16_state(q.to(DEV), k.to(DEV), v.to(DEV), g.to(DEV), beta.to(DEV), st)
+    torch.cuda.synchronize()
+    check_o(o.cpu(), o_ref)
+    check_bf16_state(st.cpu(), s_new, s_rounded)
+
+
+def test_decode_bf16_state_repeated_steps():
+    """Eight bfloat16-state steps against eight oracle bfloat16-state steps.  Each
+    side rounds its own state every step; a 1-ulp difference at one step is
+    carried (and contracted) by the next, so after m steps the state's rel-L2 is
+    within m half-ulps: 8 * 2^-9."""
+    gen = torch.Generator().manual_seed(6001)
+    N, Hqk, Hv, steps = 4, 2, 6, 8
+    state = (0.05 * torch.randn(N, Hv, 128, 128, generator=gen)).to(torch.bfloat16)
+    s_ref = state
+    st = state.to(DEV)
+    for t in range(steps):
+        q, k, v, g, beta = inputs.make_tokens(N, Hqk, Hv, 128, 128, torch.bfloat16,
+                                              inputs.G_SCALE_097, gen)
+        o_ref, _, s_ref = oracle.decode_step_bf16_state(q, k, v, g, beta, s_ref)
+        o = gdn.gdn_decode_step_bf16_state(q.to(DEV), k.to(DEV), v.to(DEV), g.to(DEV),
+                                           beta.to(DEV), st)
+        torch.cuda.synchronize()
+        check_o(o.cpu(), o_ref, what=f"o step {t}")
+    g64 = st.cpu().double().numpy()
+    rl = np.linalg.norm((g64 - s_ref).ravel()) / np.linalg.norm(s_ref.ravel())
+    assert rl <= steps * 2.0 ** -9, f"state rel-L2 after {steps} steps {rl:.3e}"
+
+
+def test_decode_bf16_state_decode256_layer():
+    """The decode workload's shape (256 sequences x 48 heads) with a bfloat16
+    state: the full layer against the oracle."""
+    wl = inputs.WORKLOADS["decode256"]
+    layer = inputs.make_decode_layer(0, device="cpu")
+    state = layer["state"].to(torch.bfloat16)
+    o_ref, s_new, s_rounded = oracle.decode_step_bf16_state(layer["q"], layer["k"], layer["v"],
+                                                             layer["g"], layer["beta"], state)
+    st = state.to(DEV)
+    o = gdn.gdn_decode_step_bf16_state(layer["q"].to(DEV), layer["k"].to(DEV), layer["v"].to(DEV),
+                                       layer["g"].to(DEV), layer["beta"].to(DEV), st)
+    torch.cuda.synchronize()
+    assert o.shape == (wl.N, wl.Hv, wl.Dv)
+    check_o(o.cpu(), o_ref)
+    check_bf16_state(st.cpu(), s_new, s_rounded)
