@@ -29,6 +29,8 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgdn.so")
 STATUS = {0: "GDN_OK", 1: "GDN_ERR_INVALID_ARGUMENT", 2: "GDN_ERR_UNSUPPORTED", 3: "GDN_ERR_CUDA",
           4: "GDN_ERR_TIMEOUT", 5: "GDN_ERR_BAD_SEQLENS"}
 DTYPE = {torch.bfloat16: 0, torch.float32: 1}
+# gdn_order values of include/gdn.h: where the recall S k is taken
+ORDERS = {"standard": 0, "recall_first": 1}
 # gdn_prefill_kernel values of include/gdn.h
 KERNELS = {"auto": 0, "cluster": 1, "single_cta": 2, "recurrent": 3, "pool": 4}
 
@@ -62,6 +64,10 @@ def library():
             lib.gdn_decode_step.restype = ctypes.c_int
             lib.gdn_decode_step_bf16_state.argtypes = lib.gdn_decode_step.argtypes
             lib.gdn_decode_step_bf16_state.restype = ctypes.c_int
+            lib.gdn_prefill_order.argtypes = lib.gdn_prefill_ex.argtypes + [ctypes.c_int]
+            lib.gdn_prefill_order.restype = ctypes.c_int
+            lib.gdn_decode_step_order.argtypes = lib.gdn_decode_step.argtypes + [ctypes.c_int]
+            lib.gdn_decode_step_order.restype = ctypes.c_int
             lib.gdn_prefill_workspace_bytes.argtypes = [i32, i64, i32, i32, i32, i32, i32]
             lib.gdn_prefill_workspace_bytes.restype = sz
             lib.gdn_prefill_ex_workspace_bytes.argtypes = [i32, i64, i32, i32, i32, i32, i32,
@@ -104,7 +110,7 @@ def gdn_prefill_workspace_bytes(N, T, Hqk, Hv, Dk, Dv, chunk=0, kernel="auto"):
 
 def gdn_prefill(q, k, v, g, beta, initial_state=None, cu_seqlens=None, *, chunk=0, o=None,
                 final_state=None, output_final_state=True, workspace=None, error_flag=None,
-                stream=None, kernel="auto"):
+                stream=None, kernel="auto", order="standard"):
     """Chunk-parallel prefill of the gated delta rule on the GPU.
 
     q, k [T,Hqk,Dk] and v [T,Hv,Dv] (bf16 or fp32, same dtype); g, beta [T,Hv] fp32;
@@ -112,6 +118,8 @@ def gdn_prefill(q, k, v, g, beta, initial_state=None, cu_seqlens=None, *, chunk=
     Returns (o [T,Hv,Dv], final_state [N,Hv,Dv,Dk] or None).  ``final_state`` may be
     ``initial_state`` for an in-place update.  Asynchronous on the current stream.
     ``kernel``: "auto", "pool", "cluster", "single_cta" or "recurrent" (see gdn_prefill_ex).
+    ``order``: "standard", or "recall_first" (the recall S k before the decay; the C
+    entry point gdn_prefill_order).
     """
     lib = library()
     dev = q.device
@@ -148,19 +156,24 @@ def gdn_prefill(q, k, v, g, beta, initial_state=None, cu_seqlens=None, *, chunk=
         if need:
             workspace = torch.empty(need, dtype=torch.uint8, device=dev)
             ws_bytes = need
-    rc = lib.gdn_prefill_ex(_ptr(q), _ptr(k), _ptr(v), DTYPE[q.dtype], _ptr(g), _ptr(beta),
-                            _ptr(initial_state), _ptr(cu_seqlens), N, T, Hqk, Hv, Dk, Dv, chunk,
-                            _ptr(o), _ptr(final_state), _ptr(workspace), ws_bytes,
-                            _ptr(error_flag), _stream(stream), KERNELS[kernel])
+    args = (_ptr(q), _ptr(k), _ptr(v), DTYPE[q.dtype], _ptr(g), _ptr(beta), _ptr(initial_state),
+            _ptr(cu_seqlens), N, T, Hqk, Hv, Dk, Dv, chunk, _ptr(o), _ptr(final_state),
+            _ptr(workspace), ws_bytes, _ptr(error_flag), _stream(stream), KERNELS[kernel])
+    if order == "standard":
+        rc = lib.gdn_prefill_ex(*args)
+    else:
+        rc = lib.gdn_prefill_order(*args, ORDERS[order])
     if rc != 0:
         raise GdnError(rc, "gdn_prefill")
     return o, final_state
 
 
-def gdn_decode_step(q, k, v, g, beta, state, *, o=None, error_flag=None, stream=None):
+def gdn_decode_step(q, k, v, g, beta, state, *, o=None, error_flag=None, stream=None,
+                    order="standard"):
     """One-token update of N sequences, in place on ``state`` [N,Hv,Dv,Dk] fp32.
 
     q, k [N,Hqk,Dk], v [N,Hv,Dv] (bf16 or fp32); g, beta [N,Hv] fp32.  Returns o [N,Hv,Dv].
+    ``order``: "standard" or "recall_first" (the C entry point gdn_decode_step_order).
     """
     lib = library()
     dev = q.device
@@ -178,9 +191,12 @@ def gdn_decode_step(q, k, v, g, beta, state, *, o=None, error_flag=None, stream=
     if o is None:
         o = torch.empty((N, Hv, Dv), dtype=q.dtype, device=dev)
     _check(o, "o", (N, Hv, Dv), q.dtype, dev)
-    rc = lib.gdn_decode_step(_ptr(q), _ptr(k), _ptr(v), DTYPE[q.dtype], _ptr(g), _ptr(beta),
-                             _ptr(state), N, Hqk, Hv, Dk, Dv, _ptr(o), _ptr(error_flag),
-                             _stream(stream))
+    args = (_ptr(q), _ptr(k), _ptr(v), DTYPE[q.dtype], _ptr(g), _ptr(beta), _ptr(state), N, Hqk,
+            Hv, Dk, Dv, _ptr(o), _ptr(error_flag), _stream(stream))
+    if order == "standard":
+        rc = lib.gdn_decode_step(*args)
+    else:
+        rc = lib.gdn_decode_step_order(*args, ORDERS[order])
     if rc != 0:
         raise GdnError(rc, "gdn_decode_step")
     return o

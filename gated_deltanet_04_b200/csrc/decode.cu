@@ -3,7 +3,8 @@
 // Section 三 of "Qwen3.8-27B 架构深读: Gated DeltaNet 混合线性注意力与 262K
 // 长上下文": at inference every step does one fixed-size matrix update.  Per
 // (sequence n, v-head h) with a = exp(g), b = beta and row i of the state:
-//     r_i   = (a S_i) . k                 (recall from the decayed state)
+//     r_i   = (a S_i) . k                 (recall from the decayed state; with
+//                                          GDN_ORDER_RECALL_FIRST: S_i . k)
 //     u_i   = b (v_i - r_i)
 //     S_i'  = a S_i + u_i k^T             (delta write)
 //     o_i   = S_i' . q = a (S_i . q) + u_i (k . q)
@@ -82,6 +83,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32)
     const float kq = group_sum<S::LPR>(kk.x * qq.x + kk.y * qq.y + kk.z * qq.z + kk.w * qq.w);
     const float gate = a.g[(int64_t)n * a.Hv + h];
     const float dec = expf(gate);
+    const float rdec = a.order == GDN_ORDER_RECALL_FIRST ? 1.f : dec;  // decay of the recall
     const float b = a.beta[(int64_t)n * a.Hv + h];
 
     float *st = static_cast<float *>(a.state) + (int64_t)unit * a.Dv * DK;
@@ -109,7 +111,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32)
             const float sk = group_sum<S::LPR>(s.x * kk.x + s.y * kk.y + s.z * kk.z + s.w * kk.w);
             const float sq = group_sum<S::LPR>(s.x * qq.x + s.y * qq.y + s.z * qq.z + s.w * qq.w);
             if (i < a.Dv) {
-                const float u = b * (vi[r] - dec * sk);
+                const float u = b * (vi[r] - rdec * sk);
                 float4 w;
                 w.x = fmaf(u, kk.x, dec * s.x);
                 w.y = fmaf(u, kk.y, dec * s.y);
@@ -308,7 +310,7 @@ __global__ void __launch_bounds__(StagedCfg<StateT>::kWarps * 32, 1)
             sk += __shfl_xor_sync(0xffffffffu, sk, off);
             sq += __shfl_xor_sync(0xffffffffu, sq, off);
         }
-        const float uu = bb * (vi - dec * sk);
+        const float uu = bb * (vi - (a.order == GDN_ORDER_RECALL_FIRST ? 1.f : dec) * sk);
         float4 w;
         w.x = fmaf(uu, k4.x, dec * row.x);
         w.y = fmaf(uu, k4.y, dec * row.y);
@@ -357,6 +359,7 @@ __global__ void __launch_bounds__(StagedCfg<StateT>::kWarps * 32, 1)
         if (!mbar_wait_bounded(&sm.full[s], (li / kStStages) & 1, kStWaitLimit)) timed_out = true;
 
         const float dec = expf(gcur);
+        const float rdec = a.order == GDN_ORDER_RECALL_FIRST ? 1.f : dec;  // decay of the recall
         const float4 kv = kIo ? load_vec4(sm.io[s][0], 4 * lane, a.dtype) : cur.k;
         const float4 qv = kIo ? load_vec4(sm.io[s][1], 4 * lane, a.dtype) : cur.q;
         float kq = kv.x * qv.x + kv.y * qv.y + kv.z * qv.z + kv.w * qv.w;
@@ -381,7 +384,7 @@ __global__ void __launch_bounds__(StagedCfg<StateT>::kWarps * 32, 1)
             // u of row rr on lanes 0..15, then to every lane
             const float vi = kIo ? load_io(sm.io[s][2], R * warp + r0 + rr, a.dtype)
                                  : __shfl_sync(0xffffffffu, cur.v, r0 + rr);
-            const float u = bcur * (vi - dec * t);
+            const float u = bcur * (vi - rdec * t);
             float uu[4];
 #pragma unroll
             for (int r = 0; r < 4; ++r) uu[r] = __shfl_sync(0xffffffffu, u, 4 * r);

@@ -79,7 +79,20 @@ gdn_status gdn_prefill_ex(const void *q, const void *k, const void *v, gdn_dtype
                           int32_t Hv, int32_t Dk, int32_t Dv, int32_t chunk, void *o,
                           float *final_state, void *workspace, size_t workspace_bytes,
                           int32_t *dev_error_flag, void *stream, gdn_prefill_kernel kernel) {
+    return gdn_prefill_order(q, k, v, io_dtype, g, beta, initial_state, cu_seqlens, N, T, Hqk, Hv,
+                             Dk, Dv, chunk, o, final_state, workspace, workspace_bytes,
+                             dev_error_flag, stream, kernel, GDN_ORDER_STANDARD);
+}
+
+gdn_status gdn_prefill_order(const void *q, const void *k, const void *v, gdn_dtype io_dtype,
+                             const float *g, const float *beta, const float *initial_state,
+                             const int32_t *cu_seqlens, int32_t N, int64_t T, int32_t Hqk,
+                             int32_t Hv, int32_t Dk, int32_t Dv, int32_t chunk, void *o,
+                             float *final_state, void *workspace, size_t workspace_bytes,
+                             int32_t *dev_error_flag, void *stream, gdn_prefill_kernel kernel,
+                             gdn_order order) {
     if (kernel < GDN_PREFILL_AUTO || kernel > GDN_PREFILL_POOL) return GDN_ERR_INVALID_ARGUMENT;
+    if (order != GDN_ORDER_STANDARD && order != GDN_ORDER_RECALL_FIRST) return GDN_ERR_INVALID_ARGUMENT;
     if (io_dtype != GDN_DTYPE_BF16 && io_dtype != GDN_DTYPE_F32) return GDN_ERR_INVALID_ARGUMENT;
     if (N < 0 || T < 0 || Hqk <= 0 || Hv <= 0 || Dk <= 0 || Dv <= 0 || chunk < 0)
         return GDN_ERR_INVALID_ARGUMENT;
@@ -107,6 +120,7 @@ gdn_status gdn_prefill_ex(const void *q, const void *k, const void *v, gdn_dtype
     a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.s0 = initial_state; a.cu = cu_seqlens;
     a.o = o; a.sT = final_state; a.err = dev_error_flag; a.ws = workspace; a.T = T; a.N = N; a.Hqk = Hqk;
     a.Hv = Hv; a.Dk = Dk; a.Dv = Dv; a.chunk = chunk == 0 ? 64 : chunk; a.dtype = io_dtype;
+    a.order = order;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (T == 0 || kernel == GDN_PREFILL_RECURRENT) return from_cuda(gdn::launch_prefill_recurrent(a, s));
     if (kernel == GDN_PREFILL_SINGLE_CTA) return from_cuda(gdn::launch_prefill_tc(a, s));
@@ -118,6 +132,15 @@ gdn_status gdn_decode_step(const void *q, const void *k, const void *v, gdn_dtyp
                            const float *g, const float *beta, float *state, int32_t N,
                            int32_t Hqk, int32_t Hv, int32_t Dk, int32_t Dv, void *o,
                            int32_t *dev_error_flag, void *stream) {
+    return gdn_decode_step_order(q, k, v, io_dtype, g, beta, state, N, Hqk, Hv, Dk, Dv, o,
+                                 dev_error_flag, stream, GDN_ORDER_STANDARD);
+}
+
+gdn_status gdn_decode_step_order(const void *q, const void *k, const void *v, gdn_dtype io_dtype,
+                                 const float *g, const float *beta, float *state, int32_t N,
+                                 int32_t Hqk, int32_t Hv, int32_t Dk, int32_t Dv, void *o,
+                                 int32_t *dev_error_flag, void *stream, gdn_order order) {
+    if (order != GDN_ORDER_STANDARD && order != GDN_ORDER_RECALL_FIRST) return GDN_ERR_INVALID_ARGUMENT;
     if (io_dtype != GDN_DTYPE_BF16 && io_dtype != GDN_DTYPE_F32) return GDN_ERR_INVALID_ARGUMENT;
     if (N < 0 || Hqk <= 0 || Hv <= 0 || Dk <= 0 || Dv <= 0) return GDN_ERR_INVALID_ARGUMENT;
     if (Hv % Hqk != 0) return GDN_ERR_INVALID_ARGUMENT;
@@ -133,6 +156,7 @@ gdn_status gdn_decode_step(const void *q, const void *k, const void *v, gdn_dtyp
     a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.state = state; a.o = o;
     a.err = dev_error_flag; a.N = N; a.Hqk = Hqk; a.Hv = Hv; a.Dk = Dk; a.Dv = Dv;
     a.dtype = io_dtype;
+    a.order = order;
     return from_cuda(gdn::launch_decode(a, static_cast<cudaStream_t>(stream)));
 }
 

@@ -22,6 +22,7 @@ struct PrefillArgs {
     int64_t T;
     int32_t N, Hqk, Hv, Dk, Dv, chunk;
     gdn_dtype dtype;
+    int32_t order = GDN_ORDER_STANDARD;  // gdn_order
 };
 
 struct DecodeArgs {
@@ -33,6 +34,7 @@ struct DecodeArgs {
     int32_t *err;
     int32_t N, Hqk, Hv, Dk, Dv;
     gdn_dtype dtype;
+    int32_t order = GDN_ORDER_STANDARD;  // gdn_order
 };
 
 // Host launchers (return cudaGetLastError() of the launch).

@@ -223,6 +223,7 @@ struct ChainParams {
     int64_t T;
     int32_t N, Hqk, Hv, units, max_chunks;
     int32_t ring_slots;  // a power of two
+    int32_t recall_first;  // GDN_ORDER_RECALL_FIRST: recall before the decay
 };
 
 __device__ __forceinline__ uint8_t *ring_slot(const ChainParams &p, int unit, int c) {
@@ -411,7 +412,12 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
             gt.eC[r0] = expf(gC - x0);  gt.eC[r0 + 1] = expf(gC - x1);
         }
         gt.bb[r0] = bpre0;              gt.bb[r0 + 1] = bpre1;
-        gt.bG[r0] = bpre0 * G0;         gt.bG[r0 + 1] = bpre1 * G1;
+        // decay of token r's recall terms (in A and W): Gamma_r, or Gamma_{r-1}
+        // when the recall is taken before the decay (Gamma_{-1} = 1)
+        const float xp = __shfl_up_sync(0xffffffffu, x1, 1);  // gamma at token 2l - 1
+        const float Gr0 = p.recall_first ? (lane > 0 ? expf(xp) : 1.f) : G0;
+        const float Gr1 = p.recall_first ? G0 : G1;
+        gt.bG[r0] = bpre0 * Gr0;        gt.bG[r0 + 1] = bpre1 * Gr1;
         if (lane == 0) {
             gt.safe = safe_;
             gt.hp = GC >= kHighPrecisionDecay;
@@ -550,7 +556,8 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
 #pragma unroll
                 for (int x = 0; x < 32; ++x) v[x] *= sr * gt.iGam[c + x];
             } else {
-                const float gr = gt.gam[r];
+                const float gr = (row < kC && p.recall_first) ? (r > 0 ? gt.gam[r - 1] : 0.f)
+                                                              : gt.gam[r];
                 const float sr = row < kC ? gt.bb[r] : 1.f;
 #pragma unroll
                 for (int x = 0; x < 32; ++x) v[x] *= sr * expf(gr - gt.gam[c + x]);
@@ -1259,6 +1266,7 @@ bool fill_params(const PrefillArgs &a, ChainParams &p, CUtensorMap &mq, CUtensor
     p.units = a.N * a.Hv;
     p.max_chunks = (int)((a.T + kC - 1) / kC);
     p.ring_slots = kClusterRingSlots;
+    p.recall_first = a.order == GDN_ORDER_RECALL_FIRST;
     return true;
 }
 }  // namespace

@@ -3,6 +3,8 @@
 // This kernel runs the rule of section 三 of "Qwen3.8-27B 架构深读: Gated
 // DeltaNet 混合线性注意力与 262K 长上下文" one token at a time:
 //     S <- a S;  r = S k;  S <- S + b (v - r) k^T;  o = S q
+// or, in the page's step function order (GDN_ORDER_RECALL_FIRST), with the
+// recall r = S k taken before the decay.
 // It serves the head sizes and dtypes the tensor-core chunked kernel does not
 // (small heads, fp32 I/O, chunk lengths other than 64), where the chunked
 // form's per-chunk set-up would cost more than it saves.
@@ -28,6 +30,7 @@ __global__ void __launch_bounds__(128)
     __shared__ float qs[kTokBlock][DK];
     __shared__ float vs[kTokBlock][128];
     __shared__ float as_[kTokBlock], bs[kTokBlock];
+    const bool recall_first = a.order == GDN_ORDER_RECALL_FIRST;  // recall before the decay
 
     const int rows = blockDim.x;
     const int rb = blockIdx.x % row_blocks;
@@ -74,7 +77,7 @@ __global__ void __launch_bounds__(128)
                 p2 = fmaf(S[d + 2], ks[tt][d + 2], p2);
                 p3 = fmaf(S[d + 3], ks[tt][d + 3], p3);
             }
-            const float r = dec * ((p0 + p1) + (p2 + p3));
+            const float r = (recall_first ? 1.f : dec) * ((p0 + p1) + (p2 + p3));
             const float u = b * (vs[tt][threadIdx.x] - r);
             float o0 = 0.f, o1 = 0.f, o2 = 0.f, o3 = 0.f;
 #pragma unroll

@@ -136,6 +136,7 @@ struct TcParams {
     int32_t *err;
     int64_t T;
     int32_t N, Hqk, Hv;
+    int32_t recall_first;  // GDN_ORDER_RECALL_FIRST: recall before the decay
 };
 
 // Sum over warp 0 of one value per lane (each lane holding the sum of its
@@ -301,7 +302,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ms->eC[r0] = expf(gC - x0);  ms->eC[r0 + 1] = expf(gC - x1);
             }
             ms->bb[r0] = bpre0;              ms->bb[r0 + 1] = bpre1;
-            ms->bG[r0] = bpre0 * G0;         ms->bG[r0 + 1] = bpre1 * G1;
+            // decay of token r's recall terms (in A and W): Gamma_r, or Gamma_{r-1}
+            // when the recall is taken before the decay (Gamma_{-1} = 1)
+            const float xp = __shfl_up_sync(0xffffffffu, x1, 1);  // gamma at token 2l - 1
+            const float Gr0 = p.recall_first ? (lane > 0 ? expf(xp) : 1.f) : G0;
+            const float Gr1 = p.recall_first ? G0 : G1;
+            ms->bG[r0] = bpre0 * Gr0;        ms->bG[r0 + 1] = bpre1 * Gr1;
             if (lane == 0) {
                 ms->safe = safe_;
                 ms->hp = GC >= kHighPrecisionDecay;
@@ -372,7 +378,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int x = 0; x < 32; ++x) v[x] *= sr * ms->iGam[c + x];
             } else {
-                const float gr = ms->gam[r];
+                const float gr = (row < kC && p.recall_first) ? (r > 0 ? ms->gam[r - 1] : 0.f)
+                                                              : ms->gam[r];
                 const float sr = row < kC ? ms->bb[r] : 1.f;
 #pragma unroll
                 for (int x = 0; x < 32; ++x) v[x] *= sr * expf(gr - ms->gam[c + x]);
@@ -668,6 +675,7 @@ cudaError_t launch_prefill_tc(const PrefillArgs &a, cudaStream_t s) {
     TcParams p;
     p.g = a.g; p.beta = a.beta; p.s0 = a.s0; p.cu = a.cu; p.o = a.o; p.sT = a.sT; p.err = a.err;
     p.T = a.T; p.N = a.N; p.Hqk = a.Hqk; p.Hv = a.Hv;
+    p.recall_first = a.order == GDN_ORDER_RECALL_FIRST;
     cudaError_t e = cudaFuncSetAttribute(gdn_prefill_tc_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;

@@ -247,6 +247,48 @@ GDN_API gdn_status gdn_prefill_static_workspace(const void *q, const void *k, co
                                                 int32_t chunk, void *o, float *final_state,
                                                 int32_t *dev_error_flag, void *stream);
 
+/*
+ * Step order.  Section 三 of the page above states the gated rule with the
+ * decay applied first and then the delta edit (the standard order used by
+ * every call above), while its per-head step function takes the recall S k
+ * from the state before the decay:
+ *   GDN_ORDER_STANDARD      S <- a S;  r = S k;  S <- S + b (v - r) k^T;  o = S q
+ *   GDN_ORDER_RECALL_FIRST  r = S k;  S <- a S;  S <- S + b (v - r) k^T;  o = S q
+ * The two differ by b (1 - a) (S k) k^T per step and agree when a = 1 or b = 0.
+ */
+typedef enum gdn_order {
+    GDN_ORDER_STANDARD = 0,
+    GDN_ORDER_RECALL_FIRST = 1
+} gdn_order;
+
+/*
+ * gdn_prefill_order -- gdn_prefill_ex in either step order.  All other
+ * arguments, layouts, kernels, workspace sizes (gdn_prefill_ex_workspace_bytes)
+ * and errors are those of gdn_prefill_ex; an order outside gdn_order returns
+ * GDN_ERR_INVALID_ARGUMENT.  In the chunked kernels the recall-first order
+ * changes only the decay factor of the recall terms: token r's recall of the
+ * chunk's earlier writes and of the entering state is scaled by the decay up
+ * to token r - 1 instead of r.
+ */
+GDN_API gdn_status gdn_prefill_order(const void *q, const void *k, const void *v,
+                                     gdn_dtype io_dtype, const float *g, const float *beta,
+                                     const float *initial_state, const int32_t *cu_seqlens,
+                                     int32_t N, int64_t T, int32_t Hqk, int32_t Hv, int32_t Dk,
+                                     int32_t Dv, int32_t chunk, void *o, float *final_state,
+                                     void *workspace, size_t workspace_bytes,
+                                     int32_t *dev_error_flag, void *stream,
+                                     gdn_prefill_kernel kernel, gdn_order order);
+
+/*
+ * gdn_decode_step_order -- gdn_decode_step in either step order (fp32 state);
+ * otherwise identical to gdn_decode_step.
+ */
+GDN_API gdn_status gdn_decode_step_order(const void *q, const void *k, const void *v,
+                                         gdn_dtype io_dtype, const float *g, const float *beta,
+                                         float *state, int32_t N, int32_t Hqk, int32_t Hv,
+                                         int32_t Dk, int32_t Dv, void *o, int32_t *dev_error_flag,
+                                         void *stream, gdn_order order);
+
 /* Human-readable name of a status code (static storage, never NULL). */
 GDN_API const char *gdn_status_string(gdn_status status);
 

@@ -176,6 +176,37 @@ def test_decode_bf16_state_empty_batch_is_ok(lib):
     assert decode_bf16_state(lib, N=0) == 0
 
 
+def test_order_entry_points_reject_unknown_orders(lib):
+    """gdn_prefill_order / gdn_decode_step_order: a gdn_order outside the enum is
+    an argument error; the rest of the checks are those of the plain calls."""
+    pf = dict(q=P, k=P + 0x1000, v=P + 0x2000, dt=0, g=P + 0x3000, beta=P + 0x4000, s0=None,
+              cu=None, N=1, T=64, Hqk=16, Hv=48, Dk=128, Dv=128, chunk=64, o=P + 0x5000,
+              sT=None, ws=None, wsb=0, err=None, stream=None)
+    def prefill_order(order, **kw):
+        a = dict(pf, **kw)
+        return lib.gdn_prefill_order(a["q"], a["k"], a["v"], a["dt"], a["g"], a["beta"], a["s0"],
+                                     a["cu"], a["N"], a["T"], a["Hqk"], a["Hv"], a["Dk"], a["Dv"],
+                                     a["chunk"], a["o"], a["sT"], a["ws"], a["wsb"], a["err"],
+                                     a["stream"], 3, order)  # kernel 3: recurrent (no workspace)
+    assert prefill_order(2) == INVALID
+    assert prefill_order(-1) == INVALID
+    assert prefill_order(1, Hv=40) == INVALID
+    assert prefill_order(1, Dk=24) == UNSUPPORTED
+    assert prefill_order(1, N=0, T=0, cu=P + 0x6000) == 0
+
+    def decode_order(order, **kw):
+        a = dict(q=P, k=P + 0x1000, v=P + 0x2000, dt=0, g=P + 0x3000, beta=P + 0x4000,
+                 state=P + 0x7000, N=256, Hqk=16, Hv=48, Dk=128, Dv=128, o=P + 0x5000)
+        a.update(kw)
+        return lib.gdn_decode_step_order(a["q"], a["k"], a["v"], a["dt"], a["g"], a["beta"],
+                                         a["state"], a["N"], a["Hqk"], a["Hv"], a["Dk"], a["Dv"],
+                                         a["o"], None, None, order)
+    assert decode_order(2) == INVALID
+    assert decode_order(1, k=MIS) == INVALID
+    assert decode_order(1, Dk=24) == UNSUPPORTED
+    assert decode_order(1, N=0) == 0
+
+
 def test_binding_refuses_cpu_tensors():
     import torch
     x = torch.zeros(4, 2, 16)
