@@ -183,3 +183,30 @@ def decode_step_bf16_state(q, k, v, g, beta, state, *, order=ORDER_STANDARD):
         raise ValueError("decode_step_bf16_state: state is not bfloat16-representable")
     o, s_new = decode_step(q, k, v, g, beta, s, order=order)
     return o, s_new, round_bf16(s_new)
+
+
+def decode_step_slots(q, k, v, g, beta, pool, slot_idx, reset=None, *, order=ORDER_STANDARD):
+    """One decode step of N batch entries whose states live in a pool of slots
+    (continuous batching): entry n uses pool[slot_idx[n]]; when reset[n] is
+    nonzero it starts from a zero state instead (a new request), whatever the
+    slot held.  The updated states are written back to their slots; slots no
+    entry names are left as they are.  slot_idx must hold distinct values in
+    [0, num_slots).
+
+    Shapes: q,k [N,Hqk,Dk], v [N,Hv,Dv], g,beta [N,Hv], pool [S,Hv,Dv,Dk],
+    slot_idx [N] int, reset [N] or None.  Returns (o [N,Hv,Dv], new pool) in
+    float64.
+    """
+    pool = _f64(pool).copy()
+    idx = np.asarray(slot_idx.detach().cpu().numpy() if hasattr(slot_idx, "detach") else slot_idx,
+                     dtype=np.int64)
+    S = pool.shape[0]
+    if idx.ndim != 1 or np.any(idx < 0) or np.any(idx >= S) or len(set(idx.tolist())) != idx.size:
+        raise ValueError("decode_step_slots: slot indices must be distinct and in range")
+    states = pool[idx].copy()
+    if reset is not None:
+        rs = np.asarray(reset.detach().cpu().numpy() if hasattr(reset, "detach") else reset)
+        states[rs != 0] = 0.0
+    o, new = decode_step(q, k, v, g, beta, states, order=order)
+    pool[idx] = new
+    return o, pool

@@ -402,3 +402,64 @@ def test_decode_bf16_state_identity_step_keeps_bf16_state():
     assert np.allclose(o, np.einsum("nhij,nhj->nhi", S, q[:, heads]), rtol=1e-13, atol=1e-13)
     with pytest.raises(ValueError):
         oracle.decode_step_bf16_state(q, k, v, np.zeros((N, Hv)), np.zeros((N, Hv)), S + 2.0 ** -20)
+
+
+# ---- decode over a pool of state slots -----------------------------------------
+
+def _slots_case(seed, N=5, S=9, Hqk=2, Hv=4, D=8):
+    r = rnd(seed)
+    q = unit_rows(r.standard_normal((N, Hqk, D)))
+    k = unit_rows(r.standard_normal((N, Hqk, D)))
+    v = r.standard_normal((N, Hv, D))
+    g = -r.uniform(0, 1, (N, Hv))
+    b = r.uniform(0, 1, (N, Hv))
+    pool = r.standard_normal((S, Hv, D, D))
+    return q, k, v, g, b, pool
+
+
+def test_slots_identity_mapping_is_decode_step():
+    q, k, v, g, b, pool = _slots_case(31, N=5, S=5)
+    o, new = oracle.decode_step_slots(q, k, v, g, b, pool, np.arange(5))
+    o_ref, s_ref = oracle.decode_step(q, k, v, g, b, pool)
+    assert np.array_equal(o, o_ref) and np.array_equal(new, s_ref)
+
+
+def test_slots_gather_scatter_and_untouched_slots():
+    """Entries read and write only their own slots, in any order; slots nobody
+    names come back bit for bit; permuting the batch permutes only o."""
+    q, k, v, g, b, pool = _slots_case(32)
+    idx = np.array([7, 2, 5, 0, 3])
+    o, new = oracle.decode_step_slots(q, k, v, g, b, pool, idx)
+    o_ref, s_ref = oracle.decode_step(q, k, v, g, b, pool[idx])
+    assert np.array_equal(o, o_ref) and np.array_equal(new[idx], s_ref)
+    untouched = np.setdiff1d(np.arange(pool.shape[0]), idx)
+    assert np.array_equal(new[untouched], pool[untouched])
+    perm = np.array([3, 0, 4, 1, 2])
+    o_p, new_p = oracle.decode_step_slots(q[perm], k[perm], v[perm], g[perm], b[perm], pool, idx[perm])
+    assert np.array_equal(o_p, o[perm]) and np.array_equal(new_p, new)
+
+
+def test_slots_reset_starts_from_zero():
+    """A reset entry ignores its slot: with S = 0 the step is S' = b v k^T and
+    o = b (k . q) v (the rule from a zero state)."""
+    q, k, v, g, b, pool = _slots_case(33)
+    idx = np.array([4, 1, 8, 6, 0])
+    reset = np.array([0, 1, 0, 1, 0])
+    o, new = oracle.decode_step_slots(q, k, v, g, b, pool, idx, reset)
+    heads = np.arange(v.shape[1]) // (v.shape[1] // q.shape[1])
+    for n in np.nonzero(reset)[0]:
+        kk, qq = k[n, heads], q[n, heads]                       # [Hv, D]
+        want_s = b[n][:, None, None] * v[n][:, :, None] * kk[:, None, :]
+        assert np.allclose(new[idx[n]], want_s, rtol=1e-13, atol=1e-14)
+        want_o = (b[n] * np.sum(kk * qq, axis=1))[:, None] * v[n]
+        assert np.allclose(o[n], want_o, rtol=1e-12, atol=1e-13)
+    keep = np.nonzero(reset == 0)[0]
+    o_k, new_k = oracle.decode_step_slots(q[keep], k[keep], v[keep], g[keep], b[keep], pool, idx[keep])
+    assert np.array_equal(o[keep], o_k) and np.array_equal(new[idx[keep]], new_k[idx[keep]])
+
+
+def test_slots_reject_bad_indices():
+    q, k, v, g, b, pool = _slots_case(34)
+    for bad in ([0, 1, 2, 3, 9], [0, 1, 2, 3, -1], [0, 1, 2, 2, 4]):
+        with pytest.raises(ValueError):
+            oracle.decode_step_slots(q, k, v, g, b, pool, np.array(bad))
