@@ -20,14 +20,14 @@ import threading
 
 import torch
 
-__all__ = ["gdn_prefill", "gdn_decode_step", "gdn_decode_step_bf16_state",
+__all__ = ["gdn_prefill", "gdn_decode_step", "gdn_decode_step_bf16_state", "gdn_decode_step_slots",
            "gdn_prefill_workspace_bytes", "library",
            "GdnError", "LIB_PATH", "STATUS", "KERNELS"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgdn.so")
 
 STATUS = {0: "GDN_OK", 1: "GDN_ERR_INVALID_ARGUMENT", 2: "GDN_ERR_UNSUPPORTED", 3: "GDN_ERR_CUDA",
-          4: "GDN_ERR_TIMEOUT", 5: "GDN_ERR_BAD_SEQLENS"}
+          4: "GDN_ERR_TIMEOUT", 5: "GDN_ERR_BAD_SEQLENS", 6: "GDN_ERR_BAD_SLOT"}
 DTYPE = {torch.bfloat16: 0, torch.float32: 1}
 # gdn_order values of include/gdn.h: where the recall S k is taken
 ORDERS = {"standard": 0, "recall_first": 1}
@@ -68,6 +68,9 @@ def library():
             lib.gdn_prefill_order.restype = ctypes.c_int
             lib.gdn_decode_step_order.argtypes = lib.gdn_decode_step.argtypes + [ctypes.c_int]
             lib.gdn_decode_step_order.restype = ctypes.c_int
+            lib.gdn_decode_step_slots.argtypes = [vp, vp, vp, ctypes.c_int, vp, vp, vp, i32, vp, vp,
+                                                  i32, i32, i32, i32, i32, vp, vp, vp]
+            lib.gdn_decode_step_slots.restype = ctypes.c_int
             lib.gdn_prefill_workspace_bytes.argtypes = [i32, i64, i32, i32, i32, i32, i32]
             lib.gdn_prefill_workspace_bytes.restype = sz
             lib.gdn_prefill_ex_workspace_bytes.argtypes = [i32, i64, i32, i32, i32, i32, i32,
@@ -199,6 +202,41 @@ def gdn_decode_step(q, k, v, g, beta, state, *, o=None, error_flag=None, stream=
         rc = lib.gdn_decode_step_order(*args, ORDERS[order])
     if rc != 0:
         raise GdnError(rc, "gdn_decode_step")
+    return o
+
+
+def gdn_decode_step_slots(q, k, v, g, beta, state_pool, slot_idx, reset=None, *, o=None,
+                          error_flag=None, stream=None):
+    """One decode step for continuous batching: entry n's state is
+    ``state_pool[slot_idx[n]]`` ([num_slots,Hv,Dv,Dk] fp32, updated in place);
+    ``reset`` (int32 [N] or None) marks entries that start from a zero state.
+    ``slot_idx`` is int32 [N] on the device, distinct values in [0, num_slots).
+    q, k [N,Hqk,Dk], v [N,Hv,Dv] (bf16 or fp32); g, beta [N,Hv] fp32.  Returns o."""
+    lib = library()
+    dev = q.device
+    if dev.type != "cuda":
+        raise ValueError("gdn_decode_step_slots runs on CUDA tensors only")
+    N, Hqk, Dk = q.shape
+    Hv, Dv = v.shape[1], v.shape[2]
+    if q.dtype not in DTYPE:
+        raise ValueError(f"unsupported io dtype {q.dtype}")
+    S = state_pool.shape[0]
+    _check(k, "k", (N, Hqk, Dk), q.dtype, dev)
+    _check(v, "v", (N, Hv, Dv), q.dtype, dev)
+    _check(g, "g", (N, Hv), torch.float32, dev)
+    _check(beta, "beta", (N, Hv), torch.float32, dev)
+    _check(state_pool, "state_pool", (S, Hv, Dv, Dk), torch.float32, dev)
+    _check(slot_idx, "slot_idx", (N,), torch.int32, dev)
+    if reset is not None:
+        _check(reset, "reset", (N,), torch.int32, dev)
+    if o is None:
+        o = torch.empty((N, Hv, Dv), dtype=q.dtype, device=dev)
+    _check(o, "o", (N, Hv, Dv), q.dtype, dev)
+    rc = lib.gdn_decode_step_slots(_ptr(q), _ptr(k), _ptr(v), DTYPE[q.dtype], _ptr(g), _ptr(beta),
+                                   _ptr(state_pool), S, _ptr(slot_idx), _ptr(reset), N, Hqk, Hv,
+                                   Dk, Dv, _ptr(o), _ptr(error_flag), _stream(stream))
+    if rc != 0:
+        raise GdnError(rc, "gdn_decode_step_slots")
     return o
 
 

@@ -86,7 +86,13 @@ __global__ void __launch_bounds__(kDecodeWarps * 32)
     const float rdec = a.order == GDN_ORDER_RECALL_FIRST ? 1.f : dec;  // decay of the recall
     const float b = a.beta[(int64_t)n * a.Hv + h];
 
-    float *st = static_cast<float *>(a.state) + (int64_t)unit * a.Dv * DK;
+    const int64_t slot = decode_state_slot(a, n);
+    if (slot < 0) {  // a bad slot index: this unit writes nothing
+        if (threadIdx.x == 0) raise_error(a.err, GDN_ERR_BAD_SLOT);
+        return;
+    }
+    const bool zero = decode_state_reset(a, n);  // a new request: start from S = 0
+    float *st = static_cast<float *>(a.state) + (slot * a.Hv + h) * a.Dv * DK;
     const int64_t vo_base = (int64_t)unit * a.Dv;
 
     // w0 is warp-uniform, so every lane runs every shuffle below; rows past Dv
@@ -100,7 +106,8 @@ __global__ void __launch_bounds__(kDecodeWarps * 32)
         for (int r = 0; r < kRowsInFlight; ++r) {
             const int i = i0 + r * S::STRIDE;
             if (i < a.Dv) {
-                row[r] = __ldcs(reinterpret_cast<const float4 *>(st + (int64_t)i * DK) + l);
+                row[r] = zero ? make_float4(0.f, 0.f, 0.f, 0.f)
+                              : __ldcs(reinterpret_cast<const float4 *>(st + (int64_t)i * DK) + l);
                 vi[r] = load_io(a.v, vo_base + i, a.dtype);
             }
         }
@@ -153,6 +160,8 @@ struct StagedCfg<__nv_bfloat16> {
     static constexpr int kStages = 6, kWarps = 16, kLateRefill = 1, kIoInStage = 1;
 };
 
+constexpr int kSlotCache = 128;  // sequences whose slot / reset a CTA keeps in shared memory
+
 template <class StateT>
 struct StagedSmem {
     static constexpr int kStages = StagedCfg<StateT>::kStages;
@@ -160,6 +169,8 @@ struct StagedSmem {
     uint8_t io[kStages][3][512];  // the unit's k, q and v rows (io dtype), loaded with its state
     float o[2][128];
     uint64_t full[kStages];
+    int32_t slot_c[kSlotCache];   // pool decode: slots (-1: bad) of this CTA's sequences
+    int32_t reset_c[kSlotCache];
 };
 template <class StateT>
 constexpr size_t staged_smem_bytes() {
@@ -242,7 +253,9 @@ __device__ __forceinline__ UnitInputs load_unit_inputs(const DecodeArgs &a, int 
     return in;
 }
 
-template <class StateT>
+// kSlots: pool decode (slot indices, reset flags); a separate instantiation
+// so the plain kernels carry none of its code.
+template <class StateT, bool kSlots>
 __global__ void __launch_bounds__(StagedCfg<StateT>::kWarps * 32, 1)
     gdn_decode_staged_kernel(DecodeArgs a, int units) {
     using namespace sm100;
@@ -263,17 +276,55 @@ __global__ void __launch_bounds__(StagedCfg<StateT>::kWarps * 32, 1)
     const int count = per;  // units of this CTA: a contiguous range (grid <= units, so >= 1)
     if (count <= 0) return;
 
+    // Pool decode: the slot and reset flag of every sequence this CTA's units
+    // belong to, read once into shared memory (from global memory when there
+    // are more than kSlotCache of them).  Slot -1 marks an index out of range.
+    const int n_lo = first / a.Hv, n_span = (first + count - 1) / a.Hv - n_lo + 1;
+    const bool cached = kSlots && n_span <= kSlotCache;
+    if (cached)
+        for (int i = tid; i < n_span; i += kStThreads) {
+            sm.slot_c[i] = (int32_t)decode_state_slot(a, n_lo + i);
+            sm.reset_c[i] = decode_state_reset(a, n_lo + i) ? 1 : 0;
+        }
+    // (the leftover rows below belong to sequences outside that range)
+    auto in_cache = [&](int n) { return cached && n >= n_lo && n - n_lo < n_span; };
+    auto slot_of = [&](int n) -> int64_t {
+        if constexpr (!kSlots) return n;
+        else return in_cache(n) ? sm.slot_c[n - n_lo] : decode_state_slot(a, n);
+    };
+    auto reset_of = [&](int n) -> bool {
+        if constexpr (!kSlots) return false;
+        else return a.reset != nullptr && (in_cache(n) ? sm.reset_c[n - n_lo] != 0 : decode_state_reset(a, n));
+    };
+    // where unit u's state lives (-1: a bad slot, nothing is read or written)
+    auto state_off = [&](int u) -> int64_t {
+        if constexpr (!kSlots) {
+            return (int64_t)u * kStUnitElems;
+        } else {
+            const int64_t sl = slot_of(u / a.Hv);
+            return sl < 0 ? -1 : (sl * a.Hv + u % a.Hv) * (int64_t)kStUnitElems;
+        }
+    };
+
     if (tid == 0) {
         for (int s = 0; s < kStStages; ++s) mbar_init(&sm.full[s], 1);
         fence_mbarrier_init();
     }
     __syncthreads();
     // A stage holds one unit: its state (and with kIo its k, q and v rows),
-    // bulk copies that complete one mbarrier (thread 0 issues them).
+    // bulk copies that complete one mbarrier (thread 0 issues them).  A unit
+    // with a bad slot, or that starts from zeros, loads no state.
     const uint32_t esz = a.dtype == GDN_DTYPE_BF16 ? 2u : 4u, row_bytes = 128u * esz;
     auto issue_stage = [&](int stg, int u) {
-        mbar_arrive_expect_tx(&sm.full[stg], kStUnitBytes + (kIo ? 3u * row_bytes : 0u));
-        bulk_load(sm.state[stg], state + (int64_t)u * kStUnitElems, kStUnitBytes, &sm.full[stg]);
+        const int64_t off = state_off(u);
+        const bool load_state = off >= 0 && !reset_of(u / a.Hv);
+        if (!load_state && !kIo) {
+            mbar_arrive(&sm.full[stg]);
+            return;
+        }
+        mbar_arrive_expect_tx(&sm.full[stg],
+                              (load_state ? kStUnitBytes : 0u) + (kIo ? 3u * row_bytes : 0u));
+        if (load_state) bulk_load(sm.state[stg], state + off, kStUnitBytes, &sm.full[stg]);
         if constexpr (kIo) {
             const int h = u % a.Hv, n = u / a.Hv;
             const int64_t qk = ((int64_t)n * a.Hqk + h / (a.Hv / a.Hqk)) * 128;
@@ -297,8 +348,13 @@ __global__ void __launch_bounds__(StagedCfg<StateT>::kWarps * 32, 1)
         const int j = h / (a.Hv / a.Hqk);
         const int64_t qk = ((int64_t)n * a.Hqk + j) * 128 + 4 * lane;
         const float4 k4 = load_vec4(a.k, qk, a.dtype), q4 = load_vec4(a.q, qk, a.dtype);
-        StateT *srow = state + (int64_t)u * kStUnitElems + i * 128 + 4 * lane;
-        const float4 row = ld_state4(srow);
+        const int64_t off = state_off(u);
+        if (off < 0) {  // a bad slot index: this unit writes nothing
+            if (lane == 0) raise_error(a.err, GDN_ERR_BAD_SLOT);
+            continue;
+        }
+        StateT *srow = state + off + i * 128 + 4 * lane;
+        const float4 row = reset_of(n) ? make_float4(0.f, 0.f, 0.f, 0.f) : ld_state4(srow);
         const float dec = expf(a.g[u]), bb = a.beta[u];
         const float vi = load_io(a.v, (int64_t)u * 128 + i, a.dtype);
         float kq = k4.x * q4.x + k4.y * q4.y + k4.z * q4.z + k4.w * q4.w;
@@ -360,6 +416,10 @@ __global__ void __launch_bounds__(StagedCfg<StateT>::kWarps * 32, 1)
 
         const float dec = expf(gcur);
         const float rdec = a.order == GDN_ORDER_RECALL_FIRST ? 1.f : dec;  // decay of the recall
+        // pool decode: a bad slot computes on a stale stage and stores nothing;
+        // a reset unit starts from zeros (its stage was not loaded)
+        const int64_t uoff = state_off(u);
+        const bool bad = uoff < 0, zero = !bad && reset_of(u / a.Hv);
         const float4 kv = kIo ? load_vec4(sm.io[s][0], 4 * lane, a.dtype) : cur.k;
         const float4 qv = kIo ? load_vec4(sm.io[s][1], 4 * lane, a.dtype) : cur.q;
         float kq = kv.x * qv.x + kv.y * qv.y + kv.z * qv.z + kv.w * qv.w;
@@ -372,7 +432,8 @@ __global__ void __launch_bounds__(StagedCfg<StateT>::kWarps * 32, 1)
             float sk[4], sq[4];
 #pragma unroll
             for (int r = 0; r < 4; ++r) {
-                row[r] = ld_state4(st + (R * warp + r0 + r) * 128 + 4 * lane);
+                row[r] = zero ? make_float4(0.f, 0.f, 0.f, 0.f)
+                              : ld_state4(st + (R * warp + r0 + r) * 128 + 4 * lane);
                 sk[r] = row[r].x * kv.x + row[r].y * kv.y + row[r].z * kv.z + row[r].w * kv.w;
                 sq[r] = row[r].x * qv.x + row[r].y * qv.y + row[r].z * qv.z + row[r].w * qv.w;
             }
@@ -407,10 +468,11 @@ __global__ void __launch_bounds__(StagedCfg<StateT>::kWarps * 32, 1)
             if (tid == 0) raise_error(a.err, GDN_ERR_TIMEOUT);
             break;
         }
-        if (tid < 128) store_io(a.o, (int64_t)u * 128 + tid, sm.o[li & 1][tid], a.dtype);
+        if (tid < 128 && !bad) store_io(a.o, (int64_t)u * 128 + tid, sm.o[li & 1][tid], a.dtype);
         if (tid == 0) {
-            bulk_store(state + (int64_t)u * kStUnitElems, st, kStUnitBytes);
-            bulk_commit();
+            if (bad) raise_error(a.err, GDN_ERR_BAD_SLOT);
+            else bulk_store(state + uoff, st, kStUnitBytes);
+            bulk_commit();  // one group per unit (empty for a bad slot)
             if constexpr (kLate) {
                 // refill the previous unit's stage: its store was issued a unit ago
                 if (li >= 1 && issued < count) {
@@ -433,18 +495,18 @@ __global__ void __launch_bounds__(StagedCfg<StateT>::kWarps * 32, 1)
     }
 }
 
-template <class StateT>
+template <class StateT, bool kSlots>
 cudaError_t launch_staged(const DecodeArgs &a, int units, cudaStream_t s) {
     int dev = 0, sms = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(gdn_decode_staged_kernel<StateT>,
+        e = cudaFuncSetAttribute(gdn_decode_staged_kernel<StateT, kSlots>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)staged_smem_bytes<StateT>());
     if (e != cudaSuccess) return e;
     const int grid = units < sms ? units : sms;
-    gdn_decode_staged_kernel<StateT>
+    gdn_decode_staged_kernel<StateT, kSlots>
         <<<grid, StagedCfg<StateT>::kWarps * 32, staged_smem_bytes<StateT>(), s>>>(a, units);
     return cudaGetLastError();
 }
@@ -455,9 +517,10 @@ cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s) {
     const int units = a.N * a.Hv;
     if (a.state_bf16) {  // bfloat16 state storage: the staged kernel only
         if (a.Dk != 128 || a.Dv != 128) return cudaErrorInvalidValue;
-        return launch_staged<__nv_bfloat16>(a, units, s);
+        return launch_staged<__nv_bfloat16, false>(a, units, s);
     }
-    if (a.Dk == 128 && a.Dv == 128) return launch_staged<float>(a, units, s);
+    if (a.Dk == 128 && a.Dv == 128)
+        return a.slot ? launch_staged<float, true>(a, units, s) : launch_staged<float, false>(a, units, s);
     const dim3 grid((unsigned)units);
     const dim3 block(kDecodeWarps * 32);
     switch (a.Dk) {

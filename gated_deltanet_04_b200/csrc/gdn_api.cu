@@ -28,6 +28,7 @@ const char *gdn_status_string(gdn_status s) {
         case GDN_ERR_CUDA: return "GDN_ERR_CUDA";
         case GDN_ERR_TIMEOUT: return "GDN_ERR_TIMEOUT";
         case GDN_ERR_BAD_SEQLENS: return "GDN_ERR_BAD_SEQLENS";
+        case GDN_ERR_BAD_SLOT: return "GDN_ERR_BAD_SLOT";
     }
     return "GDN_ERR_UNKNOWN";
 }
@@ -157,6 +158,31 @@ gdn_status gdn_decode_step_order(const void *q, const void *k, const void *v, gd
     a.err = dev_error_flag; a.N = N; a.Hqk = Hqk; a.Hv = Hv; a.Dk = Dk; a.Dv = Dv;
     a.dtype = io_dtype;
     a.order = order;
+    return from_cuda(gdn::launch_decode(a, static_cast<cudaStream_t>(stream)));
+}
+
+gdn_status gdn_decode_step_slots(const void *q, const void *k, const void *v, gdn_dtype io_dtype,
+                                 const float *g, const float *beta, float *state_pool,
+                                 int32_t num_slots, const int32_t *slot_idx, const int32_t *reset,
+                                 int32_t N, int32_t Hqk, int32_t Hv, int32_t Dk, int32_t Dv,
+                                 void *o, int32_t *dev_error_flag, void *stream) {
+    if (io_dtype != GDN_DTYPE_BF16 && io_dtype != GDN_DTYPE_F32) return GDN_ERR_INVALID_ARGUMENT;
+    if (N < 0 || Hqk <= 0 || Hv <= 0 || Dk <= 0 || Dv <= 0) return GDN_ERR_INVALID_ARGUMENT;
+    if (Hv % Hqk != 0) return GDN_ERR_INVALID_ARGUMENT;
+    if ((int64_t)N * Hv > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
+    if (N == 0) return GDN_OK;
+    if (num_slots <= 0) return GDN_ERR_INVALID_ARGUMENT;
+    if (!q || !k || !v || !g || !beta || !state_pool || !slot_idx || !o) return GDN_ERR_INVALID_ARGUMENT;
+    const void *ptrs[] = {q, k, v, g, beta, state_pool, slot_idx, reset, o, dev_error_flag};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return GDN_ERR_INVALID_ARGUMENT;
+    if (o == q || o == k || o == v || o == state_pool) return GDN_ERR_INVALID_ARGUMENT;
+    if (!supported_dim(Dk)) return GDN_ERR_UNSUPPORTED;
+    gdn::DecodeArgs a;
+    a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.state = state_pool; a.o = o;
+    a.err = dev_error_flag; a.N = N; a.Hqk = Hqk; a.Hv = Hv; a.Dk = Dk; a.Dv = Dv;
+    a.dtype = io_dtype;
+    a.slot = slot_idx; a.reset = reset; a.num_slots = num_slots;
     return from_cuda(gdn::launch_decode(a, static_cast<cudaStream_t>(stream)));
 }
 

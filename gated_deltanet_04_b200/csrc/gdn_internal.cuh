@@ -35,7 +35,23 @@ struct DecodeArgs {
     int32_t N, Hqk, Hv, Dk, Dv;
     gdn_dtype dtype;
     int32_t order = GDN_ORDER_STANDARD;  // gdn_order
+    // pool decode: sequence n's state is slot slot[n] of num_slots; reset[n]
+    // nonzero: it starts from zeros.  slot == nullptr: the state of n is n.
+    const int32_t *slot = nullptr;
+    const int32_t *reset = nullptr;
+    int32_t num_slots = 0;
 };
+
+// The state slot of decode sequence n (n itself without a slot array), or -1
+// when slot[n] is out of range.
+__device__ __forceinline__ int64_t decode_state_slot(const DecodeArgs &a, int n) {
+    if (a.slot == nullptr) return n;
+    const int s = a.slot[n];
+    return (s >= 0 && s < a.num_slots) ? s : -1;
+}
+__device__ __forceinline__ bool decode_state_reset(const DecodeArgs &a, int n) {
+    return a.reset != nullptr && a.reset[n] != 0;
+}
 
 // Host launchers (return cudaGetLastError() of the launch).
 cudaError_t launch_prefill_recurrent(const PrefillArgs &a, cudaStream_t s);

@@ -66,7 +66,8 @@ typedef enum gdn_status {
     GDN_ERR_UNSUPPORTED = 2,      /* valid but not implemented (head dims, dtype) */
     GDN_ERR_CUDA = 3,             /* a CUDA runtime call or launch failed */
     GDN_ERR_TIMEOUT = 4,          /* device: a bounded wait expired */
-    GDN_ERR_BAD_SEQLENS = 5       /* device: cu_seqlens malformed */
+    GDN_ERR_BAD_SEQLENS = 5,      /* device: cu_seqlens malformed */
+    GDN_ERR_BAD_SLOT = 6          /* device: a state slot index out of range */
 } gdn_status;
 
 typedef enum gdn_dtype {
@@ -288,6 +289,35 @@ GDN_API gdn_status gdn_decode_step_order(const void *q, const void *k, const voi
                                          float *state, int32_t N, int32_t Hqk, int32_t Hv,
                                          int32_t Dk, int32_t Dv, void *o, int32_t *dev_error_flag,
                                          void *stream, gdn_order order);
+
+/*
+ * gdn_decode_step_slots -- gdn_decode_step for continuous batching: the head
+ * states live in a pool of slots, batch entry n uses slot slot_idx[n], and an
+ * entry that starts a new request starts from a zero state.  This is the
+ * runtime's batch / reset rule for the state (page "Layouts híbridos: três
+ * DeltaNet, uma attention", section on what the runtime must support: state
+ * updates, with rules for batching and reset).
+ *
+ *   state_pool          fp32 [num_slots][Hv][Dv][Dk], updated in place; only
+ *                       the slots named in slot_idx are read or written.
+ *   num_slots           slots in the pool (>= 1 when N > 0).
+ *   slot_idx            device int32 [N]: the slot of each entry.  The values
+ *                       must be distinct (two entries naming one slot race);
+ *                       a value outside [0, num_slots) is a device-detected
+ *                       error: GDN_ERR_BAD_SLOT goes to *dev_error_flag and
+ *                       that entry writes neither state nor o.
+ *   reset               device int32 [N] or NULL: nonzero = the entry's step
+ *                       starts from a zero state; its slot's old contents are
+ *                       not read, and the step's result overwrites them.
+ *   everything else     as gdn_decode_step (fp32 state, standard order).
+ * Supported: as gdn_decode_step.
+ */
+GDN_API gdn_status gdn_decode_step_slots(const void *q, const void *k, const void *v,
+                                         gdn_dtype io_dtype, const float *g, const float *beta,
+                                         float *state_pool, int32_t num_slots,
+                                         const int32_t *slot_idx, const int32_t *reset, int32_t N,
+                                         int32_t Hqk, int32_t Hv, int32_t Dk, int32_t Dv, void *o,
+                                         int32_t *dev_error_flag, void *stream);
 
 /* Human-readable name of a status code (static storage, never NULL). */
 GDN_API const char *gdn_status_string(gdn_status status);

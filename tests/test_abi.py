@@ -207,6 +207,34 @@ def test_order_entry_points_reject_unknown_orders(lib):
     assert decode_order(1, N=0) == 0
 
 
+def decode_slots(lib, **kw):
+    a = dict(q=P, k=P + 0x1000, v=P + 0x2000, dt=0, g=P + 0x3000, beta=P + 0x4000,
+             pool=P + 0x7000, S=300, slot=P + 0x8000, reset=None, N=256, Hqk=16, Hv=48, Dk=128,
+             Dv=128, o=P + 0x5000, err=None, stream=None)
+    a.update(kw)
+    return lib.gdn_decode_step_slots(a["q"], a["k"], a["v"], a["dt"], a["g"], a["beta"], a["pool"],
+                                     a["S"], a["slot"], a["reset"], a["N"], a["Hqk"], a["Hv"],
+                                     a["Dk"], a["Dv"], a["o"], a["err"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(slot=None), INVALID),
+    (dict(pool=None), INVALID),
+    (dict(S=0), INVALID),
+    (dict(reset=MIS), INVALID),
+    (dict(slot=MIS), INVALID),
+    (dict(o=P + 0x7000), INVALID),   # o aliases the pool
+    (dict(Hv=40), INVALID),
+    (dict(Dk=24), UNSUPPORTED),
+])
+def test_decode_slots_rejects(lib, kw, code):
+    assert decode_slots(lib, **kw) == code
+
+
+def test_decode_slots_empty_batch_is_ok(lib):
+    assert decode_slots(lib, N=0, S=0, slot=None) == 0
+
+
 def test_binding_refuses_cpu_tensors():
     import torch
     x = torch.zeros(4, 2, 16)

@@ -191,3 +191,59 @@ def test_decode_bf16_state_decode256_layer():
     assert o.shape == (wl.N, wl.Hv, wl.Dv)
     check_o(o.cpu(), o_ref)
     check_bf16_state(st.cpu(), s_new, s_rounded)
+
+
+# ---- continuous batching: states in a pool of slots ----------------------------
+
+def run_slots(q, k, v, g, beta, pool, idx, reset, flag=None):
+    t = lambda x: None if x is None else x.to(DEV).contiguous()
+    pd = pool.to(DEV)
+    o = torch.full(v.shape, 7.0, dtype=v.dtype, device=DEV)
+    gdn.gdn_decode_step_slots(t(q), t(k), t(v), t(g), t(beta), pd,
+                              torch.as_tensor(idx, dtype=torch.int32).to(DEV),
+                              None if reset is None else torch.as_tensor(reset, dtype=torch.int32).to(DEV),
+                              o=o, error_flag=flag)
+    torch.cuda.synchronize()
+    return o.cpu(), pd.cpu()
+
+
+@pytest.mark.parametrize("D,N,S,Hqk,Hv", [(128, 7, 20, 2, 6), (64, 7, 20, 2, 6),
+                                          (128, 256, 300, 16, 48)])
+def test_decode_slots(D, N, S, Hqk, Hv):
+    """Entries scattered over a pool in shuffled order, about one in five
+    starting a new request: o and every named slot match the oracle, and the
+    slots nobody names come back bit for bit."""
+    gen = torch.Generator().manual_seed(7000 + D + N)
+    q, k, v, g, beta = inputs.make_tokens(N, Hqk, Hv, D, D, torch.bfloat16, inputs.G_SCALE_097, gen)
+    pool = 0.05 * torch.randn(S, Hv, D, D, generator=gen)
+    idx = torch.randperm(S, generator=gen)[:N]
+    reset = (torch.rand(N, generator=gen) < 0.2).to(torch.int32)
+    flag = torch.zeros(4, dtype=torch.int32, device=DEV)
+    o, pd = run_slots(q, k, v, g, beta, pool, idx, reset, flag)
+    assert int(flag[0]) == 0
+    o_ref, pool_ref = oracle.decode_step_slots(q, k, v, g, beta, pool, idx, reset)
+    check_o(o, o_ref)
+    check_state(pd[idx], pool_ref[idx.numpy()])
+    untouched = torch.ones(S, dtype=torch.bool)
+    untouched[idx] = False
+    assert torch.equal(pd[untouched], pool[untouched])
+
+
+@pytest.mark.parametrize("D", [128, 64])
+def test_decode_slots_bad_index_sets_flag_and_writes_nothing(D):
+    gen = torch.Generator().manual_seed(7100 + D)
+    N, S, Hqk, Hv = 5, 8, 2, 4
+    q, k, v, g, beta = inputs.make_tokens(N, Hqk, Hv, D, D, torch.bfloat16, inputs.G_SCALE_097, gen)
+    pool = 0.05 * torch.randn(S, Hv, D, D, generator=gen)
+    idx = torch.tensor([3, 8, 0, -1, 6])  # entries 1 and 3 name no slot
+    flag = torch.zeros(4, dtype=torch.int32, device=DEV)
+    o, pd = run_slots(q, k, v, g, beta, pool, idx, None, flag)
+    assert int(flag[0]) == 6  # GDN_ERR_BAD_SLOT
+    good = [0, 2, 4]
+    o_ref, pool_ref = oracle.decode_step_slots(q[good], k[good], v[good], g[good], beta[good],
+                                               pool, idx[good])
+    check_o(o[good], o_ref)
+    check_state(pd[idx[good]], pool_ref[idx[good].numpy()])
+    assert torch.all(o[[1, 3]] == 7.0)           # the bad entries wrote no output
+    others = [s for s in range(S) if s not in idx[good].tolist()]
+    assert torch.equal(pd[others], pool[others])  # ... and no state
