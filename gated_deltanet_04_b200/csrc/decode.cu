@@ -147,17 +147,21 @@ struct StagedCfg;
 // was issued (its read is done by then, so the issuing thread never waits),
 // instead of right after the store has read it.  kIoInStage: a unit's k, q and
 // v rows come with its stage (bulk copies on the stage's mbarrier) instead of
-// per-thread loads one unit ahead.  Measured on B200 (48-layer step): the fp32
-// state is bandwidth-bound with 3 stages and prefers the register path (12.8
-// vs 13.5 ms), a bfloat16 state moves half the bytes and needs the deeper,
-// never-waiting pipeline (7.4 ms; 10.0 ms with the fp32 choices).
+// per-thread loads one unit ahead.  kCtasPerSm: resident CTAs per SM.  Measured
+// on B200 (48-layer step): the fp32 state is bandwidth-bound with 3 stages and
+// prefers the register path (12.8 vs 13.5 ms); a bfloat16 state moves half the
+// bytes and needs the never-waiting pipeline (7.4 ms; 10.0 ms with the fp32
+// choices), and runs best as two 8-warp CTAs per SM whose per-unit barriers
+// do not hold each other up (7.2 ms).
 template <>
 struct StagedCfg<float> {
-    static constexpr int kStages = 3, kWarps = 16, kLateRefill = 0, kIoInStage = 0;
+    static constexpr int kStages = 3, kWarps = 16, kLateRefill = 0, kIoInStage = 0, kCtasPerSm = 1;
 };
 template <>
 struct StagedCfg<__nv_bfloat16> {
-    static constexpr int kStages = 6, kWarps = 16, kLateRefill = 1, kIoInStage = 1;
+    static constexpr int kCtasPerSm = 2;
+    static constexpr int kStages = 6 / kCtasPerSm, kWarps = 16 / kCtasPerSm, kLateRefill = 1,
+                         kIoInStage = 1;
 };
 
 constexpr int kSlotCache = 128;  // sequences whose slot / reset a CTA keeps in shared memory
@@ -176,8 +180,9 @@ template <class StateT>
 constexpr size_t staged_smem_bytes() {
     return sizeof(StagedSmem<StateT>) + 128;
 }
-static_assert(staged_smem_bytes<float>() <= 232448 && staged_smem_bytes<__nv_bfloat16>() <= 232448,
-              "stages fit the 227 KB of shared memory a CTA can opt into");
+static_assert(staged_smem_bytes<float>() * StagedCfg<float>::kCtasPerSm <= 232448 &&
+                  staged_smem_bytes<__nv_bfloat16>() * StagedCfg<__nv_bfloat16>::kCtasPerSm <= 232448,
+              "stages fit the shared memory of an SM");
 
 // Four consecutive state elements of a row, as fp32 (a lane's share of a row).
 __device__ __forceinline__ float4 ld_state4(const float *p) {
@@ -256,7 +261,7 @@ __device__ __forceinline__ UnitInputs load_unit_inputs(const DecodeArgs &a, int 
 // kSlots: pool decode (slot indices, reset flags); a separate instantiation
 // so the plain kernels carry none of its code.
 template <class StateT, bool kSlots>
-__global__ void __launch_bounds__(StagedCfg<StateT>::kWarps * 32, 1)
+__global__ void __launch_bounds__(StagedCfg<StateT>::kWarps * 32, StagedCfg<StateT>::kCtasPerSm)
     gdn_decode_staged_kernel(DecodeArgs a, int units) {
     using namespace sm100;
     constexpr int kStStages = StagedCfg<StateT>::kStages;
@@ -505,7 +510,8 @@ cudaError_t launch_staged(const DecodeArgs &a, int units, cudaStream_t s) {
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)staged_smem_bytes<StateT>());
     if (e != cudaSuccess) return e;
-    const int grid = units < sms ? units : sms;
+    const int ctas = sms * StagedCfg<StateT>::kCtasPerSm;
+    const int grid = units < ctas ? units : ctas;
     gdn_decode_staged_kernel<StateT, kSlots>
         <<<grid, StagedCfg<StateT>::kWarps * 32, staged_smem_bytes<StateT>(), s>>>(a, units);
     return cudaGetLastError();
