@@ -210,3 +210,70 @@ def decode_step_slots(q, k, v, g, beta, pool, slot_idx, reset=None, *, order=ORD
     o, new = decode_step(q, k, v, g, beta, states, order=order)
     pool[idx] = new
     return o, pool
+
+
+def short_conv(x, w, cu_seqlens=None, conv_state=None):
+    """Causal depthwise convolution with 4 taps along time, the DeltaNet
+    mixer's "kernel 4" convolution (page "Layouts híbridos: três DeltaNet, uma
+    attention", section 01), one filter per channel:
+
+        y[t, c] = w[c, 0] x[t-3, c] + w[c, 1] x[t-2, c] + w[c, 2] x[t-1, c] + w[c, 3] x[t, c]
+
+    x [T, C] packed over sequences (cu_seqlens [N+1], or None for one); w [C, 4].
+    Inputs before a sequence's first token come from conv_state [N, 3, C] (the
+    three inputs that preceded it, oldest first) or are zero when it is None.
+    Returns (y [T, C], new conv state [N, 3, C]: each sequence's last three
+    inputs, reaching into the old state when the sequence is shorter than 3).
+    All float64.
+    """
+    x, w = _f64(x), _f64(w)
+    T, C = x.shape
+    assert w.shape == (C, 4)
+    if cu_seqlens is None:
+        cu = np.array([0, T], dtype=np.int64)
+    else:
+        cu = np.asarray(cu_seqlens.detach().cpu().numpy() if hasattr(cu_seqlens, "detach")
+                        else cu_seqlens, dtype=np.int64)
+    N = cu.shape[0] - 1
+    st = np.zeros((N, 3, C)) if conv_state is None else _f64(conv_state)
+    y = np.zeros((T, C))
+    new_state = np.zeros((N, 3, C))
+    for n in range(N):
+        # the sequence's inputs with its three predecessors in front
+        ext = np.concatenate([st[n], x[cu[n]:cu[n + 1]]], axis=0)
+        for t in range(cu[n + 1] - cu[n]):
+            for j in range(4):
+                y[cu[n] + t] += w[:, j] * ext[t + j]
+        new_state[n] = ext[ext.shape[0] - 3:]
+    return y, new_state
+
+
+def l2_normalise_heads(y, H, D):
+    """Each (token, head) row of y [T, H*D] divided by its Euclidean norm (a
+    zero row stays zero).  Returns [T, H, D] float64."""
+    y = _f64(y).reshape(-1, H, D)
+    nrm = np.sqrt(np.sum(y * y, axis=-1, keepdims=True))
+    return np.divide(y, nrm, out=np.zeros_like(y), where=nrm > 0)
+
+
+def short_conv_norm(xq, xk, xv, wq, wk, wv, cu_seqlens=None, conv_state=None):
+    """The front end of the DeltaNet mixer before the delta rule: the kernel-4
+    causal convolution on the q, k and v channels, then q and k normalised per
+    head.  xq, xk [T, Hqk, Dk], xv [T, Hv, Dv]; wq, wk [Hqk*Dk, 4], wv [Hv*Dv, 4];
+    conv_state [N, 3, 2*Hqk*Dk + Hv*Dv] (q, k, v channels in that order) or
+    None.  Returns (q, k, v, new conv state), float64."""
+    xq, xk, xv = _f64(xq), _f64(xk), _f64(xv)
+    T, Hqk, Dk = xq.shape
+    Hv, Dv = xv.shape[1], xv.shape[2]
+    Cq, Cv = Hqk * Dk, Hv * Dv
+    cs = None if conv_state is None else _f64(conv_state)
+    parts = [(xq, wq, 0, Cq), (xk, wk, Cq, Cq), (xv, wv, 2 * Cq, Cv)]
+    ys, states = [], []
+    for x, w, off, C in parts:
+        y, s = short_conv(x.reshape(T, C), w, cu_seqlens, None if cs is None else cs[:, :, off:off + C])
+        ys.append(y)
+        states.append(s)
+    q = l2_normalise_heads(ys[0], Hqk, Dk)
+    k = l2_normalise_heads(ys[1], Hqk, Dk)
+    v = ys[2].reshape(T, Hv, Dv)
+    return q, k, v, np.concatenate(states, axis=2)

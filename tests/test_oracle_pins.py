@@ -463,3 +463,75 @@ def test_slots_reject_bad_indices():
     for bad in ([0, 1, 2, 3, 9], [0, 1, 2, 3, -1], [0, 1, 2, 2, 4]):
         with pytest.raises(ValueError):
             oracle.decode_step_slots(q, k, v, g, b, pool, np.array(bad))
+
+
+# ---- front end: kernel-4 causal short convolution and per-head L2 norm ---------
+
+def test_short_conv_taps_are_delays():
+    """A filter with a single 1 in tap j delays the input by 3 - j tokens, with
+    zeros (no conv state) before each sequence start."""
+    r = rnd(41)
+    T, C = 11, 5
+    x = r.standard_normal((T, C))
+    cu = np.array([0, 4, 4, 11])              # an empty sequence in the middle
+    for j in range(4):
+        w = np.zeros((C, 4))
+        w[:, j] = 1.0
+        y, _ = oracle.short_conv(x, w, cu)
+        d = 3 - j
+        for a, b in ((0, 4), (4, 11)):
+            for t in range(a, b):
+                want = x[t - d] if t - d >= a else np.zeros(C)
+                assert np.array_equal(y[t], want)
+
+
+def test_short_conv_carry_equals_one_shot():
+    """Splitting a sequence anywhere and passing the conv state gives the
+    one-shot result, for every split point (including shorter than 3)."""
+    r = rnd(42)
+    T, C = 13, 4
+    x = r.standard_normal((T, C))
+    w = r.standard_normal((C, 4))
+    y_all, s_all = oracle.short_conv(x, w)
+    for cut in range(0, T + 1):
+        y1, s1 = oracle.short_conv(x[:cut], w)
+        y2, s2 = oracle.short_conv(x[cut:], w, conv_state=s1)
+        assert np.allclose(np.concatenate([y1, y2]), y_all, rtol=0, atol=1e-14)
+        assert np.array_equal(s2, s_all)
+
+
+def test_short_conv_is_linear_and_brute_force():
+    r = rnd(43)
+    T, C = 9, 3
+    x, x2 = r.standard_normal((T, C)), r.standard_normal((T, C))
+    w = r.standard_normal((C, 4))
+    s0 = r.standard_normal((1, 3, C))
+    y, _ = oracle.short_conv(x, w, conv_state=s0)
+    ext = np.concatenate([s0[0], x])
+    brute = np.array([[sum(w[c, j] * ext[t + j, c] for j in range(4)) for c in range(C)]
+                      for t in range(T)])
+    assert np.allclose(y, brute, rtol=1e-14, atol=1e-14)
+    ya, _ = oracle.short_conv(x + 2.0 * x2, w)
+    yb, _ = oracle.short_conv(x, w)
+    yc, _ = oracle.short_conv(x2, w)
+    assert np.allclose(ya, yb + 2.0 * yc, rtol=1e-13, atol=1e-13)
+
+
+def test_short_conv_norm_heads_are_unit_and_v_is_not_normalised():
+    r = rnd(44)
+    T, Hqk, Hv, D = 7, 2, 4, 8
+    xq, xk = r.standard_normal((T, Hqk, D)), r.standard_normal((T, Hqk, D))
+    xv = r.standard_normal((T, Hv, D))
+    wq, wk, wv = (r.standard_normal((Hqk * D, 4)), r.standard_normal((Hqk * D, 4)),
+                  r.standard_normal((Hv * D, 4)))
+    q, k, v, st = oracle.short_conv_norm(xq, xk, xv, wq, wk, wv)
+    assert np.allclose(np.linalg.norm(q, axis=-1), 1.0, rtol=1e-14)
+    assert np.allclose(np.linalg.norm(k, axis=-1), 1.0, rtol=1e-14)
+    yv, _ = oracle.short_conv(xv.reshape(T, -1), wv)
+    assert np.array_equal(v, yv.reshape(T, Hv, D))
+    yq, _ = oracle.short_conv(xq.reshape(T, -1), wq)
+    yq = yq.reshape(T, Hqk, D)
+    assert np.allclose(q * np.linalg.norm(yq, axis=-1, keepdims=True), yq, rtol=1e-13, atol=1e-14)
+    assert st.shape == (1, 3, 2 * Hqk * D + Hv * D)
+    assert np.array_equal(st[0, :, :Hqk * D], xq[-3:].reshape(3, -1))
+    assert np.array_equal(st[0, :, 2 * Hqk * D:], xv[-3:].reshape(3, -1))
