@@ -21,6 +21,7 @@ import threading
 import torch
 
 __all__ = ["gdn_prefill", "gdn_decode_step", "gdn_decode_step_bf16_state", "gdn_decode_step_slots",
+           "gdn_short_conv_norm",
            "gdn_prefill_workspace_bytes", "library",
            "GdnError", "LIB_PATH", "STATUS", "KERNELS"]
 
@@ -71,6 +72,9 @@ def library():
             lib.gdn_decode_step_slots.argtypes = [vp, vp, vp, ctypes.c_int, vp, vp, vp, i32, vp, vp,
                                                   i32, i32, i32, i32, i32, vp, vp, vp]
             lib.gdn_decode_step_slots.restype = ctypes.c_int
+            lib.gdn_short_conv_norm.argtypes = [vp, vp, vp, ctypes.c_int, vp, vp, vp, vp, vp, vp,
+                                                i32, i64, i32, i32, i32, i32, vp, vp, vp, vp, vp]
+            lib.gdn_short_conv_norm.restype = ctypes.c_int
             lib.gdn_prefill_workspace_bytes.argtypes = [i32, i64, i32, i32, i32, i32, i32]
             lib.gdn_prefill_workspace_bytes.restype = sz
             lib.gdn_prefill_ex_workspace_bytes.argtypes = [i32, i64, i32, i32, i32, i32, i32,
@@ -238,6 +242,54 @@ def gdn_decode_step_slots(q, k, v, g, beta, state_pool, slot_idx, reset=None, *,
     if rc != 0:
         raise GdnError(rc, "gdn_decode_step_slots")
     return o
+
+
+def gdn_short_conv_norm(xq, xk, xv, wq, wk, wv, cu_seqlens=None, conv_state=None, *,
+                        conv_state_out=None, output_conv_state=False, error_flag=None,
+                        stream=None):
+    """The mixer's kernel-4 causal convolution on the q, k, v channels, then q, k
+    normalised per head: returns (q, k, v[, conv_state_out]) ready for gdn_prefill.
+
+    xq, xk [T,Hqk,128], xv [T,Hv,128] (bf16 or fp32); wq, wk [Hqk*128,4], wv
+    [Hv*128,4] fp32; cu_seqlens int32 [N+1] or None; conv_state [N,3,C] fp32 or
+    None with C = 2*Hqk*128 + Hv*128 (q, k, v channels).  With
+    output_conv_state (or a conv_state_out tensor, which may be conv_state) the
+    new conv state is returned too."""
+    lib = library()
+    dev = xq.device
+    if dev.type != "cuda":
+        raise ValueError("gdn_short_conv_norm runs on CUDA tensors only")
+    T, Hqk, Dk = xq.shape
+    Hv, Dv = xv.shape[1], xv.shape[2]
+    if xq.dtype not in DTYPE:
+        raise ValueError(f"unsupported io dtype {xq.dtype}")
+    _check(xk, "xk", (T, Hqk, Dk), xq.dtype, dev)
+    _check(xv, "xv", (T, Hv, Dv), xq.dtype, dev)
+    _check(wq, "wq", (Hqk * Dk, 4), torch.float32, dev)
+    _check(wk, "wk", (Hqk * Dk, 4), torch.float32, dev)
+    _check(wv, "wv", (Hv * Dv, 4), torch.float32, dev)
+    if cu_seqlens is None:
+        N = 1
+    else:
+        N = cu_seqlens.shape[0] - 1
+        _check(cu_seqlens, "cu_seqlens", (N + 1,), torch.int32, dev)
+    C = 2 * Hqk * Dk + Hv * Dv
+    if conv_state is not None:
+        _check(conv_state, "conv_state", (N, 3, C), torch.float32, dev)
+    if conv_state_out is None and output_conv_state:
+        conv_state_out = torch.empty((N, 3, C), dtype=torch.float32, device=dev)
+    if conv_state_out is not None:
+        _check(conv_state_out, "conv_state_out", (N, 3, C), torch.float32, dev)
+    q = torch.empty_like(xq)
+    k = torch.empty_like(xk)
+    v = torch.empty_like(xv)
+    rc = lib.gdn_short_conv_norm(_ptr(xq), _ptr(xk), _ptr(xv), DTYPE[xq.dtype], _ptr(wq), _ptr(wk),
+                                 _ptr(wv), _ptr(conv_state), _ptr(conv_state_out),
+                                 _ptr(cu_seqlens), N, T, Hqk, Hv, Dk, Dv, _ptr(q), _ptr(k),
+                                 _ptr(v), _ptr(error_flag), _stream(stream))
+    if rc != 0:
+        raise GdnError(rc, "gdn_short_conv_norm")
+    return (q, k, v, conv_state_out) if conv_state_out is not None else (q, k, v)
 
 
 def gdn_decode_step_bf16_state(q, k, v, g, beta, state, *, o=None, error_flag=None, stream=None):

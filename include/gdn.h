@@ -319,6 +319,44 @@ GDN_API gdn_status gdn_decode_step_slots(const void *q, const void *k, const voi
                                          int32_t Hqk, int32_t Hv, int32_t Dk, int32_t Dv, void *o,
                                          int32_t *dev_error_flag, void *stream);
 
+/*
+ * gdn_short_conv_norm -- the front end of the DeltaNet mixer before the delta
+ * rule: the mixer's "kernel 4" convolution (page "Layouts híbridos: três
+ * DeltaNet, uma attention", section 01) on the q, k and v channels, then q and
+ * k normalised per (token, head).  Per channel c, causally within each
+ * sequence,
+ *     y[t, c] = w[c,0] x[t-3, c] + w[c,1] x[t-2, c] + w[c,2] x[t-1, c] + w[c,3] x[t, c],
+ * inputs before a sequence's first token taken from conv_state_in (or zero);
+ * q, k rows divided by their Euclidean norm (a zero row stays zero); no
+ * activation (the page names none).  Computed in fp32, outputs rounded once
+ * to io_dtype; the outputs are gdn_prefill's q, k, v.
+ *
+ *   xq, xk              [T][Hqk][Dk] io_dtype, the inputs of the q and k channels.
+ *   xv                  [T][Hv][Dv] io_dtype.
+ *   wq, wk              fp32 [Hqk*Dk][4] filters (tap 3 multiplies the current token).
+ *   wv                  fp32 [Hv*Dv][4].
+ *   conv_state_in       fp32 [N][3][2*Hqk*Dk + Hv*Dv] or NULL (zeros): per
+ *                       sequence, the three inputs before its first token,
+ *                       oldest first, channels in the order q, k, v.
+ *   conv_state_out      the same layout, or NULL to skip: each sequence's last
+ *                       three inputs (reaching into conv_state_in when it is
+ *                       shorter than 3), for a later call that continues it.
+ *                       May equal conv_state_in.
+ *   cu_seqlens, N, T    as gdn_prefill.
+ *   q, k, v             outputs [T][Hqk][Dk], [T][Hqk][Dk], [T][Hv][Dv] io_dtype;
+ *                       must not alias the inputs or each other.
+ * Supported: Dk = Dv = 128.  A malformed cu_seqlens is reported as
+ * GDN_ERR_BAD_SEQLENS (when conv_state_out is given); the outputs are then
+ * unspecified, but nothing outside the arrays is touched.
+ */
+GDN_API gdn_status gdn_short_conv_norm(const void *xq, const void *xk, const void *xv,
+                                       gdn_dtype io_dtype, const float *wq, const float *wk,
+                                       const float *wv, const float *conv_state_in,
+                                       float *conv_state_out, const int32_t *cu_seqlens, int32_t N,
+                                       int64_t T, int32_t Hqk, int32_t Hv, int32_t Dk, int32_t Dv,
+                                       void *q, void *k, void *v, int32_t *dev_error_flag,
+                                       void *stream);
+
 /* Human-readable name of a status code (static storage, never NULL). */
 GDN_API const char *gdn_status_string(gdn_status status);
 

@@ -235,6 +235,35 @@ def test_decode_slots_empty_batch_is_ok(lib):
     assert decode_slots(lib, N=0, S=0, slot=None) == 0
 
 
+def short_conv(lib, **kw):
+    a = dict(xq=P, xk=P + 0x1000, xv=P + 0x2000, dt=0, wq=P + 0x3000, wk=P + 0x4000,
+             wv=P + 0x5000, sin=None, sout=None, cu=None, N=1, T=64, Hqk=16, Hv=48, Dk=128,
+             Dv=128, q=P + 0x6000, k=P + 0x7000, v=P + 0x8000, err=None, stream=None)
+    a.update(kw)
+    return lib.gdn_short_conv_norm(a["xq"], a["xk"], a["xv"], a["dt"], a["wq"], a["wk"], a["wv"],
+                                   a["sin"], a["sout"], a["cu"], a["N"], a["T"], a["Hqk"], a["Hv"],
+                                   a["Dk"], a["Dv"], a["q"], a["k"], a["v"], a["err"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(xq=None), INVALID),
+    (dict(wv=None), INVALID),
+    (dict(xk=MIS), INVALID),
+    (dict(sin=MIS), INVALID),
+    (dict(q=P), INVALID),              # q aliases xq
+    (dict(v=P + 0x6000), INVALID),     # v aliases q
+    (dict(N=2), INVALID),              # no cu_seqlens with N != 1
+    (dict(dt=2), INVALID),
+    (dict(Dk=64, Dv=64), UNSUPPORTED),
+])
+def test_short_conv_norm_rejects(lib, kw, code):
+    assert short_conv(lib, **kw) == code
+
+
+def test_short_conv_norm_nothing_to_do_is_ok(lib):
+    assert short_conv(lib, N=0, T=0, cu=P + 0x9000) == 0
+
+
 def test_binding_refuses_cpu_tensors():
     import torch
     x = torch.zeros(4, 2, 16)

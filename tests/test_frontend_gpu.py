@@ -1,0 +1,121 @@
+"""GPU parity of gdn_short_conv_norm, the mixer's kernel-4 causal convolution
+with per-head q/k normalisation (page "Layouts híbridos: três DeltaNet, uma
+attention", section 01), against the fp64 oracle, and of the front end
+followed by the prefill.
+
+The kernel computes in fp32 and rounds once to the io dtype; the oracle
+computes in fp64.  Compared after the rounding: bf16 outputs equal the
+oracle's rounding of its own result for at least 99% of elements and are
+within one bf16 ulp plus fp32 error everywhere (the two round values that
+differ by fp32 arithmetic error, which can straddle a rounding boundary).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import gated_deltanet_04_b200 as gdn
+from gated_deltanet_04_b200 import inputs
+from tests.helpers import check_o, check_state
+
+pytestmark = pytest.mark.gpu
+DEV = torch.device("cuda:0")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    from gated_deltanet_04_b200 import build
+    build.build()
+
+
+def make(T, Hqk, Hv, seed, dtype=torch.bfloat16, N_state=None):
+    gen = torch.Generator().manual_seed(seed)
+    D = 128
+    xq = torch.randn(T, Hqk, D, generator=gen).to(dtype)
+    xk = torch.randn(T, Hqk, D, generator=gen).to(dtype)
+    xv = torch.randn(T, Hv, D, generator=gen).to(dtype)
+    wq = 0.5 * torch.randn(Hqk * D, 4, generator=gen)
+    wk = 0.5 * torch.randn(Hqk * D, 4, generator=gen)
+    wv = 0.5 * torch.randn(Hv * D, 4, generator=gen)
+    st = None
+    if N_state:
+        st = torch.randn(N_state, 3, (2 * Hqk + Hv) * D, generator=gen).to(dtype).float()
+    return xq, xk, xv, wq, wk, wv, st
+
+
+def check_rounded(gpu, ref64, what):
+    """bf16 output against the fp64 oracle value."""
+    g = gpu.double().numpy()
+    want = oracle.round_bf16(ref64)
+    _, e = np.frexp(want)
+    ulp = np.ldexp(1.0, e - 8)
+    slack = 2.0 ** -20 * np.max(np.abs(ref64))
+    diff = np.abs(g - want)
+    assert np.all(diff <= ulp * 1.0000001 + slack), f"{what}: more than 1 ulp off"
+    same = float(np.mean(diff == 0))
+    assert same >= 0.99, f"{what}: only {same:.4f} identical"
+
+
+def run(xq, xk, xv, wq, wk, wv, cu, st, out_state=True):
+    t = lambda x: None if x is None else x.to(DEV).contiguous()
+    flag = torch.zeros(4, dtype=torch.int32, device=DEV)
+    res = gdn.gdn_short_conv_norm(t(xq), t(xk), t(xv), t(wq), t(wk), t(wv),
+                                  None if cu is None else cu.to(torch.int32).to(DEV), t(st),
+                                  output_conv_state=out_state, error_flag=flag)
+    torch.cuda.synchronize()
+    assert int(flag[0]) == 0
+    return [None if r is None else r.cpu() for r in res]
+
+
+@pytest.mark.parametrize("with_state", [False, True])
+def test_short_conv_norm_packed(with_state):
+    lengths = [0, 1, 2, 3, 70, 129]
+    cu = inputs.cu_from_lengths(lengths)
+    T = int(cu[-1])
+    xq, xk, xv, wq, wk, wv, st = make(T, 2, 6, seed=8000, N_state=len(lengths) if with_state else None)
+    q, k, v, s_out = run(xq, xk, xv, wq, wk, wv, cu, st)
+    q_ref, k_ref, v_ref, s_ref = oracle.short_conv_norm(xq, xk, xv, wq, wk, wv, cu, st)
+    check_rounded(q, q_ref, "q")
+    check_rounded(k, k_ref, "k")
+    check_rounded(v, v_ref, "v")
+    assert torch.equal(s_out, torch.from_numpy(s_ref).float())  # raw inputs: exact
+
+
+def test_short_conv_norm_split_and_carry_equals_one_shot():
+    xq, xk, xv, wq, wk, wv, _ = make(200, 2, 6, seed=8100)
+    full = run(xq, xk, xv, wq, wk, wv, None, None)
+    for cut in (1, 2, 64, 131):
+        a = run(xq[:cut], xk[:cut], xv[:cut], wq, wk, wv, None, None)
+        b = run(xq[cut:], xk[cut:], xv[cut:], wq, wk, wv, None, a[3])
+        for i in range(3):
+            assert torch.equal(torch.cat([a[i], b[i]]), full[i]), (cut, i)
+        assert torch.equal(b[3], full[3])
+
+
+def test_short_conv_norm_fp32():
+    xq, xk, xv, wq, wk, wv, st = make(100, 2, 6, seed=8200, dtype=torch.float32, N_state=1)
+    q, k, v, _ = run(xq, xk, xv, wq, wk, wv, None, st)
+    q_ref, k_ref, v_ref, _ = oracle.short_conv_norm(xq, xk, xv, wq, wk, wv, None, st)
+    for g_, r_ in ((q, q_ref), (k, k_ref), (v, v_ref)):
+        rel = np.linalg.norm(g_.double().numpy() - r_) / np.linalg.norm(r_)
+        assert rel <= 1e-6, rel
+
+
+def test_front_end_then_prefill_layer_shape():
+    """Front end, then the prefill (pool kernel), on a 4096-token layer of the
+    benchmark's head shape, against the oracle's front end (rounded to bf16 as
+    the GPU stores it) followed by the oracle's recurrence."""
+    T, Hqk, Hv = 4096, 16, 48
+    xq, xk, xv, wq, wk, wv, _ = make(T, Hqk, Hv, seed=8300)
+    gen = torch.Generator().manual_seed(8301)
+    g = -inputs.G_SCALE_097 * torch.nn.functional.softplus(torch.randn(T, Hv, generator=gen))
+    beta = torch.sigmoid(torch.randn(T, Hv, generator=gen))
+    q, k, v = run(xq, xk, xv, wq, wk, wv, None, None, out_state=False)
+    o, sT = gdn.gdn_prefill(q.to(DEV), k.to(DEV), v.to(DEV), g.to(DEV), beta.to(DEV))
+    torch.cuda.synchronize()
+    q_ref, k_ref, v_ref, _ = oracle.short_conv_norm(xq, xk, xv, wq, wk, wv)
+    r = lambda a: torch.from_numpy(oracle.round_bf16(a))
+    o_ref, s_ref = oracle.recurrent(r(q_ref), r(k_ref), r(v_ref), g, beta)
+    check_o(o.cpu(), o_ref)
+    check_state(sT.cpu(), s_ref)
