@@ -400,6 +400,28 @@ def main():
     p_ms = dist.max(p_total / K)
     p_launch_ms = dist.max(sum(p_each) / K)
 
+    # ------------------------------------------------------- front end --
+    # the kernel-4 short convolution + q/k norm over the same layer's q, k, v
+    # channels (the prefill inputs serve as its raw inputs), with a conv state out
+    gen = torch.Generator(device=dev).manual_seed(1200)
+    Hqk_, Hv_ = inp["q"].shape[1], inp["v"].shape[1]
+    fw = [0.5 * torch.randn(H * 128, 4, generator=gen, device=dev) for H in (Hqk_, Hqk_, Hv_)]
+    fq, fk, fv = torch.empty_like(inp["q"]), torch.empty_like(inp["k"]), torch.empty_like(inp["v"])
+    fst = torch.empty((1, 3, (2 * Hqk_ + Hv_) * 128), dtype=torch.float32, device=dev)
+    lib = gdn.library()
+
+    def front_end():
+        lib.gdn_short_conv_norm(inp["q"].data_ptr(), inp["k"].data_ptr(), inp["v"].data_ptr(), 0,
+                                fw[0].data_ptr(), fw[1].data_ptr(), fw[2].data_ptr(), None,
+                                fst.data_ptr(), None, 1, T, Hqk_, Hv_, 128, 128, fq.data_ptr(),
+                                fk.data_ptr(), fv.data_ptr(), None, stream.cuda_stream)
+
+    f_total, _ = time_launches(front_end, K, W, dist, stream, sampler)
+    f_ms = dist.max(f_total / K)
+    f_bytes = 2 * sum(t.numel() * t.element_size() for t in (fq, fk, fv)) + \
+        sum(w.numel() * 4 for w in fw) + fst.numel() * 4
+    del fq, fk, fv, fw, fst
+
     # ----------------------------------------------------------- decode --
     dwl = inputs.WORKLOADS[DECODE_WL]
     layers = [inputs.make_decode_layer(l, device=dev) for l in range(dwl.layers)]
@@ -488,6 +510,14 @@ def main():
                              "frac_of_measured_copy": b_state_gbs / dist.world / peaks["hbm_gbs"],
                              "frac_of_8TBps": b_state_gbs / dist.world / 8000.0}}
 
+    front = {"value": weak_scaling_value(T, f_ms / 1e3, dist.world) / 1e6, "unit": "Mtok/s",
+             "ms_per_step": f_ms,
+             "note": "gdn_short_conv_norm (kernel-4 causal conv on q, k, v channels, q/k L2 "
+                     "norm) over the same 262,144-token layer",
+             "hbm": {"achieved": f_bytes / (f_ms / 1e3) / 1e9, "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": f_bytes / (f_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+                     "algorithmic_bytes_per_launch": f_bytes}}
+
     cpu = None
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
         tokens = 65536
@@ -510,9 +540,10 @@ def main():
                    "parallelism": f"replica x{dist.world} (no data-path collective)"},
         "roofline": roofline,
         "decode": decode,
+        "front_end": front,
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": K * (1 + dwl.layers + 1 + dwl.layers) + K * (0 if args.no_e2e else 1),
+        "gpu_launches": K * (1 + 2 + dwl.layers + 1 + dwl.layers) + K * (0 if args.no_e2e else 1),
         "clocks": clocks,
     }
     if dist.rank == 0:

@@ -10,16 +10,17 @@
 // names the convolution and nothing after it.
 //
 // The operation is bandwidth-bound (read x once, write q/k/v once).  A warp
-// owns one (token, head) row of 128 channels, 4 per lane; a CTA's 8 warps take
-// 8 consecutive tokens of one head, so the 3-token halo of each row is read
-// from L1 rather than HBM.  A second small kernel writes the new conv state.
+// owns the 128 channels of one head, 4 per lane, and slides over 32
+// consecutive tokens with its filters and the last three inputs in registers.
+// A second small kernel writes the new conv state.
 #include "gdn_internal.cuh"
 
 namespace gdn {
 namespace {
 
 constexpr int kFeD = 128;        // head dimension served
-constexpr int kFeTokens = 8;     // tokens per CTA (one per warp)
+constexpr int kFeWarps = 8;      // warps per CTA
+constexpr int kFeRun = 64;       // consecutive tokens per warp
 
 struct FeTensor {
     const void *x;               // [T][H][128] io dtype
@@ -74,55 +75,78 @@ __device__ __forceinline__ int fe_sequence(const int32_t *cu, int N, int64_t t) 
     return lo;
 }
 
-// grid: (ceil(T / 8), Hqk + Hqk + Hv): y walks the q heads, then the k heads,
-// then the v heads; block: 8 warps, one token each
-__global__ void __launch_bounds__(kFeTokens * 32)
+// grid: (Hqk + Hqk + Hv, ceil(T / 512)): x walks the q heads, then the k heads,
+// then the v heads, so CTAs launched together cover whole token rows.  Each of
+// the CTA's 8 warps slides over kFeRun consecutive tokens of one head, keeping
+// its lanes' 16 filter taps and the last three inputs in registers, so every
+// input row is read from memory once.
+__global__ void __launch_bounds__(kFeWarps * 32)
     gdn_short_conv_kernel(FeArgs a) {
-    const int yh = blockIdx.y, Hq = a.t[0].H;
+    const int yh = blockIdx.x, Hq = a.t[0].H;
+    const unsigned tb = blockIdx.y;
     const int z = yh < Hq ? 0 : yh < 2 * Hq ? 1 : 2;
     const FeTensor ft = z == 0 ? a.t[0] : z == 1 ? a.t[1] : a.t[2];
     const int h = yh - (z == 0 ? 0 : z == 1 ? Hq : 2 * Hq);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t t = (int64_t)blockIdx.x * kFeTokens + warp;
-    if (t >= a.T) return;
-    const int n = a.cu ? fe_sequence(a.cu, a.N, t) : 0;
-    const int64_t start = a.cu ? (int64_t)a.cu[n] : 0;
+    const int64_t t0 = ((int64_t)tb * kFeWarps + warp) * kFeRun;
+    if (t0 >= a.T) return;
+    const int64_t t1 = t0 + kFeRun < a.T ? t0 + kFeRun : a.T;
     const int c = h * kFeD + 4 * lane;  // this lane's first channel within the tensor
+    const int64_t row = (int64_t)ft.H * kFeD;  // elements per token
 
     float4 w[4];  // w[i]: the 4 taps of channel c + i
 #pragma unroll
     for (int i = 0; i < 4; ++i) w[i] = *reinterpret_cast<const float4 *>(ft.w + (int64_t)(c + i) * 4);
-    float y[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {  // tap j reads token t - 3 + j
-        const int64_t tp = t - 3 + j;
-        float4 xv = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (tp >= start && tp >= 0) {
-            xv = fe_load4(ft.x, tp * ft.H * kFeD + c, a.dtype);
-        } else if (a.state_in) {  // before the sequence: its carried inputs
-            const int64_t back = start - tp;  // 1 .. 3 for a well-formed cu_seqlens
-            if (back >= 1 && back <= 3)
-                xv = *reinterpret_cast<const float4 *>(a.state_in + ((int64_t)n * 3 + 3 - back) * a.C +
-                                                        ft.chan0 + c);
+
+    // the sequence of t0, and the inputs before t0 (oldest first): from x,
+    // from the sequence's carried conv state, or zero
+    int n = a.cu ? fe_sequence(a.cu, a.N, t0) : 0;
+    int64_t start = a.cu ? (int64_t)a.cu[n] : 0;
+    int64_t next = a.cu ? (int64_t)a.cu[n + 1] : a.T;
+    auto before = [&](int64_t tp) -> float4 {  // input at token tp < t of sequence n
+        if (tp >= start && tp >= 0) return fe_load4(ft.x, tp * row + c, a.dtype);
+        const int64_t back = start - tp;
+        if (a.state_in && back >= 1 && back <= 3)
+            return *reinterpret_cast<const float4 *>(a.state_in + ((int64_t)n * 3 + 3 - back) * a.C +
+                                                     ft.chan0 + c);
+        return make_float4(0.f, 0.f, 0.f, 0.f);
+    };
+    float4 h3 = before(t0 - 3), h2 = before(t0 - 2), h1 = before(t0 - 1);  // x[t-3], x[t-2], x[t-1]
+    for (int64_t t = t0; t < t1; ++t) {
+        if (t >= next) {  // a new sequence starts at t (skip empty ones)
+            while (n + 1 < a.N && (int64_t)a.cu[n + 1] <= t) ++n;
+            start = a.cu[n];
+            next = a.cu[n + 1];
+            h3 = before(t - 3);
+            h2 = before(t - 2);
+            h1 = before(t - 1);
         }
-        const float x4[4] = {xv.x, xv.y, xv.z, xv.w};
+        const float4 x0 = fe_load4(ft.x, t * row + c, a.dtype);
+        float y[4];
+        const float xs[4][4] = {{h3.x, h3.y, h3.z, h3.w}, {h2.x, h2.y, h2.z, h2.w},
+                                {h1.x, h1.y, h1.z, h1.w}, {x0.x, x0.y, x0.z, x0.w}};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            const float wj = j == 0 ? w[i].x : j == 1 ? w[i].y : j == 2 ? w[i].z : w[i].w;
-            y[i] = fmaf(wj, x4[i], y[i]);
+            y[i] = w[i].x * xs[0][i];
+            y[i] = fmaf(w[i].y, xs[1][i], y[i]);
+            y[i] = fmaf(w[i].z, xs[2][i], y[i]);
+            y[i] = fmaf(w[i].w, xs[3][i], y[i]);
         }
-    }
-    if (ft.norm) {  // divide the (token, head) row by its norm; a zero row stays zero
-        float ss = y[0] * y[0] + y[1] * y[1] + y[2] * y[2] + y[3] * y[3];
+        if (ft.norm) {  // divide the (token, head) row by its norm; a zero row stays zero
+            float ss = y[0] * y[0] + y[1] * y[1] + y[2] * y[2] + y[3] * y[3];
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-        const float nrm = sqrtf(ss);
-        if (nrm > 0.f) {
+            for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+            const float nrm = sqrtf(ss);
+            if (nrm > 0.f) {
 #pragma unroll
-            for (int i = 0; i < 4; ++i) y[i] = y[i] / nrm;
+                for (int i = 0; i < 4; ++i) y[i] = y[i] / nrm;
+            }
         }
+        fe_store4(ft.y, t * row + c, make_float4(y[0], y[1], y[2], y[3]), a.dtype);
+        h3 = h2;
+        h2 = h1;
+        h1 = x0;
     }
-    fe_store4(ft.y, t * ft.H * kFeD + c, make_float4(y[0], y[1], y[2], y[3]), a.dtype);
 }
 
 // New conv state: each sequence's last three inputs, per channel (one thread
@@ -174,7 +198,9 @@ extern "C" GDN_API gdn_status gdn_short_conv_norm(
     if (cu_seqlens == nullptr && N != 1) return GDN_ERR_INVALID_ARGUMENT;
     if (N == 0) return T == 0 ? GDN_OK : GDN_ERR_INVALID_ARGUMENT;
     if (Dk != gdn::kFeD || Dv != gdn::kFeD) return GDN_ERR_UNSUPPORTED;
-    if (T > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
+    // token blocks are the grid's y dimension (at most 65535 of 512 tokens)
+    if ((T + (int64_t)gdn::kFeWarps * gdn::kFeRun - 1) / ((int64_t)gdn::kFeWarps * gdn::kFeRun) > 65535)
+        return GDN_ERR_UNSUPPORTED;
     if (T > 0 && (!xq || !xk || !xv || !wq || !wk || !wv || !q || !k || !v))
         return GDN_ERR_INVALID_ARGUMENT;
     const void *ptrs[] = {xq, xk, xv, wq, wk, wv, conv_state_in, conv_state_out, cu_seqlens,
@@ -203,8 +229,9 @@ extern "C" GDN_API gdn_status gdn_short_conv_norm(
     a.dtype = io_dtype;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (T > 0) {
-        const dim3 grid((unsigned)((T + gdn::kFeTokens - 1) / gdn::kFeTokens), (unsigned)(2 * Hqk + Hv));
-        gdn::gdn_short_conv_kernel<<<grid, gdn::kFeTokens * 32, 0, s>>>(a);
+        const int64_t per_cta = (int64_t)gdn::kFeWarps * gdn::kFeRun;
+        const dim3 grid((unsigned)(2 * Hqk + Hv), (unsigned)((T + per_cta - 1) / per_cta));
+        gdn::gdn_short_conv_kernel<<<grid, gdn::kFeWarps * 32, 0, s>>>(a);
         if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
     }
     if (conv_state_out) {
