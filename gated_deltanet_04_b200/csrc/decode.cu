@@ -1,4 +1,4 @@
-// One-token decode update of the gated delta rule, in place on the fp32 state.
+// One-token decode update of the gated delta rule, in place on the state.
 //
 // Section 三 of "Qwen3.8-27B 架构深读: Gated DeltaNet 混合线性注意力与 262K
 // 长上下文": at inference every step does one fixed-size matrix update.  Per
@@ -10,19 +10,21 @@
 //     o_i   = S_i' . q = a (S_i . q) + u_i (k . q)
 // The state is streamed exactly once: every row is loaded, reduced against k
 // and q, rewritten and stored by the same lanes, so the kernel is bound by
-// HBM bandwidth on 2 * Dv * Dk * 4 bytes per (n, h).
+// HBM bandwidth on 2 * Dv * Dk * sizeof(state) bytes per (n, h).
 //
 // Two kernels:
-//  * Dk = Dv = 128 (the workload shape): a persistent kernel, one CTA per SM,
-//    that streams each 64 KB head state through shared memory with bulk TMA
-//    copies (3 states in flight per SM: loads of the next two overlap the
-//    update of the current one, and the updated state leaves by a bulk store
-//    while the next is computed).  Threads only read and write shared memory.
+//  * Dk = Dv = 128 (the workload shape): a persistent kernel that streams each
+//    head state through shared-memory stages with bulk TMA copies (loads of
+//    the next units overlap the update of the current one; the updated state
+//    leaves by a bulk store).  Threads only read and write shared memory.
 //    Each CTA takes a contiguous range of (n, h) units, so every SM streams
-//    one contiguous stretch of the states (measured ~1% faster on B200 than
-//    dealing units round-robin).  The units % grid left over are split into
-//    single rows across all CTAs, so no SM runs a whole extra unit at the end.
-//  * other head sizes: the direct kernel below.
+//    one contiguous stretch of the states, and the units % grid left over are
+//    split into single rows across all CTAs.  The 8 dot products of 4 rows
+//    (S.k and S.q) are summed over a warp in 9 shuffles.  Templated on the
+//    state type (fp32, or bfloat16 storage computed in fp32) and on pool
+//    decode (slot indices and reset flags); StagedCfg gives each state type
+//    its pipeline.
+//  * other head sizes: the direct kernel below (fp32 state).
 //
 // Direct kernel: one CTA of 8 warps per (n, h).  A row of Dk fp32 values is spread
 // over LPR = Dk/4 lanes as float4 (Dk = 128: a full warp per row, 512

@@ -10,17 +10,20 @@
 // names the convolution and nothing after it.
 //
 // The operation is bandwidth-bound (read x once, write q/k/v once).  A warp
-// owns the 128 channels of one head, 4 per lane, and slides over 32
-// consecutive tokens with its filters and the last three inputs in registers.
-// A second small kernel writes the new conv state.
+// owns the 128 channels of one head, 4 per lane, and slides over 128
+// consecutive tokens with its filters and the last three inputs in registers,
+// its input rows streaming through a per-warp cp.async double buffer.  A
+// second small kernel writes the new conv state.
 #include "gdn_internal.cuh"
+#include "sm100.cuh"
 
 namespace gdn {
 namespace {
 
 constexpr int kFeD = 128;        // head dimension served
 constexpr int kFeWarps = 8;      // warps per CTA
-constexpr int kFeRun = 64;       // consecutive tokens per warp
+constexpr int kFeRun = 128;      // consecutive tokens per warp
+constexpr int kFeBlk = 16;       // rows per cp.async block (two blocks buffered per warp)
 
 struct FeTensor {
     const void *x;               // [T][H][128] io dtype
@@ -75,13 +78,22 @@ __device__ __forceinline__ int fe_sequence(const int32_t *cu, int N, int64_t t) 
     return lo;
 }
 
-// grid: (Hqk + Hqk + Hv, ceil(T / 512)): x walks the q heads, then the k heads,
+// grid: (Hqk + Hqk + Hv, ceil(T / 1024)): x walks the q heads, then the k heads,
 // then the v heads, so CTAs launched together cover whole token rows.  Each of
 // the CTA's 8 warps slides over kFeRun consecutive tokens of one head, keeping
 // its lanes' 16 filter taps and the last three inputs in registers, so every
-// input row is read from memory once.
+// input row is read from memory once.  The rows come through the warp's own
+// double buffer in shared memory, kFeBlk rows at a time by cp.async, so a
+// warp has the next kFeBlk rows in flight while it computes the current ones.
+__device__ __forceinline__ void fe_cp_async16(void *smem, const void *gmem) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sm100::smem_u32(smem)),
+                 "l"(reinterpret_cast<uint64_t>(gmem))
+                 : "memory");
+}
+
 __global__ void __launch_bounds__(kFeWarps * 32)
     gdn_short_conv_kernel(FeArgs a) {
+    extern __shared__ __align__(16) uint8_t fe_smem[];
     const int yh = blockIdx.x, Hq = a.t[0].H;
     const unsigned tb = blockIdx.y;
     const int z = yh < Hq ? 0 : yh < 2 * Hq ? 1 : 2;
@@ -93,6 +105,23 @@ __global__ void __launch_bounds__(kFeWarps * 32)
     const int64_t t1 = t0 + kFeRun < a.T ? t0 + kFeRun : a.T;
     const int c = h * kFeD + 4 * lane;  // this lane's first channel within the tensor
     const int64_t row = (int64_t)ft.H * kFeD;  // elements per token
+    const int esz = a.dtype == GDN_DTYPE_BF16 ? 2 : 4;
+    const int rb = kFeD * esz;                  // bytes of this head's slice of a row
+    uint8_t *wbuf = fe_smem + (size_t)warp * 2 * kFeBlk * rb;  // [2][kFeBlk][rb]
+
+    // rows t .. t + kFeBlk - 1 (those < t1) of this head into buffer k
+    auto issue = [&](int64_t tstart, int k) {
+        const int parts = rb / 16;              // 16-byte pieces per row slice
+        for (int idx = lane; idx < kFeBlk * parts; idx += 32) {
+            const int r = idx / parts, pc = idx % parts;
+            if (tstart + r < t1)
+                fe_cp_async16(wbuf + ((size_t)k * kFeBlk + r) * rb + pc * 16,
+                              static_cast<const uint8_t *>(ft.x) +
+                                  ((tstart + r) * row + (int64_t)h * kFeD) * esz + pc * 16);
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    issue(t0, 0);
 
     float4 w[4];  // w[i]: the 4 taps of channel c + i
 #pragma unroll
@@ -112,40 +141,53 @@ __global__ void __launch_bounds__(kFeWarps * 32)
         return make_float4(0.f, 0.f, 0.f, 0.f);
     };
     float4 h3 = before(t0 - 3), h2 = before(t0 - 2), h1 = before(t0 - 1);  // x[t-3], x[t-2], x[t-1]
-    for (int64_t t = t0; t < t1; ++t) {
-        if (t >= next) {  // a new sequence starts at t (skip empty ones)
-            while (n + 1 < a.N && (int64_t)a.cu[n + 1] <= t) ++n;
-            start = a.cu[n];
-            next = a.cu[n + 1];
-            h3 = before(t - 3);
-            h2 = before(t - 2);
-            h1 = before(t - 1);
+    int k = 0;
+    for (int64_t tb0 = t0; tb0 < t1; tb0 += kFeBlk, k ^= 1) {
+        if (tb0 + kFeBlk < t1) {  // the next block streams in while this one is computed
+            issue(tb0 + kFeBlk, k ^ 1);
+            asm volatile("cp.async.wait_group 1;" ::: "memory");
+        } else {
+            asm volatile("cp.async.wait_group 0;" ::: "memory");
         }
-        const float4 x0 = fe_load4(ft.x, t * row + c, a.dtype);
-        float y[4];
-        const float xs[4][4] = {{h3.x, h3.y, h3.z, h3.w}, {h2.x, h2.y, h2.z, h2.w},
-                                {h1.x, h1.y, h1.z, h1.w}, {x0.x, x0.y, x0.z, x0.w}};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            y[i] = w[i].x * xs[0][i];
-            y[i] = fmaf(w[i].y, xs[1][i], y[i]);
-            y[i] = fmaf(w[i].z, xs[2][i], y[i]);
-            y[i] = fmaf(w[i].w, xs[3][i], y[i]);
-        }
-        if (ft.norm) {  // divide the (token, head) row by its norm; a zero row stays zero
-            float ss = y[0] * y[0] + y[1] * y[1] + y[2] * y[2] + y[3] * y[3];
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-            const float nrm = sqrtf(ss);
-            if (nrm > 0.f) {
-#pragma unroll
-                for (int i = 0; i < 4; ++i) y[i] = y[i] / nrm;
+        __syncwarp();
+        const int nr = t1 - tb0 < kFeBlk ? (int)(t1 - tb0) : kFeBlk;
+        for (int r = 0; r < nr; ++r) {
+            const int64_t t = tb0 + r;
+            if (t >= next) {  // a new sequence starts at t (skip empty ones)
+                while (n + 1 < a.N && (int64_t)a.cu[n + 1] <= t) ++n;
+                start = a.cu[n];
+                next = a.cu[n + 1];
+                h3 = before(t - 3);
+                h2 = before(t - 2);
+                h1 = before(t - 1);
             }
+            const float4 x0 = fe_load4(wbuf + ((size_t)k * kFeBlk + r) * rb, 4 * lane, a.dtype);
+            float y[4];
+            const float xs[4][4] = {{h3.x, h3.y, h3.z, h3.w}, {h2.x, h2.y, h2.z, h2.w},
+                                    {h1.x, h1.y, h1.z, h1.w}, {x0.x, x0.y, x0.z, x0.w}};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                y[i] = w[i].x * xs[0][i];
+                y[i] = fmaf(w[i].y, xs[1][i], y[i]);
+                y[i] = fmaf(w[i].z, xs[2][i], y[i]);
+                y[i] = fmaf(w[i].w, xs[3][i], y[i]);
+            }
+            if (ft.norm) {  // divide the (token, head) row by its norm; a zero row stays zero
+                float ss = y[0] * y[0] + y[1] * y[1] + y[2] * y[2] + y[3] * y[3];
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+                const float nrm = sqrtf(ss);
+                if (nrm > 0.f) {
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) y[i] = y[i] / nrm;
+                }
+            }
+            fe_store4(ft.y, t * row + c, make_float4(y[0], y[1], y[2], y[3]), a.dtype);
+            h3 = h2;
+            h2 = h1;
+            h1 = x0;
         }
-        fe_store4(ft.y, t * row + c, make_float4(y[0], y[1], y[2], y[3]), a.dtype);
-        h3 = h2;
-        h2 = h1;
-        h1 = x0;
+        __syncwarp();  // this buffer is refilled by the next block's issue
     }
 }
 
@@ -198,7 +240,7 @@ extern "C" GDN_API gdn_status gdn_short_conv_norm(
     if (cu_seqlens == nullptr && N != 1) return GDN_ERR_INVALID_ARGUMENT;
     if (N == 0) return T == 0 ? GDN_OK : GDN_ERR_INVALID_ARGUMENT;
     if (Dk != gdn::kFeD || Dv != gdn::kFeD) return GDN_ERR_UNSUPPORTED;
-    // token blocks are the grid's y dimension (at most 65535 of 512 tokens)
+    // token blocks are the grid's y dimension (at most 65535 of 1024 tokens)
     if ((T + (int64_t)gdn::kFeWarps * gdn::kFeRun - 1) / ((int64_t)gdn::kFeWarps * gdn::kFeRun) > 65535)
         return GDN_ERR_UNSUPPORTED;
     if (T > 0 && (!xq || !xk || !xv || !wq || !wk || !wv || !q || !k || !v))
@@ -231,7 +273,12 @@ extern "C" GDN_API gdn_status gdn_short_conv_norm(
     if (T > 0) {
         const int64_t per_cta = (int64_t)gdn::kFeWarps * gdn::kFeRun;
         const dim3 grid((unsigned)(2 * Hqk + Hv), (unsigned)((T + per_cta - 1) / per_cta));
-        gdn::gdn_short_conv_kernel<<<grid, gdn::kFeWarps * 32, 0, s>>>(a);
+        const size_t smem = (size_t)gdn::kFeWarps * 2 * gdn::kFeBlk * gdn::kFeD *
+                            (io_dtype == GDN_DTYPE_BF16 ? 2 : 4);
+        if (cudaFuncSetAttribute(gdn::gdn_short_conv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)smem) != cudaSuccess)
+            return GDN_ERR_CUDA;
+        gdn::gdn_short_conv_kernel<<<grid, gdn::kFeWarps * 32, smem, s>>>(a);
         if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
     }
     if (conv_state_out) {
