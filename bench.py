@@ -61,7 +61,9 @@ def parse():
     p.add_argument("--case", default=None,
                    help="profiling mode: run one operation of a named workload (layer4k, "
                         "long256k, varlen32: one gdn_prefill call; decode256: one layer's "
-                        "gdn_decode_step; decode256_bf16: the same with a bfloat16 state) "
+                        "gdn_decode_step; decode256_bf16: the same with a bfloat16 state; "
+                        "frontend16k, frontend256k: gdn_short_conv_norm on a 16,384- or "
+                        "262,144-token layer) "
                         "W + K times and print its per-call time; no bench line")
     p.add_argument("--kernel", default="auto", choices=["auto", "pool", "cluster", "single_cta", "recurrent"],
                    help="prefill kernel for --case")
@@ -336,6 +338,20 @@ def run_case(args):
         L = inputs.make_decode_layer(0, device=dev)
         out = torch.empty_like(L["v"])
         fn = lambda: gdn.gdn_decode_step(L["q"], L["k"], L["v"], L["g"], L["beta"], L["state"], o=out)
+    elif args.case in ("frontend16k", "frontend256k"):
+        inp = (inputs.make_prefill("layer4k", device=dev, T=16384) if args.case == "frontend16k"
+               else inputs.make_prefill("long256k", device=dev))
+        gen = torch.Generator(device=dev).manual_seed(1200)
+        Hqk_, Hv_ = inp["q"].shape[1], inp["v"].shape[1]
+        fw = [0.5 * torch.randn(H * 128, 4, generator=gen, device=dev) for H in (Hqk_, Hqk_, Hv_)]
+        fo = [torch.empty_like(inp[key]) for key in ("q", "k", "v")]
+        lib = gdn.library()
+        Tn = inp["q"].shape[0]
+        fn = lambda: lib.gdn_short_conv_norm(inp["q"].data_ptr(), inp["k"].data_ptr(), inp["v"].data_ptr(),
+                                             0, fw[0].data_ptr(), fw[1].data_ptr(), fw[2].data_ptr(),
+                                             None, None, None, 1, Tn, Hqk_, Hv_, 128, 128,
+                                             fo[0].data_ptr(), fo[1].data_ptr(), fo[2].data_ptr(),
+                                             None, stream.cuda_stream)
     elif args.case == "decode256_bf16":
         L = inputs.make_decode_layer(0, device=dev)
         out = torch.empty_like(L["v"])
