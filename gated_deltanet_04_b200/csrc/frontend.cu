@@ -110,10 +110,10 @@ __global__ void __launch_bounds__(kFeWarps * 32)
     uint8_t *wbuf = fe_smem + (size_t)warp * 2 * kFeBlk * rb;  // [2][kFeBlk][rb]
 
     // rows t .. t + kFeBlk - 1 (those < t1) of this head into buffer k
+    const int lg_parts = esz == 2 ? 4 : 5;      // log2 of the 16-byte pieces per row slice
     auto issue = [&](int64_t tstart, int k) {
-        const int parts = rb / 16;              // 16-byte pieces per row slice
-        for (int idx = lane; idx < kFeBlk * parts; idx += 32) {
-            const int r = idx / parts, pc = idx % parts;
+        for (int idx = lane; idx < (kFeBlk << lg_parts); idx += 32) {
+            const int r = idx >> lg_parts, pc = idx & ((1 << lg_parts) - 1);
             if (tstart + r < t1)
                 fe_cp_async16(wbuf + ((size_t)k * kFeBlk + r) * rb + pc * 16,
                               static_cast<const uint8_t *>(ft.x) +
@@ -176,10 +176,10 @@ __global__ void __launch_bounds__(kFeWarps * 32)
                 float ss = y[0] * y[0] + y[1] * y[1] + y[2] * y[2] + y[3] * y[3];
 #pragma unroll
                 for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-                const float nrm = sqrtf(ss);
-                if (nrm > 0.f) {
+                if (ss > 0.f) {
+                    const float inv = 1.f / sqrtf(ss);
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) y[i] = y[i] / nrm;
+                    for (int i = 0; i < 4; ++i) y[i] *= inv;
                 }
             }
             fe_store4(ft.y, t * row + c, make_float4(y[0], y[1], y[2], y[3]), a.dtype);
