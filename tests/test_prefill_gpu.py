@@ -170,7 +170,7 @@ def test_kernels_agree_with_each_other():
         check_state(s2, s64.double())
 
 
-@pytest.mark.parametrize("kernel", ["cluster", "single_cta"])  # 1536 units: over the pool's 64
+@pytest.mark.parametrize("kernel", ["cluster", "single_cta"])  # 1536 units: over the pool kernel's 64-unit limit
 def test_varlen32_split_and_carry(kernel):
     """32 packed sequences, lengths U[512,16384], nonzero initial states; every
     sequence split at a random point and run as two calls carrying the state
