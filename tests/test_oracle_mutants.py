@@ -3,10 +3,13 @@
 Each case copies oracle/ to a temporary directory, plants one mistake in the
 C source (dropped decay, wrong sign of the delta write, transposed recall,
 read-out with the wrong vector, wrong head grouping, inverted decay mask,
-missing cumulative decay in W, strict instead of inclusive output mask),
-rebuilds it and runs tests/test_oracle_pins.py against the mutant.  At least
-one pin must fail for every mutant.  Mistakes are planted in the oracle on
-the CPU only.
+missing cumulative decay in W, strict instead of inclusive output mask) or in
+the Python functions (bfloat16 rounding with ties up or one bit short, a
+reset that keeps the old state, a step not written back to its slot, conv
+taps in reverse order, a conv state that is ignored, v normalised like q and
+k), rebuilds it and runs tests/test_oracle_pins.py against the mutant.  At
+least one pin must fail for every mutant.  Mistakes are planted in the oracle
+on the CPU only.
 """
 import os
 import shutil
@@ -33,11 +36,26 @@ MUTANTS = {
                                  "for (int64_t i = 0; i < r; ++i) {\n                                double qk"),
 }
 
+# mistakes in the Python functions of oracle/__init__.py
+MUTANTS_PY = {
+    "bf16_ties_up": ("return np.ldexp(np.rint(np.ldexp(m, 8)), e - 8)",
+                     "return np.ldexp(np.floor(np.ldexp(m, 8) + 0.5), e - 8)"),
+    "bf16_seven_bits": ("return np.ldexp(np.rint(np.ldexp(m, 8)), e - 8)",
+                        "return np.ldexp(np.rint(np.ldexp(m, 7)), e - 7)"),
+    "slots_reset_ignored": ("states[rs != 0] = 0.0", "states[rs != 0] = states[rs != 0]"),
+    "slots_not_written_back": ("    pool[idx] = new\n", "    pool[idx] = states\n"),
+    "conv_taps_reversed": ("y[cu[n] + t] += w[:, j] * ext[t + j]", "y[cu[n] + t] += w[:, 3 - j] * ext[t + j]"),
+    "conv_state_ignored": ("st = np.zeros((N, 3, C)) if conv_state is None else _f64(conv_state)",
+                           "st = np.zeros((N, 3, C))"),
+    "conv_v_normalised": ("v = ys[2].reshape(T, Hv, Dv)", "v = l2_normalise_heads(ys[2], Hv, Dv)"),
+}
 
-@pytest.mark.parametrize("name", sorted(MUTANTS))
+
+@pytest.mark.parametrize("name", sorted(MUTANTS) + sorted(MUTANTS_PY))
 def test_pins_catch_mutant(name, tmp_path):
-    src = open(os.path.join(ROOT, "oracle", "gdn_oracle.c")).read()
-    old, new = MUTANTS[name]
+    fname = "gdn_oracle.c" if name in MUTANTS else "__init__.py"
+    src = open(os.path.join(ROOT, "oracle", fname)).read()
+    old, new = MUTANTS[name] if name in MUTANTS else MUTANTS_PY[name]
     assert src.count(old) == 1, f"mutation site for {name} not found exactly once"
     work = tmp_path / "repo"
     shutil.copytree(os.path.join(ROOT, "oracle"), work / "oracle",
@@ -48,7 +66,7 @@ def test_pins_catch_mutant(name, tmp_path):
     for f in ("conftest.py", "test_oracle_pins.py"):
         shutil.copy(os.path.join(ROOT, "tests", f), work / "tests" / f)
     shutil.copytree(os.path.join(ROOT, "tests", "golden"), work / "tests" / "golden")
-    (work / "oracle" / "gdn_oracle.c").write_text(src.replace(old, new))
+    (work / "oracle" / fname).write_text(src.replace(old, new))
     r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-p", "no:cacheprovider",
                         "tests/test_oracle_pins.py"], cwd=work, capture_output=True, text=True,
                        timeout=600)
