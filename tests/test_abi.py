@@ -282,3 +282,34 @@ def test_product_path_never_imports_the_oracle():
                 txt = open(os.path.join(dirpath, f), encoding="utf-8").read()
                 assert "import oracle" not in txt and "from oracle" not in txt, f
                 assert "gdn_oracle" not in txt, f
+
+
+def test_header_compiles_as_c99_and_links(tmp_path):
+    """A plain C caller: include/gdn.h compiles as C99 with warnings as errors,
+    the program links against libgdn.so, and the host-only calls work (no GPU:
+    an argument error returns before any CUDA call)."""
+    import subprocess
+    gdn_build.build()
+    src = tmp_path / "caller.c"
+    src.write_text(r"""
+#include <stdio.h>
+#include <string.h>
+#include "gdn.h"
+int main(void) {
+    if (gdn_version() < 10000) return 1;
+    if (strcmp(gdn_status_string(GDN_ERR_BAD_SLOT), "GDN_ERR_BAD_SLOT") != 0) return 2;
+    /* invalid enum: rejected synchronously */
+    if (gdn_decode_step_order(0, 0, 0, GDN_DTYPE_BF16, 0, 0, 0, 1, 1, 1, 128, 128, 0, 0, 0,
+                              (gdn_order)7) != GDN_ERR_INVALID_ARGUMENT) return 3;
+    if (gdn_prefill_workspace_bytes(1, 4096, 16, 48, 128, 128, 64) == 0) return 4;
+    printf("ok\n");
+    return 0;
+}
+""")
+    lib_dir = os.path.join(ROOT, "gated_deltanet_04_b200")
+    exe = tmp_path / "caller"
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    str(src), "-o", str(exe), "-L", lib_dir, "-lgdn", "-Wl,-rpath," + lib_dir],
+                   check=True, capture_output=True, text=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0 and r.stdout.strip() == "ok", (r.returncode, r.stdout, r.stderr)
