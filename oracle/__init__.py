@@ -61,7 +61,7 @@ def _load():
                                                  ctypes.c_void_p, dp, dp]
             lib.gdn_oracle_recurrent.restype = ctypes.c_int
             lib.gdn_oracle_chunked.argtypes = [dp, dp, dp, dp, dp, dp, i64p, i64, i64, i64, i64,
-                                               i64, i64, i64, dp, dp]
+                                               i64, i64, i64, ctypes.c_int, dp, dp]
             lib.gdn_oracle_chunked.restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -127,15 +127,17 @@ def recurrent(q, k, v, gate, beta, s0=None, cu_seqlens=None, *, order=ORDER_STAN
     return o, sT
 
 
-def chunked(q, k, v, g, beta, s0=None, cu_seqlens=None, *, chunk=64):
-    """fp64 chunk-parallel form (standard order, log gate). Same shapes as recurrent()."""
+def chunked(q, k, v, g, beta, s0=None, cu_seqlens=None, *, chunk=64, order=ORDER_STANDARD):
+    """fp64 chunk-parallel form (log gate), in either step order: the
+    recall-first order moves token r's recall decay from Gamma_r to
+    Gamma_{r-1} in A and W.  Same shapes as recurrent()."""
     lib = _load()
     q, k, v, g, beta, s0, cu, N, T, Hqk, Hv, Dk, Dv = _prep(q, k, v, g, beta, s0, cu_seqlens)
     o = np.zeros((T, Hv, Dv), dtype=np.float64)
     sT = np.zeros((N, Hv, Dv, Dk), dtype=np.float64)
     rc = lib.gdn_oracle_chunked(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(s0),
                                 _ptr(cu, ctypes.c_int64), N, T, Hqk, Hv, Dk, Dv, int(chunk),
-                                _ptr(o), _ptr(sT))
+                                int(order), _ptr(o), _ptr(sT))
     if rc != 0:
         raise ValueError(f"gdn_oracle_chunked failed with code {rc}")
     return o, sT

@@ -174,15 +174,21 @@ int gdn_oracle_recurrent(const double *q, const double *k, const double *v,
  *
  * The unroll behind it: u_r = b_r (v_r - a_r S_{r-1} k_r) and
  * S_r = Gamma_r S0 + sum_{i<=r} (Gamma_r / Gamma_i) u_i k_i^T.
- * Only the log gate and the standard order are supported.
+ *
+ * order == ORACLE_ORDER_ILLUSTRATIVE (recall before the decay): u_r = b_r (v_r -
+ * S_{r-1} k_r) with the same recursion in u, so only token r's recall terms
+ * change, from Gamma_r to Gamma_{r-1} (Gamma_{-1} = 1): A's row factor
+ * becomes exp(gamma_{r-1} - gamma_i) and W = Tm diag(b Gamma_{.-1}) K.
+ * Only the log gate is supported.
  */
 int gdn_oracle_chunked(const double *q, const double *k, const double *v,
                        const double *g, const double *beta, const double *s0,
                        const int64_t *cu_seqlens, int64_t N, int64_t T,
                        int64_t Hqk, int64_t Hv, int64_t Dk, int64_t Dv,
-                       int64_t C, double *o, double *sT) {
+                       int64_t C, int order, double *o, double *sT) {
     if (N < 0 || T < 0 || Hqk <= 0 || Hv <= 0 || Dk <= 0 || Dv <= 0 || C <= 0)
         return -1;
+    if (order != ORACLE_ORDER_STANDARD && order != ORACLE_ORDER_ILLUSTRATIVE) return -1;
     if (Hv % Hqk != 0) return -1;
     if (check_seqlens(cu_seqlens, N, T)) return -2;
     const int64_t G = Hv / Hqk;
@@ -222,6 +228,9 @@ int gdn_oracle_chunked(const double *q, const double *k, const double *v,
                         acc += GB(g, r);
                         gam[r] = acc;
                     }
+/* the log-decay of token r's recall: gamma_r, or gamma_{r-1} (0 for r = 0)
+   when the recall is taken before the decay */
+#define GREC(r) (order == ORACLE_ORDER_ILLUSTRATIVE ? ((r) > 0 ? gam[(r) - 1] : 0.0) : gam[r])
                     /* A = strictly lower part of diag(b)(K K^T (.) M) */
                     for (int64_t r = 0; r < L; ++r)
                         for (int64_t i = 0; i < L; ++i) {
@@ -230,7 +239,7 @@ int gdn_oracle_chunked(const double *q, const double *k, const double *v,
                                 double kk = 0.0;
                                 for (int64_t d = 0; d < Dk; ++d)
                                     kk += KR(r)[d] * KR(i)[d];
-                                val = GB(beta, r) * kk * exp(gam[r] - gam[i]);
+                                val = GB(beta, r) * kk * exp(GREC(r) - gam[i]);
                             }
                             A[r * C + i] = val;
                         }
@@ -249,7 +258,7 @@ int gdn_oracle_chunked(const double *q, const double *k, const double *v,
                             double s = 0.0;
                             for (int64_t i = 0; i <= r; ++i)
                                 s += Tm[r * C + i] * GB(beta, i) *
-                                     exp(gam[i]) * KR(i)[d];
+                                     exp(GREC(i)) * KR(i)[d];
                             W[r * Dk + d] = s;
                         }
                         for (int64_t e = 0; e < Dv; ++e) {
@@ -296,6 +305,7 @@ int gdn_oracle_chunked(const double *q, const double *k, const double *v,
 #undef QR
 #undef VR
 #undef GB
+#undef GREC
                 }
                 if (sT)
                     memcpy(sT + (n * Hv + h) * Dv * Dk, S,

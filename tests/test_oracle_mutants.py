@@ -28,10 +28,13 @@ MUTANTS = {
                           "acc += S[d * Dk + i] * kt[d];\n                r[i] = acc;\n            }\n        }"),
     "readout_with_key": ("acc += S[i * Dk + d] * qt[d];", "acc += S[i * Dk + d] * kt[d];"),
     "head_group_modulo": ("const int64_t j = h / (Hv / Hqk);", "const int64_t j = h % Hqk;"),
-    "chunk_mask_inverted": ("val = GB(beta, r) * kk * exp(gam[r] - gam[i]);",
-                            "val = GB(beta, r) * kk * exp(gam[i] - gam[r]);"),
-    "chunk_W_without_decay": ("GB(beta, i) *\n                                     exp(gam[i]) * KR(i)[d];",
+    "chunk_mask_inverted": ("val = GB(beta, r) * kk * exp(GREC(r) - gam[i]);",
+                            "val = GB(beta, r) * kk * exp(gam[i] - GREC(r));"),
+    "chunk_W_without_decay": ("GB(beta, i) *\n                                     exp(GREC(i)) * KR(i)[d];",
                               "GB(beta, i) *\n                                     1.0 * KR(i)[d];"),
+    "chunk_recall_first_uses_gamma_r": (
+        "(order == ORACLE_ORDER_ILLUSTRATIVE ? ((r) > 0 ? gam[(r) - 1] : 0.0) : gam[r])",
+        "(gam[r])"),
     "chunk_output_mask_strict": ("for (int64_t i = 0; i <= r; ++i) {\n                                double qk",
                                  "for (int64_t i = 0; i < r; ++i) {\n                                double qk"),
 }

@@ -535,3 +535,20 @@ def test_short_conv_norm_heads_are_unit_and_v_is_not_normalised():
     assert st.shape == (1, 3, 2 * Hqk * D + Hv * D)
     assert np.array_equal(st[0, :, :Hqk * D], xq[-3:].reshape(3, -1))
     assert np.array_equal(st[0, :, 2 * Hqk * D:], xv[-3:].reshape(3, -1))
+
+
+@pytest.mark.parametrize("C", [1, 4, 16, 64])
+def test_chunked_recall_first_equals_recurrent(C):
+    """The chunked form in the recall-first order (Gamma_{r-1} in A and W)
+    reaches the recall-first recurrence, with an entering state, packed
+    sequences and decays from weak to strong; and differs from the standard
+    order."""
+    q, k, v, g, beta, s0 = make(51, T=70, N=2, s0_std=0.5)
+    cu = np.array([0, 33, 70])
+    g = g * 3.0  # stronger decay: the two orders differ more
+    o_r, s_r = oracle.recurrent(q, k, v, g, beta, s0, cu, order=ORDER_ILLUSTRATIVE)
+    o_c, s_c = oracle.chunked(q, k, v, g, beta, s0, cu, chunk=C, order=ORDER_ILLUSTRATIVE)
+    assert np.allclose(o_c, o_r, rtol=1e-10, atol=1e-11)
+    assert np.allclose(s_c, s_r, rtol=1e-10, atol=1e-11)
+    o_std, _ = oracle.chunked(q, k, v, g, beta, s0, cu, chunk=C)
+    assert np.abs(o_std - o_r).max() > 1e-3
