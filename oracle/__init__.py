@@ -279,3 +279,43 @@ def short_conv_norm(xq, xk, xv, wq, wk, wv, cu_seqlens=None, conv_state=None):
     k = l2_normalise_heads(ys[1], Hqk, Dk)
     v = ys[2].reshape(T, Hv, Dv)
     return q, k, v, np.concatenate(states, axis=2)
+
+
+def chunk_state_maps(k, v, g, beta, *, chunk=64, head_k=0, head_v=0):
+    """The chunk step of one (sequence, head) as an affine map of the entering
+    state, for a context-parallel scan over a sequence's chunks.
+
+    With the chunk quantities of chunked() (T = (I + A)^-1, W = T diag(b Gamma) K,
+    U~ = T diag(b) V, e_C = Gamma_C / Gamma), the state leaving a chunk is
+        S' = Gamma_C S + (U~ - W S^T)^T diag(e_C) K = S A_c + B_c,
+        A_c = Gamma_C I - W^T diag(e_C) K   (Dk x Dk),
+        B_c = U~^T diag(e_C) K              (Dv x Dk).
+    k [T,Hqk,Dk], v [T,Hv,Dv], g, beta [T,Hv] of one sequence; head_k / head_v
+    pick the heads.  Returns a list of (A_c, B_c), float64, one per chunk.
+    """
+    k, v, g, beta = _f64(k)[:, head_k], _f64(v)[:, head_v], _f64(g)[:, head_v], _f64(beta)[:, head_v]
+    T, Dk = k.shape
+    maps = []
+    for c0 in range(0, T, chunk):
+        K, V = k[c0:c0 + chunk], v[c0:c0 + chunk]
+        gg, b = g[c0:c0 + chunk], beta[c0:c0 + chunk]
+        L = K.shape[0]
+        gam = np.cumsum(gg)
+        M = np.tril(np.exp(gam[:, None] - gam[None, :]))
+        A = np.tril(b[:, None] * (K @ K.T) * M, -1)
+        Tm = np.linalg.solve(np.eye(L) + A, np.eye(L))
+        W = Tm @ ((b * np.exp(gam))[:, None] * K)
+        Ut = Tm @ (b[:, None] * V)
+        eC = np.exp(gam[-1] - gam)
+        Ac = np.exp(gam[-1]) * np.eye(Dk) - W.T @ (eC[:, None] * K)
+        Bc = Ut.T @ (eC[:, None] * K)
+        maps.append((Ac, Bc))
+    return maps
+
+
+def compose_state_maps(first, second):
+    """The map of running chunk map `first`, then `second`:
+    S -> (S A1 + B1) A2 + B2 = S (A1 A2) + (B1 A2 + B2).  Associative, so a
+    sequence's chunk maps can be combined by a parallel scan."""
+    (A1, B1), (A2, B2) = first, second
+    return A1 @ A2, B1 @ A2 + B2

@@ -552,3 +552,37 @@ def test_chunked_recall_first_equals_recurrent(C):
     assert np.allclose(s_c, s_r, rtol=1e-10, atol=1e-11)
     o_std, _ = oracle.chunked(q, k, v, g, beta, s0, cu, chunk=C)
     assert np.abs(o_std - o_r).max() > 1e-3
+
+
+# ---- a chunk step as an affine map of the entering state (for a scan) ---------
+
+def test_chunk_state_maps_reproduce_the_recurrence():
+    """Applying each chunk's affine map S -> S A_c + B_c in turn gives the
+    recurrence's final state, for ragged chunks and an entering state."""
+    q, k, v, g, beta, s0 = make(61, T=70, Hqk=1, Hv=2, N=1, s0_std=0.5)
+    _, s_ref = oracle.recurrent(q, k, v, g, beta, s0)
+    for h in range(2):
+        for C in (1, 7, 16, 64):
+            S = s0[0, h].copy()
+            for A, B in oracle.chunk_state_maps(k, v, g, beta, chunk=C, head_k=0, head_v=h):
+                S = S @ A + B
+            assert np.allclose(S, s_ref[0, h], rtol=1e-10, atol=1e-11), (h, C)
+
+
+def test_chunk_state_maps_compose_associatively():
+    """Composing the maps pairwise in a tree (as a parallel scan would) equals
+    composing them left to right, and equals the one-step map of the whole
+    sequence as a single chunk."""
+    q, k, v, g, beta, s0 = make(62, T=48, Hqk=1, Hv=1, N=1, s0_std=0.5)
+    maps = oracle.chunk_state_maps(k, v, g, beta, chunk=6)
+    seq = maps[0]
+    for m in maps[1:]:
+        seq = oracle.compose_state_maps(seq, m)
+    level = maps
+    while len(level) > 1:
+        level = [oracle.compose_state_maps(level[i], level[i + 1]) if i + 1 < len(level) else level[i]
+                 for i in range(0, len(level), 2)]
+    whole = oracle.chunk_state_maps(k, v, g, beta, chunk=48)[0]
+    for A, B in (level[0], whole):
+        assert np.allclose(A, seq[0], rtol=1e-10, atol=1e-11)
+        assert np.allclose(B, seq[1], rtol=1e-10, atol=1e-11)
