@@ -1,8 +1,9 @@
 // gdn_prefill_static_workspace: the cluster prefill with its workspace ring in
 // a file-scope device array, for callers that allocate no device memory per
 // call.  The contract is in include/gdn.h.  The path below calls no device
-// allocator: the array's address is looked up once per device and the call
-// is then forwarded to gdn_prefill_ex with that address as the workspace.
+// allocator: the array's address is looked up once per device and context,
+// and the call is then forwarded to gdn_prefill_ex with that address as the workspace.
+#include <cuda.h>
 #include <mutex>
 #include <stdint.h>
 
@@ -18,21 +19,61 @@ static __device__ __align__(256) unsigned char g_static_ring[kRingBytes];
 
 constexpr int kMaxDevices = 64;
 std::mutex g_setup_mu;
-void *g_ring_addr[kMaxDevices];  // device address of g_static_ring, per device
+// Per device: the device address of g_static_ring and the id of the CUDA
+// context it was looked up in.  A device reset creates a new primary context
+// (and a new copy of the array), whose different id triggers a new lookup.
+struct RingAddr {
+    void *addr;
+    unsigned long long ctx_id;
+};
+RingAddr g_ring[kMaxDevices];
 
-// The array's address on the current device, looked up on first use.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long *);
+
+// The id of the calling thread's current context (CUDA 12.0+ driver call,
+// reached through the runtime's driver entry points; libgdn links no libcuda).
+gdn_status current_context_id(unsigned long long *id) {
+    static CtxGetCurrentFn get_current = nullptr;
+    static CtxGetIdFn get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+        p = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<CtxGetIdFn>(p);
+    });
+    if (get_current == nullptr || get_id == nullptr) return GDN_ERR_CUDA;
+    CUcontext ctx = nullptr;
+    if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return GDN_ERR_CUDA;
+    return get_id(ctx, id) == CUDA_SUCCESS ? GDN_OK : GDN_ERR_CUDA;
+}
+
+// The array's address on the current device, looked up on first use in the
+// device's current context.  Before libgdn's first CUDA call on this thread no
+// context may be current yet; the symbol lookup then binds the device's
+// primary context, and its id is read afterwards.
 gdn_status ring_address(void **out) {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess) return GDN_ERR_CUDA;
     if (dev < 0 || dev >= kMaxDevices) return GDN_ERR_UNSUPPORTED;
+    unsigned long long ctx = 0;
+    const bool have_ctx = current_context_id(&ctx) == GDN_OK;
     std::lock_guard<std::mutex> lock(g_setup_mu);
-    if (g_ring_addr[dev] == nullptr) {
+    if (!have_ctx || g_ring[dev].addr == nullptr || g_ring[dev].ctx_id != ctx) {
         void *p = nullptr;
         if (cudaGetSymbolAddress(&p, g_static_ring) != cudaSuccess || p == nullptr)
             return GDN_ERR_CUDA;
-        g_ring_addr[dev] = p;
+        if (current_context_id(&ctx) != GDN_OK) return GDN_ERR_CUDA;
+        g_ring[dev].addr = p;
+        g_ring[dev].ctx_id = ctx;
     }
-    *out = g_ring_addr[dev];
+    *out = g_ring[dev].addr;
     return GDN_OK;
 }
 

@@ -77,8 +77,8 @@ typedef enum gdn_dtype {
 
 /*
  * gdn_prefill -- chunk-parallel prefill/training forward of the gated delta
- * rule over a packed batch of N sequences (section 三 of the page above:
- * "the state is accumulated chunk-parallel").
+ * rule over a packed batch of N sequences (section 三 of the page above: for
+ * training the state is built up over chunks of tokens in parallel).
  *
  *   q, k, v, io_dtype   token inputs, layouts above.
  *   g, beta             per-token log-decay and write strength, fp32 [T][Hv].
@@ -169,9 +169,9 @@ GDN_API size_t gdn_prefill_ex_workspace_bytes(int32_t N, int64_t T, int32_t Hqk,
                                               gdn_prefill_kernel kernel);
 
 /*
- * gdn_decode_step -- one-token inference update of N independent sequences
- * (section 三 of the page above: "each inference step does one fixed-size
- * matrix update"), in place on the state.
+ * gdn_decode_step -- one-token inference update of N independent sequences,
+ * in place on the state (section 三 of the page above: at inference time the
+ * state of each head takes one update of constant size per token).
  *
  *   q, k                [N][Hqk][Dk] io_dtype, this step's query and key.
  *   v                   [N][Hv][Dv]  io_dtype.
@@ -229,10 +229,15 @@ GDN_API gdn_status gdn_decode_step_bf16_state(const void *q, const void *k, cons
  * not 0 or 64) also return GDN_ERR_UNSUPPORTED.
  *
  * Set-up: the first call on a device (with that device current) looks up the
- * array's device address once and caches it per device; a failure there
- * returns GDN_ERR_CUDA.  Make that first call before any stream capture.
- * Depending on the CUDA module loading mode, the array's device memory is
- * reserved when libgdn's module is loaded or at that first call.
+ * array's device address and caches it for that device and its current CUDA
+ * context; a failure there returns GDN_ERR_CUDA.  Make that first call before
+ * any stream capture.  When the context changes (after cudaDeviceReset, the
+ * primary context is created anew and the array with it), the next call looks
+ * the address up again, so it too should come before any capture.  Devices
+ * with an index of 64 or more are not served: the call returns
+ * GDN_ERR_UNSUPPORTED for them.  Depending on the CUDA module loading mode,
+ * the array's device memory is reserved when libgdn's module is loaded or at
+ * that first call.
  *
  * Nothing in the array has to start at zero: within one call every ring slot
  * is written before it is read.  There is one array per device, so calls whose

@@ -138,7 +138,14 @@ int gdn_oracle_recurrent(const double *q, const double *k, const double *v,
         if (!S || !r) {
 #pragma omp atomic write
             failed = 1;
-        } else {
+        }
+        /* Every thread takes the same branch: the worksharing loop below is
+           reached by the whole team or by none of it. */
+#pragma omp barrier
+        int any_failed;
+#pragma omp atomic read
+        any_failed = failed;
+        if (!any_failed) {
 #pragma omp for schedule(dynamic, 1)
             for (int64_t u = 0; u < N * Hv; ++u) {
                 const int64_t n = u / Hv, h = u % Hv;
@@ -205,7 +212,14 @@ int gdn_oracle_chunked(const double *q, const double *k, const double *v,
         if (!S || !Sn || !gam || !A || !Tm || !W || !U) {
 #pragma omp atomic write
             failed = 1;
-        } else {
+        }
+        /* Every thread takes the same branch: the worksharing loop below is
+           reached by the whole team or by none of it. */
+#pragma omp barrier
+        int any_failed;
+#pragma omp atomic read
+        any_failed = failed;
+        if (!any_failed) {
 #pragma omp for schedule(dynamic, 1)
             for (int64_t unit = 0; unit < N * Hv; ++unit) {
                 const int64_t n = unit / Hv, h = unit % Hv, j = h / G;
