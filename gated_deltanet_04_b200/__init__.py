@@ -28,7 +28,7 @@ __all__ = ["gdn_prefill", "gdn_decode_step", "gdn_decode_step_bf16_state", "gdn_
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgdn.so")
 
 STATUS = {0: "GDN_OK", 1: "GDN_ERR_INVALID_ARGUMENT", 2: "GDN_ERR_UNSUPPORTED", 3: "GDN_ERR_CUDA",
-          4: "GDN_ERR_TIMEOUT", 5: "GDN_ERR_BAD_SEQLENS", 6: "GDN_ERR_BAD_SLOT"}
+          4: "GDN_ERR_TIMEOUT", 5: "GDN_ERR_BAD_SEQLENS", 6: "GDN_ERR_BAD_SLOT", 7: "GDN_ERR_RANGE"}
 DTYPE = {torch.bfloat16: 0, torch.float32: 1}
 # gdn_order values of include/gdn.h: where the recall S k is taken
 ORDERS = {"standard": 0, "recall_first": 1}

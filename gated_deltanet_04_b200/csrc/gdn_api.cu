@@ -29,6 +29,7 @@ const char *gdn_status_string(gdn_status s) {
         case GDN_ERR_TIMEOUT: return "GDN_ERR_TIMEOUT";
         case GDN_ERR_BAD_SEQLENS: return "GDN_ERR_BAD_SEQLENS";
         case GDN_ERR_BAD_SLOT: return "GDN_ERR_BAD_SLOT";
+        case GDN_ERR_RANGE: return "GDN_ERR_RANGE";
     }
     return "GDN_ERR_UNKNOWN";
 }
@@ -85,13 +86,19 @@ gdn_status gdn_prefill_ex(const void *q, const void *k, const void *v, gdn_dtype
                              dev_error_flag, stream, kernel, GDN_ORDER_STANDARD);
 }
 
-gdn_status gdn_prefill_order(const void *q, const void *k, const void *v, gdn_dtype io_dtype,
-                             const float *g, const float *beta, const float *initial_state,
-                             const int32_t *cu_seqlens, int32_t N, int64_t T, int32_t Hqk,
-                             int32_t Hv, int32_t Dk, int32_t Dv, int32_t chunk, void *o,
-                             float *final_state, void *workspace, size_t workspace_bytes,
-                             int32_t *dev_error_flag, void *stream, gdn_prefill_kernel kernel,
-                             gdn_order order) {
+}  // extern "C"
+
+namespace {
+
+// gdn_prefill_order, plus the testing-only settings of the pool kernel (a unit
+// its producers skip, and the limit of its flag spins; -1 / 0 = off).
+gdn_status prefill_impl(const void *q, const void *k, const void *v, gdn_dtype io_dtype,
+                        const float *g, const float *beta, const float *initial_state,
+                        const int32_t *cu_seqlens, int32_t N, int64_t T, int32_t Hqk, int32_t Hv,
+                        int32_t Dk, int32_t Dv, int32_t chunk, void *o, float *final_state,
+                        void *workspace, size_t workspace_bytes, int32_t *dev_error_flag,
+                        void *stream, gdn_prefill_kernel kernel, gdn_order order,
+                        int32_t debug_skip_unit, int64_t debug_flag_wait) {
     if (kernel < GDN_PREFILL_AUTO || kernel > GDN_PREFILL_POOL) return GDN_ERR_INVALID_ARGUMENT;
     if (order != GDN_ORDER_STANDARD && order != GDN_ORDER_RECALL_FIRST) return GDN_ERR_INVALID_ARGUMENT;
     if (io_dtype != GDN_DTYPE_BF16 && io_dtype != GDN_DTYPE_F32) return GDN_ERR_INVALID_ARGUMENT;
@@ -122,11 +129,43 @@ gdn_status gdn_prefill_order(const void *q, const void *k, const void *v, gdn_dt
     a.o = o; a.sT = final_state; a.err = dev_error_flag; a.ws = workspace; a.T = T; a.N = N; a.Hqk = Hqk;
     a.Hv = Hv; a.Dk = Dk; a.Dv = Dv; a.chunk = chunk == 0 ? 64 : chunk; a.dtype = io_dtype;
     a.order = order;
+    a.debug_skip_unit = debug_skip_unit;
+    a.debug_flag_wait = debug_flag_wait;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (T == 0 || kernel == GDN_PREFILL_RECURRENT) return from_cuda(gdn::launch_prefill_recurrent(a, s));
     if (kernel == GDN_PREFILL_SINGLE_CTA) return from_cuda(gdn::launch_prefill_tc(a, s));
     if (kernel == GDN_PREFILL_POOL) return from_cuda(gdn::launch_prefill_pool(a, s));
     return from_cuda(gdn::launch_prefill_cluster(a, s));
+}
+
+}  // namespace
+
+extern "C" {
+
+gdn_status gdn_prefill_order(const void *q, const void *k, const void *v, gdn_dtype io_dtype,
+                             const float *g, const float *beta, const float *initial_state,
+                             const int32_t *cu_seqlens, int32_t N, int64_t T, int32_t Hqk,
+                             int32_t Hv, int32_t Dk, int32_t Dv, int32_t chunk, void *o,
+                             float *final_state, void *workspace, size_t workspace_bytes,
+                             int32_t *dev_error_flag, void *stream, gdn_prefill_kernel kernel,
+                             gdn_order order) {
+    return prefill_impl(q, k, v, io_dtype, g, beta, initial_state, cu_seqlens, N, T, Hqk, Hv, Dk,
+                        Dv, chunk, o, final_state, workspace, workspace_bytes, dev_error_flag,
+                        stream, kernel, order, -1, 0);
+}
+
+gdn_status gdn_debug_prefill_pool_stall(const void *q, const void *k, const void *v,
+                                        gdn_dtype io_dtype, const float *g, const float *beta,
+                                        const float *initial_state, const int32_t *cu_seqlens,
+                                        int32_t N, int64_t T, int32_t Hqk, int32_t Hv, int32_t Dk,
+                                        int32_t Dv, int32_t chunk, void *o, float *final_state,
+                                        void *workspace, size_t workspace_bytes,
+                                        int32_t *dev_error_flag, void *stream, int32_t skip_unit,
+                                        int64_t flag_wait_cycles) {
+    if (skip_unit < 0 || flag_wait_cycles <= 0) return GDN_ERR_INVALID_ARGUMENT;
+    return prefill_impl(q, k, v, io_dtype, g, beta, initial_state, cu_seqlens, N, T, Hqk, Hv, Dk,
+                        Dv, chunk, o, final_state, workspace, workspace_bytes, dev_error_flag,
+                        stream, GDN_PREFILL_POOL, GDN_ORDER_STANDARD, skip_unit, flag_wait_cycles);
 }
 
 gdn_status gdn_decode_step(const void *q, const void *k, const void *v, gdn_dtype io_dtype,

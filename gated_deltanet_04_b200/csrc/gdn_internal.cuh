@@ -23,6 +23,10 @@ struct PrefillArgs {
     int32_t N, Hqk, Hv, Dk, Dv, chunk;
     gdn_dtype dtype;
     int32_t order = GDN_ORDER_STANDARD;  // gdn_order
+    // testing only (pool kernel): a unit the producers never prepare, and the
+    // SM-clock limit of every spin on a hand-off flag (0: the default)
+    int32_t debug_skip_unit = -1;
+    int64_t debug_flag_wait = 0;
 };
 
 struct DecodeArgs {

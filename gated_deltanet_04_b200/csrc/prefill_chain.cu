@@ -140,7 +140,10 @@ struct ChainMisc {
     uint64_t ready[2];
     uint64_t mma_bar;
     uint32_t tmem_base;
+    alignas(16) uint32_t vote[2][8];  // per-warp vote words of E1 and E2 (read as uint4)
+    float red[8];                     // per-warp maxima of a rescale
 };
+static_assert(offsetof(ChainMisc, vote) % 16 == 0 && C_MISC % 16 == 0, "vote words read as uint4");
 
 // chain TMEM columns (512 allocated):
 //   S    0..127   fp32 state (accumulator of nothing: read, scaled, rewritten)
@@ -162,11 +165,18 @@ constexpr uint32_t P_AS = P_X;
 constexpr uint32_t P_TS = P_X + 64 * kAS4 * 4;
 constexpr uint32_t P_XS = P_TS + 64 * kTS * 4;
 constexpr uint32_t P_P16 = 137216;      // P fp16 [64 rows][128 B], SW128
-constexpr uint32_t P_TBH = 145408, P_TBL = 153600, P_TGH = 161792, P_TGL = 169984;  // T tiles
+// T tiles: T diag(b) as bf16 hi / mid / lo and T diag(b Gamma) as fp16 hi / lo,
+// each [64 rows][128 B], SW128.  The parts of each are consecutive, so one B
+// operand of N = 192 (or 128) rows takes all of them and the MMA writes each
+// part's product to its own accumulator columns.
+constexpr uint32_t P_TBH = 145408, P_TBM = 153600, P_TBL = 161792, P_TGH = 169984,
+                   P_TGL = 178176;
 constexpr uint32_t P_UTS = P_TBH;       // then U~^T staging (same layout as SL_UT)
-constexpr uint32_t P_MISC = 178176;
-constexpr uint32_t P_ID = 182272;       // bf16 identity [64][128 B] (B operand of the Q^T product)
-static_assert(P_WST + 32768 <= P_P16 && P_UTS + 32768 <= P_MISC, "staging fits its region");
+constexpr uint32_t P_MISC = 186368;
+constexpr uint32_t P_ID = 190464;       // bf16 identity [64][128 B] (B operand of the Q^T product)
+static_assert(P_TBM == P_TBH + 8192 && P_TBL == P_TBM + 8192 && P_TGL == P_TGH + 8192,
+              "stacked B operands");
+static_assert(P_WST + 32768 <= P_P16 && P_UTS + 32768 <= P_TGL + 8192, "staging fits its region");
 static_assert(P_XS + 1024 * 4 <= P_P16, "solve scratch overflows");
 static_assert(P_TS % 16 == 0 && P_XS % 16 == 0, "float4 scratch must be aligned");
 static_assert(P_P16 % 1024 == 0 && P_TBH % 1024 == 0, "swizzled tiles start on 1 KB");
@@ -202,9 +212,12 @@ constexpr uint32_t kChainBytes = C_MISC + sizeof(ChainMisc);
 constexpr uint32_t kSmemBytes = (kProdBytes > kChainBytes ? kProdBytes : kChainBytes) + 1024;
 static_assert(kSmemBytes <= 232448, "fits the 227 KB opt-in shared memory of a CTA");
 
-// producer TMEM columns (128 allocated)
-// producer TMEM columns (256 allocated): Gram then W^T, U~^T, Q^T
-constexpr uint32_t PT_G = 0, PT_U = 64, PT_Q = 128;
+// producer TMEM columns (512 allocated): the Gram, then W^T from T diag(b Gamma)'s
+// hi part (and its lo part's product at + 64); Q^T; U~^T as three products
+// (T diag(b)'s hi, mid, lo parts) at PT_U, + 64, + 128
+constexpr uint32_t PT_G = 0, PT_Q = 128, PT_U = 256;
+constexpr uint32_t IDESC_MK_N192_BF16 = make_idesc_f16(128, 192, 1, 0, 1);
+constexpr uint32_t IDESC_MK_N128 = make_idesc_f16(128, 128, 1, 0);
 
 // pool flags: a header of kFlagHeader words ([0] the chunk counter, [1] the
 // abort flag), then 8 words per unit ([0] taken, [1 + s] ready of slot s)
@@ -224,6 +237,8 @@ struct ChainParams {
     int32_t N, Hqk, Hv, units, max_chunks;
     int32_t ring_slots;  // a power of two
     int32_t recall_first;  // GDN_ORDER_RECALL_FIRST: recall before the decay
+    long long flag_wait_limit;  // SM clocks a spin on a hand-off flag may last
+    int32_t skip_unit;          // testing: a unit no producer prepares (-1: none)
 };
 
 __device__ __forceinline__ uint8_t *ring_slot(const ChainParams &p, int unit, int c) {
@@ -253,6 +268,10 @@ __device__ Item pool_item(const ChainParams &p, uint32_t i, bool &skip) {
     const int c = (int)(i / (uint32_t)p.units);
     const int unit = (int)(i % (uint32_t)p.units);
     if (c >= p.max_chunks) return it;
+    if (unit == p.skip_unit) {  // testing: its chain waits for a chunk that never comes
+        skip = true;
+        return it;
+    }
     const int n = unit / p.Hv;
     int64_t t0, t1;
     if (!seq_range(p.cu, n, p.N, p.T, nullptr, t0, t1)) {  // the chain reports it
@@ -331,6 +350,8 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
 
     uint32_t mma_phase = 0;
     bool timed_out = false;
+    float kmax = 0.f;             // largest key-side value this thread has put into fp16
+    bool range_reported = false;
     float gpre0 = 0.f, gpre1 = 0.f, bpre0 = 0.f, bpre1 = 0.f;  // gates warp: next chunk's g, beta
     auto load_gates = [&](const Item &it) {
         gpre0 = gpre1 = bpre0 = bpre1 = 0.f;
@@ -498,9 +519,10 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
             }
             mma_commit(&ms->mma_bar);
         }
-        // bf16 -> fp16 in place with padding rows zeroed: V (A operand of U~)
-        // while the Gram products run, then K once they have read it.  Q goes
-        // to fp16 in the Q^T transpose.
+        // K goes from bf16 to fp16 in place (padding rows zeroed) once the Gram
+        // products have read it: the chain's state update takes it in fp16.
+        // V stays bf16 (the U~ product splits its other operand three ways in
+        // bf16), and Q goes to fp16 in the Q^T transpose.
         auto convert16 = [&](uint8_t *base, int x) {  // 16-byte chunk x of a [64][128 B] tile
             uint4 *ptr = reinterpret_cast<uint4 *>(base) + x;
             const int r = x >> 3;
@@ -513,17 +535,13 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
                 for (int q2 = 0; q2 < 4; ++q2) {
                     const __nv_bfloat162 b2 = *reinterpret_cast<const __nv_bfloat162 *>(&w[q2]);
                     const float2 f = __bfloat1622float2(b2);
+                    kmax = fmaxf(kmax, fmaxf(fabsf(f.x), fabsf(f.y)));
                     w[q2] = pack_half2(f.x, f.y);
                 }
                 val = make_uint4(w[0], w[1], w[2], w[3]);
             }
             *ptr = val;
         };
-#pragma unroll
-        for (int q = 0; q < 1024 / kThreads; ++q) {
-            const int x = tid + q * kThreads;  // V halves: 2 x 512 chunks
-            convert16(kqv + 32768 + (x >> 9) * 8192, x & 511);
-        }
         if (!mbar_wait_bounded(&ms->mma_bar, mma_phase, kWaitLimit)) timed_out = true;
         mma_phase ^= 1;
         tc_fence_after_sync();
@@ -572,7 +590,8 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
 #pragma unroll
                 for (int x = 0; x < 32; ++x) v[x] = (c + x <= r) ? v[x] : 0.f;
 #pragma unroll
-                for (int e = 0; e < 32; e += 8) st_row_chunk(sm + P_P16, r, (c + e) / 8, pack8(v + e));
+                for (int e = 0; e < 32; e += 8)
+                    st_row_chunk(sm + P_P16, r, (c + e) / 8, pack8_track(v + e, kmax));
             }
         }
         __syncthreads();
@@ -598,7 +617,8 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
         solve_tril64(As, Ts, Xs, tid);
         GDN_CL_PHASE(1, 6);  // solve
 
-        // ---- rows of T diag(b), T diag(b Gamma): fp16 hi / lo ----
+        // ---- rows of T diag(b) (bf16 hi / mid / lo: exact, and V needs no
+        //      conversion) and T diag(b Gamma) (fp16 hi / lo, as K) ----
         {
             const int grp = tid >> 6, r = tid & 63;
             const bool tg = grp >= 2;
@@ -615,7 +635,10 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
                     x[e + q] = (i <= r) ? tv[q] * scale[i] : 0.f;
                 }
             }
-            store_split32(sm + (tg ? P_TGH : P_TBH), sm + (tg ? P_TGL : P_TBL), r, c, x, !tg || hp);
+            if (tg)
+                store_split32(sm + P_TGH, sm + P_TGL, r, c, x, hp, kmax);
+            else
+                store_split32_bf16x3(sm + P_TBH, sm + P_TBM, sm + P_TBL, r, c, x);
         }
         publish();
         GDN_CL_PHASE(1, 7);  // T tiles
@@ -623,20 +646,18 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
         // ---- U~^T = V^T (T diag b)^T,  W^T = K^T (T diag(b Gamma))^T ----
         if (tid == 0) {
 #pragma unroll
-            for (int pass = 0; pass < 2; ++pass)
+            for (int ks = 0; ks < 4; ++ks) {  // bf16 V times [hi | mid | lo] of T diag(b)
+                const uint64_t a = make_sdesc(skqv + 32768 + ks * 2048, 8192, 1024);
+                const uint64_t b = make_sdesc(sbase + P_TBH + ks * 32, 16, 1024);
+                mma_f16_ss(tmem + PT_U, a, b, IDESC_MK_N192_BF16, ks != 0);
+            }
+            const uint32_t idesc_w = hp ? IDESC_MK_N128 : IDESC_MK_N64;
 #pragma unroll
-                for (int ks = 0; ks < 4; ++ks) {
-                    const uint64_t a = make_sdesc(skqv + 32768 + ks * 2048, 8192, 1024);
-                    const uint64_t b = make_sdesc(sbase + (pass ? P_TBL : P_TBH) + ks * 32, 16, 1024);
-                    mma_f16_ss(tmem + PT_U, a, b, IDESC_MK_N64, (pass | ks) != 0);
-                }
-            for (int pass = 0; pass < (hp ? 2 : 1); ++pass)
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks) {
-                    const uint64_t a = make_sdesc(skqv + ks * 2048, 16384, 1024);
-                    const uint64_t b = make_sdesc(sbase + (pass ? P_TGL : P_TGH) + ks * 32, 16, 1024);
-                    mma_f16_ss(tmem + PT_G, a, b, IDESC_MK_N64, (pass | ks) != 0);
-                }
+            for (int ks = 0; ks < 4; ++ks) {  // fp16 K times [hi | lo] of T diag(b Gamma)
+                const uint64_t a = make_sdesc(skqv + ks * 2048, 16384, 1024);
+                const uint64_t b = make_sdesc(sbase + P_TGH + ks * 32, 16, 1024);
+                mma_f16_ss(tmem + PT_G, a, b, idesc_w, ks != 0);
+            }
             mma_commit(&ms->mma_bar);
         }
         if (warp == kGatesWarp && ms->items[(l + 1) & 3].valid) compute_gates(ms->gt[(l + 1) & 1]);
@@ -654,7 +675,7 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
                 // depend on that observation, and the chain publishes it only after
                 // its load of the slot has completed
                 if (it.c >= p.ring_slots && early_taken < need &&
-                    !wait_flag_geq(unit_flags(p, it.unit), need, p.flags + 1, kWaitLimit))
+                    !wait_flag_geq(unit_flags(p, it.unit), need, p.flags + 1, p.flag_wait_limit))
                     timed_out = true;
             } else {
                 if (l >= 1 && !mbar_wait_cluster_bounded(&ms->taken, (l - 1) & 1, kWaitLimit))
@@ -671,10 +692,24 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
             const int c = 32 * half;
             float v[32];
             tmem_ld32(trow + PT_G + c, v);
+            if (hp) {
+                float w2[32];
+                tmem_ld32(trow + PT_G + 64 + c, w2);
+                tmem_wait_ld();
+#pragma unroll
+                for (int x = 0; x < 32; ++x) v[x] += w2[x];
+            }
             tmem_wait_ld();
-            store_split32(sm + P_WST, sm + P_WST + 16384, row, c, v, hp);
-            tmem_ld32(trow + PT_U + c, v);
-            tmem_wait_ld();
+            store_split32(sm + P_WST, sm + P_WST + 16384, row, c, v, hp, kmax);
+            {
+                float u1[32], u2[32];
+                tmem_ld32(trow + PT_U + c, v);
+                tmem_ld32(trow + PT_U + 64 + c, u1);
+                tmem_ld32(trow + PT_U + 128 + c, u2);
+                tmem_wait_ld();
+#pragma unroll
+                for (int x = 0; x < 32; ++x) v[x] += u1[x] + u2[x];
+            }
 #pragma unroll
             for (int q = 0; q < 8; ++q)
                 *reinterpret_cast<float4 *>(sm + P_UTS + ut_off(row, c / 4 + q)) =
@@ -704,9 +739,17 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
                 v[x] = (c + x < L) ? v[x] * sc : 0.f;
             }
 #pragma unroll
-            for (int e = 0; e < 32; e += 8) st_row_chunk(kqv + 32768, row, (c + e) / 8, pack8(v + e));
+            for (int e = 0; e < 32; e += 8)
+                st_row_chunk(kqv + 32768, row, (c + e) / 8, pack8_track(v + e, kmax));
         }
         fence_proxy_async_smem();  // staged data -> visible to the bulk copies
+        // a key-side fp16 operand of this chunk (K, Q^T, P, T diag(b Gamma), W^T)
+        // overflowed: report it once per thread (the unit's results are then
+        // unspecified; the computation goes on)
+        if (kmax >= kFp16Overflow && !range_reported) {
+            raise_error(p.err, GDN_ERR_RANGE);
+            range_reported = true;
+        }
         GDN_CL_PHASE(1, 9);  // staging
 
         // ---- deliver with asynchronous stores (the ring slot is free: see above) ----
@@ -762,30 +805,64 @@ __device__ void chain_role(uint8_t *sm, const CUtensorMap *tm_o, const ChainPara
     uint32_t *uflags = kPool ? unit_flags(p, unit) : nullptr;
     (void)warp;
 
-    // ---- initial state: fp32 -> TMEM accumulator, fp16 hi/lo -> TMEM A operands ----
-    {
-        const float *src = p.s0 ? p.s0 + (((int64_t)n * p.Hv + h) * kD + row) * kD + 64 * half : nullptr;
-        float v[32];
+    // Value-side operands are held with a power-of-two scale, uniform over
+    // the unit: the fp32 master state in TMEM is S * 2^-es, and its fp16 hi /
+    // lo copies (the A operand of S [Q^T | W^T]) are split from it directly,
+    // so the products come out scaled by 2^-es.  U and U' are held as
+    // U * 2^-eu, where eu is es unless U's magnitudes leave the band
+    // [kScaleLo, kScaleHi) in that scale.  Every epilogue votes on its
+    // largest scaled magnitude; the rare chunk whose values left the band
+    // recomputes them in fp32 and takes a new scale (fp16_scale_exp).  The
+    // scaling is exact, so no value-side operand over- or underflows fp16,
+    // whatever the scale of v and S0, and the results scale exactly with it.
+    int es = 0, eu = 0;
+    float s_up = 1.f, sd = 1.f;  // 2^es, 2^-es
+    auto set_es = [&](int e) {
+        es = e;
+        s_up = exp2i(e);
+        sd = exp2i(-e);
+    };
+    // 64 values of this thread's state row (scaled) -> the hi / lo TMEM operands
+    auto split_state = [&](const float (&sv)[64]) {
         uint32_t hi[32], lo[32];
 #pragma unroll
-        for (int part = 0; part < 2; ++part) {
-#pragma unroll
-            for (int x = 0; x < 32; x += 4) {
-                const float4 f = src ? *reinterpret_cast<const float4 *>(src + 32 * part + x)
-                                     : make_float4(0.f, 0.f, 0.f, 0.f);
-                v[x] = f.x; v[x + 1] = f.y; v[x + 2] = f.z; v[x + 3] = f.w;
-            }
-            tmem_st32(trow + CT_S + 64 * half + 32 * part, v);
-#pragma unroll
-            for (int x = 0; x < 32; x += 2) {
-                const __half2 hh = __floats2half2_rn(v[x], v[x + 1]);
-                const float2 hf = __half22float2(hh);
-                hi[16 * part + x / 2] = *reinterpret_cast<const uint32_t *>(&hh);
-                lo[16 * part + x / 2] = pack_half2(v[x] - hf.x, v[x + 1] - hf.y);
-            }
+        for (int x = 0; x < 64; x += 2) {
+            const __half2 hh = __floats2half2_rn(sv[x], sv[x + 1]);
+            const float2 hf = __half22float2(hh);
+            hi[x / 2] = *reinterpret_cast<const uint32_t *>(&hh);
+            lo[x / 2] = pack_half2(sv[x] - hf.x, sv[x + 1] - hf.y);
         }
         tmem_st32u(trow + CT_SH + 32 * half, hi);
         tmem_st32u(trow + CT_SL + 32 * half, lo);
+    };
+    auto store_state = [&](const float (&sv)[64]) {  // the scaled fp32 master
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {
+            float v[32];
+#pragma unroll
+            for (int x = 0; x < 32; ++x) v[x] = sv[32 * part + x];
+            tmem_st32(trow + CT_S + 64 * half + 32 * part, v);
+        }
+    };
+
+    // ---- initial state: scaled fp32 -> TMEM accumulator, fp16 hi/lo -> TMEM A operands ----
+    {
+        const float *src = p.s0 ? p.s0 + (((int64_t)n * p.Hv + h) * kD + row) * kD + 64 * half : nullptr;
+        float sv[64];
+        float am = 0.f;
+#pragma unroll
+        for (int x = 0; x < 64; x += 4) {
+            const float4 f = src ? *reinterpret_cast<const float4 *>(src + x)
+                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+            sv[x] = f.x; sv[x + 1] = f.y; sv[x + 2] = f.z; sv[x + 3] = f.w;
+            am = fmaxf(am, fmaxf(fmaxf(fabsf(f.x), fabsf(f.y)), fmaxf(fabsf(f.z), fabsf(f.w))));
+        }
+        am = cta_max(am, ms->red, warp, lane);
+        set_es(am > 0.f ? fp16_scale_exp(am) : 0);
+#pragma unroll
+        for (int x = 0; x < 64; ++x) sv[x] *= sd;
+        store_state(sv);
+        split_state(sv);
         tmem_wait_st();
     }
     tc_fence_before_sync();
@@ -835,7 +912,7 @@ __device__ void chain_role(uint8_t *sm, const CUtensorMap *tm_o, const ChainPara
     auto ready_wait = [&](int cc) -> bool {
         if constexpr (kPool)
             return wait_flag_geq(uflags + 1 + (cc & (p.ring_slots - 1)), (uint32_t)(cc + 1), p.flags + 1,
-                                 kWaitLimit);
+                                 p.flag_wait_limit);
         else
             return mbar_wait_cluster_bounded(&ms->ready[cc & 1], (cc >> 1) & 1, kWaitLimit);
     };
@@ -967,49 +1044,89 @@ __device__ void chain_role(uint8_t *sm, const CUtensorMap *tm_o, const ChainPara
         tc_fence_after_sync();
         GDN_CL_PHASE(0, 2);  // wait: S Q^T, R
 
-        // ---- O *= Gamma unless Q^T came scaled; U = U~ - R; U', U -> TMEM ----
+        // ---- U = U~ - R in the state's scale; U', U -> TMEM; O *= Gamma unless
+        //      Q^T came scaled.  A vote on U's largest scaled magnitude; if it
+        //      left the band, U takes a scale of its own and O follows it. ----
         {
             const int c32 = 32 * half;
-            float v[32], r0[32];
             const bool qs = gb->qs != 0;
-            if (!qs) tmem_ld32(trow + CT_O + c32, v);
-            tmem_ld32(trow + CT_R + c32, r0);
-            tmem_wait_ld();
-            if (hp) {
-                float r2[32];
-                tmem_ld32(trow + CT_R2 + c32, r2);
+            float v[32];
+            // R (scaled by 2^-es) into v, U~ (unscaled) into ut
+            auto load_r_ut = [&](float (&ut)[32]) {
+                tmem_ld32(trow + CT_R + c32, v);
+                tmem_wait_ld();
+                if (hp) {
+                    float r2[32];
+                    tmem_ld32(trow + CT_R2 + c32, r2);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int x = 0; x < 32; ++x) v[x] += r2[x];
+                }
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const float4 f =
+                        *reinterpret_cast<const float4 *>(slot + SL_UT + ut_off(row, c32 / 4 + q));
+                    ut[4 * q] = f.x; ut[4 * q + 1] = f.y; ut[4 * q + 2] = f.z; ut[4 * q + 3] = f.w;
+                }
+            };
+            // U (scaled) -> U' = U diag(Gamma_C / Gamma) as fp16 hi / lo, and U as fp16
+            auto store_u = [&]() {
+                uint32_t uh[16], ul[16], u16[16];
+#pragma unroll
+                for (int x = 0; x < 32; x += 2) {
+                    const float p0 = v[x] * gb->eC[c32 + x], p1 = v[x + 1] * gb->eC[c32 + x + 1];
+                    const __half2 hh = __floats2half2_rn(p0, p1);
+                    const float2 hf = __half22float2(hh);
+                    uh[x / 2] = *reinterpret_cast<const uint32_t *>(&hh);
+                    ul[x / 2] = pack_half2(p0 - hf.x, p1 - hf.y);
+                    u16[x / 2] = pack_half2(v[x], v[x + 1]);
+                }
+                tmem_st16u(trow + CT_UP + c32 / 2, uh);
+                tmem_st16u(trow + CT_UP + 32 + c32 / 2, ul);
+                tmem_st16u(trow + CT_U16 + c32 / 2, u16);
+            };
+            // O (S Q^T) times f, and times Gamma unless Q^T came scaled
+            auto scale_o = [&](float f, bool with_gamma) {
+                float ov[32];
+                tmem_ld32(trow + CT_O + c32, ov);
                 tmem_wait_ld();
 #pragma unroll
-                for (int x = 0; x < 32; ++x) r0[x] += r2[x];
-            }
-            if (!qs) {  // O = diag(Gamma) Q S^T, unless Q^T came scaled
+                for (int x = 0; x < 32; ++x) ov[x] *= with_gamma ? f * gb->Gam[c32 + x] : f;
+                tmem_st32(trow + CT_O + c32, ov);
+            };
+            float am;
+            {
+                float ut[32];
+                load_r_ut(ut);
 #pragma unroll
-                for (int x = 0; x < 32; ++x) v[x] *= gb->Gam[c32 + x];
-                tmem_st32(trow + CT_O + c32, v);
+                for (int x = 0; x < 32; ++x) v[x] = fmaf(ut[x], sd, -v[x]);  // U 2^-es (R: 2^-es)
+                am = max_abs<32>(v);
             }
+            eu = es;
+            store_u();
+            if (!qs) scale_o(1.f, true);
+            tmem_wait_st();
+            tc_fence_before_sync();
+            const unsigned b =
+                cta_or8(__reduce_or_sync(0xffffffffu, scale_bits(am)), ms->vote[0], warp, lane);
+            if (rescale_needed(b)) {  // rare: U takes its own scale, O moves to it
+                tc_fence_after_sync();
+                float ut[32];
+                load_r_ut(ut);  // R and U~ are still in place
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                const float4 f = *reinterpret_cast<const float4 *>(slot + SL_UT + ut_off(row, c32 / 4 + q));
-                v[4 * q] = f.x; v[4 * q + 1] = f.y; v[4 * q + 2] = f.z; v[4 * q + 3] = f.w;
-            }
-            uint32_t uh[16], ul[16], u16[16];
+                for (int x = 0; x < 32; ++x) v[x] = fmaf(-s_up, v[x], ut[x]);  // U in fp32, unscaled
+                am = cta_max(max_abs<32>(v), ms->red, warp, lane);
+                eu = fp16_scale_exp(am);
+                const float ud = exp2i(-eu);
 #pragma unroll
-            for (int x = 0; x < 32; x += 2) {
-                const float u0 = v[x] - r0[x], u1 = v[x + 1] - r0[x + 1];
-                const float p0 = u0 * gb->eC[c32 + x], p1 = u1 * gb->eC[c32 + x + 1];
-                const __half2 hh = __floats2half2_rn(p0, p1);
-                const float2 hf = __half22float2(hh);
-                uh[x / 2] = *reinterpret_cast<const uint32_t *>(&hh);
-                ul[x / 2] = pack_half2(p0 - hf.x, p1 - hf.y);
-                u16[x / 2] = pack_half2(u0, u1);
+                for (int x = 0; x < 32; ++x) v[x] *= ud;
+                store_u();
+                scale_o(exp2c(es - eu), false);
+                tmem_wait_st();
+                tc_fence_before_sync();
+                __syncthreads();
             }
-            tmem_st16u(trow + CT_UP + c32 / 2, uh);
-            tmem_st16u(trow + CT_UP + 32 + c32 / 2, ul);
-            tmem_st16u(trow + CT_U16 + c32 / 2, u16);
         }
-        tmem_wait_st();
-        tc_fence_before_sync();
-        __syncthreads();
         tc_fence_after_sync();
         poll_read(c);  // the load itself is issued under the next products
         GDN_CL_PHASE(0, 3);  // O scale, U, U'
@@ -1030,54 +1147,85 @@ __device__ void chain_role(uint8_t *sm, const CUtensorMap *tm_o, const ChainPara
         mma_sync_point();
         GDN_CL_PHASE(0, 4);  // state update + P MMAs
 
-        // ---- o -> staging (stored during the next chunk); S' = Gamma_C S + dS and its
-        //      fp16 hi/lo TMEM operands ----
+        // ---- o -> staging (stored during the next chunk); S' = Gamma_C S + dS in
+        //      the state's scale and its fp16 hi/lo TMEM operands; the vote
+        //      (timeout, and S' leaving the band) ----
         {
             const int c32 = 32 * half;
+            const float uu = exp2i(eu);  // O and dS come scaled by 2^-eu
             float v[32];
             tmem_ld32(trow + CT_O + c32, v);
             tmem_wait_ld();
             __nv_bfloat16 *ost = reinterpret_cast<__nv_bfloat16 *>(slot + SL_OST);
 #pragma unroll
-            for (int x = 0; x < 32; ++x) ost[(c32 + x) * kD + row] = __float2bfloat16_rn(v[x]);
-            uint32_t hi[32], lo[32];
+            for (int x = 0; x < 32; ++x) ost[(c32 + x) * kD + row] = __float2bfloat16_rn(v[x] * uu);
+            float sv[64];
+            float am;
+            const bool same = eu == es;  // uniform over the CTA
+            // same: S' in the state's scale; otherwise (U took its own scale this
+            // chunk) S' in fp32, unscaled, and a new scale for it
 #pragma unroll
             for (int part = 0; part < 2; ++part) {
                 float d[32];
                 tmem_ld32(trow + CT_S + 64 * half + 32 * part, v);
                 tmem_ld32(trow + CT_D + 64 * half + 32 * part, d);
                 tmem_wait_ld();
+                if (same) {
 #pragma unroll
-                for (int x = 0; x < 32; ++x) v[x] = fmaf(gC, v[x], d[x]);  // S' = Gamma_C S + dS
-                tmem_st32(trow + CT_S + 64 * half + 32 * part, v);
+                    for (int x = 0; x < 32; ++x) {
+                        sv[32 * part + x] = fmaf(gC, v[x], d[x]);
+                    }
+                } else {
+                    const float fs = gC * s_up;
 #pragma unroll
-                for (int x = 0; x < 32; x += 2) {
-                    const __half2 hh = __floats2half2_rn(v[x], v[x + 1]);
-                    const float2 hf = __half22float2(hh);
-                    hi[16 * part + x / 2] = *reinterpret_cast<const uint32_t *>(&hh);
-                    lo[16 * part + x / 2] = pack_half2(v[x] - hf.x, v[x + 1] - hf.y);
+                    for (int x = 0; x < 32; ++x) {
+                        sv[32 * part + x] = fmaf(fs, v[x], d[x] * uu);
+                    }
                 }
             }
-            tmem_st32u(trow + CT_SH + 32 * half, hi);
-            tmem_st32u(trow + CT_SL + 32 * half, lo);
-        }
-        poll_next(c);
-        GDN_CL_PHASE(0, 5);  // o staging, S copies
-        fence_proxy_async_smem();  // our writes to the slot precede the next bulk load into it
-        tmem_wait_st();
-        tc_fence_before_sync();
-        if (__syncthreads_or(timed_out ? 1 : 0)) {
-            if (tid == 0) {
-                raise_error(p.err, GDN_ERR_TIMEOUT);
-                if constexpr (kPool) pool_abort(p);
+            // a new scale for the unscaled sv: set es from the CTA maximum and apply it
+            auto rescale = [&]() {
+                am = cta_max(am, ms->red, warp, lane);
+                set_es(am > 0.f ? fp16_scale_exp(am) : es);
+#pragma unroll
+                for (int x = 0; x < 64; ++x) sv[x] *= sd;
+            };
+            am = max_abs<64>(sv);
+            if (!same) rescale();
+            store_state(sv);
+            split_state(sv);
+            poll_next(c);
+            GDN_CL_PHASE(0, 5);  // o staging, S copies
+            fence_proxy_async_smem();  // our writes to the slot precede the next bulk load into it
+            tmem_wait_st();
+            tc_fence_before_sync();
+            const unsigned b = cta_or8(
+                __reduce_or_sync(0xffffffffu, (same ? scale_bits(am) : 2u) | (timed_out ? 8u : 0u)),
+                ms->vote[1], warp, lane);
+            tc_fence_after_sync();
+            if (b & 8u) {
+                if (tid == 0) {
+                    raise_error(p.err, GDN_ERR_TIMEOUT);
+                    if constexpr (kPool) pool_abort(p);
+                }
+                aborted = true;
+            } else if (rescale_needed(b)) {  // rare: S' left the band
+#pragma unroll
+                for (int x = 0; x < 64; ++x) sv[x] *= s_up;  // exact: S' in fp32, unscaled
+                am = max_abs<64>(sv);
+                rescale();
+                store_state(sv);
+                split_state(sv);
+                tmem_wait_st();
+                tc_fence_before_sync();
+                __syncthreads();
+                tc_fence_after_sync();
             }
-            aborted = true;
         }
-        tc_fence_after_sync();
         GDN_CL_PHASE(0, 6);  // vote, free the slot
     }
 
-    if (!aborted && p.sT) {
+    if (!aborted && p.sT) {  // the master times 2^es
         float *dst = p.sT + (((int64_t)n * p.Hv + h) * kD + row) * kD;
 #pragma unroll 1
         for (int cc = 64 * half; cc < 64 * half + 64; cc += 32) {
@@ -1086,7 +1234,8 @@ __device__ void chain_role(uint8_t *sm, const CUtensorMap *tm_o, const ChainPara
             tmem_wait_ld();
 #pragma unroll
             for (int x = 0; x < 32; x += 4)
-                *reinterpret_cast<float4 *>(dst + cc + x) = make_float4(v[x], v[x + 1], v[x + 2], v[x + 3]);
+                *reinterpret_cast<float4 *>(dst + cc + x) =
+                    make_float4(v[x] * s_up, v[x + 1] * s_up, v[x + 2] * s_up, v[x + 3] * s_up);
         }
     }
     if (!aborted && nch > 0) store_o(nch - 1);  // the last chunk's output
@@ -1122,7 +1271,7 @@ __device__ __forceinline__ uint32_t *setup_role(uint8_t *sm, bool chain, uint32_
     } else {
         ProdMisc *ms = reinterpret_cast<ProdMisc *>(sm + P_MISC);
         tmem_slot = &ms->tmem_base;
-        ncols = 256;
+        ncols = 512;
         if (tid == 0) {
             mbar_init(&ms->tma_bar[0], 1);
             mbar_init(&ms->tma_bar[1], 1);
@@ -1267,6 +1416,8 @@ bool fill_params(const PrefillArgs &a, ChainParams &p, CUtensorMap &mq, CUtensor
     p.max_chunks = (int)((a.T + kC - 1) / kC);
     p.ring_slots = kClusterRingSlots;
     p.recall_first = a.order == GDN_ORDER_RECALL_FIRST;
+    p.flag_wait_limit = kWaitLimit;
+    p.skip_unit = -1;
     return true;
 }
 }  // namespace
@@ -1293,6 +1444,8 @@ cudaError_t launch_prefill_pool(const PrefillArgs &a, cudaStream_t s) {
     p.flags = static_cast<uint32_t *>(a.ws);
     p.ring = static_cast<uint8_t *>(a.ws) + fb;
     p.ring_slots = kPoolRingSlots;
+    if (a.debug_flag_wait > 0) p.flag_wait_limit = a.debug_flag_wait;
+    p.skip_unit = a.debug_skip_unit;
     // the chunk counter, abort flag and hand-off flags start at zero
     cudaError_t e = cudaMemsetAsync(a.ws, 0, fb, s);
     if (e != cudaSuccess) return e;

@@ -99,12 +99,17 @@ constexpr uint32_t OFF_AS = OFF_X;                   // float [64][kAS4]
 constexpr uint32_t OFF_TS = OFF_X + 64 * kAS4 * 4;      // float [64][kTS], 16-byte aligned
 constexpr uint32_t OFF_XS = OFF_TS + 64 * kTS * 4;   // float [1024] level partials
 constexpr uint32_t OFF_P16 = 163840;    // 64 rows x 128 B                  (B: P, K-major)
-constexpr uint32_t OFF_TBH = 172032;    // 64 rows x 128 B                  (B: T diag b, hi)
-constexpr uint32_t OFF_TBL = 180224;    //                                  (B: T diag b, lo)
-constexpr uint32_t OFF_TGH = 188416;    //                                  (B: T diag(b Gamma), hi)
-constexpr uint32_t OFF_TGL = 196608;    //                                  (B: T diag(b Gamma), lo)
+// T diag(b) as bf16 hi / mid / lo and T diag(b Gamma) as fp16 hi / lo, each part
+// 64 rows x 128 B; the parts of each are consecutive, so one B operand of
+// N = 192 (or 128) rows takes all of them, each part's product landing in
+// its own accumulator columns.
+constexpr uint32_t OFF_TBH = 172032;    // (B: T diag b, hi)
+constexpr uint32_t OFF_TBM = 180224;    // (B: T diag b, mid)
+constexpr uint32_t OFF_TBL = 188416;    // (B: T diag b, lo)
+constexpr uint32_t OFF_TGH = 196608;    // (B: T diag(b Gamma), hi)
+constexpr uint32_t OFF_TGL = 204800;    // (B: T diag(b Gamma), lo)
 constexpr uint32_t OFF_OST = OFF_TBH;   // o staging [64 tokens][128] bf16 (TB tiles are dead)
-constexpr uint32_t OFF_MISC = 204800;
+constexpr uint32_t OFF_MISC = 212992;
 static_assert(OFF_XS + 1024 * 4 <= OFF_P16, "solve scratch overflows");
 static_assert(OFF_TS % 16 == 0 && OFF_XS % 16 == 0, "float4 scratch must be aligned");
 
@@ -121,11 +126,23 @@ struct Misc {
     int32_t safe;     // |gamma| <= 60 over the chunk
     int32_t hp;       // Gamma_C >= kHighPrecisionDecay
     float gsum_next;  // sum of g over the next (or first) chunk
+    alignas(16) uint32_t vote[2][8];  // per-warp vote words of the U and state epilogues
+    float red[8];                     // per-warp maxima of a rescale
 };
+static_assert(offsetof(Misc, vote) % 16 == 0 && OFF_MISC % 16 == 0, "vote words read as uint4");
 constexpr uint32_t kSmemBytes = OFF_MISC + sizeof(Misc) + 1024;  // + alignment slack
 
-// TMEM column map (fp32 columns; 512 allocated, 448 used)
-constexpr uint32_t TM_S = 0, TM_G = 128, TM_U = 192, TM_WT = 256, TM_O = 320, TM_R = 384;
+// TMEM column map (fp32 columns; 512 allocated), each region used in turn:
+//   TM_S 0..127    the fp32 state
+//   TM_G 128..191  the Gram; then TM_U 128..319, U~^T as the products of T diag(b)'s
+//                  hi, mid and lo parts (64 columns each)
+//   TM_O 320..383  S Q^T, then the chunk output
+//   TM_WT 384..511 W^T as the products of T diag(b Gamma)'s hi and lo parts; then
+//   TM_R 384..447  S W^T; then TM_D 384..511, the state increment dS
+constexpr uint32_t TM_S = 0, TM_G = 128, TM_U = 128, TM_O = 320, TM_WT = 384, TM_R = 384,
+                   TM_D = 384;
+constexpr uint32_t IDESC_MK_N192_BF16 = make_idesc_f16(128, 192, 1, 0, 1);
+constexpr uint32_t IDESC_MK_N128 = make_idesc_f16(128, 128, 1, 0);
 
 
 struct TcParams {
@@ -206,24 +223,61 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem = ms->tmem_base;
     const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);  // + column
 
+    // Value-side operands are held with a power-of-two scale, uniform over
+    // the unit: the fp32 master state in TMEM is S * 2^-es (times the next
+    // chunk's Gamma_C, applied ahead), and its fp16 hi / lo copies (the A
+    // operand of S Q^T and S W^T) are split from S * 2^-es directly, so the
+    // products come out scaled by 2^-es.  U and U' are held as U * 2^-eu,
+    // where eu is es unless U's magnitudes leave the band [kScaleLo, kScaleHi)
+    // in that scale.  Both epilogues vote on their largest scaled magnitude;
+    // the rare chunk whose values left the band recomputes them in fp32 and
+    // takes a new scale (fp16_scale_exp).  The scaling is exact, so no
+    // value-side operand over- or underflows fp16, whatever the scale of v
+    // and S0, and the results scale exactly with it.
+    int es = 0, eu = 0;
+    float s_up = 1.f, sd = 1.f;  // 2^es, 2^-es
+    auto set_es = [&](int e) {
+        es = e;
+        s_up = exp2i(e);
+        sd = exp2i(-e);
+    };
+    // this thread's 64 scaled values of a state row -> the fp16 hi (and lo) tiles
+    auto split_state = [&](const float (&sv)[64], bool with_lo) {
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {
+            float v[32];
+#pragma unroll
+            for (int x = 0; x < 32; ++x) v[x] = sv[32 * part + x];
+            store_split32(sm + OFF_S16H + half * 16384, sm + OFF_S16L + half * 16384, row,
+                          32 * part, v, with_lo);
+        }
+    };
+
     // ---- initial state: Gamma_C(first chunk) * S -> TMEM accumulator; S -> fp16 hi/lo ----
     {
         const float scale0 = t_begin < t_end ? expf(ms->gsum_next) : 1.f;
-        const float *src = p.s0 ? p.s0 + (((int64_t)n * p.Hv + h) * kD + row) * kD : nullptr;
-#pragma unroll 1
-        for (int c = 64 * half; c < 64 * half + 64; c += 32) {
+        const float *src = p.s0 ? p.s0 + (((int64_t)n * p.Hv + h) * kD + row) * kD + 64 * half
+                                : nullptr;
+        float sv[64];
+        float am = 0.f;
+#pragma unroll
+        for (int x = 0; x < 64; x += 4) {
+            const float4 f = src ? *reinterpret_cast<const float4 *>(src + x)
+                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+            sv[x] = f.x; sv[x + 1] = f.y; sv[x + 2] = f.z; sv[x + 3] = f.w;
+            am = fmaxf(am, fmaxf(fmaxf(fabsf(f.x), fabsf(f.y)), fmaxf(fabsf(f.z), fabsf(f.w))));
+        }
+        am = cta_max(am, ms->red, warp, lane);
+        set_es(am > 0.f ? fp16_scale_exp(am) : 0);
+#pragma unroll
+        for (int x = 0; x < 64; ++x) sv[x] *= sd;
+        split_state(sv, true);
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {
             float v[32];
 #pragma unroll
-            for (int x = 0; x < 32; x += 4) {
-                const float4 f = src ? *reinterpret_cast<const float4 *>(src + c + x)
-                                     : make_float4(0.f, 0.f, 0.f, 0.f);
-                v[x] = f.x; v[x + 1] = f.y; v[x + 2] = f.z; v[x + 3] = f.w;
-            }
-            store_split32(sm + OFF_S16H + (c / 64) * 16384, sm + OFF_S16L + (c / 64) * 16384, row,
-                          c % 64, v, true);
-#pragma unroll
-            for (int x = 0; x < 32; ++x) v[x] *= scale0;
-            tmem_st32(trow + TM_S + c, v);
+            for (int x = 0; x < 32; ++x) v[x] = sv[32 * part + x] * scale0;
+            tmem_st32(trow + TM_S + 64 * half + 32 * part, v);
         }
     }
     fence_proxy_async_smem();
@@ -234,6 +288,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     uint32_t tma_phase = 0, mma_phase = 0;
     bool aborted = false;
+    float kmax = 0.f;             // largest key-side value this thread has put into fp16
+    bool range_reported = false;
     bool timed_out = false;  // this thread saw a bounded wait expire (voted on once per chunk)
     bool tma_outstanding = false;  // a tile load was issued and not yet waited for
 
@@ -332,7 +388,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_commit(&ms->mma_bar);
         }
         // 16-byte chunk x of the tile region starting at `base`; row = token
-        // (offset / 128 within each 8 KB box); padding rows become zeros
+        // (offset / 128 within each 8 KB box); padding rows become zeros.  K and
+        // Q go to fp16 once the Gram products have read them; V stays bf16 (the
+        // U~ product splits its other operand three ways in bf16).
         auto convert16 = [&](uint8_t *base, int x) {
             uint4 *ptr = reinterpret_cast<uint4 *>(base) + x;
             const int r = (x >> 3) & 63;
@@ -345,14 +403,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int q2 = 0; q2 < 4; ++q2) {
                     const __nv_bfloat162 b2 = *reinterpret_cast<const __nv_bfloat162 *>(&w[q2]);
                     const float2 f = __bfloat1622float2(b2);
+                    kmax = fmaxf(kmax, fmaxf(fabsf(f.x), fabsf(f.y)));
                     w[q2] = pack_half2(f.x, f.y);
                 }
                 val = make_uint4(w[0], w[1], w[2], w[3]);
             }
             *ptr = val;
         };
-#pragma unroll
-        for (int k = 0; k < 1024 / kThreads; ++k) convert16(sm + OFF_V, tid + k * kThreads);  // V
         if (!mbar_wait_bounded(&ms->mma_bar, mma_phase, kWaitLimit)) timed_out = true;
         mma_phase ^= 1;
         tc_fence_after_sync();
@@ -394,7 +451,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int x = 0; x < 32; ++x) v[x] = (c + x <= r) ? v[x] : 0.f;
 #pragma unroll
-                for (int e = 0; e < 32; e += 8) st_row_chunk(sm + OFF_P16, r, (c + e) / 8, pack8(v + e));
+                for (int e = 0; e < 32; e += 8)
+                    st_row_chunk(sm + OFF_P16, r, (c + e) / 8, pack8_track(v + e, kmax));
             }
         }
         __syncthreads();
@@ -404,7 +462,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         solve_tril64(As, Ts, Xs, tid);
         GDN_TC_PHASE(6);
 
-        // ---- B operands: rows r of T diag(b) and T diag(b Gamma), fp16 hi / lo ----
+        // ---- B operands: rows r of T diag(b) (bf16 hi / mid / lo) and
+        //      T diag(b Gamma) (fp16 hi / lo, as K) ----
         {
             const int grp = tid >> 6, r = tid & 63;
             const bool tg = grp >= 2;
@@ -421,8 +480,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     x[e + q] = (i <= r) ? tv[q] * scale[i] : 0.f;
                 }
             }
-            store_split32(sm + (tg ? OFF_TGH : OFF_TBH), sm + (tg ? OFF_TGL : OFF_TBL), r, c, x,
-                          !tg || hp);
+            if (tg)
+                store_split32(sm + OFF_TGH, sm + OFF_TGL, r, c, x, hp, kmax);
+            else
+                store_split32_bf16x3(sm + OFF_TBH, sm + OFF_TBM, sm + OFF_TBL, r, c, x);
         }
         publish();
         GDN_TC_PHASE(7);
@@ -430,22 +491,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ---- U~^T = V^T (T diag b)^T, W^T = K^T (T diag(b Gamma))^T, S Q^T ----
         if (tid == 0) {
 #pragma unroll
-            for (int pass = 0; pass < 2; ++pass)
+            for (int ks = 0; ks < 4; ++ks) {  // bf16 V times [hi | mid | lo] of T diag(b)
+                const uint64_t a = make_sdesc(sbase + OFF_V + ks * 2048, 8192, 1024);
+                const uint64_t b = make_sdesc(sbase + OFF_TBH + ks * 32, 16, 1024);
+                mma_f16_ss(tmem + TM_U, a, b, IDESC_MK_N192_BF16, ks != 0);
+            }
+            const uint32_t idesc_w = hp ? IDESC_MK_N128 : IDESC_MK_N64;
 #pragma unroll
-                for (int ks = 0; ks < 4; ++ks) {
-                    const uint64_t a = make_sdesc(sbase + OFF_V + ks * 2048, 8192, 1024);
-                    const uint64_t b =
-                        make_sdesc(sbase + (pass ? OFF_TBL : OFF_TBH) + ks * 32, 16, 1024);
-                    mma_f16_ss(tmem + TM_U, a, b, IDESC_MK_N64, (pass | ks) != 0);
-                }
-            for (int pass = 0; pass < (hp ? 2 : 1); ++pass)
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks) {
-                    const uint64_t a = make_sdesc(sbase + OFF_KQ + ks * 2048, 16384, 1024);
-                    const uint64_t b =
-                        make_sdesc(sbase + (pass ? OFF_TGL : OFF_TGH) + ks * 32, 16, 1024);
-                    mma_f16_ss(tmem + TM_WT, a, b, IDESC_MK_N64, (pass | ks) != 0);
-                }
+            for (int ks = 0; ks < 4; ++ks) {  // fp16 K times [hi | lo] of T diag(b Gamma)
+                const uint64_t a = make_sdesc(sbase + OFF_KQ + ks * 2048, 16384, 1024);
+                const uint64_t b = make_sdesc(sbase + OFF_TGH + ks * 32, 16, 1024);
+                mma_f16_ss(tmem + TM_WT, a, b, idesc_w, ks != 0);
+            }
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
                 const uint64_t a =
@@ -458,18 +515,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_sync_point();
         GDN_TC_PHASE(8);
 
-        // ---- W^T rows -> fp16 B tiles (MN-major); S Q^T rows scaled by Gamma (in place) ----
+        // ---- W^T rows -> fp16 B tiles (MN-major) ----
         {
             const int c = 32 * half;
             float v[32];
             tmem_ld32(trow + TM_WT + c, v);
-            tmem_wait_ld();
-            store_split32(sm + OFF_WST, sm + OFF_WST + 16384, row, c, v, hp);
-            tmem_ld32(trow + TM_O + c, v);
-            tmem_wait_ld();
+            if (hp) {
+                float w2[32];
+                tmem_ld32(trow + TM_WT + 64 + c, w2);
+                tmem_wait_ld();
 #pragma unroll
-            for (int x = 0; x < 32; ++x) v[x] *= ms->Gam[c + x];
-            tmem_st32(trow + TM_O + c, v);
+                for (int x = 0; x < 32; ++x) v[x] += w2[x];
+            }
+            tmem_wait_ld();
+            store_split32(sm + OFF_WST, sm + OFF_WST + 16384, row, c, v, hp, kmax);
         }
         publish();
         GDN_TC_PHASE(9);
@@ -490,34 +549,80 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_sync_point();
         GDN_TC_PHASE(10);
 
-        // ---- U = U~ - R (row i of U^T), U' = U diag(Gamma_C/Gamma) split, U fp16 ----
+        // ---- U = U~ - R (row i of U^T) in the state's scale; U' = U diag(Gamma_C/Gamma)
+        //      split and U; S Q^T rows scaled by Gamma.  A vote on U's largest
+        //      scaled magnitude; if it left the band, U takes a scale of its own
+        //      and O follows it. ----
         {
             const int c = 32 * half;
-            float u[32], r0[32];
-            tmem_ld32(trow + TM_U + c, u);
-            tmem_ld32(trow + TM_R + c, r0);
-            tmem_wait_ld();
+            float u[32];
+            // U~ (the sum of its three parts) into ut, R (scaled by 2^-es) into u
+            auto load_ut_r = [&](float (&ut)[32]) {
+                float t1[32];
+                tmem_ld32(trow + TM_U + c, ut);
+                tmem_ld32(trow + TM_U + 64 + c, t1);
+                tmem_ld32(trow + TM_U + 128 + c, u);
+                tmem_wait_ld();
 #pragma unroll
-            for (int x = 0; x < 32; ++x) {
-                u[x] -= r0[x];
-                r0[x] = u[x] * ms->eC[c + x];
+                for (int x = 0; x < 32; ++x) ut[x] += t1[x] + u[x];
+                tmem_ld32(trow + TM_R + c, u);
+                tmem_wait_ld();
+            };
+            auto store_u = [&]() {  // U' hi / lo and U (scaled) -> shared memory
+                float up[32];
+#pragma unroll
+                for (int x = 0; x < 32; ++x) up[x] = u[x] * ms->eC[c + x];
+                store_split32(sm + OFF_UP, sm + OFF_UP + 16384, row, c, up, true);
+#pragma unroll
+                for (int e = 0; e < 32; e += 8)
+                    st_row_chunk(sm + OFF_U16, row, (c + e) / 8, pack8(u + e));
+            };
+            auto scale_o = [&](float f) {  // S Q^T rows times f Gamma
+                float ov[32];
+                tmem_ld32(trow + TM_O + c, ov);
+                tmem_wait_ld();
+#pragma unroll
+                for (int x = 0; x < 32; ++x) ov[x] *= f * ms->Gam[c + x];
+                tmem_st32(trow + TM_O + c, ov);
+            };
+            float am;
+            {
+                float ut[32];
+                load_ut_r(ut);
+#pragma unroll
+                for (int x = 0; x < 32; ++x) u[x] = fmaf(ut[x], sd, -u[x]);  // U 2^-es (R: 2^-es)
+                am = max_abs<32>(u);
             }
-            store_split32(sm + OFF_UP, sm + OFF_UP + 16384, row, c, r0, true);
-#pragma unroll
-            for (int e = 0; e < 32; e += 8) st_row_chunk(sm + OFF_U16, row, (c + e) / 8, pack8(u + e));
+            eu = es;
+            store_u();
             if (warp == 0) warp0_sum_to(gpre0 + gpre1, &ms->gsum_next);  // next chunk's log-decay
+            const unsigned b =
+                cta_or8(__reduce_or_sync(0xffffffffu, scale_bits(am)), ms->vote[0], warp, lane);
+            if (rescale_needed(b)) {  // rare: U takes its own scale
+                float ut[32];
+                load_ut_r(ut);  // U~ and R are still in place
+#pragma unroll
+                for (int x = 0; x < 32; ++x) u[x] = fmaf(-s_up, u[x], ut[x]);  // U in fp32, unscaled
+                am = cta_max(max_abs<32>(u), ms->red, warp, lane);
+                eu = fp16_scale_exp(am);
+                const float ud = exp2i(-eu);
+#pragma unroll
+                for (int x = 0; x < 32; ++x) u[x] *= ud;
+                store_u();
+            }
+            scale_o(exp2c(es - eu));
         }
         publish();
         GDN_TC_PHASE(11);
 
-        // ---- S += [U'hi | U'lo] [K ; K];  O += U^T P^T ----
+        // ---- dS = [U'hi | U'lo] [K ; K] (rows scaled by 2^-eu);  O += U^T P^T ----
         if (tid == 0) {
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
                 const uint64_t a =
                     make_sdesc(sbase + OFF_UP + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
                 const uint64_t b = make_sdesc(sbase + OFF_KQ + (ks & 3) * 2048, 16384, 1024);
-                mma_f16_ss(tmem + TM_S, a, b, IDESC_KM_N128, 1);
+                mma_f16_ss(tmem + TM_D, a, b, IDESC_KM_N128, ks > 0);
             }
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) {
@@ -534,31 +639,72 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         GDN_TC_PHASE(12);
 
-        // ---- o rows -> staging tile; new S -> fp16 hi/lo; master *= Gamma_C(next) ----
+        // ---- o rows -> staging tile; new S = Gamma_C S + dS (scaled) -> fp16 hi/lo;
+        //      master = S * Gamma_C(next); a vote on S's largest scaled
+        //      magnitude (rescale if it left the band) ----
         {
             const int c = 32 * half;
+            const float uu = exp2i(eu);  // O and dS rows come scaled by 2^-eu
             float v[32];
             tmem_ld32(trow + TM_O + c, v);
             tmem_wait_ld();
             __nv_bfloat16 *ost = reinterpret_cast<__nv_bfloat16 *>(sm + OFF_OST);
 #pragma unroll
-            for (int x = 0; x < 32; ++x) ost[(c + x) * kD + row] = __float2bfloat16_rn(v[x]);
+            for (int x = 0; x < 32; ++x) ost[(c + x) * kD + row] = __float2bfloat16_rn(v[x] * uu);
             const float gnext = has_next ? expf(ms->gsum_next) : 1.f;
             const bool lo_next = gnext >= kHighPrecisionDecay;
-#pragma unroll 1
-            for (int cc = 64 * half; cc < 64 * half + 64; cc += 32) {
-                tmem_ld32(trow + TM_S + cc, v);
-                tmem_wait_ld();
-                store_split32(sm + OFF_S16H + (cc / 64) * 16384, sm + OFF_S16L + (cc / 64) * 16384,
-                              row, cc % 64, v, lo_next);
-                if (has_next) {
+            const bool same = eu == es;  // uniform over the CTA
+            // same: S' in the state's scale; otherwise (U took its own scale this
+            // chunk) S' in fp32, unscaled, and a new scale for it
+            float sv[64];
+            float am;
 #pragma unroll
-                    for (int x = 0; x < 32; ++x) v[x] *= gnext;
-                    tmem_st32(trow + TM_S + cc, v);
+            for (int part = 0; part < 2; ++part) {
+                float d[32];
+                tmem_ld32(trow + TM_S + 64 * half + 32 * part, v);
+                tmem_ld32(trow + TM_D + 64 * half + 32 * part, d);
+                tmem_wait_ld();
+                if (same) {
+#pragma unroll
+                    for (int x = 0; x < 32; ++x) {
+                        sv[32 * part + x] = v[x] + d[x];
+                    }
+                } else {
+#pragma unroll
+                    for (int x = 0; x < 32; ++x) {
+                        sv[32 * part + x] = fmaf(s_up, v[x], d[x] * uu);
+                    }
                 }
             }
+            auto rescale = [&]() {  // a new scale for the unscaled sv, from the CTA maximum
+                am = cta_max(am, ms->red, warp, lane);
+                set_es(am > 0.f ? fp16_scale_exp(am) : es);
+#pragma unroll
+                for (int x = 0; x < 64; ++x) sv[x] *= sd;
+            };
+            auto store_master = [&]() {  // gnext = 1 after the last chunk
+#pragma unroll
+                for (int part = 0; part < 2; ++part) {
+#pragma unroll
+                    for (int x = 0; x < 32; ++x) v[x] = sv[32 * part + x] * gnext;
+                    tmem_st32(trow + TM_S + 64 * half + 32 * part, v);
+                }
+            };
+            am = max_abs<64>(sv);
+            if (!same) rescale();
+            split_state(sv, lo_next);
+            store_master();
+            const unsigned b = cta_or8(__reduce_or_sync(0xffffffffu, same ? scale_bits(am) : 2u),
+                                       ms->vote[1], warp, lane);
+            if (rescale_needed(b)) {  // rare: S' left the band
+#pragma unroll
+                for (int x = 0; x < 64; ++x) sv[x] *= s_up;  // exact: S' in fp32, unscaled
+                am = max_abs<64>(sv);
+                rescale();
+                split_state(sv, lo_next);  // published by the barrier at the chunk's end
+                store_master();
+            }
         }
-        __syncthreads();
         {
             const uint4 *ost = reinterpret_cast<const uint4 *>(sm + OFF_OST);
 #pragma unroll
@@ -572,6 +718,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
         }
+        // a key-side fp16 operand of this chunk (K, Q, P, T diag(b Gamma), W^T)
+        // overflowed: report it once per thread (the unit's results are then
+        // unspecified; the computation goes on)
+        if (kmax >= kFp16Overflow && !range_reported) {
+            raise_error(p.err, GDN_ERR_RANGE);
+            range_reported = true;
+        }
         fence_proxy_async_smem();
         tmem_wait_st();
         tc_fence_before_sync();
@@ -583,7 +736,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         GDN_TC_PHASE(13);
     }
 
-    // ---- final state ----
+    // ---- final state: the master times 2^es ----
     if (!aborted && p.sT) {
         float *dst = p.sT + (((int64_t)n * p.Hv + h) * kD + row) * kD;
 #pragma unroll 1
@@ -593,7 +746,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_wait_ld();
 #pragma unroll
             for (int x = 0; x < 32; x += 4)
-                *reinterpret_cast<float4 *>(dst + c + x) = make_float4(v[x], v[x + 1], v[x + 2], v[x + 3]);
+                *reinterpret_cast<float4 *>(dst + c + x) =
+                    make_float4(v[x] * s_up, v[x + 1] * s_up, v[x + 2] * s_up, v[x + 3] * s_up);
         }
     }
     if (aborted) {

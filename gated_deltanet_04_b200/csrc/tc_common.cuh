@@ -53,6 +53,116 @@ __device__ __forceinline__ uint4 pack8(const float *x) {
                       pack_half2(x[6], x[7]));
 }
 
+// Largest |v[i]| over N values (N a multiple of 8), as a tree of eight
+// independent running maxima rather than one dependent chain.
+template <int N>
+__device__ __forceinline__ float max_abs(const float *v) {
+    float m[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) m[j] = fabsf(v[j]);
+#pragma unroll
+    for (int i = 8; i < N; i += 8)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) m[j] = fmaxf(m[j], fabsf(v[i + j]));
+    return fmaxf(fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3])),
+                 fmaxf(fmaxf(m[4], m[5]), fmaxf(m[6], m[7])));
+}
+
+// The same with the largest |x| folded into amax (range check of fp16 operands).
+__device__ __forceinline__ uint4 pack8_track(const float *x, float &amax) {
+    amax = fmaxf(amax, max_abs<8>(x));
+    return pack8(x);
+}
+
+// x = hi + mid + lo with all three parts bfloat16 (exact for normal fp32 x:
+// each residual has at most 16, then 8, significant bits), 8 values.
+__device__ __forceinline__ void split8_bf16x3(const float *x, uint4 &hi, uint4 &mid, uint4 &lo) {
+    uint32_t h[4], m[4], l[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const __nv_bfloat162 hh = __floats2bfloat162_rn(x[2 * j], x[2 * j + 1]);
+        const float2 hf = __bfloat1622float2(hh);
+        const float r0 = x[2 * j] - hf.x, r1 = x[2 * j + 1] - hf.y;
+        const __nv_bfloat162 mm = __floats2bfloat162_rn(r0, r1);
+        const float2 mf = __bfloat1622float2(mm);
+        const __nv_bfloat162 ll = __floats2bfloat162_rn(r0 - mf.x, r1 - mf.y);
+        h[j] = *reinterpret_cast<const uint32_t *>(&hh);
+        m[j] = *reinterpret_cast<const uint32_t *>(&mm);
+        l[j] = *reinterpret_cast<const uint32_t *>(&ll);
+    }
+    hi = make_uint4(h[0], h[1], h[2], h[3]);
+    mid = make_uint4(m[0], m[1], m[2], m[3]);
+    lo = make_uint4(l[0], l[1], l[2], l[3]);
+}
+
+// ---- power-of-two operand scaling ----
+// A value-side fp16 operand (the state, U, U') is stored as x * 2^-e, with e
+// chosen per accumulator row from that row's largest magnitude, and the MMA
+// result row is multiplied back by 2^e in fp32.  Both multiplications are
+// exact, so the scaling changes no bit of the arithmetic except that every
+// value now lies in fp16's normal range.
+
+// e such that amax * 2^-e lies in [2^10, 2^11), clamped so that 2^e and
+// 2^-e are normal floats.  That leaves fp16 four binades of headroom above
+// the largest scaled value (other operands that share the scale, such as U
+// beside the state, may exceed it) and six below it before a hi / lo split
+// of the largest values loses bits to subnormals.
+__device__ __forceinline__ int fp16_scale_exp(float amax) {
+    const int e = (int)((__float_as_uint(amax) >> 23) & 0xffu) - 127 - 10;
+    return min(max(e, -126), 126);
+}
+
+// 2^e for e in [-126, 127].
+__device__ __forceinline__ float exp2i(int e) { return __uint_as_float((uint32_t)(e + 127) << 23); }
+
+// Largest fp16 magnitude that does not round to infinity is just below this.
+constexpr float kFp16Overflow = 65520.f;
+
+// 2^e with e clamped to [-126, 127].
+__device__ __forceinline__ float exp2c(int e) { return exp2i(min(max(e, -126), 127)); }
+
+// The band a scaled value-side operand is kept in: its largest magnitude in
+// [kScaleLo, kScaleHi).  Above it fp16 would overflow; below it the lo parts
+// of a hi / lo split drift towards fp16's subnormals.
+constexpr float kScaleHi = 32768.f;
+constexpr float kScaleLo = 16.f;
+
+// Bits of a scale vote: some value at or above the band, some value at or
+// above its floor, some value nonzero.
+__device__ __forceinline__ unsigned scale_bits(float amax) {
+    return (amax >= kScaleHi ? 1u : 0u) | (amax >= kScaleLo ? 2u : 0u) | (amax > 0.f ? 4u : 0u);
+}
+// Whether voted bits call for a new scale: something overflowed, or nothing
+// reaches the floor although something is nonzero.
+__device__ __forceinline__ bool rescale_needed(unsigned bits) {
+    return (bits & 1u) || ((bits & 4u) && !(bits & 2u));
+}
+
+// OR of a warp-uniform word over the CTA's 8 warps: lane 0 of each warp posts
+// it to words[warp], and after the CTA barrier every thread reads all 8.  The
+// barrier is part of the call; a second use of `words` must be separated from
+// this one by another CTA barrier.
+__device__ __forceinline__ unsigned cta_or8(unsigned x, uint32_t *words, int warp, int lane) {
+    if (lane == 0) words[warp] = x;
+    __syncthreads();
+    const uint4 a = *reinterpret_cast<const uint4 *>(words);
+    const uint4 b = *reinterpret_cast<const uint4 *>(words + 4);
+    return a.x | a.y | a.z | a.w | b.x | b.y | b.z | b.w;
+}
+
+// Maximum of x (>= 0) over the CTA's 256 threads; red holds 8 floats.  Ends
+// with every thread holding the result; contains one CTA barrier, and a
+// second use of red must be separated from this one by another.
+__device__ __forceinline__ float cta_max(float x, float *red, int warp, int lane) {
+    const unsigned m = __reduce_max_sync(0xffffffffu, __float_as_uint(x));  // x >= 0: bit order
+    if (lane == 0) red[warp] = __uint_as_float(m);
+    __syncthreads();
+    float r = red[0];
+#pragma unroll
+    for (int w = 1; w < 8; ++w) r = fmaxf(r, red[w]);
+    return r;
+}
+
 __device__ __forceinline__ void st_row_chunk(uint8_t *tile, uint32_t row, uint32_t chunk,
                                              uint4 val) {
     *reinterpret_cast<uint4 *>(tile + sw128(row, chunk * 16)) = val;
@@ -68,6 +178,28 @@ __device__ __forceinline__ void store_split32(uint8_t *hi_tile, uint8_t *lo_tile
         split8(v + e, hi, lo);
         st_row_chunk(hi_tile, row, (c + e) / 8, hi);
         if (with_lo) st_row_chunk(lo_tile, row, (c + e) / 8, lo);
+    }
+}
+
+// store_split32 with the largest |v| folded into amax.
+__device__ __forceinline__ void store_split32(uint8_t *hi_tile, uint8_t *lo_tile, int row, int c,
+                                              const float *v, bool with_lo, float &amax) {
+    amax = fmaxf(amax, max_abs<32>(v));
+    store_split32(hi_tile, lo_tile, row, c, v, with_lo);
+}
+
+// Writes 32 consecutive values of a row of three 128-byte swizzled bf16 tiles
+// as the hi, mid and lo parts of an exact three-way split.
+__device__ __forceinline__ void store_split32_bf16x3(uint8_t *hi_tile, uint8_t *mid_tile,
+                                                     uint8_t *lo_tile, int row, int c,
+                                                     const float *v) {
+#pragma unroll
+    for (int e = 0; e < 32; e += 8) {
+        uint4 hi, mid, lo;
+        split8_bf16x3(v + e, hi, mid, lo);
+        st_row_chunk(hi_tile, row, (c + e) / 8, hi);
+        st_row_chunk(mid_tile, row, (c + e) / 8, mid);
+        st_row_chunk(lo_tile, row, (c + e) / 8, lo);
     }
 }
 

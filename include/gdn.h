@@ -38,7 +38,8 @@
  * Errors: argument errors are returned synchronously and nothing is launched.
  * A failed launch returns GDN_ERR_CUDA (cudaGetLastError, no synchronisation).
  * Errors only the device can see (a malformed cu_seqlens, a bounded wait that
- * expired) are written as a gdn_status value to *dev_error_flag when that
+ * expired, an fp16 range overflow of a q/k-side operand) are written as a
+ * gdn_status value to *dev_error_flag when that
  * optional device int32 is given; the caller zeroes it beforehand and reads it
  * after synchronising.  A unit (sequence, head) that detects such an error
  * writes no output for itself.  No C++ exception crosses this interface.  The
@@ -67,7 +68,8 @@ typedef enum gdn_status {
     GDN_ERR_CUDA = 3,             /* a CUDA runtime call or launch failed */
     GDN_ERR_TIMEOUT = 4,          /* device: a bounded wait expired */
     GDN_ERR_BAD_SEQLENS = 5,      /* device: cu_seqlens malformed */
-    GDN_ERR_BAD_SLOT = 6          /* device: a state slot index out of range */
+    GDN_ERR_BAD_SLOT = 6,         /* device: a state slot index out of range */
+    GDN_ERR_RANGE = 7             /* device: a q/k-side operand overflowed fp16 (see gdn_prefill) */
 } gdn_status;
 
 typedef enum gdn_dtype {
@@ -106,6 +108,19 @@ typedef enum gdn_dtype {
  * {16, 32, 64, 128} and either dtype runs an exact fp32 token-recurrent CUDA
  * kernel.  Anything else returns GDN_ERR_UNSUPPORTED.  gdn_prefill_ex below
  * selects the kernel explicitly.
+ *
+ * Value range of the tensor-core kernels.  v, the states and every quantity
+ * linear in them (U, the state increments, o) have no range limit beyond
+ * fp32's: they enter the fp16 tensor-core operands with a power-of-two scale
+ * chosen per chunk from their largest magnitude, so the results scale exactly
+ * with v and initial_state (scaling both by 2^s scales o and final_state by
+ * 2^s, bit for bit).  q and k, and the per-chunk factors built from k, beta
+ * and g (the masked Q K^T, the inverse of the chunk's triangular system times
+ * beta, W), are held in fp16 without scaling: an entry that reaches 65520 in
+ * magnitude is reported as GDN_ERR_RANGE through dev_error_flag (the results
+ * of that call are then unspecified).  q and k entries below 2^-14 in
+ * magnitude lose relative precision to fp16 subnormals; rows scaled to unit
+ * length, as the gated delta rule is used, are far from both limits.
  */
 GDN_API gdn_status gdn_prefill(const void *q, const void *k, const void *v, gdn_dtype io_dtype,
                        const float *g, const float *beta, const float *initial_state,
@@ -361,6 +376,32 @@ GDN_API gdn_status gdn_short_conv_norm(const void *xq, const void *xk, const voi
                                        int64_t T, int32_t Hqk, int32_t Hv, int32_t Dk, int32_t Dv,
                                        void *q, void *k, void *v, int32_t *dev_error_flag,
                                        void *stream);
+
+/*
+ * gdn_debug_prefill_pool_stall -- FOR TESTING THE TIMEOUT PATH ONLY.
+ * gdn_prefill_ex with kernel GDN_PREFILL_POOL, except that the producer CTAs
+ * never prepare the chunks of (sequence, head) unit `skip_unit` (n * Hv + h),
+ * and that every spin on a hand-off flag in workspace memory (a chain waiting
+ * for its next chunk, a producer waiting for a free ring slot) gives up after
+ * `flag_wait_cycles` SM clocks instead of about 2^31.  The chain of the skipped
+ * unit therefore waits for a chunk that never comes, with no copy in flight
+ * into its shared memory; when its wait gives up it reports GDN_ERR_TIMEOUT
+ * through *dev_error_flag and raises the kernel's abort flag, every other CTA
+ * stops at its next wait, and the launch ends.  Outputs are unspecified.  The
+ * context stays usable: later calls run normally.  skip_unit < 0 or
+ * flag_wait_cycles <= 0 returns GDN_ERR_INVALID_ARGUMENT; everything else as
+ * gdn_prefill_ex (a shape the pool kernel does not take returns
+ * GDN_ERR_UNSUPPORTED).  The page has no counterpart to this call.
+ */
+GDN_API gdn_status gdn_debug_prefill_pool_stall(const void *q, const void *k, const void *v,
+                                                gdn_dtype io_dtype, const float *g,
+                                                const float *beta, const float *initial_state,
+                                                const int32_t *cu_seqlens, int32_t N, int64_t T,
+                                                int32_t Hqk, int32_t Hv, int32_t Dk, int32_t Dv,
+                                                int32_t chunk, void *o, float *final_state,
+                                                void *workspace, size_t workspace_bytes,
+                                                int32_t *dev_error_flag, void *stream,
+                                                int32_t skip_unit, int64_t flag_wait_cycles);
 
 /* Human-readable name of a status code (static storage, never NULL). */
 GDN_API const char *gdn_status_string(gdn_status status);

@@ -40,3 +40,36 @@ def check_state(s_gpu, s_ref, what="state"):
     rl = rel_l2(s_gpu, s_ref)
     assert rl <= S_REL_L2, f"{what}: rel-L2 {rl:.3e}"
     return rl
+
+
+# ---- output canaries ----
+# A kernel output is placed inside a larger device buffer whose guard bytes on
+# both sides hold a sentinel; after the call the guards must be untouched, so
+# no store landed just outside the output.  (compute-sanitizer is not used
+# here; this is the stand-in for its out-of-bounds store check.)
+CANARY_BYTE = 0x7B
+CANARY_GUARD = 4096
+
+
+class Guarded:
+    """A contiguous tensor of `shape` / `dtype` inside a canary-guarded buffer."""
+
+    def __init__(self, shape, dtype, device, fill=None):
+        esz = torch.empty((), dtype=dtype).element_size()
+        n = 1
+        for s in shape:
+            n *= int(s)
+        self.nbytes = n * esz
+        self.buf = torch.full((2 * CANARY_GUARD + self.nbytes,), CANARY_BYTE, dtype=torch.uint8,
+                              device=device)
+        self.t = self.buf[CANARY_GUARD:CANARY_GUARD + self.nbytes].view(dtype).view(*shape)
+        if fill is not None:
+            self.t.copy_(fill)
+
+    def check(self, what="output"):
+        head = self.buf[:CANARY_GUARD]
+        tail = self.buf[CANARY_GUARD + self.nbytes:]
+        bad_head = int((head != CANARY_BYTE).sum())
+        bad_tail = int((tail != CANARY_BYTE).sum())
+        assert bad_head == 0 and bad_tail == 0, \
+            f"{what}: {bad_head} guard bytes before and {bad_tail} after it were overwritten"

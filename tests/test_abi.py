@@ -313,3 +313,18 @@ int main(void) {
                    check=True, capture_output=True, text=True)
     r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
     assert r.returncode == 0 and r.stdout.strip() == "ok", (r.returncode, r.stdout, r.stderr)
+
+
+def test_stall_entry_point_rejects_bad_settings(lib):
+    """The timeout-test entry point refuses a negative unit or a non-positive
+    limit before any CUDA call."""
+    f = lib.gdn_debug_prefill_pool_stall
+    vp, i32, i64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
+    f.argtypes = [vp, vp, vp, ctypes.c_int, vp, vp, vp, vp, i32, i64, i32, i32, i32, i32, i32,
+                  vp, vp, vp, ctypes.c_size_t, vp, vp, i32, i64]
+    f.restype = ctypes.c_int
+    P = 0x10000
+    args = [P, P + 0x1000, P + 0x2000, 0, P + 0x3000, P + 0x4000, None, None, 1, 64, 1, 3, 128,
+            128, 64, P + 0x5000, None, P + 0x6000, 1 << 20, None, None]
+    assert f(*args, -1, 1 << 20) == 1  # GDN_ERR_INVALID_ARGUMENT
+    assert f(*args, 0, 0) == 1

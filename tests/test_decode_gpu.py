@@ -6,7 +6,7 @@ import torch
 import oracle
 import gated_deltanet_04_b200 as gdn
 from gated_deltanet_04_b200 import inputs
-from tests.helpers import check_o, check_state
+from tests.helpers import Guarded, check_o, check_state
 
 pytestmark = pytest.mark.gpu
 DEV = torch.device("cuda:0")
@@ -35,9 +35,13 @@ def test_decode_small_shapes(Dk, Dv, dtype):
     state = 0.05 * torch.randn(N, Hv, Dv, Dk, generator=gen)
     layer = {"q": q, "k": k, "v": v, "g": g, "beta": beta, "state": state}
     o_ref, s_ref = oracle_step(layer)
-    st = state.to(DEV)
-    o = gdn.gdn_decode_step(q.to(DEV), k.to(DEV), v.to(DEV), g.to(DEV), beta.to(DEV), st)
+    gst = Guarded(state.shape, torch.float32, DEV, fill=state)
+    go = Guarded((N, Hv, v.shape[2]), v.dtype, DEV)
+    st = gst.t
+    o = gdn.gdn_decode_step(q.to(DEV), k.to(DEV), v.to(DEV), g.to(DEV), beta.to(DEV), st, o=go.t)
     torch.cuda.synchronize()
+    gst.check("state")
+    go.check("o")
     check_o(o.cpu(), o_ref)
     check_state(st.cpu(), s_ref)
 
@@ -55,9 +59,13 @@ def test_decode_staged_unit_counts(N, Hqk, Hv):
     state = 0.05 * torch.randn(N, Hv, 128, 128, generator=gen)
     layer = {"q": q, "k": k, "v": v, "g": g, "beta": beta, "state": state}
     o_ref, s_ref = oracle_step(layer)
-    st = state.to(DEV)
-    o = gdn.gdn_decode_step(q.to(DEV), k.to(DEV), v.to(DEV), g.to(DEV), beta.to(DEV), st)
+    gst = Guarded(state.shape, torch.float32, DEV, fill=state)
+    go = Guarded((N, Hv, v.shape[2]), v.dtype, DEV)
+    st = gst.t
+    o = gdn.gdn_decode_step(q.to(DEV), k.to(DEV), v.to(DEV), g.to(DEV), beta.to(DEV), st, o=go.t)
     torch.cuda.synchronize()
+    gst.check("state")
+    go.check("o")
     check_o(o.cpu(), o_ref)
     check_state(st.cpu(), s_ref)
 

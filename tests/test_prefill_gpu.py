@@ -13,7 +13,7 @@ import torch
 import oracle
 import gated_deltanet_04_b200 as gdn
 from gated_deltanet_04_b200 import inputs
-from tests.helpers import check_o, check_state
+from tests.helpers import Guarded, check_o, check_state
 
 pytestmark = pytest.mark.gpu
 DEV = torch.device("cuda:0")
@@ -30,13 +30,22 @@ TC_KERNELS = ["pool", "cluster", "single_cta"]
 
 
 def run_gpu(inp, s0=None, cu=None, chunk=0, dev=DEV, kernel="auto"):
+    """One gdn_prefill call; o and the final state are written into
+    canary-guarded buffers whose guards are checked afterwards."""
     t = lambda x: None if x is None else x.to(dev).contiguous()
     flag = torch.zeros(4, dtype=torch.int32, device=dev)
+    T, Hqk, Dk = inp["q"].shape
+    Hv, Dv = inp["v"].shape[1], inp["v"].shape[2]
+    N = 1 if cu is None else len(cu) - 1
+    go = Guarded((T, Hv, Dv), inp["v"].dtype, dev)
+    gs = Guarded((N, Hv, Dv, Dk), torch.float32, dev)
     o, sT = gdn.gdn_prefill(t(inp["q"]), t(inp["k"]), t(inp["v"]), t(inp["g"]), t(inp["beta"]),
                             t(s0), None if cu is None else cu.to(torch.int32).to(dev), chunk=chunk,
-                            kernel=kernel, error_flag=flag)
+                            kernel=kernel, error_flag=flag, o=go.t, final_state=gs.t)
     torch.cuda.synchronize()
     assert int(flag[0]) == 0, f"device error {gdn.STATUS.get(int(flag[0]))}"
+    go.check("o")
+    gs.check("final state")
     return o.cpu(), sT.cpu()
 
 
@@ -305,5 +314,84 @@ def test_auto_past_the_pool_limit():
     assert gdn.gdn_prefill_workspace_bytes(65, int(cu[-1]), 1, 1, 128, 128, 64) == 0
     o, sT = run_gpu(inp, s0, cu)
     o_ref, s_ref = run_oracle(inp, s0, cu)
+    check_o(o, o_ref)
+    check_state(sT, s_ref)
+
+
+# ---- scale robustness of the tensor-core kernels ----
+# The rule is linear in (v, S0) at fixed q, k, g, beta (oracle pin P4), so the
+# oracle's answer at scale 2^s is its answer at scale 1 times 2^s.  The
+# tolerances are compared on the results divided by 2^s, which makes them
+# scale-free.
+
+def _scaled(inp, s0, s):
+    f = 2.0 ** s
+    out = dict(inp)
+    out["v"] = (inp["v"].double() * f).to(inp["v"].dtype)  # exact: a power of two
+    return out, (None if s0 is None else s0 * f)
+
+
+@pytest.mark.parametrize("kernel", TC_KERNELS)
+@pytest.mark.parametrize("s", [-20, -14, -8, 6, 10, 20])
+def test_value_scale_robust(kernel, s):
+    inp, s0 = synth(333, 2, 6, 128, torch.bfloat16, seed=2400, s0_std=0.05)
+    o_ref, s_ref = run_oracle(inp, s0)
+    sc_inp, sc_s0 = _scaled(inp, s0, s)
+    assert torch.equal(sc_inp["v"].double(), inp["v"].double() * 2.0 ** s)
+    o, sT = run_gpu(sc_inp, sc_s0, kernel=kernel)
+    assert torch.isfinite(o.float()).all() and torch.isfinite(sT).all()
+    check_o(o.double() / 2.0 ** s, o_ref, f"o at scale 2^{s}")
+    check_state(sT.double() / 2.0 ** s, s_ref, f"state at scale 2^{s}")
+
+
+@pytest.mark.parametrize("kernel", TC_KERNELS)
+def test_scaling_inputs_scales_outputs_exactly(kernel):
+    """Every value-side operand is held with a power-of-two row scale, so the
+    kernel is exactly homogeneous: v and S0 times 2^s give o and S_T times
+    2^s, bit for bit."""
+    inp, s0 = synth(200, 2, 6, 128, torch.bfloat16, seed=2401, s0_std=0.05)
+    o1, s1 = run_gpu(inp, s0, kernel=kernel)
+    for s in (-9, 7):
+        sc_inp, sc_s0 = _scaled(inp, s0, s)
+        o2, s2 = run_gpu(sc_inp, sc_s0, kernel=kernel)
+        assert torch.equal(o2.double(), o1.double() * 2.0 ** s), s
+        assert torch.equal(s2.double(), s1.double() * 2.0 ** s), s
+
+
+@pytest.mark.parametrize("kernel", TC_KERNELS)
+def test_state_beyond_fp16_range(kernel):
+    """8192 tokens with a = 0.999, b = 1 and v ~ N(0, 2^30): the state's largest
+    entries pass 6.5e4 (fp16's largest value; with unit keys and b = 1 they
+    settle near 3.6 times v's standard deviation) and must stay accurate."""
+    T = 8192
+    inp, _ = synth(T, 1, 3, 128, torch.bfloat16, seed=2402)
+    inp["g"].fill_(float(np.log(0.999)))
+    inp["beta"].fill_(1.0)
+    inp["v"] = (inp["v"].float() * 2.0 ** 15).to(torch.bfloat16)
+    o, sT = run_gpu(inp, kernel=kernel)
+    o_ref, s_ref = run_oracle(inp)
+    assert float(np.abs(s_ref).max()) > 6.6e4  # the case this test is about
+    scale = float(np.abs(o_ref).max())
+    check_o(o.double() / scale, o_ref / scale, "o / max|o|")
+    check_state(sT, s_ref)
+
+
+@pytest.mark.parametrize("kernel", TC_KERNELS)
+def test_key_side_overflow_is_reported(kernel):
+    """A q entry beyond fp16's range (the tensor-core kernels hold q and k in
+    fp16) raises GDN_ERR_RANGE through the device flag; a normal call on the
+    same context afterwards still matches the oracle."""
+    inp, s0 = synth(130, 1, 3, 128, torch.bfloat16, seed=2403, s0_std=0.05)
+    bad = dict(inp)
+    bad["q"] = inp["q"].clone()
+    bad["q"][70, 0, 5] = 1.0e5
+    t = lambda x: x.to(DEV).contiguous()
+    flag = torch.zeros(4, dtype=torch.int32, device=DEV)
+    gdn.gdn_prefill(t(bad["q"]), t(bad["k"]), t(bad["v"]), t(bad["g"]), t(bad["beta"]), t(s0),
+                    kernel=kernel, error_flag=flag)
+    torch.cuda.synchronize()
+    assert int(flag[0]) == 7  # GDN_ERR_RANGE
+    o, sT = run_gpu(inp, s0, kernel=kernel)
+    o_ref, s_ref = run_oracle(inp, s0)
     check_o(o, o_ref)
     check_state(sT, s_ref)
