@@ -67,6 +67,9 @@ def parse():
                         "W + K times and print its per-call time; no bench line")
     p.add_argument("--kernel", default="auto", choices=["auto", "pool", "cluster", "single_cta", "recurrent"],
                    help="prefill kernel for --case")
+    p.add_argument("--tokens", type=int, default=None,
+                   help="token count of a single-sequence prefill --case (a reduced sample, e.g. "
+                        "for a DRAM-traffic capture)")
     return p.parse_args()
 
 
@@ -285,6 +288,33 @@ def time_launches(fn, K, W, dist, stream, sampler=None):
     return start.elapsed_time(end), [a.elapsed_time(b) for a, b in evs]
 
 
+def percentiles(each_ms):
+    """p50 / p95 / p99 of per-call device times (ms), nearest-rank."""
+    xs = sorted(each_ms)
+    if not xs:
+        return None
+    pick = lambda q: xs[min(len(xs) - 1, max(0, int(round(q * len(xs) + 0.5)) - 1))]
+    return {"p50": pick(0.50), "p95": pick(0.95), "p99": pick(0.99), "calls": len(xs)}
+
+
+def run_conditions():
+    """Host and device facts the numbers were taken under."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    cond = {"cpu_model": model, "nproc": os.cpu_count(), "torch": torch.__version__}
+    if torch.cuda.is_available():
+        cond["gpu"] = torch.cuda.get_device_name(0)
+        cond["cuda_runtime"] = torch.version.cuda
+    return cond
+
+
 def cpu_baseline_prefill(tokens: int):
     """The fp64 oracle on the host cores, on the first ``tokens`` tokens of the
     prefill workload (all 48 heads).  Returns (Mtok/s, seconds, threads)."""
@@ -359,7 +389,7 @@ def run_case(args):
         fn = lambda: gdn.gdn_decode_step_bf16_state(L["q"], L["k"], L["v"], L["g"], L["beta"], sb,
                                                     o=out)
     else:
-        inp = inputs.make_prefill(args.case, device=dev)
+        inp = inputs.make_prefill(args.case, device=dev, T=args.tokens)
         o = torch.empty_like(inp["v"])
         N = inp["N"]
         sT = torch.empty((N, inp["wl"].Hv, 128, 128), dtype=torch.float32, device=dev)
@@ -415,6 +445,34 @@ def main():
     p_total, p_each = time_launches(prefill, K, W, dist, stream, sampler)
     p_ms = dist.max(p_total / K)
     p_launch_ms = dist.max(sum(p_each) / K)
+    del o, sT
+
+    # ------------------------------------------- the other prefill workloads --
+    # the 4096-token layer (pool kernel) and the 32-sequence varlen batch (1,536
+    # units: the single-CTA kernel), each in Mtok/s with per-call percentiles
+    others = {}
+    for name, calls in (("layer4k", max(K, 50)), ("varlen32", K)):
+        winp = inputs.make_prefill(name, device=dev)
+        wo = torch.empty_like(winp["v"])
+        wsT = torch.empty((winp["N"], 48, 128, 128), dtype=torch.float32, device=dev)
+        wws = torch.empty(max(1, gdn.gdn_prefill_workspace_bytes(winp["N"], winp["T"], 16, 48, 128,
+                                                                 128, 64)),
+                          dtype=torch.uint8, device=dev)
+
+        def wcall(winp=winp, wo=wo, wsT=wsT, wws=wws):
+            gdn.gdn_prefill(winp["q"], winp["k"], winp["v"], winp["g"], winp["beta"], winp["s0"],
+                            winp["cu_seqlens"], chunk=64, o=wo, final_state=wsT, workspace=wws)
+
+        w_total, w_each = time_launches(wcall, calls, W, dist, stream, sampler)
+        w_ms = dist.max(w_total / calls)
+        others[name] = {"value": weak_scaling_value(winp["T"], w_ms / 1e3, dist.world) / 1e6,
+                        "unit": "Mtok/s", "ms_per_call": w_ms, "tokens": winp["T"],
+                        "units": winp["N"] * 48,
+                        "kernel": "pool" if winp["N"] * 48 <= 64 else "single_cta",
+                        "percentiles_ms": percentiles(w_each)}
+        del winp, wo, wsT, wws
+    o = torch.empty_like(inp["v"])
+    sT = torch.empty((1, 48, 128, 128), dtype=torch.float32, device=dev)
 
     # ------------------------------------------------------- front end --
     # the kernel-4 short convolution + q/k norm over the same layer's q, k, v
@@ -432,7 +490,7 @@ def main():
                                 fst.data_ptr(), None, 1, T, Hqk_, Hv_, 128, 128, fq.data_ptr(),
                                 fk.data_ptr(), fv.data_ptr(), None, stream.cuda_stream)
 
-    f_total, _ = time_launches(front_end, K, W, dist, stream, sampler)
+    f_total, f_each = time_launches(front_end, K, W, dist, stream, sampler)
     f_ms = dist.max(f_total / K)
     f_bytes = 2 * sum(t.numel() * t.element_size() for t in (fq, fk, fv)) + \
         sum(w.numel() * 4 for w in fw) + fst.numel() * 4
@@ -447,7 +505,7 @@ def main():
         for L, out in zip(layers, d_outs):
             gdn.gdn_decode_step(L["q"], L["k"], L["v"], L["g"], L["beta"], L["state"], o=out)
 
-    d_total, _ = time_launches(decode_step, K, W, dist, stream, sampler)
+    d_total, d_each = time_launches(decode_step, K, W, dist, stream, sampler)
     d_ms = dist.max(d_total / K)
     state_bytes_layer = dwl.N * dwl.Hv * dwl.Dv * dwl.Dk * 4 * 2
     io_bytes_layer = dwl.N * (2 * dwl.Hqk * dwl.Dk * 2 + 2 * dwl.Hv * dwl.Dv * 2 + 2 * dwl.Hv * 4)
@@ -465,7 +523,7 @@ def main():
         for L, st, out in zip(layers, b_states, d_outs):
             gdn.gdn_decode_step_bf16_state(L["q"], L["k"], L["v"], L["g"], L["beta"], st, o=out)
 
-    b_total, _ = time_launches(decode_step_bf16, K, W, dist, stream, sampler)
+    b_total, b_each = time_launches(decode_step_bf16, K, W, dist, stream, sampler)
     b_ms = dist.max(b_total / K)
     b_state_gbs = weak_scaling_value(state_bytes_layer // 2 * dwl.layers, b_ms / 1e3,
                                      dist.world) / 1e9
@@ -489,12 +547,13 @@ def main():
             o_host.copy_(o, non_blocking=True)
             s_host.copy_(sT, non_blocking=True)
 
-        e_total, _ = time_launches(e2e_step, K, W, dist, stream)
+        e_total, e_each = time_launches(e2e_step, K, W, dist, stream)
         e_ms = dist.max(e_total / K)
         h2d = sum(t.numel() * t.element_size() for t in host.values())
         d2h = o_host.numel() * o_host.element_size() + s_host.numel() * s_host.element_size()
         e2e = {"value": weak_scaling_value(T, e_ms / 1e3, dist.world) / 1e6, "unit": "Mtok/s",
-               "ms_per_step": e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+               "ms_per_step": e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "percentiles_ms": percentiles(e_each)}
 
     # --------------------------------------------------------- roofline --
     # Dk = Dv = 128, bf16, chunk 64, 48 units: the library's default is the pool kernel
@@ -512,6 +571,7 @@ def main():
                         "algorithmic_bytes_per_launch": PREFILL_BYTES_PER_TOKEN * T}}
     d_gbs_launch = (state_bytes_layer + io_bytes_layer) / (d1_ms / 1e3) / 1e9
     decode = {"value": d_state_gbs, "unit": "GB/s", "ms_per_step": d_ms,
+              "percentiles_ms": percentiles(d_each),
               "layers_per_step": dwl.layers, "sequences": dwl.N,
               "roofline": {"bound": "hbm", "achieved": d_gbs_launch, "peak": peaks["hbm_gbs"],
                            "unit": "GB/s", "frac": d_gbs_launch / peaks["hbm_gbs"],
@@ -521,13 +581,14 @@ def main():
                            "algorithmic_bytes_per_launch": state_bytes_layer + io_bytes_layer},
               "frac_of_8TBps": d_state_gbs / dist.world / 8000.0,
               "bf16_state": {"value": b_state_gbs, "unit": "GB/s", "ms_per_step": b_ms,
+                             "percentiles_ms": percentiles(b_each),
                              "note": "same 48-layer step with the state stored in bfloat16 "
                                      "(gdn_decode_step_bf16_state); GB/s of bf16 state bytes",
                              "frac_of_measured_copy": b_state_gbs / dist.world / peaks["hbm_gbs"],
                              "frac_of_8TBps": b_state_gbs / dist.world / 8000.0}}
 
     front = {"value": weak_scaling_value(T, f_ms / 1e3, dist.world) / 1e6, "unit": "Mtok/s",
-             "ms_per_step": f_ms,
+             "ms_per_step": f_ms, "percentiles_ms": percentiles(f_each),
              "note": "gdn_short_conv_norm (kernel-4 causal conv on q, k, v channels, q/k L2 "
                      "norm) over the same 262,144-token layer",
              "hbm": {"achieved": f_bytes / (f_ms / 1e3) / 1e9, "peak": peaks["hbm_gbs"],
@@ -554,13 +615,17 @@ def main():
                                "decode N=256 x 48 layers (see 'decode')",
                    "l2": "inputs larger than L2 (8.7 GB per prefill, 38.6 GB decode states)",
                    "parallelism": f"replica x{dist.world} (no data-path collective)"},
+        "percentiles_ms": percentiles(p_each),
         "roofline": roofline,
+        "prefill_workloads": others,
         "decode": decode,
         "front_end": front,
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": K * (1 + 2 + dwl.layers + 1 + dwl.layers) + K * (0 if args.no_e2e else 1),
+        "gpu_launches": K * (1 + 2 + dwl.layers + 1 + dwl.layers) + K * (0 if args.no_e2e else 1)
+                        + max(K, 50) + K,
         "clocks": clocks,
+        "run_conditions": run_conditions(),
     }
     if dist.rank == 0:
         print(json.dumps(line), flush=True)

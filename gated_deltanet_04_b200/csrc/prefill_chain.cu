@@ -74,7 +74,9 @@ static __shared__ unsigned int gdn_phase_acc_[16];
 #define GDN_CL_PHASE_BEGIN()                                           \
     long long phase_t_ = clock64();                                    \
     if (threadIdx.x == 0)                                              \
-        for (int i_ = 0; i_ < 16; ++i_) gdn_phase_acc_[i_] = 0u
+        for (int i_ = 0; i_ < 16; ++i_) gdn_phase_acc_[i_] = 0u;       \
+    if ((threadIdx.x & 31) == 0)                                       \
+        for (int s_ = 0; s_ < 4; ++s_) gdn_bar_acc_[s_][threadIdx.x >> 5] = 0u
 #define GDN_CL_PHASE_END(role)                                         \
     do {                                                               \
         if (threadIdx.x == 0 && phase_on_)                             \
@@ -82,10 +84,30 @@ static __shared__ unsigned int gdn_phase_acc_[16];
                 atomicAdd(&gdn_cl_phase_clk[(role)][i_],               \
                           (unsigned long long)gdn_phase_acc_[i_]);     \
     } while (0)
+// Per-warp waiting time at selected barriers of the same two CTAs:
+// [role][site][warp], accumulated by lane 0 of each warp in shared memory.
+__device__ unsigned long long gdn_cl_bar_wait[2][4][8];
+static __shared__ unsigned int gdn_bar_acc_[4][8];
+#define GDN_BAR_T0() const long long bar_t0_ = clock64()
+#define GDN_BAR_T1(site)                                                       \
+    do {                                                                       \
+        if (phase_on_ && (threadIdx.x & 31) == 0)                              \
+            gdn_bar_acc_[(site)][threadIdx.x >> 5] += (unsigned)(clock64() - bar_t0_); \
+    } while (0)
+#define GDN_BAR_END(role)                                                      \
+    do {                                                                       \
+        if (phase_on_ && (threadIdx.x & 31) == 0)                              \
+            for (int s_ = 0; s_ < 4; ++s_)                                     \
+                atomicAdd(&gdn_cl_bar_wait[(role)][s_][threadIdx.x >> 5],      \
+                          (unsigned long long)gdn_bar_acc_[s_][threadIdx.x >> 5]); \
+    } while (0)
 #else
 #define GDN_CL_PHASE(role, k) ((void)0)
 #define GDN_CL_PHASE_BEGIN() ((void)0)
 #define GDN_CL_PHASE_END(role) ((void)0)
+#define GDN_BAR_T0() ((void)0)
+#define GDN_BAR_T1(site) ((void)0)
+#define GDN_BAR_END(role) ((void)0)
 #endif
 
 namespace gdn {
@@ -106,6 +128,11 @@ constexpr int kSlotTid = 192;
 // chain thread that polls the ring, loads it, signals taken chunks and stores
 // output tiles (thread 0 only issues MMAs, and never waits on L2)
 constexpr int kLoadTid = 32;
+// chain thread that issues the output tile stores and, before each chunk's
+// first CTA barrier, waits until the store issued at the chunk's start has
+// read its shared slot (so the load thread, which fences before its ring
+// loads, never waits behind an output store)
+constexpr int kStoreTid = 64;
 constexpr int kGatesWarp = 5;  // loads g, beta and computes the next chunk's gates
 constexpr int kClusterRingSlots = 4;
 constexpr int kPoolRingSlots = 8;
@@ -131,7 +158,8 @@ struct GatesBlock {
     float eC[kC];    // exp(gamma_C - gamma_r)
     int32_t hp;      // extra precision passes for this chunk
     int32_t qs;      // Q^T arrives scaled by Gamma (so the chain need not scale O)
-    int32_t pad[2];
+    int32_t hp_next; // the unit's next chunk takes them (it reads the state's lo part)
+    int32_t pad;
 };
 static_assert(sizeof(GatesBlock) % 16 == 0, "bulk copies move multiples of 16 bytes");
 
@@ -157,53 +185,73 @@ constexpr uint32_t CT_S = 0, CT_SH = 128, CT_SL = 192, CT_U16 = 192, CT_O = 256,
                    CT_R2 = 384, CT_D = 320, CT_UP = 448;
 
 // ---- producer CTA ----
-constexpr uint32_t P_KQV = 0;           // 2 buffers: [K|Q] d-half 0, [K|Q] d-half 1, V halves
-constexpr uint32_t P_KQV_BYTES = 49152;
-constexpr uint32_t P_X = 98304;         // solve scratch: A, T, X (fp32); then W^T hi/lo staging
-constexpr uint32_t P_WST = P_X;
+// A producer work item is one chunk of one sequence for a group of nh v-heads
+// that share their q/k head (nh <= 3; 1 in the cluster kernel): the K and Q
+// tiles, the Gram matrices, K in fp16 and Q^T are made once per item, and
+// everything else once per head, a "step".
+constexpr uint32_t P_KQ = 0;            // 2 buffers (by item parity): [K|Q] d-half 0, [K|Q] d-half 1
+constexpr uint32_t P_KQ_BYTES = 32768;
+constexpr uint32_t P_V = 65536;         // 2 buffers (by step parity): a head's V halves, then its Q^T
+constexpr uint32_t P_V_BYTES = 16384;
+constexpr int kVBufs = 2;
+// Each step's ring stores read their sources asynchronously while the next
+// step runs; every source region is rewritten only as late in the next step
+// as its use allows, and the delivery thread waits for just the store groups
+// that read it right before that point:
+//   P (double-buffered)    rewritten at the A / P of the step after next
+//   W^T staging            rewritten by the next step's solve (T, X)
+//   U~ staging             rewritten by the next step's T tiles
+constexpr uint32_t P_X = 98304;         // solve scratch: A, then T and X (fp32)
 constexpr uint32_t P_AS = P_X;
 constexpr uint32_t P_TS = P_X + 64 * kAS4 * 4;
 constexpr uint32_t P_XS = P_TS + 64 * kTS * 4;
-constexpr uint32_t P_P16 = 137216;      // P fp16 [64 rows][128 B], SW128
+constexpr uint32_t P_WST = P_TS;        // W^T hi / lo staging over T and X (32 KB)
+constexpr uint32_t P_P16 = 148480;      // 2 buffers (by step parity) of P fp16 [64 rows][128 B], SW128
 // T tiles: T diag(b) as bf16 hi / mid / lo and T diag(b Gamma) as fp16 hi / lo,
 // each [64 rows][128 B], SW128.  The parts of each are consecutive, so one B
 // operand of N = 192 (or 128) rows takes all of them and the MMA writes each
 // part's product to its own accumulator columns.
-constexpr uint32_t P_TBH = 145408, P_TBM = 153600, P_TBL = 161792, P_TGH = 169984,
-                   P_TGL = 178176;
+constexpr uint32_t P_TBH = 164864, P_TBM = 173056, P_TBL = 181248, P_TGH = 189440,
+                   P_TGL = 197632;
 constexpr uint32_t P_UTS = P_TBH;       // then U~^T staging (same layout as SL_UT)
-constexpr uint32_t P_MISC = 186368;
-constexpr uint32_t P_ID = 190464;       // bf16 identity [64][128 B] (B operand of the Q^T product)
+constexpr uint32_t P_MISC = 205824;
+constexpr uint32_t P_ID = 209920;       // bf16 identity [64][128 B] (B operand of the Q^T product)
+static_assert(P_V == P_KQ + 2 * P_KQ_BYTES && P_X == P_V + kVBufs * P_V_BYTES, "tile buffers");
+static_assert(P_WST + 32768 <= P_P16 && P_TBH == P_P16 + 2 * 8192, "staging regions");
 static_assert(P_TBM == P_TBH + 8192 && P_TBL == P_TBM + 8192 && P_TGL == P_TGH + 8192,
               "stacked B operands");
-static_assert(P_WST + 32768 <= P_P16 && P_UTS + 32768 <= P_TGL + 8192, "staging fits its region");
+static_assert(P_UTS + 32768 <= P_TGL + 8192, "staging fits its region");
 static_assert(P_XS + 1024 * 4 <= P_P16, "solve scratch overflows");
 static_assert(P_TS % 16 == 0 && P_XS % 16 == 0, "float4 scratch must be aligned");
-static_assert(P_P16 % 1024 == 0 && P_TBH % 1024 == 0, "swizzled tiles start on 1 KB");
+static_assert(P_P16 % 1024 == 0 && P_TBH % 1024 == 0 && P_ID % 1024 == 0 && P_V % 1024 == 0,
+              "swizzled tiles start on 1 KB");
 
-// One chunk of one unit, as a producer sees it.
+// One work item (one chunk of one sequence for nh v-heads), as a producer
+// sees it; head i of the item is v-head h + i, unit unit + i.
 struct Item {
     int64_t c0;       // first token
-    int32_t unit, c;  // unit = n * Hv + h; chunk index within the sequence
-    int32_t h, j, L;  // v head, q/k head, valid rows
+    int32_t unit, c;  // first unit (n * Hv + h); chunk index within the sequence
+    int32_t h, j, L;  // first v head, q/k head, valid rows
     int32_t valid;
+    int32_t Lnext;    // valid rows of the sequence's next chunk (0: none)
 };
 
 // Decay and gate factors of one chunk (double-buffered by chunk parity: the
 // next chunk's are computed while this chunk's U~ / W products run).
 struct ProdGates {
     float gam[kC], Gam[kC], iGam[kC], eC[kC], bb[kC], bG[kC];
-    int32_t safe, hp, qs, pad;
+    int32_t safe, hp, qs, hp_next;
 };
 
 struct ProdMisc {
     GatesBlock gst;   // gates staging of the chunk being delivered
     ProdGates gt[2];
     Item items[4];    // this CTA's chunks l .. l + 2, by l % 4
-    uint64_t tma_bar[2];
+    uint64_t tma_bar[2];      // K / Q tiles of an item, by item parity
+    uint64_t tma_v[kVBufs];   // V tile of a step, by step parity
     uint64_t mma_bar;
     uint64_t taken;
-    uint64_t qt_bar;  // the Q^T product of the current chunk has landed
+    uint64_t qt_bar;  // the Q^T product of the current item has landed
     uint32_t tmem_base;
 };
 static_assert(P_MISC + sizeof(ProdMisc) <= P_ID, "identity tile after the misc block");
@@ -212,10 +260,14 @@ constexpr uint32_t kChainBytes = C_MISC + sizeof(ChainMisc);
 constexpr uint32_t kSmemBytes = (kProdBytes > kChainBytes ? kProdBytes : kChainBytes) + 1024;
 static_assert(kSmemBytes <= 232448, "fits the 227 KB opt-in shared memory of a CTA");
 
-// producer TMEM columns (512 allocated): the Gram, then W^T from T diag(b Gamma)'s
-// hi part (and its lo part's product at + 64); Q^T; U~^T as three products
-// (T diag(b)'s hi, mid, lo parts) at PT_U, + 64, + 128
-constexpr uint32_t PT_G = 0, PT_Q = 128, PT_U = 256;
+// producer TMEM columns (512 allocated): W^T from T diag(b Gamma)'s hi part (and
+// its lo part's product at + 64); the item's Q^T (kept for all its heads);
+// U~^T as three products (T diag(b)'s hi, mid, lo parts) at PT_U, + 64, + 128;
+// the item's Gram at PT_G, or over W^T's columns when an item has one head
+// (where it is dead by the time W^T is made).  Measured: this placement of
+// W^T, Q^T and U~^T runs the 262,144-token layer 1 ms faster than W^T at 128
+// and Q^T at 64.
+constexpr uint32_t PT_W = 0, PT_Q = 128, PT_G = 192, PT_U = 256;
 constexpr uint32_t IDESC_MK_N192_BF16 = make_idesc_f16(128, 192, 1, 0, 1);
 constexpr uint32_t IDESC_MK_N128 = make_idesc_f16(128, 128, 1, 0);
 
@@ -239,6 +291,7 @@ struct ChainParams {
     int32_t recall_first;  // GDN_ORDER_RECALL_FIRST: recall before the decay
     long long flag_wait_limit;  // SM clocks a spin on a hand-off flag may last
     int32_t skip_unit;          // testing: a unit no producer prepares (-1: none)
+    int32_t nh;                 // v-heads per pool producer item (divides Hv / Hqk, <= 3)
 };
 
 __device__ __forceinline__ uint8_t *ring_slot(const ChainParams &p, int unit, int c) {
@@ -258,17 +311,19 @@ __device__ __forceinline__ uint32_t ut_off(int i, int q) {
     return (uint32_t)i * 256u + (uint32_t)((q ^ (i & 15)) << 4);
 }
 
-// The chunk at index i of the pool kernel's chunk-major order (valid == 0 once
-// the order is exhausted).  `skip` is set when index i names no chunk (a
-// shorter or malformed sequence): the caller then takes another index.
+// The item at index i of the pool kernel's chunk-major order: chunk i / G of
+// the item's nh units, G = units / nh items per chunk (valid == 0 once the
+// order is exhausted).  `skip` is set when index i names no chunk (a shorter
+// or malformed sequence): the caller then takes another index.
 __device__ Item pool_item(const ChainParams &p, uint32_t i, bool &skip) {
     Item it;
     it.valid = 0;
     skip = false;
-    const int c = (int)(i / (uint32_t)p.units);
-    const int unit = (int)(i % (uint32_t)p.units);
+    const uint32_t per_chunk = (uint32_t)(p.units / p.nh);
+    const int c = (int)(i / per_chunk);
+    const int unit = (int)(i % per_chunk) * p.nh;
     if (c >= p.max_chunks) return it;
-    if (unit == p.skip_unit) {  // testing: its chain waits for a chunk that never comes
+    if (p.skip_unit >= unit && p.skip_unit < unit + p.nh) {  // testing: a chain starves
         skip = true;
         return it;
     }
@@ -289,6 +344,8 @@ __device__ Item pool_item(const ChainParams &p, uint32_t i, bool &skip) {
     it.h = unit % p.Hv;
     it.j = it.h / (p.Hv / p.Hqk);
     it.L = (int)((t1 - c0) < kC ? (t1 - c0) : kC);
+    const int64_t rest = t1 - c0 - kC;
+    it.Lnext = (int)(rest <= 0 ? 0 : (rest < kC ? rest : kC));
     it.valid = 1;
     return it;
 }
@@ -301,16 +358,17 @@ __device__ Item pool_fetch(const ChainParams &p, uint32_t first) {
         bool skip;
         const Item it = pool_item(p, i, skip);
         if (!skip) return it;
-        if (ld_relaxed_gpu(p.flags + 1) != 0u) return Item{0, 0, 0, 0, 0, 0, 0};
+        if (ld_relaxed_gpu(p.flags + 1) != 0u) return Item{0, 0, 0, 0, 0, 0, 0, 0};
         i = atomicAdd(p.flags, 1u);
     }
 }
 
 // ------------------------------------------------------------- producer --
 
-// kPool: the pool kernel (chunks from the global counter); otherwise producer
-// k of a cluster, whose chunks are k, k + 2, ... of `unit`.
-template <bool kPool>
+// kPool: the pool kernel (items from the global counter, p.nh heads each);
+// otherwise producer k of a cluster, whose items are chunks k, k + 2, ... of
+// `unit` (one head).  Item l's head i is step s = l * nh + i.
+template <bool kPool, int kNh>
 __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtensorMap *tm_k,
                               const CUtensorMap *tm_v, const ChainParams &p, int unit, int k,
                               int h, int j, int64_t t_begin, int64_t t_end, int nch) {
@@ -330,7 +388,7 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
     auto fetch = [&](int l) -> Item {
         if constexpr (kPool) {
             if (l < 2) {
-                if (ld_relaxed_gpu(p.flags + 1) != 0u) return Item{0, 0, 0, 0, 0, 0, 0};
+                if (ld_relaxed_gpu(p.flags + 1) != 0u) return Item{0, 0, 0, 0, 0, 0, 0, 0};
                 return pool_fetch(p, atomicAdd(p.flags, 1u));
             }
             return pool_fetch(p, pre_index);
@@ -344,31 +402,50 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
             it.h = h;
             it.j = j;
             it.L = (int)((t_end - it.c0) < kC ? (t_end - it.c0) : kC);
+            const int64_t rest = t_end - it.c0 - kC;
+            it.Lnext = (int)(rest <= 0 ? 0 : (rest < kC ? rest : kC));
             return it;
         }
     };
 
+    constexpr int nh = kNh;  // heads per item (p.nh in the pool kernel)
+    constexpr uint32_t pt_g = kNh == 1 ? PT_W : PT_G;
     uint32_t mma_phase = 0;
     bool timed_out = false;
     float kmax = 0.f;             // largest key-side value this thread has put into fp16
     bool range_reported = false;
     float gpre0 = 0.f, gpre1 = 0.f, bpre0 = 0.f, bpre1 = 0.f;  // gates warp: next chunk's g, beta
-    auto load_gates = [&](const Item &it) {
-        gpre0 = gpre1 = bpre0 = bpre1 = 0.f;
+    float gnx0 = 0.f, gnx1 = 0.f;  // ... and g of the chunk after it in the same unit
+    // g, beta of head hh (0 .. nh - 1) of item `it`, and g of the sequence's next chunk
+    auto load_gates = [&](const Item &it, int hh) {
+        gpre0 = gpre1 = bpre0 = bpre1 = gnx0 = gnx1 = 0.f;
+        const int hv = it.h + hh;
         const int64_t t0_ = it.c0 + 2 * lane, t1_ = t0_ + 1, te = it.c0 + it.L;
-        if (t0_ < te) { gpre0 = p.g[t0_ * p.Hv + it.h]; bpre0 = p.beta[t0_ * p.Hv + it.h]; }
-        if (t1_ < te) { gpre1 = p.g[t1_ * p.Hv + it.h]; bpre1 = p.beta[t1_ * p.Hv + it.h]; }
+        if (t0_ < te) { gpre0 = p.g[t0_ * p.Hv + hv]; bpre0 = p.beta[t0_ * p.Hv + hv]; }
+        if (t1_ < te) { gpre1 = p.g[t1_ * p.Hv + hv]; bpre1 = p.beta[t1_ * p.Hv + hv]; }
+        const int64_t tn = te + 2 * lane, ten = te + it.Lnext;
+        if (tn < ten) gnx0 = p.g[tn * p.Hv + hv];
+        if (tn + 1 < ten) gnx1 = p.g[(tn + 1) * p.Hv + hv];
     };
-    auto issue_tma = [&](int buf, const Item &it) {
-        uint8_t *b = sm + P_KQV + buf * P_KQV_BYTES;
-        mbar_arrive_expect_tx(&ms->tma_bar[buf], 6 * 8192);
+    // K and Q tiles of item `it` into K / Q buffer b (by item parity)
+    auto issue_kq = [&](int b, const Item &it) {
+        uint8_t *dst = sm + P_KQ + b * P_KQ_BYTES;
+        mbar_arrive_expect_tx(&ms->tma_bar[b], 4 * 8192);
         const int32_t t32 = (int32_t)it.c0;
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
-            tma_load_3d(b + hf * 16384, tm_k, &ms->tma_bar[buf], 64 * hf, it.j, t32);
-            tma_load_3d(b + hf * 16384 + 8192, tm_q, &ms->tma_bar[buf], 64 * hf, it.j, t32);
-            tma_load_3d(b + 32768 + hf * 8192, tm_v, &ms->tma_bar[buf], 64 * hf, it.h, t32);
+            tma_load_3d(dst + hf * 16384, tm_k, &ms->tma_bar[b], 64 * hf, it.j, t32);
+            tma_load_3d(dst + hf * 16384 + 8192, tm_q, &ms->tma_bar[b], 64 * hf, it.j, t32);
         }
+    };
+    // V tile of head hh of item `it` into V buffer b (by step % 3)
+    auto issue_v = [&](int b, const Item &it, int hh) {
+        uint8_t *dst = sm + P_V + b * P_V_BYTES;
+        mbar_arrive_expect_tx(&ms->tma_v[b], 2 * 8192);
+        const int32_t t32 = (int32_t)it.c0;
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf)
+            tma_load_3d(dst + hf * 8192, tm_v, &ms->tma_v[b], 64 * hf, it.h + hh, t32);
     };
     auto mma_sync_point = [&]() {
         if (tid == 0) mma_commit(&ms->mma_bar);
@@ -384,20 +461,39 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
         tc_fence_after_sync();
     };
 
-    // The delivery thread's last chunk whose ring stores are in flight and not
-    // yet reported ready (valid == 0: none).
-    Item pending;
+    // The delivery thread's chunks whose ring stores are in flight and not yet
+    // reported ready: the last one delivered (pending) and, in the pool kernel,
+    // the one before it (older).  valid == 0: none.
+    Item pending, older;
     pending.valid = 0;
-    auto flush_delivery = [&]() {  // delivery thread only
-        if (!pending.valid) return;
-        bulk_wait_all();              // written to global memory
-        fence_proxy_async_global();   // ... ordered before the signal below
+    older.valid = 0;
+    auto signal_ready = [&](const Item &d) {  // its stores have completed
         if constexpr (kPool)
-            st_release_gpu(unit_flags(p, pending.unit) + 1 + (pending.c & (p.ring_slots - 1)),
-                           (uint32_t)(pending.c + 1));
+            st_release_gpu(unit_flags(p, d.unit) + 1 + (d.c & (p.ring_slots - 1)),
+                           (uint32_t)(d.c + 1));
         else
             mbar_arrive_remote(c_ready);
+    };
+    auto flush_delivery = [&]() {  // delivery thread only: every delivery held
+        if (!pending.valid && !older.valid) return;
+        bulk_wait_all();              // written to global memory
+        fence_proxy_async_global();   // ... ordered before the signals below
+        if (older.valid) signal_ready(older);
+        if (pending.valid) signal_ready(pending);
+        older.valid = 0;
         pending.valid = 0;
+    };
+    // Pool kernel: the delivery before the last one, whose stores landed long
+    // ago (two bulk groups per delivery: the last delivery's may still be in
+    // flight).  Signalling one chunk late keeps the wait for the 105 KB of
+    // stores to land off the producer's path; the ring's depth absorbs the
+    // extra latency.
+    auto flush_older = [&]() {
+        if (!older.valid) return;
+        bulk_wait_all_but_two();
+        fence_proxy_async_global();
+        signal_ready(older);
+        older.valid = 0;
     };
 
     // Gates of a chunk from the g, beta values in gpre / bpre (the gates warp, two
@@ -439,23 +535,29 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
         const float Gr0 = p.recall_first ? (lane > 0 ? expf(xp) : 1.f) : G0;
         const float Gr1 = p.recall_first ? G0 : G1;
         gt.bG[r0] = bpre0 * Gr0;        gt.bG[r0 + 1] = bpre1 * Gr1;
+        // the precision choice of this chunk and of the unit's next one, from the
+        // same sum in the same order as the next chunk's own producer takes it
+        const float gsum = warp_sum(gpre0 + gpre1), gsum_next = warp_sum(gnx0 + gnx1);
         if (lane == 0) {
             gt.safe = safe_;
-            gt.hp = GC >= kHighPrecisionDecay;
+            gt.hp = gsum >= kLogHighPrecisionDecay;
+            gt.hp_next = gsum_next >= kLogHighPrecisionDecay;
             // Q^T is scaled by Gamma <= 1 only: Gamma q then cannot overflow fp16
             gt.qs = safe_ && top <= 0.f;
         }
     };
 
-    // Chunks l and l + 1 are known when chunk l starts (tile loads of chunks
-    // 0 and 1 are issued here, those of chunk l + 1 > 1 during the U~ / W
-    // products of chunk l, after the stores of chunk l - 1 have landed); chunk
-    // l + 2 is fetched during those products too.
+    // Items l and l + 1 are known when item l starts (item l + 2 is fetched
+    // during the U~ / W products of its first step).  The K / Q tiles of item
+    // 0 and the V tile of step 0 are loaded here; those of item l + 1 during
+    // the U~ / W products of item l's last step, and the V tile of step s + 1
+    // during those of step s (its buffer held step s - 2's, whose stores have
+    // read it by then).
     if (tid == kFetchTid) {
-        for (int l = 0; l < 2; ++l) {
-            const Item it = fetch(l);
-            ms->items[l] = it;
-            if (it.valid) issue_tma(l, it);
+        for (int l = 0; l < 2; ++l) ms->items[l] = fetch(l);
+        if (ms->items[0].valid) {
+            issue_kq(0, ms->items[0]);
+            issue_v(0, ms->items[0], 0);
         }
     }
     // the bf16 identity, K-major with the 128-byte swizzle: row n holds 1 at k = n
@@ -471,7 +573,7 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
     fence_proxy_async_smem();
     __syncthreads();
     if (warp == kGatesWarp && ms->items[0].valid) {
-        load_gates(ms->items[0]);
+        load_gates(ms->items[0], 0);
         compute_gates(ms->gt[0]);
     }
     __syncthreads();
@@ -479,42 +581,54 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
     const bool phase_on_ = blockIdx.x == (kPool ? (unsigned)p.units : 1u);
 #endif
     GDN_CL_PHASE_BEGIN();
-    int l = 0;
+    int s = 0, l = 0, hi = 0;  // step, its item and head within the item
     bool broke = false;
+    int v_loaded = 1;  // steps whose V tile load has been issued
+    int kq_loaded = 1; // items whose K / Q tile load has been issued
 #pragma unroll 1
-    for (;; ++l) {
-        const Item it = ms->items[l & 3];
-        if (!it.valid) break;
+    for (;; ++s) {
+        l = s / nh;
+        hi = s - l * nh;
+        const Item item = ms->items[l & 3];
+        if (!item.valid) break;
+        Item it = item;  // this step's head: v-head item.h + hi, unit item.unit + hi
+        it.h += hi;
+        it.unit += hi;
         const int L = it.L;
         const int buf = l & 1;
-        const ProdGates &gt = ms->gt[l & 1];
+        const int vb = s % kVBufs;
+        const ProdGates &gt = ms->gt[s & 1];
 
-        // the next chunk's g, beta: in flight until its gates are computed
+        // the next step's g, beta: in flight until its gates are computed
         if (warp == kGatesWarp) {
-            const Item nx = ms->items[(l + 1) & 3];
-            if (nx.valid) load_gates(nx);
+            const int ln = (s + 1) / nh, hn = (s + 1) - ln * nh;
+            const Item nx = ms->items[ln & 3];
+            if (nx.valid) load_gates(nx, hn);
         }
-        // pool: the index of chunk l + 2 and an early look at this chunk's ring
-        // slot, both consumed at the end of the chunk
+        // pool: the index of item l + 2 (first step of an item) and an early
+        // look at this step's ring slot, both consumed later in the step
         uint32_t early_taken = 0;
         if constexpr (kPool) {
-            if (tid == kFetchTid) pre_index = atomicAdd(p.flags, 1u);
-            if (tid == kSlotTid && it.c >= p.ring_slots)
+            if (tid == kFetchTid && hi == 0) pre_index = atomicAdd(p.flags, 1u);
+            if (tid == kDeliverTid && it.c >= p.ring_slots)
                 early_taken = ld_relaxed_gpu(unit_flags(p, it.unit));
         }
         GDN_CL_PHASE(1, 0);  // gates
         GDN_CL_PHASE(1, 1);  // (no wait)
+        uint8_t *kqv = sm + P_KQ + buf * P_KQ_BYTES;
+        const uint32_t skqv = sbase + P_KQ + buf * P_KQ_BYTES;
+        uint8_t *vt = sm + P_V + vb * P_V_BYTES;
+        const uint32_t svt = sbase + P_V + vb * P_V_BYTES;
+        // ---- first step of an item: K / Q tiles, the Gram [K;Q] K^T straight from
+        //      the bf16 tiles (exact products either way), K to fp16 ----
+        if (hi == 0) {
         if (!mbar_wait_bounded(&ms->tma_bar[buf], (l >> 1) & 1, kWaitLimit)) timed_out = true;
         GDN_CL_PHASE(1, 2);  // wait: tiles
-
-        // ---- Gram [K;Q] K^T straight from the bf16 tiles (exact products either way) ----
-        uint8_t *kqv = sm + P_KQV + buf * P_KQV_BYTES;
-        const uint32_t skqv = sbase + P_KQV + buf * P_KQV_BYTES;
         if (tid == 0) {
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
                 const uint32_t a = skqv + (ks >> 2) * 16384 + (ks & 3) * 32;
-                mma_f16_ss(tmem + PT_G, make_sdesc(a, 16, 1024), make_sdesc(a, 16, 1024),
+                mma_f16_ss(tmem + pt_g, make_sdesc(a, 16, 1024), make_sdesc(a, 16, 1024),
                            IDESC_KK_N64_BF16, ks > 0);
             }
             mma_commit(&ms->mma_bar);
@@ -545,14 +659,28 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
         if (!mbar_wait_bounded(&ms->mma_bar, mma_phase, kWaitLimit)) timed_out = true;
         mma_phase ^= 1;
         tc_fence_after_sync();
-        // A / P, the solve and the W^T staging rewrite what the previous chunk's
-        // first store group (W^T, P, gates) reads: wait until it has been read.
-        if (tid == kDeliverTid) bulk_wait_read_all_but_one();
-        __syncthreads();
+        // A / P rewrites the P buffer that the step before last's first store
+        // group read: wait until it has been read (the last step's groups may
+        // still be reading).
+        if (tid == kDeliverTid) bulk_wait_read_all_but_two();
+        {
+            GDN_BAR_T0();
+            __syncthreads();
+            GDN_BAR_T1(1);
+        }
 #pragma unroll
         for (int q = 0; q < 1024 / kThreads; ++q) {
             const int x = tid + q * kThreads;  // K halves: 2 x 512 chunks
             convert16(kqv + (x >> 9) * 16384, x & 511);
+        }
+        } else {
+        // a later step of the item: only the store-group wait above
+        if (tid == kDeliverTid) bulk_wait_read_all_but_two();
+        {
+            GDN_BAR_T0();
+            __syncthreads();
+            GDN_BAR_T1(1);
+        }
         }
         const bool hp = gt.hp;
         const bool safe = gt.safe;
@@ -567,7 +695,7 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
             const int r = row & 63;
             const int c = 32 * half;
             float v[32];
-            tmem_ld32(trow + PT_G + c, v);
+            tmem_ld32(trow + pt_g + c, v);
             tmem_wait_ld();
             if (safe) {
                 const float sr = row < kC ? gt.bG[r] : gt.Gam[r];
@@ -591,21 +719,18 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
                 for (int x = 0; x < 32; ++x) v[x] = (c + x <= r) ? v[x] : 0.f;
 #pragma unroll
                 for (int e = 0; e < 32; e += 8)
-                    st_row_chunk(sm + P_P16, r, (c + e) / 8, pack8_track(v + e, kmax));
+                    st_row_chunk(sm + P_P16 + (s & 1) * 8192, r, (c + e) / 8,
+                                 pack8_track(v + e, kmax));
             }
         }
+        // the solve rewrites the last step's W^T staging (its first store group)
+        if (tid == kDeliverTid) bulk_wait_read_all_but_one();
         __syncthreads();
         GDN_CL_PHASE(1, 5);  // A / P
 
-        // The T tiles below overwrite the previous chunk's U~ staging: its
-        // stores must have read it (long done by now; the solve's first
-        // barrier orders this before every thread's writes).  Waiting for
-        // those stores to land, and signalling the chunk ready, comes later,
-        // in the U~ / W window, where this warp idles.
-        if (tid == kDeliverTid) bulk_wait_read_all();
-
-        // ---- Q^T = Q^T I on the tensor cores while the solve runs (exact: bf16 x 1) ----
-        if (tid == 0) {
+        // ---- Q^T = Q^T I on the tensor cores while the solve runs (exact: bf16 x 1),
+        //      once per item ----
+        if (tid == 0 && hi == 0) {
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
                 mma_f16_ss(tmem + PT_Q, make_sdesc(skqv + 8192 + ks * 2048, 16384, 1024),
@@ -615,39 +740,61 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
 
         // ---- T = (I + A)^-1 ----
         solve_tril64(As, Ts, Xs, tid);
+        // The T tiles below overwrite the last step's U~ staging: its stores
+        // must have read it.  (Waiting for those stores to land, and signalling
+        // the chunk ready, comes later, in the U~ / W window.)
+        if (tid == kDeliverTid) bulk_wait_read_all();
+        {
+            GDN_BAR_T0();
+            __syncthreads();
+            GDN_BAR_T1(2);
+        }
         GDN_CL_PHASE(1, 6);  // solve
 
         // ---- rows of T diag(b) (bf16 hi / mid / lo: exact, and V needs no
-        //      conversion) and T diag(b Gamma) (fp16 hi / lo, as K) ----
+        //      conversion) and T diag(b Gamma) (fp16 hi / lo, as K): thread
+        //      (row r, quarter cq) does columns 16 cq .. 16 cq + 15 of both ----
         {
-            const int grp = tid >> 6, r = tid & 63;
-            const bool tg = grp >= 2;
-            const int c = 32 * (grp & 1);
-            const float *scale = tg ? gt.bG : gt.bb;
-            float x[32];
+            const int r = tid & 63, cq = tid >> 6;
+            float tb[16], tg[16];
 #pragma unroll
-            for (int e = 0; e < 32; e += 4) {
-                const float4 t4 = *reinterpret_cast<const float4 *>(Ts + r * kTS + c + e);
+            for (int e = 0; e < 16; e += 4) {
+                const float4 t4 = *reinterpret_cast<const float4 *>(Ts + r * kTS + 16 * cq + e);
                 const float tv[4] = {t4.x, t4.y, t4.z, t4.w};
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
-                    const int i = c + e + q;
-                    x[e + q] = (i <= r) ? tv[q] * scale[i] : 0.f;
+                    const int i = 16 * cq + e + q;
+                    tb[e + q] = (i <= r) ? tv[q] * gt.bb[i] : 0.f;
+                    tg[e + q] = (i <= r) ? tv[q] * gt.bG[i] : 0.f;
                 }
             }
-            if (tg)
-                store_split32(sm + P_TGH, sm + P_TGL, r, c, x, hp, kmax);
-            else
-                store_split32_bf16x3(sm + P_TBH, sm + P_TBM, sm + P_TBL, r, c, x);
+            kmax = fmaxf(kmax, max_abs<16>(tg));
+#pragma unroll
+            for (int e = 0; e < 16; e += 8) {
+                uint4 hi, mid, lo;
+                split8_bf16x3(tb + e, hi, mid, lo);
+                const int ch = (16 * cq + e) / 8;
+                st_row_chunk(sm + P_TBH, r, ch, hi);
+                st_row_chunk(sm + P_TBM, r, ch, mid);
+                st_row_chunk(sm + P_TBL, r, ch, lo);
+                split8(tg + e, hi, lo);
+                st_row_chunk(sm + P_TGH, r, ch, hi);
+                if (hp) st_row_chunk(sm + P_TGL, r, ch, lo);
+            }
         }
-        publish();
+        {
+            GDN_BAR_T0();
+            publish();
+            GDN_BAR_T1(3);
+        }
         GDN_CL_PHASE(1, 7);  // T tiles
 
         // ---- U~^T = V^T (T diag b)^T,  W^T = K^T (T diag(b Gamma))^T ----
         if (tid == 0) {
+            if (!mbar_wait_bounded(&ms->tma_v[vb], (s / kVBufs) & 1, kWaitLimit)) timed_out = true;
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) {  // bf16 V times [hi | mid | lo] of T diag(b)
-                const uint64_t a = make_sdesc(skqv + 32768 + ks * 2048, 8192, 1024);
+                const uint64_t a = make_sdesc(svt + ks * 2048, 8192, 1024);
                 const uint64_t b = make_sdesc(sbase + P_TBH + ks * 32, 16, 1024);
                 mma_f16_ss(tmem + PT_U, a, b, IDESC_MK_N192_BF16, ks != 0);
             }
@@ -656,28 +803,49 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
             for (int ks = 0; ks < 4; ++ks) {  // fp16 K times [hi | lo] of T diag(b Gamma)
                 const uint64_t a = make_sdesc(skqv + ks * 2048, 16384, 1024);
                 const uint64_t b = make_sdesc(sbase + P_TGH + ks * 32, 16, 1024);
-                mma_f16_ss(tmem + PT_G, a, b, idesc_w, ks != 0);
+                mma_f16_ss(tmem + PT_W, a, b, idesc_w, ks != 0);
             }
             mma_commit(&ms->mma_bar);
         }
-        if (warp == kGatesWarp && ms->items[(l + 1) & 3].valid) compute_gates(ms->gt[(l + 1) & 1]);
-        // side duties while these products run
-        if (tid == kRefillTid) {  // refill its tile buffer (its stores have read it)
-            const Item nx = ms->items[(l + 1) & 3];
-            if (l >= 1 && nx.valid) issue_tma((l + 1) & 1, nx);
+        if (warp == kGatesWarp) {
+            const int ln = (s + 1) / nh;
+            if (ms->items[ln & 3].valid) compute_gates(ms->gt[(s + 1) & 1]);
         }
-        if (tid == kFetchTid) ms->items[(l + 2) & 3] = fetch(l + 2);  // decode chunk l + 2
-        if (tid == kDeliverTid) flush_delivery();  // the previous chunk, landed -> ready
-        if (tid == kSlotTid) {  // make sure this chunk's ring slot is free
-            if constexpr (kPool) {
+        // side duties while these products run
+        if (tid == kRefillTid) {  // tile loads into buffers whose stores have read them
+            const int ln = (s + 1) / nh, hn = (s + 1) - ln * nh;
+            const Item nv = ms->items[ln & 3];
+            if (nv.valid) {  // step s + 1's V tile
+                issue_v((s + 1) % kVBufs, nv, hn);
+                v_loaded = s + 2;
+            }
+            const Item nk = ms->items[(l + 1) & 3];
+            if (hi == nh - 1 && nk.valid) {  // item l + 1's K / Q tiles
+                issue_kq((l + 1) & 1, nk);
+                kq_loaded = l + 2;
+            }
+        }
+        if (tid == kFetchTid && hi == 0) ms->items[(l + 2) & 3] = fetch(l + 2);  // decode item l + 2
+        if constexpr (kPool) {
+            if (tid == kDeliverTid) {  // earlier deliveries -> ready; this chunk's ring slot free
                 const uint32_t need = (uint32_t)(it.c - p.ring_slots + 1);
                 // a free slot seen early needs no fence: the stores that refill it
                 // depend on that observation, and the chain publishes it only after
                 // its load of the slot has completed
-                if (it.c >= p.ring_slots && early_taken < need &&
-                    !wait_flag_geq(unit_flags(p, it.unit), need, p.flags + 1, p.flag_wait_limit))
-                    timed_out = true;
-            } else {
+                if (it.c >= p.ring_slots && early_taken < need) {
+                    // about to wait on a chain: first report every delivery held,
+                    // so that no producer waits while holding one back
+                    flush_delivery();
+                    if (!wait_flag_geq(unit_flags(p, it.unit), need, p.flags + 1,
+                                       p.flag_wait_limit))
+                        timed_out = true;
+                } else {
+                    flush_older();
+                }
+            }
+        } else {
+            if (tid == kDeliverTid) flush_delivery();  // the previous chunk, landed -> ready
+            if (tid == kSlotTid) {  // make sure this chunk's ring slot is free
                 if (l >= 1 && !mbar_wait_cluster_bounded(&ms->taken, (l - 1) & 1, kWaitLimit))
                     timed_out = true;
             }
@@ -691,10 +859,10 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
         {
             const int c = 32 * half;
             float v[32];
-            tmem_ld32(trow + PT_G + c, v);
+            tmem_ld32(trow + PT_W + c, v);
             if (hp) {
                 float w2[32];
-                tmem_ld32(trow + PT_G + 64 + c, w2);
+                tmem_ld32(trow + PT_W + 64 + c, w2);
                 tmem_wait_ld();
 #pragma unroll
                 for (int x = 0; x < 32; ++x) v[x] += w2[x];
@@ -721,11 +889,12 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
             if (tid == 0) {
                 ms->gst.hp = hp;
                 ms->gst.qs = gt.qs;
+                ms->gst.hp_next = gt.hp_next;
             }
         }
-        {   // Q^T fp16 (MN-major: row d holds 64 tokens) from TMEM into the V half
-            // of the tile buffer, which the U~ product has finished reading;
-            // scaled by Gamma when the gates allow (qs); tokens past L zeroed
+        {   // Q^T fp16 (MN-major: row d holds 64 tokens) from TMEM into this step's V
+            // buffer, which the U~ product has finished reading; scaled by this
+            // head's Gamma when the gates allow (qs); tokens past L zeroed
             if (!mbar_wait_bounded(&ms->qt_bar, l & 1, kWaitLimit)) timed_out = true;
             tc_fence_after_sync();
             const int c = 32 * half;
@@ -740,7 +909,7 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
             }
 #pragma unroll
             for (int e = 0; e < 32; e += 8)
-                st_row_chunk(kqv + 32768, row, (c + e) / 8, pack8_track(v + e, kmax));
+                st_row_chunk(vt, row, (c + e) / 8, pack8_track(v + e, kmax));
         }
         fence_proxy_async_smem();  // staged data -> visible to the bulk copies
         // a key-side fp16 operand of this chunk (K, Q^T, P, T diag(b Gamma), W^T)
@@ -753,7 +922,10 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
         GDN_CL_PHASE(1, 9);  // staging
 
         // ---- deliver with asynchronous stores (the ring slot is free: see above) ----
-        if (__syncthreads_or(timed_out ? 1 : 0)) {
+        GDN_BAR_T0();
+        const int voted_ = __syncthreads_or(timed_out ? 1 : 0);
+        GDN_BAR_T1(0);
+        if (voted_) {
             if (tid == 0) {
                 raise_error(p.err, GDN_ERR_TIMEOUT);
                 if constexpr (kPool) pool_abort(p);
@@ -767,26 +939,33 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
             fence_proxy_async_global();  // the chain's reads of this slot precede our writes
             // group 1: what the next chunk rewrites first (read before its A / P)
             bulk_store(dst + SL_WH, sm + P_WST, hp ? 32768 : 16384);
-            bulk_store(dst + SL_P16, sm + P_P16, 8192);
+            bulk_store(dst + SL_P16, sm + P_P16 + (s & 1) * 8192, 8192);
             bulk_store(dst + SL_GATES, &ms->gst, (uint32_t)sizeof(GatesBlock));
             bulk_commit();
-            // group 2: U~ (in the T tiles' space), K and Q^T (in the tile buffer)
+            // group 2: U~ (in the T tiles' space), K (in the item's K / Q buffer)
+            // and Q^T (in the step's V buffer)
             bulk_store(dst + SL_UT, sm + P_UTS, 32768);
             bulk_store(dst + SL_K16, kqv, 8192);
             bulk_store(dst + SL_K16 + 8192, kqv + 16384, 8192);
-            bulk_store(dst + SL_QT, kqv + 32768, 16384);
+            bulk_store(dst + SL_QT, vt, 16384);
             bulk_commit();
+            older = pending;  // pool: signalled during the next chunk (cluster: already)
             pending = it;
         }
         GDN_CL_PHASE(1, 11);  // deliver (issue)
     }
     if (tid == kDeliverTid) flush_delivery();  // the last chunk delivered
     GDN_CL_PHASE_END(1);
-    // A tile load issued for a chunk this loop never reached must land before
-    // this CTA's shared memory can go away (chunk l + 1's, after a timeout;
-    // on a normal exit chunks l and l + 1 do not exist).
-    if (broke && ms->items[(l + 1) & 3].valid)
-        mbar_wait_bounded(&ms->tma_bar[(l + 1) & 1], ((l + 1) >> 1) & 1, kWaitLimit);
+    GDN_BAR_END(1);
+    // Tile loads issued for steps or items this loop never reached must land
+    // before this CTA's shared memory can go away (after a timeout; on a
+    // normal exit nothing is in flight).
+    if (broke) {  // (waiting again on a phase that completed returns at once)
+        for (int ss = s; ss < v_loaded; ++ss)
+            mbar_wait_bounded(&ms->tma_v[ss % kVBufs], (ss / kVBufs) & 1, kWaitLimit);
+        for (int ll = l; ll < kq_loaded; ++ll)
+            mbar_wait_bounded(&ms->tma_bar[ll & 1], (ll >> 1) & 1, kWaitLimit);
+    }
 }
 
 // ---------------------------------------------------------------- chain --
@@ -822,18 +1001,25 @@ __device__ void chain_role(uint8_t *sm, const CUtensorMap *tm_o, const ChainPara
         s_up = exp2i(e);
         sd = exp2i(-e);
     };
-    // 64 values of this thread's state row (scaled) -> the hi / lo TMEM operands
-    auto split_state = [&](const float (&sv)[64]) {
-        uint32_t hi[32], lo[32];
+    // 64 values of this thread's state row (scaled) -> the hi (and lo) TMEM
+    // operands; the lo part only when the next chunk's products read it
+    auto split_state = [&](const float (&sv)[64], bool with_lo) {
+        uint32_t hi[32];
+        if (with_lo) {
+            uint32_t lo[32];
 #pragma unroll
-        for (int x = 0; x < 64; x += 2) {
-            const __half2 hh = __floats2half2_rn(sv[x], sv[x + 1]);
-            const float2 hf = __half22float2(hh);
-            hi[x / 2] = *reinterpret_cast<const uint32_t *>(&hh);
-            lo[x / 2] = pack_half2(sv[x] - hf.x, sv[x + 1] - hf.y);
+            for (int x = 0; x < 64; x += 2) {
+                const __half2 hh = __floats2half2_rn(sv[x], sv[x + 1]);
+                const float2 hf = __half22float2(hh);
+                hi[x / 2] = *reinterpret_cast<const uint32_t *>(&hh);
+                lo[x / 2] = pack_half2(sv[x] - hf.x, sv[x + 1] - hf.y);
+            }
+            tmem_st32u(trow + CT_SL + 32 * half, lo);
+        } else {
+#pragma unroll
+            for (int x = 0; x < 64; x += 2) hi[x / 2] = pack_half2(sv[x], sv[x + 1]);
         }
         tmem_st32u(trow + CT_SH + 32 * half, hi);
-        tmem_st32u(trow + CT_SL + 32 * half, lo);
     };
     auto store_state = [&](const float (&sv)[64]) {  // the scaled fp32 master
 #pragma unroll
@@ -862,7 +1048,7 @@ __device__ void chain_role(uint8_t *sm, const CUtensorMap *tm_o, const ChainPara
 #pragma unroll
         for (int x = 0; x < 64; ++x) sv[x] *= sd;
         store_state(sv);
-        split_state(sv);
+        split_state(sv, true);
         tmem_wait_st();
     }
     tc_fence_before_sync();
@@ -887,7 +1073,9 @@ __device__ void chain_role(uint8_t *sm, const CUtensorMap *tm_o, const ChainPara
     // Has chunk cc reached the ring?  (load thread)  The pool kernel reads the
     // flag with a relaxed load whose value is only examined on a later call,
     // so the L2 round trip overlaps other work; an observed flag is turned
-    // into an acquire by a fence.
+    // into an acquire by reading it again with an acquire load (a gpu-scope
+    // fence there held the load thread, and the barrier after it, for over a
+    // thousand cycles).
     uint32_t polled = 0;
     int polled_for = -1;  // the chunk whose flag `polled` holds
     auto read_flag = [&](int cc) {
@@ -899,7 +1087,9 @@ __device__ void chain_role(uint8_t *sm, const CUtensorMap *tm_o, const ChainPara
     auto ready_try = [&](int cc) -> bool {
         if constexpr (kPool) {
             if (polled_for == cc && polled >= (uint32_t)(cc + 1)) {
-                fence_acq_rel_gpu();
+                // acquire: re-read the flag (it only grows) with an acquire load,
+                // which costs far less than a gpu-scope fence
+                (void)ld_acquire_gpu(uflags + 1 + (cc & (p.ring_slots - 1)));
                 polled_for = -1;
                 return true;
             }
@@ -925,8 +1115,9 @@ __device__ void chain_role(uint8_t *sm, const CUtensorMap *tm_o, const ChainPara
     // soon as it is reported ready, while chunk c is processed; the shared
     // slot held chunk c - 1, which is finished.
     int loaded = 0;  // chunks whose load has been issued
+    // (the output tile store from this shared slot has read it: the store
+    // thread waited for that before an earlier CTA barrier)
     auto issue_load = [&](int cc) {  // four copies, which the copy engine can overlap
-        bulk_wait_read_all();        // an output tile store from this shared slot has read it
         fence_proxy_async_global();  // the producer's stores, acquired, precede our bulk load
         uint64_t *bar = &ms->full[cc & 1];
         mbar_arrive_expect_tx(bar, SLOT_BYTES);
@@ -957,17 +1148,18 @@ __device__ void chain_role(uint8_t *sm, const CUtensorMap *tm_o, const ChainPara
     };
     // Chunk cc's output from its staging area (the consumed Q^T region of its
     // shared slot) to global memory: a full chunk as one tile store issued by
-    // the load thread (read back before the slot is reloaded, see issue_load);
-    // the last, partial chunk of a sequence with 16-byte stores of warps 2..7,
-    // so nothing past the sequence is written.  Warps 0 and 1 take no part in
-    // those: the load thread fences before its ring loads, and a fence waits
-    // for the issuing thread's own outstanding stores.
+    // the store thread (which waits for it to read the slot before the next
+    // CTA barrier: the slot is reloaded after that); the last, partial chunk
+    // of a sequence with 16-byte stores of warps 2..7, so nothing past the
+    // sequence is written.  Warps 0 and 1 take no part in either: the MMA
+    // thread and the load thread fence, and a fence waits for the issuing
+    // thread's own outstanding stores.
     auto store_o = [&](int cc) {
         const int64_t cc0 = t_begin + (int64_t)kC * cc;
         const int cL = (int)((t_end - cc0) < kC ? (t_end - cc0) : kC);
         const uint8_t *ostb = sm + (cc & 1) * SLOT_BYTES + SL_OST;
         if (cL == kC) {
-            if (tid == kLoadTid) {
+            if (tid == kStoreTid) {
                 tma_store_3d(tm_o, ostb, 0, h, (int32_t)cc0);
                 bulk_commit();
             }
@@ -1006,7 +1198,11 @@ __device__ void chain_role(uint8_t *sm, const CUtensorMap *tm_o, const ChainPara
                 mbar_arrive(&ms->full[k]);
             }
         }
-        if (!mbar_wait_bounded(&ms->full[k], (c >> 1) & 1, kWaitLimit)) timed_out = true;
+        {
+            GDN_BAR_T0();
+            if (!mbar_wait_bounded(&ms->full[k], (c >> 1) & 1, kWaitLimit)) timed_out = true;
+            GDN_BAR_T1(3);
+        }
         GDN_CL_PHASE(0, 0);  // wait: delivery
         if (tid == kLoadTid && have) {  // the chunk is out of the ring: its slot may be refilled
             if constexpr (kPool)
@@ -1039,7 +1235,11 @@ __device__ void chain_role(uint8_t *sm, const CUtensorMap *tm_o, const ChainPara
         if (c > 0) store_o(c - 1);
         fence_proxy_async_smem();
         GDN_CL_PHASE(0, 1);  // issue S Q^T, R
-        if (!mbar_wait_bounded(&ms->mma_bar, mma_phase, kWaitLimit)) timed_out = true;
+        {
+            GDN_BAR_T0();
+            if (!mbar_wait_bounded(&ms->mma_bar, mma_phase, kWaitLimit)) timed_out = true;
+            GDN_BAR_T1(2);
+        }
         mma_phase ^= 1;
         tc_fence_after_sync();
         GDN_CL_PHASE(0, 2);  // wait: S Q^T, R
@@ -1105,10 +1305,13 @@ __device__ void chain_role(uint8_t *sm, const CUtensorMap *tm_o, const ChainPara
             eu = es;
             store_u();
             if (!qs) scale_o(1.f, true);
+            if (tid == kStoreTid) bulk_wait_read_all();  // the chunk's output store has read its slot
             tmem_wait_st();
             tc_fence_before_sync();
+            GDN_BAR_T0();
             const unsigned b =
                 cta_or8(__reduce_or_sync(0xffffffffu, scale_bits(am)), ms->vote[0], warp, lane);
+            GDN_BAR_T1(0);
             if (rescale_needed(b)) {  // rare: U takes its own scale, O moves to it
                 tc_fence_after_sync();
                 float ut[32];
@@ -1192,16 +1395,19 @@ __device__ void chain_role(uint8_t *sm, const CUtensorMap *tm_o, const ChainPara
             };
             am = max_abs<64>(sv);
             if (!same) rescale();
+            const bool lo_next = gb->hp_next != 0;
             store_state(sv);
-            split_state(sv);
+            split_state(sv, lo_next);
             poll_next(c);
             GDN_CL_PHASE(0, 5);  // o staging, S copies
             fence_proxy_async_smem();  // our writes to the slot precede the next bulk load into it
             tmem_wait_st();
             tc_fence_before_sync();
+            GDN_BAR_T0();
             const unsigned b = cta_or8(
                 __reduce_or_sync(0xffffffffu, (same ? scale_bits(am) : 2u) | (timed_out ? 8u : 0u)),
                 ms->vote[1], warp, lane);
+            GDN_BAR_T1(1);
             tc_fence_after_sync();
             if (b & 8u) {
                 if (tid == 0) {
@@ -1215,7 +1421,7 @@ __device__ void chain_role(uint8_t *sm, const CUtensorMap *tm_o, const ChainPara
                 am = max_abs<64>(sv);
                 rescale();
                 store_state(sv);
-                split_state(sv);
+                split_state(sv, lo_next);
                 tmem_wait_st();
                 tc_fence_before_sync();
                 __syncthreads();
@@ -1239,8 +1445,9 @@ __device__ void chain_role(uint8_t *sm, const CUtensorMap *tm_o, const ChainPara
         }
     }
     if (!aborted && nch > 0) store_o(nch - 1);  // the last chunk's output
-    if (tid == kLoadTid) bulk_wait_all();  // every output tile store has landed
+    if (tid == kStoreTid) bulk_wait_all();  // every output tile store has landed
     GDN_CL_PHASE_END(0);
+    GDN_BAR_END(0);
     if (aborted) {
         // A prefetch still landing in shared memory must finish (c is one past
         // the chunk that voted; every earlier load has been waited for).
@@ -1275,6 +1482,7 @@ __device__ __forceinline__ uint32_t *setup_role(uint8_t *sm, bool chain, uint32_
         if (tid == 0) {
             mbar_init(&ms->tma_bar[0], 1);
             mbar_init(&ms->tma_bar[1], 1);
+            for (int b = 0; b < kVBufs; ++b) mbar_init(&ms->tma_v[b], 1);
             mbar_init(&ms->mma_bar, 1);
             mbar_init(&ms->taken, 1);
             mbar_init(&ms->qt_bar, 1);
@@ -1322,7 +1530,8 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
     if (rank == 0)
         chain_role<false>(sm, &tm_o, p, unit, n, h, t_begin, t_end, nch);
     else
-        producer_role<false>(sm, &tm_q, &tm_k, &tm_v, p, unit, rank - 1, h, j, t_begin, t_end, nch);
+        producer_role<false, 1>(sm, &tm_q, &tm_k, &tm_v, p, unit, rank - 1, h, j, t_begin, t_end,
+                                nch);
 
     tc_fence_before_sync();
     __syncthreads();
@@ -1331,6 +1540,8 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
     cluster_sync();  // nobody's shared memory goes away while another CTA may address it
 }
 
+// kNh: v-heads per producer item (p.nh)
+template <int kNh>
 __global__ void __launch_bounds__(kThreads, 1)
     gdn_prefill_pool_kernel(const __grid_constant__ CUtensorMap tm_q,
                             const __grid_constant__ CUtensorMap tm_k,
@@ -1357,7 +1568,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (chain)
         chain_role<true>(sm, &tm_o, p, unit, n, h, t_begin, t_end, nch);
     else
-        producer_role<true>(sm, &tm_q, &tm_k, &tm_v, p, 0, 0, 0, 0, 0, 0, 0);
+        producer_role<true, kNh>(sm, &tm_q, &tm_k, &tm_v, p, 0, 0, 0, 0, 0, 0, 0);
 
     tc_fence_before_sync();
     __syncthreads();
@@ -1418,6 +1629,10 @@ bool fill_params(const PrefillArgs &a, ChainParams &p, CUtensorMap &mq, CUtensor
     p.recall_first = a.order == GDN_ORDER_RECALL_FIRST;
     p.flag_wait_limit = kWaitLimit;
     p.skip_unit = -1;
+    // heads per pool producer item: the largest of 3, 2, 1 that divides the
+    // v-heads per q/k head
+    const int G = a.Hv / a.Hqk;
+    p.nh = G % 3 == 0 ? 3 : (G % 2 == 0 ? 2 : 1);
     return true;
 }
 }  // namespace
@@ -1449,8 +1664,9 @@ cudaError_t launch_prefill_pool(const PrefillArgs &a, cudaStream_t s) {
     // the chunk counter, abort flag and hand-off flags start at zero
     cudaError_t e = cudaMemsetAsync(a.ws, 0, fb, s);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(gdn_prefill_pool_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kSmemBytes);
+    auto kern = p.nh == 3 ? gdn_prefill_pool_kernel<3>
+                          : (p.nh == 2 ? gdn_prefill_pool_kernel<2> : gdn_prefill_pool_kernel<1>);
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)sms);
@@ -1462,7 +1678,7 @@ cudaError_t launch_prefill_pool(const PrefillArgs &a, cudaStream_t s) {
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, gdn_prefill_pool_kernel, mq, mk, mv, mo, p);
+    e = cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, mo, p);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
@@ -1470,6 +1686,17 @@ cudaError_t launch_prefill_pool(const PrefillArgs &a, cudaStream_t s) {
 }  // namespace gdn
 
 #ifdef GDN_TC_PHASES
+extern "C" GDN_API int gdn_debug_bar_waits(long long *out, int reset) {
+    unsigned long long host[64];
+    if (cudaMemcpyFromSymbol(host, gdn_cl_bar_wait, sizeof(host)) != cudaSuccess) return -1;
+    for (int i = 0; i < 64; ++i) out[i] = (long long)host[i];
+    if (reset) {
+        const unsigned long long zero[64] = {0};
+        cudaMemcpyToSymbol(gdn_cl_bar_wait, zero, sizeof(zero));
+    }
+    return 0;
+}
+
 extern "C" GDN_API int gdn_debug_cluster_phases(long long *out, int reset) {
     unsigned long long host[32];
     if (cudaMemcpyFromSymbol(host, gdn_cl_phase_clk, sizeof(host)) != cudaSuccess) return -1;

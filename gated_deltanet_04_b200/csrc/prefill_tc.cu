@@ -366,7 +366,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             ms->bG[r0] = bpre0 * Gr0;        ms->bG[r0 + 1] = bpre1 * Gr1;
             if (lane == 0) {
                 ms->safe = safe_;
-                ms->hp = GC >= kHighPrecisionDecay;
+                // from the chunk's summed log-decay, the number the previous
+                // chunk used to decide whether to write the state's lo part
+                ms->hp = ms->gsum_next >= kLogHighPrecisionDecay;
             }
             if (has_next) load_gates(c0 + kC);  // prefetch the next chunk's gates
         }
@@ -652,7 +654,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int x = 0; x < 32; ++x) ost[(c + x) * kD + row] = __float2bfloat16_rn(v[x] * uu);
             const float gnext = has_next ? expf(ms->gsum_next) : 1.f;
-            const bool lo_next = gnext >= kHighPrecisionDecay;
+            const bool lo_next = has_next && ms->gsum_next >= kLogHighPrecisionDecay;
             const bool same = eu == es;  // uniform over the CTA
             // same: S' in the state's scale; otherwise (U took its own scale this
             // chunk) S' in fp32, unscaled, and a new scale for it

@@ -153,9 +153,21 @@ __device__ __forceinline__ void bulk_wait_read_all_but_one() {
     asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
 }
 
+// Waits until the sources of all but the two most recent committed bulk
+// store groups have been read.
+__device__ __forceinline__ void bulk_wait_read_all_but_two() {
+    asm volatile("cp.async.bulk.wait_group.read 2;" ::: "memory");
+}
+
 // Waits until every committed bulk store has completed.
 __device__ __forceinline__ void bulk_wait_all() {
     asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
+// Waits until all but the two most recent committed bulk store groups have
+// completed.
+__device__ __forceinline__ void bulk_wait_all_but_two() {
+    asm volatile("cp.async.bulk.wait_group 2;" ::: "memory");
 }
 
 // -------------------------------------------------------------- clusters --

@@ -18,6 +18,10 @@ constexpr int kC = 64;      // chunk length
 constexpr int kD = 128;     // Dk = Dv
 constexpr long long kWaitLimit = 1ll << 31;  // SM clocks (about a second)
 constexpr float kHighPrecisionDecay = 0.2f;  // Gamma_C at or above -> extra passes
+// The same threshold on the chunk's summed log-decay, log(0.2), which is how
+// the kernels decide it: one sum, in one fixed order, for every party that
+// needs the decision of a chunk.
+constexpr float kLogHighPrecisionDecay = -1.6094379f;
 constexpr int kAS4 = 68; // row stride of A for solve_tril64 (16-byte aligned rows)
 constexpr int kTS = 68;  // row stride of T (16-byte aligned rows for float4 access)
 
@@ -117,6 +121,15 @@ __device__ __forceinline__ float exp2i(int e) { return __uint_as_float((uint32_t
 
 // Largest fp16 magnitude that does not round to infinity is just below this.
 constexpr float kFp16Overflow = 65520.f;
+
+// Sum over the warp of one value per lane, by xor butterflies: every lane
+// ends with the same, bit-identical total (each step adds a pair of equal
+// partial sums in both lanes of the pair).
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+    return x;
+}
 
 // 2^e with e clamped to [-126, 127].
 __device__ __forceinline__ float exp2c(int e) { return exp2i(min(max(e, -126), 127)); }
@@ -288,8 +301,10 @@ __device__ __forceinline__ void mm16x8_tf32(const float *Lp, int ls, const float
 // T = (I + A)^-1 for the 64 x 64 strictly lower A in As (row stride kAS4),
 // into Ts (row stride kTS), fp32, 256 threads.  Three steps:
 //   1. the four 16 x 16 diagonal blocks D_i = (I + A_ii)^-1, by forward
-//      substitution (one thread per (block, column)); the threads idle there
-//      write zeros above the diagonal blocks;
+//      substitution (lanes 0-15 of warp 4 + i, one per column of block i, so
+//      the four blocks run on the four SM sub-partitions, on warps that carry
+//      no other duties here); the other threads write zeros above the
+//      diagonal blocks;
 //   2. T_10 = -D_1 A_10 D_0 and T_32 = -D_3 A_32 D_2 (the 32 x 32 halves);
 //   3. the lower-left 32 x 32 block T_bl = -T_bot (A_bl T_top), where T_top and
 //      T_bot are the two lower-triangular 32 x 32 diagonal halves.
@@ -299,8 +314,8 @@ __device__ __forceinline__ void mm16x8_tf32(const float *Lp, int ls, const float
 // before (As complete); the function ends with a barrier.
 __device__ __forceinline__ void solve_tril64(const float *As, float *Ts, float *Xs, int tid) {
     const int warp = tid >> 5, lane = tid & 31;
-    if (tid < kC) {  // 1. diagonal blocks
-        const int bi = tid >> 4, col = tid & 15;
+    if (warp >= 4 && lane < 16) {  // 1. diagonal block warp - 4 (one warp per block: 4 SMSPs)
+        const int bi = warp - 4, col = lane;
         const float *Ab = As + (16 * bi) * kAS4 + 16 * bi;
         float x[16];
 #pragma unroll
@@ -312,7 +327,7 @@ __device__ __forceinline__ void solve_tril64(const float *As, float *Ts, float *
 #pragma unroll
         for (int rr = 0; rr < 16; ++rr) Ts[(16 * bi + rr) * kTS + 16 * bi + col] = x[rr];
     } else {  // zeros above the diagonal blocks: 6 blocks of 16 x 16, 8 floats per thread
-        const int z = tid - kC;              // 0 .. 191
+        const int z = warp >= 4 ? 128 + 16 * (warp - 4) + (lane - 16) : tid;  // 0 .. 191
         const int blk = z >> 5, part = z & 31;
         // upper blocks (bi, bj), bi < bj: (0,1) (0,2) (0,3) (1,2) (1,3) (2,3)
         const int bi = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
