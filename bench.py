@@ -63,7 +63,8 @@ def parse():
                         "long256k, varlen32: one gdn_prefill call; decode256: one layer's "
                         "gdn_decode_step; decode256_bf16: the same with a bfloat16 state; "
                         "frontend16k, frontend256k: gdn_short_conv_norm on a 16,384- or "
-                        "262,144-token layer) "
+                        "262,144-token layer; fused16k, fused256k: gdn_prefill_conv, the front "
+                        "end fused into the pool prefill, on the same) "
                         "W + K times and print its per-call time; no bench line")
     p.add_argument("--kernel", default="auto", choices=["auto", "pool", "cluster", "single_cta", "recurrent"],
                    help="prefill kernel for --case")
@@ -382,6 +383,20 @@ def run_case(args):
                                              None, None, None, 1, Tn, Hqk_, Hv_, 128, 128,
                                              fo[0].data_ptr(), fo[1].data_ptr(), fo[2].data_ptr(),
                                              None, stream.cuda_stream)
+    elif args.case in ("fused16k", "fused256k"):
+        inp = (inputs.make_prefill("layer4k", device=dev, T=16384) if args.case == "fused16k"
+               else inputs.make_prefill("long256k", device=dev))
+        gen = torch.Generator(device=dev).manual_seed(1200)
+        Hqk_, Hv_ = inp["q"].shape[1], inp["v"].shape[1]
+        fw = [0.5 * torch.randn(H * 128, 4, generator=gen, device=dev) for H in (Hqk_, Hqk_, Hv_)]
+        o = torch.empty_like(inp["v"])
+        sT = torch.empty((1, Hv_, 128, 128), dtype=torch.float32, device=dev)
+        fst = torch.empty((1, 3, (2 * Hqk_ + Hv_) * 128), dtype=torch.float32, device=dev)
+        ws = torch.empty(gdn.gdn_prefill_conv_workspace_bytes(1, inp["T"], Hqk_, Hv_, 128, 128),
+                         dtype=torch.uint8, device=dev)
+        fn = lambda: gdn.gdn_prefill_conv(inp["q"], inp["k"], inp["v"], fw[0], fw[1], fw[2], inp["g"],
+                                          inp["beta"], conv_state_out=fst, o=o, final_state=sT,
+                                          workspace=ws)
     elif args.case == "decode256_bf16":
         L = inputs.make_decode_layer(0, device=dev)
         out = torch.empty_like(L["v"])

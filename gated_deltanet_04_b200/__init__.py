@@ -21,7 +21,7 @@ import threading
 import torch
 
 __all__ = ["gdn_prefill", "gdn_decode_step", "gdn_decode_step_bf16_state", "gdn_decode_step_slots",
-           "gdn_short_conv_norm",
+           "gdn_short_conv_norm", "gdn_prefill_conv", "gdn_prefill_conv_workspace_bytes",
            "gdn_prefill_workspace_bytes", "library",
            "GdnError", "LIB_PATH", "STATUS", "KERNELS"]
 
@@ -75,6 +75,12 @@ def library():
             lib.gdn_short_conv_norm.argtypes = [vp, vp, vp, ctypes.c_int, vp, vp, vp, vp, vp, vp,
                                                 i32, i64, i32, i32, i32, i32, vp, vp, vp, vp, vp]
             lib.gdn_short_conv_norm.restype = ctypes.c_int
+            lib.gdn_prefill_conv.argtypes = [vp, vp, vp, ctypes.c_int, vp, vp, vp, vp, vp, vp, vp,
+                                             vp, vp, i32, i64, i32, i32, i32, i32, i32, vp, vp,
+                                             vp, sz, vp, vp]
+            lib.gdn_prefill_conv.restype = ctypes.c_int
+            lib.gdn_prefill_conv_workspace_bytes.argtypes = [i32, i64, i32, i32, i32, i32]
+            lib.gdn_prefill_conv_workspace_bytes.restype = sz
             lib.gdn_prefill_workspace_bytes.argtypes = [i32, i64, i32, i32, i32, i32, i32]
             lib.gdn_prefill_workspace_bytes.restype = sz
             lib.gdn_prefill_ex_workspace_bytes.argtypes = [i32, i64, i32, i32, i32, i32, i32,
@@ -108,6 +114,11 @@ def _check(t, name, shape, dtype, device):
         raise ValueError(f"{name} has dtype {t.dtype}, expected {dtype}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
+
+
+def gdn_prefill_conv_workspace_bytes(N, T, Hqk, Hv, Dk, Dv):
+    """Scratch bytes gdn_prefill_conv needs (0: none, or unsupported shapes)."""
+    return int(library().gdn_prefill_conv_workspace_bytes(N, T, Hqk, Hv, Dk, Dv))
 
 
 def gdn_prefill_workspace_bytes(N, T, Hqk, Hv, Dk, Dv, chunk=0, kernel="auto"):
@@ -319,3 +330,68 @@ def gdn_decode_step_bf16_state(q, k, v, g, beta, state, *, o=None, error_flag=No
     if rc != 0:
         raise GdnError(rc, "gdn_decode_step_bf16_state")
     return o
+
+
+def gdn_prefill_conv(xq, xk, xv, wq, wk, wv, g, beta, initial_state=None, cu_seqlens=None,
+                     conv_state=None, *, conv_state_out=None, output_conv_state=False, o=None,
+                     final_state=None, output_final_state=True, workspace=None, error_flag=None,
+                     stream=None):
+    """gdn_short_conv_norm followed by gdn_prefill in one call, with the front end
+    fused into the pool prefill kernel's load stage (the C entry point
+    gdn_prefill_conv).  Arguments as the two calls: raw channel inputs xq, xk
+    [T,Hqk,128], xv [T,Hv,128] bf16, filters, conv state, then the prefill's.
+    Returns (o, final_state[, conv_state_out])."""
+    lib = library()
+    dev = xq.device
+    if dev.type != "cuda":
+        raise ValueError("gdn_prefill_conv runs on CUDA tensors only")
+    T, Hqk, Dk = xq.shape
+    Hv, Dv = xv.shape[1], xv.shape[2]
+    if xq.dtype not in DTYPE:
+        raise ValueError(f"unsupported io dtype {xq.dtype}")
+    _check(xk, "xk", (T, Hqk, Dk), xq.dtype, dev)
+    _check(xv, "xv", (T, Hv, Dv), xq.dtype, dev)
+    _check(wq, "wq", (Hqk * Dk, 4), torch.float32, dev)
+    _check(wk, "wk", (Hqk * Dk, 4), torch.float32, dev)
+    _check(wv, "wv", (Hv * Dv, 4), torch.float32, dev)
+    _check(g, "g", (T, Hv), torch.float32, dev)
+    _check(beta, "beta", (T, Hv), torch.float32, dev)
+    if cu_seqlens is None:
+        N = 1
+    else:
+        N = cu_seqlens.shape[0] - 1
+        _check(cu_seqlens, "cu_seqlens", (N + 1,), torch.int32, dev)
+    C = 2 * Hqk * Dk + Hv * Dv
+    if conv_state is not None:
+        _check(conv_state, "conv_state", (N, 3, C), torch.float32, dev)
+    if conv_state_out is None and output_conv_state:
+        conv_state_out = torch.empty((N, 3, C), dtype=torch.float32, device=dev)
+    if conv_state_out is not None:
+        _check(conv_state_out, "conv_state_out", (N, 3, C), torch.float32, dev)
+    if initial_state is not None:
+        _check(initial_state, "initial_state", (N, Hv, Dv, Dk), torch.float32, dev)
+    if o is None:
+        o = torch.empty((T, Hv, Dv), dtype=xq.dtype, device=dev)
+    _check(o, "o", (T, Hv, Dv), xq.dtype, dev)
+    if final_state is None and output_final_state:
+        final_state = torch.empty((N, Hv, Dv, Dk), dtype=torch.float32, device=dev)
+    if final_state is not None:
+        _check(final_state, "final_state", (N, Hv, Dv, Dk), torch.float32, dev)
+    ws_bytes = 0
+    if workspace is not None:
+        ws_bytes = workspace.numel() * workspace.element_size()
+    else:
+        need = int(lib.gdn_prefill_conv_workspace_bytes(N, T, Hqk, Hv, Dk, Dv))
+        if need:
+            workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+            ws_bytes = need
+    rc = lib.gdn_prefill_conv(_ptr(xq), _ptr(xk), _ptr(xv), DTYPE[xq.dtype], _ptr(wq), _ptr(wk),
+                              _ptr(wv), _ptr(conv_state), _ptr(conv_state_out), _ptr(g), _ptr(beta),
+                              _ptr(initial_state), _ptr(cu_seqlens), N, T, Hqk, Hv, Dk, Dv, 0,
+                              _ptr(o), _ptr(final_state), _ptr(workspace), ws_bytes,
+                              _ptr(error_flag), _stream(stream))
+    if rc != 0:
+        raise GdnError(rc, "gdn_prefill_conv")
+    if conv_state_out is not None:
+        return o, final_state, conv_state_out
+    return o, final_state

@@ -224,9 +224,55 @@ __global__ void gdn_conv_state_kernel(FeArgs a) {
     for (int i = 0; i < 3; ++i) a.state_out[((int64_t)n * 3 + i) * a.C + cc] = v[i];
 }
 
+// The fused prefill's copy of the filters: per (tensor, head) block of 128
+// channels (q heads, then k heads, then v heads, the conv state's order),
+// 512 floats ordered [tap k][part p][chunk cc][i] for channel 8 cc + 4 p + i,
+// so that the sixteen threads convolving the sixteen 8-channel chunks of a
+// row read one tap's filters as consecutive 16-byte words.
+__global__ void gdn_conv_filter_kernel(const float *wq, const float *wk, const float *wv,
+                                       int32_t Hqk, int32_t Hv, float *dst) {
+    const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx >= (int64_t)(2 * Hqk + Hv) * 512) return;
+    const int blk = (int)(idx >> 9), r = (int)(idx & 511);
+    const int k = r >> 7, part = (r >> 6) & 1, cc = (r >> 2) & 15, i = r & 3;
+    const float *w = blk < Hqk ? wq : blk < 2 * Hqk ? wk : wv;
+    const int head = blk < Hqk ? blk : blk < 2 * Hqk ? blk - Hqk : blk - 2 * Hqk;
+    dst[idx] = w[((int64_t)head * kFeD + 8 * cc + 4 * part + i) * 4 + k];
+}
+
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 }  // namespace
+
+cudaError_t launch_conv_filters(const float *wq, const float *wk, const float *wv, int32_t Hqk,
+                                int32_t Hv, float *dst, cudaStream_t s) {
+    const int64_t total = (int64_t)(2 * Hqk + Hv) * 512;
+    gdn_conv_filter_kernel<<<(unsigned)((total + 255) / 256), 256, 0, s>>>(wq, wk, wv, Hqk, Hv, dst);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_conv_state(const void *xq, const void *xk, const void *xv, gdn_dtype dt,
+                              const float *state_in, float *state_out, const int32_t *cu,
+                              int32_t N, int64_t T, int32_t Hqk, int32_t Hv, int32_t *err,
+                              cudaStream_t s) {
+    FeArgs a;
+    const int32_t Cq = Hqk * kFeD;
+    a.t[0] = {xq, nullptr, nullptr, Hqk, 0, 1};
+    a.t[1] = {xk, nullptr, nullptr, Hqk, Cq, 1};
+    a.t[2] = {xv, nullptr, nullptr, Hv, 2 * Cq, 0};
+    a.cu = cu;
+    a.state_in = state_in;
+    a.state_out = state_out;
+    a.err = err;
+    a.T = T;
+    a.N = N;
+    a.C = 2 * Cq + Hv * kFeD;
+    a.dtype = dt;
+    const int64_t total = (int64_t)N * a.C;
+    gdn_conv_state_kernel<<<(unsigned)((total + 255) / 256), 256, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
 }  // namespace gdn
 
 extern "C" GDN_API gdn_status gdn_short_conv_norm(

@@ -154,6 +154,76 @@ gdn_status gdn_prefill_order(const void *q, const void *k, const void *v, gdn_dt
                         stream, kernel, order, -1, 0);
 }
 
+// gdn_prefill_conv's scratch: the pool kernel's, then (from a 256-byte
+// boundary) the rearranged filters.
+size_t conv_filter_offset(int64_t units) {
+    return (gdn::prefill_pool_workspace_bytes(units) + 255) & ~(size_t)255;
+}
+
+size_t gdn_prefill_conv_workspace_bytes(int32_t N, int64_t T, int32_t Hqk, int32_t Hv, int32_t Dk,
+                                        int32_t Dv) {
+    if (N <= 0 || T <= 0 || Hqk <= 0 || Hv <= 0 || Hv % Hqk != 0 || Dk != 128 || Dv != 128)
+        return 0;
+    const int64_t units = (int64_t)N * Hv;
+    if (units > gdn::kPoolMaxUnits) return 0;
+    return conv_filter_offset(units) + gdn::conv_filter_bytes(Hqk, Hv);
+}
+
+gdn_status gdn_prefill_conv(const void *xq, const void *xk, const void *xv, gdn_dtype io_dtype,
+                            const float *wq, const float *wk, const float *wv,
+                            const float *conv_state_in, float *conv_state_out, const float *g,
+                            const float *beta, const float *initial_state,
+                            const int32_t *cu_seqlens, int32_t N, int64_t T, int32_t Hqk,
+                            int32_t Hv, int32_t Dk, int32_t Dv, int32_t chunk, void *o,
+                            float *final_state, void *workspace, size_t workspace_bytes,
+                            int32_t *dev_error_flag, void *stream) {
+    if (io_dtype != GDN_DTYPE_BF16 && io_dtype != GDN_DTYPE_F32) return GDN_ERR_INVALID_ARGUMENT;
+    if (N < 0 || T < 0 || Hqk <= 0 || Hv <= 0 || Dk <= 0 || Dv <= 0 || chunk < 0)
+        return GDN_ERR_INVALID_ARGUMENT;
+    if (Hv % Hqk != 0) return GDN_ERR_INVALID_ARGUMENT;
+    if (cu_seqlens == nullptr && N != 1) return GDN_ERR_INVALID_ARGUMENT;
+    if (N == 0) return T == 0 ? GDN_OK : GDN_ERR_INVALID_ARGUMENT;
+    if (T > 0 && (!xq || !xk || !xv || !wq || !wk || !wv || !g || !beta || !o))
+        return GDN_ERR_INVALID_ARGUMENT;
+    const void *ptrs[] = {xq, xk, xv, wq, wk, wv, conv_state_in, conv_state_out, g, beta,
+                          initial_state, cu_seqlens, o, final_state, workspace, dev_error_flag};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return GDN_ERR_INVALID_ARGUMENT;
+    const void *ins[] = {xq, xk, xv, wq, wk, wv, g, beta};
+    for (const void *i : ins)
+        if (i && (i == o || i == conv_state_out)) return GDN_ERR_INVALID_ARGUMENT;
+    if (!tc_path(io_dtype, Dk, Dv, chunk)) return GDN_ERR_UNSUPPORTED;
+    const int64_t units = (int64_t)N * Hv;
+    if (units > gdn::kPoolMaxUnits || !gdn::prefill_pool_fits(units)) return GDN_ERR_UNSUPPORTED;
+    const size_t need = gdn_prefill_conv_workspace_bytes(N, T, Hqk, Hv, Dk, Dv);
+    if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return GDN_ERR_INVALID_ARGUMENT;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    float *filters = nullptr;
+    if (T > 0) {
+        filters = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + conv_filter_offset(units));
+        const cudaError_t e = gdn::launch_conv_filters(wq, wk, wv, Hqk, Hv, filters, s);
+        if (e != cudaSuccess) return GDN_ERR_CUDA;
+    }
+    if (T > 0 || final_state != nullptr) {
+        gdn::PrefillArgs a;
+        a.q = xq; a.k = xk; a.v = xv; a.g = g; a.beta = beta; a.s0 = initial_state;
+        a.cu = cu_seqlens; a.o = o; a.sT = final_state; a.err = dev_error_flag; a.ws = workspace;
+        a.T = T; a.N = N; a.Hqk = Hqk; a.Hv = Hv; a.Dk = Dk; a.Dv = Dv; a.chunk = 64;
+        a.dtype = io_dtype;
+        a.conv = true;
+        a.cf = filters;
+        a.cstate_in = conv_state_in;
+        const cudaError_t e = T > 0 ? gdn::launch_prefill_pool(a, s) : gdn::launch_prefill_recurrent(a, s);
+        if (e == cudaErrorNotSupported) return GDN_ERR_UNSUPPORTED;
+        if (e != cudaSuccess) return GDN_ERR_CUDA;
+    }
+    // the new conv state after the prefill, which reads the old one (so the two may alias)
+    if (conv_state_out)
+        return from_cuda(gdn::launch_conv_state(xq, xk, xv, io_dtype, conv_state_in, conv_state_out,
+                                                cu_seqlens, N, T, Hqk, Hv, dev_error_flag, s));
+    return GDN_OK;
+}
+
 gdn_status gdn_debug_prefill_pool_stall(const void *q, const void *k, const void *v,
                                         gdn_dtype io_dtype, const float *g, const float *beta,
                                         const float *initial_state, const int32_t *cu_seqlens,

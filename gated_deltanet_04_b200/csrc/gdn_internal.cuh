@@ -27,6 +27,11 @@ struct PrefillArgs {
     // SM-clock limit of every spin on a hand-off flag (0: the default)
     int32_t debug_skip_unit = -1;
     int64_t debug_flag_wait = 0;
+    // front end fused into the pool kernel's load stage: q, k, v above are then
+    // the raw inputs of the q, k, v channels (see gdn_prefill_conv)
+    bool conv = false;
+    const float *cf = nullptr;  // filters as launch_conv_filters writes them
+    const float *cstate_in = nullptr;                  // [N][3][C] or null (zeros)
 };
 
 struct DecodeArgs {
@@ -77,6 +82,17 @@ size_t prefill_pool_workspace_bytes(int64_t units);
 constexpr int64_t kPoolMaxUnits = 64;
 // Whether the current device has SMs enough for the pool kernel with `units`.
 bool prefill_pool_fits(int64_t units);
+// The new conv state of gdn_short_conv_norm's contract (each sequence's last
+// three inputs of every q, k, v channel), also checking cu_seqlens.
+cudaError_t launch_conv_state(const void *xq, const void *xk, const void *xv, gdn_dtype dt,
+                              const float *state_in, float *state_out, const int32_t *cu,
+                              int32_t N, int64_t T, int32_t Hqk, int32_t Hv, int32_t *err,
+                              cudaStream_t s);
+// The filters wq, wk, wv ([H * 128][4] fp32 each) rearranged for the fused
+// prefill into dst, conv_filter_bytes(Hqk, Hv) bytes.
+cudaError_t launch_conv_filters(const float *wq, const float *wk, const float *wv, int32_t Hqk,
+                                int32_t Hv, float *dst, cudaStream_t s);
+constexpr size_t conv_filter_bytes(int32_t Hqk, int32_t Hv) { return (size_t)(2 * Hqk + Hv) * 2048; }
 
 // ---------------------------------------------------------------- device --
 

@@ -255,7 +255,18 @@ struct ProdMisc {
     uint32_t tmem_base;
 };
 static_assert(P_MISC + sizeof(ProdMisc) <= P_ID, "identity tile after the misc block");
-constexpr uint32_t kProdBytes = P_ID + 8192;
+// Front end fused into the load stage (kConv): 8-row halo tiles (the 8 tokens
+// before a chunk, 128-byte swizzle, 1 KB each) of the raw K and Q inputs (K
+// half 0, K half 1, Q half 0, Q half 1) and of the raw V input (half 0, half
+// 1), and the filters of the item's k and q heads (2 KB each) and of the
+// step's v head (2 KB), in launch_conv_filters' order.  One buffer each: a
+// tile's convolution is over before the load of the next one is issued.
+constexpr uint32_t P_HKQ = P_ID + 8192;
+constexpr uint32_t P_HV = P_HKQ + 4096;
+constexpr uint32_t P_FKQ = P_HV + 2048;
+constexpr uint32_t P_FV = P_FKQ + 4096;
+static_assert(P_HKQ % 1024 == 0 && P_HV % 1024 == 0, "swizzled halo tiles start on 1 KB");
+constexpr uint32_t kProdBytes = P_FV + 2048;
 constexpr uint32_t kChainBytes = C_MISC + sizeof(ChainMisc);
 constexpr uint32_t kSmemBytes = (kProdBytes > kChainBytes ? kProdBytes : kChainBytes) + 1024;
 static_assert(kSmemBytes <= 232448, "fits the 227 KB opt-in shared memory of a CTA");
@@ -292,6 +303,12 @@ struct ChainParams {
     long long flag_wait_limit;  // SM clocks a spin on a hand-off flag may last
     int32_t skip_unit;          // testing: a unit no producer prepares (-1: none)
     int32_t nh;                 // v-heads per pool producer item (divides Hv / Hqk, <= 3)
+    // front end fused into the load stage: the tiles are the raw inputs of
+    // the q, k, v channels, convolved (kernel 4, causal) and, for q and k,
+    // normalised per (token, head) before use
+    const float *cf;            // filters, as launch_conv_filters writes them
+    const float *cstate;        // conv state in, [N][3][cC] (oldest first), or null (zeros)
+    int32_t cC;                 // conv-state channels: q (Hqk 128), k (Hqk 128), v (Hv 128)
 };
 
 __device__ __forceinline__ uint8_t *ring_slot(const ChainParams &p, int unit, int c) {
@@ -368,10 +385,16 @@ __device__ Item pool_fetch(const ChainParams &p, uint32_t first) {
 // kPool: the pool kernel (items from the global counter, p.nh heads each);
 // otherwise producer k of a cluster, whose items are chunks k, k + 2, ... of
 // `unit` (one head).  Item l's head i is step s = l * nh + i.
-template <bool kPool, int kNh>
+// kConv: the front end is fused into the load stage (pool kernel only): tm_q,
+// tm_k, tm_v map the raw inputs of the q, k, v channels and tm_hq, tm_hk,
+// tm_hv the same inputs in 8-token boxes, for the tokens before a chunk.
+template <bool kPool, int kNh, bool kConv = false>
 __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtensorMap *tm_k,
                               const CUtensorMap *tm_v, const ChainParams &p, int unit, int k,
-                              int h, int j, int64_t t_begin, int64_t t_end, int nch) {
+                              int h, int j, int64_t t_begin, int64_t t_end, int nch,
+                              const CUtensorMap *tm_hq = nullptr,
+                              const CUtensorMap *tm_hk = nullptr,
+                              const CUtensorMap *tm_hv = nullptr) {
     ProdMisc *ms = reinterpret_cast<ProdMisc *>(sm + P_MISC);
     const uint32_t sbase = smem_u32(sm);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -427,25 +450,122 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
         if (tn < ten) gnx0 = p.g[tn * p.Hv + hv];
         if (tn + 1 < ten) gnx1 = p.g[(tn + 1) * p.Hv + hv];
     };
-    // K and Q tiles of item `it` into K / Q buffer b (by item parity)
+    // K and Q tiles of item `it` into K / Q buffer b (by item parity); with the
+    // fused front end also the 8 tokens before the chunk (the coordinate may be
+    // negative: the load fills zeros there)
     auto issue_kq = [&](int b, const Item &it) {
         uint8_t *dst = sm + P_KQ + b * P_KQ_BYTES;
-        mbar_arrive_expect_tx(&ms->tma_bar[b], 4 * 8192);
+        mbar_arrive_expect_tx(&ms->tma_bar[b], kConv ? 4 * 8192 + 4 * 1024 + 4096 : 4 * 8192);
         const int32_t t32 = (int32_t)it.c0;
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
             tma_load_3d(dst + hf * 16384, tm_k, &ms->tma_bar[b], 64 * hf, it.j, t32);
             tma_load_3d(dst + hf * 16384 + 8192, tm_q, &ms->tma_bar[b], 64 * hf, it.j, t32);
+            if constexpr (kConv) {
+                uint8_t *hd = sm + P_HKQ;
+                tma_load_3d(hd + hf * 1024, tm_hk, &ms->tma_bar[b], 64 * hf, it.j, t32 - 8);
+                tma_load_3d(hd + 2048 + hf * 1024, tm_hq, &ms->tma_bar[b], 64 * hf, it.j, t32 - 8);
+            }
+        }
+        if constexpr (kConv) {  // k head's filters, then q head's
+            bulk_load(sm + P_FKQ, p.cf + (int64_t)(p.Hqk + it.j) * 512, 2048, &ms->tma_bar[b]);
+            bulk_load(sm + P_FKQ + 2048, p.cf + (int64_t)it.j * 512, 2048, &ms->tma_bar[b]);
         }
     };
-    // V tile of head hh of item `it` into V buffer b (by step % 3)
+    // V tile of head hh of item `it` into V buffer b (by step parity), and its halo
     auto issue_v = [&](int b, const Item &it, int hh) {
         uint8_t *dst = sm + P_V + b * P_V_BYTES;
-        mbar_arrive_expect_tx(&ms->tma_v[b], 2 * 8192);
+        mbar_arrive_expect_tx(&ms->tma_v[b], kConv ? 2 * 8192 + 2 * 1024 + 2048 : 2 * 8192);
         const int32_t t32 = (int32_t)it.c0;
 #pragma unroll
-        for (int hf = 0; hf < 2; ++hf)
+        for (int hf = 0; hf < 2; ++hf) {
             tma_load_3d(dst + hf * 8192, tm_v, &ms->tma_v[b], 64 * hf, it.h + hh, t32);
+            if constexpr (kConv)
+                tma_load_3d(sm + P_HV + hf * 1024, tm_hv, &ms->tma_v[b], 64 * hf, it.h + hh,
+                            t32 - 8);
+        }
+        if constexpr (kConv)
+            bulk_load(sm + P_FV, p.cf + (int64_t)(2 * p.Hqk + it.h + hh) * 512, 2048, &ms->tma_v[b]);
+    };
+    // Fused front end: the "kernel 4" causal convolution of one [64 tokens][128]
+    // bf16 tile (two 64-feature halves `half0` and `half0` + hstride, 128-byte
+    // swizzle), in place, rounded to bf16 once; with `norm`, each token row is
+    // divided by its norm first (a zero row stays zero).  Thread (16-byte chunk
+    // cch of 8 features, rows 4 rb .. 4 rb + 3) reads its rows and the three
+    // before them and works on channel pairs with the two-wide fp32 FMA; the
+    // rows before the chunk come from the halo tile (rows 5 .. 7 of the 8
+    // tokens before the chunk) or, for a sequence's first chunk, from the
+    // carried conv state (or zeros).  `filt`: the head's filters in shared
+    // memory (launch_conv_filters' order); `sch`: the conv state's channel of
+    // the tile's channel 0.  Every thread reads before anyone writes (one CTA
+    // barrier inside).
+    auto conv_tile = [&](uint8_t *half0, uint32_t hstride, const uint8_t *halo0, uint32_t halostride,
+                         const uint8_t *filt, int sch, const Item &it, bool norm) {
+        const int cch = tid & 15, rb = tid >> 4;
+        const int hf = cch >> 3, cb = (cch & 7) * 16;
+        uint8_t *tile = half0 + hf * hstride;
+        const uint8_t *halo = halo0 + hf * halostride;
+        float2 x[7][4];  // rows 4 rb - 3 .. 4 rb + 3; channel pairs
+#pragma unroll
+        for (int i = 0; i < 7; ++i) {
+            const int rr = 4 * rb - 3 + i;
+            if (rr >= 0 || it.c > 0) {
+                const uint4 u = *reinterpret_cast<const uint4 *>(rr >= 0 ? tile + sw128(rr, cb)
+                                                                         : halo + sw128(rr + 8, cb));
+                const uint32_t wv[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    x[i][e] = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&wv[e]));
+            } else if (p.cstate != nullptr) {  // a sequence's first chunk
+                const float *st = p.cstate + ((int64_t)(it.unit / p.Hv) * 3 + rr + 3) * p.cC + sch + 8 * cch;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) x[i][e] = make_float2(st[2 * e], st[2 * e + 1]);
+            } else {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) x[i][e] = make_float2(0.f, 0.f);
+            }
+        }
+        float2 y[4][4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {  // tap k multiplies row t - 3 + k
+            const float4 w0 = *reinterpret_cast<const float4 *>(filt + k * 512 + cch * 16);
+            const float4 w1 = *reinterpret_cast<const float4 *>(filt + k * 512 + 256 + cch * 16);
+            const float2 wk[4] = {make_float2(w0.x, w0.y), make_float2(w0.z, w0.w),
+                                  make_float2(w1.x, w1.y), make_float2(w1.z, w1.w)};
+#pragma unroll
+            for (int jr = 0; jr < 4; ++jr)
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    y[jr][e] = k == 0 ? fmul2(wk[e], x[jr][e]) : ffma2(wk[e], x[jr + k][e], y[jr][e]);
+        }
+        float2 inv[4];
+#pragma unroll
+        for (int jr = 0; jr < 4; ++jr) inv[jr] = make_float2(1.f, 1.f);
+        if (norm) {  // the 16 lanes of a row (lanes 16 (rb & 1) .. + 15) hold its 128 features
+#pragma unroll
+            for (int jr = 0; jr < 4; ++jr) {
+                float2 s2 = fmul2(y[jr][0], y[jr][0]);
+#pragma unroll
+                for (int e = 1; e < 4; ++e) s2 = ffma2(y[jr][e], y[jr][e], s2);
+                float ss = s2.x + s2.y;
+#pragma unroll
+                for (int off = 1; off < 16; off <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+                const float iv = ss > 0.f ? 1.f / sqrtf(ss) : 1.f;
+                inv[jr] = make_float2(iv, iv);
+            }
+        }
+        __syncthreads();  // every read of the tile is done
+#pragma unroll
+        for (int jr = 0; jr < 4; ++jr) {
+            uint32_t wv[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 o2 = fmul2(y[jr][e], inv[jr]);
+                const __nv_bfloat162 b2 = __floats2bfloat162_rn(o2.x, o2.y);
+                wv[e] = *reinterpret_cast<const uint32_t *>(&b2);
+            }
+            *reinterpret_cast<uint4 *>(tile + sw128(4 * rb + jr, cb)) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+        }
     };
     auto mma_sync_point = [&]() {
         if (tid == 0) mma_commit(&ms->mma_bar);
@@ -624,6 +744,15 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
         if (hi == 0) {
         if (!mbar_wait_bounded(&ms->tma_bar[buf], (l >> 1) & 1, kWaitLimit)) timed_out = true;
         GDN_CL_PHASE(1, 2);  // wait: tiles
+        if constexpr (kConv) {
+            // the item's raw k and q tiles -> convolved, each (token, head) row
+            // normalised, rounded to bf16 once, in place
+            conv_tile(kqv, 16384, sm + P_HKQ, 1024, sm + P_FKQ, p.Hqk * kD + item.j * kD, item, true);
+            conv_tile(kqv + 8192, 16384, sm + P_HKQ + 2048, 1024, sm + P_FKQ + 2048, item.j * kD,
+                      item, true);
+            fence_proxy_async_smem();  // -> visible to the Gram and Q^T products
+            __syncthreads();
+        }
         if (tid == 0) {
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
@@ -781,6 +910,11 @@ __device__ void producer_role(uint8_t *sm, const CUtensorMap *tm_q, const CUtens
                 st_row_chunk(sm + P_TGH, r, ch, hi);
                 if (hp) st_row_chunk(sm + P_TGL, r, ch, lo);
             }
+        }
+        if constexpr (kConv) {
+            // this head's raw v tile -> convolved, rounded to bf16 in place
+            if (!mbar_wait_bounded(&ms->tma_v[vb], (s / kVBufs) & 1, kWaitLimit)) timed_out = true;
+            conv_tile(vt, 8192, sm + P_HV, 1024, sm + P_FV, 2 * p.Hqk * kD + it.h * kD, it, false);
         }
         {
             GDN_BAR_T0();
@@ -1540,13 +1674,18 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
     cluster_sync();  // nobody's shared memory goes away while another CTA may address it
 }
 
-// kNh: v-heads per producer item (p.nh)
-template <int kNh>
+// kNh: v-heads per producer item (p.nh).  kConv: the front end fused into the
+// load stage (tm_q, tm_k, tm_v map the raw channel inputs; tm_hq, tm_hk, tm_hv
+// the same in 8-token boxes); otherwise the halo maps are unused.
+template <int kNh, bool kConv>
 __global__ void __launch_bounds__(kThreads, 1)
     gdn_prefill_pool_kernel(const __grid_constant__ CUtensorMap tm_q,
                             const __grid_constant__ CUtensorMap tm_k,
                             const __grid_constant__ CUtensorMap tm_v,
-                            const __grid_constant__ CUtensorMap tm_o, ChainParams p) {
+                            const __grid_constant__ CUtensorMap tm_o,
+                            const __grid_constant__ CUtensorMap tm_hq,
+                            const __grid_constant__ CUtensorMap tm_hk,
+                            const __grid_constant__ CUtensorMap tm_hv, ChainParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = aligned_smem(smem_raw);
     const bool chain = (int)blockIdx.x < p.units;
@@ -1568,7 +1707,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (chain)
         chain_role<true>(sm, &tm_o, p, unit, n, h, t_begin, t_end, nch);
     else
-        producer_role<true, kNh>(sm, &tm_q, &tm_k, &tm_v, p, 0, 0, 0, 0, 0, 0, 0);
+        producer_role<true, kNh, kConv>(sm, &tm_q, &tm_k, &tm_v, p, 0, 0, 0, 0, 0, 0, 0, &tm_hq,
+                                        &tm_hk, &tm_hv);
 
     tc_fence_before_sync();
     __syncthreads();
@@ -1609,6 +1749,7 @@ bool prefill_pool_fits(int64_t units) {
 }
 
 bool make_tile_map_bf16_128(CUtensorMap *m, const void *base, int64_t T, int32_t H);
+bool make_halo_map_bf16_128(CUtensorMap *m, const void *base, int64_t T, int32_t H);
 bool make_store_map_bf16_128(CUtensorMap *m, void *base, int64_t T, int32_t H);
 
 namespace {
@@ -1633,6 +1774,9 @@ bool fill_params(const PrefillArgs &a, ChainParams &p, CUtensorMap &mq, CUtensor
     // v-heads per q/k head
     const int G = a.Hv / a.Hqk;
     p.nh = G % 3 == 0 ? 3 : (G % 2 == 0 ? 2 : 1);
+    p.cf = a.cf;
+    p.cstate = a.cstate_in;
+    p.cC = 2 * a.Hqk * kD + a.Hv * kD;
     return true;
 }
 }  // namespace
@@ -1654,7 +1798,10 @@ cudaError_t launch_prefill_pool(const PrefillArgs &a, cudaStream_t s) {
     CUtensorMap mq, mk, mv, mo;
     if (!fill_params(a, p, mq, mk, mv, mo)) return cudaErrorInvalidValue;
     const int sms = sm_count();
-    if (!prefill_pool_fits(p.units) || sms <= 0) return launch_prefill_tc(a, s);
+    if (!prefill_pool_fits(p.units) || sms <= 0) {
+        if (a.conv) return cudaErrorNotSupported;  // the fused front end runs in the pool kernel only
+        return launch_prefill_tc(a, s);
+    }
     const size_t fb = pool_flag_bytes(p.units);
     p.flags = static_cast<uint32_t *>(a.ws);
     p.ring = static_cast<uint8_t *>(a.ws) + fb;
@@ -1664,8 +1811,17 @@ cudaError_t launch_prefill_pool(const PrefillArgs &a, cudaStream_t s) {
     // the chunk counter, abort flag and hand-off flags start at zero
     cudaError_t e = cudaMemsetAsync(a.ws, 0, fb, s);
     if (e != cudaSuccess) return e;
-    auto kern = p.nh == 3 ? gdn_prefill_pool_kernel<3>
-                          : (p.nh == 2 ? gdn_prefill_pool_kernel<2> : gdn_prefill_pool_kernel<1>);
+    CUtensorMap hq = mq, hk = mk, hv = mv;  // halo maps (the fused front end only)
+    if (a.conv && (!make_halo_map_bf16_128(&hq, a.q, a.T > 0 ? a.T : 1, a.Hqk) ||
+                   !make_halo_map_bf16_128(&hk, a.k, a.T > 0 ? a.T : 1, a.Hqk) ||
+                   !make_halo_map_bf16_128(&hv, a.v, a.T > 0 ? a.T : 1, a.Hv)))
+        return cudaErrorInvalidValue;
+    auto kern = a.conv ? (p.nh == 3 ? gdn_prefill_pool_kernel<3, true>
+                                    : (p.nh == 2 ? gdn_prefill_pool_kernel<2, true>
+                                                 : gdn_prefill_pool_kernel<1, true>))
+                       : (p.nh == 3 ? gdn_prefill_pool_kernel<3, false>
+                                    : (p.nh == 2 ? gdn_prefill_pool_kernel<2, false>
+                                                 : gdn_prefill_pool_kernel<1, false>));
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
@@ -1678,7 +1834,7 @@ cudaError_t launch_prefill_pool(const PrefillArgs &a, cudaStream_t s) {
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, mo, p);
+    e = cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, mo, hq, hk, hv, p);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }

@@ -807,6 +807,21 @@ bool make_tile_map_bf16_128(CUtensorMap *m, const void *base, int64_t T, int32_t
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The same map with 8-token boxes (the tokens before a chunk, for the fused
+// front end's convolution).
+bool make_halo_map_bf16_128(CUtensorMap *m, const void *base, int64_t T, int32_t H) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)H, (cuuint64_t)T};
+    const cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)H * kD * 2};
+    const cuuint32_t box[3] = {64, 1, 8};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
+              box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // [T][H][128] bf16 tensor map for storing whole 64-token tiles of one head
 // (box 128 x 1 x 64, no swizzle: the tile is [64 tokens][128] row-major).
 bool make_store_map_bf16_128(CUtensorMap *m, void *base, int64_t T, int32_t H) {

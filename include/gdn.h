@@ -378,6 +378,52 @@ GDN_API gdn_status gdn_short_conv_norm(const void *xq, const void *xk, const voi
                                        void *stream);
 
 /*
+ * gdn_prefill_conv -- gdn_short_conv_norm followed by gdn_prefill, as one
+ * operation: the mixer's front end (the "kernel 4" convolution of the q, k, v
+ * channels and the per-(token, head) normalisation of q and k, page "Layouts
+ * híbridos: três DeltaNet, uma attention", section 01) is fused into the load
+ * stage of the pool prefill kernel, so the convolved q, k, v never go through
+ * HBM.
+ *
+ *   xq, xk, xv, wq, wk, wv, conv_state_in, conv_state_out
+ *                       as gdn_short_conv_norm (raw channel inputs, filters,
+ *                       carried conv states; conv_state_out may equal
+ *                       conv_state_in).
+ *   g, beta, initial_state, cu_seqlens, N, T, Hqk, Hv, Dk, Dv, chunk, o,
+ *   final_state, dev_error_flag, stream
+ *                       as gdn_prefill with kernel GDN_PREFILL_POOL.
+ *   workspace, workspace_bytes
+ *                       device scratch of at least
+ *                       gdn_prefill_conv_workspace_bytes() (the pool
+ *                       kernel's, then a copy of the filters rearranged for
+ *                       its load stage), 16-byte aligned, caller-owned;
+ *                       contents need not be preserved between calls.
+ * Arithmetic: as the two calls -- the convolution and the norm in fp32, q, k
+ * and v rounded to bf16 once -- up to the order in which a norm's squares are
+ * summed.  Supported: the pool kernel's shapes (bf16, Dk = Dv = 128, chunk 0
+ * or 64, N * Hv <= 64 and SMs enough for it on this GPU); anything else
+ * returns GDN_ERR_UNSUPPORTED (run the two calls instead).  Errors as the two
+ * calls, and GDN_ERR_INVALID_ARGUMENT for a workspace that is too small.
+ */
+/*
+ * gdn_prefill_conv_workspace_bytes -- scratch bytes gdn_prefill_conv needs for
+ * these sizes; 0 when T <= 0 or the shapes are outside the ones it supports
+ * (the call then needs none, or returns GDN_ERR_UNSUPPORTED).
+ */
+GDN_API size_t gdn_prefill_conv_workspace_bytes(int32_t N, int64_t T, int32_t Hqk, int32_t Hv,
+                                                int32_t Dk, int32_t Dv);
+
+GDN_API gdn_status gdn_prefill_conv(const void *xq, const void *xk, const void *xv,
+                                    gdn_dtype io_dtype, const float *wq, const float *wk,
+                                    const float *wv, const float *conv_state_in,
+                                    float *conv_state_out, const float *g, const float *beta,
+                                    const float *initial_state, const int32_t *cu_seqlens,
+                                    int32_t N, int64_t T, int32_t Hqk, int32_t Hv, int32_t Dk,
+                                    int32_t Dv, int32_t chunk, void *o, float *final_state,
+                                    void *workspace, size_t workspace_bytes,
+                                    int32_t *dev_error_flag, void *stream);
+
+/*
  * gdn_debug_prefill_pool_stall -- FOR TESTING THE TIMEOUT PATH ONLY.
  * gdn_prefill_ex with kernel GDN_PREFILL_POOL, except that the producer CTAs
  * never prepare the chunks of (sequence, head) unit `skip_unit` (n * Hv + h),

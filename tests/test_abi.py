@@ -49,6 +49,18 @@ def test_workspace_bytes_is_pure(lib):
     assert a == b and a >= 0
 
 
+def test_conv_workspace_holds_pool_scratch_and_filters(lib):
+    """gdn_prefill_conv's scratch: the pool kernel's, then one 2 KB filter block
+    per q, k and v head; none for an empty call or an unsupported shape."""
+    pool = lib.gdn_prefill_ex_workspace_bytes(1, 262144, 16, 48, 128, 128, 64, 4)
+    conv = lib.gdn_prefill_conv_workspace_bytes(1, 262144, 16, 48, 128, 128)
+    assert pool > 0 and conv >= pool + (2 * 16 + 48) * 2048
+    assert conv - (2 * 16 + 48) * 2048 < pool + 256
+    assert lib.gdn_prefill_conv_workspace_bytes(1, 0, 16, 48, 128, 128) == 0
+    assert lib.gdn_prefill_conv_workspace_bytes(1, 4096, 16, 48, 64, 128) == 0
+    assert lib.gdn_prefill_conv_workspace_bytes(2, 4096, 16, 48, 128, 128) == 0  # 96 units
+
+
 # fake, 16-byte aligned "device" addresses: validation rejects the call before
 # any of them could be dereferenced
 P = 0x10000

@@ -119,3 +119,125 @@ def test_front_end_then_prefill_layer_shape():
     o_ref, s_ref = oracle.recurrent(r(q_ref), r(k_ref), r(v_ref), g, beta)
     check_o(o.cpu(), o_ref)
     check_state(sT.cpu(), s_ref)
+
+
+# ---- the front end fused into the pool prefill (gdn_prefill_conv) ----
+
+def _fused_inputs(lengths, Hqk, Hv, seed, with_state):
+    cu = inputs.cu_from_lengths(lengths)
+    T = int(cu[-1])
+    xq, xk, xv, wq, wk, wv, st = make(T, Hqk, Hv, seed=seed,
+                                      N_state=len(lengths) if with_state else None)
+    gen = torch.Generator().manual_seed(seed + 1)
+    g = -inputs.G_SCALE_097 * torch.nn.functional.softplus(torch.randn(T, Hv, generator=gen))
+    beta = torch.sigmoid(torch.randn(T, Hv, generator=gen))
+    s0 = 0.05 * torch.randn(len(lengths), Hv, 128, 128, generator=gen) if with_state else None
+    return cu, xq, xk, xv, wq, wk, wv, st, g, beta, s0
+
+
+def _fused(cu, xq, xk, xv, wq, wk, wv, st, g, beta, s0):
+    t = lambda x: None if x is None else x.to(DEV).contiguous()
+    flag = torch.zeros(4, dtype=torch.int32, device=DEV)
+    o, sT, st_out = gdn.gdn_prefill_conv(t(xq), t(xk), t(xv), t(wq), t(wk), t(wv), t(g), t(beta),
+                                         t(s0), None if cu is None else cu.to(torch.int32).to(DEV),
+                                         t(st), output_conv_state=True, error_flag=flag)
+    torch.cuda.synchronize()
+    assert int(flag[0]) == 0, gdn.STATUS.get(int(flag[0]))
+    return o.cpu(), sT.cpu(), st_out.cpu()
+
+
+def _oracle_chain(cu, xq, xk, xv, wq, wk, wv, st, g, beta, s0):
+    q_ref, k_ref, v_ref, st_ref = oracle.short_conv_norm(xq, xk, xv, wq, wk, wv, cu, st)
+    r = lambda a: torch.from_numpy(oracle.round_bf16(a))
+    o_ref, s_ref = oracle.recurrent(r(q_ref), r(k_ref), r(v_ref), g, beta, s0,
+                                    None if cu is None else cu.to(torch.int64))
+    return o_ref, s_ref, st_ref
+
+
+@pytest.mark.parametrize("with_state", [False, True])
+def test_fused_front_end_prefill_packed(with_state):
+    """Packed sequences (an empty one, a single chunk, ragged tails, chunks past
+    the first) with and without carried conv and recurrent states, against the
+    oracle's front end (rounded to bf16) then its recurrence."""
+    args = _fused_inputs([0, 64, 200, 1, 777, 130], 2, 6, 8400, with_state)
+    o, sT, st_out = _fused(*args)
+    o_ref, s_ref, st_ref = _oracle_chain(*args)
+    check_o(o, o_ref)
+    check_state(sT, s_ref)
+    assert torch.equal(st_out, torch.from_numpy(st_ref).float())  # raw inputs: exact
+
+
+def test_fused_front_end_split_and_carry():
+    """Each sequence split in two calls that carry the conv state and the
+    recurrent state: matches the one-shot call and the oracle."""
+    lengths = [300, 129, 64, 1000]
+    split = [100, 64, 1, 555]
+    cu, xq, xk, xv, wq, wk, wv, st, g, beta, s0 = _fused_inputs(lengths, 2, 6, 8500, True)
+    o1, s1, c1 = _fused(cu, xq, xk, xv, wq, wk, wv, st, g, beta, s0)
+    o_ref, s_ref, _ = _oracle_chain(cu, xq, xk, xv, wq, wk, wv, st, g, beta, s0)
+    check_o(o1, o_ref, "one-shot o")
+    check_state(s1, s_ref, "one-shot state")
+    pieces = [[], []]
+    for n, L in enumerate(lengths):
+        b = int(cu[n])
+        pieces[0].append((b, b + split[n]))
+        pieces[1].append((b + split[n], b + L))
+    idx = lambda part: torch.cat([torch.arange(a, e) for a, e in part])
+    lens = lambda part: [e - a for a, e in part]
+    sel = lambda x, part: x[idx(part)]
+    ia, ib = pieces
+    cua, cub = inputs.cu_from_lengths(lens(ia)), inputs.cu_from_lengths(lens(ib))
+    oa, sa, ca = _fused(cua, sel(xq, ia), sel(xk, ia), sel(xv, ia), wq, wk, wv, st, sel(g, ia),
+                        sel(beta, ia), s0)
+    ob, sb, cb = _fused(cub, sel(xq, ib), sel(xk, ib), sel(xv, ib), wq, wk, wv, ca, sel(g, ib),
+                        sel(beta, ib), sa)
+    o2 = torch.empty_like(o1)
+    o2[idx(ia)] = oa
+    o2[idx(ib)] = ob
+    check_o(o2, o_ref, "segmented o")
+    check_state(sb, s_ref, "segmented state")
+    assert torch.equal(cb, c1)
+
+
+def test_fused_front_end_layer_shape_matches_separate_calls():
+    """The 4096-token layer of the benchmark's head shape: the fused call
+    against the separate front end then prefill (pool kernel), and against
+    the oracle chain."""
+    T, Hqk, Hv = 4096, 16, 48
+    xq, xk, xv, wq, wk, wv, _ = make(T, Hqk, Hv, seed=8600)
+    gen = torch.Generator().manual_seed(8601)
+    g = -inputs.G_SCALE_097 * torch.nn.functional.softplus(torch.randn(T, Hv, generator=gen))
+    beta = torch.sigmoid(torch.randn(T, Hv, generator=gen))
+    o, sT, _ = _fused(None, xq, xk, xv, wq, wk, wv, None, g, beta, None)
+    q, k, v = run(xq, xk, xv, wq, wk, wv, None, None, out_state=False)
+    o2, s2 = gdn.gdn_prefill(q.to(DEV), k.to(DEV), v.to(DEV), g.to(DEV), beta.to(DEV), kernel="pool")
+    torch.cuda.synchronize()
+    check_o(o, o2.cpu().double(), "fused vs separate o")
+    check_state(sT, s2.cpu().double(), "fused vs separate state")
+    o_ref, s_ref, _ = _oracle_chain(None, xq, xk, xv, wq, wk, wv, None, g, beta, None)
+    check_o(o, o_ref)
+    check_state(sT, s_ref)
+
+
+def test_fused_front_end_rejects_small_workspace_and_fp32():
+    """gdn_prefill_conv validates before launching: a workspace one byte short
+    of gdn_prefill_conv_workspace_bytes, and fp32 inputs (the pool kernel is
+    bf16 only), are errors and leave the output untouched."""
+    args = _fused_inputs([200], 2, 6, 8700, False)
+    cu, xq, xk, xv, wq, wk, wv, st, g, beta, s0 = args
+    T = xq.shape[0]
+    t = lambda x: x.to(DEV).contiguous()
+    need = gdn.gdn_prefill_conv_workspace_bytes(1, T, 2, 6, 128, 128)
+    assert need > 0
+    ws = torch.empty(need - 1, dtype=torch.uint8, device=DEV)
+    o = torch.full((T, 6, 128), 3.0, dtype=torch.bfloat16, device=DEV)
+    with pytest.raises(gdn.GdnError) as e:
+        gdn.gdn_prefill_conv(t(xq), t(xk), t(xv), t(wq), t(wk), t(wv), t(g), t(beta), o=o,
+                             workspace=ws)
+    assert e.value.code == 1
+    with pytest.raises(gdn.GdnError) as e:
+        gdn.gdn_prefill_conv(t(xq).float(), t(xk).float(), t(xv).float(), t(wq), t(wk), t(wv),
+                             t(g), t(beta))
+    assert e.value.code == 2
+    torch.cuda.synchronize()
+    assert bool((o == 3.0).all())
