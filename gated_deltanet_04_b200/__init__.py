@@ -22,6 +22,7 @@ import torch
 
 __all__ = ["gdn_prefill", "gdn_decode_step", "gdn_decode_step_bf16_state", "gdn_decode_step_slots",
            "gdn_short_conv_norm", "gdn_prefill_conv", "gdn_prefill_conv_workspace_bytes",
+           "gdn_prefill_host", "gdn_prefill_host_scratch_bytes", "gdn_prefill_slots",
            "gdn_prefill_workspace_bytes", "library",
            "GdnError", "LIB_PATH", "STATUS", "KERNELS"]
 
@@ -81,6 +82,18 @@ def library():
             lib.gdn_prefill_conv.restype = ctypes.c_int
             lib.gdn_prefill_conv_workspace_bytes.argtypes = [i32, i64, i32, i32, i32, i32]
             lib.gdn_prefill_conv_workspace_bytes.restype = sz
+            lib.gdn_prefill_slots.argtypes = [vp, vp, vp, ctypes.c_int, vp, vp, vp, i32, vp, vp,
+                                              vp, i32, i64, i32, i32, i32, i32, i32, vp, vp, sz,
+                                              vp, vp]
+            lib.gdn_prefill_slots.restype = ctypes.c_int
+            lib.gdn_prefill_slots_workspace_bytes.argtypes = [i32, i64, i32, i32, i32, i32, i32]
+            lib.gdn_prefill_slots_workspace_bytes.restype = sz
+            lib.gdn_prefill_host.argtypes = [vp, vp, vp, ctypes.c_int, vp, vp, vp, i64, i32, i32,
+                                             i32, i32, i32, vp, vp, i64, vp, sz, vp, vp]
+            lib.gdn_prefill_host.restype = ctypes.c_int
+            lib.gdn_prefill_host_scratch_bytes.argtypes = [i64, i32, i32, i32, i32, i32,
+                                                           ctypes.c_int, i64]
+            lib.gdn_prefill_host_scratch_bytes.restype = sz
             lib.gdn_prefill_workspace_bytes.argtypes = [i32, i64, i32, i32, i32, i32, i32]
             lib.gdn_prefill_workspace_bytes.restype = sz
             lib.gdn_prefill_ex_workspace_bytes.argtypes = [i32, i64, i32, i32, i32, i32, i32,
@@ -119,6 +132,60 @@ def _check(t, name, shape, dtype, device):
 def gdn_prefill_conv_workspace_bytes(N, T, Hqk, Hv, Dk, Dv):
     """Scratch bytes gdn_prefill_conv needs (0: none, or unsupported shapes)."""
     return int(library().gdn_prefill_conv_workspace_bytes(N, T, Hqk, Hv, Dk, Dv))
+
+
+def gdn_prefill_host_scratch_bytes(T, Hqk, Hv, Dk, Dv, chunk=0, dtype=torch.bfloat16,
+                                   segment_tokens=0):
+    """Device scratch bytes gdn_prefill_host needs."""
+    return int(library().gdn_prefill_host_scratch_bytes(T, Hqk, Hv, Dk, Dv, chunk, DTYPE[dtype],
+                                                        segment_tokens))
+
+
+def gdn_prefill_host(q, k, v, g, beta, initial_state=None, *, o=None, final_state=None,
+                     output_final_state=True, chunk=0, segment_tokens=0, scratch=None,
+                     error_flag=None, device=None, stream=None):
+    """One sequence's prefill from HOST tensors (the C entry point
+    gdn_prefill_host): q, k [T,Hqk,Dk], v [T,Hv,Dv], g, beta [T,Hv], optional
+    initial_state [Hv,Dv,Dk], all on the CPU (pinned for overlapped copies).
+    The sequence streams through the device in segments.  Returns (o,
+    final_state) as CPU tensors; the copies into them are complete when
+    `stream` (default: the current stream of `device`) has reached them."""
+    lib = library()
+    cpu = torch.device("cpu")
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    T, Hqk, Dk = q.shape
+    Hv, Dv = v.shape[1], v.shape[2]
+    if q.dtype not in DTYPE:
+        raise ValueError(f"unsupported io dtype {q.dtype}")
+    _check(q, "q", (T, Hqk, Dk), q.dtype, cpu)
+    _check(k, "k", (T, Hqk, Dk), q.dtype, cpu)
+    _check(v, "v", (T, Hv, Dv), q.dtype, cpu)
+    _check(g, "g", (T, Hv), torch.float32, cpu)
+    _check(beta, "beta", (T, Hv), torch.float32, cpu)
+    if initial_state is not None:
+        _check(initial_state, "initial_state", (Hv, Dv, Dk), torch.float32, cpu)
+    if o is None:
+        o = torch.empty((T, Hv, Dv), dtype=q.dtype).pin_memory()
+    _check(o, "o", (T, Hv, Dv), q.dtype, cpu)
+    if final_state is None and output_final_state:
+        final_state = torch.empty((Hv, Dv, Dk), dtype=torch.float32).pin_memory()
+    if final_state is not None:
+        _check(final_state, "final_state", (Hv, Dv, Dk), torch.float32, cpu)
+    need = int(lib.gdn_prefill_host_scratch_bytes(T, Hqk, Hv, Dk, Dv, chunk, DTYPE[q.dtype],
+                                                  segment_tokens))
+    if scratch is None:
+        scratch = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    if error_flag is not None:
+        _check(error_flag, "error_flag", tuple(error_flag.shape), torch.int32, dev)
+    st = torch.cuda.current_stream(dev) if stream is None else stream
+    rc = lib.gdn_prefill_host(_ptr(q), _ptr(k), _ptr(v), DTYPE[q.dtype], _ptr(g), _ptr(beta),
+                              _ptr(initial_state), T, Hqk, Hv, Dk, Dv, chunk, _ptr(o),
+                              _ptr(final_state), segment_tokens, _ptr(scratch),
+                              scratch.numel() * scratch.element_size(), _ptr(error_flag),
+                              ctypes.c_void_p(st.cuda_stream))
+    if rc != 0:
+        raise GdnError(rc, "gdn_prefill_host")
+    return o, final_state
 
 
 def gdn_prefill_workspace_bytes(N, T, Hqk, Hv, Dk, Dv, chunk=0, kernel="auto"):
@@ -252,6 +319,50 @@ def gdn_decode_step_slots(q, k, v, g, beta, state_pool, slot_idx, reset=None, *,
                                    Dk, Dv, _ptr(o), _ptr(error_flag), _stream(stream))
     if rc != 0:
         raise GdnError(rc, "gdn_decode_step_slots")
+    return o
+
+
+def gdn_prefill_slots(q, k, v, g, beta, state_pool, slot_idx, reset=None, cu_seqlens=None, *,
+                      chunk=0, o=None, workspace=None, error_flag=None, stream=None):
+    """Prefill for continuous batching: sequence n starts from
+    ``state_pool[slot_idx[n]]`` ([num_slots,Hv,Dv,Dk] fp32, updated in place),
+    or from zeros when ``reset[n]`` is nonzero, and its final state goes back
+    to that slot.  q, k [T,Hqk,Dk], v [T,Hv,Dv], g, beta [T,Hv] as gdn_prefill;
+    slot_idx (and reset) int32 [N] on the device; cu_seqlens int32 [N+1] or
+    None (N = 1).  Returns o."""
+    lib = library()
+    dev = q.device
+    if dev.type != "cuda":
+        raise ValueError("gdn_prefill_slots runs on CUDA tensors only")
+    T, Hqk, Dk = q.shape
+    Hv, Dv = v.shape[1], v.shape[2]
+    if q.dtype not in DTYPE:
+        raise ValueError(f"unsupported io dtype {q.dtype}")
+    N = 1 if cu_seqlens is None else cu_seqlens.shape[0] - 1
+    S = state_pool.shape[0]
+    _check(k, "k", (T, Hqk, Dk), q.dtype, dev)
+    _check(v, "v", (T, Hv, Dv), q.dtype, dev)
+    _check(g, "g", (T, Hv), torch.float32, dev)
+    _check(beta, "beta", (T, Hv), torch.float32, dev)
+    _check(state_pool, "state_pool", (S, Hv, Dv, Dk), torch.float32, dev)
+    _check(slot_idx, "slot_idx", (N,), torch.int32, dev)
+    if reset is not None:
+        _check(reset, "reset", (N,), torch.int32, dev)
+    if cu_seqlens is not None:
+        _check(cu_seqlens, "cu_seqlens", (N + 1,), torch.int32, dev)
+    if o is None:
+        o = torch.empty((T, Hv, Dv), dtype=q.dtype, device=dev)
+    _check(o, "o", (T, Hv, Dv), q.dtype, dev)
+    need = int(lib.gdn_prefill_slots_workspace_bytes(N, T, Hqk, Hv, Dk, Dv, chunk))
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    rc = lib.gdn_prefill_slots(_ptr(q), _ptr(k), _ptr(v), DTYPE[q.dtype], _ptr(g), _ptr(beta),
+                               _ptr(state_pool), S, _ptr(slot_idx), _ptr(reset), _ptr(cu_seqlens),
+                               N, T, Hqk, Hv, Dk, Dv, chunk, _ptr(o), _ptr(workspace),
+                               workspace.numel() * workspace.element_size(), _ptr(error_flag),
+                               _stream(stream))
+    if rc != 0:
+        raise GdnError(rc, "gdn_prefill_slots")
     return o
 
 

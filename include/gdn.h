@@ -424,6 +424,103 @@ GDN_API gdn_status gdn_prefill_conv(const void *xq, const void *xk, const void *
                                     int32_t *dev_error_flag, void *stream);
 
 /*
+ * gdn_prefill_slots -- gdn_prefill over a packed batch whose states live in
+ * the same pool of slots as gdn_decode_step_slots (continuous batching: page
+ * "Hybrid · kết hợp…", section 3, state updates with batch and reset rules).
+ * Sequence n starts from state_pool[slot_idx[n]], or from zeros when reset[n]
+ * is nonzero (a new request; its slot is not read), and its final state is
+ * written back to that slot.  Slots no sequence names are not touched.
+ *
+ *   q, k, v, io_dtype, g, beta, cu_seqlens, N, T, Hqk, Hv, Dk, Dv, chunk, o,
+ *   dev_error_flag, stream
+ *                       as gdn_prefill.
+ *   state_pool          fp32 [num_slots][Hv][Dv][Dk], device, updated in place.
+ *   slot_idx            device int32 [N], distinct values in [0, num_slots).
+ *                       An index out of range is reported as GDN_ERR_BAD_SLOT
+ *                       through dev_error_flag; that sequence runs from zeros
+ *                       and its state is not stored.  Repeated indices are a
+ *                       caller error (the slot ends with one of the states).
+ *   reset               device int32 [N], or NULL for none.
+ *   workspace, workspace_bytes
+ *                       device scratch of at least
+ *                       gdn_prefill_slots_workspace_bytes(): the N gathered
+ *                       states, then gdn_prefill's workspace.
+ * The states are gathered into the workspace, gdn_prefill runs in place on
+ * them, and they are scattered back: 2 N Hv Dv Dk fp32 values of copies.
+ * Errors as gdn_prefill, and GDN_ERR_INVALID_ARGUMENT for a null pool or
+ * slot list, num_slots <= 0 or a short workspace.
+ */
+GDN_API gdn_status gdn_prefill_slots(const void *q, const void *k, const void *v,
+                                     gdn_dtype io_dtype, const float *g, const float *beta,
+                                     float *state_pool, int32_t num_slots,
+                                     const int32_t *slot_idx, const int32_t *reset,
+                                     const int32_t *cu_seqlens, int32_t N, int64_t T, int32_t Hqk,
+                                     int32_t Hv, int32_t Dk, int32_t Dv, int32_t chunk, void *o,
+                                     void *workspace, size_t workspace_bytes,
+                                     int32_t *dev_error_flag, void *stream);
+
+/*
+ * gdn_prefill_slots_workspace_bytes -- scratch bytes gdn_prefill_slots needs
+ * for these sizes (0 for invalid ones).
+ */
+GDN_API size_t gdn_prefill_slots_workspace_bytes(int32_t N, int64_t T, int32_t Hqk, int32_t Hv,
+                                                 int32_t Dk, int32_t Dv, int32_t chunk);
+
+/*
+ * gdn_prefill_host -- gdn_prefill of ONE sequence whose inputs and outputs
+ * are in host memory.  The state carries everything one part of a sequence
+ * hands to the next (page "Qwen3.8-27B 架构深读…", section 三), so the
+ * sequence runs as consecutive segments of segment_tokens tokens, each a
+ * gdn_prefill call on `stream` that starts from the state the previous one
+ * left (in place, in scratch).  Two internal streams overlap the copies: the
+ * next segment's q, k, v, g, beta go in while a segment computes and the
+ * previous segment's o comes back.
+ *
+ *   q, k, v, g, beta    HOST memory, layouts as gdn_prefill with N = 1.  Pin
+ *                       it (cudaHostAlloc / cudaHostRegister) for the copies
+ *                       to overlap; pageable memory works, serialised.
+ *   initial_state       HOST fp32 [Hv][Dv][Dk], or NULL for zeros.
+ *   T, Hqk, Hv, Dk, Dv, chunk
+ *                       as gdn_prefill.
+ *   o                   HOST output [T][Hv][Dv] in io_dtype.
+ *   final_state         HOST fp32 [Hv][Dv][Dk], or NULL to skip.
+ *   segment_tokens      tokens per segment, a multiple of 64 so that
+ *                       segments end on chunk boundaries; 0 picks 16,384.
+ *   scratch, scratch_bytes
+ *                       DEVICE scratch of at least
+ *                       gdn_prefill_host_scratch_bytes(), 16-byte aligned,
+ *                       caller-owned: the state, the prefill workspace and
+ *                       two segment buffers.
+ *   dev_error_flag      optional device int32, as gdn_prefill.
+ *   stream              cudaStream_t.  The call is asynchronous like a copy
+ *                       on `stream`: it starts after the work queued there
+ *                       and `stream` sees it complete; the host buffers must
+ *                       stay valid and unread until then.
+ * Arithmetic: the segments' kernels are gdn_prefill's for segment_tokens
+ * tokens; the result equals one gdn_prefill call over the whole sequence
+ * within the prefill's tolerances (a state that crosses a segment boundary
+ * passes through fp32 memory exactly).  Errors: GDN_ERR_INVALID_ARGUMENT for
+ * bad sizes, a segment length that is not a multiple of 64 or a short
+ * scratch; gdn_prefill's otherwise.  It creates two streams and eight events
+ * per call and releases them before returning (CUDA frees them once the
+ * queued work is done).
+ */
+GDN_API gdn_status gdn_prefill_host(const void *q, const void *k, const void *v,
+                                    gdn_dtype io_dtype, const float *g, const float *beta,
+                                    const float *initial_state, int64_t T, int32_t Hqk,
+                                    int32_t Hv, int32_t Dk, int32_t Dv, int32_t chunk, void *o,
+                                    float *final_state, int64_t segment_tokens, void *scratch,
+                                    size_t scratch_bytes, int32_t *dev_error_flag, void *stream);
+
+/*
+ * gdn_prefill_host_scratch_bytes -- device scratch gdn_prefill_host needs for
+ * these sizes (0 for invalid ones).
+ */
+GDN_API size_t gdn_prefill_host_scratch_bytes(int64_t T, int32_t Hqk, int32_t Hv, int32_t Dk,
+                                              int32_t Dv, int32_t chunk, gdn_dtype io_dtype,
+                                              int64_t segment_tokens);
+
+/*
  * gdn_debug_prefill_pool_stall -- FOR TESTING THE TIMEOUT PATH ONLY.
  * gdn_prefill_ex with kernel GDN_PREFILL_POOL, except that the producer CTAs
  * never prepare the chunks of (sequence, head) unit `skip_unit` (n * Hv + h),

@@ -214,6 +214,33 @@ def decode_step_slots(q, k, v, g, beta, pool, slot_idx, reset=None, *, order=ORD
     return o, pool
 
 
+def prefill_slots(q, k, v, g, beta, pool, slot_idx, reset=None, cu_seqlens=None, *,
+                  order=ORDER_STANDARD):
+    """A prefill of N packed sequences whose states live in a pool of slots
+    (continuous batching, page "Hybrid · kết hợp…", section 3: state updates
+    with batch and reset rules): sequence n starts from pool[slot_idx[n]], or
+    from zeros when reset[n] is nonzero (a new request), and its final state is
+    written back to that slot; slots no sequence names are left as they are.
+    slot_idx must hold distinct values in [0, num_slots).
+
+    Shapes as ``recurrent`` with N sequences; pool [S,Hv,Dv,Dk], slot_idx [N]
+    int, reset [N] or None.  Returns (o [T,Hv,Dv], new pool) in float64.
+    """
+    pool = _f64(pool).copy()
+    idx = np.asarray(slot_idx.detach().cpu().numpy() if hasattr(slot_idx, "detach") else slot_idx,
+                     dtype=np.int64)
+    S = pool.shape[0]
+    if idx.ndim != 1 or np.any(idx < 0) or np.any(idx >= S) or len(set(idx.tolist())) != idx.size:
+        raise ValueError("prefill_slots: slot indices must be distinct and in range")
+    states = pool[idx].copy()
+    if reset is not None:
+        rs = np.asarray(reset.detach().cpu().numpy() if hasattr(reset, "detach") else reset)
+        states[rs != 0] = 0.0
+    o, new = recurrent(q, k, v, g, beta, states, cu_seqlens, order=order)
+    pool[idx] = new
+    return o, pool
+
+
 def short_conv(x, w, cu_seqlens=None, conv_state=None):
     """Causal depthwise convolution with 4 taps along time, the DeltaNet
     mixer's "kernel 4" convolution (page "Layouts híbridos: três DeltaNet, uma

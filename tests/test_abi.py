@@ -61,6 +61,31 @@ def test_conv_workspace_holds_pool_scratch_and_filters(lib):
     assert lib.gdn_prefill_conv_workspace_bytes(2, 4096, 16, 48, 128, 128) == 0  # 96 units
 
 
+def test_host_scratch_bytes(lib):
+    """gdn_prefill_host's scratch: state, workspace and two segment buffers,
+    growing with the segment length up to the sequence length; 0 for bad sizes."""
+    per_token = 2 * (2 * 16 * 128 * 2 + 2 * 48 * 128 * 2 + 2 * 48 * 4)  # two buffers, bf16
+    a = lib.gdn_prefill_host_scratch_bytes(262144, 16, 48, 128, 128, 64, 0, 16384)
+    b = lib.gdn_prefill_host_scratch_bytes(262144, 16, 48, 128, 128, 64, 0, 32768)
+    assert a >= 16384 * per_token + 48 * 128 * 128 * 4
+    assert b - a >= 16384 * per_token
+    assert lib.gdn_prefill_host_scratch_bytes(1000, 16, 48, 128, 128, 64, 0, 16384) == \
+        lib.gdn_prefill_host_scratch_bytes(1000, 16, 48, 128, 128, 64, 0, 0)
+    assert lib.gdn_prefill_host_scratch_bytes(-1, 16, 48, 128, 128, 64, 0, 0) == 0
+    assert lib.gdn_prefill_host_scratch_bytes(100, 16, 48, 128, 128, 64, 5, 0) == 0
+
+
+def test_host_prefill_rejects_bad_segments_before_any_copy(lib):
+    """A segment length that is not a multiple of 64, or no scratch, fails
+    validation without touching the (fake) pointers."""
+    rc = lib.gdn_prefill_host(P, P, P, 0, P, P, None, 100, 16, 48, 128, 128, 64, P, None, 100, P,
+                              1 << 40, None, None)
+    assert rc == INVALID
+    rc = lib.gdn_prefill_host(P, P, P, 0, P, P, None, 100, 16, 48, 128, 128, 64, P, None, 0, None,
+                              0, None, None)
+    assert rc == INVALID
+
+
 # fake, 16-byte aligned "device" addresses: validation rejects the call before
 # any of them could be dereferenced
 P = 0x10000

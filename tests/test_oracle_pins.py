@@ -465,6 +465,76 @@ def test_slots_reject_bad_indices():
             oracle.decode_step_slots(q, k, v, g, b, pool, np.array(bad))
 
 
+# ---- prefill over a pool of state slots ----------------------------------------
+
+def _pslots_case(seed, lengths=(3, 1, 5), S=7, Hqk=2, Hv=4, D=8):
+    r = rnd(seed)
+    T = sum(lengths)
+    q = unit_rows(r.standard_normal((T, Hqk, D)))
+    k = unit_rows(r.standard_normal((T, Hqk, D)))
+    v = r.standard_normal((T, Hv, D))
+    g = -r.uniform(0, 1, (T, Hv))
+    b = r.uniform(0, 1, (T, Hv))
+    pool = r.standard_normal((S, Hv, D, D))
+    cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int64)
+    return q, k, v, g, b, pool, cu
+
+
+def test_prefill_slots_identity_mapping_is_recurrent():
+    q, k, v, g, b, pool, cu = _pslots_case(41, S=3)
+    o, new = oracle.prefill_slots(q, k, v, g, b, pool, np.arange(3), cu_seqlens=cu)
+    o_ref, s_ref = oracle.recurrent(q, k, v, g, b, pool, cu)
+    assert np.array_equal(o, o_ref) and np.array_equal(new, s_ref)
+
+
+def test_prefill_slots_gather_scatter_untouched_and_permuted():
+    """Sequences read and write only their own slots; slots nobody names come
+    back bit for bit; reordering the packed sequences (tokens and slot list
+    together) reorders only o."""
+    lengths = (3, 1, 5)
+    q, k, v, g, b, pool, cu = _pslots_case(42, lengths)
+    idx = np.array([5, 1, 3])
+    o, new = oracle.prefill_slots(q, k, v, g, b, pool, idx, cu_seqlens=cu)
+    o_ref, s_ref = oracle.recurrent(q, k, v, g, b, pool[idx], cu)
+    assert np.array_equal(o, o_ref) and np.array_equal(new[idx], s_ref)
+    untouched = np.setdiff1d(np.arange(pool.shape[0]), idx)
+    assert np.array_equal(new[untouched], pool[untouched])
+    perm = [2, 0, 1]
+    tok = np.concatenate([np.arange(cu[n], cu[n + 1]) for n in perm])
+    cu_p = np.concatenate([[0], np.cumsum([lengths[n] for n in perm])]).astype(np.int64)
+    o_p, new_p = oracle.prefill_slots(q[tok], k[tok], v[tok], g[tok], b[tok], pool, idx[perm],
+                                      cu_seqlens=cu_p)
+    assert np.array_equal(o_p, o[tok]) and np.array_equal(new_p, new)
+
+
+def test_prefill_slots_reset_starts_from_zero():
+    """A reset sequence ignores its slot: one token from S = 0 gives
+    S' = b v k^T and o = b (k . q) v; a longer reset sequence equals the same
+    sequence started from a slot that holds zeros."""
+    lengths = (1, 4, 2)
+    q, k, v, g, b, pool, cu = _pslots_case(43, lengths)
+    idx = np.array([6, 2, 0])
+    reset = np.array([1, 1, 0])
+    o, new = oracle.prefill_slots(q, k, v, g, b, pool, idx, reset, cu)
+    heads = np.arange(v.shape[1]) // (v.shape[1] // q.shape[1])
+    kk, qq = k[0, heads], q[0, heads]
+    want_s = b[0][:, None, None] * v[0][:, :, None] * kk[:, None, :]
+    assert np.allclose(new[6], want_s, rtol=1e-13, atol=1e-14)
+    want_o = (b[0] * np.sum(kk * qq, axis=1))[:, None] * v[0]
+    assert np.allclose(o[0], want_o, rtol=1e-12, atol=1e-13)
+    zeroed = pool.copy()
+    zeroed[[6, 2]] = 0.0
+    o_z, new_z = oracle.prefill_slots(q, k, v, g, b, zeroed, idx, None, cu)
+    assert np.array_equal(o, o_z) and np.array_equal(new[idx], new_z[idx])
+
+
+def test_prefill_slots_reject_bad_indices():
+    q, k, v, g, b, pool, cu = _pslots_case(44)
+    for bad in ([0, 1, 7], [0, -1, 2], [3, 3, 4]):
+        with pytest.raises(ValueError):
+            oracle.prefill_slots(q, k, v, g, b, pool, np.array(bad), cu_seqlens=cu)
+
+
 # ---- front end: kernel-4 causal short convolution and per-head L2 norm ---------
 
 def test_short_conv_taps_are_delays():
