@@ -16,6 +16,7 @@
 // second small kernel writes the new conv state.
 #include "gdn_internal.cuh"
 #include "sm100.cuh"
+#include "trace.cuh"
 
 namespace gdn {
 namespace {
@@ -280,6 +281,7 @@ extern "C" GDN_API gdn_status gdn_short_conv_norm(
     const float *wk, const float *wv, const float *conv_state_in, float *conv_state_out,
     const int32_t *cu_seqlens, int32_t N, int64_t T, int32_t Hqk, int32_t Hv, int32_t Dk,
     int32_t Dv, void *q, void *k, void *v, int32_t *dev_error_flag, void *stream) {
+    GDN_TRACE("gdn_short_conv_norm");
     using gdn::aligned16;
     if (io_dtype != GDN_DTYPE_BF16 && io_dtype != GDN_DTYPE_F32) return GDN_ERR_INVALID_ARGUMENT;
     if (N < 0 || T < 0 || Hqk <= 0 || Hv <= 0 || Dk <= 0 || Dv <= 0) return GDN_ERR_INVALID_ARGUMENT;

@@ -3,6 +3,7 @@
 #include <stdint.h>
 
 #include "gdn_internal.cuh"
+#include "trace.cuh"
 
 namespace {
 
@@ -99,6 +100,7 @@ gdn_status prefill_impl(const void *q, const void *k, const void *v, gdn_dtype i
                         void *workspace, size_t workspace_bytes, int32_t *dev_error_flag,
                         void *stream, gdn_prefill_kernel kernel, gdn_order order,
                         int32_t debug_skip_unit, int64_t debug_flag_wait) {
+    GDN_TRACE("gdn_prefill");
     if (kernel < GDN_PREFILL_AUTO || kernel > GDN_PREFILL_POOL) return GDN_ERR_INVALID_ARGUMENT;
     if (order != GDN_ORDER_STANDARD && order != GDN_ORDER_RECALL_FIRST) return GDN_ERR_INVALID_ARGUMENT;
     if (io_dtype != GDN_DTYPE_BF16 && io_dtype != GDN_DTYPE_F32) return GDN_ERR_INVALID_ARGUMENT;
@@ -177,6 +179,7 @@ gdn_status gdn_prefill_conv(const void *xq, const void *xk, const void *xv, gdn_
                             int32_t Hv, int32_t Dk, int32_t Dv, int32_t chunk, void *o,
                             float *final_state, void *workspace, size_t workspace_bytes,
                             int32_t *dev_error_flag, void *stream) {
+    GDN_TRACE("gdn_prefill_conv");
     if (io_dtype != GDN_DTYPE_BF16 && io_dtype != GDN_DTYPE_F32) return GDN_ERR_INVALID_ARGUMENT;
     if (N < 0 || T < 0 || Hqk <= 0 || Hv <= 0 || Dk <= 0 || Dv <= 0 || chunk < 0)
         return GDN_ERR_INVALID_ARGUMENT;
@@ -250,6 +253,7 @@ gdn_status gdn_decode_step_order(const void *q, const void *k, const void *v, gd
                                  const float *g, const float *beta, float *state, int32_t N,
                                  int32_t Hqk, int32_t Hv, int32_t Dk, int32_t Dv, void *o,
                                  int32_t *dev_error_flag, void *stream, gdn_order order) {
+    GDN_TRACE("gdn_decode_step");
     if (order != GDN_ORDER_STANDARD && order != GDN_ORDER_RECALL_FIRST) return GDN_ERR_INVALID_ARGUMENT;
     if (io_dtype != GDN_DTYPE_BF16 && io_dtype != GDN_DTYPE_F32) return GDN_ERR_INVALID_ARGUMENT;
     if (N < 0 || Hqk <= 0 || Hv <= 0 || Dk <= 0 || Dv <= 0) return GDN_ERR_INVALID_ARGUMENT;
@@ -275,6 +279,7 @@ gdn_status gdn_decode_step_slots(const void *q, const void *k, const void *v, gd
                                  int32_t num_slots, const int32_t *slot_idx, const int32_t *reset,
                                  int32_t N, int32_t Hqk, int32_t Hv, int32_t Dk, int32_t Dv,
                                  void *o, int32_t *dev_error_flag, void *stream) {
+    GDN_TRACE("gdn_decode_step_slots");
     if (io_dtype != GDN_DTYPE_BF16 && io_dtype != GDN_DTYPE_F32) return GDN_ERR_INVALID_ARGUMENT;
     if (N < 0 || Hqk <= 0 || Hv <= 0 || Dk <= 0 || Dv <= 0) return GDN_ERR_INVALID_ARGUMENT;
     if (Hv % Hqk != 0) return GDN_ERR_INVALID_ARGUMENT;
@@ -299,6 +304,7 @@ gdn_status gdn_decode_step_bf16_state(const void *q, const void *k, const void *
                                       gdn_dtype io_dtype, const float *g, const float *beta,
                                       void *state, int32_t N, int32_t Hqk, int32_t Hv, int32_t Dk,
                                       int32_t Dv, void *o, int32_t *dev_error_flag, void *stream) {
+    GDN_TRACE("gdn_decode_step_bf16_state");
     if (io_dtype != GDN_DTYPE_BF16 && io_dtype != GDN_DTYPE_F32) return GDN_ERR_INVALID_ARGUMENT;
     if (N < 0 || Hqk <= 0 || Hv <= 0 || Dk <= 0 || Dv <= 0) return GDN_ERR_INVALID_ARGUMENT;
     if (Hv % Hqk != 0) return GDN_ERR_INVALID_ARGUMENT;

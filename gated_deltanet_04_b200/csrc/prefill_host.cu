@@ -14,6 +14,7 @@
 #include <cstdint>
 
 #include "gdn.h"
+#include "trace.cuh"
 
 namespace {
 
@@ -104,6 +105,7 @@ gdn_status gdn_prefill_host(const void *q, const void *k, const void *v, gdn_dty
                             int32_t Hqk, int32_t Hv, int32_t Dk, int32_t Dv, int32_t chunk, void *o,
                             float *final_state, int64_t segment_tokens, void *scratch,
                             size_t scratch_bytes, int32_t *dev_error_flag, void *stream) {
+    GDN_TRACE("gdn_prefill_host");
     if (io_dtype != GDN_DTYPE_BF16 && io_dtype != GDN_DTYPE_F32) return GDN_ERR_INVALID_ARGUMENT;
     if (T < 0 || Hqk <= 0 || Hv <= 0 || Dk <= 0 || Dv <= 0 || chunk < 0) return GDN_ERR_INVALID_ARGUMENT;
     if (Hv % Hqk != 0) return GDN_ERR_INVALID_ARGUMENT;

@@ -13,6 +13,7 @@
 
 #include "gdn.h"
 #include "gdn_internal.cuh"
+#include "trace.cuh"
 
 namespace {
 
@@ -83,6 +84,7 @@ gdn_status gdn_prefill_slots(const void *q, const void *k, const void *v, gdn_dt
                              int32_t Hv, int32_t Dk, int32_t Dv, int32_t chunk, void *o,
                              void *workspace, size_t workspace_bytes, int32_t *dev_error_flag,
                              void *stream) {
+    GDN_TRACE("gdn_prefill_slots");
     if (N < 0 || T < 0 || Hqk <= 0 || Hv <= 0 || Dk <= 0 || Dv <= 0 || chunk < 0)
         return GDN_ERR_INVALID_ARGUMENT;
     if (N == 0) return T == 0 ? GDN_OK : GDN_ERR_INVALID_ARGUMENT;
