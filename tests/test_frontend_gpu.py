@@ -167,6 +167,19 @@ def test_fused_front_end_prefill_packed(with_state):
     assert torch.equal(st_out, torch.from_numpy(st_ref).float())  # raw inputs: exact
 
 
+@pytest.mark.parametrize("Hqk,Hv", [(3, 3), (2, 4), (1, 5)])
+def test_fused_front_end_other_group_sizes(Hqk, Hv):
+    """Producer items of one and of two v-heads per q/k head (the group sizes
+    other than 3 that the pool kernel uses: 3 heads share q/k with 1, 4 heads
+    over 2 with 2, 5 over 1 with 1), packed sequences with carried states."""
+    args = _fused_inputs([130, 1, 64, 257], Hqk, Hv, 8800 + 10 * Hqk + Hv, True)
+    o, sT, st_out = _fused(*args)
+    o_ref, s_ref, st_ref = _oracle_chain(*args)
+    check_o(o, o_ref)
+    check_state(sT, s_ref)
+    assert torch.equal(st_out, torch.from_numpy(st_ref).float())
+
+
 def test_fused_front_end_split_and_carry():
     """Each sequence split in two calls that carry the conv state and the
     recurrent state: matches the one-shot call and the oracle."""
