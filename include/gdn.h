@@ -501,9 +501,12 @@ GDN_API size_t gdn_prefill_slots_workspace_bytes(int32_t N, int64_t T, int32_t H
  * within the prefill's tolerances (a state that crosses a segment boundary
  * passes through fp32 memory exactly).  Errors: GDN_ERR_INVALID_ARGUMENT for
  * bad sizes, a segment length that is not a multiple of 64 or a short
- * scratch; gdn_prefill's otherwise.  It creates two streams and eight events
- * per call and releases them before returning (CUDA frees them once the
- * queued work is done).
+ * scratch; gdn_prefill's otherwise.  After GDN_ERR_CUDA (or an error from a
+ * segment's gdn_prefill) copies of earlier segments may still be in flight
+ * on the internal streams, which `stream` does not wait for: synchronise the
+ * device before reusing the host buffers or the scratch.  It creates two
+ * streams and eight events per call and releases them before returning (CUDA
+ * frees them once the queued work is done).
  */
 GDN_API gdn_status gdn_prefill_host(const void *q, const void *k, const void *v,
                                     gdn_dtype io_dtype, const float *g, const float *beta,
