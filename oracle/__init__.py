@@ -187,6 +187,30 @@ def decode_step_bf16_state(q, k, v, g, beta, state, *, order=ORDER_STANDARD):
     return o, s_new, round_bf16(s_new)
 
 
+def _gather_slots(pool, slot_idx, reset, what):
+    """The batch/reset rule of a state pool: a copy of the pool (fp64), the
+    slot of each entry, and each entry's starting state -- its slot's, or
+    zeros when reset[n] is nonzero.  Slot indices must be distinct and in
+    range."""
+    pool = _f64(pool).copy()
+    idx = np.asarray(slot_idx.detach().cpu().numpy() if hasattr(slot_idx, "detach") else slot_idx,
+                     dtype=np.int64)
+    S = pool.shape[0]
+    if idx.ndim != 1 or np.any(idx < 0) or np.any(idx >= S) or len(set(idx.tolist())) != idx.size:
+        raise ValueError(f"{what}: slot indices must be distinct and in range")
+    states = pool[idx].copy()
+    if reset is not None:
+        rs = np.asarray(reset.detach().cpu().numpy() if hasattr(reset, "detach") else reset)
+        states[rs != 0] = 0.0
+    return pool, idx, states
+
+
+def _scatter_slots(pool, idx, new):
+    """Each entry's final state back into its slot; other slots unchanged."""
+    pool[idx] = new
+    return pool
+
+
 def decode_step_slots(q, k, v, g, beta, pool, slot_idx, reset=None, *, order=ORDER_STANDARD):
     """One decode step of N batch entries whose states live in a pool of slots
     (continuous batching): entry n uses pool[slot_idx[n]]; when reset[n] is
@@ -199,19 +223,9 @@ def decode_step_slots(q, k, v, g, beta, pool, slot_idx, reset=None, *, order=ORD
     slot_idx [N] int, reset [N] or None.  Returns (o [N,Hv,Dv], new pool) in
     float64.
     """
-    pool = _f64(pool).copy()
-    idx = np.asarray(slot_idx.detach().cpu().numpy() if hasattr(slot_idx, "detach") else slot_idx,
-                     dtype=np.int64)
-    S = pool.shape[0]
-    if idx.ndim != 1 or np.any(idx < 0) or np.any(idx >= S) or len(set(idx.tolist())) != idx.size:
-        raise ValueError("decode_step_slots: slot indices must be distinct and in range")
-    states = pool[idx].copy()
-    if reset is not None:
-        rs = np.asarray(reset.detach().cpu().numpy() if hasattr(reset, "detach") else reset)
-        states[rs != 0] = 0.0
+    pool, idx, states = _gather_slots(pool, slot_idx, reset, "decode_step_slots")
     o, new = decode_step(q, k, v, g, beta, states, order=order)
-    pool[idx] = new
-    return o, pool
+    return o, _scatter_slots(pool, idx, new)
 
 
 def prefill_slots(q, k, v, g, beta, pool, slot_idx, reset=None, cu_seqlens=None, *,
@@ -226,19 +240,9 @@ def prefill_slots(q, k, v, g, beta, pool, slot_idx, reset=None, cu_seqlens=None,
     Shapes as ``recurrent`` with N sequences; pool [S,Hv,Dv,Dk], slot_idx [N]
     int, reset [N] or None.  Returns (o [T,Hv,Dv], new pool) in float64.
     """
-    pool = _f64(pool).copy()
-    idx = np.asarray(slot_idx.detach().cpu().numpy() if hasattr(slot_idx, "detach") else slot_idx,
-                     dtype=np.int64)
-    S = pool.shape[0]
-    if idx.ndim != 1 or np.any(idx < 0) or np.any(idx >= S) or len(set(idx.tolist())) != idx.size:
-        raise ValueError("prefill_slots: slot indices must be distinct and in range")
-    states = pool[idx].copy()
-    if reset is not None:
-        rs = np.asarray(reset.detach().cpu().numpy() if hasattr(reset, "detach") else reset)
-        states[rs != 0] = 0.0
+    pool, idx, states = _gather_slots(pool, slot_idx, reset, "prefill_slots")
     o, new = recurrent(q, k, v, g, beta, states, cu_seqlens, order=order)
-    pool[idx] = new
-    return o, pool
+    return o, _scatter_slots(pool, idx, new)
 
 
 def short_conv(x, w, cu_seqlens=None, conv_state=None):

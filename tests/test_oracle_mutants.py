@@ -46,7 +46,7 @@ MUTANTS_PY = {
     "bf16_seven_bits": ("return np.ldexp(np.rint(np.ldexp(m, 8)), e - 8)",
                         "return np.ldexp(np.rint(np.ldexp(m, 7)), e - 7)"),
     "slots_reset_ignored": ("states[rs != 0] = 0.0", "states[rs != 0] = states[rs != 0]"),
-    "slots_not_written_back": ("    pool[idx] = new\n", "    pool[idx] = states\n"),
+    "slots_not_written_back": ("    pool[idx] = new\n", "    pool[idx] = pool[idx]\n"),
     "conv_taps_reversed": ("y[cu[n] + t] += w[:, j] * ext[t + j]", "y[cu[n] + t] += w[:, 3 - j] * ext[t + j]"),
     "conv_state_ignored": ("st = np.zeros((N, 3, C)) if conv_state is None else _f64(conv_state)",
                            "st = np.zeros((N, 3, C))"),
