@@ -27,6 +27,7 @@ import argparse
 import datetime
 import hashlib
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -294,7 +295,8 @@ def percentiles(each_ms):
     xs = sorted(each_ms)
     if not xs:
         return None
-    pick = lambda q: xs[min(len(xs) - 1, max(0, int(round(q * len(xs) + 0.5)) - 1))]
+    # rank ceil(q n), 1-based; the epsilon keeps q n = 95.00000000000001 at 95
+    pick = lambda q: xs[min(len(xs), max(1, math.ceil(q * len(xs) - 1e-9))) - 1]
     return {"p50": pick(0.50), "p95": pick(0.95), "p99": pick(0.99), "calls": len(xs)}
 
 
