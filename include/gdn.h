@@ -29,21 +29,27 @@
  * v-head h reads q/k head h / (Hv / Hqk): groups of Hv/Hqk consecutive v-heads
  * share one q/k head.
  *
- * Ownership: every pointer is a DEVICE pointer owned by the caller.  The
- * library allocates nothing, frees nothing and never synchronises; all work
- * is enqueued on `stream` (a cudaStream_t; NULL is the legacy default stream)
- * and completes asynchronously.  Inputs are only read.  Outputs must not alias
- * inputs, except where stated.  Every pointer must be 16-byte aligned.
+ * Ownership: every pointer is a DEVICE pointer owned by the caller, except
+ * the host buffers of gdn_prefill_host.  The library allocates no memory,
+ * frees nothing and never synchronises; all work is enqueued on `stream` (a
+ * cudaStream_t; NULL is the legacy default stream) and completes
+ * asynchronously.  (gdn_prefill_host creates and releases two streams and
+ * eight events per call, and its copies to or from pageable host memory are
+ * synchronous, as CUDA makes them.)  Inputs are only read.  Outputs must not
+ * alias inputs, except where stated.  Every pointer must be 16-byte aligned.
  *
  * Errors: argument errors are returned synchronously and nothing is launched.
  * A failed launch returns GDN_ERR_CUDA (cudaGetLastError, no synchronisation).
  * Errors only the device can see (a malformed cu_seqlens, a bounded wait that
- * expired, an fp16 range overflow of a q/k-side operand) are written as a
+ * expired, an fp16 range overflow of a q/k-side operand, a state slot index
+ * out of range) are written as a
  * gdn_status value to *dev_error_flag when that
  * optional device int32 is given; the caller zeroes it beforehand and reads it
  * after synchronising.  A unit (sequence, head) that detects such an error
  * writes no output for itself.  No C++ exception crosses this interface.  The
- * calls keep no global mutable state and are safe to call from any thread.
+ * calls keep no global mutable state and are safe to call from any thread,
+ * except gdn_prefill_static_workspace, whose one scratch array per device is
+ * shared by its calls (see its contract).
  */
 #ifndef GDN_H_
 #define GDN_H_
